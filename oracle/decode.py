@@ -1,0 +1,185 @@
+"""Oracle: context encoding, one denoising step of the canvas, and the block
+decoding loop.
+
+The pages (the arXiv abstract page "DiffusionGemma 技术报告" and the
+laozijiushiniubi.cn article "谷歌DeepMind如何将一台'逐字打稿机'改造成
+'整段喷墨机'", §一, §二, §四) describe generation as: encode the prompt
+causally; start a 256-token block from uniformly random tokens; refine every
+position in parallel each round; lock confident positions and re-randomise
+the others; stop adaptively; the block then becomes context for the next one.
+
+One step, in order (steps a1-a9):
+  a1  x0 = E_emb[canvas] (+ bf16(e_prev) W_sc^T when self-conditioning)
+  a2-a6 the transformer layers over the canvas (forward_layers, no mask,
+      canvas keys not kept)
+  a7  LM-head logits and per-position H, pmax, argmax, Gumbel sample at T_s
+  a8  the expected embedding e = sum_v softmax(l)_v E_emb[v] (next step's
+      self-conditioning input)
+  a9  mean entropy, stop flag, lock mask, and the next canvas: locked
+      positions keep their sample, the others get uniform random tokens; on
+      stop (or at the last budgeted step) the canvas becomes the argmax
+      sequence and the canvas is frozen.
+
+Canvases of a batch are independent (own context, own random stream, own stop).
+"""
+
+from dataclasses import dataclass, field
+
+import numpy as np
+
+from . import sampler as smp
+from .model import ModelConfig, Weights, KVCache, forward_layers, lm_logits
+from .numerics import f32_round
+from .philox import method_draw, uniform_token, PURPOSE_INIT
+
+
+@dataclass
+class CanvasState:
+    tokens: np.ndarray            # [B, N] int64
+    sc: np.ndarray                # [B, N, d] float64 (bf16 values); zeros before step 0
+    prev_argmax: np.ndarray       # [B, N] int64, -1 before step 0
+    done: np.ndarray              # [B] bool
+
+
+@dataclass
+class StepOutput:
+    logits: np.ndarray            # [B, N, V] float32
+    argmax: np.ndarray            # [B, N]
+    sample: np.ndarray            # [B, N]
+    entropy: np.ndarray           # [B, N] float64
+    pmax: np.ndarray              # [B, N] float64
+    mean_entropy: np.ndarray      # [B]
+    stop: np.ndarray              # [B] bool (stopped at this step)
+    final: np.ndarray             # [B] bool (stopped, or the last budgeted step)
+    lock: np.ndarray              # [B, N] bool
+    tokens_in: np.ndarray         # [B, N] canvas the step consumed
+    tokens_out: np.ndarray        # [B, N] canvas after the update
+    sample_margin: np.ndarray     # [B, N] top-2 gap of the Gumbel keys
+    argmax_margin: np.ndarray     # [B, N] top-2 gap of the logits
+    routing: list = field(default_factory=list)  # per layer (idx [B,N,k], w [B,N,k])
+    expected_emb: np.ndarray = None
+
+
+def init_canvas(seed: int, block: int, batch: int, n_pos: int, vocab: int) -> np.ndarray:
+    """Uniform random starting tokens (draw purpose 1)."""
+    toks = np.empty((batch, n_pos), np.int64)
+    for b in range(batch):
+        w0, _, _, _ = method_draw(seed, PURPOSE_INIT, b, block, 0, np.arange(n_pos, dtype=np.uint64))
+        toks[b] = uniform_token(w0, vocab)
+    return toks
+
+
+def new_state(tokens, d_model) -> CanvasState:
+    B, N = tokens.shape
+    return CanvasState(tokens=np.array(tokens, np.int64), sc=np.zeros((B, N, d_model)),
+                       prev_argmax=np.full((B, N), -1, np.int64), done=np.zeros(B, bool))
+
+
+def encode_context(cfg: ModelConfig, W: Weights, kv: KVCache, tokens):
+    """Causal encoding of tokens [B, n] appended at kv.length (keys stored)."""
+    tokens = np.asarray(tokens)
+    B, n = tokens.shape
+    x = W.emb_rows(tokens).reshape(B, n, cfg.d_model)
+    forward_layers(cfg, W, x, kv, causal=True, append=True)
+
+
+def _top2_gap(v):
+    v = np.asarray(v, dtype=np.float64)
+    if v.size < 2:
+        return np.inf
+    top = np.partition(v, -2)[-2:]
+    return float(top[1] - top[0])
+
+
+def denoise_step(cfg: ModelConfig, W: Weights, kv: KVCache, state: CanvasState,
+                 sc: smp.SamplerConfig, block: int, step: int, keep_logits: bool = True,
+                 record_routing: bool = False) -> StepOutput:
+    """One denoising round over every canvas of the batch; updates `state`."""
+    B, N = state.tokens.shape
+    d, V = cfg.d_model, cfg.vocab
+    tokens_in = state.tokens.copy()
+
+    # a1: canvas embedding plus the self-conditioning input
+    x = W.emb_rows(tokens_in).reshape(B, N, d)
+    if cfg.self_cond:
+        x = f32_round(x + f32_round(state.sc.reshape(B * N, d) @ W.sc().T).reshape(B, N, d))
+
+    # a2-a6: transformer layers, bidirectional over the canvas
+    routing = [] if record_routing else None
+    x = forward_layers(cfg, W, x, kv, causal=False, append=False, record=routing)
+
+    # a7: logits and per-position statistics / samples
+    logits = lm_logits(cfg, W, x.reshape(B * N, d)).reshape(B, N, V)
+    inv_t = smp.inv_temperature_f32(step, sc.max_steps, sc.t_start, sc.t_end)
+    H = np.empty((B, N))
+    pmax = np.empty((B, N))
+    amax = np.empty((B, N), np.int64)
+    samp = np.empty((B, N), np.int64)
+    s_gap = np.empty((B, N))
+    a_gap = np.empty((B, N))
+    probs = np.empty((B, N, V)) if cfg.self_cond else None
+    for b in range(B):
+        for i in range(N):
+            H[b, i], pmax[b, i], amax[b, i], p = smp.position_stats(logits[b, i])
+            samp[b, i], keys = smp.position_sample(logits[b, i], inv_t, sc.seed, b, block, step, i)
+            s_gap[b, i] = _top2_gap(keys)
+            a_gap[b, i] = _top2_gap(logits[b, i])
+            if probs is not None:
+                probs[b, i] = p
+
+    # a8: expected embedding for the next round's self-conditioning input
+    e_new = None
+    if cfg.self_cond:
+        e_new = smp.expected_embedding(probs.reshape(B * N, V), W).reshape(B, N, d)
+
+    # a9: stop, lock and the next canvas
+    meanH = H.mean(axis=1)
+    stop = np.zeros(B, bool)
+    final = np.zeros(B, bool)
+    lock = np.zeros((B, N), bool)
+    for b in range(B):
+        lock[b] = smp.lock_mask(H[b], pmax[b], sc.lock_policy, sc.lock_threshold)
+        if state.done[b]:
+            continue
+        prev = state.prev_argmax[b] if step > 0 else None
+        stop[b] = smp.stop_flag(meanH[b], sc.stop_entropy, sc.stop_require_stable_argmax, step,
+                                amax[b], prev)
+        final[b] = stop[b] or step == sc.max_steps - 1
+        if final[b]:
+            state.tokens[b] = amax[b]
+            state.done[b] = True
+        else:
+            noise = smp.renoise_tokens(sc.seed, b, block, step, N, V)
+            state.tokens[b] = np.where(lock[b], samp[b], noise)
+        state.prev_argmax[b] = amax[b]
+        if cfg.self_cond:
+            state.sc[b] = e_new[b]
+
+    return StepOutput(logits=logits if keep_logits else None, argmax=amax, sample=samp, entropy=H,
+                      pmax=pmax, mean_entropy=meanH, stop=stop, final=final, lock=lock,
+                      tokens_in=tokens_in, tokens_out=state.tokens.copy(), sample_margin=s_gap,
+                      argmax_margin=a_gap, routing=routing or [], expected_emb=e_new)
+
+
+def decode_block(cfg: ModelConfig, W: Weights, kv: KVCache, sc: smp.SamplerConfig, block: int,
+                 batch: int, keep_logits: bool = False, on_step=None):
+    """Generate one block per canvas: initialise, step until every canvas has
+    stopped or the budget is spent, then append the block to the context.
+    Returns (tokens [B, N], steps taken per canvas [B], list of StepOutput)."""
+    N = cfg.canvas
+    state = new_state(init_canvas(sc.seed, block, batch, N, cfg.vocab), cfg.d_model)
+    steps = np.zeros(batch, np.int64)
+    outs = []
+    for s in range(sc.max_steps):
+        active = ~state.done
+        o = denoise_step(cfg, W, kv, state, sc, block, s, keep_logits=keep_logits)
+        steps[active] += 1
+        outs.append(o)
+        if on_step is not None:
+            on_step(s, o)
+        if state.done.all():
+            break
+    tokens = state.tokens.copy()
+    encode_context(cfg, W, kv, tokens)
+    return tokens, steps, outs
+

@@ -1,0 +1,196 @@
+"""Pins of the oracle's transformer pieces against closed forms, invariants
+and independent formulations (no GPU)."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import model as M
+from oracle.numerics import bf16_round, f32_round
+
+
+# ---- rounding helpers -------------------------------------------------------
+
+def test_bf16_round_ties_to_even():
+    one = 1.0
+    ulp = 2.0 ** -7  # bf16 spacing in [1, 2)
+    assert bf16_round(one + ulp / 2) == one                 # tie, even stays
+    assert bf16_round(one + 3 * ulp / 2) == one + 2 * ulp   # tie, odd rounds up
+    assert bf16_round(one + ulp / 2 + 2.0 ** -30) == one + ulp
+    assert bf16_round(-(one + 3 * ulp / 2)) == -(one + 2 * ulp)
+    assert bf16_round(0.0) == 0.0
+
+
+def test_bf16_round_matches_torch_on_float32_inputs():
+    rng = np.random.default_rng(0)
+    x = (rng.standard_normal(100000) * np.exp(rng.uniform(-20, 20, 100000))).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(bf16_round(x.astype(np.float64)), ref)
+
+
+def test_f32_round():
+    assert f32_round(1.0 + 2.0 ** -30) == 1.0
+    assert f32_round(1.0 + 2.0 ** -23) == 1.0 + 2.0 ** -23
+
+
+# ---- RMSNorm, RoPE, SwiGLU ----------------------------------------------------
+
+def test_rmsnorm_closed_form():
+    x = np.array([3.0, 4.0])
+    rms = math.sqrt((9 + 16) / 2 + 1e-6)
+    assert np.allclose(M.rmsnorm(x, 1e-6), x / rms, rtol=0, atol=1e-15)
+    assert np.allclose(M.rmsnorm(x, 1e-6, gain=np.array([2.0, 0.5])), x / rms * [2.0, 0.5])
+
+
+def test_rope_identity_at_position_zero():
+    x = np.random.default_rng(1).standard_normal((3, 2, 8))
+    assert np.allclose(M.rope(x, np.zeros(3), 10000.0), x, atol=0)
+
+
+def test_rope_relative_position_and_norm():
+    rng = np.random.default_rng(2)
+    q = rng.standard_normal((1, 1, 16))
+    k = rng.standard_normal((1, 1, 16))
+    dots = []
+    for shift in (0, 5, 1000):
+        qr = M.rope(q, np.array([7 + shift]), 10000.0)
+        kr = M.rope(k, np.array([3 + shift]), 10000.0)
+        dots.append(float((qr * kr).sum()))
+        assert np.isclose(np.linalg.norm(qr), np.linalg.norm(q))
+    assert np.allclose(dots, dots[0], rtol=1e-10)
+
+
+def test_rope_pairs_rotate_halves():
+    # one pair (i, i + hd/2) at position p rotates by p * theta^(-2i/hd)
+    hd, i, p, theta = 8, 1, 3, 10000.0
+    x = np.zeros((1, 1, hd))
+    x[0, 0, i] = 1.0
+    ang = p * theta ** (-2.0 * i / hd)
+    r = M.rope(x, np.array([p]), theta)[0, 0]
+    assert np.isclose(r[i], math.cos(ang)) and np.isclose(r[i + hd // 2], math.sin(ang))
+    assert np.allclose(np.delete(r, [i, i + hd // 2]), 0)
+
+
+def test_silu_and_expert_closed_form():
+    assert M.silu(np.array([0.0]))[0] == 0.0
+    assert np.isclose(M.silu(np.array([1.0]))[0], 1 / (1 + math.exp(-1)))
+    # one-hot weights pick single products: y = silu(a) * u * wd
+    x = np.array([[1.0, 0.0]])
+    wg = np.array([[2.0, 0.0]])
+    wu = np.array([[0.5, 0.0]])
+    wd = np.array([[1.0], [0.0]])
+    want = bf16_round(2.0 / (1 + math.exp(-2.0)) * 0.5)
+    assert np.isclose(M.expert_ffn(x, wg, wu, wd)[0, 0], want)
+
+
+# ---- attention ----------------------------------------------------------------
+
+def _attention_loop(q, k, v, q_pos, k_pos, causal):
+    """A second formulation: per query and head, log-sum-exp weighted sum."""
+    nq, Hq, hd = q.shape
+    group = Hq // k.shape[1]
+    out = np.zeros_like(q)
+    for i in range(nq):
+        for h in range(Hq):
+            g = h // group
+            keys = [j for j in range(k.shape[0]) if not causal or k_pos[j] <= q_pos[i]]
+            s = [sum(q[i, h, t] * k[j, g, t] for t in range(hd)) / math.sqrt(hd) for j in keys]
+            lse = max(s) + math.log(sum(math.exp(a - max(s)) for a in s))
+            for j, a in zip(keys, s):
+                out[i, h] += math.exp(a - lse) * v[j, g]
+    return out
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_attention_matches_second_formulation(causal):
+    rng = np.random.default_rng(3)
+    q = rng.standard_normal((5, 4, 6))
+    k = rng.standard_normal((7, 2, 6))
+    v = rng.standard_normal((7, 2, 6))
+    q_pos = np.arange(2, 7)
+    k_pos = np.arange(7)
+    got = M.attention(q, k, v, q_pos, k_pos, causal)
+    assert np.allclose(got, _attention_loop(q, k, v, q_pos, k_pos, causal), atol=1e-12)
+
+
+def test_attention_permutation_equivariant_without_mask():
+    rng = np.random.default_rng(4)
+    n, ctx = 9, 4
+    q = rng.standard_normal((n, 2, 8))
+    kc = rng.standard_normal((n, 1, 8))
+    vc = rng.standard_normal((n, 1, 8))
+    kx = rng.standard_normal((ctx, 1, 8))
+    vx = rng.standard_normal((ctx, 1, 8))
+    perm = rng.permutation(n)
+    pos = np.arange(ctx, ctx + n)
+    kp = np.arange(ctx + n)
+    a = M.attention(q, np.concatenate([kx, kc]), np.concatenate([vx, vc]), pos, kp, False)
+    b = M.attention(q[perm], np.concatenate([kx, kc[perm]]), np.concatenate([vx, vc[perm]]),
+                    pos, kp, False)
+    assert np.allclose(a[perm], b, atol=1e-12)
+
+
+def test_attention_equal_keys_give_mean_of_values():
+    rng = np.random.default_rng(5)
+    k = np.repeat(rng.standard_normal((1, 1, 8)), 6, axis=0)
+    v = rng.standard_normal((6, 1, 8))
+    q = rng.standard_normal((3, 1, 8))
+    out = M.attention(q, k, v, np.arange(3), np.arange(6), False)
+    assert np.allclose(out, v.mean(axis=0, keepdims=True), atol=1e-12)
+
+
+def test_causal_first_row_sees_only_itself():
+    rng = np.random.default_rng(6)
+    q, k, v = (rng.standard_normal((4, 1, 8)) for _ in range(3))
+    out = M.attention(q, k, v, np.arange(4), np.arange(4), True)
+    assert np.allclose(out[0], v[0])
+
+
+# ---- routing / mixture of experts --------------------------------------------
+
+def _toy_layer(rng, E, d, f):
+    from oracle.numerics import f64_to_bf16_bits
+    mk = lambda *s: bf16_round(rng.standard_normal(s) * 0.3)  # noqa: E731
+    return {"wr": mk(E, d), "wg": f64_to_bf16_bits(mk(E, f, d)), "wu": f64_to_bf16_bits(mk(E, f, d)),
+            "wd": f64_to_bf16_bits(mk(E, d, f))}
+
+
+def test_moe_topk_all_equals_dense_softmax_mixture():
+    from oracle.numerics import bf16_bits_to_f64 as dec
+    rng = np.random.default_rng(7)
+    E, d, f = 4, 8, 6
+    layer = _toy_layer(rng, E, d, f)
+    h = bf16_round(rng.standard_normal((5, d)))
+    out, idx, w = M.moe_ffn(h, layer, top_k=E)
+    logits = f32_round(h @ layer["wr"].T)
+    p = np.exp(logits - logits.max(1, keepdims=True))
+    p /= p.sum(1, keepdims=True)
+    dense = sum(p[:, [e]] * M.expert_ffn(h, dec(layer["wg"][e]), dec(layer["wu"][e]),
+                                         dec(layer["wd"][e])) for e in range(E))
+    assert np.allclose(out, dense, rtol=1e-6, atol=1e-6)
+
+
+def test_moe_single_expert_is_plain_ffn():
+    from oracle.numerics import bf16_bits_to_f64 as dec
+    rng = np.random.default_rng(8)
+    layer = _toy_layer(rng, 1, 8, 6)
+    h = bf16_round(rng.standard_normal((3, 8)))
+    out, idx, w = M.moe_ffn(h, layer, top_k=1)
+    assert np.all(idx == 0) and np.all(w == 1.0)
+    assert np.array_equal(out, M.expert_ffn(h, dec(layer["wg"][0]), dec(layer["wu"][0]),
+                                            dec(layer["wd"][0])))
+
+
+def test_route_weights_sum_to_one_and_ties_go_low():
+    wr = np.array([[1.0, 0.0], [1.0, 0.0], [0.5, 0.0], [1.0, 0.0]])  # experts 0, 1, 3 tie
+    h = np.array([[1.0, 2.0]])
+    idx, w, _ = M.route(h, wr, 2)
+    assert list(idx[0]) == [0, 1]
+    assert np.isclose(w.sum(), 1.0) and np.allclose(w, 0.5)
+    rng = np.random.default_rng(9)
+    idx, w, logits = M.route(rng.standard_normal((20, 8)), rng.standard_normal((16, 8)), 4)
+    assert np.allclose(w.sum(1), 1.0, atol=1e-6)
+    for t in range(20):
+        assert set(idx[t]) == set(np.argsort(-logits[t], kind="stable")[:4])

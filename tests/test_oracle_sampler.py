@@ -1,0 +1,160 @@
+"""Pins of the oracle's vocabulary statistics, sampler, lock rules, stop rule,
+temperature schedule and expected embedding (no GPU)."""
+
+import itertools
+import math
+
+import numpy as np
+import pytest
+
+from oracle import sampler as S
+from oracle import philox
+
+
+def test_uniform_logits_entropy_is_log_v():
+    for V in (4096, 262144):
+        H, pmax, amax, p = S.position_stats(np.zeros(V, np.float32))
+        assert abs(H - math.log(V)) < 1e-9
+        assert abs(pmax - 1.0 / V) < 1e-15
+        assert amax == 0  # ties go to the lower id
+        assert abs(p.sum() - 1.0) < 1e-12
+    assert abs(math.log(262144) - 12.4766) < 1e-4
+
+
+def test_two_level_logits_closed_form():
+    # one logit a, V-1 logits 0: p1 = e^a / (e^a + V - 1)
+    V, a = 1000, 3.0
+    l = np.zeros(V, np.float32)
+    l[17] = a
+    H, pmax, amax, p = S.position_stats(l)
+    Z = math.exp(a) + V - 1
+    p1, p0 = math.exp(a) / Z, 1.0 / Z
+    assert abs(pmax - p1) < 1e-12 and amax == 17
+    assert abs(H - (-(p1 * math.log(p1)) - (V - 1) * p0 * math.log(p0))) < 1e-10
+
+
+def test_entropy_bounds_random_logits():
+    rng = np.random.default_rng(0)
+    for scale in (0.01, 1.0, 30.0):
+        l = (rng.standard_normal(5000) * scale).astype(np.float32)
+        H, pmax, amax, p = S.position_stats(l)
+        assert 0.0 <= H <= math.log(5000) + 1e-12
+        assert abs(p.sum() - 1.0) < 1e-12
+        assert amax == int(np.argmax(l))
+
+
+def test_gumbel_max_frequencies_match_softmax():
+    logits = np.array([0.0, 0.5, 1.0, -1.0, 2.0, 0.2, -0.3, 1.5], np.float32)
+    inv_t = np.float32(1.0 / 0.7)
+    n = 60000
+    # independent draws: 60000 positions of the counter space, two Philox
+    # blocks (c0 = 0, 1) give the 8 per-id words of each draw
+    pos = np.arange(n, dtype=np.uint64)
+    words = np.stack(philox.method_draw(99, philox.PURPOSE_GUMBEL, 0, 0, 0, pos, 0), axis=1)
+    words = np.concatenate([words, np.stack(philox.method_draw(99, philox.PURPOSE_GUMBEL, 0, 0, 0,
+                                                               pos, 1), axis=1)], axis=1)
+    keys = (logits * inv_t)[None, :] + (-np.log(-np.log(philox.gumbel_u(words))))
+    counts = np.bincount(np.argmax(keys, axis=1), minlength=8)
+    p = np.exp(logits.astype(np.float64) * float(inv_t))
+    p /= p.sum()
+    exp = n * p
+    chi2 = float(((counts - exp) ** 2 / exp).sum())
+    assert chi2 < 40, chi2  # 7 degrees of freedom; p < 1e-5 beyond ~33
+
+
+def test_gumbel_sample_low_temperature_is_argmax():
+    rng = np.random.default_rng(1)
+    l = rng.standard_normal(300).astype(np.float32)
+    words = philox.gumbel_words(5, 0, 0, 0, 3, 300)
+    tok, _ = S.gumbel_sample(l, np.float32(1e6), words)
+    assert tok == int(np.argmax(l))
+
+
+def test_gumbel_words_layout():
+    w = philox.gumbel_words(11, 2, 1, 3, 7, 10)
+    blk = philox.method_draw(11, philox.PURPOSE_GUMBEL, 2, 1, 3, 7, 2)  # c0 = 2 covers ids 8..11
+    assert int(w[8]) == int(blk[0]) and int(w[9]) == int(blk[1])
+
+
+def test_temperature_schedule():
+    assert S.temperature(0, 48) == 0.8
+    assert abs(S.temperature(47, 48) - 0.4) < 1e-15
+    assert abs(S.temperature(1, 3) - 0.6) < 1e-15
+    assert [round(S.temperature(s, 4), 4) for s in range(4)] == [0.8, 0.6667, 0.5333, 0.4]
+    assert S.temperature(0, 1) == 0.8
+
+
+def test_prob_lock_is_strict_threshold():
+    pmax = np.array([0.9, 0.9 + 1e-9, 0.5, 0.99])
+    assert list(S.lock_mask(np.zeros(4), pmax, S.LOCK_PROB, 0.9)) == [False, True, False, True]
+
+
+def _cumsum_lock_brute(H, theta):
+    """Independent formulation: i is locked iff the total entropy of all
+    positions ordered at or before i (by (H, index)) is <= theta."""
+    n = len(H)
+    out = np.zeros(n, bool)
+    for i in range(n):
+        before = [j for j in range(n) if (H[j], j) <= (H[i], i)]
+        out[i] = sum(H[j] for j in before) <= theta
+    return out
+
+
+def test_cumsum_lock_matches_enumeration():
+    rng = np.random.default_rng(2)
+    for trial in range(300):
+        H = rng.choice([0.0, 0.01, 0.02, 0.05, 0.1, 0.3], size=8) * rng.uniform(0.5, 1.5)
+        if trial % 3 == 0:
+            H = rng.exponential(0.04, size=8)
+        got = S.lock_mask(H, np.zeros(8), S.LOCK_ENTROPY_CUMSUM, 0.1)
+        assert np.array_equal(got, _cumsum_lock_brute(list(H), 0.1)), H
+    # every subset size reachable; the crossing position is not locked
+    H = np.array([0.05, 0.04, 0.02, 0.5])
+    assert list(S.lock_mask(H, None, S.LOCK_ENTROPY_CUMSUM, 0.1)) == [False, True, True, False]
+
+
+def test_stop_fires_exactly_below_threshold():
+    assert S.stop_flag(0.4999, 0.5, False, 0, None, None)
+    assert not S.stop_flag(0.5, 0.5, False, 0, None, None)
+    a = np.array([1, 2, 3])
+    assert not S.stop_flag(0.0, 0.5, True, 0, a, None)          # never at step 0
+    assert S.stop_flag(0.0, 0.5, True, 3, a, a.copy())
+    assert not S.stop_flag(0.0, 0.5, True, 3, a, np.array([1, 2, 4]))
+
+
+def test_stop_on_constructed_logits():
+    # two-level logits with entropy straddling the threshold
+    V = 100
+    def H_of(a):
+        l = np.zeros(V, np.float32)
+        l[0] = a
+        return S.position_stats(l)[0]
+    lo, hi = H_of(12.0), H_of(2.0)
+    assert lo < 0.5 < hi
+    assert S.stop_flag(np.mean([lo] * 4), 0.5, False, 1, None, None)
+    assert not S.stop_flag(np.mean([hi] * 4), 0.5, False, 1, None, None)
+    mixed = np.mean([lo, lo, lo, hi])
+    assert S.stop_flag(mixed, 0.5, False, 1, None, None) == (mixed < 0.5)
+
+
+def test_expected_embedding_one_hot_returns_row():
+    from oracle.model import ModelConfig, Weights
+    cfg = ModelConfig(1, 16, 1, 1, 16, 1, 1, 16, 64)
+    W = Weights(cfg, seed=3)
+    p = np.zeros((2, 64))
+    p[0, 5] = 1.0
+    p[1, 63] = 1.0
+    e = S.expected_embedding(p, W, chunk=16)
+    assert np.array_equal(e[0], W.emb_chunk(5, 1)[0])
+    assert np.array_equal(e[1], W.emb_chunk(63, 1)[0])
+    # uniform p gives the mean row (within bf16 rounding of the result)
+    e = S.expected_embedding(np.full((1, 64), 1 / 64), W, chunk=64)
+    assert np.allclose(e[0], W.emb_chunk(0, 64).mean(0), atol=2 ** -9 * np.abs(e).max() + 1e-6)
+
+
+def test_renoise_uniform_and_deterministic():
+    a = S.renoise_tokens(1, 0, 2, 3, 256, 4096)
+    b = S.renoise_tokens(1, 0, 2, 3, 256, 4096)
+    c = S.renoise_tokens(1, 0, 2, 4, 256, 4096)
+    assert np.array_equal(a, b) and not np.array_equal(a, c)
+    assert a.min() >= 0 and a.max() < 4096
