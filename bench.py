@@ -1,0 +1,448 @@
+#!/usr/bin/env python
+"""Benchmark of one DiffusionGemma denoising round (dg_denoise_step) on B200.
+
+Workload (default, "full"): the full-size single step — 30 layers, d_model
+2816, 16 query / 8 KV heads x 176, 128 experts top-8 (SwiGLU, ffn 704), vocab
+262144, self-conditioning projection, random-init bf16 weights N(0, 0.02)
+(seeded generator), a causally encoded context of 1024 random tokens, one
+256-token canvas (batch 1).  A step is one dg_denoise_step: embedding and
+self-conditioning input, 30 transformer layers, LM head with vocabulary
+statistics and Gumbel sampling, expected embedding, canvas update.
+
+Prints one JSON line (rank 0).  value = denoise steps/s summed over ranks
+(replicas, one per GPU; no collective on the data path).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+
+import argparse
+import ctypes
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOADS = {
+    # full-size single step: 30 layers, self-conditioning, context 1024, batch 1
+    "full": dict(cfg=dict(n_layers=30, d_model=2816, n_q_heads=16, n_kv_heads=8, head_dim=176,
+                          n_experts=128, top_k=8, d_ff=704, vocab=262144, self_cond=True),
+                 ctx=1024, batch=1),
+    # single-layer full-width step: context 2048, no self-conditioning
+    "layer1": dict(cfg=dict(n_layers=1, d_model=2816, n_q_heads=16, n_kv_heads=8, head_dim=176,
+                            n_experts=128, top_k=8, d_ff=704, vocab=262144, self_cond=False),
+                   ctx=2048, batch=1),
+    # tiny: 2 layers, d 256, 16 experts top-2, vocab 4096, context 64
+    "tiny": dict(cfg=dict(n_layers=2, d_model=256, n_q_heads=8, n_kv_heads=8, head_dim=32, n_experts=16,
+                          top_k=2, d_ff=512, vocab=4096, self_cond=False),
+                 ctx=64, batch=1),
+}
+METRIC = "denoise steps/s on 256-token canvas"
+UNIT = "steps/s"
+CANVAS = 256
+MAX_STEPS = 48
+SEED = 7
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        j = json.load(open(p))
+        return dict(hbm_gbs=j["hbm_gbs"], bf16_tflops=j["bf16_tflops"],
+                    bf16_tflops_sustained=j.get("bf16_tflops_sustained", j["bf16_tflops"]),
+                    source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+def step_cost(cfg, batch, ctx, distinct_per_layer):
+    """Algorithmic FLOPs and HBM bytes of one denoising round."""
+    d, hd, Hq, Hkv, E, k, f, V, L = (cfg[x] for x in ("d_model", "head_dim", "n_q_heads", "n_kv_heads",
+                                                      "n_experts", "top_k", "d_ff", "vocab", "n_layers"))
+    T = batch * CANVAS
+    qkv_rows = (Hq + 2 * Hkv) * hd
+    keys = ctx + CANVAS
+    flops = 0.0
+    bytes_ = 0.0
+    for l in range(L):
+        macs = T * (qkv_rows * d + d * Hq * hd + E * d + k * 3 * f * d)
+        flops += 2.0 * macs + 4.0 * batch * CANVAS * Hq * hd * keys
+        bytes_ += 2.0 * (qkv_rows * d + d * Hq * hd + E * d)
+        bytes_ += distinct_per_layer[l] * 3 * f * d * 2.0
+        bytes_ += 2.0 * batch * Hkv * keys * hd * 2  # K and V of the context and the canvas
+    flops += 2.0 * T * V * d  # LM head
+    bytes_ += V * d * 2.0
+    if cfg["self_cond"]:
+        flops += 2.0 * T * V * d + 2.0 * T * d * d
+        bytes_ += V * d * 2.0 + d * d * 2.0
+    return flops, bytes_
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"dg_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = [r.split(",") for r in open(self.path).read().strip().splitlines() if r.strip()]
+        os.unlink(self.path)
+        sm, smax, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for r in rows:
+            try:
+                sm.append(float(r[1].split()[0]))
+                smax.append(float(r[2].split()[0]))
+            except (ValueError, IndexError):
+                continue
+            for nm, v in zip(names, r[5:9]):
+                if "Active" in v and "Not" not in v:
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for rel in ("discrete_diffusion_moe_b200/csrc/gemm_tc.cuh", "discrete_diffusion_moe_b200/csrc/epilogues.cuh",
+                "discrete_diffusion_moe_b200/csrc/common.cuh"):
+        h.update(open(os.path.join(ROOT, rel), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_key):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary, or None when missing or taken on a different kernel source."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(p):
+        return None
+    j = json.load(open(p))
+    e = j.get(kernel_key)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("bytes_per_launch_full")
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the oracle, timed on a bounded sample of the workload
+
+def oracle_sample(wl, threads):
+    """Time the oracle on a sample of one step and scale it to the whole
+    step.  Sample: transformer layer 0 over the 256 canvas tokens (keys: a
+    synthetic context of the workload's length + the canvas), the LM head over
+    one 16384-id block of the vocabulary, and the per-position statistics,
+    Gumbel sample and expected embedding of 8 positions over the full
+    vocabulary.  Weights are generated before timing (inputs).  Returns
+    (seconds per step, description)."""
+    import numpy as np
+    import oracle
+    import synth
+    from oracle import decode as OD
+    from oracle import sampler as OS
+    from oracle.model import forward_layers, lm_logits
+    c = wl["cfg"]
+    ocfg1 = oracle.ModelConfig(**dict(c, n_layers=1))
+    W = oracle.Weights(ocfg1, seed=0, threads=threads, keep_chunks=True)
+    W.layer(0)
+    ctx = wl["ctx"]
+    kv = oracle.KVCache(ocfg1, 1, ctx + CANVAS)
+    kv.k[0][:, :ctx] = synth.f32_tensor(ctx * c["n_kv_heads"] * c["head_dim"], 3, 900, 1.0).reshape(
+        1, ctx, c["n_kv_heads"], c["head_dim"])
+    kv.v[0][:, :ctx] = synth.f32_tensor(ctx * c["n_kv_heads"] * c["head_dim"], 3, 901, 1.0).reshape(
+        1, ctx, c["n_kv_heads"], c["head_dim"])
+    kv.length = ctx
+    toks = OD.init_canvas(SEED, 0, 1, CANVAS, c["vocab"])
+    x0 = W.emb_rows(toks).reshape(1, CANVAS, c["d_model"])
+    chunk = 16384
+    vcfg = oracle.ModelConfig(**dict(c, n_layers=1, vocab=chunk))
+    Wv = oracle.Weights(vcfg, seed=0, threads=threads, keep_chunks=True)
+    Wv.lm_chunk(0, chunk)
+    n_pos = 8
+    W.emb_chunk(0, chunk)
+    t0 = time.perf_counter()
+    x = forward_layers(ocfg1, W, x0, kv, causal=False, append=False)
+    t1 = time.perf_counter()
+    lm_logits(vcfg, Wv, x.reshape(CANVAS, -1), chunk=chunk)
+    t2 = time.perf_counter()
+    rng_logits = synth.f32_tensor(n_pos * c["vocab"], 5, 902, 1.0).reshape(n_pos, c["vocab"])
+    probs = []
+    for i in range(n_pos):
+        _, _, _, p = OS.position_stats(rng_logits[i])
+        OS.position_sample(rng_logits[i], np.float32(1.25), SEED, 0, 0, 0, i)
+        probs.append(p)
+    t3 = time.perf_counter()
+    t4 = t3
+    if c["self_cond"]:
+        vc = oracle.ModelConfig(**dict(c, n_layers=1, vocab=chunk))
+        We = oracle.Weights(vc, seed=0, threads=threads, keep_chunks=True)
+        We._chunks[(synth.KIND_EMB, 0, chunk)] = W.emb_chunk(0, chunk)
+        p_all = np.full((CANVAS, chunk), 1.0 / c["vocab"])
+        t3 = time.perf_counter()
+        OS.expected_embedding(p_all, We, chunk=chunk)
+        t4 = time.perf_counter()
+    per_step = ((t1 - t0) * c["n_layers"] + (t2 - t1) * (c["vocab"] / chunk)
+                + (t3 - t2) * (CANVAS / n_pos) + (t4 - t3) * (c["vocab"] / chunk))
+    desc = (f"oracle (numpy float64) timed on: layer 0 of {c['n_layers']} over the 256-token canvas with "
+            f"{ctx} context keys (x{c['n_layers']}), LM head over 16384 of {c['vocab']} ids "
+            f"(x{c['vocab'] // chunk}), statistics and Gumbel sample of {n_pos} of 256 positions "
+            f"(x{CANVAS // n_pos}), expected embedding over 16384 ids (x{c['vocab'] // chunk}); "
+            f"weight generation excluded")
+    return per_step, desc, t4 - t0
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+def reference_arm(args, wl, rank, world):
+    if rank != 0:
+        return 0
+    cores = cpu_cores()
+    times = []
+    desc = ""
+    for i in range(args.warmup + args.steps):
+        per_step, desc, _ = oracle_sample(wl, threads=cores)
+        if i >= args.warmup:
+            times.append(per_step)
+    v = 1.0 / statistics.mean(times)
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * statistics.mean(times),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(args, wl, world),
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(args, wl, world):
+    c = wl["cfg"]
+    return {"workload": {"full": "full-size single step (30 layers, self-conditioning, context 1024, batch 1)",
+                         "layer1": "single-layer full-width step (context 2048, batch 1)",
+                         "tiny": "tiny 2-layer step (context 64, batch 1)"}[args.workload],
+            "n_layers": c["n_layers"], "d_model": c["d_model"], "heads": f"{c['n_q_heads']}q/{c['n_kv_heads']}kv x {c['head_dim']}",
+            "experts": f"{c['n_experts']} top-{c['top_k']} ffn {c['d_ff']}", "vocab": c["vocab"],
+            "self_cond": bool(c["self_cond"]), "context": wl["ctx"], "canvas": CANVAS, "batch_per_gpu": wl["batch"],
+            "global_batch": wl["batch"] * world, "parallelism": f"replicas x{world}",
+            "l2": "inputs larger than L2: every step streams the full weight set (no flush needed)"
+            if args.workload != "tiny" else "L2 flushed between steps (256 MiB write)",
+            "weights": "random-init bf16, seeded generator, std 0.02"}
+
+
+# ---------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="full", choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    wl = WORKLOADS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return reference_arm(args, wl, rank, world)
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.warmup + args.steps >= MAX_STEPS:
+        args.steps = MAX_STEPS - 1 - args.warmup
+
+    import torch
+    import torch.distributed as dist
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    import discrete_diffusion_moe_b200 as dg
+    import synth
+
+    c = wl["cfg"]
+    B, ctx = wl["batch"], wl["ctx"]
+    cfg = dg.model_config(**c)
+    stream = torch.cuda.current_stream()
+    model = dg.Model(cfg, B, seed=0)
+    kv = dg.KVCache(cfg, B, ctx + CANVAS)
+    ctx_tok = torch.from_numpy(synth.context_tokens(B, ctx, 1234 + rank, c["vocab"])).cuda()
+    model.encode(kv, ctx_tok)
+    cv = dg.Canvas(cfg, B)
+    model.canvas_init(cv, 0, SEED + rank)
+    samp = dg.sampler_config(max_steps=MAX_STEPS, stop_entropy=0.5, lock_threshold=0.9, seed=SEED + rank)
+    model.check_device()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda") if args.workload == "tiny" else None
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    step_i = 0
+    for _ in range(args.warmup):
+        model.step(kv, cv, 0, step_i, samp)
+        step_i += 1
+    barrier()
+
+    # ---- device-timed region -------------------------------------------------------
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    prof = dg.dg_profile()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    dg.check(dg.lib.dg_profile_start(model.ctx))
+    e0.record(stream)
+    for _ in range(args.steps):
+        if flush is not None:
+            flush.zero_()
+        model.step(kv, cv, 0, step_i, samp)
+        step_i += 1
+    e1.record(stream)
+    barrier()
+    dg.check(dg.lib.dg_profile_stop(model.ctx, ctypes.byref(prof)))
+    clk = clocks.stop()
+    model.check_device()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per_step = ms / args.steps
+    value = world * args.steps / (ms / 1000.0)
+
+    # ---- routing of one more round: distinct experts per layer ----------------------
+    out = dg.StepOutputs(cfg, B, routing=True)
+    model.canvas_init(cv, 1, SEED + rank)
+    model.step(kv, cv, 1, 0, samp, out)
+    torch.cuda.synchronize()
+    ridx = out.route_idx.cpu()
+    distinct = [int(torch.unique(ridx[l]).numel()) for l in range(c["n_layers"])]
+
+    # ---- end to end through the public API with host buffers -------------------------
+    e2e = None
+    if not args.no_e2e:
+        h_tok = torch.empty(B, CANVAS, dtype=torch.int32).pin_memory()
+        h_sc = torch.empty(B, CANVAS, c["d_model"], dtype=torch.bfloat16).pin_memory()
+        h_tok.copy_(cv.tokens.cpu())
+        h_sc.copy_(cv.sc_state.cpu())
+        res = dg.StepOutputs(cfg, B)
+        outs = [res.argmax, res.sample, res.entropy, res.pmax, res.lock, res.mean_entropy, res.stop,
+                res.final_round]
+        h_outs = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs]
+        h_tok_out = torch.empty_like(h_tok).pin_memory()
+        h_sc_out = torch.empty_like(h_sc).pin_memory()
+        n_e2e = max(3, min(args.steps, 10))
+        h2d = h_tok.numel() * 4 + h_sc.numel() * 2
+        d2h = h_tok_out.numel() * 4 + h_sc_out.numel() * 2 + sum(t.numel() * t.element_size() for t in outs)
+        model.canvas_init(cv, 2, SEED + rank)
+        barrier()
+        f0 = torch.cuda.Event(enable_timing=True)
+        f1 = torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for s in range(n_e2e):
+            cv.tokens.copy_(h_tok, non_blocking=True)
+            cv.sc_state.copy_(h_sc, non_blocking=True)
+            model.step(kv, cv, 2, s, samp, res)
+            h_tok_out.copy_(cv.tokens, non_blocking=True)
+            h_sc_out.copy_(cv.sc_state, non_blocking=True)
+            for d_, h_ in zip(outs, h_outs):
+                h_.copy_(d_, non_blocking=True)
+            stream.synchronize()  # the host reads the round's result
+            h_tok.copy_(h_tok_out)
+            h_sc.copy_(h_sc_out)
+        f1.record(stream)
+        barrier()
+        ms_e2e = f0.elapsed_time(f1)
+        if world > 1:
+            t = torch.tensor([ms_e2e], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms_e2e = float(t.item())
+        e2e = {"value": world * n_e2e / (ms_e2e / 1000.0), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "steps": n_e2e}
+
+    peaks = load_peaks()
+    flops, nbytes = step_cost(c, B, ctx, distinct)
+    t_roof = max(flops / (peaks["bf16_tflops_sustained"] * 1e12), nbytes / (peaks["hbm_gbs"] * 1e9))
+    # dominant kernel: grouped expert gate/up projection + SwiGLU (one launch per layer)
+    gu = dg.DG_PROF_EXPERT_GATE_UP
+    gu_ms = prof.ms[gu] / max(prof.launches[gu], 1)
+    P = B * CANVAS * c["top_k"]
+    avg_distinct = sum(distinct) / len(distinct)
+    gu_bytes = avg_distinct * 2 * c["d_ff"] * c["d_model"] * 2 + P * c["d_model"] * 2 + P * c["d_ff"] * 2
+    achieved = gu_bytes / (gu_ms / 1000.0) / 1e9
+    kinds = ["expert_gate_up", "expert_down", "lm_head", "attention", "dense_proj", "expected_emb"]
+    breakdown = {kinds[i]: {"ms_per_step": prof.ms[i] / args.steps, "launches_per_step": prof.launches[i] / args.steps}
+                 for i in range(6)}
+
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            cores = cpu_cores()
+            per_step, desc, wall = oracle_sample(wl, threads=cores)
+            cpu = {"value": 1.0 / per_step, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc,
+                   "sample_wall_s": wall}
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (random-init weights, random tokens)",
+            "config": workload_config(args, wl, world),
+            "output_tok_per_s": {"at_48_rounds_per_block": value * CANVAS / MAX_STEPS,
+                                 "projected_at_12_rounds_per_block": value * CANVAS / 12},
+            "step_roofline": {"flops": flops, "bytes": nbytes, "t_ms": 1000 * t_roof,
+                              "frac": t_roof / (ms_per_step / 1000.0),
+                              "bound": "hbm" if nbytes / (peaks["hbm_gbs"] * 1e9) >= flops / (peaks["bf16_tflops_sustained"] * 1e12) else "tensor",
+                              "peaks": f"{peaks['source']}: {peaks['hbm_gbs']} GB/s, {peaks['bf16_tflops_sustained']} TF/s sustained bf16"},
+            "roofline": {"kernel": "gemm_tc_kernel<EpiSwiGLU> (grouped expert gate/up + SwiGLU)", "bound": "hbm",
+                         "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / peaks["hbm_gbs"], "traffic": ncu_traffic("expert_gate_up"),
+                         "bytes_per_launch": gu_bytes, "launch_ms": gu_ms,
+                         "peak_source": f"{peaks['source']} (of {peaks['source']})"},
+            "kernel_breakdown": breakdown,
+            "distinct_experts_per_layer": avg_distinct,
+            "gpu_launches": int(prof.launches_total),
+            "clocks": clk,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    model.close()
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,915 @@
+// dg_api.cu - host side of the library: weight / workspace layouts, TMA
+// tensor maps, kernel orchestration of one denoising round, context encoding
+// and the block loop, behind the C ABI of include/dg.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <vector>
+
+#include "../../include/dg.h"
+#include "../../include/dg_testing.h"
+#include "../../synth/synth.h"
+#include "attention.cuh"
+#include "epilogues.cuh"
+#include "gemm_tc.cuh"
+#include "kernels.cuh"
+
+using namespace dg;
+
+// ============================================================================
+// errors
+static thread_local char g_err[512] = "";
+
+static dg_status fail(dg_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+#define DG_CUDA(call)                                                                        \
+  do {                                                                                       \
+    cudaError_t e_ = (call);                                                                 \
+    if (e_ != cudaSuccess) return fail(DG_ERR_CUDA, "%s: %s (%s:%d)", #call,                \
+                                       cudaGetErrorString(e_), __FILE__, __LINE__);          \
+  } while (0)
+
+#define DG_TRY(expr)                  \
+  do {                                \
+    dg_status s_ = (expr);            \
+    if (s_ != DG_OK) return s_;       \
+  } while (0)
+
+extern "C" const char* dg_last_error(void) { return g_err; }
+
+// ============================================================================
+// configuration checks and layouts
+static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+static int next_pow2(int x) {
+  int p = 1;
+  while (p < x) p <<= 1;
+  return p;
+}
+
+static bool cfg_ok(const dg_model_config* c, char* why, size_t n) {
+  if (!c) { snprintf(why, n, "null config"); return false; }
+  if (c->n_layers < 1 || c->d_model < 128 || c->d_model % 64) { snprintf(why, n, "d_model must be a multiple of 64, >= 128"); return false; }
+  if (c->head_dim < 16 || c->head_dim % 16 || c->head_dim > 256) { snprintf(why, n, "head_dim must be a multiple of 16 in [16, 256]"); return false; }
+  if (c->head_dim != 32 && c->head_dim != 64 && c->head_dim != 128 && c->head_dim != 176) {
+    snprintf(why, n, "head_dim %d not built (32, 64, 128, 176)", c->head_dim); return false;
+  }
+  if (c->n_q_heads < 1 || c->n_kv_heads < 1 || c->n_q_heads % c->n_kv_heads) { snprintf(why, n, "n_q_heads must be a multiple of n_kv_heads"); return false; }
+  if ((c->n_q_heads * c->head_dim) % 64) { snprintf(why, n, "n_q_heads * head_dim must be a multiple of 64"); return false; }
+  if (c->n_experts < 1 || c->n_experts > 256) { snprintf(why, n, "n_experts must be in [1, 256]"); return false; }
+  if (c->top_k < 1 || c->top_k > 8 || c->top_k > c->n_experts) { snprintf(why, n, "top_k must be in [1, min(8, n_experts)]"); return false; }
+  if (c->d_ff < 64 || c->d_ff % 64) { snprintf(why, n, "d_ff must be a multiple of 64"); return false; }
+  if (c->vocab < 256 || c->vocab % 256) { snprintf(why, n, "vocab must be a multiple of 256"); return false; }
+  if (!(c->rope_theta > 0.f) || !(c->rms_eps > 0.f)) { snprintf(why, n, "rope_theta and rms_eps must be > 0"); return false; }
+  return true;
+}
+
+namespace {
+
+struct LayerW {
+  size_t wqkv, wo, wr, wgu, wd, g_attn, g_moe;
+};
+struct WLayout {
+  size_t emb, embT, lm, sc, g_final;
+  std::vector<LayerW> layers;
+  size_t total;  // elements
+  int qkv_rows, wr_rows;
+};
+
+WLayout weight_layout(const dg_model_config& c) {
+  WLayout w;
+  size_t off = 0;
+  auto take = [&](size_t n) { size_t o = off; off = align_up(off + n, 128); return o; };
+  const size_t d = c.d_model, V = c.vocab;
+  w.qkv_rows = (c.n_q_heads + 2 * c.n_kv_heads) * c.head_dim;
+  w.wr_rows = (int)align_up(c.n_experts, 128);
+  w.emb = take(V * d);
+  w.embT = take(V * d);
+  w.lm = take(V * d);
+  w.sc = c.self_cond ? take(d * d) : 0;
+  w.g_final = take(d);
+  for (int l = 0; l < c.n_layers; ++l) {
+    LayerW L;
+    L.wqkv = take((size_t)w.qkv_rows * d);
+    L.wo = take(d * (size_t)c.n_q_heads * c.head_dim);
+    L.wr = take((size_t)w.wr_rows * d);
+    L.wgu = take((size_t)c.n_experts * 2 * c.d_ff * d);
+    L.wd = take((size_t)c.n_experts * d * c.d_ff);
+    L.g_attn = take(d);
+    L.g_moe = take(d);
+    w.layers.push_back(L);
+  }
+  w.total = off;
+  return w;
+}
+
+constexpr int kMaxAttnSplits = 8;
+
+struct WsLayout {
+  size_t err, flags, x, xn, qkv, q, attn, attn_po, attn_pml, rpart, idx, w, off, perm, inv, wperm,
+      xperm, hperm, yperm, logits, vp_m, vp_z, vp_s, vp_av, vp_ai, vp_gv, vp_gi, st_m, st_iz, st_h,
+      st_pmax, st_amax, st_samp, probs, epart, total;
+  int T_alloc, P_alloc, ks_r, n_vt, attn_rows_cap;
+  long long epart_rows;
+};
+
+int router_splits(const dg_model_config& c) { return std::min(c.d_model / 64, 16); }
+
+int esum_splits(const dg_model_config& c, int T, int num_sms) {
+  const int m_tiles = (c.d_model + 127) / 128;
+  const int n_tiles = (T + 255) / 256;
+  int ks = (2 * num_sms + m_tiles * n_tiles - 1) / (m_tiles * n_tiles);
+  ks = std::max(1, std::min(ks, 32));
+  return std::min(ks, c.vocab / 64);
+}
+
+WsLayout ws_layout(const dg_model_config& c, int batch, int num_sms) {
+  WsLayout L;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes, 256); return o; };
+  const size_t T = (size_t)batch * DG_CANVAS;
+  const size_t d = c.d_model, V = c.vocab, k = c.top_k, E = c.n_experts;
+  const size_t P = T * k;
+  const size_t hq = (size_t)c.n_q_heads * c.head_dim;
+  L.T_alloc = (int)T;
+  L.P_alloc = (int)P;
+  L.ks_r = router_splits(c);
+  L.n_vt = c.vocab / 256;
+  L.attn_rows_cap = std::max(batch, kMaxAttnSplits);
+  long long er = 0;
+  for (int b = 1; b <= batch; ++b)
+    er = std::max(er, (long long)esum_splits(c, b * DG_CANVAS, num_sms) * b * DG_CANVAS);
+  L.epart_rows = er;
+  L.err = take(64);
+  L.flags = take(std::max<size_t>(batch, 64));
+  L.x = take(T * d * 4);
+  L.xn = take(T * d * 2);
+  L.qkv = take(T * (size_t)((c.n_q_heads + 2 * c.n_kv_heads) * c.head_dim) * 4);
+  L.q = take(T * hq * 2);
+  L.attn = take(T * hq * 2);
+  L.attn_po = take((size_t)L.attn_rows_cap * DG_CANVAS * hq * 4);
+  L.attn_pml = take((size_t)L.attn_rows_cap * DG_CANVAS * c.n_q_heads * 2 * 4);
+  L.rpart = take((size_t)L.ks_r * T * E * 4);
+  L.idx = take(P * 4);
+  L.w = take(P * 4);
+  L.off = take((E + 1) * 4);
+  L.perm = take(P * 4);
+  L.inv = take(P * 4);
+  L.wperm = take(P * 4);
+  L.xperm = take(P * d * 2);
+  L.hperm = take(P * (size_t)c.d_ff * 2);
+  L.yperm = take(P * d * 4);
+  L.logits = take(T * V * 4);
+  const size_t nvp = T * (size_t)L.n_vt * 4;
+  L.vp_m = take(nvp); L.vp_z = take(nvp); L.vp_s = take(nvp); L.vp_av = take(nvp);
+  L.vp_ai = take(nvp); L.vp_gv = take(nvp); L.vp_gi = take(nvp);
+  L.st_m = take(T * 4); L.st_iz = take(T * 4); L.st_h = take(T * 4); L.st_pmax = take(T * 4);
+  L.st_amax = take(T * 4); L.st_samp = take(T * 4);
+  L.probs = c.self_cond ? take(T * V * 2) : 0;
+  L.epart = c.self_cond ? take((size_t)er * d * 4) : 0;
+  L.total = off;
+  return L;
+}
+
+// ---------------------------------------------------------------------------
+// TMA tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)p;
+  }
+  return fn;
+}
+
+// K-major bf16 matrix [rows, K] (row stride K elements), box 64 x box_rows,
+// 128-byte swizzle.
+dg_status make_tmap(CUtensorMap* m, const void* base, long long K, long long rows, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(DG_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  if (((uintptr_t)base & 15) || K % 64 || rows < 1)
+    return fail(DG_ERR_INVALID_ARG, "tensor map: bad base/K/rows (%p, %lld, %lld)", base, K, rows);
+  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(DG_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return DG_OK;
+}
+
+int device_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
+
+template <class Epi>
+dg_status run_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmPlan& p, const Epi& epi,
+                   int num_sms, cudaStream_t st, long long* launches = nullptr) {
+  if (p.bn < 16 || p.bn > 256 || (p.bn & (p.bn - 1)) || p.bn % p.b_box || p.K % 64 || p.K < 64)
+    return fail(DG_ERR_INVALID_ARG, "gemm plan: bn %d b_box %d K %d", p.bn, p.b_box, p.K);
+  static bool attr_done = false;
+  if (!attr_done) {
+    DG_CUDA(cudaFuncSetAttribute(gemm_tc_kernel<Epi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 227 * 1024));
+    attr_done = true;
+  }
+  const int stages = gemm_pick_stages(p.bn);
+  const size_t smem = gemm_smem_bytes(p.bn, stages);
+  long long units;
+  if (p.group_off) units = (long long)p.n_groups * p.m_tiles;
+  else units = (long long)p.m_tiles * ((p.n_total + p.bn - 1) / p.bn) * p.k_splits;
+  if (units <= 0) return DG_OK;
+  const int grid = (int)std::min<long long>(units, num_sms);
+  gemm_tc_kernel<Epi><<<grid, kGemmThreads, smem, st>>>(ta, tb, p, epi, stages);
+  DG_CUDA(cudaGetLastError());
+  if (launches) ++*launches;
+  return DG_OK;
+}
+
+GemmPlan dense_plan(int K, int a_rows, int n_total, int bn, int b_box, int k_splits, int* err) {
+  GemmPlan p{};
+  p.K = K;
+  p.a_rows = a_rows;
+  p.m_tiles = (a_rows + 127) / 128;
+  p.n_total = n_total;
+  p.bn = bn;
+  p.b_box = b_box;
+  p.k_splits = k_splits;
+  p.n_fast = 1;
+  p.group_off = nullptr;
+  p.err = err;
+  return p;
+}
+
+GemmPlan grouped_plan(int K, int rows_per_group, const int* off, int n_groups, int bn, int* err) {
+  GemmPlan p{};
+  p.K = K;
+  p.a_rows = rows_per_group;
+  p.m_tiles = (rows_per_group + 127) / 128;
+  p.n_total = 0;
+  p.bn = bn;
+  p.b_box = 16;
+  p.k_splits = 1;
+  p.group_off = off;
+  p.n_groups = n_groups;
+  p.a_rows_per_group = rows_per_group;
+  p.err = err;
+  return p;
+}
+
+int token_bn(int T) { return std::min(256, std::max(16, next_pow2(T))); }
+int box_for(int bn) { return std::min(64, bn); }
+
+}  // namespace
+
+// ============================================================================
+struct dg_ctx {
+  // measurement hooks: launch counter and per-class CUDA-event brackets
+  bool prof = false;
+  long long n_launch = 0;
+  std::vector<cudaEvent_t> ev_pool;
+  std::vector<std::pair<int, int>> prof_recs;  // (class, index of the start event)
+  int ev_used = 0;
+  int prof_begin(int kind, cudaStream_t st) {
+    if (!prof || prof_recs.size() >= 65536) return -1;
+    while ((int)ev_pool.size() < ev_used + 2) {
+      cudaEvent_t e;
+      if (cudaEventCreate(&e) != cudaSuccess) return -1;
+      ev_pool.push_back(e);
+    }
+    const int i = ev_used;
+    ev_used += 2;
+    cudaEventRecord(ev_pool[i], st);
+    prof_recs.push_back({kind, i});
+    return i;
+  }
+  void prof_end(int i, cudaStream_t st) {
+    if (i >= 0) cudaEventRecord(ev_pool[i + 1], st);
+  }
+  ~dg_ctx() {
+    for (cudaEvent_t e : ev_pool) cudaEventDestroy(e);
+  }
+  dg_model_config cfg;
+  const uint16_t* w;
+  uint8_t* ws;
+  size_t ws_bytes;
+  int batch_max;
+  int num_sms;
+  WLayout wl;
+  WsLayout L;
+  template <class T>
+  T* at(size_t off) const { return reinterpret_cast<T*>(ws + off); }
+  const uint16_t* wp(size_t off) const { return w + off; }
+  int* err() const { return at<int>(L.err); }
+};
+
+// Brackets the launches of one profiled class with CUDA events (no-op when
+// profiling is off).
+struct ProfScope {
+  dg_ctx* c;
+  cudaStream_t st;
+  int idx;
+  ProfScope(dg_ctx* c_, int kind, cudaStream_t s) : c(c_), st(s), idx(c_->prof_begin(kind, s)) {}
+  ~ProfScope() { c->prof_end(idx, st); }
+};
+#define CNT(c) (++(c)->n_launch)
+
+extern "C" size_t dg_weights_bytes(const dg_model_config* cfg) {
+  char why[256];
+  if (!cfg_ok(cfg, why, sizeof why)) { fail(DG_ERR_INVALID_ARG, "%s", why); return 0; }
+  return weight_layout(*cfg).total * 2;
+}
+
+extern "C" size_t dg_kv_bytes(const dg_model_config* cfg, int32_t batch, int32_t c_max) {
+  char why[256];
+  if (!cfg_ok(cfg, why, sizeof why) || batch < 1 || c_max < 1) { fail(DG_ERR_INVALID_ARG, "bad kv size query"); return 0; }
+  return (size_t)cfg->n_layers * batch * cfg->n_kv_heads * c_max * cfg->head_dim * 2;
+}
+
+extern "C" size_t dg_workspace_bytes(const dg_model_config* cfg, int32_t batch) {
+  char why[256];
+  if (!cfg_ok(cfg, why, sizeof why) || batch < 1) { fail(DG_ERR_INVALID_ARG, "bad workspace query"); return 0; }
+  return ws_layout(*cfg, batch, device_sms()).total;
+}
+
+extern "C" dg_status dg_model_init_random(const dg_model_config* cfg, uint64_t seed, const float* kind_std,
+                                          void* d_weights, void* stream) {
+  char why[256];
+  if (!cfg_ok(cfg, why, sizeof why)) return fail(DG_ERR_INVALID_ARG, "%s", why);
+  if (!d_weights || ((uintptr_t)d_weights & 255)) return fail(DG_ERR_INVALID_ARG, "weights must be 256-byte aligned");
+  const dg_model_config& c = *cfg;
+  const WLayout wl = weight_layout(c);
+  uint16_t* W = (uint16_t*)d_weights;
+  cudaStream_t st = (cudaStream_t)stream;
+  auto sd = [&](int kind) -> double {
+    return (kind_std && kind_std[kind] > 0.f) ? (double)kind_std[kind] : 0.02;
+  };
+  auto fill = [&](uint16_t* dst, long long rows, long long cols, long long sr, long long sc, uint32_t tid,
+                  int kind) -> dg_status {
+    int r = synth_fill_bf16_device(dst, 0, rows, cols, sr, sc, seed, tid, sd(kind), st);
+    if (r) return fail(DG_ERR_CUDA, "weight init: %s", cudaGetErrorString((cudaError_t)r));
+    return DG_OK;
+  };
+  auto ones = [&](uint16_t* dst, long long n) -> dg_status {
+    fill_u16_kernel<<<(unsigned)std::min<long long>((n + 255) / 256, 4096), 256, 0, st>>>(dst, n, 0x3F80);
+    DG_CUDA(cudaGetLastError());
+    return DG_OK;
+  };
+  const long long d = c.d_model, V = c.vocab, hd = c.head_dim, E = c.n_experts, f = c.d_ff;
+  DG_CUDA(cudaMemsetAsync(W, 0, wl.total * 2, st));
+  DG_TRY(fill(W + wl.emb, V, d, d, 1, SYNTH_KIND_EMB, SYNTH_KIND_EMB));
+  DG_TRY(fill(W + wl.embT, V, d, 1, V, SYNTH_KIND_EMB, SYNTH_KIND_EMB));  // transposed copy
+  DG_TRY(fill(W + wl.lm, V, d, d, 1, SYNTH_KIND_LM, SYNTH_KIND_LM));
+  if (c.self_cond) DG_TRY(fill(W + wl.sc, d, d, d, 1, SYNTH_KIND_SC, SYNTH_KIND_SC));
+  DG_TRY(ones(W + wl.g_final, d));
+  for (int l = 0; l < c.n_layers; ++l) {
+    const LayerW& L = wl.layers[l];
+    uint16_t* qkv = W + L.wqkv;
+    DG_TRY(fill(qkv, c.n_q_heads * hd, d, d, 1, synth_layer_tid(l, SYNTH_KIND_WQ), SYNTH_KIND_WQ));
+    DG_TRY(fill(qkv + (long long)c.n_q_heads * hd * d, c.n_kv_heads * hd, d, d, 1,
+                synth_layer_tid(l, SYNTH_KIND_WK), SYNTH_KIND_WK));
+    DG_TRY(fill(qkv + (long long)(c.n_q_heads + c.n_kv_heads) * hd * d, c.n_kv_heads * hd, d, d, 1,
+                synth_layer_tid(l, SYNTH_KIND_WV), SYNTH_KIND_WV));
+    DG_TRY(fill(W + L.wo, d, c.n_q_heads * hd, c.n_q_heads * hd, 1, synth_layer_tid(l, SYNTH_KIND_WO),
+                SYNTH_KIND_WO));
+    DG_TRY(fill(W + L.wr, E, d, d, 1, synth_layer_tid(l, SYNTH_KIND_WR), SYNTH_KIND_WR));
+    // gate row j of expert e -> physical row 2(e f + j), up row -> 2(e f + j) + 1
+    DG_TRY(fill(W + L.wgu, E * f, d, 2 * d, 1, synth_layer_tid(l, SYNTH_KIND_WG), SYNTH_KIND_WG));
+    DG_TRY(fill(W + L.wgu + d, E * f, d, 2 * d, 1, synth_layer_tid(l, SYNTH_KIND_WU), SYNTH_KIND_WU));
+    DG_TRY(fill(W + L.wd, E * d, f, f, 1, synth_layer_tid(l, SYNTH_KIND_WD), SYNTH_KIND_WD));
+    DG_TRY(ones(W + L.g_attn, d));
+    DG_TRY(ones(W + L.g_moe, d));
+  }
+  return DG_OK;
+}
+
+extern "C" dg_status dg_context_create(const dg_model_config* cfg, const void* d_weights, void* d_workspace,
+                                       size_t ws_bytes, int32_t batch, dg_ctx** out) {
+  if (!out) return fail(DG_ERR_INVALID_ARG, "out is null");
+  *out = nullptr;
+  char why[256];
+  if (!cfg_ok(cfg, why, sizeof why)) return fail(DG_ERR_INVALID_ARG, "%s", why);
+  if (batch < 1 || batch > 64) return fail(DG_ERR_INVALID_ARG, "batch must be in [1, 64]");
+  if (!d_weights || !d_workspace || ((uintptr_t)d_workspace & 255) || ((uintptr_t)d_weights & 255))
+    return fail(DG_ERR_INVALID_ARG, "weights and workspace must be non-null and 256-byte aligned");
+  dg_ctx* c = new (std::nothrow) dg_ctx();
+  if (!c) return fail(DG_ERR_INVALID_ARG, "host allocation failed");
+  c->cfg = *cfg;
+  c->w = (const uint16_t*)d_weights;
+  c->ws = (uint8_t*)d_workspace;
+  c->ws_bytes = ws_bytes;
+  c->batch_max = batch;
+  c->num_sms = device_sms();
+  c->wl = weight_layout(*cfg);
+  c->L = ws_layout(*cfg, batch, c->num_sms);
+  if (ws_bytes < c->L.total) {
+    size_t need = c->L.total;
+    delete c;
+    return fail(DG_ERR_WORKSPACE, "workspace too small: %zu < %zu", ws_bytes, need);
+  }
+  cudaError_t e = cudaMemset(c->ws + c->L.err, 0, 64);
+  if (e != cudaSuccess) {
+    delete c;
+    return fail(DG_ERR_CUDA, "cudaMemset: %s", cudaGetErrorString(e));
+  }
+  *out = c;
+  return DG_OK;
+}
+
+extern "C" void dg_context_destroy(dg_ctx* ctx) { delete ctx; }
+
+// ============================================================================
+// one pass of the transformer layers over T = B * nq tokens at positions
+// L0 .. L0 + nq - 1 (x already holds the embedded inputs)
+static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L0, bool causal,
+                                int32_t* dbg_idx, float* dbg_w, cudaStream_t st) {
+  const dg_model_config& m = c->cfg;
+  const WsLayout& L = c->L;
+  const int T = B * nq, d = m.d_model, hd = m.head_dim, Hq = m.n_q_heads, Hkv = m.n_kv_heads;
+  const int E = m.n_experts, k = m.top_k, f = m.d_ff, P = T * k;
+  const int qkv_rows = c->wl.qkv_rows;
+  int* err = c->err();
+  float* x = c->at<float>(L.x);
+  uint16_t* xn = c->at<uint16_t>(L.xn);
+  const int bnT = token_bn(T), boxT = box_for(bnT);
+  const int avg = std::max(1, P / E);
+  const int bnG = std::min(256, std::max(32, next_pow2(3 * avg)));
+  const size_t kv_layer = (size_t)kv->batch * Hkv * kv->c_max * hd;
+
+  CUtensorMap t_xn, t_attn, t_xperm, t_hperm;
+  DG_TRY(make_tmap(&t_xn, xn, d, L.T_alloc, boxT));
+  DG_TRY(make_tmap(&t_attn, c->at<uint16_t>(L.attn), (long long)Hq * hd, L.T_alloc, boxT));
+  DG_TRY(make_tmap(&t_xperm, c->at<uint16_t>(L.xperm), d, L.P_alloc, 16));
+  DG_TRY(make_tmap(&t_hperm, c->at<uint16_t>(L.hperm), f, L.P_alloc, 16));
+
+  // attention launch shape
+  const int q_tiles = ((Hq / Hkv) * nq + 63) / 64;
+  const int base_ctas = q_tiles * Hkv * B;
+  const int n_kt = (L0 + nq + 63) / 64;
+  int splits = std::max(1, std::min((2 * c->num_sms + base_ctas - 1) / base_ctas, kMaxAttnSplits));
+  splits = std::min(splits, n_kt);
+  while (splits > 1 && (long long)splits * B > L.attn_rows_cap) --splits;
+
+  for (int l = 0; l < m.n_layers; ++l) {
+    const LayerW& W = c->wl.layers[l];
+    uint16_t* kc = (uint16_t*)kv->k + (size_t)l * kv_layer;
+    uint16_t* vc = (uint16_t*)kv->v + (size_t)l * kv_layer;
+
+    // --- attention block ---
+    rmsnorm_kernel<256><<<T, 256, 0, st>>>(x, c->wp(W.g_attn), xn, d, m.rms_eps);
+    CNT(c);
+    {
+      ProfScope ps_(c, DG_PROF_DENSE, st);
+      CUtensorMap ta;
+      DG_TRY(make_tmap(&ta, c->wp(W.wqkv), d, qkv_rows, 128));
+      GemmPlan p = dense_plan(d, qkv_rows, T, bnT, boxT, 1, err);
+      p.a_hint = 1;
+      EpiStoreT e{c->at<float>(L.qkv), qkv_rows, 0, 0, nullptr, nullptr, 0, err};
+      DG_TRY(run_gemm(ta, t_xn, p, e, c->num_sms, st, &c->n_launch));
+    }
+    {
+      RopeParams rp{c->at<float>(L.qkv), c->at<uint16_t>(L.q), kc, vc, T, nq, L0, kv->c_max, Hq, Hkv, hd,
+                    (double)m.rope_theta};
+      rope_kv_kernel<<<std::min(4096, (T * (Hq + 2 * Hkv) * hd / 2 + 255) / 256), 256, 0, st>>>(rp);
+      CNT(c);
+    }
+    {
+      ProfScope ps_(c, DG_PROF_ATTENTION, st);
+      AttnParams ap{c->at<uint16_t>(L.q), kc, vc, c->at<uint16_t>(L.attn), c->at<float>(L.attn_po),
+                    c->at<float>(L.attn_pml), B, nq, L0, kv->c_max, Hq, Hkv, splits, causal ? 1 : 0,
+                    (float)(1.4426950408889634 / sqrt((double)hd))};
+      dim3 grid(q_tiles, Hkv, B * splits);
+      switch (hd) {
+        case 32: attn_kernel<32><<<grid, 128, attn_smem_bytes<32>(), st>>>(ap); break;
+        case 64: attn_kernel<64><<<grid, 128, attn_smem_bytes<64>(), st>>>(ap); break;
+        case 128: attn_kernel<128><<<grid, 128, attn_smem_bytes<128>(), st>>>(ap); break;
+        case 176: attn_kernel<176><<<grid, 128, attn_smem_bytes<176>(), st>>>(ap); break;
+        default: return fail(DG_ERR_UNSUPPORTED, "head_dim %d", hd);
+      }
+      CNT(c);
+      DG_CUDA(cudaGetLastError());
+      if (splits > 1) {
+        const long long n = (long long)B * Hq * nq * hd;
+        attn_combine_kernel<<<(unsigned)std::min<long long>((n + 255) / 256, 8192), 256, 0, st>>>(
+            c->at<float>(L.attn_po), c->at<float>(L.attn_pml), c->at<uint16_t>(L.attn), splits, B, Hq, nq, hd);
+            CNT(c);
+      }
+    }
+    {
+      ProfScope ps_(c, DG_PROF_DENSE, st);
+      CUtensorMap ta;
+      DG_TRY(make_tmap(&ta, c->wp(W.wo), (long long)Hq * hd, d, 128));
+      GemmPlan p = dense_plan(Hq * hd, d, T, bnT, boxT, 1, err);
+      p.a_hint = 1;
+      EpiStoreT e{x, d, 0, 1, nullptr, nullptr, 0, err};
+      DG_TRY(run_gemm(ta, t_attn, p, e, c->num_sms, st, &c->n_launch));
+    }
+
+    // --- mixture of experts block ---
+    rmsnorm_kernel<256><<<T, 256, 0, st>>>(x, c->wp(W.g_moe), xn, d, m.rms_eps);
+    CNT(c);
+    {
+      ProfScope ps_(c, DG_PROF_DENSE, st);
+      CUtensorMap ta;
+      DG_TRY(make_tmap(&ta, c->wp(W.wr), d, c->wl.wr_rows, 128));
+      GemmPlan p = dense_plan(d, E, T, bnT, boxT, L.ks_r, err);
+      EpiStoreT e{c->at<float>(L.rpart), E, (long long)T * E, 0, nullptr, nullptr, 0, err};
+      DG_TRY(run_gemm(ta, t_xn, p, e, c->num_sms, st, &c->n_launch));
+    }
+    router_topk_kernel<<<(T * 32 + 255) / 256, 256, 0, st>>>(
+        c->at<float>(L.rpart), L.ks_r, T, E, k, c->at<int>(L.idx), c->at<float>(L.w),
+        dbg_idx ? dbg_idx + (size_t)l * T * k : nullptr, dbg_w ? dbg_w + (size_t)l * T * k : nullptr);
+        CNT(c);
+    permute_kernel<<<1, kPermThreads, (size_t)34 * E * sizeof(int), st>>>(
+        c->at<int>(L.idx), c->at<float>(L.w), P, E, c->at<int>(L.off), c->at<int>(L.perm),
+        c->at<int>(L.inv), c->at<float>(L.wperm), err);
+        CNT(c);
+    gather_rows_kernel<<<P, 128, 0, st>>>(xn, c->at<int>(L.perm), c->at<uint16_t>(L.xperm), P, k, d);
+    CNT(c);
+    {
+      ProfScope ps_(c, DG_PROF_EXPERT_GATE_UP, st);
+      CUtensorMap ta;
+      DG_TRY(make_tmap(&ta, c->wp(W.wgu), d, (long long)E * 2 * f, 128));
+      GemmPlan p = grouped_plan(d, 2 * f, c->at<int>(L.off), E, bnG, err);
+      p.a_hint = 1;
+      p.b_hint = 2;
+      EpiSwiGLU e{c->at<uint16_t>(L.hperm), f};
+      DG_TRY(run_gemm(ta, t_xperm, p, e, c->num_sms, st, &c->n_launch));
+    }
+    {
+      ProfScope ps_(c, DG_PROF_EXPERT_DOWN, st);
+      CUtensorMap ta;
+      DG_TRY(make_tmap(&ta, c->wp(W.wd), f, (long long)E * d, 128));
+      GemmPlan p = grouped_plan(f, d, c->at<int>(L.off), E, bnG, err);
+      p.a_hint = 1;
+      p.b_hint = 2;
+      EpiDown e{c->at<float>(L.yperm), d, c->at<float>(L.wperm)};
+      DG_TRY(run_gemm(ta, t_hperm, p, e, c->num_sms, st, &c->n_launch));
+    }
+    moe_combine_kernel<<<T, 256, 0, st>>>(x, c->at<float>(L.yperm), c->at<int>(L.inv), T, k, d);
+    CNT(c);
+    DG_CUDA(cudaGetLastError());
+  }
+  return DG_OK;
+}
+
+static dg_status check_kv(const dg_ctx* c, const dg_kv* kv, int extra) {
+  if (!kv || !kv->k || !kv->v) return fail(DG_ERR_INVALID_ARG, "kv buffers are null");
+  if (kv->batch < 1 || kv->batch > c->batch_max) return fail(DG_ERR_INVALID_ARG, "kv batch %d outside [1, %d]", kv->batch, c->batch_max);
+  if (kv->length < 0 || kv->c_max < 1 || (long long)kv->length + extra > kv->c_max)
+    return fail(DG_ERR_INVALID_ARG, "kv length %d + %d exceeds c_max %d", kv->length, extra, kv->c_max);
+  return DG_OK;
+}
+
+static bool attn_smem_ready(int hd) {
+  static bool done[4] = {false, false, false, false};
+  int slot = hd == 32 ? 0 : hd == 64 ? 1 : hd == 128 ? 2 : 3;
+  if (done[slot]) return true;
+  cudaError_t e = cudaSuccess;
+  switch (hd) {
+    case 32: e = cudaFuncSetAttribute(attn_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, attn_smem_bytes<32>()); break;
+    case 64: e = cudaFuncSetAttribute(attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, attn_smem_bytes<64>()); break;
+    case 128: e = cudaFuncSetAttribute(attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, attn_smem_bytes<128>()); break;
+    case 176: e = cudaFuncSetAttribute(attn_kernel<176>, cudaFuncAttributeMaxDynamicSharedMemorySize, attn_smem_bytes<176>()); break;
+  }
+  done[slot] = e == cudaSuccess;
+  return done[slot];
+}
+
+extern "C" dg_status dg_encode_context(dg_ctx* c, dg_kv* kv, const int32_t* d_tokens, int32_t n, void* stream) {
+  if (!c) return fail(DG_ERR_INVALID_ARG, "null context");
+  if (n < 0) return fail(DG_ERR_INVALID_ARG, "n < 0");
+  DG_TRY(check_kv(c, kv, n));
+  if (n == 0) return DG_OK;
+  if (!d_tokens) return fail(DG_ERR_INVALID_ARG, "tokens are null");
+  if (!attn_smem_ready(c->cfg.head_dim)) return fail(DG_ERR_CUDA, "attention smem attribute");
+  cudaStream_t st = (cudaStream_t)stream;
+  const int B = kv->batch, d = c->cfg.d_model;
+  int* tok_tmp = c->at<int>(c->L.st_samp);  // [T] staging of the chunk's token ids
+  for (int s0 = 0; s0 < n; s0 += DG_CANVAS) {
+    const int nq = std::min(DG_CANVAS, n - s0);
+    const int T = B * nq;
+    // gather the chunk's tokens into a dense [B, nq] block
+    DG_CUDA(cudaMemcpy2DAsync(tok_tmp, (size_t)nq * 4, d_tokens + s0, (size_t)n * 4, (size_t)nq * 4, B,
+                              cudaMemcpyDeviceToDevice, st));
+    embed_kernel<<<T, 128, 0, st>>>(c->wp(c->wl.emb), tok_tmp, c->at<float>(c->L.x), T, d, c->cfg.vocab, c->err());
+    CNT(c);
+    DG_CUDA(cudaGetLastError());
+    DG_TRY(forward_layers(c, kv, B, nq, kv->length, true, nullptr, nullptr, st));
+    kv->length += nq;
+  }
+  return DG_OK;
+}
+
+extern "C" dg_status dg_canvas_init(dg_ctx* c, dg_canvas* cv, int32_t block, uint64_t seed, void* stream) {
+  if (!c || !cv || !cv->tokens || !cv->prev_argmax || !cv->done) return fail(DG_ERR_INVALID_ARG, "null canvas");
+  if (cv->batch < 1 || cv->batch > c->batch_max) return fail(DG_ERR_INVALID_ARG, "canvas batch");
+  if (block < 0 || block > (1 << 23)) return fail(DG_ERR_INVALID_ARG, "block index");
+  cudaStream_t st = (cudaStream_t)stream;
+  const int n = cv->batch * DG_CANVAS;
+  canvas_init_kernel<<<(n + 255) / 256, 256, 0, st>>>(cv->tokens, cv->prev_argmax, cv->done, cv->batch, block,
+                                                      (uint32_t)seed, (uint32_t)(seed >> 32), c->cfg.vocab);
+                                                      CNT(c);
+  DG_CUDA(cudaGetLastError());
+  if (c->cfg.self_cond) {
+    if (!cv->sc_state) return fail(DG_ERR_INVALID_ARG, "self-conditioning state is null");
+    DG_CUDA(cudaMemsetAsync(cv->sc_state, 0, (size_t)n * c->cfg.d_model * 2, st));
+  }
+  return DG_OK;
+}
+
+extern "C" dg_status dg_denoise_step(dg_ctx* c, const dg_kv* kv, dg_canvas* cv, const dg_step_args* a,
+                                     const dg_step_out* o, void* stream) {
+  if (!c || !cv || !a) return fail(DG_ERR_INVALID_ARG, "null argument");
+  DG_TRY(check_kv(c, kv, DG_CANVAS));
+  if (cv->batch != kv->batch) return fail(DG_ERR_INVALID_ARG, "canvas batch %d != kv batch %d", cv->batch, kv->batch);
+  if (!cv->tokens || !cv->prev_argmax || !cv->done || (c->cfg.self_cond && !cv->sc_state))
+    return fail(DG_ERR_INVALID_ARG, "canvas buffers are null");
+  const dg_sampler_config& s = a->sampler;
+  if (s.max_steps < 1 || s.max_steps > 256 || a->step < 0 || a->step >= s.max_steps || a->block < 0 ||
+      a->block > (1 << 23))
+    return fail(DG_ERR_INVALID_ARG, "step %d / max_steps %d / block %d out of range", a->step, s.max_steps, a->block);
+  if (s.lock_policy != DG_LOCK_PROB && s.lock_policy != DG_LOCK_ENTROPY_CUMSUM)
+    return fail(DG_ERR_INVALID_ARG, "lock policy");
+  if (!(s.t_start > 0.f) || !(s.t_end > 0.f)) return fail(DG_ERR_INVALID_ARG, "temperatures must be > 0");
+  if (!attn_smem_ready(c->cfg.head_dim)) return fail(DG_ERR_CUDA, "attention smem attribute");
+
+  const dg_model_config& m = c->cfg;
+  const WsLayout& L = c->L;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int B = cv->batch, T = B * DG_CANVAS, d = m.d_model, V = m.vocab;
+  int* err = c->err();
+  const int bnT = token_bn(T), boxT = box_for(bnT);
+  dg_step_out none{};
+  if (!o) o = &none;
+
+  // a1: canvas embedding (+ self-conditioning input)
+  if (m.self_cond) {
+    ProfScope ps_(c, DG_PROF_DENSE, st);
+    CUtensorMap ta, tb;
+    DG_TRY(make_tmap(&ta, c->wp(c->wl.sc), d, d, 128));
+    DG_TRY(make_tmap(&tb, cv->sc_state, d, T, boxT));
+    GemmPlan p = dense_plan(d, d, T, bnT, boxT, 1, err);
+    p.a_hint = 1;
+    EpiStoreT e{c->at<float>(L.x), d, 0, 2, c->wp(c->wl.emb), cv->tokens, V, err};
+    DG_TRY(run_gemm(ta, tb, p, e, c->num_sms, st, &c->n_launch));
+  } else {
+    embed_kernel<<<T, 128, 0, st>>>(c->wp(c->wl.emb), cv->tokens, c->at<float>(L.x), T, d, V, err);
+    CNT(c);
+    DG_CUDA(cudaGetLastError());
+  }
+
+  // a2-a6: transformer layers, bidirectional over the canvas
+  DG_TRY(forward_layers(c, kv, B, DG_CANVAS, kv->length, false, o->route_idx, o->route_w, st));
+
+  // a7: final norm, LM head with online vocabulary statistics and sampling
+  uint16_t* xn = c->at<uint16_t>(L.xn);
+  rmsnorm_kernel<256><<<T, 256, 0, st>>>(c->at<float>(L.x), c->wp(c->wl.g_final), xn, d, m.rms_eps);
+  CNT(c);
+  float* logits = o->logits ? o->logits : c->at<float>(L.logits);
+  const double Ts = s.max_steps <= 1 ? (double)s.t_start
+                                     : (double)s.t_start + ((double)s.t_end - (double)s.t_start) * a->step /
+                                                               (double)(s.max_steps - 1);
+  const float inv_t = (float)(1.0 / Ts);
+  VocabPartials vp{c->at<float>(L.vp_m), c->at<float>(L.vp_z), c->at<float>(L.vp_s), c->at<float>(L.vp_av),
+                   c->at<int>(L.vp_ai), c->at<float>(L.vp_gv), c->at<int>(L.vp_gi)};
+  {
+    ProfScope ps_(c, DG_PROF_LM_HEAD, st);
+    CUtensorMap ta, tb;
+    DG_TRY(make_tmap(&ta, xn, d, L.T_alloc, 128));
+    DG_TRY(make_tmap(&tb, c->wp(c->wl.lm), d, V, 64));
+    GemmPlan p = dense_plan(d, T, V, 256, 64, 1, err);
+    p.n_fast = 0;
+    p.a_hint = 2;
+    p.b_hint = 1;
+    EpiLMHead e{logits, V, vp, L.n_vt, 256, (uint32_t)s.seed, (uint32_t)(s.seed >> 32),
+                (uint32_t)(a->block * 256 + a->step), inv_t, DG_CANVAS};
+    DG_TRY(run_gemm(ta, tb, p, e, c->num_sms, st, &c->n_launch));
+  }
+  PosStats ps{c->at<float>(L.st_m), c->at<float>(L.st_iz), o->entropy ? o->entropy : c->at<float>(L.st_h),
+              o->pmax ? o->pmax : c->at<float>(L.st_pmax), o->argmax ? o->argmax : c->at<int>(L.st_amax),
+              o->sample ? o->sample : c->at<int>(L.st_samp)};
+  vocab_merge_kernel<<<(T * 32 + 255) / 256, 256, 0, st>>>(vp.m, vp.z, vp.s, vp.amax_v, vp.amax_i, vp.gkey_v,
+                                                           vp.gkey_i, L.n_vt, T, log((double)V), ps);
+                                                           CNT(c);
+  DG_CUDA(cudaGetLastError());
+
+  // a8: expected embedding for the next round's self-conditioning input
+  if (m.self_cond) {
+    ProfScope ps_(c, DG_PROF_EXPECTED_EMB, st);
+    uint16_t* probs = c->at<uint16_t>(L.probs);
+    const long long n4 = (long long)T * V / 4;
+    probs_kernel<<<(unsigned)std::min<long long>((n4 + 255) / 256, 148 * 16), 256, 0, st>>>(
+        logits, ps.m, ps.inv_z, probs, T, V);
+        CNT(c);
+    const int ks = esum_splits(m, T, c->num_sms);
+    CUtensorMap ta, tb;
+    DG_TRY(make_tmap(&ta, c->wp(c->wl.embT), V, d, 128));
+    DG_TRY(make_tmap(&tb, probs, V, L.T_alloc, boxT));
+    GemmPlan p = dense_plan(V, d, T, bnT, boxT, ks, err);
+    p.a_hint = 1;
+    p.b_hint = 2;
+    EpiStoreT e{c->at<float>(L.epart), d, (long long)T * d, 0, nullptr, nullptr, 0, err};
+    DG_TRY(run_gemm(ta, tb, p, e, c->num_sms, st, &c->n_launch));
+    const long long n = (long long)T * d;
+    esum_kernel<<<(unsigned)std::min<long long>((n + 255) / 256, 148 * 16), 256, 0, st>>>(
+        c->at<float>(L.epart), ks, T, d, DG_CANVAS, cv->done, cv->sc_state);
+        CNT(c);
+    DG_CUDA(cudaGetLastError());
+  }
+
+  // a9: mean entropy, stop, lock, next canvas
+  UpdateParams up{};
+  up.entropy = ps.entropy;
+  up.pmax = ps.pmax;
+  up.argmax = ps.argmax;
+  up.sample = ps.sample;
+  up.tokens = cv->tokens;
+  up.prev_argmax = cv->prev_argmax;
+  up.done = cv->done;
+  up.lock_out = o->lock;
+  up.mean_out = o->mean_entropy;
+  up.stop_out = o->stop;
+  up.final_out = o->final_round;
+  up.flags = c->at<uint8_t>(L.flags);
+  up.policy = s.lock_policy;
+  up.lock_threshold = s.lock_threshold;
+  up.stop_entropy = s.stop_entropy;
+  up.require_stable = s.stop_require_stable_argmax;
+  up.step = a->step;
+  up.max_steps = s.max_steps;
+  up.block = a->block;
+  up.k0 = (uint32_t)s.seed;
+  up.k1 = (uint32_t)(s.seed >> 32);
+  up.vocab = V;
+  canvas_update_kernel<<<B, 256, 0, st>>>(up);
+  CNT(c);
+  DG_CUDA(cudaGetLastError());
+  return DG_OK;
+}
+
+extern "C" dg_status dg_check_device_error(dg_ctx* c, void* stream) {
+  if (!c) return fail(DG_ERR_INVALID_ARG, "null context");
+  DG_CUDA(cudaStreamSynchronize((cudaStream_t)stream));
+  int e = 0;
+  DG_CUDA(cudaMemcpy(&e, c->err(), sizeof(int), cudaMemcpyDeviceToHost));
+  if (e) {
+    DG_CUDA(cudaMemset(c->err(), 0, sizeof(int)));
+    if (e == kDevErrBadToken) return fail(DG_ERR_BAD_TOKEN, "a token id outside [0, vocab) reached the device");
+    if (e == kDevErrTimeout) return fail(DG_ERR_TIMEOUT, "a bounded device wait ran out");
+    return fail(DG_ERR_CUDA, "device error word %d", e);
+  }
+  return DG_OK;
+}
+
+extern "C" dg_status dg_decode_block(dg_ctx* c, dg_kv* kv, dg_canvas* cv, const dg_step_args* a, int32_t* d_out,
+                                     dg_block_stats* h_stats, void* stream) {
+  if (!c || !cv || !a || !d_out) return fail(DG_ERR_INVALID_ARG, "null argument");
+  DG_TRY(check_kv(c, kv, DG_CANVAS));
+  cudaStream_t st = (cudaStream_t)stream;
+  const int B = cv->batch;
+  DG_TRY(dg_canvas_init(c, cv, a->block, a->sampler.seed, stream));
+  std::vector<uint8_t> flags(B, 0);
+  std::vector<int32_t> steps(B, 0);
+  int rounds = 0;
+  for (int s = 0; s < a->sampler.max_steps; ++s) {
+    dg_step_args sa = *a;
+    sa.step = s;
+    DG_TRY(dg_denoise_step(c, kv, cv, &sa, nullptr, stream));
+    ++rounds;
+    for (int b = 0; b < B; ++b)
+      if (!flags[b]) ++steps[b];
+    DG_CUDA(cudaMemcpyAsync(flags.data(), c->at<uint8_t>(c->L.flags), B, cudaMemcpyDeviceToHost, st));
+    DG_TRY(dg_check_device_error(c, stream));  // synchronises the stream
+    bool all = true;
+    for (int b = 0; b < B; ++b) all = all && flags[b];
+    if (all) break;
+  }
+  DG_CUDA(cudaMemcpyAsync(d_out, cv->tokens, (size_t)B * DG_CANVAS * 4, cudaMemcpyDeviceToDevice, st));
+  DG_TRY(dg_encode_context(c, kv, d_out, DG_CANVAS, stream));
+  if (h_stats) {
+    h_stats->rounds = rounds;
+    if (h_stats->steps_taken) memcpy(h_stats->steps_taken, steps.data(), B * sizeof(int32_t));
+  }
+  return DG_OK;
+}
+
+extern "C" dg_status dg_profile_start(dg_ctx* c) {
+  if (!c) return fail(DG_ERR_INVALID_ARG, "null context");
+  c->prof = true;
+  c->n_launch = 0;
+  c->ev_used = 0;
+  c->prof_recs.clear();
+  return DG_OK;
+}
+
+extern "C" dg_status dg_profile_stop(dg_ctx* c, dg_profile* out) {
+  if (!c || !out) return fail(DG_ERR_INVALID_ARG, "null argument");
+  c->prof = false;
+  memset(out, 0, sizeof(*out));
+  for (const auto& r : c->prof_recs) {
+    DG_CUDA(cudaEventSynchronize(c->ev_pool[r.second + 1]));
+    float ms = 0.f;
+    DG_CUDA(cudaEventElapsedTime(&ms, c->ev_pool[r.second], c->ev_pool[r.second + 1]));
+    out->ms[r.first] += ms;
+    out->launches[r.first] += 1;
+  }
+  out->launches_total = c->n_launch;
+  c->prof_recs.clear();
+  c->ev_used = 0;
+  return DG_OK;
+}
+
+// ============================================================================
+// test hooks
+namespace {
+struct EpiGroupedT {
+  float* out;
+  int ld;
+  struct State {};
+  __device__ __forceinline__ void begin(const GemmJob&, int, State&) const {}
+  __device__ __forceinline__ void end(const GemmJob&, int, State&) const {}
+  __device__ __forceinline__ void chunk(const GemmJob& j, int row, int c0, const float (&v)[16], State&) const {
+    if (row >= j.m_valid) return;
+    const int f = j.m_tile * 128 + row;
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if (c0 + i < j.n_valid) out[(long long)(j.n0 + c0 + i) * ld + f] = v[i];
+  }
+};
+
+// row-major store; k split s writes the matrix at D + s * M * N
+struct EpiSplitRows {
+  float* out;
+  long long M, N;
+  struct State {};
+  __device__ __forceinline__ void begin(const GemmJob&, int, State&) const {}
+  __device__ __forceinline__ void end(const GemmJob&, int, State&) const {}
+  __device__ __forceinline__ void chunk(const GemmJob& j, int row, int c0, const float (&v)[16], State&) const {
+    if (row >= j.m_valid) return;
+    const long long m = (long long)j.m_tile * 128 + row;
+    float* o = out + (long long)j.ks * M * N + m * N + j.n0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if (c0 + i < j.n_valid) o[c0 + i] = v[i];
+  }
+};
+}  // namespace
+
+extern "C" dg_status dg_test_gemm(const uint16_t* A, int32_t M, const uint16_t* B, int32_t N, int32_t K, float* D,
+                                  int32_t k_splits, void* stream) {
+  if (!A || !B || !D || M < 128 || N < 16 || K < 64 || K % 64 || k_splits < 1 || k_splits > K / 64)
+    return fail(DG_ERR_INVALID_ARG, "dg_test_gemm: bad arguments");
+  cudaStream_t st = (cudaStream_t)stream;
+  int* err = nullptr;
+  const int bn = token_bn(N), box = box_for(bn);
+  CUtensorMap ta, tb;
+  DG_TRY(make_tmap(&ta, A, K, M, 128));
+  DG_TRY(make_tmap(&tb, B, K, N, box));
+  GemmPlan p = dense_plan(K, M, N, bn, box, k_splits, err);
+  p.n_fast = 0;
+  EpiSplitRows e{D, M, N};
+  DG_TRY(run_gemm(ta, tb, p, e, device_sms(), st));
+  DG_CUDA(cudaStreamSynchronize(st));
+  return DG_OK;
+}
+
+extern "C" dg_status dg_test_grouped_gemm(const uint16_t* A, int32_t rows_per_group, int32_t n_groups,
+                                          const uint16_t* B, int32_t n_rows, int32_t K, const int32_t* off,
+                                          float* D, int32_t bn, void* stream) {
+  if (!A || !B || !D || !off || rows_per_group < 1 || n_groups < 1 || n_rows < 16 || K < 64 || K % 64 ||
+      bn < 16 || bn > 256 || (bn & (bn - 1)))
+    return fail(DG_ERR_INVALID_ARG, "dg_test_grouped_gemm: bad arguments");
+  if ((long long)rows_per_group * n_groups < 128) return fail(DG_ERR_INVALID_ARG, "A needs >= 128 rows");
+  cudaStream_t st = (cudaStream_t)stream;
+  CUtensorMap ta, tb;
+  DG_TRY(make_tmap(&ta, A, K, (long long)rows_per_group * n_groups, 128));
+  DG_TRY(make_tmap(&tb, B, K, n_rows, 16));
+  GemmPlan p = grouped_plan(K, rows_per_group, off, n_groups, bn, nullptr);
+  EpiGroupedT e{D, rows_per_group};
+  DG_TRY(run_gemm(ta, tb, p, e, device_sms(), st));
+  DG_CUDA(cudaStreamSynchronize(st));
+  return DG_OK;
+}

@@ -1,0 +1,207 @@
+// epilogues.cuh - per-thread epilogue functors of the tcgen05 GEMM core.
+// Each epilogue thread owns one accumulator row (tile row `row`, 0..127) and
+// receives its values 16 columns at a time.
+#pragma once
+
+#include "gemm_tc.cuh"
+
+namespace dg {
+
+// Transposed store of a weight-stationary product (A = weights, one row per
+// output feature; B = tokens): out[t * ld + f] for feature f = a_row0 + row and
+// token t = n0 + column.  Consecutive threads write consecutive features, so
+// each warp store is one contiguous 128-byte line.
+//   mode 0: out  = D           (split k: out + ks * split_stride)
+//   mode 1: out += D           (residual add)
+//   mode 2: out  = E_emb[tok[t], f] + D   (canvas embedding + self-conditioning)
+struct EpiStoreT {
+  float* out;
+  long long ld;
+  long long split_stride;
+  int mode;
+  const uint16_t* emb;   // mode 2: [V, ld] bf16
+  const int* tokens;     // mode 2: [T]
+  int vocab;             // mode 2
+  int* err;
+  struct State {};
+  __device__ __forceinline__ void begin(const GemmJob&, int, State&) const {}
+  __device__ __forceinline__ void end(const GemmJob&, int, State&) const {}
+  __device__ __forceinline__ void chunk(const GemmJob& j, int row, int c0, const float (&v)[16],
+                                        State&) const {
+    if (row >= j.m_valid) return;
+    const int f = j.m_tile * 128 + row;
+    float* base = out + (long long)j.ks * split_stride + f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int n = c0 + i;
+      if (n < j.n_valid) {
+        const long long t = j.n0 + n;
+        float* p = base + t * ld;
+        if (mode == 0) {
+          *p = v[i];
+        } else if (mode == 1) {
+          *p += v[i];
+        } else {
+          int tok = __ldg(tokens + t);
+          if (tok < 0 || tok >= vocab) { set_error(err, kDevErrBadToken); tok = 0; }
+          *p = bf16_to_f32(__ldg(emb + (long long)tok * ld + f)) + v[i];
+        }
+      }
+    }
+  }
+};
+
+// Grouped gate/up projection with SwiGLU.  The expert's [2 f, d] weight has
+// gate row j at 2j and up row j at 2j+1, so the pair sits in adjacent lanes:
+// h[slot, j] = bf16(silu(gate) * up) with silu(z) = z / (1 + e^-z).
+struct EpiSwiGLU {
+  uint16_t* h;   // [rows, f_dim] bf16, rows in expert (permuted) order
+  int f_dim;
+  struct State {};
+  __device__ __forceinline__ void begin(const GemmJob&, int, State&) const {}
+  __device__ __forceinline__ void end(const GemmJob&, int, State&) const {}
+  __device__ __forceinline__ void chunk(const GemmJob& j, int row, int c0, const float (&v)[16],
+                                        State&) const {
+    const int feat = (j.m_tile * 128 + row) >> 1;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float other = __shfl_xor_sync(0xffffffffu, v[i], 1);
+      const int n = c0 + i;
+      if ((row & 1) == 0 && row < j.m_valid && n < j.n_valid) {
+        const float g = v[i], u = other;
+        const float act = g / (1.0f + __expf(-g));
+        h[(long long)(j.n0 + n) * f_dim + feat] = f32_to_bf16(act * u);
+      }
+    }
+  }
+};
+
+// Grouped down projection: y[slot, f] = w[slot] * D (fp32), f = output feature.
+struct EpiDown {
+  float* y;
+  int d;
+  const float* w_slot;
+  struct State {};
+  __device__ __forceinline__ void begin(const GemmJob&, int, State&) const {}
+  __device__ __forceinline__ void end(const GemmJob&, int, State&) const {}
+  __device__ __forceinline__ void chunk(const GemmJob& j, int row, int c0, const float (&v)[16],
+                                        State&) const {
+    if (row >= j.m_valid) return;
+    const int f = j.m_tile * 128 + row;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int n = c0 + i;
+      if (n < j.n_valid) {
+        const long long slot = j.n0 + n;
+        y[slot * d + f] = __ldg(w_slot + slot) * v[i];
+      }
+    }
+  }
+};
+
+// LM head (A = final normalised hidden states, one row per canvas position;
+// B = W_lm rows = vocabulary ids).  Stores the fp32 logits and keeps, per
+// position and per vocabulary tile, the online softmax statistics
+//   m = max l, Z = sum e^(l - m), S = sum e^(l - m) l,
+// the argmax (first maximum) and the Gumbel-max key argmax_v (l_v / T + g_v)
+// with g = -ln(-ln u) from Philox (purpose 2, c0 = v / 4, word v % 4).
+struct VocabPartials {
+  float* m;
+  float* z;
+  float* s;
+  float* amax_v;
+  int* amax_i;
+  float* gkey_v;
+  int* gkey_i;
+};
+
+struct EpiLMHead {
+  float* logits;         // [T, V]
+  long long V;
+  VocabPartials part;    // each [T, n_vt]
+  int n_vt;              // vocabulary tiles (V / bn)
+  int bn;
+  uint32_t k0, k1;       // Philox key (seed)
+  uint32_t c2;           // block * 256 + step
+  float inv_t;           // 1 / T_step, fp32
+  int canvas;            // positions per canvas (256)
+  struct State {
+    float m, z, s, av, gv;
+    int ai, gi;
+  };
+  __device__ __forceinline__ void begin(const GemmJob&, int, State& st) const {
+    st.m = -INFINITY; st.z = 0.f; st.s = 0.f;
+    st.av = -INFINITY; st.ai = 0; st.gv = -INFINITY; st.gi = 0;
+  }
+  __device__ __forceinline__ void chunk(const GemmJob& j, int row, int c0, const float (&v)[16],
+                                        State& st) const {
+    if (row >= j.m_valid) return;
+    const int t = j.m_tile * 128 + row;
+    const int vb = j.n0 + c0;  // first vocabulary id of this chunk (multiple of 16)
+    float4* dst = reinterpret_cast<float4*>(logits + (long long)t * V + vb);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+
+    float cm = v[0];
+#pragma unroll
+    for (int i = 1; i < 16; ++i) cm = fmaxf(cm, v[i]);
+    if (cm > st.m) {
+      const float sc = __expf(st.m - cm);  // 0 when st.m = -inf
+      st.z *= sc;
+      st.s *= sc;
+      st.m = cm;
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float e = __expf(v[i] - st.m);
+      st.z += e;
+      st.s = fmaf(e, v[i], st.s);
+      if (v[i] > st.av) { st.av = v[i]; st.ai = vb + i; }
+    }
+    const int b = t / canvas, pos = t - b * canvas;
+    const uint32_t c3 = (kPurposeGumbel << 24) | (uint32_t)b;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const Philox4 r = philox4x32_10((uint32_t)(vb >> 2) + q, (uint32_t)pos, c2, c3, k0, k1);
+      const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float u = gumbel_u(w[e]);
+        const float g = -__logf(-__logf(u));
+        const float key = __fadd_rn(__fmul_rn(v[4 * q + e], inv_t), g);
+        if (key > st.gv) { st.gv = key; st.gi = vb + 4 * q + e; }
+      }
+    }
+  }
+  __device__ __forceinline__ void end(const GemmJob& j, int row, State& st) const {
+    if (row >= j.m_valid) return;
+    const int t = j.m_tile * 128 + row;
+    const long long idx = (long long)t * n_vt + j.n0 / bn;
+    part.m[idx] = st.m;
+    part.z[idx] = st.z;
+    part.s[idx] = st.s;
+    part.amax_v[idx] = st.av;
+    part.amax_i[idx] = st.ai;
+    part.gkey_v[idx] = st.gv;
+    part.gkey_i[idx] = st.gi;
+  }
+};
+
+// Plain row-major store D[m, n] -> out[m * ld + n] (the GEMM test hook).
+struct EpiStoreRows {
+  float* out;
+  long long ld;
+  struct State {};
+  __device__ __forceinline__ void begin(const GemmJob&, int, State&) const {}
+  __device__ __forceinline__ void end(const GemmJob&, int, State&) const {}
+  __device__ __forceinline__ void chunk(const GemmJob& j, int row, int c0, const float (&v)[16],
+                                        State&) const {
+    if (row >= j.m_valid) return;
+    const long long m = (long long)j.m_tile * 128 + row;
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if (c0 + i < j.n_valid) out[m * ld + j.n0 + c0 + i] = v[i];
+  }
+};
+
+}  // namespace dg

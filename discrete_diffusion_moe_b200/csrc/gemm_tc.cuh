@@ -1,0 +1,283 @@
+// gemm_tc.cuh - persistent, warp-specialised tcgen05 GEMM core for sm_100a.
+//
+//   D[m, n] = sum_k A[m, k] * B[n, k]      (bf16 inputs, fp32 accumulate)
+//
+// A and B are K-major bf16 matrices read through 2-D TMA tensor maps with the
+// 128-byte swizzle (box: 64 elements of K x 128 rows for A, x b_box rows for
+// B).  One CTA per SM loops over work units:
+//   warp 0      TMA producer (one elected lane) filling a ring of smem stages
+//   warp 1      allocates tensor memory; one lane issues tcgen05.mma (M = 128,
+//               N = the unit's columns rounded up to 16) into one of two
+//               accumulator buffers and commits stage / accumulator barriers
+//   warps 2..5  epilogue: tcgen05.ld of the 128 x N accumulator (warp w owns
+//               TMEM lanes 32*(w%4) .. +31, i.e. tile rows) into registers and
+//               a caller-supplied functor; the second accumulator buffer lets
+//               the next unit's MMAs overlap this epilogue.
+//
+// Two schedules:
+//   dense    units = (m_tile, n_tile, k_split); B rows [n_tile*bn, +bn)
+//   grouped  units = (group, m_tile); group g uses A rows
+//            [g * a_rows_per_group + m_tile*128, +128) and B rows
+//            [group_off[g], group_off[g+1]) in passes of at most bn columns
+//            (a mixture-of-experts layer: one group per expert, B rows are the
+//            tokens routed to it, typically a few dozen).
+//
+// Every mbarrier wait is bounded (see mbar_wait); a unit whose wait ran out
+// is abandoned, the error word is set, in-flight copies are drained and the
+// tensor memory is released before the CTA exits.
+#pragma once
+
+#include "common.cuh"
+
+namespace dg {
+
+struct GemmPlan {
+  int K;                 // reduction length, multiple of 64
+  int a_rows;            // dense: rows of A (M); grouped: rows per group actually valid
+  int m_tiles;           // dense: ceil(M / 128); grouped: tiles per group
+  int n_total;           // dense: rows of B (N)
+  int bn;                // columns per pass: multiple of 16, <= 256
+  int b_box;             // rows per TMA box of B (divides bn)
+  int k_splits;          // dense: K loop split into this many units (>= 1)
+  int n_fast;            // dense: 1 = consecutive units walk the N tiles of one A tile
+  const int* group_off;  // grouped when non-null: [n_groups + 1] B row offsets
+  int n_groups;
+  int a_rows_per_group;  // grouped: A row stride between groups
+  int a_hint, b_hint;    // L2 policy of the A / B loads: 0 none, 1 evict_first, 2 evict_last
+  int* err;              // device error word
+};
+
+struct GemmJob {
+  int m_tile;    // tile index within the group (grouped) or within A (dense)
+  int a_row0;    // first A row of the tile
+  int m_valid;   // valid rows in this tile (<= 128)
+  int group;     // grouped: group id; dense: -1
+  int n0;        // first B row of this pass
+  int n_local0;  // first column of this pass relative to the group / matrix start
+  int n_valid;   // valid columns (B rows) in this pass, 1..bn
+  int ks;        // k split index
+  int kb0, kb1;  // k blocks [kb0, kb1) of 64
+};
+
+__device__ __forceinline__ int gemm_num_units(const GemmPlan& p) {
+  if (p.group_off) return p.n_groups * p.m_tiles;
+  const int n_tiles = (p.n_total + p.bn - 1) / p.bn;
+  return p.m_tiles * n_tiles * p.k_splits;
+}
+
+// Number of passes of unit u (0 for an empty group) and the job of pass `pass`.
+__device__ __forceinline__ int gemm_unit_passes(const GemmPlan& p, int u) {
+  if (!p.group_off) return 1;
+  const int g = u / p.m_tiles;
+  const int n = __ldg(p.group_off + g + 1) - __ldg(p.group_off + g);
+  return n <= 0 ? 0 : (n + p.bn - 1) / p.bn;
+}
+
+__device__ __forceinline__ GemmJob gemm_job(const GemmPlan& p, int u, int pass) {
+  GemmJob j;
+  const int kb_total = p.K / 64;
+  if (p.group_off) {
+    const int g = u / p.m_tiles;
+    j.m_tile = u - g * p.m_tiles;
+    j.group = g;
+    j.a_row0 = g * p.a_rows_per_group + j.m_tile * 128;
+    j.m_valid = min(128, p.a_rows - j.m_tile * 128);
+    const int off0 = __ldg(p.group_off + g), off1 = __ldg(p.group_off + g + 1);
+    j.n_local0 = pass * p.bn;
+    j.n0 = off0 + j.n_local0;
+    j.n_valid = min(p.bn, off1 - j.n0);
+    j.ks = 0;
+    j.kb0 = 0;
+    j.kb1 = kb_total;
+  } else {
+    const int n_tiles = (p.n_total + p.bn - 1) / p.bn;
+    const int ks = u % p.k_splits;
+    const int r = u / p.k_splits;
+    int mt, nt;
+    if (p.n_fast) { nt = r % n_tiles; mt = r / n_tiles; }
+    else          { mt = r % p.m_tiles; nt = r / p.m_tiles; }
+    j.m_tile = mt;
+    j.group = -1;
+    j.a_row0 = mt * 128;
+    j.m_valid = min(128, p.a_rows - mt * 128);
+    j.n_local0 = nt * p.bn;
+    j.n0 = j.n_local0;
+    j.n_valid = min(p.bn, p.n_total - j.n0);
+    j.ks = ks;
+    j.kb0 = (int)((long long)kb_total * ks / p.k_splits);
+    j.kb1 = (int)((long long)kb_total * (ks + 1) / p.k_splits);
+  }
+  return j;
+}
+
+constexpr int kGemmThreads = 192;
+constexpr int kATileBytes = 128 * 128;  // 128 rows x 64 bf16
+
+template <class Epi>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const GemmPlan p, const Epi epi, const int stages) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // 1024-byte alignment for the swizzled tiles
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const int b_stage_bytes = p.bn * 128;
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + (size_t)stages * kATileBytes;
+  uint64_t* bars = (uint64_t*)(sB + (size_t)stages * b_stage_bytes);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + stages;
+  uint64_t* acc_full = bars + 2 * stages;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* drain = acc_empty + 2;
+  uint32_t* tmem_slot = (uint32_t*)(drain + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t tmem_cols = 2u * (uint32_t)p.bn < 32u ? 32u : 2u * (uint32_t)p.bn;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(smem_u32(&acc_full[a]), 1);
+      mbar_init(smem_u32(&acc_empty[a]), 128);
+    }
+    mbar_init(smem_u32(drain), 1);
+    fence_mbar_init();
+    fence_proxy_async_smem();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int U = gemm_num_units(p);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      uint32_t it = 0;
+      bool ok = true;
+      const uint64_t pol_first = l2_policy_evict_first(), pol_last = l2_policy_evict_last();
+      const uint64_t pol_a = p.a_hint == 1 ? pol_first : pol_last;
+      const uint64_t pol_b = p.b_hint == 1 ? pol_first : pol_last;
+      for (int u = blockIdx.x; u < U && ok; u += gridDim.x) {
+        const int np = gemm_unit_passes(p, u);
+        for (int pass = 0; pass < np && ok; ++pass) {
+          const GemmJob j = gemm_job(p, u, pass);
+          const int n_mma = (j.n_valid + 15) & ~15;
+          const int nbox = (n_mma + p.b_box - 1) / p.b_box;
+          const uint32_t tx = kATileBytes + (uint32_t)nbox * p.b_box * 128;
+          for (int kb = j.kb0; kb < j.kb1; ++kb, ++it) {
+            const int s = it % stages;
+            const uint32_t ph = (it / stages) & 1;
+            if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1, p.err)) { ok = false; break; }
+            const uint32_t fb = smem_u32(&full[s]);
+            mbar_arrive_expect_tx(fb, tx);
+            const uint32_t dA = smem_u32(sA + (size_t)s * kATileBytes);
+            if (p.a_hint) tma_load_2d_hint(dA, &tmA, fb, kb * 64, j.a_row0, pol_a);
+            else          tma_load_2d(dA, &tmA, fb, kb * 64, j.a_row0);
+            for (int b = 0; b < nbox; ++b) {
+              const uint32_t dB = smem_u32(sB + (size_t)s * b_stage_bytes + b * p.b_box * 128);
+              if (p.b_hint) tma_load_2d_hint(dB, &tmB, fb, kb * 64, j.n0 + b * p.b_box, pol_b);
+              else          tma_load_2d(dB, &tmB, fb, kb * 64, j.n0 + b * p.b_box);
+            }
+          }
+        }
+      }
+      // drain: wait until every issued copy has landed before the CTA may exit
+      const uint32_t n_issued = it;
+      const uint32_t first = n_issued > (uint32_t)stages ? n_issued - stages : 0;
+      for (uint32_t q = first; q < n_issued; ++q)
+        mbar_wait(smem_u32(&full[q % stages]), (q / stages) & 1, p.err);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer ----------------
+      uint32_t it = 0, jc = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < U && ok; u += gridDim.x) {
+        const int np = gemm_unit_passes(p, u);
+        for (int pass = 0; pass < np && ok; ++pass, ++jc) {
+          const GemmJob j = gemm_job(p, u, pass);
+          const int n_mma = (j.n_valid + 15) & ~15;
+          const uint32_t idesc = idesc_bf16_f32(128, n_mma);
+          const uint32_t acc = jc & 1;
+          if (!mbar_wait(smem_u32(&acc_empty[acc]), ((jc >> 1) & 1) ^ 1, p.err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t d_tmem = tmem_base + acc * (uint32_t)p.bn;
+          for (int kb = j.kb0; kb < j.kb1; ++kb, ++it) {
+            const int s = it % stages;
+            const uint32_t ph = (it / stages) & 1;
+            if (!mbar_wait(smem_u32(&full[s]), ph, p.err)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t a0 = smem_u32(sA + (size_t)s * kATileBytes);
+            const uint32_t b0 = smem_u32(sB + (size_t)s * b_stage_bytes);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_bf16(d_tmem, sdesc_k128(a0 + kk * 32), sdesc_k128(b0 + kk * 32), idesc,
+                        (kb > j.kb0 || kk > 0) ? 1u : 0u);
+            umma_commit(smem_u32(&empty[s]));
+          }
+          if (ok) umma_commit(smem_u32(&acc_full[acc]));
+        }
+      }
+      // all issued tensor-core work must finish before the memory is released
+      umma_commit(smem_u32(drain));
+      mbar_wait(smem_u32(drain), 0, p.err);
+    }
+  } else {
+    // ---------------- epilogue (warps 2..5) ----------------
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    uint32_t jc = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < U && ok; u += gridDim.x) {
+      const int np = gemm_unit_passes(p, u);
+      for (int pass = 0; pass < np && ok; ++pass, ++jc) {
+        const GemmJob j = gemm_job(p, u, pass);
+        const uint32_t acc = jc & 1;
+        if (!mbar_wait(smem_u32(&acc_full[acc]), (jc >> 1) & 1, p.err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t t0 = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * (uint32_t)p.bn;
+        typename Epi::State st;
+        epi.begin(j, row, st);
+        const int nch = (j.n_valid + 15) >> 4;
+        for (int c = 0; c < nch; ++c) {
+          float v[16];
+          tmem_ld16(t0 + c * 16, v);
+          epi.chunk(j, row, c * 16, v, st);
+        }
+        epi.end(j, row, st);
+        tc_fence_before();
+        mbar_arrive(smem_u32(&acc_empty[acc]));
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, tmem_cols);
+}
+
+// Dynamic shared memory of one CTA for `stages` stages.
+inline size_t gemm_smem_bytes(int bn, int stages) {
+  return 1024 + (size_t)stages * (kATileBytes + (size_t)bn * 128) + (2 * stages + 5) * 8 + 16;
+}
+
+inline int gemm_pick_stages(int bn, int max_stages = 8) {
+  const size_t budget = 227 * 1024;
+  int s = max_stages;
+  while (s > 2 && gemm_smem_bytes(bn, s) > budget) --s;
+  return s;
+}
+
+}  // namespace dg

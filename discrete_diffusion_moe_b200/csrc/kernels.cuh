@@ -1,0 +1,513 @@
+// kernels.cuh - bandwidth-bound kernels of the denoising step: embedding,
+// RMSNorm, RoPE + KV write, router top-k, token permutation, expert combine,
+// vocabulary statistics merge, softmax probabilities, split-k reduction of
+// the expected embedding, the canvas update (entropy / lock / stop /
+// re-noise) and canvas initialisation.  All reductions that carry results
+// run in a fixed order (no atomics on values), so results are deterministic.
+#pragma once
+
+#include "common.cuh"
+
+namespace dg {
+
+// ---------------------------------------------------------------------------
+// a1: x[t, :] = E_emb[tok[t], :]   (fp32 residual stream)
+__global__ void embed_kernel(const uint16_t* __restrict__ emb, const int* __restrict__ tokens,
+                             float* __restrict__ x, int T, int d, int vocab, int* err) {
+  const int t = blockIdx.x;
+  if (t >= T) return;
+  int tok = tokens[t];
+  if (tok < 0 || tok >= vocab) {
+    if (threadIdx.x == 0) set_error(err, kDevErrBadToken);
+    tok = 0;
+  }
+  const uint16_t* src = emb + (long long)tok * d;
+  float* dst = x + (long long)t * d;
+  for (int c = threadIdx.x * 8; c < d; c += blockDim.x * 8) {
+    const uint4 u = *reinterpret_cast<const uint4*>(src + c);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    float4 a, b;
+    a.x = bf16_to_f32(w[0] & 0xFFFF); a.y = bf16_to_f32(w[0] >> 16);
+    a.z = bf16_to_f32(w[1] & 0xFFFF); a.w = bf16_to_f32(w[1] >> 16);
+    b.x = bf16_to_f32(w[2] & 0xFFFF); b.y = bf16_to_f32(w[2] >> 16);
+    b.z = bf16_to_f32(w[3] & 0xFFFF); b.w = bf16_to_f32(w[3] >> 16);
+    *reinterpret_cast<float4*>(dst + c) = a;
+    *reinterpret_cast<float4*>(dst + c + 4) = b;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// RMSNorm: y = bf16(x / sqrt(mean(x^2) + eps) * g), one CTA per row.
+template <int THREADS>
+__global__ void __launch_bounds__(THREADS) rmsnorm_kernel(const float* __restrict__ x,
+                                                          const uint16_t* __restrict__ gain,
+                                                          uint16_t* __restrict__ y, int d, float eps) {
+  const int t = blockIdx.x;
+  const float* xr = x + (long long)t * d;
+  float ss = 0.f;
+  for (int c = threadIdx.x * 4; c < d; c += THREADS * 4) {
+    const float4 v = *reinterpret_cast<const float4*>(xr + c);
+    ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+  }
+  __shared__ float red[THREADS / 32];
+  ss = warp_sum(ss);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  float tot = 0.f;
+#pragma unroll
+  for (int w = 0; w < THREADS / 32; ++w) tot += red[w];
+  const float r = rsqrtf(tot / (float)d + eps);
+  uint16_t* yr = y + (long long)t * d;
+  for (int c = threadIdx.x * 4; c < d; c += THREADS * 4) {
+    const float4 v = *reinterpret_cast<const float4*>(xr + c);
+    const uint2 gg = *reinterpret_cast<const uint2*>(gain + c);
+    uint2 o;
+    o.x = pack_bf16x2(v.x * r * bf16_to_f32(gg.x & 0xFFFF), v.y * r * bf16_to_f32(gg.x >> 16));
+    o.y = pack_bf16x2(v.z * r * bf16_to_f32(gg.y & 0xFFFF), v.w * r * bf16_to_f32(gg.y >> 16));
+    *reinterpret_cast<uint2*>(yr + c) = o;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// RoPE on q and k (pairs (i, i + hd/2) rotated by pos * theta^(-2i/hd), angle
+// and rotation in double), q -> bf16 [T, Hq*hd]; k, v -> bf16 KV cache of this
+// layer at position L0 + i of each canvas ([B][Hkv][c_max][hd]).
+struct RopeParams {
+  const float* qkv;   // [T, (Hq + 2 Hkv) * hd]
+  uint16_t* q;        // [T, Hq * hd]
+  uint16_t* kc;       // layer base of K cache
+  uint16_t* vc;       // layer base of V cache
+  int T, nq, L0, c_max, Hq, Hkv, hd;
+  double theta;
+};
+
+__global__ void rope_kv_kernel(const RopeParams p) {
+  const int half = p.hd / 2;
+  const int heads = p.Hq + p.Hkv;                   // heads that are rotated
+  const long long n_rot = (long long)p.T * heads * half;
+  const long long n_v = (long long)p.T * p.Hkv * half;  // v copied in pairs
+  const int row_w = (p.Hq + 2 * p.Hkv) * p.hd;
+  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n_rot + n_v;
+       e += (long long)gridDim.x * blockDim.x) {
+    if (e < n_rot) {
+      const int i = (int)(e % half);
+      const long long r = e / half;
+      const int h = (int)(r % heads);
+      const int t = (int)(r / heads);
+      const int b = t / p.nq, pos_in = t - b * p.nq;
+      const double pos = (double)(p.L0 + pos_in);
+      const double inv_freq = pow(p.theta, -2.0 * (double)i / (double)p.hd);
+      double sn, cs;
+      sincos(pos * inv_freq, &sn, &cs);
+      const float* src = p.qkv + (long long)t * row_w + h * p.hd;
+      const double x1 = src[i], x2 = src[i + half];
+      const float o1 = (float)(x1 * cs - x2 * sn), o2 = (float)(x2 * cs + x1 * sn);
+      uint16_t* dst;
+      if (h < p.Hq) {
+        dst = p.q + (long long)t * p.Hq * p.hd + h * p.hd;
+      } else {
+        const int g = h - p.Hq;
+        dst = p.kc + (((long long)b * p.Hkv + g) * p.c_max + p.L0 + pos_in) * p.hd;
+      }
+      dst[i] = f32_to_bf16(o1);
+      dst[i + half] = f32_to_bf16(o2);
+    } else {
+      const long long e2 = e - n_rot;
+      const int i = (int)(e2 % half);
+      const long long r = e2 / half;
+      const int g = (int)(r % p.Hkv);
+      const int t = (int)(r / p.Hkv);
+      const int b = t / p.nq, pos_in = t - b * p.nq;
+      const float* src = p.qkv + (long long)t * row_w + (p.Hq + p.Hkv + g) * p.hd;
+      uint16_t* dst = p.vc + (((long long)b * p.Hkv + g) * p.c_max + p.L0 + pos_in) * p.hd;
+      dst[2 * i] = f32_to_bf16(src[2 * i]);
+      dst[2 * i + 1] = f32_to_bf16(src[2 * i + 1]);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Router: sum the split-k partial logits (fixed order), pick the top-k
+// experts by logit (ties to the lower id), softmax over the chosen k.
+// One warp per token; E <= 256.
+__global__ void router_topk_kernel(const float* __restrict__ part, int ks, int T, int E, int k,
+                                   int* __restrict__ idx, float* __restrict__ w,
+                                   int* __restrict__ dbg_idx, float* __restrict__ dbg_w) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= T) return;
+  const int t = warp;
+  float l[8];
+  bool taken[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const int e = lane + 32 * q;
+    float s = -INFINITY;
+    if (e < E) {
+      s = 0.f;
+      for (int p = 0; p < ks; ++p) s += part[((long long)p * T + t) * E + e];
+    }
+    l[q] = s;
+    taken[q] = false;
+  }
+  float sel_l[8];
+  int sel_e[8];
+  for (int r = 0; r < k; ++r) {
+    float bv = -INFINITY;
+    int be = 0x7fffffff;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int e = lane + 32 * q;
+      if (e < E && !taken[q] && (l[q] > bv || (l[q] == bv && e < be))) { bv = l[q]; be = e; }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+      if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
+    }
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      if (lane + 32 * q == be) taken[q] = true;
+    sel_l[r] = bv;
+    sel_e[r] = be;
+  }
+  if (lane == 0) {
+    float den = 0.f;
+    float ex[8];
+    for (int r = 0; r < k; ++r) { ex[r] = expf(sel_l[r] - sel_l[0]); den += ex[r]; }
+    for (int r = 0; r < k; ++r) {
+      idx[t * k + r] = sel_e[r];
+      w[t * k + r] = ex[r] / den;
+      if (dbg_idx) dbg_idx[t * k + r] = sel_e[r];
+      if (dbg_w) dbg_w[t * k + r] = ex[r] / den;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Token permutation: stable counting sort of the T*k (token, slot) pairs by
+// expert.  One CTA of 1024 threads.  Outputs off[E+1], perm[slot] = pair,
+// inv[pair] = slot, w_perm[slot] = w[pair].  Within an expert, pairs keep
+// ascending pair order (token-major), so the layout is deterministic.
+constexpr int kPermThreads = 1024;
+__global__ void __launch_bounds__(kPermThreads) permute_kernel(const int* __restrict__ idx,
+                                                               const float* __restrict__ w, int P,
+                                                               int E, int* __restrict__ off,
+                                                               int* __restrict__ perm,
+                                                               int* __restrict__ inv,
+                                                               float* __restrict__ w_perm, int* err) {
+  extern __shared__ int sm[];
+  int* cnt = sm;                    // [E]
+  int* base = sm + E;               // [E] running base within expert
+  int* wcnt = sm + 2 * E;           // [32 warps][E]
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int e = tid; e < E; e += kPermThreads) cnt[e] = 0;
+  __syncthreads();
+  for (int q = tid; q < P; q += kPermThreads) {
+    int e = idx[q];
+    if (e < 0 || e >= E) { set_error(err, kDevErrBadToken); e = 0; }
+    atomicAdd(&cnt[e], 1);
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int acc = 0;
+    for (int e = 0; e < E; ++e) { off[e] = acc; base[e] = acc; acc += cnt[e]; }
+    off[E] = acc;
+  }
+  __syncthreads();
+  for (int c0 = 0; c0 < P; c0 += kPermThreads) {
+    const int q = c0 + tid;
+    int e = -1;
+    if (q < P) { e = idx[q]; if (e < 0 || e >= E) e = 0; }
+    for (int i = tid; i < 32 * E; i += kPermThreads) wcnt[i] = 0;
+    __syncthreads();
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int rank_in_warp = __popc(peers & ((1u << lane) - 1));
+    if (e >= 0 && rank_in_warp == 0) wcnt[warp * E + e] = __popc(peers);
+    __syncthreads();
+    // exclusive scan over warps per expert (fixed order), then advance bases
+    for (int ee = tid; ee < E; ee += kPermThreads) {
+      int acc = base[ee];
+      for (int wv = 0; wv < 32; ++wv) {
+        const int c = wcnt[wv * E + ee];
+        wcnt[wv * E + ee] = acc;
+        acc += c;
+      }
+      base[ee] = acc;
+    }
+    __syncthreads();
+    if (e >= 0) {
+      const int slot = wcnt[warp * E + e] + rank_in_warp;
+      perm[slot] = q;
+      inv[q] = slot;
+      w_perm[slot] = w[q];
+    }
+    __syncthreads();
+  }
+}
+
+// X_perm[slot, :] = xn[perm[slot] / k, :]  (bf16 rows, 16-byte vectors)
+__global__ void gather_rows_kernel(const uint16_t* __restrict__ xn, const int* __restrict__ perm,
+                                   uint16_t* __restrict__ xp, int P, int k, int d) {
+  const int slot = blockIdx.x;
+  if (slot >= P) return;
+  const int t = perm[slot] / k;
+  const uint4* src = reinterpret_cast<const uint4*>(xn + (long long)t * d);
+  uint4* dst = reinterpret_cast<uint4*>(xp + (long long)slot * d);
+  for (int c = threadIdx.x; c < d / 8; c += blockDim.x) dst[c] = src[c];
+}
+
+// x[t, :] += sum_{j < k} y[inv[t*k + j], :]   (fixed j order, fp32)
+__global__ void moe_combine_kernel(float* __restrict__ x, const float* __restrict__ y,
+                                   const int* __restrict__ inv, int T, int k, int d) {
+  const int t = blockIdx.x;
+  if (t >= T) return;
+  int slots[8];
+  for (int j = 0; j < k; ++j) slots[j] = inv[t * k + j];
+  float* xr = x + (long long)t * d;
+  for (int c = threadIdx.x * 4; c < d; c += blockDim.x * 4) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < k; ++j) {
+      const float4 v = *reinterpret_cast<const float4*>(y + (long long)slots[j] * d + c);
+      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+    float4 r = *reinterpret_cast<float4*>(xr + c);
+    r.x += acc.x; r.y += acc.y; r.z += acc.z; r.w += acc.w;
+    *reinterpret_cast<float4*>(xr + c) = r;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Merge the per-tile vocabulary statistics of each position (fixed order:
+// lane l folds tiles l, l+32, ...; then a fixed shuffle tree), in double.
+// Writes m, 1/Z, entropy H = m + ln Z - S/Z (clamped to [0, ln V]), pmax = 1/Z,
+// argmax and Gumbel sample.
+struct PosStats {
+  float* m;
+  float* inv_z;
+  float* entropy;
+  float* pmax;
+  int* argmax;
+  int* sample;
+};
+
+__device__ __forceinline__ void merge_ms(double& m, double& z, double& s, double m2, double z2,
+                                         double s2) {
+  if (m2 == -INFINITY) return;
+  if (m == -INFINITY) { m = m2; z = z2; s = s2; return; }
+  const double mn = fmax(m, m2);
+  const double a = exp(m - mn), b = exp(m2 - mn);
+  z = z * a + z2 * b;
+  s = s * a + s2 * b;
+  m = mn;
+}
+
+__global__ void vocab_merge_kernel(const float* __restrict__ pm, const float* __restrict__ pz,
+                                   const float* __restrict__ ps, const float* __restrict__ pav,
+                                   const int* __restrict__ pai, const float* __restrict__ pgv,
+                                   const int* __restrict__ pgi, int n_vt, int T, double log_v,
+                                   PosStats out) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= T) return;
+  const long long base = (long long)warp * n_vt;
+  double m = -INFINITY, z = 0.0, s = 0.0;
+  float av = -INFINITY, gv = -INFINITY;
+  int ai = 0x7fffffff, gi = 0x7fffffff;
+  for (int v = lane; v < n_vt; v += 32) {
+    merge_ms(m, z, s, (double)pm[base + v], (double)pz[base + v], (double)ps[base + v]);
+    const float a = pav[base + v];
+    const int a_i = pai[base + v];
+    if (a > av || (a == av && a_i < ai)) { av = a; ai = a_i; }
+    const float g = pgv[base + v];
+    const int g_i = pgi[base + v];
+    if (g > gv || (g == gv && g_i < gi)) { gv = g; gi = g_i; }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const double m2 = __shfl_xor_sync(0xffffffffu, m, o);
+    const double z2 = __shfl_xor_sync(0xffffffffu, z, o);
+    const double s2 = __shfl_xor_sync(0xffffffffu, s, o);
+    merge_ms(m, z, s, m2, z2, s2);
+    const float a2 = __shfl_xor_sync(0xffffffffu, av, o);
+    const int ai2 = __shfl_xor_sync(0xffffffffu, ai, o);
+    if (a2 > av || (a2 == av && ai2 < ai)) { av = a2; ai = ai2; }
+    const float g2 = __shfl_xor_sync(0xffffffffu, gv, o);
+    const int gi2 = __shfl_xor_sync(0xffffffffu, gi, o);
+    if (g2 > gv || (g2 == gv && gi2 < gi)) { gv = g2; gi = gi2; }
+  }
+  if (lane == 0) {
+    double H = m + log(z) - s / z;
+    H = fmin(fmax(H, 0.0), log_v);
+    out.m[warp] = (float)m;
+    out.inv_z[warp] = (float)(1.0 / z);
+    out.entropy[warp] = (float)H;
+    out.pmax[warp] = (float)(1.0 / z);
+    out.argmax[warp] = ai;
+    out.sample[warp] = gi;
+  }
+}
+
+// p[t, v] = bf16(exp(l[t, v] - m_t) / Z_t) — the softmax operand of the
+// expected-embedding product.
+__global__ void probs_kernel(const float* __restrict__ logits, const float* __restrict__ m,
+                             const float* __restrict__ inv_z, uint16_t* __restrict__ p, int T,
+                             long long V) {
+  const long long n4 = (long long)T * V / 4;
+  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n4;
+       e += (long long)gridDim.x * blockDim.x) {
+    const long long t = (e * 4) / V;
+    const float mm = m[t], iz = inv_z[t];
+    const float4 l = reinterpret_cast<const float4*>(logits)[e];
+    uint2 o;
+    o.x = pack_bf16x2(__expf(l.x - mm) * iz, __expf(l.y - mm) * iz);
+    o.y = pack_bf16x2(__expf(l.z - mm) * iz, __expf(l.w - mm) * iz);
+    reinterpret_cast<uint2*>(p)[e] = o;
+  }
+}
+
+// e[t, f] = bf16(sum_s part[s, t, f]) for canvases that are still running.
+__global__ void esum_kernel(const float* __restrict__ part, int ks, int T, int d, int canvas,
+                            const uint8_t* __restrict__ done, uint16_t* __restrict__ sc_state) {
+  const long long n = (long long)T * d;
+  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n;
+       e += (long long)gridDim.x * blockDim.x) {
+    const int t = (int)(e / d);
+    if (done[t / canvas]) continue;
+    float acc = 0.f;
+    for (int s = 0; s < ks; ++s) acc += part[(long long)s * n + e];
+    sc_state[e] = f32_to_bf16(acc);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Canvas update (a9), one CTA of 256 threads per canvas (thread = position).
+struct UpdateParams {
+  const float* entropy;
+  const float* pmax;
+  const int* argmax;
+  const int* sample;
+  int* tokens;          // canvas in/out
+  int* prev_argmax;
+  uint8_t* done;
+  uint8_t* lock_out;    // may be null
+  float* mean_out;      // may be null
+  uint8_t* stop_out;    // may be null
+  uint8_t* final_out;   // may be null
+  uint8_t* flags;       // [B] internal copy of done after the update (host readback)
+  int policy;
+  float lock_threshold;
+  float stop_entropy;
+  int require_stable;
+  int step, max_steps, block;
+  uint32_t k0, k1;
+  int vocab;
+};
+
+__global__ void __launch_bounds__(256) canvas_update_kernel(const UpdateParams p) {
+  const int b = blockIdx.x, i = threadIdx.x;
+  const int t = b * 256 + i;
+  __shared__ float red[8];
+  __shared__ int same_w[8];
+  __shared__ float key[256];
+  __shared__ int kid[256];
+  __shared__ float csum[256];
+  const float H = p.entropy[t];
+  const float pm = p.pmax[t];
+  const int am = p.argmax[t];
+  const int smp = p.sample[t];
+  const bool was_done = p.done[b] != 0;
+
+  // mean entropy (fixed reduction order)
+  float v = warp_sum(H);
+  const int same = __all_sync(0xffffffffu, am == p.prev_argmax[t]);
+  if ((i & 31) == 0) { red[i >> 5] = v; same_w[i >> 5] = same; }
+  __syncthreads();
+  float tot = 0.f;
+  int all_same = 1;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) { tot += red[w]; all_same &= same_w[w]; }
+  const float meanH = tot / 256.0f;
+
+  // lock mask
+  bool lock;
+  if (p.policy == 0) {
+    lock = pm > p.lock_threshold;
+  } else {
+    // bitonic sort of (H, position) ascending, then a fixed-order running sum
+    key[i] = H;
+    kid[i] = i;
+    __syncthreads();
+    for (int size = 2; size <= 256; size <<= 1) {
+      for (int stride = size >> 1; stride > 0; stride >>= 1) {
+        const int j = i ^ stride;
+        if (j > i) {
+          const bool up = (i & size) == 0;
+          const float a = key[i], c = key[j];
+          const int ia = kid[i], ic = kid[j];
+          const bool gt = (a > c) || (a == c && ia > ic);
+          if (gt == up) { key[i] = c; key[j] = a; kid[i] = ic; kid[j] = ia; }
+        }
+        __syncthreads();
+      }
+    }
+    if (i == 0) {
+      float acc = 0.f;
+      for (int r = 0; r < 256; ++r) { acc += key[r]; csum[r] = acc; }
+    }
+    __syncthreads();
+    // rank of this position in sorted order
+    lock = false;
+    for (int r = 0; r < 256; ++r)
+      if (kid[r] == i) { lock = csum[r] <= p.lock_threshold; break; }
+  }
+  if (p.lock_out) p.lock_out[t] = lock ? 1 : 0;
+
+  const bool stable = p.step > 0 && all_same;
+  const bool stop = !was_done && (meanH < p.stop_entropy) && (!p.require_stable || stable);
+  const bool fin = !was_done && (stop || p.step == p.max_steps - 1);
+  if (!was_done) {
+    int nt;
+    if (fin) {
+      nt = am;
+    } else if (lock) {
+      nt = smp;
+    } else {
+      const Philox4 r = philox4x32_10(0u, (uint32_t)i, (uint32_t)(p.block * 256 + p.step),
+                                      (kPurposeRenoise << 24) | (uint32_t)b, p.k0, p.k1);
+      nt = uniform_token(r.x, (uint32_t)p.vocab);
+    }
+    p.tokens[t] = nt;
+    p.prev_argmax[t] = am;
+  }
+  __syncthreads();
+  if (i == 0) {
+    if (p.mean_out) p.mean_out[b] = meanH;
+    if (p.stop_out) p.stop_out[b] = stop ? 1 : 0;
+    if (p.final_out) p.final_out[b] = fin ? 1 : 0;
+    if (fin) p.done[b] = 1;
+    p.flags[b] = (was_done || fin) ? 1 : 0;
+  }
+}
+
+// Canvas initialisation: uniform tokens (purpose 1), prev_argmax = -1, done = 0.
+__global__ void canvas_init_kernel(int* tokens, int* prev_argmax, uint8_t* done, int B, int block,
+                                   uint32_t k0, uint32_t k1, int vocab) {
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= B * 256) return;
+  const int b = t / 256, i = t % 256;
+  const Philox4 r = philox4x32_10(0u, (uint32_t)i, (uint32_t)(block * 256),
+                                  (kPurposeInit << 24) | (uint32_t)b, k0, k1);
+  tokens[t] = uniform_token(r.x, (uint32_t)vocab);
+  prev_argmax[t] = -1;
+  if (i == 0) done[b] = 0;
+}
+
+__global__ void fill_u16_kernel(uint16_t* p, long long n, uint16_t v) {
+  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n;
+       e += (long long)gridDim.x * blockDim.x)
+    p[e] = v;
+}
+
+}  // namespace dg

@@ -1,0 +1,151 @@
+"""Device-memory plumbing around the C ABI: torch tensors for the weights,
+workspace, KV cache, canvas state and step outputs, and calls into libdg.so.
+No arithmetic of the method happens here."""
+
+import ctypes
+
+import torch
+
+from . import (DG_CANVAS, DG_LOCK_PROB, check, dg_block_stats, dg_canvas, dg_kv, dg_model_config,
+               dg_sampler_config, dg_step_args, dg_step_out, lib)
+
+
+def model_config(n_layers, d_model, n_q_heads, n_kv_heads, head_dim, n_experts, top_k, d_ff, vocab,
+                 self_cond=False, rope_theta=10000.0, rms_eps=1e-6) -> dg_model_config:
+    return dg_model_config(n_layers, d_model, n_q_heads, n_kv_heads, head_dim, n_experts, top_k, d_ff,
+                           vocab, int(bool(self_cond)), rope_theta, rms_eps)
+
+
+def sampler_config(lock_policy=DG_LOCK_PROB, lock_threshold=0.9, t_start=0.8, t_end=0.4, max_steps=48,
+                   stop_entropy=0.5, stop_require_stable_argmax=False, seed=0) -> dg_sampler_config:
+    return dg_sampler_config(lock_policy, lock_threshold, t_start, t_end, max_steps, stop_entropy,
+                             int(bool(stop_require_stable_argmax)), seed)
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+class KVCache:
+    def __init__(self, cfg: dg_model_config, batch: int, c_max: int, device="cuda"):
+        n = lib.dg_kv_bytes(ctypes.byref(cfg), batch, c_max)
+        if n == 0:
+            raise ValueError("bad KV cache size")
+        self.k = torch.zeros(n, dtype=torch.uint8, device=device)
+        self.v = torch.zeros(n, dtype=torch.uint8, device=device)
+        self.s = dg_kv(self.k.data_ptr(), self.v.data_ptr(), batch, c_max, 0)
+        self.cfg = cfg
+
+    @property
+    def length(self):
+        return self.s.length
+
+    def layer_kv(self, layer):
+        """(K, V) of one layer as bf16 [B, Hkv, c_max, hd] views."""
+        c = self.cfg
+        shape = (self.s.batch, c.n_kv_heads, self.s.c_max, c.head_dim)
+        per = self.k.numel() // 2 // c.n_layers
+        k = self.k.view(torch.bfloat16)[layer * per:(layer + 1) * per].view(shape)
+        v = self.v.view(torch.bfloat16)[layer * per:(layer + 1) * per].view(shape)
+        return k, v
+
+
+class Canvas:
+    def __init__(self, cfg: dg_model_config, batch: int, device="cuda"):
+        self.tokens = torch.zeros(batch, DG_CANVAS, dtype=torch.int32, device=device)
+        self.sc_state = torch.zeros(batch, DG_CANVAS, cfg.d_model, dtype=torch.bfloat16, device=device)
+        self.prev_argmax = torch.full((batch, DG_CANVAS), -1, dtype=torch.int32, device=device)
+        self.done = torch.zeros(batch, dtype=torch.uint8, device=device)
+        self.s = dg_canvas(self.tokens.data_ptr(), self.sc_state.data_ptr(), self.prev_argmax.data_ptr(),
+                           self.done.data_ptr(), batch)
+
+
+class StepOutputs:
+    def __init__(self, cfg: dg_model_config, batch: int, logits=False, routing=False, device="cuda"):
+        T = batch * DG_CANVAS
+        self.argmax = torch.zeros(batch, DG_CANVAS, dtype=torch.int32, device=device)
+        self.sample = torch.zeros_like(self.argmax)
+        self.entropy = torch.zeros(batch, DG_CANVAS, dtype=torch.float32, device=device)
+        self.pmax = torch.zeros_like(self.entropy)
+        self.lock = torch.zeros(batch, DG_CANVAS, dtype=torch.uint8, device=device)
+        self.mean_entropy = torch.zeros(batch, dtype=torch.float32, device=device)
+        self.stop = torch.zeros(batch, dtype=torch.uint8, device=device)
+        self.final_round = torch.zeros(batch, dtype=torch.uint8, device=device)
+        self.logits = (torch.zeros(batch, DG_CANVAS, cfg.vocab, dtype=torch.float32, device=device)
+                       if logits else None)
+        self.route_idx = (torch.zeros(cfg.n_layers, T, cfg.top_k, dtype=torch.int32, device=device)
+                          if routing else None)
+        self.route_w = (torch.zeros(cfg.n_layers, T, cfg.top_k, dtype=torch.float32, device=device)
+                        if routing else None)
+        self.s = dg_step_out(*[t.data_ptr() if t is not None else None for t in (
+            self.argmax, self.sample, self.entropy, self.pmax, self.lock, self.mean_entropy, self.stop,
+            self.final_round, self.logits, self.route_idx, self.route_w)])
+
+
+class Model:
+    """Weights + workspace + context handle for up to `batch` canvases."""
+
+    def __init__(self, cfg: dg_model_config, batch: int, seed: int = 0, kind_std=None, device="cuda",
+                 stream=None):
+        self.cfg = cfg
+        self.batch = batch
+        nw = lib.dg_weights_bytes(ctypes.byref(cfg))
+        if nw == 0:
+            raise ValueError(lib.dg_last_error().decode())
+        self.weights = torch.empty(nw, dtype=torch.uint8, device=device)
+        nws = lib.dg_workspace_bytes(ctypes.byref(cfg), batch)
+        self.workspace = torch.empty(nws, dtype=torch.uint8, device=device)
+        std = None
+        if kind_std:
+            arr = (ctypes.c_float * 32)()
+            for kind, v in kind_std.items():
+                arr[kind] = v
+            std = ctypes.cast(arr, ctypes.c_void_p)
+            self._std = arr
+        check(lib.dg_model_init_random(ctypes.byref(cfg), seed, std, _ptr(self.weights), _stream(stream)))
+        ctx = ctypes.c_void_p()
+        check(lib.dg_context_create(ctypes.byref(cfg), _ptr(self.weights), _ptr(self.workspace), nws, batch,
+                                    ctypes.byref(ctx)))
+        self.ctx = ctx
+
+    def close(self):
+        if getattr(self, "ctx", None):
+            lib.dg_context_destroy(self.ctx)
+            self.ctx = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def encode(self, kv: KVCache, tokens: torch.Tensor, stream=None):
+        assert tokens.dtype == torch.int32 and tokens.is_contiguous()
+        check(lib.dg_encode_context(self.ctx, ctypes.byref(kv.s), _ptr(tokens), tokens.shape[1],
+                                    _stream(stream)))
+
+    def canvas_init(self, cv: Canvas, block: int, seed: int, stream=None):
+        check(lib.dg_canvas_init(self.ctx, ctypes.byref(cv.s), block, seed, _stream(stream)))
+
+    def step(self, kv: KVCache, cv: Canvas, block: int, step: int, sampler: dg_sampler_config,
+             out: StepOutputs = None, stream=None):
+        args = dg_step_args(block, step, sampler)
+        check(lib.dg_denoise_step(self.ctx, ctypes.byref(kv.s), ctypes.byref(cv.s), ctypes.byref(args),
+                                  ctypes.byref(out.s) if out is not None else None, _stream(stream)))
+
+    def decode_block(self, kv: KVCache, cv: Canvas, block: int, sampler: dg_sampler_config, out_tokens,
+                     stream=None):
+        steps = (ctypes.c_int32 * cv.s.batch)()
+        stats = dg_block_stats(steps, 0)
+        args = dg_step_args(block, 0, sampler)
+        check(lib.dg_decode_block(self.ctx, ctypes.byref(kv.s), ctypes.byref(cv.s), ctypes.byref(args),
+                                  _ptr(out_tokens), ctypes.byref(stats), _stream(stream)))
+        return list(steps), stats.rounds
+
+    def check_device(self, stream=None):
+        check(lib.dg_check_device_error(self.ctx, _stream(stream)))

@@ -58,13 +58,17 @@ class Weights:
     lazily as float64 (one layer at a time).  `std` maps a tensor kind to its
     init standard deviation (default 0.02 for all)."""
 
-    def __init__(self, cfg: ModelConfig, seed: int = 0, std=None, threads: int = 0):
+    def __init__(self, cfg: ModelConfig, seed: int = 0, std=None, threads: int = 0,
+                 keep_chunks: bool = False):
         self.cfg = cfg
         self.seed = seed
         self.std = dict(std or {})
         self.threads = threads
         self._layer_idx = None
         self._layer = None
+        # keep_chunks: remember generated embedding / LM-head row blocks so
+        # that a timing run measures the arithmetic, not the input generator
+        self._chunks = {} if keep_chunks else None
 
     def _std(self, kind):
         return self.std.get(kind, synth.WEIGHT_STD)
@@ -103,11 +107,20 @@ class Weights:
             out[i] = self._mat(int(tok), 1, d, synth.KIND_EMB, synth.KIND_EMB)[0]
         return out
 
+    def _chunk(self, kind, v0, n):
+        key = (kind, v0, n)
+        if self._chunks is not None and key in self._chunks:
+            return self._chunks[key]
+        m = self._mat(v0, n, self.cfg.d_model, kind, kind)
+        if self._chunks is not None:
+            self._chunks[key] = m
+        return m
+
     def emb_chunk(self, v0: int, n: int) -> np.ndarray:
-        return self._mat(v0, n, self.cfg.d_model, synth.KIND_EMB, synth.KIND_EMB)
+        return self._chunk(synth.KIND_EMB, v0, n)
 
     def lm_chunk(self, v0: int, n: int) -> np.ndarray:
-        return self._mat(v0, n, self.cfg.d_model, synth.KIND_LM, synth.KIND_LM)
+        return self._chunk(synth.KIND_LM, v0, n)
 
     def sc(self) -> np.ndarray:
         d = self.cfg.d_model
@@ -182,7 +195,9 @@ def route(h, wr, top_k):
     experts by logit (ties to the lower expert id; the softmax over all
     experts is monotone in the logit) and their softmax probabilities
     renormalised over the chosen k (the full-softmax denominator cancels).
-    Returns (idx [T, k] int64, w [T, k] fp32 values, logits [T, E])."""
+    Returns (idx [T, k] int64, w [T, k] fp32 values, logits [T, E]).
+    route_margin() gives each token's smallest gap between consecutive
+    sorted logits among the first k + 1 (how close the choice is to a tie)."""
     logits = f32_round(h @ wr.T)
     T, E = logits.shape
     idx = np.empty((T, top_k), np.int64)
@@ -194,6 +209,13 @@ def route(h, wr, top_k):
         ex = np.exp(sel - sel.max())
         w[t] = ex / ex.sum()
     return idx, f32_round(w), logits
+
+
+def route_margin(logits, top_k):
+    s = -np.sort(-np.asarray(logits, dtype=np.float64), axis=1)[:, :top_k + 1]
+    if s.shape[1] < 2:
+        return np.full(s.shape[0], np.inf)
+    return np.min(s[:, :-1] - s[:, 1:], axis=1)
 
 
 def silu(a):
@@ -210,10 +232,10 @@ def expert_ffn(x, wg, wu, wd):
 def moe_ffn(h, layer, top_k):
     """Mixture-of-experts FFN on bf16 inputs h [T, d]: route, run each
     expert on the tokens sent to it, and combine sum_k w_k y_k (fp32 result).
-    Returns (out, idx, w)."""
+    Returns (out, idx, w, routing margin)."""
     wg, wu, wd = layer["wg"], layer["wu"], layer["wd"]
     E = wg.shape[0]
-    idx, w, _ = route(h, layer["wr"], top_k)
+    idx, w, logits = route(h, layer["wr"], top_k)
     T = h.shape[0]
     y = np.zeros((T, top_k, h.shape[1]))
     for e in range(E):
@@ -223,7 +245,7 @@ def moe_ffn(h, layer, top_k):
         y[tok, slot] = expert_ffn(h[tok], bf16_bits_to_f64(wg[e]), bf16_bits_to_f64(wu[e]),
                                   bf16_bits_to_f64(wd[e]))
     out = f32_round(np.sum(w[:, :, None] * y, axis=1))
-    return out, idx, w
+    return out, idx, w, route_margin(logits, top_k)
 
 
 def forward_layers(cfg: ModelConfig, W: Weights, x, kv: KVCache, causal: bool, append: bool,
@@ -236,7 +258,7 @@ def forward_layers(cfg: ModelConfig, W: Weights, x, kv: KVCache, causal: bool, a
     kv.length grows); a canvas pass uses causal=False and append=False (the
     canvas attends to the whole context and to itself, and its keys are not
     kept).  Returns the final residual stream.  `record`, if a list, receives
-    per-layer routing (idx, w)."""
+    per-layer routing (idx, w, margin)."""
     c = cfg
     B, n, d = x.shape
     L0 = kv.length
@@ -263,9 +285,9 @@ def forward_layers(cfg: ModelConfig, W: Weights, x, kv: KVCache, causal: bool, a
                 kv.v[l][b, L0:L0 + n] = vb
         x = f32_round(x + f32_round(o @ lw["wo"].T))
         h2 = bf16_round(rmsnorm(x, c.rms_eps)).reshape(B * n, d)
-        m, idx, w = moe_ffn(h2, lw, c.top_k)
+        m, idx, w, margin = moe_ffn(h2, lw, c.top_k)
         if record is not None:
-            record.append((idx.reshape(B, n, -1), w.reshape(B, n, -1)))
+            record.append((idx.reshape(B, n, -1), w.reshape(B, n, -1), margin.reshape(B, n)))
         x = f32_round(x + m.reshape(B, n, d))
     if append:
         kv.length = L0 + n

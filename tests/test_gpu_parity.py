@@ -1,0 +1,40 @@
+"""GPU (C ABI) vs oracle parity of the denoising step on seeded synthetic
+inputs: context encoding, canvas initialisation, logits, routing, per-position
+statistics, samples, lock masks, stop flags, the next canvas and the
+self-conditioning state, step by step."""
+
+import pytest
+
+from parity import Case, TINY, LAYER1, run_case
+
+pytestmark = pytest.mark.gpu
+
+
+def test_tiny_decode_prob_lock():
+    """2 layers, d 256, 8 heads x 32, 16 experts top-2, vocab 4096, 64 context
+    tokens, one canvas, 4 rounds, lock on max prob > 0.9, Philox seed 1234."""
+    rep = run_case(Case(cfg=TINY, ctx_len=64, steps=4))
+    assert rep.steps == 4 and rep.diverged_at == -1, rep
+
+
+def test_tiny_self_cond_entropy_cumsum_lock_batch2():
+    """Peaked LM head so that positions lock; cumulative-entropy lock rule;
+    self-conditioning; two canvases with their own contexts and streams;
+    ragged context length (not a multiple of 64)."""
+    rep = run_case(Case(cfg=TINY, self_cond=True, ctx_len=77, batch=2, steps=3, lm_std=2.0,
+                        sampler=dict(lock_policy="entropy_cumsum", lock_threshold=0.1)))
+    assert rep.steps >= 1, rep
+
+
+def test_tiny_peaked_prob_lock_and_stop():
+    """Locks fire (pmax > 0.9) and the adaptive stop fires at its threshold."""
+    rep = run_case(Case(cfg=TINY, ctx_len=300, steps=3, lm_std=2.5,
+                        sampler=dict(stop_entropy=3.0, stop_require_stable_argmax=False)))
+    assert rep.steps >= 1, rep
+
+
+def test_single_layer_full_width_step():
+    """1 layer, d 2816, 16 q / 8 kv heads x 176, 128 experts top-8, ffn 704,
+    vocab 262144, 2048 context tokens, one canvas, one round."""
+    rep = run_case(Case(cfg=LAYER1, ctx_len=2048, steps=1))
+    assert rep.steps == 1, rep
