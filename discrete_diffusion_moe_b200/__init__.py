@@ -61,7 +61,7 @@ class dg_step_out(ctypes.Structure):
     _fields_ = [("argmax", ctypes.c_void_p), ("sample", ctypes.c_void_p), ("entropy", ctypes.c_void_p),
                 ("pmax", ctypes.c_void_p), ("lock", ctypes.c_void_p), ("mean_entropy", ctypes.c_void_p),
                 ("stop", ctypes.c_void_p), ("final_round", ctypes.c_void_p), ("logits", ctypes.c_void_p),
-                ("route_idx", ctypes.c_void_p), ("route_w", ctypes.c_void_p)]
+                ("route_idx", ctypes.c_void_p), ("route_w", ctypes.c_void_p), ("hidden", ctypes.c_void_p)]
 
 
 DG_PROF_EXPERT_GATE_UP, DG_PROF_EXPERT_DOWN, DG_PROF_LM_HEAD, DG_PROF_ATTENTION, DG_PROF_DENSE, \
@@ -102,7 +102,9 @@ def _load():
         "dg_profile_start": (I32, [P]),
         "dg_profile_stop": (I32, [P, ctypes.POINTER(dg_profile)]),
         "dg_test_gemm": (I32, [P, I32, P, I32, I32, P, I32, P]),
-        "dg_test_grouped_gemm": (I32, [P, I32, I32, P, I32, I32, P, P, I32, P]),
+        "dg_test_grouped_gemm": (I32, [P, I32, I32, P, I32, I32, P, P, I32, P, P]),
+        "dg_test_attention": (I32, [P, P, P, P, I32, I32, I32, I32, I32, I32, I32, I32, I32, P, P, P]),
+        "dg_test_workspace_buffer": (I32, [P, ctypes.c_char_p, ctypes.POINTER(P), ctypes.POINTER(S)]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -185,8 +187,9 @@ def dg_test_gemm(d_a, M, d_b, N, K, d_d, k_splits, stream):
     return lib.dg_test_gemm(d_a, M, d_b, N, K, d_d, k_splits, stream)
 
 
-def dg_test_grouped_gemm(d_a, rows_per_group, n_groups, d_b, n_rows, K, d_off, d_d, bn, stream):
-    return lib.dg_test_grouped_gemm(d_a, rows_per_group, n_groups, d_b, n_rows, K, d_off, d_d, bn, stream)
+def dg_test_grouped_gemm(d_a, rows_per_group, n_groups, d_b, n_rows, K, d_off, d_d, bn, d_chunk_off, stream):
+    return lib.dg_test_grouped_gemm(d_a, rows_per_group, n_groups, d_b, n_rows, K, d_off, d_d, bn, d_chunk_off,
+                                    stream)
 
 
 from .runtime import Model, KVCache, Canvas, StepOutputs, sampler_config, model_config  # noqa: E402,F401

@@ -10,8 +10,12 @@
 // packed into G * nq rows, so one CTA's 64-row tile reuses each K/V tile for
 // all heads of the group.  Flash-style online softmax in the exp2 domain;
 // QK^T and PV run on bf16 mma.sync tensor-core instructions (m16n8k16, fp32
-// accumulate; P is rounded to bf16 as the PV operand).  Keys can be split
-// across CTAs (split-KV); partial (m, l, O) are merged in a fixed order.
+// accumulate).  The probabilities are split into a bf16 high part and a bf16
+// residual (P = P_hi + P_lo, two PV products), so the PV operand carries about
+// 16 significant bits instead of 8: the attention output of a long, nearly
+// uniform softmax is a heavily cancelling average, and plain bf16 P would put
+// a relative error of order 2^-9 on it.  Keys can be split across CTAs
+// (split-KV); partial (m, l, O) are merged in a fixed order.
 #pragma once
 
 #include "common.cuh"
@@ -193,19 +197,26 @@ __global__ void __launch_bounds__(128) attn_kernel(const AttnParams p) {
           l_r[rr] += pv;
         }
     }
-    // O += P V
+    // O += (P_hi + P_lo) V
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) {
-      const uint32_t a0 = pack_bf16x2(s[2 * kk][0], s[2 * kk][1]);
-      const uint32_t a1 = pack_bf16x2(s[2 * kk][2], s[2 * kk][3]);
-      const uint32_t a2 = pack_bf16x2(s[2 * kk + 1][0], s[2 * kk + 1][1]);
-      const uint32_t a3 = pack_bf16x2(s[2 * kk + 1][2], s[2 * kk + 1][3]);
+      uint32_t hi[4], lo[4];
+      const float* pr[4] = {&s[2 * kk][0], &s[2 * kk][2], &s[2 * kk + 1][0], &s[2 * kk + 1][2]};
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const float p0 = pr[r][0], p1 = pr[r][1];
+        hi[r] = pack_bf16x2(p0, p1);
+        const float h0 = bf16_to_f32(hi[r] & 0xFFFF), h1 = bf16_to_f32(hi[r] >> 16);
+        lo[r] = pack_bf16x2(p0 - h0, p1 - h1);
+      }
 #pragma unroll
       for (int dp = 0; dp < NT / 2; ++dp) {
         uint32_t b0, b1, b2, b3;
         ldsm_x4_t(smem_u32(cV + (kk * 16 + (lane & 15)) * LD + dp * 16 + (lane >> 4) * 8), b0, b1, b2, b3);
-        mma_bf16_16816(o[2 * dp], a0, a1, a2, a3, b0, b1);
-        mma_bf16_16816(o[2 * dp + 1], a0, a1, a2, a3, b2, b3);
+        mma_bf16_16816(o[2 * dp], hi[0], hi[1], hi[2], hi[3], b0, b1);
+        mma_bf16_16816(o[2 * dp + 1], hi[0], hi[1], hi[2], hi[3], b2, b3);
+        mma_bf16_16816(o[2 * dp], lo[0], lo[1], lo[2], lo[3], b0, b1);
+        mma_bf16_16816(o[2 * dp + 1], lo[0], lo[1], lo[2], lo[3], b2, b3);
       }
     }
     __syncthreads();

@@ -116,7 +116,7 @@ WLayout weight_layout(const dg_model_config& c) {
 constexpr int kMaxAttnSplits = 8;
 
 struct WsLayout {
-  size_t err, flags, x, xn, qkv, q, attn, attn_po, attn_pml, rpart, idx, w, off, perm, inv, wperm,
+  size_t err, flags, x, xn, qkv, q, attn, attn_po, attn_pml, rpart, idx, w, off, choff, perm, inv, wperm,
       xperm, hperm, yperm, logits, vp_m, vp_z, vp_s, vp_av, vp_ai, vp_gv, vp_gi, st_m, st_iz, st_h,
       st_pmax, st_amax, st_samp, probs, epart, total;
   int T_alloc, P_alloc, ks_r, n_vt, attn_rows_cap;
@@ -163,6 +163,7 @@ WsLayout ws_layout(const dg_model_config& c, int batch, int num_sms) {
   L.idx = take(P * 4);
   L.w = take(P * 4);
   L.off = take((E + 1) * 4);
+  L.choff = take((E + 1) * 4);
   L.perm = take(P * 4);
   L.inv = take(P * 4);
   L.wperm = take(P * 4);
@@ -237,8 +238,8 @@ dg_status run_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmPlan&
   }
   const int stages = gemm_pick_stages(p.bn);
   const size_t smem = gemm_smem_bytes(p.bn, stages);
-  long long units;
-  if (p.group_off) units = (long long)p.n_groups * p.m_tiles;
+  long long units;  // grouped: known only on the device; one persistent CTA per SM
+  if (p.group_off) units = num_sms;
   else units = (long long)p.m_tiles * ((p.n_total + p.bn - 1) / p.bn) * p.k_splits;
   if (units <= 0) return DG_OK;
   const int grid = (int)std::min<long long>(units, num_sms);
@@ -263,8 +264,10 @@ GemmPlan dense_plan(int K, int a_rows, int n_total, int bn, int b_box, int k_spl
   return p;
 }
 
-GemmPlan grouped_plan(int K, int rows_per_group, const int* off, int n_groups, int bn, int* err) {
+GemmPlan grouped_plan(int K, int rows_per_group, const int* off, const int* chunk_off, int n_groups, int bn,
+                      int* err) {
   GemmPlan p{};
+  p.chunk_off = chunk_off;
   p.K = K;
   p.a_rows = rows_per_group;
   p.m_tiles = (rows_per_group + 127) / 128;
@@ -444,7 +447,7 @@ extern "C" void dg_context_destroy(dg_ctx* ctx) { delete ctx; }
 // one pass of the transformer layers over T = B * nq tokens at positions
 // L0 .. L0 + nq - 1 (x already holds the embedded inputs)
 static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L0, bool causal,
-                                int32_t* dbg_idx, float* dbg_w, cudaStream_t st) {
+                                int32_t* dbg_idx, float* dbg_w, float* dbg_hidden, cudaStream_t st) {
   const dg_model_config& m = c->cfg;
   const WsLayout& L = c->L;
   const int T = B * nq, d = m.d_model, hd = m.head_dim, Hq = m.n_q_heads, Hkv = m.n_kv_heads;
@@ -454,8 +457,9 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
   float* x = c->at<float>(L.x);
   uint16_t* xn = c->at<uint16_t>(L.xn);
   const int bnT = token_bn(T), boxT = box_for(bnT);
+  // token rows per grouped unit: about twice the mean tokens per expert
   const int avg = std::max(1, P / E);
-  const int bnG = std::min(256, std::max(32, next_pow2(3 * avg)));
+  const int bnG = std::min(256, std::max(32, next_pow2(2 * avg)));
   const size_t kv_layer = (size_t)kv->batch * Hkv * kv->c_max * hd;
 
   CUtensorMap t_xn, t_attn, t_xperm, t_hperm;
@@ -543,8 +547,8 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
         dbg_idx ? dbg_idx + (size_t)l * T * k : nullptr, dbg_w ? dbg_w + (size_t)l * T * k : nullptr);
         CNT(c);
     permute_kernel<<<1, kPermThreads, (size_t)34 * E * sizeof(int), st>>>(
-        c->at<int>(L.idx), c->at<float>(L.w), P, E, c->at<int>(L.off), c->at<int>(L.perm),
-        c->at<int>(L.inv), c->at<float>(L.wperm), err);
+        c->at<int>(L.idx), c->at<float>(L.w), P, E, bnG, c->at<int>(L.off), c->at<int>(L.choff),
+        c->at<int>(L.perm), c->at<int>(L.inv), c->at<float>(L.wperm), err);
         CNT(c);
     gather_rows_kernel<<<P, 128, 0, st>>>(xn, c->at<int>(L.perm), c->at<uint16_t>(L.xperm), P, k, d);
     CNT(c);
@@ -552,7 +556,7 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
       ProfScope ps_(c, DG_PROF_EXPERT_GATE_UP, st);
       CUtensorMap ta;
       DG_TRY(make_tmap(&ta, c->wp(W.wgu), d, (long long)E * 2 * f, 128));
-      GemmPlan p = grouped_plan(d, 2 * f, c->at<int>(L.off), E, bnG, err);
+      GemmPlan p = grouped_plan(d, 2 * f, c->at<int>(L.off), c->at<int>(L.choff), E, bnG, err);
       p.a_hint = 1;
       p.b_hint = 2;
       EpiSwiGLU e{c->at<uint16_t>(L.hperm), f};
@@ -562,7 +566,7 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
       ProfScope ps_(c, DG_PROF_EXPERT_DOWN, st);
       CUtensorMap ta;
       DG_TRY(make_tmap(&ta, c->wp(W.wd), f, (long long)E * d, 128));
-      GemmPlan p = grouped_plan(f, d, c->at<int>(L.off), E, bnG, err);
+      GemmPlan p = grouped_plan(f, d, c->at<int>(L.off), c->at<int>(L.choff), E, bnG, err);
       p.a_hint = 1;
       p.b_hint = 2;
       EpiDown e{c->at<float>(L.yperm), d, c->at<float>(L.wperm)};
@@ -571,6 +575,9 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
     moe_combine_kernel<<<T, 256, 0, st>>>(x, c->at<float>(L.yperm), c->at<int>(L.inv), T, k, d);
     CNT(c);
     DG_CUDA(cudaGetLastError());
+    if (dbg_hidden)
+      DG_CUDA(cudaMemcpyAsync(dbg_hidden + (size_t)(l + 1) * T * d, x, (size_t)T * d * 4,
+                              cudaMemcpyDeviceToDevice, st));
   }
   return DG_OK;
 }
@@ -617,7 +624,7 @@ extern "C" dg_status dg_encode_context(dg_ctx* c, dg_kv* kv, const int32_t* d_to
     embed_kernel<<<T, 128, 0, st>>>(c->wp(c->wl.emb), tok_tmp, c->at<float>(c->L.x), T, d, c->cfg.vocab, c->err());
     CNT(c);
     DG_CUDA(cudaGetLastError());
-    DG_TRY(forward_layers(c, kv, B, nq, kv->length, true, nullptr, nullptr, st));
+    DG_TRY(forward_layers(c, kv, B, nq, kv->length, true, nullptr, nullptr, nullptr, st));
     kv->length += nq;
   }
   return DG_OK;
@@ -681,8 +688,11 @@ extern "C" dg_status dg_denoise_step(dg_ctx* c, const dg_kv* kv, dg_canvas* cv, 
     DG_CUDA(cudaGetLastError());
   }
 
+  if (o->hidden)
+    DG_CUDA(cudaMemcpyAsync(o->hidden, c->at<float>(L.x), (size_t)T * d * 4, cudaMemcpyDeviceToDevice, st));
+
   // a2-a6: transformer layers, bidirectional over the canvas
-  DG_TRY(forward_layers(c, kv, B, DG_CANVAS, kv->length, false, o->route_idx, o->route_w, st));
+  DG_TRY(forward_layers(c, kv, B, DG_CANVAS, kv->length, false, o->route_idx, o->route_w, o->hidden, st));
 
   // a7: final norm, LM head with online vocabulary statistics and sampling
   uint16_t* xn = c->at<uint16_t>(L.xn);
@@ -898,8 +908,8 @@ extern "C" dg_status dg_test_gemm(const uint16_t* A, int32_t M, const uint16_t* 
 
 extern "C" dg_status dg_test_grouped_gemm(const uint16_t* A, int32_t rows_per_group, int32_t n_groups,
                                           const uint16_t* B, int32_t n_rows, int32_t K, const int32_t* off,
-                                          float* D, int32_t bn, void* stream) {
-  if (!A || !B || !D || !off || rows_per_group < 1 || n_groups < 1 || n_rows < 16 || K < 64 || K % 64 ||
+                                          float* D, int32_t bn, int32_t* choff, void* stream) {
+  if (!A || !B || !D || !off || !choff || rows_per_group < 1 || n_groups < 1 || n_rows < 16 || K < 64 || K % 64 ||
       bn < 16 || bn > 256 || (bn & (bn - 1)))
     return fail(DG_ERR_INVALID_ARG, "dg_test_grouped_gemm: bad arguments");
   if ((long long)rows_per_group * n_groups < 128) return fail(DG_ERR_INVALID_ARG, "A needs >= 128 rows");
@@ -907,9 +917,63 @@ extern "C" dg_status dg_test_grouped_gemm(const uint16_t* A, int32_t rows_per_gr
   CUtensorMap ta, tb;
   DG_TRY(make_tmap(&ta, A, K, (long long)rows_per_group * n_groups, 128));
   DG_TRY(make_tmap(&tb, B, K, n_rows, 16));
-  GemmPlan p = grouped_plan(K, rows_per_group, off, n_groups, bn, nullptr);
+  chunk_offsets_kernel<<<1, 1, 0, st>>>(off, n_groups, bn, choff);
+  GemmPlan p = grouped_plan(K, rows_per_group, off, choff, n_groups, bn, nullptr);
   EpiGroupedT e{D, rows_per_group};
   DG_TRY(run_gemm(ta, tb, p, e, device_sms(), st));
   DG_CUDA(cudaStreamSynchronize(st));
   return DG_OK;
+}
+
+extern "C" dg_status dg_test_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out,
+                                       int32_t B, int32_t nq, int32_t L0, int32_t c_max, int32_t Hq, int32_t Hkv,
+                                       int32_t hd, int32_t causal, int32_t splits, float* part_o, float* part_ml,
+                                       void* stream) {
+  if (!q || !k || !v || !out || B < 1 || nq < 1 || L0 < 0 || L0 + nq > c_max || Hq < 1 || Hkv < 1 ||
+      Hq % Hkv || splits < 0 || splits > kMaxAttnSplits)
+    return fail(DG_ERR_INVALID_ARG, "dg_test_attention: bad arguments");
+  if (splits > 1 && (!part_o || !part_ml)) return fail(DG_ERR_INVALID_ARG, "split buffers are null");
+  if (!attn_smem_ready(hd)) return fail(DG_ERR_UNSUPPORTED, "head_dim %d", hd);
+  cudaStream_t st = (cudaStream_t)stream;
+  if (splits == 0) splits = 1;
+  const int q_tiles = ((Hq / Hkv) * nq + 63) / 64;
+  AttnParams ap{q, k, v, out, part_o, part_ml, B, nq, L0, c_max, Hq, Hkv, splits, causal,
+                (float)(1.4426950408889634 / sqrt((double)hd))};
+  dim3 grid(q_tiles, Hkv, B * splits);
+  switch (hd) {
+    case 32: attn_kernel<32><<<grid, 128, attn_smem_bytes<32>(), st>>>(ap); break;
+    case 64: attn_kernel<64><<<grid, 128, attn_smem_bytes<64>(), st>>>(ap); break;
+    case 128: attn_kernel<128><<<grid, 128, attn_smem_bytes<128>(), st>>>(ap); break;
+    case 176: attn_kernel<176><<<grid, 128, attn_smem_bytes<176>(), st>>>(ap); break;
+    default: return fail(DG_ERR_UNSUPPORTED, "head_dim %d", hd);
+  }
+  DG_CUDA(cudaGetLastError());
+  if (splits > 1) {
+    const long long n = (long long)B * Hq * nq * hd;
+    attn_combine_kernel<<<(unsigned)std::min<long long>((n + 255) / 256, 8192), 256, 0, st>>>(
+        part_o, part_ml, out, splits, B, Hq, nq, hd);
+    DG_CUDA(cudaGetLastError());
+  }
+  DG_CUDA(cudaStreamSynchronize(st));
+  return DG_OK;
+}
+
+extern "C" dg_status dg_test_workspace_buffer(dg_ctx* c, const char* name, void** ptr, size_t* bytes) {
+  if (!c || !name || !ptr || !bytes) return fail(DG_ERR_INVALID_ARG, "null argument");
+  const WsLayout& L = c->L;
+  struct Entry { const char* n; size_t off, next; };
+  const Entry tab[] = {{"x", L.x, L.xn}, {"xn", L.xn, L.qkv}, {"qkv", L.qkv, L.q}, {"q", L.q, L.attn},
+                       {"attn", L.attn, L.attn_po}, {"idx", L.idx, L.w}, {"w", L.w, L.off},
+                       {"off", L.off, L.perm}, {"perm", L.perm, L.inv}, {"inv", L.inv, L.wperm},
+                       {"wperm", L.wperm, L.xperm}, {"xperm", L.xperm, L.hperm}, {"hperm", L.hperm, L.yperm},
+                       {"yperm", L.yperm, L.logits}, {"logits", L.logits, L.vp_m},
+                       {"probs", L.probs, L.epart}};
+  for (const Entry& e : tab)
+    if (!strcmp(e.n, name)) {
+      if (!e.off && strcmp(name, "x")) return fail(DG_ERR_INVALID_ARG, "buffer %s not allocated", name);
+      *ptr = c->ws + e.off;
+      *bytes = e.next - e.off;
+      return DG_OK;
+    }
+  return fail(DG_ERR_INVALID_ARG, "unknown workspace buffer %s", name);
 }

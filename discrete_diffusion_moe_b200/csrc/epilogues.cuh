@@ -31,22 +31,33 @@ struct EpiStoreT {
     if (row >= j.m_valid) return;
     const int f = j.m_tile * 128 + row;
     float* base = out + (long long)j.ks * split_stride + f;
+    const int nv = j.n_valid - c0;  // valid columns in this chunk (may exceed 16)
+    if (mode == 0) {
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int n = c0 + i;
-      if (n < j.n_valid) {
-        const long long t = j.n0 + n;
-        float* p = base + t * ld;
-        if (mode == 0) {
-          *p = v[i];
-        } else if (mode == 1) {
-          *p += v[i];
-        } else {
-          int tok = __ldg(tokens + t);
-          if (tok < 0 || tok >= vocab) { set_error(err, kDevErrBadToken); tok = 0; }
-          *p = bf16_to_f32(__ldg(emb + (long long)tok * ld + f)) + v[i];
-        }
+      for (int i = 0; i < 16; ++i)
+        if (i < nv) base[(long long)(j.n0 + c0 + i) * ld] = v[i];
+    } else if (mode == 1) {
+      // all loads first: the 16 read-modify-writes then overlap their latency
+      float old[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) old[i] = i < nv ? base[(long long)(j.n0 + c0 + i) * ld] : 0.f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        if (i < nv) base[(long long)(j.n0 + c0 + i) * ld] = old[i] + v[i];
+    } else {
+      int tok[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) tok[i] = i < nv ? __ldg(tokens + j.n0 + c0 + i) : 0;
+      float e[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        int t = tok[i];
+        if (t < 0 || t >= vocab) { set_error(err, kDevErrBadToken); t = 0; }
+        e[i] = bf16_to_f32(__ldg(emb + (long long)t * ld + f));
       }
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        if (i < nv) base[(long long)(j.n0 + c0 + i) * ld] = e[i] + v[i];
     }
   }
 };
@@ -88,14 +99,13 @@ struct EpiDown {
                                         State&) const {
     if (row >= j.m_valid) return;
     const int f = j.m_tile * 128 + row;
+    const int nv = j.n_valid - c0;
+    float w[16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int n = c0 + i;
-      if (n < j.n_valid) {
-        const long long slot = j.n0 + n;
-        y[slot * d + f] = __ldg(w_slot + slot) * v[i];
-      }
-    }
+    for (int i = 0; i < 16; ++i) w[i] = i < nv ? __ldg(w_slot + j.n0 + c0 + i) : 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if (i < nv) y[(long long)(j.n0 + c0 + i) * d + f] = w[i] * v[i];
   }
 };
 

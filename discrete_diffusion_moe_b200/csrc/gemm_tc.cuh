@@ -16,11 +16,14 @@
 //
 // Two schedules:
 //   dense    units = (m_tile, n_tile, k_split); B rows [n_tile*bn, +bn)
-//   grouped  units = (group, m_tile); group g uses A rows
+//   grouped  units = (group, m_tile, chunk); group g uses A rows
 //            [g * a_rows_per_group + m_tile*128, +128) and B rows
-//            [group_off[g], group_off[g+1]) in passes of at most bn columns
+//            [group_off[g], group_off[g+1]) in chunks of at most bn rows
 //            (a mixture-of-experts layer: one group per expert, B rows are the
-//            tokens routed to it, typically a few dozen).
+//            tokens routed to it).  chunk_off[g] = sum over groups < g of
+//            ceil(rows / bn), built on the device; units are ordered group,
+//            then m_tile, then chunk, so the CTAs that run at the same time
+//            share each weight tile through L2 instead of re-reading HBM.
 //
 // Every mbarrier wait is bounded (see mbar_wait); a unit whose wait ran out
 // is abandoned, the error word is set, in-flight copies are drained and the
@@ -41,6 +44,7 @@ struct GemmPlan {
   int k_splits;          // dense: K loop split into this many units (>= 1)
   int n_fast;            // dense: 1 = consecutive units walk the N tiles of one A tile
   const int* group_off;  // grouped when non-null: [n_groups + 1] B row offsets
+  const int* chunk_off;  // grouped: [n_groups + 1] prefix sums of ceil(rows / bn)
   int n_groups;
   int a_rows_per_group;  // grouped: A row stride between groups
   int a_hint, b_hint;    // L2 policy of the A / B loads: 0 none, 1 evict_first, 2 evict_last
@@ -60,30 +64,36 @@ struct GemmJob {
 };
 
 __device__ __forceinline__ int gemm_num_units(const GemmPlan& p) {
-  if (p.group_off) return p.n_groups * p.m_tiles;
+  if (p.group_off) return p.m_tiles * __ldg(p.chunk_off + p.n_groups);
   const int n_tiles = (p.n_total + p.bn - 1) / p.bn;
   return p.m_tiles * n_tiles * p.k_splits;
 }
 
-// Number of passes of unit u (0 for an empty group) and the job of pass `pass`.
-__device__ __forceinline__ int gemm_unit_passes(const GemmPlan& p, int u) {
-  if (!p.group_off) return 1;
-  const int g = u / p.m_tiles;
-  const int n = __ldg(p.group_off + g + 1) - __ldg(p.group_off + g);
-  return n <= 0 ? 0 : (n + p.bn - 1) / p.bn;
-}
+// Every unit is one pass (kept as a loop level so a unit could be split).
+__device__ __forceinline__ int gemm_unit_passes(const GemmPlan&, int) { return 1; }
 
-__device__ __forceinline__ GemmJob gemm_job(const GemmPlan& p, int u, int pass) {
+__device__ __forceinline__ GemmJob gemm_job(const GemmPlan& p, int u, int) {
   GemmJob j;
   const int kb_total = p.K / 64;
   if (p.group_off) {
-    const int g = u / p.m_tiles;
-    j.m_tile = u - g * p.m_tiles;
+    // group g with m_tiles * chunk_off[g] <= u < m_tiles * chunk_off[g + 1]
+    int lo = 0, hi = p.n_groups;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (p.m_tiles * __ldg(p.chunk_off + mid) <= u) lo = mid;
+      else hi = mid;
+    }
+    const int g = lo;
+    const int c0 = __ldg(p.chunk_off + g);
+    const int nch = __ldg(p.chunk_off + g + 1) - c0;
+    const int r = u - p.m_tiles * c0;
+    j.m_tile = r / nch;
+    const int ch = r - j.m_tile * nch;
     j.group = g;
     j.a_row0 = g * p.a_rows_per_group + j.m_tile * 128;
     j.m_valid = min(128, p.a_rows - j.m_tile * 128);
     const int off0 = __ldg(p.group_off + g), off1 = __ldg(p.group_off + g + 1);
-    j.n_local0 = pass * p.bn;
+    j.n_local0 = ch * p.bn;
     j.n0 = off0 + j.n_local0;
     j.n_valid = min(p.bn, off1 - j.n0);
     j.ks = 0;

@@ -193,7 +193,8 @@ __global__ void router_topk_kernel(const float* __restrict__ part, int ks, int T
 constexpr int kPermThreads = 1024;
 __global__ void __launch_bounds__(kPermThreads) permute_kernel(const int* __restrict__ idx,
                                                                const float* __restrict__ w, int P,
-                                                               int E, int* __restrict__ off,
+                                                               int E, int bn, int* __restrict__ off,
+                                                               int* __restrict__ chunk_off,
                                                                int* __restrict__ perm,
                                                                int* __restrict__ inv,
                                                                float* __restrict__ w_perm, int* err) {
@@ -211,9 +212,16 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(const int* __rest
   }
   __syncthreads();
   if (tid == 0) {
-    int acc = 0;
-    for (int e = 0; e < E; ++e) { off[e] = acc; base[e] = acc; acc += cnt[e]; }
+    int acc = 0, acc_c = 0;
+    for (int e = 0; e < E; ++e) {
+      off[e] = acc;
+      base[e] = acc;
+      chunk_off[e] = acc_c;
+      acc += cnt[e];
+      acc_c += (cnt[e] + bn - 1) / bn;
+    }
     off[E] = acc;
+    chunk_off[E] = acc_c;
   }
   __syncthreads();
   for (int c0 = 0; c0 < P; c0 += kPermThreads) {
@@ -245,6 +253,18 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(const int* __rest
     }
     __syncthreads();
   }
+}
+
+// chunk_off[g] = sum_{h < g} ceil((off[h+1] - off[h]) / bn)  (one thread)
+__global__ void chunk_offsets_kernel(const int* __restrict__ off, int G, int bn, int* __restrict__ chunk_off) {
+  if (blockIdx.x != 0 || threadIdx.x != 0) return;
+  int acc = 0;
+  for (int g = 0; g < G; ++g) {
+    chunk_off[g] = acc;
+    const int n = off[g + 1] - off[g];
+    acc += n > 0 ? (n + bn - 1) / bn : 0;
+  }
+  chunk_off[G] = acc;
 }
 
 // X_perm[slot, :] = xn[perm[slot] / k, :]  (bf16 rows, 16-byte vectors)

@@ -66,7 +66,8 @@ class Canvas:
 
 
 class StepOutputs:
-    def __init__(self, cfg: dg_model_config, batch: int, logits=False, routing=False, device="cuda"):
+    def __init__(self, cfg: dg_model_config, batch: int, logits=False, routing=False, hidden=False,
+                 device="cuda"):
         T = batch * DG_CANVAS
         self.argmax = torch.zeros(batch, DG_CANVAS, dtype=torch.int32, device=device)
         self.sample = torch.zeros_like(self.argmax)
@@ -82,9 +83,11 @@ class StepOutputs:
                           if routing else None)
         self.route_w = (torch.zeros(cfg.n_layers, T, cfg.top_k, dtype=torch.float32, device=device)
                         if routing else None)
+        self.hidden = (torch.zeros(cfg.n_layers + 1, T, cfg.d_model, dtype=torch.float32, device=device)
+                       if hidden else None)
         self.s = dg_step_out(*[t.data_ptr() if t is not None else None for t in (
             self.argmax, self.sample, self.entropy, self.pmax, self.lock, self.mean_entropy, self.stop,
-            self.final_round, self.logits, self.route_idx, self.route_w)])
+            self.final_round, self.logits, self.route_idx, self.route_w, self.hidden)])
 
 
 class Model:

@@ -29,10 +29,32 @@ dg_status dg_test_gemm(const uint16_t* d_a, int32_t M, const uint16_t* d_b, int3
    [off[g], off[g+1]) and writes D[r, f] (fp32, [n_rows, rows_per_group]) for
    each B row r of the group and each A row f of the group.  d_off is a
    device int32 array of n_groups + 1 non-decreasing offsets ending at n_rows.
-   bn (16..256, power of two) is the number of B rows per pass.  Synchronous. */
+   bn (16..256, power of two) is the number of B rows per unit; d_chunk_off
+   is caller-provided device scratch of n_groups + 1 int32.  Synchronous. */
 dg_status dg_test_grouped_gemm(const uint16_t* d_a, int32_t rows_per_group, int32_t n_groups,
                                const uint16_t* d_b, int32_t n_rows, int32_t K, const int32_t* d_off,
-                               float* d_d, int32_t bn, void* stream);
+                               float* d_d, int32_t bn, int32_t* d_chunk_off, void* stream);
+
+/* The library's attention kernel on its own: q bf16 [B * nq, Hq * hd]
+   (token-major), K/V caches bf16 [B][Hkv][c_max][hd] holding keys
+   [0, L0 + nq), out bf16 [B * nq, Hq * hd].  causal = 0: every query sees
+   all L0 + nq keys; causal = 1: query i sees keys [0, L0 + i].  splits > 0
+   forces that many key splits (0: the library's own choice).  The split
+   partial buffers come from the caller: part_o fp32 [splits * B * Hq * nq * hd]
+   and part_ml fp32 [splits * B * Hq * nq * 2].  Synchronous. */
+dg_status dg_test_attention(const uint16_t* d_q, const uint16_t* d_k, const uint16_t* d_v, uint16_t* d_out,
+                            int32_t B, int32_t nq, int32_t L0, int32_t c_max, int32_t Hq, int32_t Hkv,
+                            int32_t hd, int32_t causal, int32_t splits, float* d_part_o,
+                            float* d_part_ml, void* stream);
+
+/* Device address and size of one named scratch buffer of a context's
+   workspace (for inspecting the last layer's intermediates after a call):
+   "x" fp32 residual [T, d], "xn" bf16 normed activations, "qkv" fp32,
+   "q" bf16 [T, Hq*hd], "attn" bf16 [T, Hq*hd], "idx" int32 [T, k],
+   "w" fp32 [T, k], "off" int32 [E+1], "perm", "inv" int32 [T*k],
+   "wperm" fp32 [T*k], "xperm" bf16 [T*k, d], "hperm" bf16 [T*k, f],
+   "yperm" fp32 [T*k, d], "logits" fp32 [T, V], "probs" bf16 [T, V]. */
+dg_status dg_test_workspace_buffer(dg_ctx* ctx, const char* name, void** d_ptr, size_t* bytes);
 
 #ifdef __cplusplus
 }

@@ -258,7 +258,7 @@ def forward_layers(cfg: ModelConfig, W: Weights, x, kv: KVCache, causal: bool, a
     kv.length grows); a canvas pass uses causal=False and append=False (the
     canvas attends to the whole context and to itself, and its keys are not
     kept).  Returns the final residual stream.  `record`, if a list, receives
-    per-layer routing (idx, w, margin)."""
+    per layer (routing idx, weights, routing margin, residual stream after the layer)."""
     c = cfg
     B, n, d = x.shape
     L0 = kv.length
@@ -286,9 +286,9 @@ def forward_layers(cfg: ModelConfig, W: Weights, x, kv: KVCache, causal: bool, a
         x = f32_round(x + f32_round(o @ lw["wo"].T))
         h2 = bf16_round(rmsnorm(x, c.rms_eps)).reshape(B * n, d)
         m, idx, w, margin = moe_ffn(h2, lw, c.top_k)
-        if record is not None:
-            record.append((idx.reshape(B, n, -1), w.reshape(B, n, -1), margin.reshape(B, n)))
         x = f32_round(x + m.reshape(B, n, d))
+        if record is not None:
+            record.append((idx.reshape(B, n, -1), w.reshape(B, n, -1), margin.reshape(B, n), x.copy()))
     if append:
         kv.length = L0 + n
     return x

@@ -44,20 +44,23 @@ def test_dense_gemm(dg, M, N, K, ks):
     assert np.abs(got - ref).max() <= tol * np.abs(ref).max() + 1e-4, np.abs(got - ref).max()
 
 
-@pytest.mark.parametrize("bn", [16, 32, 64, 256])
-def test_grouped_gemm(dg, bn):
-    rng = np.random.default_rng(bn)
+@pytest.mark.parametrize("bn,sizes", [(16, [17, 0, 43, 1, 90, 5]), (32, [17, 0, 43, 1, 90, 5]),
+                                      (64, [17, 0, 43, 1, 90, 5]), (256, [17, 0, 43, 1, 90, 5]),
+                                      # skewed routing: one group holds most rows
+                                      (64, [3, 600, 0, 0, 9, 300])])
+def test_grouped_gemm(dg, bn, sizes):
+    rng = np.random.default_rng(bn + len(sizes) + sizes[1])
     G, R, K = 6, 256, 192
-    sizes = [17, 0, 43, 1, 90, 5]
     off = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
     n = int(off[-1])
     a, b = _bf16(rng, (G * R, K)), _bf16(rng, (n, K))
     dd = torch.full((n, R), float("nan"), device="cuda")
     doff = torch.from_numpy(off).cuda()
     da, db = a.cuda(), b.cuda()  # keep the device copies alive across the call
+    choff = torch.zeros(G + 1, dtype=torch.int32, device="cuda")
     st = torch.cuda.current_stream().cuda_stream
     dg.check(dg.dg_test_grouped_gemm(da.data_ptr(), R, G, db.data_ptr(), n, K, doff.data_ptr(),
-                                     dd.data_ptr(), bn, st))
+                                     dd.data_ptr(), bn, choff.data_ptr(), st))
     got = dd.double().cpu().numpy()
     A = a.double().numpy().reshape(G, R, K)
     B = b.double().numpy()
