@@ -61,7 +61,8 @@ class dg_step_out(ctypes.Structure):
     _fields_ = [("argmax", ctypes.c_void_p), ("sample", ctypes.c_void_p), ("entropy", ctypes.c_void_p),
                 ("pmax", ctypes.c_void_p), ("lock", ctypes.c_void_p), ("mean_entropy", ctypes.c_void_p),
                 ("stop", ctypes.c_void_p), ("final_round", ctypes.c_void_p), ("logits", ctypes.c_void_p),
-                ("route_idx", ctypes.c_void_p), ("route_w", ctypes.c_void_p), ("hidden", ctypes.c_void_p)]
+                ("route_idx", ctypes.c_void_p), ("route_w", ctypes.c_void_p), ("route_logits", ctypes.c_void_p),
+                ("hidden", ctypes.c_void_p)]
 
 
 DG_PROF_EXPERT_GATE_UP, DG_PROF_EXPERT_DOWN, DG_PROF_LM_HEAD, DG_PROF_ATTENTION, DG_PROF_DENSE, \

@@ -118,7 +118,7 @@ constexpr int kMaxAttnSplits = 8;
 struct WsLayout {
   size_t err, flags, x, xn, qkv, q, attn, attn_po, attn_pml, rpart, idx, w, off, choff, perm, inv, wperm,
       xperm, hperm, yperm, logits, vp_m, vp_z, vp_s, vp_av, vp_ai, vp_gv, vp_gi, st_m, st_iz, st_h,
-      st_pmax, st_amax, st_samp, probs, epart, total;
+      st_pmax, st_amax, st_samp, probs, epart, rope, total;
   int T_alloc, P_alloc, ks_r, n_vt, attn_rows_cap;
   long long epart_rows;
 };
@@ -176,6 +176,7 @@ WsLayout ws_layout(const dg_model_config& c, int batch, int num_sms) {
   L.vp_ai = take(nvp); L.vp_gv = take(nvp); L.vp_gi = take(nvp);
   L.st_m = take(T * 4); L.st_iz = take(T * 4); L.st_h = take(T * 4); L.st_pmax = take(T * 4);
   L.st_amax = take(T * 4); L.st_samp = take(T * 4);
+  L.rope = take((size_t)DG_CANVAS * (c.head_dim / 2) * 16);
   L.probs = c.self_cond ? take(T * V * 2) : 0;
   L.epart = c.self_cond ? take((size_t)er * d * 4) : 0;
   L.total = off;
@@ -447,7 +448,8 @@ extern "C" void dg_context_destroy(dg_ctx* ctx) { delete ctx; }
 // one pass of the transformer layers over T = B * nq tokens at positions
 // L0 .. L0 + nq - 1 (x already holds the embedded inputs)
 static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L0, bool causal,
-                                int32_t* dbg_idx, float* dbg_w, float* dbg_hidden, cudaStream_t st) {
+                                int32_t* dbg_idx, float* dbg_w, float* dbg_logits, float* dbg_hidden,
+                                cudaStream_t st) {
   const dg_model_config& m = c->cfg;
   const WsLayout& L = c->L;
   const int T = B * nq, d = m.d_model, hd = m.head_dim, Hq = m.n_q_heads, Hkv = m.n_kv_heads;
@@ -467,6 +469,14 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
   DG_TRY(make_tmap(&t_attn, c->at<uint16_t>(L.attn), (long long)Hq * hd, L.T_alloc, boxT));
   DG_TRY(make_tmap(&t_xperm, c->at<uint16_t>(L.xperm), d, L.P_alloc, 16));
   DG_TRY(make_tmap(&t_hperm, c->at<uint16_t>(L.hperm), f, L.P_alloc, 16));
+
+  // cos/sin of this pass's positions, shared by all layers
+  {
+    const int n = nq * (hd / 2);
+    rope_table_kernel<<<(n + 255) / 256, 256, 0, st>>>(c->at<double2>(L.rope), nq, L0, hd / 2, hd,
+                                                       (double)m.rope_theta);
+    CNT(c);
+  }
 
   // attention launch shape
   const int q_tiles = ((Hq / Hkv) * nq + 63) / 64;
@@ -494,8 +504,8 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
       DG_TRY(run_gemm(ta, t_xn, p, e, c->num_sms, st, &c->n_launch));
     }
     {
-      RopeParams rp{c->at<float>(L.qkv), c->at<uint16_t>(L.q), kc, vc, T, nq, L0, kv->c_max, Hq, Hkv, hd,
-                    (double)m.rope_theta};
+      RopeParams rp{c->at<float>(L.qkv), c->at<double2>(L.rope), c->at<uint16_t>(L.q), kc, vc, T, nq, L0,
+                    kv->c_max, Hq, Hkv, hd};
       rope_kv_kernel<<<std::min(4096, (T * (Hq + 2 * Hkv) * hd / 2 + 255) / 256), 256, 0, st>>>(rp);
       CNT(c);
     }
@@ -544,7 +554,8 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
     }
     router_topk_kernel<<<(T * 32 + 255) / 256, 256, 0, st>>>(
         c->at<float>(L.rpart), L.ks_r, T, E, k, c->at<int>(L.idx), c->at<float>(L.w),
-        dbg_idx ? dbg_idx + (size_t)l * T * k : nullptr, dbg_w ? dbg_w + (size_t)l * T * k : nullptr);
+        dbg_idx ? dbg_idx + (size_t)l * T * k : nullptr, dbg_w ? dbg_w + (size_t)l * T * k : nullptr,
+        dbg_logits ? dbg_logits + (size_t)l * T * E : nullptr);
         CNT(c);
     permute_kernel<<<1, kPermThreads, (size_t)34 * E * sizeof(int), st>>>(
         c->at<int>(L.idx), c->at<float>(L.w), P, E, bnG, c->at<int>(L.off), c->at<int>(L.choff),
@@ -624,7 +635,7 @@ extern "C" dg_status dg_encode_context(dg_ctx* c, dg_kv* kv, const int32_t* d_to
     embed_kernel<<<T, 128, 0, st>>>(c->wp(c->wl.emb), tok_tmp, c->at<float>(c->L.x), T, d, c->cfg.vocab, c->err());
     CNT(c);
     DG_CUDA(cudaGetLastError());
-    DG_TRY(forward_layers(c, kv, B, nq, kv->length, true, nullptr, nullptr, nullptr, st));
+    DG_TRY(forward_layers(c, kv, B, nq, kv->length, true, nullptr, nullptr, nullptr, nullptr, st));
     kv->length += nq;
   }
   return DG_OK;
@@ -692,7 +703,8 @@ extern "C" dg_status dg_denoise_step(dg_ctx* c, const dg_kv* kv, dg_canvas* cv, 
     DG_CUDA(cudaMemcpyAsync(o->hidden, c->at<float>(L.x), (size_t)T * d * 4, cudaMemcpyDeviceToDevice, st));
 
   // a2-a6: transformer layers, bidirectional over the canvas
-  DG_TRY(forward_layers(c, kv, B, DG_CANVAS, kv->length, false, o->route_idx, o->route_w, o->hidden, st));
+  DG_TRY(forward_layers(c, kv, B, DG_CANVAS, kv->length, false, o->route_idx, o->route_w, o->route_logits,
+                        o->hidden, st));
 
   // a7: final norm, LM head with online vocabulary statistics and sampling
   uint16_t* xn = c->at<uint16_t>(L.xn);
@@ -721,8 +733,8 @@ extern "C" dg_status dg_denoise_step(dg_ctx* c, const dg_kv* kv, dg_canvas* cv, 
   PosStats ps{c->at<float>(L.st_m), c->at<float>(L.st_iz), o->entropy ? o->entropy : c->at<float>(L.st_h),
               o->pmax ? o->pmax : c->at<float>(L.st_pmax), o->argmax ? o->argmax : c->at<int>(L.st_amax),
               o->sample ? o->sample : c->at<int>(L.st_samp)};
-  vocab_merge_kernel<<<(T * 32 + 255) / 256, 256, 0, st>>>(vp.m, vp.z, vp.s, vp.amax_v, vp.amax_i, vp.gkey_v,
-                                                           vp.gkey_i, L.n_vt, T, log((double)V), ps);
+  vocab_merge_kernel<<<T, kMergeThreads, 0, st>>>(vp.m, vp.z, vp.s, vp.amax_v, vp.amax_i, vp.gkey_v,
+                                                  vp.gkey_i, L.n_vt, T, log((double)V), ps);
                                                            CNT(c);
   DG_CUDA(cudaGetLastError());
 
@@ -963,7 +975,8 @@ extern "C" dg_status dg_test_workspace_buffer(dg_ctx* c, const char* name, void*
   const WsLayout& L = c->L;
   struct Entry { const char* n; size_t off, next; };
   const Entry tab[] = {{"x", L.x, L.xn}, {"xn", L.xn, L.qkv}, {"qkv", L.qkv, L.q}, {"q", L.q, L.attn},
-                       {"attn", L.attn, L.attn_po}, {"idx", L.idx, L.w}, {"w", L.w, L.off},
+                       {"attn", L.attn, L.attn_po}, {"rpart", L.rpart, L.idx}, {"idx", L.idx, L.w},
+                       {"w", L.w, L.off},
                        {"off", L.off, L.perm}, {"perm", L.perm, L.inv}, {"inv", L.inv, L.wperm},
                        {"wperm", L.wperm, L.xperm}, {"xperm", L.xperm, L.hperm}, {"hperm", L.hperm, L.yperm},
                        {"yperm", L.yperm, L.logits}, {"logits", L.logits, L.vp_m},

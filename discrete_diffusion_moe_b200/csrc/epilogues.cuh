@@ -114,7 +114,9 @@ struct EpiDown {
 // position and per vocabulary tile, the online softmax statistics
 //   m = max l, Z = sum e^(l - m), S = sum e^(l - m) l,
 // the argmax (first maximum) and the Gumbel-max key argmax_v (l_v / T + g_v)
-// with g = -ln(-ln u) from Philox (purpose 2, c0 = v / 4, word v % 4).
+// with g = -ln(-ln u) from Philox (purpose 2, c0 = v / 4, word v % 4).  The
+// inner logarithm uses the accurate logf: for u within ~1e-5 of 1, where the
+// largest keys come from, the fast __logf has only absolute accuracy.
 struct VocabPartials {
   float* m;
   float* z;
@@ -177,7 +179,9 @@ struct EpiLMHead {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float u = gumbel_u(w[e]);
-        const float g = -__logf(-__logf(u));
+        // -ln(u) needs relative accuracy for u near 1 (the largest Gumbel keys,
+        // which decide the sample): the accurate logf there, the fast one outside
+        const float g = -__logf(-logf(u));
         const float key = __fadd_rn(__fmul_rn(v[4 * q + e], inv_t), g);
         if (key > st.gv) { st.gv = key; st.gi = vb + 4 * q + e; }
       }

@@ -69,16 +69,29 @@ __global__ void __launch_bounds__(THREADS) rmsnorm_kernel(const float* __restric
 }
 
 // ---------------------------------------------------------------------------
-// RoPE on q and k (pairs (i, i + hd/2) rotated by pos * theta^(-2i/hd), angle
-// and rotation in double), q -> bf16 [T, Hq*hd]; k, v -> bf16 KV cache of this
-// layer at position L0 + i of each canvas ([B][Hkv][c_max][hd]).
+// RoPE: pairs (i, i + hd/2) rotated by the angle pos * theta^(-2i/hd).  The
+// cos/sin of each (position, pair) are computed once per pass in double
+// (rope_table_kernel) and shared by all layers; the rotation is done in
+// double from the fp32 projection and rounded once to bf16.
+// q -> bf16 [T, Hq*hd]; k, v -> bf16 KV cache of this layer at position
+// L0 + i of each canvas ([B][Hkv][c_max][hd]).
+__global__ void rope_table_kernel(double2* __restrict__ tab, int nq, int L0, int half, int hd, double theta) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= nq * half) return;
+  const int pos_in = e / half, i = e - pos_in * half;
+  const double inv_freq = pow(theta, -2.0 * (double)i / (double)hd);
+  double sn, cs;
+  sincos((double)(L0 + pos_in) * inv_freq, &sn, &cs);
+  tab[e] = make_double2(cs, sn);
+}
+
 struct RopeParams {
   const float* qkv;   // [T, (Hq + 2 Hkv) * hd]
+  const double2* tab; // [nq, hd/2] (cos, sin)
   uint16_t* q;        // [T, Hq * hd]
   uint16_t* kc;       // layer base of K cache
   uint16_t* vc;       // layer base of V cache
   int T, nq, L0, c_max, Hq, Hkv, hd;
-  double theta;
 };
 
 __global__ void rope_kv_kernel(const RopeParams p) {
@@ -95,13 +108,10 @@ __global__ void rope_kv_kernel(const RopeParams p) {
       const int h = (int)(r % heads);
       const int t = (int)(r / heads);
       const int b = t / p.nq, pos_in = t - b * p.nq;
-      const double pos = (double)(p.L0 + pos_in);
-      const double inv_freq = pow(p.theta, -2.0 * (double)i / (double)p.hd);
-      double sn, cs;
-      sincos(pos * inv_freq, &sn, &cs);
+      const double2 cs = p.tab[pos_in * half + i];
       const float* src = p.qkv + (long long)t * row_w + h * p.hd;
       const double x1 = src[i], x2 = src[i + half];
-      const float o1 = (float)(x1 * cs - x2 * sn), o2 = (float)(x2 * cs + x1 * sn);
+      const float o1 = (float)(x1 * cs.x - x2 * cs.y), o2 = (float)(x2 * cs.x + x1 * cs.y);
       uint16_t* dst;
       if (h < p.Hq) {
         dst = p.q + (long long)t * p.Hq * p.hd + h * p.hd;
@@ -132,7 +142,8 @@ __global__ void rope_kv_kernel(const RopeParams p) {
 // One warp per token; E <= 256.
 __global__ void router_topk_kernel(const float* __restrict__ part, int ks, int T, int E, int k,
                                    int* __restrict__ idx, float* __restrict__ w,
-                                   int* __restrict__ dbg_idx, float* __restrict__ dbg_w) {
+                                   int* __restrict__ dbg_idx, float* __restrict__ dbg_w,
+                                   float* __restrict__ dbg_logits) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= T) return;
@@ -140,15 +151,21 @@ __global__ void router_topk_kernel(const float* __restrict__ part, int ks, int T
   float l[8];
   bool taken[8];
 #pragma unroll
+  for (int q = 0; q < 8; ++q) { l[q] = 0.f; taken[q] = false; }
+  // split-k partials summed in split order; the 8 expert slots of a lane are
+  // independent, so their loads are issued together
+  for (int p = 0; p < ks; ++p) {
+    const float* row = part + ((long long)p * T + t) * E;
+    float v[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) v[q] = (lane + 32 * q < E) ? row[lane + 32 * q] : 0.f;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) l[q] += v[q];
+  }
+#pragma unroll
   for (int q = 0; q < 8; ++q) {
-    const int e = lane + 32 * q;
-    float s = -INFINITY;
-    if (e < E) {
-      s = 0.f;
-      for (int p = 0; p < ks; ++p) s += part[((long long)p * T + t) * E + e];
-    }
-    l[q] = s;
-    taken[q] = false;
+    if (lane + 32 * q >= E) l[q] = -INFINITY;
+    else if (dbg_logits) dbg_logits[(long long)t * E + lane + 32 * q] = l[q];
   }
   float sel_l[8];
   int sel_e[8];
@@ -323,20 +340,24 @@ __device__ __forceinline__ void merge_ms(double& m, double& z, double& s, double
   m = mn;
 }
 
-__global__ void vocab_merge_kernel(const float* __restrict__ pm, const float* __restrict__ pz,
-                                   const float* __restrict__ ps, const float* __restrict__ pav,
-                                   const int* __restrict__ pai, const float* __restrict__ pgv,
-                                   const int* __restrict__ pgi, int n_vt, int T, double log_v,
-                                   PosStats out) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (warp >= T) return;
-  const long long base = (long long)warp * n_vt;
-  double m = -INFINITY, z = 0.0, s = 0.0;
+constexpr int kMergeThreads = 256;
+// One CTA per position: thread i folds tiles i, i + 256, ... in order, then a
+// fixed binary tree over the 256 partial states (shared memory) in double.
+__global__ void __launch_bounds__(kMergeThreads) vocab_merge_kernel(
+    const float* __restrict__ pm, const float* __restrict__ pz, const float* __restrict__ ps,
+    const float* __restrict__ pav, const int* __restrict__ pai, const float* __restrict__ pgv,
+    const int* __restrict__ pgi, int n_vt, int T, double log_v, PosStats out) {
+  __shared__ double sm_m[kMergeThreads], sm_z[kMergeThreads], sm_s[kMergeThreads];
+  __shared__ float sa_v[kMergeThreads], sg_v[kMergeThreads];
+  __shared__ int sa_i[kMergeThreads], sg_i[kMergeThreads];
+  const int t = blockIdx.x, tid = threadIdx.x;
+  if (t >= T) return;
+  const long long base = (long long)t * n_vt;
+  double m = -INFINITY, z = 0.0, s_ = 0.0;
   float av = -INFINITY, gv = -INFINITY;
   int ai = 0x7fffffff, gi = 0x7fffffff;
-  for (int v = lane; v < n_vt; v += 32) {
-    merge_ms(m, z, s, (double)pm[base + v], (double)pz[base + v], (double)ps[base + v]);
+  for (int v = tid; v < n_vt; v += kMergeThreads) {
+    merge_ms(m, z, s_, (double)pm[base + v], (double)pz[base + v], (double)ps[base + v]);
     const float a = pav[base + v];
     const int a_i = pai[base + v];
     if (a > av || (a == av && a_i < ai)) { av = a; ai = a_i; }
@@ -344,28 +365,33 @@ __global__ void vocab_merge_kernel(const float* __restrict__ pm, const float* __
     const int g_i = pgi[base + v];
     if (g > gv || (g == gv && g_i < gi)) { gv = g; gi = g_i; }
   }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const double m2 = __shfl_xor_sync(0xffffffffu, m, o);
-    const double z2 = __shfl_xor_sync(0xffffffffu, z, o);
-    const double s2 = __shfl_xor_sync(0xffffffffu, s, o);
-    merge_ms(m, z, s, m2, z2, s2);
-    const float a2 = __shfl_xor_sync(0xffffffffu, av, o);
-    const int ai2 = __shfl_xor_sync(0xffffffffu, ai, o);
-    if (a2 > av || (a2 == av && ai2 < ai)) { av = a2; ai = ai2; }
-    const float g2 = __shfl_xor_sync(0xffffffffu, gv, o);
-    const int gi2 = __shfl_xor_sync(0xffffffffu, gi, o);
-    if (g2 > gv || (g2 == gv && gi2 < gi)) { gv = g2; gi = gi2; }
+  sm_m[tid] = m; sm_z[tid] = z; sm_s[tid] = s_;
+  sa_v[tid] = av; sa_i[tid] = ai; sg_v[tid] = gv; sg_i[tid] = gi;
+  __syncthreads();
+  for (int h = kMergeThreads / 2; h > 0; h >>= 1) {
+    if (tid < h) {
+      double mm = sm_m[tid], zz = sm_z[tid], ss = sm_s[tid];
+      merge_ms(mm, zz, ss, sm_m[tid + h], sm_z[tid + h], sm_s[tid + h]);
+      sm_m[tid] = mm; sm_z[tid] = zz; sm_s[tid] = ss;
+      if (sa_v[tid + h] > sa_v[tid] || (sa_v[tid + h] == sa_v[tid] && sa_i[tid + h] < sa_i[tid])) {
+        sa_v[tid] = sa_v[tid + h]; sa_i[tid] = sa_i[tid + h];
+      }
+      if (sg_v[tid + h] > sg_v[tid] || (sg_v[tid + h] == sg_v[tid] && sg_i[tid + h] < sg_i[tid])) {
+        sg_v[tid] = sg_v[tid + h]; sg_i[tid] = sg_i[tid + h];
+      }
+    }
+    __syncthreads();
   }
-  if (lane == 0) {
-    double H = m + log(z) - s / z;
+  if (tid == 0) {
+    const double mm = sm_m[0], zz = sm_z[0], ss = sm_s[0];
+    double H = mm + log(zz) - ss / zz;
     H = fmin(fmax(H, 0.0), log_v);
-    out.m[warp] = (float)m;
-    out.inv_z[warp] = (float)(1.0 / z);
-    out.entropy[warp] = (float)H;
-    out.pmax[warp] = (float)(1.0 / z);
-    out.argmax[warp] = ai;
-    out.sample[warp] = gi;
+    out.m[t] = (float)mm;
+    out.inv_z[t] = (float)(1.0 / zz);
+    out.entropy[t] = (float)H;
+    out.pmax[t] = (float)(1.0 / zz);
+    out.argmax[t] = sa_i[0];
+    out.sample[t] = sg_i[0];
   }
 }
 

@@ -83,11 +83,13 @@ class StepOutputs:
                           if routing else None)
         self.route_w = (torch.zeros(cfg.n_layers, T, cfg.top_k, dtype=torch.float32, device=device)
                         if routing else None)
+        self.route_logits = (torch.zeros(cfg.n_layers, T, cfg.n_experts, dtype=torch.float32, device=device)
+                             if routing else None)
         self.hidden = (torch.zeros(cfg.n_layers + 1, T, cfg.d_model, dtype=torch.float32, device=device)
                        if hidden else None)
         self.s = dg_step_out(*[t.data_ptr() if t is not None else None for t in (
             self.argmax, self.sample, self.entropy, self.pmax, self.lock, self.mean_entropy, self.stop,
-            self.final_round, self.logits, self.route_idx, self.route_w, self.hidden)])
+            self.final_round, self.logits, self.route_idx, self.route_w, self.route_logits, self.hidden)])
 
 
 class Model:

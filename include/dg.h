@@ -137,6 +137,7 @@ typedef struct dg_step_out {
   float* logits;          /* optional [B, 256, vocab] fp32 LM-head logits */
   int32_t* route_idx;     /* optional [n_layers, B*256, top_k] expert ids */
   float* route_w;         /* optional [n_layers, B*256, top_k] renormalised weights */
+  float* route_logits;    /* optional [n_layers, B*256, n_experts] fp32 router logits */
   float* hidden;          /* optional [n_layers + 1, B*256, d_model] fp32 residual stream after
                              the embedding (a1) and after each layer */
 } dg_step_out;

@@ -50,7 +50,8 @@ dg_status dg_test_attention(const uint16_t* d_q, const uint16_t* d_k, const uint
 /* Device address and size of one named scratch buffer of a context's
    workspace (for inspecting the last layer's intermediates after a call):
    "x" fp32 residual [T, d], "xn" bf16 normed activations, "qkv" fp32,
-   "q" bf16 [T, Hq*hd], "attn" bf16 [T, Hq*hd], "idx" int32 [T, k],
+   "q" bf16 [T, Hq*hd], "attn" bf16 [T, Hq*hd], "rpart" fp32 split-k router
+   partial logits [splits, T, E], "idx" int32 [T, k],
    "w" fp32 [T, k], "off" int32 [E+1], "perm", "inv" int32 [T*k],
    "wperm" fp32 [T*k], "xperm" bf16 [T*k, d], "hperm" bf16 [T*k, f],
    "yperm" fp32 [T*k, d], "logits" fp32 [T, V], "probs" bf16 [T, V]. */

@@ -232,7 +232,7 @@ def expert_ffn(x, wg, wu, wd):
 def moe_ffn(h, layer, top_k):
     """Mixture-of-experts FFN on bf16 inputs h [T, d]: route, run each
     expert on the tokens sent to it, and combine sum_k w_k y_k (fp32 result).
-    Returns (out, idx, w, routing margin)."""
+    Returns (out, idx, w, routing margin, router logits)."""
     wg, wu, wd = layer["wg"], layer["wu"], layer["wd"]
     E = wg.shape[0]
     idx, w, logits = route(h, layer["wr"], top_k)
@@ -245,7 +245,7 @@ def moe_ffn(h, layer, top_k):
         y[tok, slot] = expert_ffn(h[tok], bf16_bits_to_f64(wg[e]), bf16_bits_to_f64(wu[e]),
                                   bf16_bits_to_f64(wd[e]))
     out = f32_round(np.sum(w[:, :, None] * y, axis=1))
-    return out, idx, w, route_margin(logits, top_k)
+    return out, idx, w, route_margin(logits, top_k), logits
 
 
 def forward_layers(cfg: ModelConfig, W: Weights, x, kv: KVCache, causal: bool, append: bool,
@@ -258,7 +258,8 @@ def forward_layers(cfg: ModelConfig, W: Weights, x, kv: KVCache, causal: bool, a
     kv.length grows); a canvas pass uses causal=False and append=False (the
     canvas attends to the whole context and to itself, and its keys are not
     kept).  Returns the final residual stream.  `record`, if a list, receives
-    per layer (routing idx, weights, routing margin, residual stream after the layer)."""
+    per layer (routing idx, weights, routing margin, residual stream after the
+    layer, router logits)."""
     c = cfg
     B, n, d = x.shape
     L0 = kv.length
@@ -285,10 +286,11 @@ def forward_layers(cfg: ModelConfig, W: Weights, x, kv: KVCache, causal: bool, a
                 kv.v[l][b, L0:L0 + n] = vb
         x = f32_round(x + f32_round(o @ lw["wo"].T))
         h2 = bf16_round(rmsnorm(x, c.rms_eps)).reshape(B * n, d)
-        m, idx, w, margin = moe_ffn(h2, lw, c.top_k)
+        m, idx, w, margin, rlog = moe_ffn(h2, lw, c.top_k)
         x = f32_round(x + m.reshape(B, n, d))
         if record is not None:
-            record.append((idx.reshape(B, n, -1), w.reshape(B, n, -1), margin.reshape(B, n), x.copy()))
+            record.append((idx.reshape(B, n, -1), w.reshape(B, n, -1), margin.reshape(B, n), x.copy(),
+                           rlog.reshape(B, n, -1)))
     if append:
         kv.length = L0 + n
     return x

@@ -163,7 +163,7 @@ def test_moe_topk_all_equals_dense_softmax_mixture():
     E, d, f = 4, 8, 6
     layer = _toy_layer(rng, E, d, f)
     h = bf16_round(rng.standard_normal((5, d)))
-    out, idx, w, _ = M.moe_ffn(h, layer, top_k=E)
+    out, idx, w, _, _ = M.moe_ffn(h, layer, top_k=E)
     logits = f32_round(h @ layer["wr"].T)
     p = np.exp(logits - logits.max(1, keepdims=True))
     p /= p.sum(1, keepdims=True)
@@ -177,7 +177,7 @@ def test_moe_single_expert_is_plain_ffn():
     rng = np.random.default_rng(8)
     layer = _toy_layer(rng, 1, 8, 6)
     h = bf16_round(rng.standard_normal((3, 8)))
-    out, idx, w, _ = M.moe_ffn(h, layer, top_k=1)
+    out, idx, w, _, _ = M.moe_ffn(h, layer, top_k=1)
     assert np.all(idx == 0) and np.all(w == 1.0)
     assert np.array_equal(out, M.expert_ffn(h, dec(layer["wg"][0]), dec(layer["wu"][0]),
                                             dec(layer["wd"][0])))
