@@ -250,30 +250,45 @@ __global__ void __launch_bounds__(128) attn_kernel(const AttnParams p) {
   }
 }
 
-// Merge split-KV partials (fixed split order) -> bf16 output.
+// Merge split-KV partials (fixed split order) -> bf16 output.  One warp per
+// (canvas, head, query) row: the split maxima and sums are read once per row,
+// the row's HD values are merged with 16-byte vector loads.
 __global__ void attn_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml,
-                                    uint16_t* __restrict__ out, int splits, int B, int Hq, int nq,
-                                    int HD) {
+                                    uint16_t* __restrict__ out, int splits, int B, int Hq, int nq, int HD) {
   const long long rows = (long long)B * Hq * nq;
-  const long long n = rows * HD;
-  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n;
-       e += (long long)gridDim.x * blockDim.x) {
-    const long long row = e / HD;
-    const int dd = (int)(e - row * HD);
-    float mx = -INFINITY;
-    for (int s = 0; s < splits; ++s) mx = fmaxf(mx, part_ml[(s * rows + row) * 2]);
-    float den = 0.f, num = 0.f;
-    for (int s = 0; s < splits; ++s) {
+  const long long row = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  float mx = -INFINITY;
+  for (int s = 0; s < splits; ++s) mx = fmaxf(mx, part_ml[(s * rows + row) * 2]);
+  float wgt[8];
+  float den = 0.f;
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    wgt[s] = 0.f;
+    if (s < splits) {
       const float ms = part_ml[(s * rows + row) * 2];
-      if (ms == -INFINITY) continue;
-      const float wgt = exp2f(ms - mx);
-      den += wgt * part_ml[(s * rows + row) * 2 + 1];
-      num += wgt * part_o[(s * rows + row) * HD + dd];
+      if (ms != -INFINITY) wgt[s] = exp2f(ms - mx);
+      den += wgt[s] * part_ml[(s * rows + row) * 2 + 1];
     }
-    const int i = (int)(row % nq);
-    const long long bh = row / nq;
-    const int h = (int)(bh % Hq), b = (int)(bh / Hq);
-    out[((long long)(b * nq + i) * Hq + h) * HD + dd] = f32_to_bf16(den > 0.f ? num / den : 0.f);
+  }
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+  const int i = (int)(row % nq);
+  const long long bh = row / nq;
+  const int h = (int)(bh % Hq), b = (int)(bh / Hq);
+  uint16_t* dst = out + ((long long)(b * nq + i) * Hq + h) * HD;
+  for (int c = lane * 4; c < HD; c += 128) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int s = 0; s < 8; ++s)
+      if (s < splits) {
+        const float4 v = *reinterpret_cast<const float4*>(part_o + (s * rows + row) * HD + c);
+        acc.x += wgt[s] * v.x; acc.y += wgt[s] * v.y; acc.z += wgt[s] * v.z; acc.w += wgt[s] * v.w;
+      }
+    uint2 o;
+    o.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+    o.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+    *reinterpret_cast<uint2*>(dst + c) = o;
   }
 }
 

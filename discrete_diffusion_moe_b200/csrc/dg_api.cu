@@ -59,7 +59,7 @@ static int next_pow2(int x) {
 
 static bool cfg_ok(const dg_model_config* c, char* why, size_t n) {
   if (!c) { snprintf(why, n, "null config"); return false; }
-  if (c->n_layers < 1 || c->d_model < 128 || c->d_model % 64) { snprintf(why, n, "d_model must be a multiple of 64, >= 128"); return false; }
+  if (c->n_layers < 1 || c->d_model < 256 || c->d_model % 64 || c->d_model > 4096) { snprintf(why, n, "d_model must be a multiple of 64 in [256, 4096]"); return false; }
   if (c->head_dim < 16 || c->head_dim % 16 || c->head_dim > 256) { snprintf(why, n, "head_dim must be a multiple of 16 in [16, 256]"); return false; }
   if (c->head_dim != 32 && c->head_dim != 64 && c->head_dim != 128 && c->head_dim != 176) {
     snprintf(why, n, "head_dim %d not built (32, 64, 128, 176)", c->head_dim); return false;
@@ -123,7 +123,8 @@ struct WsLayout {
   long long epart_rows;
 };
 
-int router_splits(const dg_model_config& c) { return std::min(c.d_model / 64, 16); }
+constexpr int kRouterSplits = 4;  // split-k of the router product (needs d_model >= 256)
+int router_splits(const dg_model_config&) { return kRouterSplits; }
 
 int esum_splits(const dg_model_config& c, int T, int num_sms) {
   const int m_tiles = (c.d_model + 127) / 128;
@@ -284,6 +285,15 @@ GemmPlan grouped_plan(int K, int rows_per_group, const int* off, const int* chun
 }
 
 int token_bn(int T) { return std::min(256, std::max(16, next_pow2(T))); }
+
+// Token columns per unit of a weight-stationary dense GEMM: the largest tile
+// (up to 256) that still gives about one unit per SM, so small batches spread
+// the weight stream over the whole GPU (tiles re-read their weights from L2).
+int dense_bn(int m_tiles, int T, int num_sms) {
+  int bn = token_bn(T);
+  while (bn > 16 && (long long)m_tiles * ((T + bn - 1) / bn) < (3 * num_sms) / 4) bn >>= 1;
+  return bn;
+}
 int box_for(int bn) { return std::min(64, bn); }
 
 }  // namespace
@@ -459,9 +469,10 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
   float* x = c->at<float>(L.x);
   uint16_t* xn = c->at<uint16_t>(L.xn);
   const int bnT = token_bn(T), boxT = box_for(bnT);
-  // token rows per grouped unit: about twice the mean tokens per expert
-  const int avg = std::max(1, P / E);
-  const int bnG = std::min(256, std::max(32, next_pow2(2 * avg)));
+  // token rows per grouped unit: 128 (256 for large batches).  Routing can be
+  // very uneven; one unit per 128 tokens of an expert keeps the number of times
+  // a weight tile is read small while the units of one tile run side by side.
+  const int bnG = P / E > 64 ? 256 : 128;
   const size_t kv_layer = (size_t)kv->batch * Hkv * kv->c_max * hd;
 
   CUtensorMap t_xn, t_attn, t_xperm, t_hperm;
@@ -491,17 +502,21 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
     uint16_t* kc = (uint16_t*)kv->k + (size_t)l * kv_layer;
     uint16_t* vc = (uint16_t*)kv->v + (size_t)l * kv_layer;
 
-    // --- attention block ---
-    rmsnorm_kernel<256><<<T, 256, 0, st>>>(x, c->wp(W.g_attn), xn, d, m.rms_eps);
-    CNT(c);
+    // --- attention block (its RMSNorm ran at the end of the previous layer) ---
+    if (l == 0) {
+      rmsnorm_kernel<256><<<T, 256, 0, st>>>(x, c->wp(W.g_attn), xn, d, m.rms_eps);
+      CNT(c);
+    }
     {
       ProfScope ps_(c, DG_PROF_DENSE, st);
-      CUtensorMap ta;
+      CUtensorMap ta, tb;
+      const int bn = dense_bn((qkv_rows + 127) / 128, T, c->num_sms);
       DG_TRY(make_tmap(&ta, c->wp(W.wqkv), d, qkv_rows, 128));
-      GemmPlan p = dense_plan(d, qkv_rows, T, bnT, boxT, 1, err);
+      DG_TRY(make_tmap(&tb, xn, d, L.T_alloc, box_for(bn)));
+      GemmPlan p = dense_plan(d, qkv_rows, T, bn, box_for(bn), 1, err);
       p.a_hint = 1;
       EpiStoreT e{c->at<float>(L.qkv), qkv_rows, 0, 0, nullptr, nullptr, 0, err};
-      DG_TRY(run_gemm(ta, t_xn, p, e, c->num_sms, st, &c->n_launch));
+      DG_TRY(run_gemm(ta, tb, p, e, c->num_sms, st, &c->n_launch));
     }
     {
       RopeParams rp{c->at<float>(L.qkv), c->at<double2>(L.rope), c->at<uint16_t>(L.q), kc, vc, T, nq, L0,
@@ -525,20 +540,22 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
       CNT(c);
       DG_CUDA(cudaGetLastError());
       if (splits > 1) {
-        const long long n = (long long)B * Hq * nq * hd;
-        attn_combine_kernel<<<(unsigned)std::min<long long>((n + 255) / 256, 8192), 256, 0, st>>>(
+        const long long rows = (long long)B * Hq * nq;
+        attn_combine_kernel<<<(unsigned)((rows * 32 + 255) / 256), 256, 0, st>>>(
             c->at<float>(L.attn_po), c->at<float>(L.attn_pml), c->at<uint16_t>(L.attn), splits, B, Hq, nq, hd);
             CNT(c);
       }
     }
     {
       ProfScope ps_(c, DG_PROF_DENSE, st);
-      CUtensorMap ta;
+      CUtensorMap ta, tb;
+      const int bn = dense_bn((d + 127) / 128, T, c->num_sms);
       DG_TRY(make_tmap(&ta, c->wp(W.wo), (long long)Hq * hd, d, 128));
-      GemmPlan p = dense_plan(Hq * hd, d, T, bnT, boxT, 1, err);
+      DG_TRY(make_tmap(&tb, c->at<uint16_t>(L.attn), (long long)Hq * hd, L.T_alloc, box_for(bn)));
+      GemmPlan p = dense_plan(Hq * hd, d, T, bn, box_for(bn), 1, err);
       p.a_hint = 1;
       EpiStoreT e{x, d, 0, 1, nullptr, nullptr, 0, err};
-      DG_TRY(run_gemm(ta, t_attn, p, e, c->num_sms, st, &c->n_launch));
+      DG_TRY(run_gemm(ta, tb, p, e, c->num_sms, st, &c->n_launch));
     }
 
     // --- mixture of experts block ---
@@ -546,14 +563,17 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
     CNT(c);
     {
       ProfScope ps_(c, DG_PROF_DENSE, st);
-      CUtensorMap ta;
+      CUtensorMap ta, tb;
+      const int bn = std::max(32, dense_bn((E + 127) / 128, T, c->num_sms / L.ks_r));
       DG_TRY(make_tmap(&ta, c->wp(W.wr), d, c->wl.wr_rows, 128));
-      GemmPlan p = dense_plan(d, E, T, bnT, boxT, L.ks_r, err);
+      DG_TRY(make_tmap(&tb, xn, d, L.T_alloc, box_for(bn)));
+      GemmPlan p = dense_plan(d, E, T, bn, box_for(bn), L.ks_r, err);
       EpiStoreT e{c->at<float>(L.rpart), E, (long long)T * E, 0, nullptr, nullptr, 0, err};
-      DG_TRY(run_gemm(ta, t_xn, p, e, c->num_sms, st, &c->n_launch));
+      DG_TRY(run_gemm(ta, tb, p, e, c->num_sms, st, &c->n_launch));
     }
-    router_topk_kernel<<<(T * 32 + 255) / 256, 256, 0, st>>>(
-        c->at<float>(L.rpart), L.ks_r, T, E, k, c->at<int>(L.idx), c->at<float>(L.w),
+    if (L.ks_r != kRouterSplits) return fail(DG_ERR_UNSUPPORTED, "router split count %d", L.ks_r);
+    router_topk_kernel<kRouterSplits><<<(T * 32 + 255) / 256, 256, 0, st>>>(
+        c->at<float>(L.rpart), T, E, k, c->at<int>(L.idx), c->at<float>(L.w),
         dbg_idx ? dbg_idx + (size_t)l * T * k : nullptr, dbg_w ? dbg_w + (size_t)l * T * k : nullptr,
         dbg_logits ? dbg_logits + (size_t)l * T * E : nullptr);
         CNT(c);
@@ -583,8 +603,14 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
       EpiDown e{c->at<float>(L.yperm), d, c->at<float>(L.wperm)};
       DG_TRY(run_gemm(ta, t_hperm, p, e, c->num_sms, st, &c->n_launch));
     }
-    moe_combine_kernel<<<T, 256, 0, st>>>(x, c->at<float>(L.yperm), c->at<int>(L.inv), T, k, d);
-    CNT(c);
+    // combine + residual, fused with the next RMSNorm (next layer's attention
+    // norm, or the final norm before the LM head)
+    {
+      const uint16_t* g_next = l + 1 < m.n_layers ? c->wp(c->wl.layers[l + 1].g_attn) : c->wp(c->wl.g_final);
+      moe_combine_norm_kernel<<<T, 256, 0, st>>>(x, c->at<float>(L.yperm), c->at<int>(L.inv), T, k, d, g_next,
+                                                 xn, m.rms_eps);
+      CNT(c);
+    }
     DG_CUDA(cudaGetLastError());
     if (dbg_hidden)
       DG_CUDA(cudaMemcpyAsync(dbg_hidden + (size_t)(l + 1) * T * d, x, (size_t)T * d * 4,
@@ -687,9 +713,10 @@ extern "C" dg_status dg_denoise_step(dg_ctx* c, const dg_kv* kv, dg_canvas* cv, 
   if (m.self_cond) {
     ProfScope ps_(c, DG_PROF_DENSE, st);
     CUtensorMap ta, tb;
+    const int bn = dense_bn((d + 127) / 128, T, c->num_sms);
     DG_TRY(make_tmap(&ta, c->wp(c->wl.sc), d, d, 128));
-    DG_TRY(make_tmap(&tb, cv->sc_state, d, T, boxT));
-    GemmPlan p = dense_plan(d, d, T, bnT, boxT, 1, err);
+    DG_TRY(make_tmap(&tb, cv->sc_state, d, T, box_for(bn)));
+    GemmPlan p = dense_plan(d, d, T, bn, box_for(bn), 1, err);
     p.a_hint = 1;
     EpiStoreT e{c->at<float>(L.x), d, 0, 2, c->wp(c->wl.emb), cv->tokens, V, err};
     DG_TRY(run_gemm(ta, tb, p, e, c->num_sms, st, &c->n_launch));
@@ -707,9 +734,7 @@ extern "C" dg_status dg_denoise_step(dg_ctx* c, const dg_kv* kv, dg_canvas* cv, 
                         o->hidden, st));
 
   // a7: final norm, LM head with online vocabulary statistics and sampling
-  uint16_t* xn = c->at<uint16_t>(L.xn);
-  rmsnorm_kernel<256><<<T, 256, 0, st>>>(c->at<float>(L.x), c->wp(c->wl.g_final), xn, d, m.rms_eps);
-  CNT(c);
+  uint16_t* xn = c->at<uint16_t>(L.xn);  // final RMSNorm: fused into the last layer's combine
   float* logits = o->logits ? o->logits : c->at<float>(L.logits);
   const double Ts = s.max_steps <= 1 ? (double)s.t_start
                                      : (double)s.t_start + ((double)s.t_end - (double)s.t_start) * a->step /
@@ -961,9 +986,9 @@ extern "C" dg_status dg_test_attention(const uint16_t* q, const uint16_t* k, con
   }
   DG_CUDA(cudaGetLastError());
   if (splits > 1) {
-    const long long n = (long long)B * Hq * nq * hd;
-    attn_combine_kernel<<<(unsigned)std::min<long long>((n + 255) / 256, 8192), 256, 0, st>>>(
-        part_o, part_ml, out, splits, B, Hq, nq, hd);
+    const long long rows = (long long)B * Hq * nq;
+    attn_combine_kernel<<<(unsigned)((rows * 32 + 255) / 256), 256, 0, st>>>(part_o, part_ml, out, splits, B,
+                                                                             Hq, nq, hd);
     DG_CUDA(cudaGetLastError());
   }
   DG_CUDA(cudaStreamSynchronize(st));

@@ -140,7 +140,8 @@ __global__ void rope_kv_kernel(const RopeParams p) {
 // Router: sum the split-k partial logits (fixed order), pick the top-k
 // experts by logit (ties to the lower id), softmax over the chosen k.
 // One warp per token; E <= 256.
-__global__ void router_topk_kernel(const float* __restrict__ part, int ks, int T, int E, int k,
+template <int KS>
+__global__ void router_topk_kernel(const float* __restrict__ part, int T, int E, int k,
                                    int* __restrict__ idx, float* __restrict__ w,
                                    int* __restrict__ dbg_idx, float* __restrict__ dbg_w,
                                    float* __restrict__ dbg_logits) {
@@ -154,7 +155,8 @@ __global__ void router_topk_kernel(const float* __restrict__ part, int ks, int T
   for (int q = 0; q < 8; ++q) { l[q] = 0.f; taken[q] = false; }
   // split-k partials summed in split order; the 8 expert slots of a lane are
   // independent, so their loads are issued together
-  for (int p = 0; p < ks; ++p) {
+#pragma unroll
+  for (int p = 0; p < KS; ++p) {
     const float* row = part + ((long long)p * T + t) * E;
     float v[8];
 #pragma unroll
@@ -228,17 +230,32 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(const int* __rest
     atomicAdd(&cnt[e], 1);
   }
   __syncthreads();
-  if (tid == 0) {
-    int acc = 0, acc_c = 0;
-    for (int e = 0; e < E; ++e) {
-      off[e] = acc;
-      base[e] = acc;
-      chunk_off[e] = acc_c;
-      acc += cnt[e];
-      acc_c += (cnt[e] + bn - 1) / bn;
+  if (warp == 0) {
+    // exclusive scans of the counts and chunk counts, 8 experts per lane (E <= 256)
+    int c8[8], k8[8], sc = 0, sk = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = lane * 8 + j;
+      c8[j] = e < E ? cnt[e] : 0;
+      k8[j] = (c8[j] + bn - 1) / bn;
+      sc += c8[j];
+      sk += k8[j];
     }
-    off[E] = acc;
-    chunk_off[E] = acc_c;
+    int ic = sc, ik = sk;  // inclusive lane sums
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int a = __shfl_up_sync(0xffffffffu, ic, o), b2 = __shfl_up_sync(0xffffffffu, ik, o);
+      if (lane >= o) { ic += a; ik += b2; }
+    }
+    int pc = ic - sc, pk = ik - sk;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = lane * 8 + j;
+      if (e < E) { off[e] = pc; base[e] = pc; chunk_off[e] = pk; }
+      pc += c8[j];
+      pk += k8[j];
+    }
+    if (lane == 31) { off[E] = ic; chunk_off[E] = ik; }
   }
   __syncthreads();
   for (int c0 = 0; c0 < P; c0 += kPermThreads) {
@@ -295,23 +312,62 @@ __global__ void gather_rows_kernel(const uint16_t* __restrict__ xn, const int* _
   for (int c = threadIdx.x; c < d / 8; c += blockDim.x) dst[c] = src[c];
 }
 
-// x[t, :] += sum_{j < k} y[inv[t*k + j], :]   (fixed j order, fp32)
-__global__ void moe_combine_kernel(float* __restrict__ x, const float* __restrict__ y,
-                                   const int* __restrict__ inv, int T, int k, int d) {
+// x[t, :] += sum_{j < k} y[inv[t*k + j], :]   (fixed j order, fp32), then
+// the RMSNorm that starts the next block: xn[t, :] = bf16(x / rms(x) * gain).
+// One CTA of 256 threads per token; the row stays in registers between the
+// two passes (d <= 256 * 4 * kCombineVec).
+constexpr int kCombineVec = 4;
+__global__ void __launch_bounds__(256) moe_combine_norm_kernel(float* __restrict__ x, const float* __restrict__ y,
+                                                               const int* __restrict__ inv, int T, int k, int d,
+                                                               const uint16_t* __restrict__ gain,
+                                                               uint16_t* __restrict__ xn, float eps) {
   const int t = blockIdx.x;
   if (t >= T) return;
   int slots[8];
-  for (int j = 0; j < k; ++j) slots[j] = inv[t * k + j];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) slots[j] = j < k ? inv[t * k + j] : 0;
   float* xr = x + (long long)t * d;
-  for (int c = threadIdx.x * 4; c < d; c += blockDim.x * 4) {
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j = 0; j < k; ++j) {
-      const float4 v = *reinterpret_cast<const float4*>(y + (long long)slots[j] * d + c);
-      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+  float4 r[kCombineVec];
+  float ss = 0.f;
+#pragma unroll
+  for (int q = 0; q < kCombineVec; ++q) {
+    const int c = (q * 256 + threadIdx.x) * 4;
+    if (c < d) {
+      float4 acc = *reinterpret_cast<const float4*>(xr + c);
+      float4 v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (j < k) v[j] = *reinterpret_cast<const float4*>(y + (long long)slots[j] * d + c);
+      float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (j < k) { sum.x += v[j].x; sum.y += v[j].y; sum.z += v[j].z; sum.w += v[j].w; }
+      acc.x += sum.x; acc.y += sum.y; acc.z += sum.z; acc.w += sum.w;
+      *reinterpret_cast<float4*>(xr + c) = acc;
+      r[q] = acc;
+      ss += acc.x * acc.x + acc.y * acc.y + acc.z * acc.z + acc.w * acc.w;
     }
-    float4 r = *reinterpret_cast<float4*>(xr + c);
-    r.x += acc.x; r.y += acc.y; r.z += acc.z; r.w += acc.w;
-    *reinterpret_cast<float4*>(xr + c) = r;
+  }
+  if (!xn) return;
+  __shared__ float red[8];
+  ss = warp_sum(ss);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  float tot = 0.f;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) tot += red[w];
+  const float rs = rsqrtf(tot / (float)d + eps);
+  uint16_t* yr = xn + (long long)t * d;
+#pragma unroll
+  for (int q = 0; q < kCombineVec; ++q) {
+    const int c = (q * 256 + threadIdx.x) * 4;
+    if (c < d) {
+      const uint2 gg = *reinterpret_cast<const uint2*>(gain + c);
+      uint2 o;
+      o.x = pack_bf16x2(r[q].x * rs * bf16_to_f32(gg.x & 0xFFFF), r[q].y * rs * bf16_to_f32(gg.x >> 16));
+      o.y = pack_bf16x2(r[q].z * rs * bf16_to_f32(gg.y & 0xFFFF), r[q].w * rs * bf16_to_f32(gg.y >> 16));
+      *reinterpret_cast<uint2*>(yr + c) = o;
+    }
   }
 }
 

@@ -54,9 +54,9 @@ typedef enum dg_status {
 
 /* Model dimensions.  The pages fix 128 experts with 8 active per token
    (laozijiushiniubi.cn article §二); the other dimensions are the caller's.
-   Limits of this build: d_model % 64 == 0, head_dim % 16 == 0 and
-   head_dim <= 256, n_q_heads % n_kv_heads == 0, d_ff % 64 == 0,
-   vocab % 256 == 0, top_k <= 8, n_experts <= 256. */
+   Limits of this build: d_model % 64 == 0 and 256 <= d_model <= 4096,
+   head_dim in {32, 64, 128, 176}, n_q_heads % n_kv_heads == 0,
+   d_ff % 64 == 0, vocab % 256 == 0, top_k <= 8, n_experts <= 256. */
 typedef struct dg_model_config {
   int32_t n_layers;
   int32_t d_model;
