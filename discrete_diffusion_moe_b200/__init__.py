@@ -97,6 +97,8 @@ def _load():
         "dg_canvas_init": (I32, [P, ctypes.POINTER(dg_canvas), I32, U64, P]),
         "dg_denoise_step": (I32, [P, ctypes.POINTER(dg_kv), ctypes.POINTER(dg_canvas),
                                   ctypes.POINTER(dg_step_args), ctypes.POINTER(dg_step_out), P]),
+        "dg_denoise_step_graph": (I32, [P, ctypes.POINTER(dg_kv), ctypes.POINTER(dg_canvas),
+                                        ctypes.POINTER(dg_step_args), ctypes.POINTER(dg_step_out), P]),
         "dg_decode_block": (I32, [P, ctypes.POINTER(dg_kv), ctypes.POINTER(dg_canvas),
                                   ctypes.POINTER(dg_step_args), P, ctypes.POINTER(dg_block_stats), P]),
         "dg_check_device_error": (I32, [P, P]),
@@ -165,6 +167,11 @@ def dg_canvas_init(ctx, cv: dg_canvas, block, seed, stream):
 def dg_denoise_step(ctx, kv: dg_kv, cv: dg_canvas, args: dg_step_args, out, stream):
     return lib.dg_denoise_step(ctx, ctypes.byref(kv), ctypes.byref(cv), ctypes.byref(args),
                                ctypes.byref(out) if out is not None else None, stream)
+
+
+def dg_denoise_step_graph(ctx, kv: dg_kv, cv: dg_canvas, args: dg_step_args, out, stream):
+    return lib.dg_denoise_step_graph(ctx, ctypes.byref(kv), ctypes.byref(cv), ctypes.byref(args),
+                                     ctypes.byref(out) if out is not None else None, stream)
 
 
 def dg_decode_block(ctx, kv: dg_kv, cv: dg_canvas, args: dg_step_args, d_out, stats, stream):

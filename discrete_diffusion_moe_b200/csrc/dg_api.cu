@@ -116,15 +116,22 @@ WLayout weight_layout(const dg_model_config& c) {
 constexpr int kMaxAttnSplits = 8;
 
 struct WsLayout {
-  size_t err, flags, x, xn, qkv, q, attn, attn_po, attn_pml, rpart, idx, w, off, choff, perm, inv, wperm,
+  size_t err, flags, x, xn, qkv, opart, q, attn, attn_po, attn_pml, rpart, idx, w, off, choff, perm, inv, wperm,
       xperm, hperm, yperm, logits, vp_m, vp_z, vp_s, vp_av, vp_ai, vp_gv, vp_gi, st_m, st_iz, st_h,
-      st_pmax, st_amax, st_samp, probs, epart, rope, total;
+      st_pmax, st_amax, st_samp, probs, epart, rope, stepdev, total;
   int T_alloc, P_alloc, ks_r, n_vt, attn_rows_cap;
   long long epart_rows;
 };
 
 constexpr int kRouterSplits = 4;  // split-k of the router product (needs d_model >= 256)
 int router_splits(const dg_model_config&) { return kRouterSplits; }
+
+// Split-k factor of a weight-stationary dense GEMM with m_tiles x n_tiles
+// output tiles: as many k splits as keep the units within one wave.
+int dense_splits(int m_tiles, int n_tiles, int kb, int num_sms) {
+  int ks = num_sms / std::max(1, m_tiles * n_tiles);
+  return std::max(1, std::min({ks, 8, kb / 4}));
+}
 
 int esum_splits(const dg_model_config& c, int T, int num_sms) {
   const int m_tiles = (c.d_model + 127) / 128;
@@ -155,7 +162,17 @@ WsLayout ws_layout(const dg_model_config& c, int batch, int num_sms) {
   L.flags = take(std::max<size_t>(batch, 64));
   L.x = take(T * d * 4);
   L.xn = take(T * d * 2);
-  L.qkv = take(T * (size_t)((c.n_q_heads + 2 * c.n_kv_heads) * c.head_dim) * 4);
+  {
+    const int qkv_rows = (c.n_q_heads + 2 * c.n_kv_heads) * c.head_dim;
+    size_t rq = 0, ro = 0;
+    for (int tt = DG_CANVAS; tt <= (int)T; tt += DG_CANVAS) {
+      const int nt = (tt + 255) / 256;
+      rq = std::max(rq, (size_t)dense_splits((qkv_rows + 127) / 128, nt, c.d_model / 64, num_sms) * tt);
+      ro = std::max(ro, (size_t)dense_splits((c.d_model + 127) / 128, nt, (int)hq / 64, num_sms) * tt);
+    }
+    L.qkv = take(rq * qkv_rows * 4);
+    L.opart = take(ro * d * 4);
+  }
   L.q = take(T * hq * 2);
   L.attn = take(T * hq * 2);
   L.attn_po = take((size_t)L.attn_rows_cap * DG_CANVAS * hq * 4);
@@ -178,6 +195,7 @@ WsLayout ws_layout(const dg_model_config& c, int batch, int num_sms) {
   L.st_m = take(T * 4); L.st_iz = take(T * 4); L.st_h = take(T * 4); L.st_pmax = take(T * 4);
   L.st_amax = take(T * 4); L.st_samp = take(T * 4);
   L.rope = take((size_t)DG_CANVAS * (c.head_dim / 2) * 16);
+  L.stepdev = take(sizeof(StepDev));
   L.probs = c.self_cond ? take(T * V * 2) : 0;
   L.epart = c.self_cond ? take((size_t)er * d * 4) : 0;
   L.total = off;
@@ -322,7 +340,30 @@ struct dg_ctx {
   void prof_end(int i, cudaStream_t st) {
     if (i >= 0) cudaEventRecord(ev_pool[i + 1], st);
   }
+  // cached CUDA graph of one round (dg_denoise_step_graph)
+  struct GraphKey {
+    dg_kv kv;
+    dg_canvas cv;
+    dg_step_out out;
+  };
+  bool g_valid = false;
+  GraphKey g_key;
+  cudaGraph_t g_graph = nullptr;
+  cudaGraphExec_t g_exec = nullptr;
+  cudaGraphNode_t g_param_node = nullptr;
+  cudaStream_t g_stream = nullptr;
+  long long g_kernels = 0;  // kernels launched by one replay
+  void drop_graph() {
+    if (g_exec) cudaGraphExecDestroy(g_exec);
+    if (g_graph) cudaGraphDestroy(g_graph);
+    g_exec = nullptr;
+    g_graph = nullptr;
+    g_param_node = nullptr;
+    g_valid = false;
+  }
   ~dg_ctx() {
+    drop_graph();
+    if (g_stream) cudaStreamDestroy(g_stream);
     for (cudaEvent_t e : ev_pool) cudaEventDestroy(e);
   }
   dg_model_config cfg;
@@ -489,6 +530,10 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
     CNT(c);
   }
 
+  // split-k of the two dense projections (partials summed by their consumers)
+  const int ks_qkv = dense_splits((qkv_rows + 127) / 128, (T + 255) / 256, d / 64, c->num_sms);
+  const int ks_o = dense_splits((d + 127) / 128, (T + 255) / 256, Hq * hd / 64, c->num_sms);
+
   // attention launch shape
   const int q_tiles = ((Hq / Hkv) * nq + 63) / 64;
   const int base_ctas = q_tiles * Hkv * B;
@@ -510,17 +555,17 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
     {
       ProfScope ps_(c, DG_PROF_DENSE, st);
       CUtensorMap ta, tb;
-      const int bn = dense_bn((qkv_rows + 127) / 128, T, c->num_sms);
+      const int bn = token_bn(T);
       DG_TRY(make_tmap(&ta, c->wp(W.wqkv), d, qkv_rows, 128));
       DG_TRY(make_tmap(&tb, xn, d, L.T_alloc, box_for(bn)));
-      GemmPlan p = dense_plan(d, qkv_rows, T, bn, box_for(bn), 1, err);
+      GemmPlan p = dense_plan(d, qkv_rows, T, bn, box_for(bn), ks_qkv, err);
       p.a_hint = 1;
-      EpiStoreT e{c->at<float>(L.qkv), qkv_rows, 0, 0, nullptr, nullptr, 0, err};
+      EpiStoreT e{c->at<float>(L.qkv), qkv_rows, (long long)T * qkv_rows, 0, nullptr, nullptr, 0, err};
       DG_TRY(run_gemm(ta, tb, p, e, c->num_sms, st, &c->n_launch));
     }
     {
-      RopeParams rp{c->at<float>(L.qkv), c->at<double2>(L.rope), c->at<uint16_t>(L.q), kc, vc, T, nq, L0,
-                    kv->c_max, Hq, Hkv, hd};
+      RopeParams rp{c->at<float>(L.qkv), ks_qkv, (long long)T * qkv_rows, c->at<double2>(L.rope),
+                    c->at<uint16_t>(L.q), kc, vc, T, nq, L0, kv->c_max, Hq, Hkv, hd};
       rope_kv_kernel<<<std::min(4096, (T * (Hq + 2 * Hkv) * hd / 2 + 255) / 256), 256, 0, st>>>(rp);
       CNT(c);
     }
@@ -549,17 +594,18 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
     {
       ProfScope ps_(c, DG_PROF_DENSE, st);
       CUtensorMap ta, tb;
-      const int bn = dense_bn((d + 127) / 128, T, c->num_sms);
+      const int bn = token_bn(T);
       DG_TRY(make_tmap(&ta, c->wp(W.wo), (long long)Hq * hd, d, 128));
       DG_TRY(make_tmap(&tb, c->at<uint16_t>(L.attn), (long long)Hq * hd, L.T_alloc, box_for(bn)));
-      GemmPlan p = dense_plan(Hq * hd, d, T, bn, box_for(bn), 1, err);
+      GemmPlan p = dense_plan(Hq * hd, d, T, bn, box_for(bn), ks_o, err);
       p.a_hint = 1;
-      EpiStoreT e{x, d, 0, 1, nullptr, nullptr, 0, err};
+      EpiStoreT e{c->at<float>(L.opart), d, (long long)T * d, 0, nullptr, nullptr, 0, err};
       DG_TRY(run_gemm(ta, tb, p, e, c->num_sms, st, &c->n_launch));
     }
 
-    // --- mixture of experts block ---
-    rmsnorm_kernel<256><<<T, 256, 0, st>>>(x, c->wp(W.g_moe), xn, d, m.rms_eps);
+    // --- mixture of experts block: residual add of the output projection + RMSNorm ---
+    residual_norm_kernel<<<T, 256, 0, st>>>(x, c->at<float>(L.opart), ks_o, (long long)T * d, d,
+                                            c->wp(W.g_moe), xn, m.rms_eps);
     CNT(c);
     {
       ProfScope ps_(c, DG_PROF_DENSE, st);
@@ -684,8 +730,26 @@ extern "C" dg_status dg_canvas_init(dg_ctx* c, dg_canvas* cv, int32_t block, uin
   return DG_OK;
 }
 
-extern "C" dg_status dg_denoise_step(dg_ctx* c, const dg_kv* kv, dg_canvas* cv, const dg_step_args* a,
-                                     const dg_step_out* o, void* stream) {
+static StepDev step_dev(const dg_step_args* a) {
+  const dg_sampler_config& s = a->sampler;
+  const double Ts = s.max_steps <= 1 ? (double)s.t_start
+                                     : (double)s.t_start + ((double)s.t_end - (double)s.t_start) * a->step /
+                                                               (double)(s.max_steps - 1);
+  StepDev v;
+  v.step = a->step;
+  v.max_steps = s.max_steps;
+  v.block = a->block;
+  v.policy = s.lock_policy;
+  v.lock_threshold = s.lock_threshold;
+  v.stop_entropy = s.stop_entropy;
+  v.inv_t = (float)(1.0 / Ts);
+  v.require_stable = s.stop_require_stable_argmax;
+  v.k0 = (uint32_t)s.seed;
+  v.k1 = (uint32_t)(s.seed >> 32);
+  return v;
+}
+
+static dg_status check_round_args(dg_ctx* c, const dg_kv* kv, dg_canvas* cv, const dg_step_args* a) {
   if (!c || !cv || !a) return fail(DG_ERR_INVALID_ARG, "null argument");
   DG_TRY(check_kv(c, kv, DG_CANVAS));
   if (cv->batch != kv->batch) return fail(DG_ERR_INVALID_ARG, "canvas batch %d != kv batch %d", cv->batch, kv->batch);
@@ -699,15 +763,33 @@ extern "C" dg_status dg_denoise_step(dg_ctx* c, const dg_kv* kv, dg_canvas* cv, 
     return fail(DG_ERR_INVALID_ARG, "lock policy");
   if (!(s.t_start > 0.f) || !(s.t_end > 0.f)) return fail(DG_ERR_INVALID_ARG, "temperatures must be > 0");
   if (!attn_smem_ready(c->cfg.head_dim)) return fail(DG_ERR_CUDA, "attention smem attribute");
+  return DG_OK;
+}
 
+// Enqueue one round.  The first launch writes the round parameters to the
+// device (its node is returned when the stream is being captured).
+static dg_status enqueue_round(dg_ctx* c, const dg_kv* kv, dg_canvas* cv, const dg_step_args* a,
+                               const dg_step_out* o, cudaStream_t st, cudaGraphNode_t* param_node) {
   const dg_model_config& m = c->cfg;
   const WsLayout& L = c->L;
-  cudaStream_t st = (cudaStream_t)stream;
+  const dg_sampler_config& s = a->sampler;
   const int B = cv->batch, T = B * DG_CANVAS, d = m.d_model, V = m.vocab;
   int* err = c->err();
   const int bnT = token_bn(T), boxT = box_for(bnT);
   dg_step_out none{};
   if (!o) o = &none;
+  StepDev* sp = c->at<StepDev>(L.stepdev);
+  step_params_kernel<<<1, 32, 0, st>>>(sp, step_dev(a));
+  CNT(c);
+  DG_CUDA(cudaGetLastError());
+  if (param_node) {
+    cudaStreamCaptureStatus cs;
+    const cudaGraphNode_t* deps = nullptr;
+    size_t nd = 0;
+    DG_CUDA(cudaStreamGetCaptureInfo(st, &cs, nullptr, nullptr, &deps, &nd));
+    if (cs != cudaStreamCaptureStatusActive || nd != 1) return fail(DG_ERR_CUDA, "capture of the round failed");
+    *param_node = deps[0];
+  }
 
   // a1: canvas embedding (+ self-conditioning input)
   if (m.self_cond) {
@@ -736,10 +818,7 @@ extern "C" dg_status dg_denoise_step(dg_ctx* c, const dg_kv* kv, dg_canvas* cv, 
   // a7: final norm, LM head with online vocabulary statistics and sampling
   uint16_t* xn = c->at<uint16_t>(L.xn);  // final RMSNorm: fused into the last layer's combine
   float* logits = o->logits ? o->logits : c->at<float>(L.logits);
-  const double Ts = s.max_steps <= 1 ? (double)s.t_start
-                                     : (double)s.t_start + ((double)s.t_end - (double)s.t_start) * a->step /
-                                                               (double)(s.max_steps - 1);
-  const float inv_t = (float)(1.0 / Ts);
+  (void)s;
   VocabPartials vp{c->at<float>(L.vp_m), c->at<float>(L.vp_z), c->at<float>(L.vp_s), c->at<float>(L.vp_av),
                    c->at<int>(L.vp_ai), c->at<float>(L.vp_gv), c->at<int>(L.vp_gi)};
   {
@@ -751,8 +830,7 @@ extern "C" dg_status dg_denoise_step(dg_ctx* c, const dg_kv* kv, dg_canvas* cv, 
     p.n_fast = 0;
     p.a_hint = 2;
     p.b_hint = 1;
-    EpiLMHead e{logits, V, vp, L.n_vt, 256, (uint32_t)s.seed, (uint32_t)(s.seed >> 32),
-                (uint32_t)(a->block * 256 + a->step), inv_t, DG_CANVAS};
+    EpiLMHead e{logits, V, vp, L.n_vt, 256, sp, DG_CANVAS};
     DG_TRY(run_gemm(ta, tb, p, e, c->num_sms, st, &c->n_launch));
   }
   PosStats ps{c->at<float>(L.st_m), c->at<float>(L.st_iz), o->entropy ? o->entropy : c->at<float>(L.st_h),
@@ -801,19 +879,85 @@ extern "C" dg_status dg_denoise_step(dg_ctx* c, const dg_kv* kv, dg_canvas* cv, 
   up.stop_out = o->stop;
   up.final_out = o->final_round;
   up.flags = c->at<uint8_t>(L.flags);
-  up.policy = s.lock_policy;
-  up.lock_threshold = s.lock_threshold;
-  up.stop_entropy = s.stop_entropy;
-  up.require_stable = s.stop_require_stable_argmax;
-  up.step = a->step;
-  up.max_steps = s.max_steps;
-  up.block = a->block;
-  up.k0 = (uint32_t)s.seed;
-  up.k1 = (uint32_t)(s.seed >> 32);
+  up.sp = sp;
   up.vocab = V;
   canvas_update_kernel<<<B, 256, 0, st>>>(up);
   CNT(c);
   DG_CUDA(cudaGetLastError());
+  return DG_OK;
+}
+
+extern "C" dg_status dg_denoise_step(dg_ctx* c, const dg_kv* kv, dg_canvas* cv, const dg_step_args* a,
+                                     const dg_step_out* o, void* stream) {
+  DG_TRY(check_round_args(c, kv, cv, a));
+  return enqueue_round(c, kv, cv, a, o, (cudaStream_t)stream, nullptr);
+}
+
+static bool same_key(const dg_ctx::GraphKey& a, const dg_ctx::GraphKey& b) {
+  const dg_kv &x = a.kv, &y = b.kv;
+  const dg_canvas &p = a.cv, &q = b.cv;
+  const dg_step_out &u = a.out, &w = b.out;
+  return x.k == y.k && x.v == y.v && x.batch == y.batch && x.c_max == y.c_max && x.length == y.length &&
+         p.tokens == q.tokens && p.sc_state == q.sc_state && p.prev_argmax == q.prev_argmax && p.done == q.done &&
+         p.batch == q.batch && u.argmax == w.argmax && u.sample == w.sample && u.entropy == w.entropy &&
+         u.pmax == w.pmax && u.lock == w.lock && u.mean_entropy == w.mean_entropy && u.stop == w.stop &&
+         u.final_round == w.final_round && u.logits == w.logits && u.route_idx == w.route_idx &&
+         u.route_w == w.route_w && u.route_logits == w.route_logits && u.hidden == w.hidden;
+}
+
+extern "C" dg_status dg_denoise_step_graph(dg_ctx* c, const dg_kv* kv, dg_canvas* cv, const dg_step_args* a,
+                                           const dg_step_out* o, void* stream) {
+  DG_TRY(check_round_args(c, kv, cv, a));
+  if (c->prof) return enqueue_round(c, kv, cv, a, o, (cudaStream_t)stream, nullptr);
+  dg_ctx::GraphKey key;
+  memset(&key, 0, sizeof(key));
+  key.kv = *kv;
+  key.cv = *cv;
+  if (o) key.out = *o;
+  if (!c->g_valid || !same_key(key, c->g_key)) {
+    c->drop_graph();
+    if (!c->g_stream) DG_CUDA(cudaStreamCreateWithFlags(&c->g_stream, cudaStreamNonBlocking));
+    // make sure one-time attribute calls happen outside the capture
+    DG_TRY(check_round_args(c, kv, cv, a));
+    DG_CUDA(cudaStreamBeginCapture(c->g_stream, cudaStreamCaptureModeThreadLocal));
+    cudaGraphNode_t node = nullptr;
+    const long long n0 = c->n_launch;
+    const dg_status r = enqueue_round(c, kv, cv, a, o, c->g_stream, &node);
+    c->g_kernels = c->n_launch - n0;
+    c->n_launch = n0;
+    cudaGraph_t g = nullptr;
+    const cudaError_t e = cudaStreamEndCapture(c->g_stream, &g);
+    if (r != DG_OK) {
+      if (g) cudaGraphDestroy(g);
+      return r;
+    }
+    if (e != cudaSuccess) return fail(DG_ERR_CUDA, "cudaStreamEndCapture: %s", cudaGetErrorString(e));
+    cudaGraphExec_t ex = nullptr;
+    const cudaError_t e2 = cudaGraphInstantiate(&ex, g, 0);
+    if (e2 != cudaSuccess) {
+      cudaGraphDestroy(g);
+      return fail(DG_ERR_CUDA, "cudaGraphInstantiate: %s", cudaGetErrorString(e2));
+    }
+    c->g_graph = g;
+    c->g_exec = ex;
+    c->g_param_node = node;
+    c->g_key = key;
+    c->g_valid = true;
+  }
+  // this round's parameters go into the captured parameter node
+  StepDev v = step_dev(a);
+  StepDev* sp = c->at<StepDev>(c->L.stepdev);
+  void* args[2] = {(void*)&sp, (void*)&v};
+  cudaKernelNodeParams kp{};
+  kp.func = (void*)step_params_kernel;
+  kp.gridDim = dim3(1);
+  kp.blockDim = dim3(32);
+  kp.sharedMemBytes = 0;
+  kp.kernelParams = args;
+  kp.extra = nullptr;
+  DG_CUDA(cudaGraphExecKernelNodeSetParams(c->g_exec, c->g_param_node, &kp));
+  DG_CUDA(cudaGraphLaunch(c->g_exec, (cudaStream_t)stream));
+  c->n_launch += c->g_kernels;
   return DG_OK;
 }
 
@@ -844,7 +988,7 @@ extern "C" dg_status dg_decode_block(dg_ctx* c, dg_kv* kv, dg_canvas* cv, const 
   for (int s = 0; s < a->sampler.max_steps; ++s) {
     dg_step_args sa = *a;
     sa.step = s;
-    DG_TRY(dg_denoise_step(c, kv, cv, &sa, nullptr, stream));
+    DG_TRY(dg_denoise_step_graph(c, kv, cv, &sa, nullptr, stream));
     ++rounds;
     for (int b = 0; b < B; ++b)
       if (!flags[b]) ++steps[b];

@@ -4,6 +4,7 @@
 #pragma once
 
 #include "gemm_tc.cuh"
+#include "kernels.cuh"
 
 namespace dg {
 
@@ -133,17 +134,20 @@ struct EpiLMHead {
   VocabPartials part;    // each [T, n_vt]
   int n_vt;              // vocabulary tiles (V / bn)
   int bn;
-  uint32_t k0, k1;       // Philox key (seed)
-  uint32_t c2;           // block * 256 + step
-  float inv_t;           // 1 / T_step, fp32
+  const StepDev* sp;     // round parameters: Philox key, block, step, 1 / T_step
   int canvas;            // positions per canvas (256)
   struct State {
     float m, z, s, av, gv;
     int ai, gi;
+    uint32_t k0, k1, c2;
+    float inv_t;
   };
   __device__ __forceinline__ void begin(const GemmJob&, int, State& st) const {
     st.m = -INFINITY; st.z = 0.f; st.s = 0.f;
     st.av = -INFINITY; st.ai = 0; st.gv = -INFINITY; st.gi = 0;
+    st.k0 = sp->k0; st.k1 = sp->k1;
+    st.c2 = (uint32_t)(sp->block * 256 + sp->step);
+    st.inv_t = sp->inv_t;
   }
   __device__ __forceinline__ void chunk(const GemmJob& j, int row, int c0, const float (&v)[16],
                                         State& st) const {
@@ -174,7 +178,7 @@ struct EpiLMHead {
     const uint32_t c3 = (kPurposeGumbel << 24) | (uint32_t)b;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const Philox4 r = philox4x32_10((uint32_t)(vb >> 2) + q, (uint32_t)pos, c2, c3, k0, k1);
+      const Philox4 r = philox4x32_10((uint32_t)(vb >> 2) + q, (uint32_t)pos, st.c2, c3, st.k0, st.k1);
       const uint32_t w[4] = {r.x, r.y, r.z, r.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -182,7 +186,7 @@ struct EpiLMHead {
         // -ln(u) needs relative accuracy for u near 1 (the largest Gumbel keys,
         // which decide the sample): the accurate logf there, the fast one outside
         const float g = -__logf(-logf(u));
-        const float key = __fadd_rn(__fmul_rn(v[4 * q + e], inv_t), g);
+        const float key = __fadd_rn(__fmul_rn(v[4 * q + e], st.inv_t), g);
         if (key > st.gv) { st.gv = key; st.gi = vb + 4 * q + e; }
       }
     }

@@ -69,6 +69,57 @@ __global__ void __launch_bounds__(THREADS) rmsnorm_kernel(const float* __restric
 }
 
 // ---------------------------------------------------------------------------
+// x[t, :] += sum_s part[s, t, :] (split-k partials of the output projection, in
+// split order), then xn = bf16(x / rms(x) * gain).  One CTA of 256 threads per
+// token; the row stays in registers between the two passes.
+__global__ void __launch_bounds__(256) residual_norm_kernel(float* __restrict__ x, const float* __restrict__ part,
+                                                            int ks, long long split_stride, int d,
+                                                            const uint16_t* __restrict__ gain,
+                                                            uint16_t* __restrict__ xn, float eps) {
+  const int t = blockIdx.x;
+  float* xr = x + (long long)t * d;
+  float4 r[4];
+  float ss = 0.f;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int c = (q * 256 + threadIdx.x) * 4;
+    if (c < d) {
+      const float* pp = part + (long long)t * d + c;
+      float4 sum = *reinterpret_cast<const float4*>(pp);
+      for (int sp = 1; sp < ks; ++sp) {
+        const float4 v = *reinterpret_cast<const float4*>(pp + sp * split_stride);
+        sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
+      }
+      float4 acc = *reinterpret_cast<const float4*>(xr + c);
+      acc.x += sum.x; acc.y += sum.y; acc.z += sum.z; acc.w += sum.w;
+      *reinterpret_cast<float4*>(xr + c) = acc;
+      r[q] = acc;
+      ss += acc.x * acc.x + acc.y * acc.y + acc.z * acc.z + acc.w * acc.w;
+    }
+  }
+  __shared__ float red[8];
+  ss = warp_sum(ss);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  float tot = 0.f;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) tot += red[w];
+  const float rs = rsqrtf(tot / (float)d + eps);
+  uint16_t* yr = xn + (long long)t * d;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int c = (q * 256 + threadIdx.x) * 4;
+    if (c < d) {
+      const uint2 gg = *reinterpret_cast<const uint2*>(gain + c);
+      uint2 o;
+      o.x = pack_bf16x2(r[q].x * rs * bf16_to_f32(gg.x & 0xFFFF), r[q].y * rs * bf16_to_f32(gg.x >> 16));
+      o.y = pack_bf16x2(r[q].z * rs * bf16_to_f32(gg.y & 0xFFFF), r[q].w * rs * bf16_to_f32(gg.y >> 16));
+      *reinterpret_cast<uint2*>(yr + c) = o;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // RoPE: pairs (i, i + hd/2) rotated by the angle pos * theta^(-2i/hd).  The
 // cos/sin of each (position, pair) are computed once per pass in double
 // (rope_table_kernel) and shared by all layers; the rotation is done in
@@ -86,7 +137,9 @@ __global__ void rope_table_kernel(double2* __restrict__ tab, int nq, int L0, int
 }
 
 struct RopeParams {
-  const float* qkv;   // [T, (Hq + 2 Hkv) * hd]
+  const float* qkv;   // [ks][T, (Hq + 2 Hkv) * hd] split-k partial products (summed in order)
+  int ks;
+  long long split_stride;
   const double2* tab; // [nq, hd/2] (cos, sin)
   uint16_t* q;        // [T, Hq * hd]
   uint16_t* kc;       // layer base of K cache
@@ -110,7 +163,9 @@ __global__ void rope_kv_kernel(const RopeParams p) {
       const int b = t / p.nq, pos_in = t - b * p.nq;
       const double2 cs = p.tab[pos_in * half + i];
       const float* src = p.qkv + (long long)t * row_w + h * p.hd;
-      const double x1 = src[i], x2 = src[i + half];
+      float a1 = src[i], a2 = src[i + half];
+      for (int q = 1; q < p.ks; ++q) { a1 += src[q * p.split_stride + i]; a2 += src[q * p.split_stride + i + half]; }
+      const double x1 = a1, x2 = a2;
       const float o1 = (float)(x1 * cs.x - x2 * cs.y), o2 = (float)(x2 * cs.x + x1 * cs.y);
       uint16_t* dst;
       if (h < p.Hq) {
@@ -130,8 +185,10 @@ __global__ void rope_kv_kernel(const RopeParams p) {
       const int b = t / p.nq, pos_in = t - b * p.nq;
       const float* src = p.qkv + (long long)t * row_w + (p.Hq + p.Hkv + g) * p.hd;
       uint16_t* dst = p.vc + (((long long)b * p.Hkv + g) * p.c_max + p.L0 + pos_in) * p.hd;
-      dst[2 * i] = f32_to_bf16(src[2 * i]);
-      dst[2 * i + 1] = f32_to_bf16(src[2 * i + 1]);
+      float a1 = src[2 * i], a2 = src[2 * i + 1];
+      for (int q = 1; q < p.ks; ++q) { a1 += src[q * p.split_stride + 2 * i]; a2 += src[q * p.split_stride + 2 * i + 1]; }
+      dst[2 * i] = f32_to_bf16(a1);
+      dst[2 * i + 1] = f32_to_bf16(a2);
     }
   }
 }
@@ -484,6 +541,19 @@ __global__ void esum_kernel(const float* __restrict__ part, int ks, int T, int d
 }
 
 // ---------------------------------------------------------------------------
+// Per-round parameters read on the device (written by step_params_kernel as
+// the first node of a round, so a captured round can be replayed for any step).
+struct StepDev {
+  int step, max_steps, block, policy;
+  float lock_threshold, stop_entropy, inv_t;
+  int require_stable;
+  uint32_t k0, k1;
+};
+
+__global__ void step_params_kernel(StepDev* dst, const StepDev v) {
+  if (threadIdx.x == 0 && blockIdx.x == 0) *dst = v;
+}
+
 // Canvas update (a9), one CTA of 256 threads per canvas (thread = position).
 struct UpdateParams {
   const float* entropy;
@@ -498,12 +568,7 @@ struct UpdateParams {
   uint8_t* stop_out;    // may be null
   uint8_t* final_out;   // may be null
   uint8_t* flags;       // [B] internal copy of done after the update (host readback)
-  int policy;
-  float lock_threshold;
-  float stop_entropy;
-  int require_stable;
-  int step, max_steps, block;
-  uint32_t k0, k1;
+  const StepDev* sp;    // round parameters
   int vocab;
 };
 
@@ -515,6 +580,7 @@ __global__ void __launch_bounds__(256) canvas_update_kernel(const UpdateParams p
   __shared__ float key[256];
   __shared__ int kid[256];
   __shared__ float csum[256];
+  const StepDev sp = *p.sp;
   const float H = p.entropy[t];
   const float pm = p.pmax[t];
   const int am = p.argmax[t];
@@ -534,8 +600,8 @@ __global__ void __launch_bounds__(256) canvas_update_kernel(const UpdateParams p
 
   // lock mask
   bool lock;
-  if (p.policy == 0) {
-    lock = pm > p.lock_threshold;
+  if (sp.policy == 0) {
+    lock = pm > sp.lock_threshold;
   } else {
     // bitonic sort of (H, position) ascending, then a fixed-order running sum
     key[i] = H;
@@ -562,13 +628,13 @@ __global__ void __launch_bounds__(256) canvas_update_kernel(const UpdateParams p
     // rank of this position in sorted order
     lock = false;
     for (int r = 0; r < 256; ++r)
-      if (kid[r] == i) { lock = csum[r] <= p.lock_threshold; break; }
+      if (kid[r] == i) { lock = csum[r] <= sp.lock_threshold; break; }
   }
   if (p.lock_out) p.lock_out[t] = lock ? 1 : 0;
 
-  const bool stable = p.step > 0 && all_same;
-  const bool stop = !was_done && (meanH < p.stop_entropy) && (!p.require_stable || stable);
-  const bool fin = !was_done && (stop || p.step == p.max_steps - 1);
+  const bool stable = sp.step > 0 && all_same;
+  const bool stop = !was_done && (meanH < sp.stop_entropy) && (!sp.require_stable || stable);
+  const bool fin = !was_done && (stop || sp.step == sp.max_steps - 1);
   if (!was_done) {
     int nt;
     if (fin) {
@@ -576,8 +642,8 @@ __global__ void __launch_bounds__(256) canvas_update_kernel(const UpdateParams p
     } else if (lock) {
       nt = smp;
     } else {
-      const Philox4 r = philox4x32_10(0u, (uint32_t)i, (uint32_t)(p.block * 256 + p.step),
-                                      (kPurposeRenoise << 24) | (uint32_t)b, p.k0, p.k1);
+      const Philox4 r = philox4x32_10(0u, (uint32_t)i, (uint32_t)(sp.block * 256 + sp.step),
+                                      (kPurposeRenoise << 24) | (uint32_t)b, sp.k0, sp.k1);
       nt = uniform_token(r.x, (uint32_t)p.vocab);
     }
     p.tokens[t] = nt;

@@ -138,10 +138,11 @@ class Model:
         check(lib.dg_canvas_init(self.ctx, ctypes.byref(cv.s), block, seed, _stream(stream)))
 
     def step(self, kv: KVCache, cv: Canvas, block: int, step: int, sampler: dg_sampler_config,
-             out: StepOutputs = None, stream=None):
+             out: StepOutputs = None, stream=None, graph: bool = False):
         args = dg_step_args(block, step, sampler)
-        check(lib.dg_denoise_step(self.ctx, ctypes.byref(kv.s), ctypes.byref(cv.s), ctypes.byref(args),
-                                  ctypes.byref(out.s) if out is not None else None, _stream(stream)))
+        fn = lib.dg_denoise_step_graph if graph else lib.dg_denoise_step
+        check(fn(self.ctx, ctypes.byref(kv.s), ctypes.byref(cv.s), ctypes.byref(args),
+                 ctypes.byref(out.s) if out is not None else None, _stream(stream)))
 
     def decode_block(self, kv: KVCache, cv: Canvas, block: int, sampler: dg_sampler_config, out_tokens,
                      stream=None):

@@ -199,6 +199,15 @@ dg_status dg_canvas_init(dg_ctx* ctx, dg_canvas* cv, int32_t block, uint64_t see
 dg_status dg_denoise_step(dg_ctx* ctx, const dg_kv* kv, dg_canvas* cv, const dg_step_args* args,
                           const dg_step_out* out, void* stream);
 
+/* The same round as dg_denoise_step, replayed from a CUDA graph that the
+   context captures on first use and keeps while the KV cache (pointers and
+   length), canvas and output pointers stay the same (a change re-captures
+   it).  Results are bit-identical to dg_denoise_step.  Falls back to direct
+   launches while profiling is on.  The graph belongs to the context: do not
+   call this concurrently on one context. */
+dg_status dg_denoise_step_graph(dg_ctx* ctx, const dg_kv* kv, dg_canvas* cv, const dg_step_args* args,
+                                const dg_step_out* out, void* stream);
+
 /* Decode one block per canvas: dg_canvas_init, rounds until every canvas has
    stopped or the budget is spent (one 8-byte device-to-host read per round),
    copy the blocks to d_out [B, 256] and append them to the context with
