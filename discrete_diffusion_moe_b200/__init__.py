@@ -19,6 +19,9 @@ DG_OK, DG_ERR_INVALID_ARG, DG_ERR_CUDA, DG_ERR_WORKSPACE, DG_ERR_TIMEOUT, DG_ERR
     DG_ERR_BAD_TOKEN = range(7)
 DG_LOCK_PROB, DG_LOCK_ENTROPY_CUMSUM = 0, 1
 
+# size of the library's fixed split-KV scratch array (dg_attention_static_scratch)
+DG_ATTN_STATIC_SCRATCH_BYTES = 16 << 20
+
 _STATUS_NAMES = {0: "DG_OK", 1: "DG_ERR_INVALID_ARG", 2: "DG_ERR_CUDA", 3: "DG_ERR_WORKSPACE",
                  4: "DG_ERR_TIMEOUT", 5: "DG_ERR_UNSUPPORTED", 6: "DG_ERR_BAD_TOKEN"}
 
@@ -108,6 +111,7 @@ def _load():
         "dg_test_grouped_gemm": (I32, [P, I32, I32, P, I32, I32, P, P, I32, P, P]),
         "dg_test_attention": (I32, [P, P, P, P, I32, I32, I32, I32, I32, I32, I32, I32, I32, P, P, P]),
         "dg_test_workspace_buffer": (I32, [P, ctypes.c_char_p, ctypes.POINTER(P), ctypes.POINTER(S)]),
+        "dg_attention_static_scratch": (I32, [P, P, P, P, I32, I32, I32, I32, I32, I32, I32, I32, I32, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)

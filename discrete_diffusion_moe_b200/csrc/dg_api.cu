@@ -1159,3 +1159,45 @@ extern "C" dg_status dg_test_workspace_buffer(dg_ctx* c, const char* name, void*
     }
   return fail(DG_ERR_INVALID_ARG, "unknown workspace buffer %s", name);
 }
+
+// ============================================================================
+// attention whose split-KV partials live in a fixed array of this library
+// (for callers that cannot allocate device memory)
+#include <mutex>
+
+static __device__ __align__(256) float g_attn_scratch[DG_ATTN_STATIC_SCRATCH_BYTES / sizeof(float)];
+
+static float* attn_scratch_address() {
+  static std::mutex mu;
+  static float* addr[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_attn_scratch) != cudaSuccess) return nullptr;
+    addr[dev] = (float*)p;
+  }
+  return addr[dev];
+}
+
+extern "C" dg_status dg_attention_static_scratch(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                                 uint16_t* out, int32_t B, int32_t nq, int32_t L0, int32_t c_max,
+                                                 int32_t Hq, int32_t Hkv, int32_t hd, int32_t causal,
+                                                 int32_t splits, void* stream) {
+  if (!q || !k || !v || !out || B < 1 || nq < 1 || L0 < 0 || L0 + nq > c_max || Hq < 1 || Hkv < 1 ||
+      Hq % Hkv || splits < 0 || splits > kMaxAttnSplits)
+    return fail(DG_ERR_INVALID_ARG, "dg_attention_static_scratch: bad arguments");
+  const int sp = splits == 0 ? 1 : splits;
+  const size_t rows = (size_t)sp * B * Hq * nq;
+  const size_t o_floats = align_up(rows * hd, 64);
+  const size_t need = (o_floats + rows * 2) * sizeof(float);
+  if (sp > 1 && need > DG_ATTN_STATIC_SCRATCH_BYTES)
+    return fail(DG_ERR_INVALID_ARG,
+                "dg_attention_static_scratch: %zu bytes of split partials exceed the %u-byte scratch array",
+                need, (unsigned)DG_ATTN_STATIC_SCRATCH_BYTES);
+  float* base = attn_scratch_address();
+  if (!base) return fail(DG_ERR_CUDA, "cudaGetSymbolAddress of the attention scratch failed");
+  return dg_test_attention(q, k, v, out, B, nq, L0, c_max, Hq, Hkv, hd, causal, sp, base, base + o_floats,
+                           stream);
+}

@@ -244,6 +244,38 @@ dg_status dg_profile_start(dg_ctx* ctx);
 /* Stop, synchronise the recorded events and fill *out. */
 dg_status dg_profile_stop(dg_ctx* ctx, dg_profile* out);
 
+/* ---- attention without caller-provided scratch ---------------------------
+   The pages have no counterpart for this call.  It is for callers that cannot
+   allocate device memory when they call in: code that runs inside a memory
+   pool sized once at start-up, a host program whose allocator is closed after
+   initialisation, or a caller that has no CUDA allocator of its own.
+
+   Computes the same attention as dg_test_attention (dg_testing.h), with the
+   same argument meaning and layout: q bf16 [B * nq, Hq * hd] (token-major),
+   K/V caches bf16 [B][Hkv][c_max][hd] holding keys [0, L0 + nq), out bf16
+   [B * nq, Hq * hd]; causal as there; splits 1..8 key splits (0 means 1).
+   All four pointers are device memory owned by the caller.  The split-KV partial
+   results, which dg_test_attention takes from the caller, live here in one
+   fixed array inside the library, DG_ATTN_STATIC_SCRATCH_BYTES long (16 MiB);
+   every GPU the library runs on holds its own copy for the life of the
+   process.  No cudaMalloc, cudaFree or other allocating routine is called.
+
+   Limit: splits * B * Hq * nq * (hd + 2) * 4 bytes (plus up to 256 bytes of
+   alignment) must fit the array; a larger request returns DG_ERR_INVALID_ARG
+   and launches nothing.  splits 0 or 1 uses no scratch.
+   Set-up: the first call on each GPU (that GPU current) looks up the array's
+   address; make that first call before any stream capture begins.
+   Nothing has to start at zero: each call writes every partial it reads.
+   One array per GPU: calls on the same GPU that may run at the same time
+   (several host threads, or streams with no ordering between them) race on
+   it, so the caller serialises them.  The call returns after its work on
+   `stream` has finished. */
+#define DG_ATTN_STATIC_SCRATCH_BYTES (16u << 20)
+dg_status dg_attention_static_scratch(const uint16_t* d_q, const uint16_t* d_k, const uint16_t* d_v,
+                                      uint16_t* d_out, int32_t B, int32_t nq, int32_t L0, int32_t c_max,
+                                      int32_t Hq, int32_t Hkv, int32_t hd, int32_t causal, int32_t splits,
+                                      void* stream);
+
 #ifdef __cplusplus
 }
 #endif
