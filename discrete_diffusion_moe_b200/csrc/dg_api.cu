@@ -239,6 +239,22 @@ dg_status make_tmap(CUtensorMap* m, const void* base, long long K, long long row
   return DG_OK;
 }
 
+// B operand of a GEMM: three tensor maps of the same matrix with boxes of 16,
+// min(64, bn) and bn rows (each at most the matrix's rows).
+struct BOperand {
+  BMaps maps;
+  int rows[3];
+};
+
+dg_status make_bop(BOperand* b, const void* base, long long K, long long rows, int bn) {
+  const int want[3] = {16, std::min(64, bn), bn};
+  for (int i = 0; i < 3; ++i) {
+    b->rows[i] = (int)std::min<long long>(want[i], rows);
+    DG_TRY(make_tmap(&b->maps.m[i], base, K, rows, b->rows[i]));
+  }
+  return DG_OK;
+}
+
 int device_sms() {
   int dev = 0, n = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
@@ -246,37 +262,43 @@ int device_sms() {
 }
 
 template <class Epi>
-dg_status run_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmPlan& p, const Epi& epi,
-                   int num_sms, cudaStream_t st, long long* launches = nullptr) {
-  if (p.bn < 16 || p.bn > 256 || (p.bn & (p.bn - 1)) || p.bn % p.b_box || p.K % 64 || p.K < 64)
-    return fail(DG_ERR_INVALID_ARG, "gemm plan: bn %d b_box %d K %d", p.bn, p.b_box, p.K);
+dg_status run_gemm(const CUtensorMap& ta, const BOperand& tb, GemmPlan p, const Epi& epi, int num_sms,
+                   cudaStream_t st, long long* launches = nullptr) {
+  if (p.bn < 16 || p.bn > 256 || (p.bn & (p.bn - 1)) || p.K % 64 || p.K < 64)
+    return fail(DG_ERR_INVALID_ARG, "gemm plan: bn %d K %d", p.bn, p.K);
+  for (int i = 0; i < 3; ++i) {
+    if (tb.rows[i] < 1 || tb.rows[i] > p.bn || (i && tb.rows[i] < tb.rows[i - 1]))
+      return fail(DG_ERR_INVALID_ARG, "gemm plan: B box rows %d of bn %d", tb.rows[i], p.bn);
+    p.b_rows[i] = tb.rows[i];
+  }
   static bool attr_done = false;
   if (!attr_done) {
     DG_CUDA(cudaFuncSetAttribute(gemm_tc_kernel<Epi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  227 * 1024));
+    DG_CUDA(cudaFuncSetAttribute(gemm_tc_kernel<Epi>, cudaFuncAttributePreferredSharedMemoryCarveout, 100));
     attr_done = true;
   }
-  const int stages = gemm_pick_stages(p.bn);
+  const int ctas = gemm_ctas_per_sm(p.bn);
+  const int stages = gemm_pick_stages(p.bn, ctas);
   const size_t smem = gemm_smem_bytes(p.bn, stages);
-  long long units;  // grouped: known only on the device; one persistent CTA per SM
-  if (p.group_off) units = num_sms;
+  long long units;  // grouped: known only on the device; persistent CTAs
+  if (p.group_off) units = (long long)ctas * num_sms;
   else units = (long long)p.m_tiles * ((p.n_total + p.bn - 1) / p.bn) * p.k_splits;
   if (units <= 0) return DG_OK;
-  const int grid = (int)std::min<long long>(units, num_sms);
-  gemm_tc_kernel<Epi><<<grid, kGemmThreads, smem, st>>>(ta, tb, p, epi, stages);
+  const int grid = (int)std::min<long long>(units, (long long)ctas * num_sms);
+  gemm_tc_kernel<Epi><<<grid, kGemmThreads, smem, st>>>(ta, tb.maps, p, epi, stages);
   DG_CUDA(cudaGetLastError());
   if (launches) ++*launches;
   return DG_OK;
 }
 
-GemmPlan dense_plan(int K, int a_rows, int n_total, int bn, int b_box, int k_splits, int* err) {
+GemmPlan dense_plan(int K, int a_rows, int n_total, int bn, int k_splits, int* err) {
   GemmPlan p{};
   p.K = K;
   p.a_rows = a_rows;
   p.m_tiles = (a_rows + 127) / 128;
   p.n_total = n_total;
   p.bn = bn;
-  p.b_box = b_box;
   p.k_splits = k_splits;
   p.n_fast = 1;
   p.group_off = nullptr;
@@ -293,7 +315,6 @@ GemmPlan grouped_plan(int K, int rows_per_group, const int* off, const int* chun
   p.m_tiles = (rows_per_group + 127) / 128;
   p.n_total = 0;
   p.bn = bn;
-  p.b_box = 16;
   p.k_splits = 1;
   p.group_off = off;
   p.n_groups = n_groups;
@@ -312,7 +333,6 @@ int dense_bn(int m_tiles, int T, int num_sms) {
   while (bn > 16 && (long long)m_tiles * ((T + bn - 1) / bn) < (3 * num_sms) / 4) bn >>= 1;
   return bn;
 }
-int box_for(int bn) { return std::min(64, bn); }
 
 }  // namespace
 
@@ -509,18 +529,15 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
   int* err = c->err();
   float* x = c->at<float>(L.x);
   uint16_t* xn = c->at<uint16_t>(L.xn);
-  const int bnT = token_bn(T), boxT = box_for(bnT);
   // token rows per grouped unit: 128 (256 for large batches).  Routing can be
   // very uneven; one unit per 128 tokens of an expert keeps the number of times
   // a weight tile is read small while the units of one tile run side by side.
   const int bnG = P / E > 64 ? 256 : 128;
   const size_t kv_layer = (size_t)kv->batch * Hkv * kv->c_max * hd;
 
-  CUtensorMap t_xn, t_attn, t_xperm, t_hperm;
-  DG_TRY(make_tmap(&t_xn, xn, d, L.T_alloc, boxT));
-  DG_TRY(make_tmap(&t_attn, c->at<uint16_t>(L.attn), (long long)Hq * hd, L.T_alloc, boxT));
-  DG_TRY(make_tmap(&t_xperm, c->at<uint16_t>(L.xperm), d, L.P_alloc, 16));
-  DG_TRY(make_tmap(&t_hperm, c->at<uint16_t>(L.hperm), f, L.P_alloc, 16));
+  BOperand t_xperm, t_hperm;
+  DG_TRY(make_bop(&t_xperm, c->at<uint16_t>(L.xperm), d, L.P_alloc, bnG));
+  DG_TRY(make_bop(&t_hperm, c->at<uint16_t>(L.hperm), f, L.P_alloc, bnG));
 
   // cos/sin of this pass's positions, shared by all layers
   {
@@ -554,11 +571,12 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
     }
     {
       ProfScope ps_(c, DG_PROF_DENSE, st);
-      CUtensorMap ta, tb;
+      CUtensorMap ta;
+      BOperand tb;
       const int bn = token_bn(T);
       DG_TRY(make_tmap(&ta, c->wp(W.wqkv), d, qkv_rows, 128));
-      DG_TRY(make_tmap(&tb, xn, d, L.T_alloc, box_for(bn)));
-      GemmPlan p = dense_plan(d, qkv_rows, T, bn, box_for(bn), ks_qkv, err);
+      DG_TRY(make_bop(&tb, xn, d, L.T_alloc, bn));
+      GemmPlan p = dense_plan(d, qkv_rows, T, bn, ks_qkv, err);
       p.a_hint = 1;
       EpiStoreT e{c->at<float>(L.qkv), qkv_rows, (long long)T * qkv_rows, 0, nullptr, nullptr, 0, err};
       DG_TRY(run_gemm(ta, tb, p, e, c->num_sms, st, &c->n_launch));
@@ -593,11 +611,12 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
     }
     {
       ProfScope ps_(c, DG_PROF_DENSE, st);
-      CUtensorMap ta, tb;
+      CUtensorMap ta;
+      BOperand tb;
       const int bn = token_bn(T);
       DG_TRY(make_tmap(&ta, c->wp(W.wo), (long long)Hq * hd, d, 128));
-      DG_TRY(make_tmap(&tb, c->at<uint16_t>(L.attn), (long long)Hq * hd, L.T_alloc, box_for(bn)));
-      GemmPlan p = dense_plan(Hq * hd, d, T, bn, box_for(bn), ks_o, err);
+      DG_TRY(make_bop(&tb, c->at<uint16_t>(L.attn), (long long)Hq * hd, L.T_alloc, bn));
+      GemmPlan p = dense_plan(Hq * hd, d, T, bn, ks_o, err);
       p.a_hint = 1;
       EpiStoreT e{c->at<float>(L.opart), d, (long long)T * d, 0, nullptr, nullptr, 0, err};
       DG_TRY(run_gemm(ta, tb, p, e, c->num_sms, st, &c->n_launch));
@@ -609,11 +628,12 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
     CNT(c);
     {
       ProfScope ps_(c, DG_PROF_DENSE, st);
-      CUtensorMap ta, tb;
+      CUtensorMap ta;
+      BOperand tb;
       const int bn = std::max(32, dense_bn((E + 127) / 128, T, c->num_sms / L.ks_r));
       DG_TRY(make_tmap(&ta, c->wp(W.wr), d, c->wl.wr_rows, 128));
-      DG_TRY(make_tmap(&tb, xn, d, L.T_alloc, box_for(bn)));
-      GemmPlan p = dense_plan(d, E, T, bn, box_for(bn), L.ks_r, err);
+      DG_TRY(make_bop(&tb, xn, d, L.T_alloc, bn));
+      GemmPlan p = dense_plan(d, E, T, bn, L.ks_r, err);
       EpiStoreT e{c->at<float>(L.rpart), E, (long long)T * E, 0, nullptr, nullptr, 0, err};
       DG_TRY(run_gemm(ta, tb, p, e, c->num_sms, st, &c->n_launch));
     }
@@ -775,7 +795,7 @@ static dg_status enqueue_round(dg_ctx* c, const dg_kv* kv, dg_canvas* cv, const 
   const dg_sampler_config& s = a->sampler;
   const int B = cv->batch, T = B * DG_CANVAS, d = m.d_model, V = m.vocab;
   int* err = c->err();
-  const int bnT = token_bn(T), boxT = box_for(bnT);
+  const int bnT = token_bn(T);
   dg_step_out none{};
   if (!o) o = &none;
   StepDev* sp = c->at<StepDev>(L.stepdev);
@@ -794,11 +814,12 @@ static dg_status enqueue_round(dg_ctx* c, const dg_kv* kv, dg_canvas* cv, const 
   // a1: canvas embedding (+ self-conditioning input)
   if (m.self_cond) {
     ProfScope ps_(c, DG_PROF_DENSE, st);
-    CUtensorMap ta, tb;
+    CUtensorMap ta;
+    BOperand tb;
     const int bn = dense_bn((d + 127) / 128, T, c->num_sms);
     DG_TRY(make_tmap(&ta, c->wp(c->wl.sc), d, d, 128));
-    DG_TRY(make_tmap(&tb, cv->sc_state, d, T, box_for(bn)));
-    GemmPlan p = dense_plan(d, d, T, bn, box_for(bn), 1, err);
+    DG_TRY(make_bop(&tb, cv->sc_state, d, T, bn));
+    GemmPlan p = dense_plan(d, d, T, bn, 1, err);
     p.a_hint = 1;
     EpiStoreT e{c->at<float>(L.x), d, 0, 2, c->wp(c->wl.emb), cv->tokens, V, err};
     DG_TRY(run_gemm(ta, tb, p, e, c->num_sms, st, &c->n_launch));
@@ -823,10 +844,11 @@ static dg_status enqueue_round(dg_ctx* c, const dg_kv* kv, dg_canvas* cv, const 
                    c->at<int>(L.vp_ai), c->at<float>(L.vp_gv), c->at<int>(L.vp_gi)};
   {
     ProfScope ps_(c, DG_PROF_LM_HEAD, st);
-    CUtensorMap ta, tb;
+    CUtensorMap ta;
+    BOperand tb;
     DG_TRY(make_tmap(&ta, xn, d, L.T_alloc, 128));
-    DG_TRY(make_tmap(&tb, c->wp(c->wl.lm), d, V, 64));
-    GemmPlan p = dense_plan(d, T, V, 256, 64, 1, err);
+    DG_TRY(make_bop(&tb, c->wp(c->wl.lm), d, V, 256));
+    GemmPlan p = dense_plan(d, T, V, 256, 1, err);
     p.n_fast = 0;
     p.a_hint = 2;
     p.b_hint = 1;
@@ -850,10 +872,11 @@ static dg_status enqueue_round(dg_ctx* c, const dg_kv* kv, dg_canvas* cv, const 
         logits, ps.m, ps.inv_z, probs, T, V);
         CNT(c);
     const int ks = esum_splits(m, T, c->num_sms);
-    CUtensorMap ta, tb;
+    CUtensorMap ta;
+    BOperand tb;
     DG_TRY(make_tmap(&ta, c->wp(c->wl.embT), V, d, 128));
-    DG_TRY(make_tmap(&tb, probs, V, L.T_alloc, boxT));
-    GemmPlan p = dense_plan(V, d, T, bnT, boxT, ks, err);
+    DG_TRY(make_bop(&tb, probs, V, L.T_alloc, bnT));
+    GemmPlan p = dense_plan(V, d, T, bnT, ks, err);
     p.a_hint = 1;
     p.b_hint = 2;
     EpiStoreT e{c->at<float>(L.epart), d, (long long)T * d, 0, nullptr, nullptr, 0, err};
@@ -1075,11 +1098,12 @@ extern "C" dg_status dg_test_gemm(const uint16_t* A, int32_t M, const uint16_t* 
     return fail(DG_ERR_INVALID_ARG, "dg_test_gemm: bad arguments");
   cudaStream_t st = (cudaStream_t)stream;
   int* err = nullptr;
-  const int bn = token_bn(N), box = box_for(bn);
-  CUtensorMap ta, tb;
+  const int bn = token_bn(N);
+  CUtensorMap ta;
+  BOperand tb;
   DG_TRY(make_tmap(&ta, A, K, M, 128));
-  DG_TRY(make_tmap(&tb, B, K, N, box));
-  GemmPlan p = dense_plan(K, M, N, bn, box, k_splits, err);
+  DG_TRY(make_bop(&tb, B, K, N, bn));
+  GemmPlan p = dense_plan(K, M, N, bn, k_splits, err);
   p.n_fast = 0;
   EpiSplitRows e{D, M, N};
   DG_TRY(run_gemm(ta, tb, p, e, device_sms(), st));
@@ -1095,9 +1119,10 @@ extern "C" dg_status dg_test_grouped_gemm(const uint16_t* A, int32_t rows_per_gr
     return fail(DG_ERR_INVALID_ARG, "dg_test_grouped_gemm: bad arguments");
   if ((long long)rows_per_group * n_groups < 128) return fail(DG_ERR_INVALID_ARG, "A needs >= 128 rows");
   cudaStream_t st = (cudaStream_t)stream;
-  CUtensorMap ta, tb;
+  CUtensorMap ta;
+  BOperand tb;
   DG_TRY(make_tmap(&ta, A, K, (long long)rows_per_group * n_groups, 128));
-  DG_TRY(make_tmap(&tb, B, K, n_rows, 16));
+  DG_TRY(make_bop(&tb, B, K, n_rows, bn));
   chunk_offsets_kernel<<<1, 1, 0, st>>>(off, n_groups, bn, choff);
   GemmPlan p = grouped_plan(K, rows_per_group, off, choff, n_groups, bn, nullptr);
   EpiGroupedT e{D, rows_per_group};

@@ -3,8 +3,14 @@
 //   D[m, n] = sum_k A[m, k] * B[n, k]      (bf16 inputs, fp32 accumulate)
 //
 // A and B are K-major bf16 matrices read through 2-D TMA tensor maps with the
-// 128-byte swizzle (box: 64 elements of K x 128 rows for A, x b_box rows for
-// B).  One CTA per SM loops over work units:
+// 128-byte swizzle (box: 64 elements of K x 128 rows for A).  B comes with
+// three tensor maps of 16, min(64, bn) and bn rows per box: every stage loads
+// its B rows with ONE copy, the smallest box that covers the unit's columns.
+// The per-CTA copy engine rate, not the number of bytes in flight, limits how
+// fast a CTA fills its stages (a few hundred cycles per 32 KB stage, plus
+// about a hundred per copy), so each stage is exactly two copies and, for
+// tiles of at most 128 columns, two CTAs share an SM.  Each CTA loops over
+// work units:
 //   warp 0      TMA producer (one elected lane) filling a ring of smem stages
 //   warp 1      allocates tensor memory; one lane issues tcgen05.mma (M = 128,
 //               N = the unit's columns rounded up to 16) into one of two
@@ -40,7 +46,7 @@ struct GemmPlan {
   int m_tiles;           // dense: ceil(M / 128); grouped: tiles per group
   int n_total;           // dense: rows of B (N)
   int bn;                // columns per pass: multiple of 16, <= 256
-  int b_box;             // rows per TMA box of B (divides bn)
+  int b_rows[3];         // rows per box of the three B tensor maps (ascending, last covers bn)
   int k_splits;          // dense: K loop split into this many units (>= 1)
   int n_fast;            // dense: 1 = consecutive units walk the N tiles of one A tile
   const int* group_off;  // grouped when non-null: [n_groups + 1] B row offsets
@@ -123,9 +129,14 @@ __device__ __forceinline__ GemmJob gemm_job(const GemmPlan& p, int u, int) {
 constexpr int kGemmThreads = 192;
 constexpr int kATileBytes = 128 * 128;  // 128 rows x 64 bf16
 
+// B tensor maps: boxes of b_rows[0] / b_rows[1] / b_rows[2] rows
+struct BMaps {
+  CUtensorMap m[3];
+};
+
 template <class Epi>
-__global__ void __launch_bounds__(kGemmThreads, 1)
-    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+__global__ void __launch_bounds__(kGemmThreads, 2)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ BMaps tmB,
                    const GemmPlan p, const Epi epi, const int stages) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte alignment for the swizzled tiles
@@ -157,7 +168,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     fence_mbar_init();
     fence_proxy_async_smem();
     tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB);
+    for (int i = 0; i < 3; ++i) tma_prefetch_desc(&tmB.m[i]);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), tmem_cols);
@@ -183,8 +194,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int pass = 0; pass < np && ok; ++pass) {
           const GemmJob j = gemm_job(p, u, pass);
           const int n_mma = (j.n_valid + 15) & ~15;
-          const int nbox = (n_mma + p.b_box - 1) / p.b_box;
-          const uint32_t tx = kATileBytes + (uint32_t)nbox * p.b_box * 128;
+          const int bi = n_mma <= p.b_rows[0] ? 0 : (n_mma <= p.b_rows[1] ? 1 : 2);
+          const CUtensorMap* mb = &tmB.m[bi];
+          const uint32_t tx = kATileBytes + (uint32_t)p.b_rows[bi] * 128;
           for (int kb = j.kb0; kb < j.kb1; ++kb, ++it) {
             const int s = it % stages;
             const uint32_t ph = (it / stages) & 1;
@@ -194,11 +206,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const uint32_t dA = smem_u32(sA + (size_t)s * kATileBytes);
             if (p.a_hint) tma_load_2d_hint(dA, &tmA, fb, kb * 64, j.a_row0, pol_a);
             else          tma_load_2d(dA, &tmA, fb, kb * 64, j.a_row0);
-            for (int b = 0; b < nbox; ++b) {
-              const uint32_t dB = smem_u32(sB + (size_t)s * b_stage_bytes + b * p.b_box * 128);
-              if (p.b_hint) tma_load_2d_hint(dB, &tmB, fb, kb * 64, j.n0 + b * p.b_box, pol_b);
-              else          tma_load_2d(dB, &tmB, fb, kb * 64, j.n0 + b * p.b_box);
-            }
+            const uint32_t dB = smem_u32(sB + (size_t)s * b_stage_bytes);
+            if (p.b_hint) tma_load_2d_hint(dB, mb, fb, kb * 64, j.n0, pol_b);
+            else          tma_load_2d(dB, mb, fb, kb * 64, j.n0);
           }
         }
       }
@@ -283,8 +293,14 @@ inline size_t gemm_smem_bytes(int bn, int stages) {
   return 1024 + (size_t)stages * (kATileBytes + (size_t)bn * 128) + (2 * stages + 5) * 8 + 16;
 }
 
-inline int gemm_pick_stages(int bn, int max_stages = 8) {
-  const size_t budget = 227 * 1024;
+// CTAs per SM: two when both fit (tensor memory: 2 x 2 x bn columns <= 512;
+// shared memory: at least three stages each), else one.
+inline int gemm_ctas_per_sm(int bn) { return bn <= 128 ? 2 : 1; }
+
+// Stages that fit `ctas` CTAs in one SM's 228 KB (1 KB of each CTA's share is
+// reserved by the system).
+inline int gemm_pick_stages(int bn, int ctas, int max_stages = 8) {
+  const size_t budget = (size_t)228 * 1024 / ctas - 1024;
   int s = max_stages;
   while (s > 2 && gemm_smem_bytes(bn, s) > budget) --s;
   return s;
