@@ -14,7 +14,7 @@
 #include "../../include/dg.h"
 #include "../../include/dg_testing.h"
 #include "../../synth/synth.h"
-#include "attention.cuh"
+#include "attention_tc.cuh"
 #include "epilogues.cuh"
 #include "gemm_tc.cuh"
 #include "kernels.cuh"
@@ -239,6 +239,28 @@ dg_status make_tmap(CUtensorMap* m, const void* base, long long K, long long row
   return DG_OK;
 }
 
+// General 2-D bf16 tensor map: `rows` rows of `inner` elements, `stride_bytes`
+// apart; box box_inner x box_rows with the 128-byte swizzle (box_inner = 64).
+// Elements past `inner` or `rows` read as zero.
+dg_status make_tmap_2d(CUtensorMap* m, const void* base, long long inner, long long rows, long long stride_bytes,
+                       int box_inner, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(DG_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  if (((uintptr_t)base & 15) || inner < 1 || rows < 1 || stride_bytes % 16 || box_inner * 2 != 128 ||
+      box_rows < 1 || box_rows > 256)
+    return fail(DG_ERR_INVALID_ARG, "tensor map: bad base/extent/stride (%p, %lld, %lld, %lld)", base, inner, rows,
+                stride_bytes);
+  cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)stride_bytes};
+  cuuint32_t box[2] = {(cuuint32_t)box_inner, (cuuint32_t)box_rows};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(DG_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return DG_OK;
+}
+
 // B operand of a GEMM: three tensor maps of the same matrix with boxes of 16,
 // min(64, bn) and bn rows (each at most the matrix's rows).
 struct BOperand {
@@ -419,7 +441,10 @@ extern "C" size_t dg_weights_bytes(const dg_model_config* cfg) {
 
 extern "C" size_t dg_kv_bytes(const dg_model_config* cfg, int32_t batch, int32_t c_max) {
   char why[256];
-  if (!cfg_ok(cfg, why, sizeof why) || batch < 1 || c_max < 1) { fail(DG_ERR_INVALID_ARG, "bad kv size query"); return 0; }
+  if (!cfg_ok(cfg, why, sizeof why) || batch < 1 || c_max < 8 || c_max % 8) {
+    fail(DG_ERR_INVALID_ARG, "bad kv size query (c_max must be a positive multiple of 8)");
+    return 0;
+  }
   return (size_t)cfg->n_layers * batch * cfg->n_kv_heads * c_max * cfg->head_dim * 2;
 }
 
@@ -515,6 +540,64 @@ extern "C" dg_status dg_context_create(const dg_model_config* cfg, const void* d
 
 extern "C" void dg_context_destroy(dg_ctx* ctx) { delete ctx; }
 
+// ---------------------------------------------------------------------------
+// Attention of one pass on the tensor cores: q packed [B][Hkv][nq][G][hd],
+// K cache [B][Hkv][c_max][hd], V^T cache [B][Hkv][hd][c_max]; splits > 1
+// writes per-split partials and merges them (fixed split order) into out.
+template <int HD>
+static bool attn_tc_ready() {
+  static bool done = false;
+  if (!done)
+    done = cudaFuncSetAttribute(attn_tc_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)AttnTcShape<HD>::SMEM) == cudaSuccess;
+  return done;
+}
+
+static dg_status run_attention(const uint16_t* q, const uint16_t* kc, const uint16_t* vc, uint16_t* out,
+                               float* part_o, float* part_ml, int B, int nq, int L0, int c_max, int Hq, int Hkv,
+                               int hd, bool causal, int splits, int* err, cudaStream_t st, long long* launches) {
+  if (c_max % 8) return fail(DG_ERR_INVALID_ARG, "c_max %d is not a multiple of 8", c_max);
+  if (splits > 1 && (!part_o || !part_ml)) return fail(DG_ERR_INVALID_ARG, "split buffers are null");
+  const int G = Hq / Hkv;
+  CUtensorMap tq, tk, tv;
+  DG_TRY(make_tmap_2d(&tq, q, hd, (long long)B * Hkv * nq * G, (long long)hd * 2, 64, kAttnRows));
+  DG_TRY(make_tmap_2d(&tk, kc, hd, (long long)B * Hkv * c_max, (long long)hd * 2, 64, kAttnKeys));
+  DG_TRY(make_tmap_2d(&tv, vc, L0 + nq, (long long)B * Hkv * hd, (long long)c_max * 2, 64, hd));
+  AttnTcParams ap{out, part_o, part_ml, B, nq, L0, c_max, Hq, Hkv, splits, causal ? 1 : 0,
+                  (float)(1.4426950408889634 / sqrt((double)hd)), err};
+  dim3 grid((G * nq + kAttnRows - 1) / kAttnRows, Hkv, B * splits);
+  bool ready = false;
+  switch (hd) {
+    case 32: if ((ready = attn_tc_ready<32>())) attn_tc_kernel<32><<<grid, kAttnThreads, AttnTcShape<32>::SMEM, st>>>(tq, tk, tv, ap); break;
+    case 64: if ((ready = attn_tc_ready<64>())) attn_tc_kernel<64><<<grid, kAttnThreads, AttnTcShape<64>::SMEM, st>>>(tq, tk, tv, ap); break;
+    case 128: if ((ready = attn_tc_ready<128>())) attn_tc_kernel<128><<<grid, kAttnThreads, AttnTcShape<128>::SMEM, st>>>(tq, tk, tv, ap); break;
+    case 176: if ((ready = attn_tc_ready<176>())) attn_tc_kernel<176><<<grid, kAttnThreads, AttnTcShape<176>::SMEM, st>>>(tq, tk, tv, ap); break;
+    default: return fail(DG_ERR_UNSUPPORTED, "head_dim %d", hd);
+  }
+  if (!ready) return fail(DG_ERR_CUDA, "attention shared-memory attribute");
+  DG_CUDA(cudaGetLastError());
+  if (launches) ++*launches;
+  if (splits > 1) {
+    const long long rows = (long long)B * Hq * nq;
+    attn_combine_kernel<<<(unsigned)((rows * 32 + 255) / 256), 256, 0, st>>>(part_o, part_ml, out, splits, B, Hq,
+                                                                             nq, hd);
+    DG_CUDA(cudaGetLastError());
+    if (launches) ++*launches;
+  }
+  return DG_OK;
+}
+
+// Key splits of a pass: enough CTAs to cover the SMs once (at most 8 splits,
+// at most one split per 64-key tile).
+static int attn_splits(int B, int nq, int L0, int Hq, int Hkv, int num_sms, int cap_rows) {
+  const int base = ((Hq / Hkv) * nq + kAttnRows - 1) / kAttnRows * Hkv * B;
+  const int n_kt = (L0 + nq + kAttnKeys - 1) / kAttnKeys;
+  int s = std::max(1, std::min(num_sms / std::max(1, base), kMaxAttnSplits));
+  s = std::min(s, n_kt);
+  while (s > 1 && (long long)s * B > cap_rows) --s;
+  return s;
+}
+
 // ============================================================================
 // one pass of the transformer layers over T = B * nq tokens at positions
 // L0 .. L0 + nq - 1 (x already holds the embedded inputs)
@@ -551,13 +634,8 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
   const int ks_qkv = dense_splits((qkv_rows + 127) / 128, (T + 255) / 256, d / 64, c->num_sms);
   const int ks_o = dense_splits((d + 127) / 128, (T + 255) / 256, Hq * hd / 64, c->num_sms);
 
-  // attention launch shape
-  const int q_tiles = ((Hq / Hkv) * nq + 63) / 64;
-  const int base_ctas = q_tiles * Hkv * B;
-  const int n_kt = (L0 + nq + 63) / 64;
-  int splits = std::max(1, std::min((2 * c->num_sms + base_ctas - 1) / base_ctas, kMaxAttnSplits));
-  splits = std::min(splits, n_kt);
-  while (splits > 1 && (long long)splits * B > L.attn_rows_cap) --splits;
+  // attention key splits
+  const int splits = attn_splits(B, nq, L0, Hq, Hkv, c->num_sms, L.attn_rows_cap);
 
   for (int l = 0; l < m.n_layers; ++l) {
     const LayerW& W = c->wl.layers[l];
@@ -582,32 +660,18 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
       DG_TRY(run_gemm(ta, tb, p, e, c->num_sms, st, &c->n_launch));
     }
     {
+      const int rot_blocks = std::min(4096, (T * (Hq + Hkv) * hd / 2 + 255) / 256);
+      const int v_blocks = B * Hkv * ((nq + kRopeVTok - 1) / kRopeVTok);
       RopeParams rp{c->at<float>(L.qkv), ks_qkv, (long long)T * qkv_rows, c->at<double2>(L.rope),
-                    c->at<uint16_t>(L.q), kc, vc, T, nq, L0, kv->c_max, Hq, Hkv, hd};
-      rope_kv_kernel<<<std::min(4096, (T * (Hq + 2 * Hkv) * hd / 2 + 255) / 256), 256, 0, st>>>(rp);
+                    c->at<uint16_t>(L.q), kc, vc, T, nq, L0, kv->c_max, Hq, Hkv, hd, rot_blocks};
+      rope_kv_kernel<<<rot_blocks + v_blocks, 256, 0, st>>>(rp);
       CNT(c);
     }
     {
       ProfScope ps_(c, DG_PROF_ATTENTION, st);
-      AttnParams ap{c->at<uint16_t>(L.q), kc, vc, c->at<uint16_t>(L.attn), c->at<float>(L.attn_po),
-                    c->at<float>(L.attn_pml), B, nq, L0, kv->c_max, Hq, Hkv, splits, causal ? 1 : 0,
-                    (float)(1.4426950408889634 / sqrt((double)hd))};
-      dim3 grid(q_tiles, Hkv, B * splits);
-      switch (hd) {
-        case 32: attn_kernel<32><<<grid, 128, attn_smem_bytes<32>(), st>>>(ap); break;
-        case 64: attn_kernel<64><<<grid, 128, attn_smem_bytes<64>(), st>>>(ap); break;
-        case 128: attn_kernel<128><<<grid, 128, attn_smem_bytes<128>(), st>>>(ap); break;
-        case 176: attn_kernel<176><<<grid, 128, attn_smem_bytes<176>(), st>>>(ap); break;
-        default: return fail(DG_ERR_UNSUPPORTED, "head_dim %d", hd);
-      }
-      CNT(c);
-      DG_CUDA(cudaGetLastError());
-      if (splits > 1) {
-        const long long rows = (long long)B * Hq * nq;
-        attn_combine_kernel<<<(unsigned)((rows * 32 + 255) / 256), 256, 0, st>>>(
-            c->at<float>(L.attn_po), c->at<float>(L.attn_pml), c->at<uint16_t>(L.attn), splits, B, Hq, nq, hd);
-            CNT(c);
-      }
+      DG_TRY(run_attention(c->at<uint16_t>(L.q), kc, vc, c->at<uint16_t>(L.attn), c->at<float>(L.attn_po),
+                           c->at<float>(L.attn_pml), B, nq, L0, kv->c_max, Hq, Hkv, hd, causal, splits, err, st,
+                           &c->n_launch));
     }
     {
       ProfScope ps_(c, DG_PROF_DENSE, st);
@@ -688,25 +752,12 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
 static dg_status check_kv(const dg_ctx* c, const dg_kv* kv, int extra) {
   if (!kv || !kv->k || !kv->v) return fail(DG_ERR_INVALID_ARG, "kv buffers are null");
   if (kv->batch < 1 || kv->batch > c->batch_max) return fail(DG_ERR_INVALID_ARG, "kv batch %d outside [1, %d]", kv->batch, c->batch_max);
-  if (kv->length < 0 || kv->c_max < 1 || (long long)kv->length + extra > kv->c_max)
+  if (kv->c_max < 8 || kv->c_max % 8) return fail(DG_ERR_INVALID_ARG, "kv c_max %d is not a positive multiple of 8", kv->c_max);
+  if (kv->length < 0 || (long long)kv->length + extra > kv->c_max)
     return fail(DG_ERR_INVALID_ARG, "kv length %d + %d exceeds c_max %d", kv->length, extra, kv->c_max);
   return DG_OK;
 }
 
-static bool attn_smem_ready(int hd) {
-  static bool done[4] = {false, false, false, false};
-  int slot = hd == 32 ? 0 : hd == 64 ? 1 : hd == 128 ? 2 : 3;
-  if (done[slot]) return true;
-  cudaError_t e = cudaSuccess;
-  switch (hd) {
-    case 32: e = cudaFuncSetAttribute(attn_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, attn_smem_bytes<32>()); break;
-    case 64: e = cudaFuncSetAttribute(attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, attn_smem_bytes<64>()); break;
-    case 128: e = cudaFuncSetAttribute(attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, attn_smem_bytes<128>()); break;
-    case 176: e = cudaFuncSetAttribute(attn_kernel<176>, cudaFuncAttributeMaxDynamicSharedMemorySize, attn_smem_bytes<176>()); break;
-  }
-  done[slot] = e == cudaSuccess;
-  return done[slot];
-}
 
 extern "C" dg_status dg_encode_context(dg_ctx* c, dg_kv* kv, const int32_t* d_tokens, int32_t n, void* stream) {
   if (!c) return fail(DG_ERR_INVALID_ARG, "null context");
@@ -714,7 +765,6 @@ extern "C" dg_status dg_encode_context(dg_ctx* c, dg_kv* kv, const int32_t* d_to
   DG_TRY(check_kv(c, kv, n));
   if (n == 0) return DG_OK;
   if (!d_tokens) return fail(DG_ERR_INVALID_ARG, "tokens are null");
-  if (!attn_smem_ready(c->cfg.head_dim)) return fail(DG_ERR_CUDA, "attention smem attribute");
   cudaStream_t st = (cudaStream_t)stream;
   const int B = kv->batch, d = c->cfg.d_model;
   int* tok_tmp = c->at<int>(c->L.st_samp);  // [T] staging of the chunk's token ids
@@ -782,7 +832,6 @@ static dg_status check_round_args(dg_ctx* c, const dg_kv* kv, dg_canvas* cv, con
   if (s.lock_policy != DG_LOCK_PROB && s.lock_policy != DG_LOCK_ENTROPY_CUMSUM)
     return fail(DG_ERR_INVALID_ARG, "lock policy");
   if (!(s.t_start > 0.f) || !(s.t_end > 0.f)) return fail(DG_ERR_INVALID_ARG, "temperatures must be > 0");
-  if (!attn_smem_ready(c->cfg.head_dim)) return fail(DG_ERR_CUDA, "attention smem attribute");
   return DG_OK;
 }
 
@@ -1138,28 +1187,10 @@ extern "C" dg_status dg_test_attention(const uint16_t* q, const uint16_t* k, con
   if (!q || !k || !v || !out || B < 1 || nq < 1 || L0 < 0 || L0 + nq > c_max || Hq < 1 || Hkv < 1 ||
       Hq % Hkv || splits < 0 || splits > kMaxAttnSplits)
     return fail(DG_ERR_INVALID_ARG, "dg_test_attention: bad arguments");
-  if (splits > 1 && (!part_o || !part_ml)) return fail(DG_ERR_INVALID_ARG, "split buffers are null");
-  if (!attn_smem_ready(hd)) return fail(DG_ERR_UNSUPPORTED, "head_dim %d", hd);
   cudaStream_t st = (cudaStream_t)stream;
   if (splits == 0) splits = 1;
-  const int q_tiles = ((Hq / Hkv) * nq + 63) / 64;
-  AttnParams ap{q, k, v, out, part_o, part_ml, B, nq, L0, c_max, Hq, Hkv, splits, causal,
-                (float)(1.4426950408889634 / sqrt((double)hd))};
-  dim3 grid(q_tiles, Hkv, B * splits);
-  switch (hd) {
-    case 32: attn_kernel<32><<<grid, 128, attn_smem_bytes<32>(), st>>>(ap); break;
-    case 64: attn_kernel<64><<<grid, 128, attn_smem_bytes<64>(), st>>>(ap); break;
-    case 128: attn_kernel<128><<<grid, 128, attn_smem_bytes<128>(), st>>>(ap); break;
-    case 176: attn_kernel<176><<<grid, 128, attn_smem_bytes<176>(), st>>>(ap); break;
-    default: return fail(DG_ERR_UNSUPPORTED, "head_dim %d", hd);
-  }
-  DG_CUDA(cudaGetLastError());
-  if (splits > 1) {
-    const long long rows = (long long)B * Hq * nq;
-    attn_combine_kernel<<<(unsigned)((rows * 32 + 255) / 256), 256, 0, st>>>(part_o, part_ml, out, splits, B,
-                                                                             Hq, nq, hd);
-    DG_CUDA(cudaGetLastError());
-  }
+  DG_TRY(run_attention(q, k, v, out, part_o, part_ml, B, nq, L0, c_max, Hq, Hkv, hd, causal != 0, splits, nullptr,
+                       st, nullptr));
   DG_CUDA(cudaStreamSynchronize(st));
   return DG_OK;
 }

@@ -141,21 +141,30 @@ struct RopeParams {
   int ks;
   long long split_stride;
   const double2* tab; // [nq, hd/2] (cos, sin)
-  uint16_t* q;        // [T, Hq * hd]
-  uint16_t* kc;       // layer base of K cache
-  uint16_t* vc;       // layer base of V cache
+  uint16_t* q;        // packed queries [B][Hkv][nq][G][hd], G = Hq / Hkv
+  uint16_t* kc;       // layer base of K cache   [B][Hkv][c_max][hd]
+  uint16_t* vc;       // layer base of V^T cache [B][Hkv][hd][c_max]
   int T, nq, L0, c_max, Hq, Hkv, hd;
+  int rot_blocks;     // blocks [0, rot_blocks) rotate q and k; the rest transpose v
 };
 
-__global__ void rope_kv_kernel(const RopeParams p) {
+constexpr int kRopeVTok = 32;  // tokens per v-transpose block
+
+// Blocks [0, rot_blocks): RoPE of q (into the packed grouped-query layout)
+// and k (into the cache), one thread per rotated pair, the split-k partials
+// summed in order.  Remaining blocks: one block per (canvas, kv head, 32
+// tokens) copies v into the transposed cache through shared memory, so both
+// the reads (along the head dimension) and the writes (along positions) are
+// contiguous.
+__global__ void __launch_bounds__(256) rope_kv_kernel(const RopeParams p) {
   const int half = p.hd / 2;
-  const int heads = p.Hq + p.Hkv;                   // heads that are rotated
-  const long long n_rot = (long long)p.T * heads * half;
-  const long long n_v = (long long)p.T * p.Hkv * half;  // v copied in pairs
   const int row_w = (p.Hq + 2 * p.Hkv) * p.hd;
-  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n_rot + n_v;
-       e += (long long)gridDim.x * blockDim.x) {
-    if (e < n_rot) {
+  if ((int)blockIdx.x < p.rot_blocks) {
+    const int heads = p.Hq + p.Hkv;                   // heads that are rotated
+    const int G = p.Hq / p.Hkv;
+    const long long n_rot = (long long)p.T * heads * half;
+    for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n_rot;
+         e += (long long)p.rot_blocks * blockDim.x) {
       const int i = (int)(e % half);
       const long long r = e / half;
       const int h = (int)(r % heads);
@@ -169,26 +178,36 @@ __global__ void rope_kv_kernel(const RopeParams p) {
       const float o1 = (float)(x1 * cs.x - x2 * cs.y), o2 = (float)(x2 * cs.x + x1 * cs.y);
       uint16_t* dst;
       if (h < p.Hq) {
-        dst = p.q + (long long)t * p.Hq * p.hd + h * p.hd;
+        const int g = h / G, hh = h - g * G;
+        dst = p.q + ((((long long)b * p.Hkv + g) * p.nq + pos_in) * G + hh) * p.hd;
       } else {
         const int g = h - p.Hq;
         dst = p.kc + (((long long)b * p.Hkv + g) * p.c_max + p.L0 + pos_in) * p.hd;
       }
       dst[i] = f32_to_bf16(o1);
       dst[i + half] = f32_to_bf16(o2);
-    } else {
-      const long long e2 = e - n_rot;
-      const int i = (int)(e2 % half);
-      const long long r = e2 / half;
-      const int g = (int)(r % p.Hkv);
-      const int t = (int)(r / p.Hkv);
-      const int b = t / p.nq, pos_in = t - b * p.nq;
-      const float* src = p.qkv + (long long)t * row_w + (p.Hq + p.Hkv + g) * p.hd;
-      uint16_t* dst = p.vc + (((long long)b * p.Hkv + g) * p.c_max + p.L0 + pos_in) * p.hd;
-      float a1 = src[2 * i], a2 = src[2 * i + 1];
-      for (int q = 1; q < p.ks; ++q) { a1 += src[q * p.split_stride + 2 * i]; a2 += src[q * p.split_stride + 2 * i + 1]; }
-      dst[2 * i] = f32_to_bf16(a1);
-      dst[2 * i + 1] = f32_to_bf16(a2);
+    }
+  } else {
+    __shared__ uint16_t tile[kRopeVTok * 256];  // [token][dim], hd <= 256
+    const int tiles_per_seq = (p.nq + kRopeVTok - 1) / kRopeVTok;
+    int blk = (int)blockIdx.x - p.rot_blocks;
+    const int tt = blk % tiles_per_seq;
+    blk /= tiles_per_seq;
+    const int g = blk % p.Hkv, b = blk / p.Hkv;
+    const int pos0 = tt * kRopeVTok;
+    const int ntok = min(kRopeVTok, p.nq - pos0);
+    for (int e = threadIdx.x; e < ntok * p.hd; e += blockDim.x) {
+      const int tok = e / p.hd, dim = e - tok * p.hd;
+      const float* src = p.qkv + (long long)(b * p.nq + pos0 + tok) * row_w + (p.Hq + p.Hkv + g) * p.hd + dim;
+      float a = src[0];
+      for (int q = 1; q < p.ks; ++q) a += src[q * p.split_stride];
+      tile[tok * p.hd + dim] = f32_to_bf16(a);
+    }
+    __syncthreads();
+    uint16_t* dst = p.vc + ((long long)b * p.Hkv + g) * p.hd * p.c_max + p.L0 + pos0;
+    for (int e = threadIdx.x; e < ntok * p.hd; e += blockDim.x) {
+      const int dim = e / ntok, tok = e - dim * ntok;
+      dst[(long long)dim * p.c_max + tok] = tile[tok * p.hd + dim];
     }
   }
 }

@@ -96,7 +96,9 @@ typedef struct dg_sampler_config {
 } dg_sampler_config;
 
 /* Causally encoded context, one K and one V buffer of dg_kv_bytes() each:
-   bf16 [n_layers][batch][n_kv_heads][c_max][head_dim], keys after RoPE.
+   K bf16 [n_layers][batch][n_kv_heads][c_max][head_dim] (keys after RoPE),
+   V bf16 transposed, [n_layers][batch][n_kv_heads][head_dim][c_max].
+   c_max must be a multiple of 8 (16-byte row pitch of the transposed V).
    Positions [0, length) hold the context; a denoising round uses positions
    [length, length + 256) as scratch for the canvas keys, so
    c_max >= length + 256 is required. */
@@ -156,7 +158,8 @@ const char* dg_last_error(void);
 /* Bytes of the weight buffer (bf16; layout private to the library). 0 on a
    bad configuration. */
 size_t dg_weights_bytes(const dg_model_config* cfg);
-/* Bytes of ONE of the two KV buffers (K or V) for `batch` canvases. */
+/* Bytes of ONE of the two KV buffers (K or V) for `batch` canvases; 0 when
+   c_max is not a positive multiple of 8. */
 size_t dg_kv_bytes(const dg_model_config* cfg, int32_t batch, int32_t c_max);
 /* Bytes of the scratch workspace for up to `batch` canvases. */
 size_t dg_workspace_bytes(const dg_model_config* cfg, int32_t batch);
@@ -251,10 +254,12 @@ dg_status dg_profile_stop(dg_ctx* ctx, dg_profile* out);
    initialisation, or a caller that has no CUDA allocator of its own.
 
    Computes the same attention as dg_test_attention (dg_testing.h), with the
-   same argument meaning and layout: q bf16 [B * nq, Hq * hd] (token-major),
-   K/V caches bf16 [B][Hkv][c_max][hd] holding keys [0, L0 + nq), out bf16
-   [B * nq, Hq * hd]; causal as there; splits 1..8 key splits (0 means 1).
-   All four pointers are device memory owned by the caller.  The split-KV partial
+   same argument meaning and layout: q bf16 packed by kv head
+   [B][Hkv][nq][Hq / Hkv][hd], K cache bf16 [B][Hkv][c_max][hd], V cache
+   transposed bf16 [B][Hkv][hd][c_max], both holding keys [0, L0 + nq),
+   c_max a multiple of 8; out bf16 [B * nq, Hq * hd]; causal as there;
+   splits 1..8 key splits (0 means 1).  All four pointers are device memory
+   owned by the caller.  The split-KV partial
    results, which dg_test_attention takes from the caller, live here in one
    fixed array inside the library, DG_ATTN_STATIC_SCRATCH_BYTES long (16 MiB);
    every GPU the library runs on holds its own copy for the life of the

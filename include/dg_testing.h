@@ -35,13 +35,16 @@ dg_status dg_test_grouped_gemm(const uint16_t* d_a, int32_t rows_per_group, int3
                                const uint16_t* d_b, int32_t n_rows, int32_t K, const int32_t* d_off,
                                float* d_d, int32_t bn, int32_t* d_chunk_off, void* stream);
 
-/* The library's attention kernel on its own: q bf16 [B * nq, Hq * hd]
-   (token-major), K/V caches bf16 [B][Hkv][c_max][hd] holding keys
-   [0, L0 + nq), out bf16 [B * nq, Hq * hd].  causal = 0: every query sees
-   all L0 + nq keys; causal = 1: query i sees keys [0, L0 + i].  splits > 0
-   forces that many key splits (0: the library's own choice).  The split
-   partial buffers come from the caller: part_o fp32 [splits * B * Hq * nq * hd]
-   and part_ml fp32 [splits * B * Hq * nq * 2].  Synchronous. */
+/* The library's attention kernel on its own (tcgen05 tensor cores):
+   q bf16 packed by kv head [B][Hkv][nq][G][hd] (G = Hq / Hkv, query head
+   g * G + j is row j of token t's group g), K cache bf16 [B][Hkv][c_max][hd],
+   V cache transposed, bf16 [B][Hkv][hd][c_max], both holding keys
+   [0, L0 + nq); c_max a multiple of 8; out bf16 [B * nq, Hq * hd]
+   (token-major).  causal = 0: every query sees all L0 + nq keys; causal = 1:
+   query i sees keys [0, L0 + i].  splits (1..8; 0 means 1) key splits; for
+   splits > 1 the partial buffers come from the caller: part_o fp32
+   [splits * B * Hq * nq * hd] and part_ml fp32 [splits * B * Hq * nq * 2].
+   head_dim one of 32, 64, 128, 176.  Synchronous. */
 dg_status dg_test_attention(const uint16_t* d_q, const uint16_t* d_k, const uint16_t* d_v, uint16_t* d_out,
                             int32_t B, int32_t nq, int32_t L0, int32_t c_max, int32_t Hq, int32_t Hkv,
                             int32_t hd, int32_t causal, int32_t splits, float* d_part_o,

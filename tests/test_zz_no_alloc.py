@@ -9,31 +9,18 @@ import numpy as np
 import pytest
 import torch
 
+import attn_inputs
 from oracle.model import attention as oracle_attention
 
 pytestmark = pytest.mark.gpu
-
-
-def _inputs(B, nq, L0, Hq, Hkv, hd, seed):
-    rng = np.random.default_rng(seed)
-    c_max = L0 + nq + 3
-    q = torch.from_numpy(rng.standard_normal((B * nq, Hq * hd)).astype(np.float32)).to(torch.bfloat16)
-    k = torch.from_numpy(rng.standard_normal((B, Hkv, c_max, hd)).astype(np.float32)).to(torch.bfloat16)
-    v = torch.from_numpy(rng.standard_normal((B, Hkv, c_max, hd)).astype(np.float32)).to(torch.bfloat16)
-    return q, k, v, c_max
-
-
-def _bound(ref):
-    # one bf16 ulp of the output (2^-7 relative) plus a floor for cancelling sums
-    return 2.0 ** -7 * np.abs(ref) + 2.0 ** -20 * np.abs(ref).max()
 
 
 @pytest.mark.parametrize("B,nq,L0,Hq,Hkv,hd,causal,splits", [
     (1, 256, 1024, 16, 8, 176, 0, 5), (2, 256, 77, 8, 8, 32, 0, 4), (1, 44, 256, 8, 8, 32, 1, 3)])
 def test_static_scratch_matches_caller_scratch(B, nq, L0, Hq, Hkv, hd, causal, splits):
     import discrete_diffusion_moe_b200 as dg
-    q, k, v, c_max = _inputs(B, nq, L0, Hq, Hkv, hd, seed=nq + L0 + hd)
-    dq, dk, dv = q.cuda(), k.cuda(), v.cuda()
+    dev, ref_in = attn_inputs.make(B, nq, L0, Hq, Hkv, hd, seed=nq + L0 + hd, pad=3)
+    dq, dk, dv, c_max = dev["q"], dev["k"], dev["v"], dev["c_max"]
     stream = torch.cuda.current_stream().cuda_stream
     want = torch.zeros(B * nq, Hq * hd, dtype=torch.bfloat16, device="cuda")
     po = torch.zeros(splits * B * Hq * nq * hd, device="cuda")
@@ -41,11 +28,8 @@ def test_static_scratch_matches_caller_scratch(B, nq, L0, Hq, Hkv, hd, causal, s
     dg.check(dg.lib.dg_test_attention(dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), want.data_ptr(), B, nq, L0,
                                       c_max, Hq, Hkv, hd, causal, splits, po.data_ptr(), pml.data_ptr(), stream))
     want_np = want.float().cpu().numpy()
-    qn = q.double().numpy().reshape(B, nq, Hq, hd)
-    kn = k.double().numpy().transpose(0, 2, 1, 3)[:, :L0 + nq]
-    vn = v.double().numpy().transpose(0, 2, 1, 3)[:, :L0 + nq]
-    ref = np.stack([oracle_attention(qn[b], kn[b], vn[b], np.arange(L0, L0 + nq), np.arange(L0 + nq),
-                                     bool(causal)) for b in range(B)]).reshape(B * nq, Hq * hd)
+    ref = np.stack([oracle_attention(ref_in["q"][b], ref_in["k"][b], ref_in["v"][b], np.arange(L0, L0 + nq),
+                                     np.arange(L0 + nq), bool(causal)) for b in range(B)]).reshape(B * nq, Hq * hd)
     for call in range(2):
         out = torch.full((B * nq, Hq * hd), float("nan"), dtype=torch.bfloat16, device="cuda")
         dg.check(dg.lib.dg_attention_static_scratch(dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), out.data_ptr(),
@@ -53,17 +37,19 @@ def test_static_scratch_matches_caller_scratch(B, nq, L0, Hq, Hkv, hd, causal, s
         got = out.float().cpu().numpy()
         assert np.all(np.isfinite(got)), call
         diff = np.abs(got - want_np)
-        assert np.all(diff <= _bound(want_np)), (call, float((diff / np.maximum(_bound(want_np), 1e-30)).max()))
+        bw = attn_inputs.bound(want_np, L0 + nq)
+        assert np.all(diff <= bw), (call, float((diff / np.maximum(bw, 1e-30)).max()))
         err = np.abs(got - ref)
-        assert np.all(err <= _bound(ref)), (call, float((err / np.maximum(_bound(ref), 1e-30)).max()))
+        br = attn_inputs.bound(ref, L0 + nq)
+        assert np.all(err <= br), (call, float((err / np.maximum(br, 1e-30)).max()))
 
 
 def test_static_scratch_rejects_requests_beyond_its_array():
     import discrete_diffusion_moe_b200 as dg
     B, nq, L0, Hq, Hkv, hd, splits = 4, 256, 64, 16, 8, 176, 8   # 8*4*16*256*178*4 B > 16 MiB
     assert splits * B * Hq * nq * (hd + 2) * 4 > dg.DG_ATTN_STATIC_SCRATCH_BYTES
-    q, k, v, c_max = _inputs(B, nq, L0, Hq, Hkv, hd, seed=7)
-    dq, dk, dv = q.cuda(), k.cuda(), v.cuda()
+    dev, _ = attn_inputs.make(B, nq, L0, Hq, Hkv, hd, seed=7)
+    dq, dk, dv, c_max = dev["q"], dev["k"], dev["v"], dev["c_max"]
     out = torch.zeros(B * nq, Hq * hd, dtype=torch.bfloat16, device="cuda")
     rc = dg.lib.dg_attention_static_scratch(dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), out.data_ptr(), B, nq,
                                             L0, c_max, Hq, Hkv, hd, 0, splits,
