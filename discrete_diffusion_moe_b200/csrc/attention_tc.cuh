@@ -18,9 +18,12 @@
 //                 O += P_hi V + P_lo V  (M 128, N hd, K 64)    -> TMEM cols [64, 64 + hd)
 //               S of tile j + 1 is issued as soon as S of tile j has been read,
 //               before P V of tile j, so the next scores overlap the softmax.
-//   warps 2..5  softmax, one thread per query row (tensor-memory lane): read
-//               its 64 scores, online max / sum in the exp2 domain, rescale its
-//               row of O in tensor memory when the max grew, write P split
+//   warps 2..9  softmax, two threads per query row (tensor-memory lane), each
+//               taking 32 of the tile's 64 scores; the pair exchanges its
+//               partial maxima through shared memory (bounded mbarrier wait),
+//               keeps an online max / sum in the exp2 domain, rescales its
+//               half of the row of O in tensor memory when the reference max
+//               moved, writes P split
 //               into a bf16 high part and a bf16 residual (P = P_hi + P_lo,
 //               about 16 significant bits for the P V product) into shared
 //               memory in the 128-byte-swizzled K-major layout the MMA reads;
@@ -45,9 +48,10 @@ struct AttnTcParams {
   int* err;
 };
 
-constexpr int kAttnThreads = 192;
+constexpr int kAttnThreads = 320;
 constexpr int kAttnKeys = 64;   // keys per tile
 constexpr int kAttnRows = 128;  // packed query rows per CTA
+constexpr float kAttnLazyLog2 = 8.f;  // reference-max slack (log2 units)
 
 template <int HD>
 struct AttnTcShape {
@@ -56,7 +60,7 @@ struct AttnTcShape {
   static constexpr uint32_t K_BYTES = NA * kAttnKeys * 128;
   static constexpr uint32_t V_BYTES = HD * 128;      // hd rows x 64 keys
   static constexpr uint32_t P_BYTES = kAttnRows * 128;
-  static constexpr size_t SMEM = 1024 + Q_BYTES + 2 * (K_BYTES + V_BYTES) + 2 * P_BYTES + 16 * 8;
+  static constexpr size_t SMEM = 1024 + Q_BYTES + 2 * (K_BYTES + V_BYTES) + 2 * P_BYTES + 16 * 8 + 6 * 128 * 4;
   static constexpr uint32_t TMEM_COLS = (64 + HD) <= 128 ? 128 : 256;
 };
 
@@ -72,6 +76,52 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) 
       : "memory");
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// 32 lanes x 32 consecutive fp32 columns in one load and one wait.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+#define DG_R8(i) "=r"(r[i]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3]), "=r"(r[i + 4]), "=r"(r[i + 5]), "=r"(r[i + 6]), "=r"(r[i + 7])
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,"
+      "%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : DG_R8(0), DG_R8(8), DG_R8(16), DG_R8(24)
+      : "r"(taddr));
+#undef DG_R8
+#define DG_W8(i) "+r"(r[i]), "+r"(r[i + 1]), "+r"(r[i + 2]), "+r"(r[i + 3]), "+r"(r[i + 4]), "+r"(r[i + 5]), "+r"(r[i + 6]), "+r"(r[i + 7])
+  asm volatile("tcgen05.wait::ld.sync.aligned;" : DG_W8(0), DG_W8(8), DG_W8(16), DG_W8(24) : : "memory");
+#undef DG_W8
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 2^x on the special-function unit (PTX ex2.approx.ftz; 2^-inf = 0).
+__device__ __forceinline__ float ex2_fast(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// 32 lanes x 64 consecutive fp32 columns in one load and one wait (the wait
+// names every destination register so no use is scheduled before it).
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
+  uint32_t r[64];
+#define DG_R8(i) "=r"(r[i]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3]), "=r"(r[i + 4]), "=r"(r[i + 5]), "=r"(r[i + 6]), "=r"(r[i + 7])
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,"
+      "%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,"
+      "%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];"
+      : DG_R8(0), DG_R8(8), DG_R8(16), DG_R8(24), DG_R8(32), DG_R8(40), DG_R8(48), DG_R8(56)
+      : "r"(taddr));
+#undef DG_R8
+#define DG_W8(i) "+r"(r[i]), "+r"(r[i + 1]), "+r"(r[i + 2]), "+r"(r[i + 3]), "+r"(r[i + 4]), "+r"(r[i + 5]), "+r"(r[i + 6]), "+r"(r[i + 7])
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : DG_W8(0), DG_W8(8), DG_W8(16), DG_W8(24), DG_W8(32), DG_W8(40), DG_W8(48), DG_W8(56)
+               :
+               : "memory");
+#undef DG_W8
+#pragma unroll
+  for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
+}
 
 // tmQ: packed queries [B * Hkv * nq * G rows, hd], box 64 x 128
 // tmK: keys [B * Hkv * c_max rows, hd], box 64 x 64
@@ -96,7 +146,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* p_full = bars + 7;
   uint64_t* pv_done = bars + 8;
   uint64_t* drain = bars + 9;
-  uint32_t* tmem_slot = (uint32_t*)(bars + 10);
+  uint64_t* pair_bar = bars + 10;  // [4] per tensor-memory lane quarter: the two halves of a row
+  uint32_t* tmem_slot = (uint32_t*)(bars + 14);
+  float* xchg = (float*)(bars + 16);  // [2 tile parities][2 halves][128 rows] maxima, then [2][128] sums
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.Hq / p.Hkv;
@@ -122,8 +174,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(smem_u32(&kv_empty[s]), 1);
     }
     mbar_init(smem_u32(s_full), 1);
-    mbar_init(smem_u32(s_free), 128);
-    mbar_init(smem_u32(p_full), 128);
+    mbar_init(smem_u32(s_free), 256);
+    mbar_init(smem_u32(p_full), 256);
+    for (int q = 0; q < 4; ++q) mbar_init(smem_u32(&pair_bar[q]), 64);
     mbar_init(smem_u32(pv_done), 1);
     mbar_init(smem_u32(drain), 1);
     fence_mbar_init();
@@ -208,61 +261,80 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_wait(smem_u32(drain), 0, p.err);
     }
   } else {
-    // ---------------- softmax + epilogue (warps 2..5) ----------------
+    // ---------------- softmax + epilogue (warps 2..9) ----------------
     const int quarter = warp & 3;
-    const int row = quarter * 32 + lane;  // tensor-memory lane = query row of the tile
+    const int half = (warp - 2) >> 2;      // which 32 of the tile's 64 keys
+    const int row = quarter * 32 + lane;   // tensor-memory lane = query row of the tile
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const int r = r0 + row;
     const int t_in = (r < rows_total ? r : rows_total - 1) / G;  // token within the pass
     const int lim = p.causal ? min(kv_len - 1, p.L0 + t_in) : kv_len - 1;
-    float m = -INFINITY, l = 0.f;
+    const float scale = p.scale_log2;
+    float m = -INFINITY, l = 0.f;  // reference max (scaled, log2 units) and this half's sum
     bool ok = true;
     uint8_t* p_hi = sP;
     uint8_t* p_lo = sP + S::P_BYTES;
     const uint32_t prow = (uint32_t)row * 128;
+    const uint32_t pb = smem_u32(&pair_bar[quarter]);
+    constexpr int NCH = HD / 16;
+    const int oc0 = half ? (NCH + 1) / 2 : 0, oc1 = half ? NCH : (NCH + 1) / 2;  // this half's O chunks
     // waits are made warp-uniform: tensor-memory loads and stores are
     // warp-collective and must never run in a diverged warp
-    auto wait_all = [&](uint64_t* bar, uint32_t parity) {
-      return __all_sync(0xffffffffu, mbar_wait(smem_u32(bar), parity, p.err)) != 0;
+    auto wait_all = [&](uint32_t bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, p.err)) != 0;
     };
     for (int i = 0; i < n_tiles && ok; ++i) {
-      if (!wait_all(s_full, i & 1)) { ok = false; break; }
+      if (!wait_all(smem_u32(s_full), i & 1)) { ok = false; break; }
       tc_fence_after();
-      float sv[kAttnKeys];
-#pragma unroll
-      for (int c = 0; c < kAttnKeys / 16; ++c) {
-        float v[16];
-        tmem_ld16(t_s + lane_off + c * 16, v);
-#pragma unroll
-        for (int e = 0; e < 16; ++e) sv[c * 16 + e] = v[e];
-      }
+      float sv[32];
+      tmem_ld32(t_s + lane_off + half * 32, sv);
       tc_fence_before();
       mbar_arrive(smem_u32(s_free));
-      const int key0 = (kt0 + i) * kAttnKeys;
-      float mx = -INFINITY;
+      const int key0 = (kt0 + i) * kAttnKeys + half * 32;
+      // raw maximum of this half (scale > 0 commutes with max); mask only a
+      // tile that reaches past the row's last visible key
+      float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      if (key0 + 31 <= lim) {
 #pragma unroll
-      for (int c = 0; c < kAttnKeys; ++c) {
-        const float v = key0 + c <= lim ? sv[c] * p.scale_log2 : -INFINITY;
-        sv[c] = v;
-        mx = fmaxf(mx, v);
+        for (int c = 0; c < 32; ++c) mq[c & 3] = fmaxf(mq[c & 3], sv[c]);
+      } else {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          sv[c] = key0 + c <= lim ? sv[c] : -INFINITY;
+          mq[c & 3] = fmaxf(mq[c & 3], sv[c]);
+        }
       }
-      const float m_new = fmaxf(m, mx);
-      const float alpha = (m_new == -INFINITY) ? 1.f : exp2f(m - m_new);
-      float sum = 0.f;
+      // exchange the halves' maxima (double-buffered by tile parity)
+      float* xm = xchg + (i & 1) * 256;
+      xm[half * 128 + row] = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
+      mbar_arrive(pb);
+      if (!wait_all(pb, i & 1)) { ok = false; break; }
+      const float raw = fmaxf(xm[row], xm[128 + row]);
+      const float mx = raw * scale;  // -inf stays -inf
+      // The reference max only moves when the tile's max exceeds it by more
+      // than 2^8: the exponentials stay <= 256 (the same 16-bit P precision,
+      // fp32 sums), and O is rescaled rarely instead of on nearly every tile.
+      // The final normalisation divides by the sum taken against the same
+      // reference, so the result is unchanged.
+      const bool move = mx > m + kAttnLazyLog2 || (m == -INFINITY && mx != -INFINITY);
+      const float m_new = move ? mx : m;
+      const float alpha = (move && m != -INFINITY) ? ex2_fast(m - m_new) : 1.f;
+      const float nref = m_new == -INFINITY ? 0.f : -m_new;
+      float sq[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < kAttnKeys; ++c) {
-        const float pv = (m_new == -INFINITY) ? 0.f : exp2f(sv[c] - m_new);
+      for (int c = 0; c < 32; ++c) {
+        const float pv = ex2_fast(fmaf(sv[c], scale, nref));  // masked: 2^-inf = 0
         sv[c] = pv;
-        sum += pv;
+        sq[c & 3] += pv;
       }
-      l = l * alpha + sum;
+      l = l * alpha + ((sq[0] + sq[1]) + (sq[2] + sq[3]));
       m = m_new;
       // P of the previous tile has been consumed and O is up to date
       if (i > 0) {
-        if (!wait_all(pv_done, (i - 1) & 1)) { ok = false; break; }
+        if (!wait_all(smem_u32(pv_done), (i - 1) & 1)) { ok = false; break; }
         tc_fence_after();
         if (__any_sync(0xffffffffu, alpha != 1.f)) {
-          for (int c = 0; c < HD / 16; ++c) {
+          for (int c = oc0; c < oc1; ++c) {
             float v[16];
             tmem_ld16(t_o + lane_off + c * 16, v);
 #pragma unroll
@@ -274,13 +346,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       // P_hi / P_lo rows into the swizzled K-major operand tiles
 #pragma unroll
-      for (int ch = 0; ch < kAttnKeys / 8; ++ch) {
+      for (int cc = 0; cc < 4; ++cc) {
+        const int ch = half * 4 + cc;
         uint32_t hi[4], lo[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float a0 = sv[ch * 8 + 2 * e], a1 = sv[ch * 8 + 2 * e + 1];
+          const float a0 = sv[cc * 8 + 2 * e], a1 = sv[cc * 8 + 2 * e + 1];
           hi[e] = pack_bf16x2(a0, a1);
-          lo[e] = pack_bf16x2(a0 - bf16_to_f32(hi[e] & 0xFFFF), a1 - bf16_to_f32(hi[e] >> 16));
+          lo[e] = pack_bf16x2(a0 - __uint_as_float(hi[e] << 16), a1 - __uint_as_float(hi[e] & 0xFFFF0000u));
         }
         const uint32_t off = prow + (((uint32_t)ch ^ ((uint32_t)row & 7)) << 4);
         *reinterpret_cast<uint4*>(p_hi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
@@ -290,14 +363,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       tc_fence_before();
       mbar_arrive(smem_u32(p_full));
     }
-    if (ok && n_tiles > 0) ok = wait_all(pv_done, (n_tiles - 1) & 1);
+    if (ok && n_tiles > 0) ok = wait_all(smem_u32(pv_done), (n_tiles - 1) & 1);
     tc_fence_after();
-    const bool have = ok && n_tiles > 0;  // uniform across the warp
+    // total sum of the row: both halves used the same reference max
+    float* xl = xchg + 512;
+    xl[half * 128 + row] = l;
+    mbar_arrive(pb);
+    const bool have = ok && n_tiles > 0 && wait_all(pb, n_tiles & 1);  // uniform across the warp
+    const float l_row = have ? xl[row] + xl[128 + row] : 0.f;
     const bool valid = r < rows_total;
     const int h = g * G + (valid ? r % G : 0);
-    const float inv = (have && l > 0.f) ? 1.f / l : 0.f;
+    const float inv = (have && l_row > 0.f) ? 1.f / l_row : 0.f;
     const long long prow_g = (((long long)split * p.B + b) * p.Hq + h) * p.nq + t_in;
-    for (int c = 0; c < HD / 16; ++c) {
+    for (int c = oc0; c < oc1; ++c) {
       float v[16];
       if (have) {
         tmem_ld16(t_o + lane_off + c * 16, v);
@@ -320,9 +398,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           *reinterpret_cast<float4*>(dst + 4 * e) = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
       }
     }
-    if (valid && p.splits > 1) {
+    if (valid && p.splits > 1 && half == 0) {
       p.part_ml[prow_g * 2] = have ? m : -INFINITY;
-      p.part_ml[prow_g * 2 + 1] = have ? l : 0.f;
+      p.part_ml[prow_g * 2 + 1] = have ? l_row : 0.f;
     }
   }
 
