@@ -660,11 +660,10 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
       DG_TRY(run_gemm(ta, tb, p, e, c->num_sms, st, &c->n_launch));
     }
     {
-      const int rot_blocks = std::min(4096, (T * (Hq + Hkv) * hd / 2 + 255) / 256);
       const int v_blocks = B * Hkv * ((nq + kRopeVTok - 1) / kRopeVTok);
       RopeParams rp{c->at<float>(L.qkv), ks_qkv, (long long)T * qkv_rows, c->at<double2>(L.rope),
-                    c->at<uint16_t>(L.q), kc, vc, T, nq, L0, kv->c_max, Hq, Hkv, hd, rot_blocks};
-      rope_kv_kernel<<<rot_blocks + v_blocks, 256, 0, st>>>(rp);
+                    c->at<uint16_t>(L.q), kc, vc, T, nq, L0, kv->c_max, Hq, Hkv, hd};
+      rope_kv_kernel<<<T + v_blocks, 256, 0, st>>>(rp);
       CNT(c);
     }
     {

@@ -145,35 +145,35 @@ struct RopeParams {
   uint16_t* kc;       // layer base of K cache   [B][Hkv][c_max][hd]
   uint16_t* vc;       // layer base of V^T cache [B][Hkv][hd][c_max]
   int T, nq, L0, c_max, Hq, Hkv, hd;
-  int rot_blocks;     // blocks [0, rot_blocks) rotate q and k; the rest transpose v
 };
 
-constexpr int kRopeVTok = 32;  // tokens per v-transpose block
+constexpr int kRopeVTok = 16;  // tokens per v-transpose block
 
-// Blocks [0, rot_blocks): RoPE of q (into the packed grouped-query layout)
-// and k (into the cache), one thread per rotated pair, the split-k partials
-// summed in order.  Remaining blocks: one block per (canvas, kv head, 32
-// tokens) copies v into the transposed cache through shared memory, so both
-// the reads (along the head dimension) and the writes (along positions) are
-// contiguous.
+// Blocks [0, T): one block per token rotates its q heads (into the packed
+// grouped-query layout) and k heads (into the cache), one thread per rotated
+// pair, the split-k partials summed in order.  Blocks [T, ...): one block per
+// (canvas, kv head, 16 tokens) copies v into the transposed cache through
+// shared memory, so both the reads (along the head dimension) and the writes
+// (along positions) are contiguous; every thread issues the loads of several
+// elements before it uses them, so the block is not a chain of dependent
+// loads.
 __global__ void __launch_bounds__(256) rope_kv_kernel(const RopeParams p) {
   const int half = p.hd / 2;
   const int row_w = (p.Hq + 2 * p.Hkv) * p.hd;
-  if ((int)blockIdx.x < p.rot_blocks) {
-    const int heads = p.Hq + p.Hkv;                   // heads that are rotated
+  if ((int)blockIdx.x < p.T) {
+    const int t = blockIdx.x;
     const int G = p.Hq / p.Hkv;
-    const long long n_rot = (long long)p.T * heads * half;
-    for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n_rot;
-         e += (long long)p.rot_blocks * blockDim.x) {
-      const int i = (int)(e % half);
-      const long long r = e / half;
-      const int h = (int)(r % heads);
-      const int t = (int)(r / heads);
-      const int b = t / p.nq, pos_in = t - b * p.nq;
-      const double2 cs = p.tab[pos_in * half + i];
-      const float* src = p.qkv + (long long)t * row_w + h * p.hd;
-      float a1 = src[i], a2 = src[i + half];
-      for (int q = 1; q < p.ks; ++q) { a1 += src[q * p.split_stride + i]; a2 += src[q * p.split_stride + i + half]; }
+    const int b = t / p.nq, pos_in = t - b * p.nq;
+    const int n_pairs = (p.Hq + p.Hkv) * half;
+    const float* row = p.qkv + (long long)t * row_w;
+    const double2* tab = p.tab + (long long)pos_in * half;
+#pragma unroll 2
+    for (int j = threadIdx.x; j < n_pairs; j += blockDim.x) {
+      const int h = j / half, i = j - h * half;
+      const float* src = row + h * p.hd + i;
+      float a1 = src[0], a2 = src[half];
+      for (int q = 1; q < p.ks; ++q) { a1 += src[q * p.split_stride]; a2 += src[q * p.split_stride + half]; }
+      const double2 cs = tab[i];
       const double x1 = a1, x2 = a2;
       const float o1 = (float)(x1 * cs.x - x2 * cs.y), o2 = (float)(x2 * cs.x + x1 * cs.y);
       uint16_t* dst;
@@ -190,22 +190,37 @@ __global__ void __launch_bounds__(256) rope_kv_kernel(const RopeParams p) {
   } else {
     __shared__ uint16_t tile[kRopeVTok * 256];  // [token][dim], hd <= 256
     const int tiles_per_seq = (p.nq + kRopeVTok - 1) / kRopeVTok;
-    int blk = (int)blockIdx.x - p.rot_blocks;
+    int blk = (int)blockIdx.x - p.T;
     const int tt = blk % tiles_per_seq;
     blk /= tiles_per_seq;
     const int g = blk % p.Hkv, b = blk / p.Hkv;
     const int pos0 = tt * kRopeVTok;
     const int ntok = min(kRopeVTok, p.nq - pos0);
-    for (int e = threadIdx.x; e < ntok * p.hd; e += blockDim.x) {
+    const int n = ntok * p.hd;
+    const float* base = p.qkv + (long long)(b * p.nq + pos0) * row_w + (p.Hq + p.Hkv + g) * p.hd;
+    constexpr int kPer = (kRopeVTok * 256 + 255) / 256;  // elements per thread at most
+    float a[kPer];
+    int off[kPer];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int e = threadIdx.x + u * 256;
       const int tok = e / p.hd, dim = e - tok * p.hd;
-      const float* src = p.qkv + (long long)(b * p.nq + pos0 + tok) * row_w + (p.Hq + p.Hkv + g) * p.hd + dim;
-      float a = src[0];
-      for (int q = 1; q < p.ks; ++q) a += src[q * p.split_stride];
-      tile[tok * p.hd + dim] = f32_to_bf16(a);
+      off[u] = tok * row_w + dim;
+      a[u] = e < n ? base[off[u]] : 0.f;
+    }
+    for (int q = 1; q < p.ks; ++q) {
+#pragma unroll
+      for (int u = 0; u < kPer; ++u)
+        if (threadIdx.x + u * 256 < n) a[u] += base[q * p.split_stride + off[u]];
+    }
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int e = threadIdx.x + u * 256;
+      if (e < n) tile[e] = f32_to_bf16(a[u]);  // e = tok * hd + dim
     }
     __syncthreads();
     uint16_t* dst = p.vc + ((long long)b * p.Hkv + g) * p.hd * p.c_max + p.L0 + pos0;
-    for (int e = threadIdx.x; e < ntok * p.hd; e += blockDim.x) {
+    for (int e = threadIdx.x; e < n; e += blockDim.x) {
       const int dim = e / ntok, tok = e - dim * ntok;
       dst[(long long)dim * p.c_max + tok] = tile[tok * p.hd + dim];
     }
