@@ -65,7 +65,12 @@ struct EpiStoreT {
 
 // Grouped gate/up projection with SwiGLU.  The expert's [2 f, d] weight has
 // gate row j at 2j and up row j at 2j+1, so the pair sits in adjacent lanes:
-// h[slot, j] = bf16(silu(gate) * up) with silu(z) = z / (1 + e^-z).
+// h[slot, j] = bf16(silu(gate) * up) with silu(z) = z / (1 + e^-z).  The two
+// lanes of a pair exchange their 16 values, then the even lane finishes the
+// chunk's first 8 columns and the odd lane the last 8: every lane works, and
+// all 8 activations are computed before any store, so the exponentials and
+// divisions of different columns overlap instead of running one column at a
+// time behind a branch.
 struct EpiSwiGLU {
   uint16_t* h;   // [rows, f_dim] bf16, rows in expert (permuted) order
   int f_dim;
@@ -75,15 +80,22 @@ struct EpiSwiGLU {
   __device__ __forceinline__ void chunk(const GemmJob& j, int row, int c0, const float (&v)[16],
                                         State&) const {
     const int feat = (j.m_tile * 128 + row) >> 1;
+    const bool odd = (row & 1) != 0;
+    float o[16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const float other = __shfl_xor_sync(0xffffffffu, v[i], 1);
-      const int n = c0 + i;
-      if ((row & 1) == 0 && row < j.m_valid && n < j.n_valid) {
-        const float g = v[i], u = other;
-        const float act = g / (1.0f + __expf(-g));
-        h[(long long)(j.n0 + n) * f_dim + feat] = f32_to_bf16(act * u);
-      }
+    for (int i = 0; i < 16; ++i) o[i] = __shfl_xor_sync(0xffffffffu, v[i], 1);
+    uint16_t r[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const float g = odd ? o[q + 8] : v[q];
+      const float u = odd ? v[q + 8] : o[q];
+      r[q] = f32_to_bf16(__fdividef(g, 1.0f + __expf(-g)) * u);
+    }
+    if (row < j.m_valid) {
+      const int nb = c0 + (odd ? 8 : 0);
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        if (nb + q < j.n_valid) h[(long long)(j.n0 + nb + q) * f_dim + feat] = r[q];
     }
   }
 };
