@@ -274,6 +274,7 @@ def main():
     ap.add_argument("--workload", default="full", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-decode-loop", action="store_true")
     args = ap.parse_args()
     wl = WORKLOADS[args.workload]
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -369,6 +370,35 @@ def main():
     ridx = out.route_idx.cpu()
     distinct = [int(torch.unique(ridx[l]).numel()) for l in range(c["n_layers"])]
 
+    # ---- the decode loop (dg_decode_block): 4 blocks of up to 48 steps after a
+    # prompt of the workload's context length; block appends are included, the
+    # prompt encode is not ------------------------------------------------------------
+    loop = None
+    if not args.no_decode_loop and B == 1:
+        n_blocks = 4
+        kv_l = dg.KVCache(cfg, 1, ctx + n_blocks * CANVAS)
+        model.encode(kv_l, ctx_tok[:1].contiguous())
+        cv_l = dg.Canvas(cfg, 1)
+        toks = torch.zeros(1, CANVAS, dtype=torch.int32, device="cuda")
+        g0 = torch.cuda.Event(enable_timing=True)
+        g1 = torch.cuda.Event(enable_timing=True)
+        barrier()
+        g0.record(stream)
+        passes = 0
+        for blk in range(n_blocks):
+            st_, _ = model.decode_block(kv_l, cv_l, blk, samp, toks)
+            passes += st_[0]
+        g1.record(stream)
+        barrier()
+        model.check_device()
+        ms_l = g0.elapsed_time(g1)
+        loop = {"blocks": n_blocks, "max_steps_per_block": MAX_STEPS, "output_tokens": n_blocks * CANVAS,
+                "denoise_passes": passes, "tokens_per_pass": n_blocks * CANVAS / passes, "ms": ms_l,
+                "output_tok_per_s": n_blocks * CANVAS / (ms_l / 1000.0),
+                "note": "random-init weights: predictions stay near uniform, so no position locks and the "
+                        "entropy stop never fires; every block runs its full step budget"}
+        del kv_l
+
     # ---- end to end through the public API with host buffers -------------------------
     e2e = None
     if not args.no_e2e:
@@ -437,6 +467,7 @@ def main():
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (random-init weights, random tokens)",
             "config": workload_config(args, wl, world),
+            "decode_loop": loop,
             "output_tok_per_s": {"at_48_rounds_per_block": value * CANVAS / MAX_STEPS,
                                  "projected_at_12_rounds_per_block": value * CANVAS / 12},
             "step_roofline": {"flops": flops, "bytes": nbytes, "t_ms": 1000 * t_roof,

@@ -34,9 +34,15 @@ struct EpiStoreT {
     float* base = out + (long long)j.ks * split_stride + f;
     const int nv = j.n_valid - c0;  // valid columns in this chunk (may exceed 16)
     if (mode == 0) {
+      // streaming stores (evict-first): the partial products are read once
+      if (nv >= 16) {
 #pragma unroll
-      for (int i = 0; i < 16; ++i)
-        if (i < nv) base[(long long)(j.n0 + c0 + i) * ld] = v[i];
+        for (int i = 0; i < 16; ++i) __stcs(base + (long long)(j.n0 + c0 + i) * ld, v[i]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          if (i < nv) __stcs(base + (long long)(j.n0 + c0 + i) * ld, v[i]);
+      }
     } else if (mode == 1) {
       // all loads first: the 16 read-modify-writes then overlap their latency
       float old[16];
@@ -116,9 +122,14 @@ struct EpiDown {
     float w[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) w[i] = i < nv ? __ldg(w_slot + j.n0 + c0 + i) : 0.f;
+    if (nv >= 16) {
 #pragma unroll
-    for (int i = 0; i < 16; ++i)
-      if (i < nv) y[(long long)(j.n0 + c0 + i) * d + f] = w[i] * v[i];
+      for (int i = 0; i < 16; ++i) __stcs(y + (long long)(j.n0 + c0 + i) * d + f, w[i] * v[i]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        if (i < nv) __stcs(y + (long long)(j.n0 + c0 + i) * d + f, w[i] * v[i]);
+    }
   }
 };
 

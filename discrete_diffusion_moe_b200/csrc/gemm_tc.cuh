@@ -270,10 +270,21 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
         typename Epi::State st;
         epi.begin(j, row, st);
         const int nch = (j.n_valid + 15) >> 4;
+        // the load of chunk c + 1 is in flight while chunk c is processed
+        uint32_t ra[16], rb[16];
+        tmem_ld16_nowait(t0, ra);
+        tmem_wait_ld16(ra);
         for (int c = 0; c < nch; ++c) {
+          if (c + 1 < nch) tmem_ld16_nowait(t0 + (c + 1) * 16, rb);
           float v[16];
-          tmem_ld16(t0 + c * 16, v);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(ra[i]);
           epi.chunk(j, row, c * 16, v, st);
+          if (c + 1 < nch) {
+            tmem_wait_ld16(rb);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) ra[i] = rb[i];
+          }
         }
         epi.end(j, row, st);
         tc_fence_before();
