@@ -91,6 +91,39 @@ def _top2_gap(v):
     return float(top[1] - top[0])
 
 
+def update_canvas(cfg: ModelConfig, sc: smp.SamplerConfig, state: CanvasState, block: int, step: int,
+                  H, pmax, amax, samp, e_new=None):
+    """a9 on the per-position statistics of one step (H, pmax, argmax and
+    sample [B, N]): the mean entropy, the stop flag, the lock mask and the next
+    canvas (locked positions keep their sample, the others get the re-noise
+    draw; a stopping or last-budget canvas becomes its argmax and is frozen);
+    `state` is updated in place.  Returns (meanH, stop, final, lock)."""
+    B, N = state.tokens.shape
+    V = cfg.vocab
+    meanH = H.mean(axis=1)
+    stop = np.zeros(B, bool)
+    final = np.zeros(B, bool)
+    lock = np.zeros((B, N), bool)
+    for b in range(B):
+        lock[b] = smp.lock_mask(H[b], pmax[b], sc.lock_policy, sc.lock_threshold)
+        if state.done[b]:
+            continue
+        prev = state.prev_argmax[b] if step > 0 else None
+        stop[b] = smp.stop_flag(meanH[b], sc.stop_entropy, sc.stop_require_stable_argmax, step,
+                                amax[b], prev)
+        final[b] = stop[b] or step == sc.max_steps - 1
+        if final[b]:
+            state.tokens[b] = amax[b]
+            state.done[b] = True
+        else:
+            noise = smp.renoise_tokens(sc.seed, b, block, step, N, V)
+            state.tokens[b] = np.where(lock[b], samp[b], noise)
+        state.prev_argmax[b] = amax[b]
+        if cfg.self_cond and e_new is not None:
+            state.sc[b] = e_new[b]
+    return meanH, stop, final, lock
+
+
 def denoise_step(cfg: ModelConfig, W: Weights, kv: KVCache, state: CanvasState,
                  sc: smp.SamplerConfig, block: int, step: int, keep_logits: bool = True,
                  record_routing: bool = False) -> StepOutput:
@@ -133,27 +166,7 @@ def denoise_step(cfg: ModelConfig, W: Weights, kv: KVCache, state: CanvasState,
         e_new = smp.expected_embedding(probs.reshape(B * N, V), W).reshape(B, N, d)
 
     # a9: stop, lock and the next canvas
-    meanH = H.mean(axis=1)
-    stop = np.zeros(B, bool)
-    final = np.zeros(B, bool)
-    lock = np.zeros((B, N), bool)
-    for b in range(B):
-        lock[b] = smp.lock_mask(H[b], pmax[b], sc.lock_policy, sc.lock_threshold)
-        if state.done[b]:
-            continue
-        prev = state.prev_argmax[b] if step > 0 else None
-        stop[b] = smp.stop_flag(meanH[b], sc.stop_entropy, sc.stop_require_stable_argmax, step,
-                                amax[b], prev)
-        final[b] = stop[b] or step == sc.max_steps - 1
-        if final[b]:
-            state.tokens[b] = amax[b]
-            state.done[b] = True
-        else:
-            noise = smp.renoise_tokens(sc.seed, b, block, step, N, V)
-            state.tokens[b] = np.where(lock[b], samp[b], noise)
-        state.prev_argmax[b] = amax[b]
-        if cfg.self_cond:
-            state.sc[b] = e_new[b]
+    meanH, stop, final, lock = update_canvas(cfg, sc, state, block, step, H, pmax, amax, samp, e_new)
 
     return StepOutput(logits=logits if keep_logits else None, argmax=amax, sample=samp, entropy=H,
                       pmax=pmax, mean_entropy=meanH, stop=stop, final=final, lock=lock,

@@ -248,6 +248,41 @@ def moe_ffn(h, layer, top_k):
     return out, idx, w, route_margin(logits, top_k), logits
 
 
+def layer_forward(cfg: ModelConfig, lw: dict, x, kv_k, kv_v, L0: int, causal: bool, append: bool):
+    """One transformer layer on the residual stream x [B, n, d] (fp32 values)
+    whose tokens sit at positions L0 .. L0 + n - 1.  kv_k / kv_v are this
+    layer's cached keys (after RoPE) and values [B, C_max, H_kv, hd]; the
+    pass attends to keys [0, L0) from the cache plus its own n keys, which are
+    written to the cache at [L0, L0 + n) when `append`.  Returns the residual
+    stream after the layer and (routing idx, weights, routing margin, router
+    logits)."""
+    c = cfg
+    B, n, d = x.shape
+    pos = np.arange(L0, L0 + n)
+    k_pos = np.arange(0, L0 + n)
+    hd, Hq, Hkv = c.head_dim, c.n_q_heads, c.n_kv_heads
+    h = bf16_round(rmsnorm(x, c.rms_eps))
+    q = h @ lw["wq"].T
+    k = h @ lw["wk"].T
+    v = bf16_round(h @ lw["wv"].T)
+    o = np.empty((B, n, Hq * hd))
+    for b in range(B):
+        qb = bf16_round(rope(q[b].reshape(n, Hq, hd), pos, c.rope_theta))
+        kb = bf16_round(rope(k[b].reshape(n, Hkv, hd), pos, c.rope_theta))
+        vb = v[b].reshape(n, Hkv, hd)
+        k_all = np.concatenate([kv_k[b, :L0].astype(np.float64), kb], axis=0)
+        v_all = np.concatenate([kv_v[b, :L0].astype(np.float64), vb], axis=0)
+        o[b] = bf16_round(attention(qb, k_all, v_all, pos, k_pos, causal)).reshape(n, Hq * hd)
+        if append:
+            kv_k[b, L0:L0 + n] = kb
+            kv_v[b, L0:L0 + n] = vb
+    x = f32_round(x + f32_round(o @ lw["wo"].T))
+    h2 = bf16_round(rmsnorm(x, c.rms_eps)).reshape(B * n, d)
+    m, idx, w, margin, rlog = moe_ffn(h2, lw, c.top_k)
+    x = f32_round(x + m.reshape(B, n, d))
+    return x, (idx.reshape(B, n, -1), w.reshape(B, n, -1), margin.reshape(B, n), rlog.reshape(B, n, -1))
+
+
 def forward_layers(cfg: ModelConfig, W: Weights, x, kv: KVCache, causal: bool, append: bool,
                    record=None):
     """Run all transformer layers on the residual stream x [B, n, d] (fp32
@@ -260,37 +295,13 @@ def forward_layers(cfg: ModelConfig, W: Weights, x, kv: KVCache, causal: bool, a
     kept).  Returns the final residual stream.  `record`, if a list, receives
     per layer (routing idx, weights, routing margin, residual stream after the
     layer, router logits)."""
-    c = cfg
-    B, n, d = x.shape
     L0 = kv.length
-    pos = np.arange(L0, L0 + n)
-    k_pos = np.arange(0, L0 + n)
-    hd, Hq, Hkv = c.head_dim, c.n_q_heads, c.n_kv_heads
+    n = x.shape[1]
     x = f32_round(x)
-    for l in range(c.n_layers):
-        lw = W.layer(l)
-        h = bf16_round(rmsnorm(x, c.rms_eps))
-        q = h @ lw["wq"].T
-        k = h @ lw["wk"].T
-        v = bf16_round(h @ lw["wv"].T)
-        o = np.empty((B, n, Hq * hd))
-        for b in range(B):
-            qb = bf16_round(rope(q[b].reshape(n, Hq, hd), pos, c.rope_theta))
-            kb = bf16_round(rope(k[b].reshape(n, Hkv, hd), pos, c.rope_theta))
-            vb = v[b].reshape(n, Hkv, hd)
-            k_all = np.concatenate([kv.k[l][b, :L0].astype(np.float64), kb], axis=0)
-            v_all = np.concatenate([kv.v[l][b, :L0].astype(np.float64), vb], axis=0)
-            o[b] = bf16_round(attention(qb, k_all, v_all, pos, k_pos, causal)).reshape(n, Hq * hd)
-            if append:
-                kv.k[l][b, L0:L0 + n] = kb
-                kv.v[l][b, L0:L0 + n] = vb
-        x = f32_round(x + f32_round(o @ lw["wo"].T))
-        h2 = bf16_round(rmsnorm(x, c.rms_eps)).reshape(B * n, d)
-        m, idx, w, margin, rlog = moe_ffn(h2, lw, c.top_k)
-        x = f32_round(x + m.reshape(B, n, d))
+    for l in range(cfg.n_layers):
+        x, (idx, w, margin, rlog) = layer_forward(cfg, W.layer(l), x, kv.k[l], kv.v[l], L0, causal, append)
         if record is not None:
-            record.append((idx.reshape(B, n, -1), w.reshape(B, n, -1), margin.reshape(B, n), x.copy(),
-                           rlog.reshape(B, n, -1)))
+            record.append((idx, w, margin, x.copy(), rlog))
     if append:
         kv.length = L0 + n
     return x
