@@ -6,6 +6,7 @@
 #include <math.h>
 #include <stdarg.h>
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <algorithm>
@@ -126,11 +127,17 @@ struct WsLayout {
 constexpr int kRouterSplits = 4;  // split-k of the router product (needs d_model >= 256)
 int router_splits(const dg_model_config&) { return kRouterSplits; }
 
-// Split-k factor of a weight-stationary dense GEMM with m_tiles x n_tiles
-// output tiles: as many k splits as keep the units within one wave.
-int dense_splits(int m_tiles, int n_tiles, int kb, int num_sms) {
-  int ks = num_sms / std::max(1, m_tiles * n_tiles);
-  return std::max(1, std::min({ks, 8, kb / 4}));
+// Token columns per unit of the QKV and output projections: 128 from 256
+// tokens on (two CTAs share an SM, each weight tile is read by two CTAs at the
+// same time, the second time from L2).
+int proj_bn(int T) { return T >= 256 ? 128 : std::min(256, std::max(16, next_pow2(T))); }
+
+// Split-k of the QKV and output projections: enough units for two CTAs per
+// SM, at most 3 (every split is one more fp32 partial its consumer reads).
+int proj_splits(int m_tiles, int T, int kb, int num_sms) {
+  const int n_tiles = (T + proj_bn(T) - 1) / proj_bn(T);
+  const int ks = (2 * num_sms) / std::max(1, m_tiles * n_tiles);
+  return std::max(1, std::min({ks, 3, kb / 4}));
 }
 
 int esum_splits(const dg_model_config& c, int T, int num_sms) {
@@ -166,9 +173,8 @@ WsLayout ws_layout(const dg_model_config& c, int batch, int num_sms) {
     const int qkv_rows = (c.n_q_heads + 2 * c.n_kv_heads) * c.head_dim;
     size_t rq = 0, ro = 0;
     for (int tt = DG_CANVAS; tt <= (int)T; tt += DG_CANVAS) {
-      const int nt = (tt + 255) / 256;
-      rq = std::max(rq, (size_t)dense_splits((qkv_rows + 127) / 128, nt, c.d_model / 64, num_sms) * tt);
-      ro = std::max(ro, (size_t)dense_splits((c.d_model + 127) / 128, nt, (int)hq / 64, num_sms) * tt);
+      rq = std::max(rq, (size_t)proj_splits((qkv_rows + 127) / 128, tt, c.d_model / 64, num_sms) * tt);
+      ro = std::max(ro, (size_t)proj_splits((c.d_model + 127) / 128, tt, (int)hq / 64, num_sms) * tt);
     }
     L.qkv = take(rq * qkv_rows * 4);
     L.opart = take(ro * d * 4);
@@ -631,8 +637,9 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
   }
 
   // split-k of the two dense projections (partials summed by their consumers)
-  const int ks_qkv = dense_splits((qkv_rows + 127) / 128, (T + 255) / 256, d / 64, c->num_sms);
-  const int ks_o = dense_splits((d + 127) / 128, (T + 255) / 256, Hq * hd / 64, c->num_sms);
+  const int dense_bn_x = proj_bn(T);
+  const int ks_qkv = proj_splits((qkv_rows + 127) / 128, T, d / 64, c->num_sms);
+  const int ks_o = proj_splits((d + 127) / 128, T, Hq * hd / 64, c->num_sms);
 
   // attention key splits
   const int splits = attn_splits(B, nq, L0, Hq, Hkv, c->num_sms, L.attn_rows_cap);
@@ -651,7 +658,7 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
       ProfScope ps_(c, DG_PROF_DENSE, st);
       CUtensorMap ta;
       BOperand tb;
-      const int bn = token_bn(T);
+      const int bn = dense_bn_x;
       DG_TRY(make_tmap(&ta, c->wp(W.wqkv), d, qkv_rows, 128));
       DG_TRY(make_bop(&tb, xn, d, L.T_alloc, bn));
       GemmPlan p = dense_plan(d, qkv_rows, T, bn, ks_qkv, err);
@@ -676,7 +683,7 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
       ProfScope ps_(c, DG_PROF_DENSE, st);
       CUtensorMap ta;
       BOperand tb;
-      const int bn = token_bn(T);
+      const int bn = dense_bn_x;
       DG_TRY(make_tmap(&ta, c->wp(W.wo), (long long)Hq * hd, d, 128));
       DG_TRY(make_bop(&tb, c->at<uint16_t>(L.attn), (long long)Hq * hd, L.T_alloc, bn));
       GemmPlan p = dense_plan(Hq * hd, d, T, bn, ks_o, err);
