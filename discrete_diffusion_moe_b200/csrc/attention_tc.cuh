@@ -15,7 +15,8 @@
 //               keys, so keys past it arrive as zeros
 //   warp 1      tensor memory owner and MMA issuer:
 //                 S  = Q K^T            (M 128, N 64, K hd)    -> TMEM cols [0, 64)
-//                 O += P_hi V + P_lo V  (M 128, N hd, K 64)    -> TMEM cols [64, 64 + hd)
+//                 O += P V              (M 128, N hd, K 64)    -> TMEM cols [64, 64 + hd)
+//                                       (P and V in fp16)
 //               S of tile j + 1 is issued as soon as S of tile j has been read,
 //               before P V of tile j, so the next scores overlap the softmax.
 //   warps 2..9  softmax, two threads per query row (tensor-memory lane), each
@@ -23,10 +24,11 @@
 //               partial maxima through shared memory (bounded mbarrier wait),
 //               keeps an online max / sum in the exp2 domain, rescales its
 //               half of the row of O in tensor memory when the reference max
-//               moved, writes P split
-//               into a bf16 high part and a bf16 residual (P = P_hi + P_lo,
-//               about 16 significant bits for the P V product) into shared
-//               memory in the 128-byte-swizzled K-major layout the MMA reads;
+//               moved, writes P in fp16 (11 significant bits; scaled by 2^7
+//               so that the values lie in (0, 2^15])
+//               into shared memory in the 128-byte-swizzled K-major layout the
+//               MMA reads (the V^T cache holds the bf16-rounded values in
+//               fp16, exact above 2^-14, for this product);
 //               finally read O and write the normalised bf16 output or the
 //               split's unnormalised partial (with its max and sum).
 //
@@ -52,6 +54,10 @@ constexpr int kAttnThreads = 320;
 constexpr int kAttnKeys = 64;   // keys per tile
 constexpr int kAttnRows = 128;  // packed query rows per CTA
 constexpr float kAttnLazyLog2 = 8.f;  // reference-max slack (log2 units)
+// P is computed as 2^(s - m + 7): the values lie in (0, 2^15] (below the fp16
+// maximum) and only those below 2^-21 of the reference fall to fp16
+// subnormals.  The row sum carries the same factor, so it cancels.
+constexpr float kAttnPScaleLog2 = 7.f;
 
 template <int HD>
 struct AttnTcShape {
@@ -60,7 +66,7 @@ struct AttnTcShape {
   static constexpr uint32_t K_BYTES = NA * kAttnKeys * 128;
   static constexpr uint32_t V_BYTES = HD * 128;      // hd rows x 64 keys
   static constexpr uint32_t P_BYTES = kAttnRows * 128;
-  static constexpr size_t SMEM = 1024 + Q_BYTES + 2 * (K_BYTES + V_BYTES) + 2 * P_BYTES + 16 * 8 + 6 * 128 * 4;
+  static constexpr size_t SMEM = 1024 + Q_BYTES + 2 * (K_BYTES + V_BYTES) + P_BYTES + 16 * 8 + 6 * 128 * 4;
   static constexpr uint32_t TMEM_COLS = (64 + HD) <= 128 ? 128 : 256;
 };
 
@@ -136,8 +142,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint8_t* sQ = smem;
   uint8_t* sK = sQ + S::Q_BYTES;               // 2 stages
   uint8_t* sV = sK + 2 * S::K_BYTES;           // 2 stages
-  uint8_t* sP = sV + 2 * S::V_BYTES;           // P_hi, P_lo
-  uint64_t* bars = (uint64_t*)(sP + 2 * S::P_BYTES);
+  uint8_t* sP = sV + 2 * S::V_BYTES;           // P (fp16)
+  uint64_t* bars = (uint64_t*)(sP + S::P_BYTES);
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;   // [2]
   uint64_t* kv_empty = bars + 3;  // [2]
@@ -223,7 +229,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (lane == 0 && n_tiles > 0) {
       // ---------------- MMA issuer ----------------
       const uint32_t id_s = idesc_bf16_f32(128, kAttnKeys);
-      const uint32_t id_o = idesc_bf16_f32(128, HD);
+      const uint32_t id_o = idesc_f16_f32(128, HD);
       bool ok = mbar_wait(smem_u32(q_full), 0, p.err);
       auto issue_s = [&](int i) -> bool {
         const int s = i & 1;
@@ -246,14 +252,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (!mbar_wait(smem_u32(p_full), i & 1, p.err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t va = smem_u32(sV + (i & 1) * S::V_BYTES);
+        const uint32_t pa = smem_u32(sP);
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {
-          const uint32_t pa = smem_u32(sP + part * S::P_BYTES);
-#pragma unroll
-          for (int k = 0; k < kAttnKeys / 16; ++k)
-            umma_bf16(t_o, sdesc_k128(pa + k * 32), sdesc_k128(va + k * 32), id_o,
-                      (i > 0 || part > 0 || k > 0) ? 1u : 0u);
-        }
+        for (int k = 0; k < kAttnKeys / 16; ++k)
+          umma_bf16(t_o, sdesc_k128(pa + k * 32), sdesc_k128(va + k * 32), id_o, (i > 0 || k > 0) ? 1u : 0u);
         umma_commit(smem_u32(pv_done));
         umma_commit(smem_u32(&kv_empty[i & 1]));
       }
@@ -272,8 +274,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const float scale = p.scale_log2;
     float m = -INFINITY, l = 0.f;  // reference max (scaled, log2 units) and this half's sum
     bool ok = true;
-    uint8_t* p_hi = sP;
-    uint8_t* p_lo = sP + S::P_BYTES;
+    uint8_t* p_s = sP;
     const uint32_t prow = (uint32_t)row * 128;
     const uint32_t pb = smem_u32(&pair_bar[quarter]);
     constexpr int NCH = HD / 16;
@@ -319,7 +320,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const bool move = mx > m + kAttnLazyLog2 || (m == -INFINITY && mx != -INFINITY);
       const float m_new = move ? mx : m;
       const float alpha = (move && m != -INFINITY) ? ex2_fast(m - m_new) : 1.f;
-      const float nref = m_new == -INFINITY ? 0.f : -m_new;
+      const float nref = m_new == -INFINITY ? 0.f : kAttnPScaleLog2 - m_new;
       float sq[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
@@ -344,20 +345,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           tmem_wait_st();
         }
       }
-      // P_hi / P_lo rows into the swizzled K-major operand tiles
+      // P rows (fp16) into the swizzled K-major operand tile
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
         const int ch = half * 4 + cc;
-        uint32_t hi[4], lo[4];
+        uint32_t hv[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float a0 = sv[cc * 8 + 2 * e], a1 = sv[cc * 8 + 2 * e + 1];
-          hi[e] = pack_bf16x2(a0, a1);
-          lo[e] = pack_bf16x2(a0 - __uint_as_float(hi[e] << 16), a1 - __uint_as_float(hi[e] & 0xFFFF0000u));
-        }
+        for (int e = 0; e < 4; ++e) hv[e] = pack_f16x2(sv[cc * 8 + 2 * e], sv[cc * 8 + 2 * e + 1]);
         const uint32_t off = prow + (((uint32_t)ch ^ ((uint32_t)row & 7)) << 4);
-        *reinterpret_cast<uint4*>(p_hi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4*>(p_lo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        *reinterpret_cast<uint4*>(p_s + off) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
       }
       fence_proxy_async_smem();
       tc_fence_before();

@@ -143,7 +143,7 @@ struct RopeParams {
   const double2* tab; // [nq, hd/2] (cos, sin)
   uint16_t* q;        // packed queries [B][Hkv][nq][G][hd], G = Hq / Hkv
   uint16_t* kc;       // layer base of K cache   [B][Hkv][c_max][hd]
-  uint16_t* vc;       // layer base of V^T cache [B][Hkv][hd][c_max]
+  uint16_t* vc;       // layer base of V^T cache [B][Hkv][hd][c_max] (fp16 holding the bf16 values)
   int T, nq, L0, c_max, Hq, Hkv, hd;
 };
 
@@ -216,7 +216,7 @@ __global__ void __launch_bounds__(256) rope_kv_kernel(const RopeParams p) {
 #pragma unroll
     for (int u = 0; u < kPer; ++u) {
       const int e = threadIdx.x + u * 256;
-      if (e < n) tile[e] = f32_to_bf16(a[u]);  // e = tok * hd + dim
+      if (e < n) tile[e] = bf16_to_f16(f32_to_bf16(a[u]));  // e = tok * hd + dim; the bf16 value, held in fp16
     }
     __syncthreads();
     uint16_t* dst = p.vc + ((long long)b * p.Hkv + g) * p.hd * p.c_max + p.L0 + pos0;

@@ -32,8 +32,8 @@ def _ptr(t):
 
 
 class KVCache:
-    """Per-layer K cache [B, Hkv, c_max, hd] and transposed V cache
-    [B, Hkv, hd, c_max] (bf16).  The capacity is rounded up to a multiple of 8
+    """Per-layer K cache [B, Hkv, c_max, hd] (bf16) and transposed V cache
+    [B, Hkv, hd, c_max] (fp16 holding the bf16-rounded values).  The capacity is rounded up to a multiple of 8
     positions (the row pitch of the transposed cache must be 16-byte aligned)."""
 
     def __init__(self, cfg: dg_model_config, batch: int, c_max: int, device="cuda"):
@@ -51,13 +51,13 @@ class KVCache:
         return self.s.length
 
     def layer_kv(self, layer):
-        """(K, V) of one layer as bf16 [B, Hkv, c_max, hd] views (V is a
-        transposed view of the [B, Hkv, hd, c_max] storage)."""
+        """(K, V) of one layer as [B, Hkv, c_max, hd] views, K bf16 and V fp16
+        (V is a transposed view of the [B, Hkv, hd, c_max] storage)."""
         c = self.cfg
         per = self.k.numel() // 2 // c.n_layers
         k = self.k.view(torch.bfloat16)[layer * per:(layer + 1) * per].view(
             self.s.batch, c.n_kv_heads, self.s.c_max, c.head_dim)
-        vt = self.v.view(torch.bfloat16)[layer * per:(layer + 1) * per].view(
+        vt = self.v.view(torch.float16)[layer * per:(layer + 1) * per].view(
             self.s.batch, c.n_kv_heads, c.head_dim, self.s.c_max)
         return k, vt.transpose(-1, -2)
 

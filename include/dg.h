@@ -97,7 +97,9 @@ typedef struct dg_sampler_config {
 
 /* Causally encoded context, one K and one V buffer of dg_kv_bytes() each:
    K bf16 [n_layers][batch][n_kv_heads][c_max][head_dim] (keys after RoPE),
-   V bf16 transposed, [n_layers][batch][n_kv_heads][head_dim][c_max].
+   V transposed, [n_layers][batch][n_kv_heads][head_dim][c_max], in fp16:
+   the bf16-rounded values (exact in fp16 for magnitudes >= 2^-14), the
+   operand type of the attention's P V product.
    c_max must be a multiple of 8 (16-byte row pitch of the transposed V).
    Positions [0, length) hold the context; a denoising round uses positions
    [length, length + 256) as scratch for the canvas keys, so
@@ -256,7 +258,7 @@ dg_status dg_profile_stop(dg_ctx* ctx, dg_profile* out);
    Computes the same attention as dg_test_attention (dg_testing.h), with the
    same argument meaning and layout: q bf16 packed by kv head
    [B][Hkv][nq][Hq / Hkv][hd], K cache bf16 [B][Hkv][c_max][hd], V cache
-   transposed bf16 [B][Hkv][hd][c_max], both holding keys [0, L0 + nq),
+   transposed fp16 [B][Hkv][hd][c_max], both holding keys [0, L0 + nq),
    c_max a multiple of 8; out bf16 [B * nq, Hq * hd]; causal as there;
    splits 1..8 key splits (0 means 1).  All four pointers are device memory
    owned by the caller.  The split-KV partial

@@ -38,7 +38,7 @@ dg_status dg_test_grouped_gemm(const uint16_t* d_a, int32_t rows_per_group, int3
 /* The library's attention kernel on its own (tcgen05 tensor cores):
    q bf16 packed by kv head [B][Hkv][nq][G][hd] (G = Hq / Hkv, query head
    g * G + j is row j of token t's group g), K cache bf16 [B][Hkv][c_max][hd],
-   V cache transposed, bf16 [B][Hkv][hd][c_max], both holding keys
+   V cache transposed, fp16 [B][Hkv][hd][c_max], both holding keys
    [0, L0 + nq); c_max a multiple of 8; out bf16 [B * nq, Hq * hd]
    (token-major).  causal = 0: every query sees all L0 + nq keys; causal = 1:
    query i sees keys [0, L0 + i].  splits (1..8; 0 means 1) key splits; for

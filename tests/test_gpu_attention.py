@@ -31,10 +31,11 @@ def test_attention_matches_oracle(B, nq, L0, Hq, Hkv, hd, causal, splits):
                                       pml.data_ptr(), torch.cuda.current_stream().cuda_stream))
     got = out.float().cpu().numpy().reshape(B, nq, Hq, hd)
     for b in range(B):
-        want = oracle_attention(ref["q"][b], ref["k"][b], ref["v"][b], np.arange(L0, L0 + nq), np.arange(L0 + nq),
-                                bool(causal))
-        # P is carried as bf16 hi + lo parts, so the error is the bf16 rounding of the
-        # output plus fp32 accumulation noise (see attn_inputs.bound)
+        pos, kpos = np.arange(L0, L0 + nq), np.arange(L0 + nq)
+        want = oracle_attention(ref["q"][b], ref["k"][b], ref["v"][b], pos, kpos, bool(causal))
+        want_abs = oracle_attention(ref["q"][b], ref["k"][b], np.abs(ref["v"][b]), pos, kpos, bool(causal))
+        # bf16 rounding of the output, fp16 probabilities in the P V product and
+        # fp32 accumulation noise (see attn_inputs.bound)
         err = np.abs(got[b] - want)
-        bound = attn_inputs.bound(want, L0 + nq)
+        bound = attn_inputs.bound(want, L0 + nq, want_abs)
         assert np.all(err <= bound), (b, float((err / np.maximum(bound, 1e-30)).max()))

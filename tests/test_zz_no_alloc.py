@@ -30,6 +30,9 @@ def test_static_scratch_matches_caller_scratch(B, nq, L0, Hq, Hkv, hd, causal, s
     want_np = want.float().cpu().numpy()
     ref = np.stack([oracle_attention(ref_in["q"][b], ref_in["k"][b], ref_in["v"][b], np.arange(L0, L0 + nq),
                                      np.arange(L0 + nq), bool(causal)) for b in range(B)]).reshape(B * nq, Hq * hd)
+    ref_abs = np.stack([oracle_attention(ref_in["q"][b], ref_in["k"][b], np.abs(ref_in["v"][b]),
+                                         np.arange(L0, L0 + nq), np.arange(L0 + nq), bool(causal))
+                        for b in range(B)]).reshape(B * nq, Hq * hd)
     for call in range(2):
         out = torch.full((B * nq, Hq * hd), float("nan"), dtype=torch.bfloat16, device="cuda")
         dg.check(dg.lib.dg_attention_static_scratch(dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), out.data_ptr(),
@@ -37,10 +40,10 @@ def test_static_scratch_matches_caller_scratch(B, nq, L0, Hq, Hkv, hd, causal, s
         got = out.float().cpu().numpy()
         assert np.all(np.isfinite(got)), call
         diff = np.abs(got - want_np)
-        bw = attn_inputs.bound(want_np, L0 + nq)
+        bw = attn_inputs.bound(want_np, L0 + nq, ref_abs)
         assert np.all(diff <= bw), (call, float((diff / np.maximum(bw, 1e-30)).max()))
         err = np.abs(got - ref)
-        br = attn_inputs.bound(ref, L0 + nq)
+        br = attn_inputs.bound(ref, L0 + nq, ref_abs)
         assert np.all(err <= br), (call, float((err / np.maximum(br, 1e-30)).max()))
 
 
