@@ -669,8 +669,9 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
     {
       const int v_blocks = B * Hkv * ((nq + kRopeVTok - 1) / kRopeVTok);
       RopeParams rp{c->at<float>(L.qkv), ks_qkv, (long long)T * qkv_rows, c->at<double2>(L.rope),
-                    c->at<uint16_t>(L.q), kc, vc, T, nq, L0, kv->c_max, Hq, Hkv, hd};
-      rope_kv_kernel<<<T + v_blocks, 256, 0, st>>>(rp);
+                    c->at<uint16_t>(L.q), kc, vc, T, nq, L0, kv->c_max, Hq, Hkv, hd, v_blocks};
+      const int rot_blocks = T * ((Hq + Hkv + kRopeHeadsPerBlock - 1) / kRopeHeadsPerBlock);
+      rope_kv_kernel<<<rot_blocks + v_blocks, 256, 0, st>>>(rp);
       CNT(c);
     }
     {
@@ -693,8 +694,9 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
     }
 
     // --- mixture of experts block: residual add of the output projection + RMSNorm ---
-    residual_norm_kernel<<<T, 256, 0, st>>>(x, c->at<float>(L.opart), ks_o, (long long)T * d, d,
-                                            c->wp(W.g_moe), xn, m.rms_eps);
+    residual_norm_kernel<1><<<T, row_launch(d).threads, 0, st>>>(x, c->at<float>(L.opart), ks_o,
+                                                                 (long long)T * d, d, c->wp(W.g_moe), xn,
+                                                                 m.rms_eps);
     CNT(c);
     {
       ProfScope ps_(c, DG_PROF_DENSE, st);
@@ -743,7 +745,9 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
     // norm, or the final norm before the LM head)
     {
       const uint16_t* g_next = l + 1 < m.n_layers ? c->wp(c->wl.layers[l + 1].g_attn) : c->wp(c->wl.g_final);
-      moe_combine_norm_kernel<<<T, 256, 0, st>>>(x, c->at<float>(L.yperm), c->at<int>(L.inv), T, k, d, g_next,
+      // two float4s per thread: the eight expert rows per float4 keep the
+      // register count high, and two CTAs per SM keep every token resident
+      moe_combine_norm_kernel<2><<<T, ((d / 4 + 1) / 2 + 31) / 32 * 32, 0, st>>>(x, c->at<float>(L.yperm), c->at<int>(L.inv), T, k, d, g_next,
                                                  xn, m.rms_eps);
       CNT(c);
     }

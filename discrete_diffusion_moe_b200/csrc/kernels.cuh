@@ -70,19 +70,24 @@ __global__ void __launch_bounds__(THREADS) rmsnorm_kernel(const float* __restric
 
 // ---------------------------------------------------------------------------
 // x[t, :] += sum_s part[s, t, :] (split-k partials of the output projection, in
-// split order), then xn = bf16(x / rms(x) * gain).  One CTA of 256 threads per
-// token; the row stays in registers between the two passes.
-__global__ void __launch_bounds__(256) residual_norm_kernel(float* __restrict__ x, const float* __restrict__ part,
-                                                            int ks, long long split_stride, int d,
-                                                            const uint16_t* __restrict__ gain,
-                                                            uint16_t* __restrict__ xn, float eps) {
+// split order), then xn = bf16(x / rms(x) * gain).  One CTA per token with
+// one float4 of the row per thread (NV per thread when the row is longer than
+// 4096): every load of the row is in flight at once and all tokens' CTAs are
+// resident together; the row stays in registers between the two passes.
+template <int NV>
+__global__ void __launch_bounds__(1024) residual_norm_kernel(float* __restrict__ x, const float* __restrict__ part,
+                                                             int ks, long long split_stride, int d,
+                                                             const uint16_t* __restrict__ gain,
+                                                             uint16_t* __restrict__ xn, float eps) {
   const int t = blockIdx.x;
+  const int nt = blockDim.x;
   float* xr = x + (long long)t * d;
-  float4 r[4];
+  float4 r[NV];
   float ss = 0.f;
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int c = (q * 256 + threadIdx.x) * 4;
+  for (int q = 0; q < NV; ++q) {
+    const int c = (q * nt + threadIdx.x) * 4;
+    r[q] = make_float4(0.f, 0.f, 0.f, 0.f);
     if (c < d) {
       const float* pp = part + (long long)t * d + c;
       float4 sum = *reinterpret_cast<const float4*>(pp);
@@ -97,18 +102,17 @@ __global__ void __launch_bounds__(256) residual_norm_kernel(float* __restrict__ 
       ss += acc.x * acc.x + acc.y * acc.y + acc.z * acc.z + acc.w * acc.w;
     }
   }
-  __shared__ float red[8];
+  __shared__ float red[32];
   ss = warp_sum(ss);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
   __syncthreads();
   float tot = 0.f;
-#pragma unroll
-  for (int w = 0; w < 8; ++w) tot += red[w];
+  for (int w = 0; w < (nt >> 5); ++w) tot += red[w];
   const float rs = rsqrtf(tot / (float)d + eps);
   uint16_t* yr = xn + (long long)t * d;
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int c = (q * 256 + threadIdx.x) * 4;
+  for (int q = 0; q < NV; ++q) {
+    const int c = (q * nt + threadIdx.x) * 4;
     if (c < d) {
       const uint2 gg = *reinterpret_cast<const uint2*>(gain + c);
       uint2 o;
@@ -117,6 +121,18 @@ __global__ void __launch_bounds__(256) residual_norm_kernel(float* __restrict__ 
       *reinterpret_cast<uint2*>(yr + c) = o;
     }
   }
+}
+
+// Threads and float4s per thread of the one-CTA-per-row kernels for a row of
+// d floats (d a multiple of 4).
+struct RowLaunch {
+  int threads, nv;
+};
+inline RowLaunch row_launch(int d) {
+  const int n4 = d / 4;
+  const int nv = n4 <= 1024 ? 1 : (n4 <= 2048 ? 2 : 4);
+  const int per = (n4 + nv - 1) / nv;
+  return {(per + 31) / 32 * 32, nv};
 }
 
 // ---------------------------------------------------------------------------
@@ -145,13 +161,16 @@ struct RopeParams {
   uint16_t* kc;       // layer base of K cache   [B][Hkv][c_max][hd]
   uint16_t* vc;       // layer base of V^T cache [B][Hkv][hd][c_max] (fp16 holding the bf16 values)
   int T, nq, L0, c_max, Hq, Hkv, hd;
+  int v_blocks;       // blocks [0, v_blocks) transpose v; the rest rotate q and k
 };
 
-constexpr int kRopeVTok = 16;  // tokens per v-transpose block
+constexpr int kRopeVTok = 16;          // tokens per v-transpose block
+constexpr int kRopeHeadsPerBlock = 32; // q / k heads rotated per block
 
-// Blocks [0, T): one block per token rotates its q heads (into the packed
-// grouped-query layout) and k heads (into the cache), one thread per rotated
-// pair, the split-k partials summed in order.  Blocks [T, ...): one block per
+// Blocks [v_blocks, ...): one block per (token, group of up to 32 heads) rotates its
+// q heads (into the packed grouped-query layout) and k heads (into the
+// cache), one thread per rotated pair, the split-k partials summed in order.
+// Blocks [0, v_blocks) (scheduled first: they are the long ones): one block per
 // (canvas, kv head, 16 tokens) copies v into the transposed cache through
 // shared memory, so both the reads (along the head dimension) and the writes
 // (along positions) are contiguous; every thread issues the loads of several
@@ -160,16 +179,19 @@ constexpr int kRopeVTok = 16;  // tokens per v-transpose block
 __global__ void __launch_bounds__(256) rope_kv_kernel(const RopeParams p) {
   const int half = p.hd / 2;
   const int row_w = (p.Hq + 2 * p.Hkv) * p.hd;
-  if ((int)blockIdx.x < p.T) {
-    const int t = blockIdx.x;
+  const int parts = (p.Hq + p.Hkv + kRopeHeadsPerBlock - 1) / kRopeHeadsPerBlock;
+  const int rot_blk = (int)blockIdx.x - p.v_blocks;
+  if (rot_blk >= 0) {
+    const int t = rot_blk / parts, part = rot_blk - t * parts;
     const int G = p.Hq / p.Hkv;
     const int b = t / p.nq, pos_in = t - b * p.nq;
-    const int n_pairs = (p.Hq + p.Hkv) * half;
+    const int h0 = part * kRopeHeadsPerBlock;
+    const int n_pairs = (min(p.Hq + p.Hkv, h0 + kRopeHeadsPerBlock) - h0) * half;
     const float* row = p.qkv + (long long)t * row_w;
     const double2* tab = p.tab + (long long)pos_in * half;
 #pragma unroll 2
     for (int j = threadIdx.x; j < n_pairs; j += blockDim.x) {
-      const int h = j / half, i = j - h * half;
+      const int h = h0 + j / half, i = j - (h - h0) * half;
       const float* src = row + h * p.hd + i;
       float a1 = src[0], a2 = src[half];
       for (int q = 1; q < p.ks; ++q) { a1 += src[q * p.split_stride]; a2 += src[q * p.split_stride + half]; }
@@ -190,7 +212,7 @@ __global__ void __launch_bounds__(256) rope_kv_kernel(const RopeParams p) {
   } else {
     __shared__ uint16_t tile[kRopeVTok * 256];  // [token][dim], hd <= 256
     const int tiles_per_seq = (p.nq + kRopeVTok - 1) / kRopeVTok;
-    int blk = (int)blockIdx.x - p.T;
+    int blk = (int)blockIdx.x;
     const int tt = blk % tiles_per_seq;
     blk /= tiles_per_seq;
     const int g = blk % p.Hkv, b = blk / p.Hkv;
@@ -403,26 +425,29 @@ __global__ void gather_rows_kernel(const uint16_t* __restrict__ xn, const int* _
   for (int c = threadIdx.x; c < d / 8; c += blockDim.x) dst[c] = src[c];
 }
 
-// x[t, :] += sum_{j < k} y[inv[t*k + j], :]   (fixed j order, fp32), then
-// the RMSNorm that starts the next block: xn[t, :] = bf16(x / rms(x) * gain).
-// One CTA of 256 threads per token; the row stays in registers between the
-// two passes (d <= 256 * 4 * kCombineVec).
-constexpr int kCombineVec = 4;
-__global__ void __launch_bounds__(256) moe_combine_norm_kernel(float* __restrict__ x, const float* __restrict__ y,
-                                                               const int* __restrict__ inv, int T, int k, int d,
-                                                               const uint16_t* __restrict__ gain,
-                                                               uint16_t* __restrict__ xn, float eps) {
+// Mixture-of-experts combine + residual, fused with the next RMSNorm:
+// x[t, :] += sum_{j < k} y[inv[t, j], :] (the expert outputs already carry
+// their routing weights; fixed order j = 0..k-1), then, when xn is given,
+// xn = bf16(x / rms(x) * gain).  One CTA per token, one float4 of the row per
+// thread (NV when the row is longer than 4096).
+template <int NV>
+__global__ void __launch_bounds__(1024) moe_combine_norm_kernel(float* __restrict__ x, const float* __restrict__ y,
+                                                                const int* __restrict__ inv, int T, int k, int d,
+                                                                const uint16_t* __restrict__ gain,
+                                                                uint16_t* __restrict__ xn, float eps) {
   const int t = blockIdx.x;
   if (t >= T) return;
+  const int nt = blockDim.x;
   int slots[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) slots[j] = j < k ? inv[t * k + j] : 0;
   float* xr = x + (long long)t * d;
-  float4 r[kCombineVec];
+  float4 r[NV];
   float ss = 0.f;
 #pragma unroll
-  for (int q = 0; q < kCombineVec; ++q) {
-    const int c = (q * 256 + threadIdx.x) * 4;
+  for (int q = 0; q < NV; ++q) {
+    const int c = (q * nt + threadIdx.x) * 4;
+    r[q] = make_float4(0.f, 0.f, 0.f, 0.f);
     if (c < d) {
       float4 acc = *reinterpret_cast<const float4*>(xr + c);
       float4 v[8];
@@ -440,18 +465,17 @@ __global__ void __launch_bounds__(256) moe_combine_norm_kernel(float* __restrict
     }
   }
   if (!xn) return;
-  __shared__ float red[8];
+  __shared__ float red[32];
   ss = warp_sum(ss);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
   __syncthreads();
   float tot = 0.f;
-#pragma unroll
-  for (int w = 0; w < 8; ++w) tot += red[w];
+  for (int w = 0; w < (nt >> 5); ++w) tot += red[w];
   const float rs = rsqrtf(tot / (float)d + eps);
   uint16_t* yr = xn + (long long)t * d;
 #pragma unroll
-  for (int q = 0; q < kCombineVec; ++q) {
-    const int c = (q * 256 + threadIdx.x) * 4;
+  for (int q = 0; q < NV; ++q) {
+    const int c = (q * nt + threadIdx.x) * 4;
     if (c < d) {
       const uint2 gg = *reinterpret_cast<const uint2*>(gain + c);
       uint2 o;
