@@ -294,6 +294,8 @@ dg_status run_gemm(const CUtensorMap& ta, const BOperand& tb, GemmPlan p, const 
                    cudaStream_t st, long long* launches = nullptr) {
   if (p.bn < 16 || p.bn > 256 || (p.bn & (p.bn - 1)) || p.K % 64 || p.K < 64)
     return fail(DG_ERR_INVALID_ARG, "gemm plan: bn %d K %d", p.bn, p.K);
+  if (p.group_off && (p.n_groups < 1 || p.n_groups > kGemmMaxGroups))
+    return fail(DG_ERR_INVALID_ARG, "gemm plan: %d groups (1..%d)", p.n_groups, kGemmMaxGroups);
   for (int i = 0; i < 3; ++i) {
     if (tb.rows[i] < 1 || tb.rows[i] > p.bn || (i && tb.rows[i] < tb.rows[i - 1]))
       return fail(DG_ERR_INVALID_ARG, "gemm plan: B box rows %d of bn %d", tb.rows[i], p.bn);
@@ -302,7 +304,7 @@ dg_status run_gemm(const CUtensorMap& ta, const BOperand& tb, GemmPlan p, const 
   static bool attr_done = false;
   if (!attr_done) {
     DG_CUDA(cudaFuncSetAttribute(gemm_tc_kernel<Epi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 227 * 1024));
+                                 (int)(227 * 1024 - kGemmStaticSmem)));
     DG_CUDA(cudaFuncSetAttribute(gemm_tc_kernel<Epi>, cudaFuncAttributePreferredSharedMemoryCarveout, 100));
     attr_done = true;
   }

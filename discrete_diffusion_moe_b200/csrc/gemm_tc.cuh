@@ -69,8 +69,21 @@ struct GemmJob {
   int kb0, kb1;  // k blocks [kb0, kb1) of 64
 };
 
-__device__ __forceinline__ int gemm_num_units(const GemmPlan& p) {
-  if (p.group_off) return p.m_tiles * __ldg(p.chunk_off + p.n_groups);
+// The grouped schedule's offset tables are copied into shared memory at the
+// start of the kernel (a binary search over them in global memory would be a
+// chain of dependent loads before the first copy is issued).
+constexpr int kGemmMaxGroups = 256;
+struct GemmTables {
+  int chunk_off[kGemmMaxGroups + 1];
+  int group_off[kGemmMaxGroups + 1];
+};
+// static shared memory set aside for the tables (and rounding) when sizing
+// the dynamic part
+constexpr size_t kGemmStaticSmem = 4096;
+static_assert(sizeof(GemmTables) <= kGemmStaticSmem, "offset tables");
+
+__device__ __forceinline__ int gemm_num_units(const GemmPlan& p, const GemmTables& tb) {
+  if (p.group_off) return p.m_tiles * tb.chunk_off[p.n_groups];
   const int n_tiles = (p.n_total + p.bn - 1) / p.bn;
   return p.m_tiles * n_tiles * p.k_splits;
 }
@@ -78,7 +91,7 @@ __device__ __forceinline__ int gemm_num_units(const GemmPlan& p) {
 // Every unit is one pass (kept as a loop level so a unit could be split).
 __device__ __forceinline__ int gemm_unit_passes(const GemmPlan&, int) { return 1; }
 
-__device__ __forceinline__ GemmJob gemm_job(const GemmPlan& p, int u, int) {
+__device__ __forceinline__ GemmJob gemm_job(const GemmPlan& p, const GemmTables& tb, int u, int) {
   GemmJob j;
   const int kb_total = p.K / 64;
   if (p.group_off) {
@@ -86,19 +99,19 @@ __device__ __forceinline__ GemmJob gemm_job(const GemmPlan& p, int u, int) {
     int lo = 0, hi = p.n_groups;
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
-      if (p.m_tiles * __ldg(p.chunk_off + mid) <= u) lo = mid;
+      if (p.m_tiles * tb.chunk_off[mid] <= u) lo = mid;
       else hi = mid;
     }
     const int g = lo;
-    const int c0 = __ldg(p.chunk_off + g);
-    const int nch = __ldg(p.chunk_off + g + 1) - c0;
+    const int c0 = tb.chunk_off[g];
+    const int nch = tb.chunk_off[g + 1] - c0;
     const int r = u - p.m_tiles * c0;
     j.m_tile = r / nch;
     const int ch = r - j.m_tile * nch;
     j.group = g;
     j.a_row0 = g * p.a_rows_per_group + j.m_tile * 128;
     j.m_valid = min(128, p.a_rows - j.m_tile * 128);
-    const int off0 = __ldg(p.group_off + g), off1 = __ldg(p.group_off + g + 1);
+    const int off0 = tb.group_off[g], off1 = tb.group_off[g + 1];
     j.n_local0 = ch * p.bn;
     j.n0 = off0 + j.n_local0;
     j.n_valid = min(p.bn, off1 - j.n0);
@@ -139,6 +152,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ BMaps tmB,
                    const GemmPlan p, const Epi epi, const int stages) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
+  __shared__ GemmTables tabs;
   // 1024-byte alignment for the swizzled tiles
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const int b_stage_bytes = p.bn * 128;
@@ -174,12 +188,18 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
     tmem_alloc(smem_u32(tmem_slot), tmem_cols);
     tmem_relinquish();
   }
+  if (p.group_off && warp >= 2) {
+    for (int g = threadIdx.x - 64; g <= p.n_groups; g += kGemmThreads - 64) {
+      tabs.chunk_off[g] = __ldg(p.chunk_off + g);
+      tabs.group_off[g] = __ldg(p.group_off + g);
+    }
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int U = gemm_num_units(p);
+  const int U = gemm_num_units(p, tabs);
 
   if (warp == 0) {
     if (lane == 0) {
@@ -192,7 +212,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
       for (int u = blockIdx.x; u < U && ok; u += gridDim.x) {
         const int np = gemm_unit_passes(p, u);
         for (int pass = 0; pass < np && ok; ++pass) {
-          const GemmJob j = gemm_job(p, u, pass);
+          const GemmJob j = gemm_job(p, tabs, u, pass);
           const int n_mma = (j.n_valid + 15) & ~15;
           const int bi = n_mma <= p.b_rows[0] ? 0 : (n_mma <= p.b_rows[1] ? 1 : 2);
           const CUtensorMap* mb = &tmB.m[bi];
@@ -226,7 +246,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
       for (int u = blockIdx.x; u < U && ok; u += gridDim.x) {
         const int np = gemm_unit_passes(p, u);
         for (int pass = 0; pass < np && ok; ++pass, ++jc) {
-          const GemmJob j = gemm_job(p, u, pass);
+          const GemmJob j = gemm_job(p, tabs, u, pass);
           const int n_mma = (j.n_valid + 15) & ~15;
           const uint32_t idesc = idesc_bf16_f32(128, n_mma);
           const uint32_t acc = jc & 1;
@@ -262,7 +282,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
     for (int u = blockIdx.x; u < U && ok; u += gridDim.x) {
       const int np = gemm_unit_passes(p, u);
       for (int pass = 0; pass < np && ok; ++pass, ++jc) {
-        const GemmJob j = gemm_job(p, u, pass);
+        const GemmJob j = gemm_job(p, tabs, u, pass);
         const uint32_t acc = jc & 1;
         if (!mbar_wait(smem_u32(&acc_full[acc]), (jc >> 1) & 1, p.err)) { ok = false; break; }
         tc_fence_after();
@@ -311,7 +331,7 @@ inline int gemm_ctas_per_sm(int bn) { return bn <= 128 ? 2 : 1; }
 // Stages that fit `ctas` CTAs in one SM's 228 KB (1 KB of each CTA's share is
 // reserved by the system).
 inline int gemm_pick_stages(int bn, int ctas, int max_stages = 8) {
-  const size_t budget = (size_t)228 * 1024 / ctas - 1024;
+  const size_t budget = (size_t)228 * 1024 / ctas - 1024 - kGemmStaticSmem;
   int s = max_stages;
   while (s > 2 && gemm_smem_bytes(bn, s) > budget) --s;
   return s;
