@@ -108,6 +108,7 @@ def _load():
         "dg_profile_start": (I32, [P]),
         "dg_profile_stop": (I32, [P, ctypes.POINTER(dg_profile)]),
         "dg_test_gemm": (I32, [P, I32, P, I32, I32, P, I32, P]),
+        "dg_test_gemm_tiles": (I32, [P, I32, P, I32, I32, P, I32, I32, I32, P]),
         "dg_test_grouped_gemm": (I32, [P, I32, I32, P, I32, I32, P, P, I32, P, P]),
         "dg_test_attention": (I32, [P, P, P, P, I32, I32, I32, I32, I32, I32, I32, I32, I32, P, P, P]),
         "dg_test_workspace_buffer": (I32, [P, ctypes.c_char_p, ctypes.POINTER(P), ctypes.POINTER(S)]),

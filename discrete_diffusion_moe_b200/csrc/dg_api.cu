@@ -140,10 +140,16 @@ int proj_splits(int m_tiles, int T, int kb, int num_sms) {
   return std::max(1, std::min({ks, 3, kb / 4}));
 }
 
+// Split-k (over the vocabulary) of the expected-embedding product
+// e = probs . E_emb: units of two 128-row tiles of E_emb^T (one token tile
+// feeding both) and about one unit per SM (one CTA per SM: the two
+// accumulators of 256 columns fill the tensor memory).
+constexpr int kEsumMt = 2;
 int esum_splits(const dg_model_config& c, int T, int num_sms) {
-  const int m_tiles = (c.d_model + 127) / 128;
-  const int n_tiles = (T + 255) / 256;
-  int ks = (2 * num_sms + m_tiles * n_tiles - 1) / (m_tiles * n_tiles);
+  const int m_units = ((c.d_model + 127) / 128 + kEsumMt - 1) / kEsumMt;
+  const int bn = std::min(256, std::max(16, next_pow2(T)));
+  const int n_tiles = (T + bn - 1) / bn;
+  int ks = num_sms / std::max(1, m_units * n_tiles);
   ks = std::max(1, std::min(ks, 32));
   return std::min(ks, c.vocab / 64);
 }
@@ -296,6 +302,8 @@ dg_status run_gemm(const CUtensorMap& ta, const BOperand& tb, GemmPlan p, const 
     return fail(DG_ERR_INVALID_ARG, "gemm plan: bn %d K %d", p.bn, p.K);
   if (p.group_off && (p.n_groups < 1 || p.n_groups > kGemmMaxGroups))
     return fail(DG_ERR_INVALID_ARG, "gemm plan: %d groups (1..%d)", p.n_groups, kGemmMaxGroups);
+  if (p.mt != 1 && (p.mt != 2 || p.group_off))
+    return fail(DG_ERR_INVALID_ARG, "gemm plan: %d A tiles per unit", p.mt);
   for (int i = 0; i < 3; ++i) {
     if (tb.rows[i] < 1 || tb.rows[i] > p.bn || (i && tb.rows[i] < tb.rows[i - 1]))
       return fail(DG_ERR_INVALID_ARG, "gemm plan: B box rows %d of bn %d", tb.rows[i], p.bn);
@@ -308,12 +316,12 @@ dg_status run_gemm(const CUtensorMap& ta, const BOperand& tb, GemmPlan p, const 
     DG_CUDA(cudaFuncSetAttribute(gemm_tc_kernel<Epi>, cudaFuncAttributePreferredSharedMemoryCarveout, 100));
     attr_done = true;
   }
-  const int ctas = gemm_ctas_per_sm(p.bn);
-  const int stages = gemm_pick_stages(p.bn, ctas);
-  const size_t smem = gemm_smem_bytes(p.bn, stages);
+  const int ctas = gemm_ctas_per_sm(p.bn, p.mt);
+  const int stages = gemm_pick_stages(p.bn, ctas, 8, p.mt);
+  const size_t smem = gemm_smem_bytes(p.bn, stages, p.mt);
   long long units;  // grouped: known only on the device; persistent CTAs
   if (p.group_off) units = (long long)ctas * num_sms;
-  else units = (long long)p.m_tiles * ((p.n_total + p.bn - 1) / p.bn) * p.k_splits;
+  else units = (long long)((p.m_tiles + p.mt - 1) / p.mt) * ((p.n_total + p.bn - 1) / p.bn) * p.k_splits;
   if (units <= 0) return DG_OK;
   const int grid = (int)std::min<long long>(units, (long long)ctas * num_sms);
   gemm_tc_kernel<Epi><<<grid, kGemmThreads, smem, st>>>(ta, tb.maps, p, epi, stages);
@@ -332,6 +340,7 @@ GemmPlan dense_plan(int K, int a_rows, int n_total, int bn, int k_splits, int* e
   p.k_splits = k_splits;
   p.n_fast = 1;
   p.group_off = nullptr;
+  p.mt = 1;
   p.err = err;
   return p;
 }
@@ -349,6 +358,7 @@ GemmPlan grouped_plan(int K, int rows_per_group, const int* off, const int* chun
   p.group_off = off;
   p.n_groups = n_groups;
   p.a_rows_per_group = rows_per_group;
+  p.mt = 1;
   p.err = err;
   return p;
 }
@@ -938,6 +948,7 @@ static dg_status enqueue_round(dg_ctx* c, const dg_kv* kv, dg_canvas* cv, const 
     DG_TRY(make_tmap(&ta, c->wp(c->wl.embT), V, d, 128));
     DG_TRY(make_bop(&tb, probs, V, L.T_alloc, bnT));
     GemmPlan p = dense_plan(V, d, T, bnT, ks, err);
+    p.mt = kEsumMt;
     p.a_hint = 1;
     p.b_hint = 2;
     EpiStoreT e{c->at<float>(L.epart), d, (long long)T * d, 0, nullptr, nullptr, 0, err};
@@ -1166,6 +1177,26 @@ extern "C" dg_status dg_test_gemm(const uint16_t* A, int32_t M, const uint16_t* 
   DG_TRY(make_bop(&tb, B, K, N, bn));
   GemmPlan p = dense_plan(K, M, N, bn, k_splits, err);
   p.n_fast = 0;
+  EpiSplitRows e{D, M, N};
+  DG_TRY(run_gemm(ta, tb, p, e, device_sms(), st));
+  DG_CUDA(cudaStreamSynchronize(st));
+  return DG_OK;
+}
+
+extern "C" dg_status dg_test_gemm_tiles(const uint16_t* A, int32_t M, const uint16_t* B, int32_t N, int32_t K,
+                                        float* D, int32_t k_splits, int32_t mt, int32_t bn, void* stream) {
+  if (!A || !B || !D || M < 128 || N < 16 || K < 64 || K % 64 || k_splits < 1 || k_splits > K / 64 ||
+      (mt != 1 && mt != 2) || (bn != 0 && (bn < 16 || bn > 256 || (bn & (bn - 1)))))
+    return fail(DG_ERR_INVALID_ARG, "dg_test_gemm_tiles: bad arguments");
+  cudaStream_t st = (cudaStream_t)stream;
+  if (bn == 0) bn = token_bn(N);
+  CUtensorMap ta;
+  BOperand tb;
+  DG_TRY(make_tmap(&ta, A, K, M, 128));
+  DG_TRY(make_bop(&tb, B, K, N, bn));
+  GemmPlan p = dense_plan(K, M, N, bn, k_splits, nullptr);
+  p.n_fast = 0;
+  p.mt = mt;
   EpiSplitRows e{D, M, N};
   DG_TRY(run_gemm(ta, tb, p, e, device_sms(), st));
   DG_CUDA(cudaStreamSynchronize(st));

@@ -54,6 +54,7 @@ struct GemmPlan {
   int n_groups;
   int a_rows_per_group;  // grouped: A row stride between groups
   int a_hint, b_hint;    // L2 policy of the A / B loads: 0 none, 1 evict_first, 2 evict_last
+  int mt;                // dense: 128-row A tiles per unit (1 or 2; grouped: 1)
   int* err;              // device error word
 };
 
@@ -67,6 +68,7 @@ struct GemmJob {
   int n_valid;   // valid columns (B rows) in this pass, 1..bn
   int ks;        // k split index
   int kb0, kb1;  // k blocks [kb0, kb1) of 64
+  int mt_eff;    // A tiles in this unit (dense units may cover two, tiles m_tile, m_tile + 1)
 };
 
 // The grouped schedule's offset tables are copied into shared memory at the
@@ -85,7 +87,8 @@ static_assert(sizeof(GemmTables) <= kGemmStaticSmem, "offset tables");
 __device__ __forceinline__ int gemm_num_units(const GemmPlan& p, const GemmTables& tb) {
   if (p.group_off) return p.m_tiles * tb.chunk_off[p.n_groups];
   const int n_tiles = (p.n_total + p.bn - 1) / p.bn;
-  return p.m_tiles * n_tiles * p.k_splits;
+  const int m_units = (p.m_tiles + p.mt - 1) / p.mt;
+  return m_units * n_tiles * p.k_splits;
 }
 
 // Every unit is one pass (kept as a loop level so a unit could be split).
@@ -118,13 +121,17 @@ __device__ __forceinline__ GemmJob gemm_job(const GemmPlan& p, const GemmTables&
     j.ks = 0;
     j.kb0 = 0;
     j.kb1 = kb_total;
+    j.mt_eff = 1;
   } else {
     const int n_tiles = (p.n_total + p.bn - 1) / p.bn;
+    const int m_units = (p.m_tiles + p.mt - 1) / p.mt;
     const int ks = u % p.k_splits;
     const int r = u / p.k_splits;
-    int mt, nt;
-    if (p.n_fast) { nt = r % n_tiles; mt = r / n_tiles; }
-    else          { mt = r % p.m_tiles; nt = r / p.m_tiles; }
+    int mu, nt;
+    if (p.n_fast) { nt = r % n_tiles; mu = r / n_tiles; }
+    else          { mu = r % m_units; nt = r / m_units; }
+    const int mt = mu * p.mt;
+    j.mt_eff = min(p.mt, p.m_tiles - mt);
     j.m_tile = mt;
     j.group = -1;
     j.a_row0 = mt * 128;
@@ -156,8 +163,9 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
   // 1024-byte alignment for the swizzled tiles
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const int b_stage_bytes = p.bn * 128;
+  const int a_stage_bytes = p.mt * kATileBytes;
   uint8_t* sA = smem;
-  uint8_t* sB = smem + (size_t)stages * kATileBytes;
+  uint8_t* sB = smem + (size_t)stages * a_stage_bytes;
   uint64_t* bars = (uint64_t*)(sB + (size_t)stages * b_stage_bytes);
   uint64_t* full = bars;
   uint64_t* empty = bars + stages;
@@ -167,7 +175,12 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
   uint32_t* tmem_slot = (uint32_t*)(drain + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t tmem_cols = 2u * (uint32_t)p.bn < 32u ? 32u : 2u * (uint32_t)p.bn;
+  // accumulator buffers: two (the next unit's MMAs overlap this unit's
+  // epilogue) unless two A tiles of 256 columns fill the tensor memory
+  const uint32_t buf_cols = (uint32_t)(p.mt * p.bn);
+  const int nbuf = buf_cols <= 256u ? 2 : 1;
+  const uint32_t tmem_need = buf_cols * nbuf;
+  const uint32_t tmem_cols = tmem_need <= 32u ? 32u : (tmem_need <= 64u ? 64u : (tmem_need <= 128u ? 128u : (tmem_need <= 256u ? 256u : 512u)));
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) {
@@ -216,16 +229,18 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
           const int n_mma = (j.n_valid + 15) & ~15;
           const int bi = n_mma <= p.b_rows[0] ? 0 : (n_mma <= p.b_rows[1] ? 1 : 2);
           const CUtensorMap* mb = &tmB.m[bi];
-          const uint32_t tx = kATileBytes + (uint32_t)p.b_rows[bi] * 128;
+          const uint32_t tx = (uint32_t)j.mt_eff * kATileBytes + (uint32_t)p.b_rows[bi] * 128;
           for (int kb = j.kb0; kb < j.kb1; ++kb, ++it) {
             const int s = it % stages;
             const uint32_t ph = (it / stages) & 1;
             if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1, p.err)) { ok = false; break; }
             const uint32_t fb = smem_u32(&full[s]);
             mbar_arrive_expect_tx(fb, tx);
-            const uint32_t dA = smem_u32(sA + (size_t)s * kATileBytes);
-            if (p.a_hint) tma_load_2d_hint(dA, &tmA, fb, kb * 64, j.a_row0, pol_a);
-            else          tma_load_2d(dA, &tmA, fb, kb * 64, j.a_row0);
+            for (int t = 0; t < j.mt_eff; ++t) {
+              const uint32_t dA = smem_u32(sA + (size_t)s * a_stage_bytes + t * kATileBytes);
+              if (p.a_hint) tma_load_2d_hint(dA, &tmA, fb, kb * 64, j.a_row0 + t * 128, pol_a);
+              else          tma_load_2d(dA, &tmA, fb, kb * 64, j.a_row0 + t * 128);
+            }
             const uint32_t dB = smem_u32(sB + (size_t)s * b_stage_bytes);
             if (p.b_hint) tma_load_2d_hint(dB, mb, fb, kb * 64, j.n0, pol_b);
             else          tma_load_2d(dB, mb, fb, kb * 64, j.n0);
@@ -249,21 +264,24 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
           const GemmJob j = gemm_job(p, tabs, u, pass);
           const int n_mma = (j.n_valid + 15) & ~15;
           const uint32_t idesc = idesc_bf16_f32(128, n_mma);
-          const uint32_t acc = jc & 1;
-          if (!mbar_wait(smem_u32(&acc_empty[acc]), ((jc >> 1) & 1) ^ 1, p.err)) { ok = false; break; }
+          const uint32_t acc = nbuf == 2 ? (jc & 1) : 0;
+          const uint32_t use = nbuf == 2 ? (jc >> 1) : jc;
+          if (!mbar_wait(smem_u32(&acc_empty[acc]), (use & 1) ^ 1, p.err)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t d_tmem = tmem_base + acc * (uint32_t)p.bn;
+          const uint32_t d_tmem = tmem_base + acc * buf_cols;
           for (int kb = j.kb0; kb < j.kb1; ++kb, ++it) {
             const int s = it % stages;
             const uint32_t ph = (it / stages) & 1;
             if (!mbar_wait(smem_u32(&full[s]), ph, p.err)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t a0 = smem_u32(sA + (size_t)s * kATileBytes);
             const uint32_t b0 = smem_u32(sB + (size_t)s * b_stage_bytes);
+            for (int t = 0; t < j.mt_eff; ++t) {
+              const uint32_t a0 = smem_u32(sA + (size_t)s * a_stage_bytes + t * kATileBytes);
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              umma_bf16(d_tmem, sdesc_k128(a0 + kk * 32), sdesc_k128(b0 + kk * 32), idesc,
-                        (kb > j.kb0 || kk > 0) ? 1u : 0u);
+              for (int kk = 0; kk < 4; ++kk)
+                umma_bf16(d_tmem + t * (uint32_t)p.bn, sdesc_k128(a0 + kk * 32), sdesc_k128(b0 + kk * 32), idesc,
+                          (kb > j.kb0 || kk > 0) ? 1u : 0u);
+            }
             umma_commit(smem_u32(&empty[s]));
           }
           if (ok) umma_commit(smem_u32(&acc_full[acc]));
@@ -282,11 +300,17 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
     for (int u = blockIdx.x; u < U && ok; u += gridDim.x) {
       const int np = gemm_unit_passes(p, u);
       for (int pass = 0; pass < np && ok; ++pass, ++jc) {
-        const GemmJob j = gemm_job(p, tabs, u, pass);
-        const uint32_t acc = jc & 1;
-        if (!mbar_wait(smem_u32(&acc_full[acc]), (jc >> 1) & 1, p.err)) { ok = false; break; }
+        const GemmJob ju = gemm_job(p, tabs, u, pass);
+        const uint32_t acc = nbuf == 2 ? (jc & 1) : 0;
+        const uint32_t use = nbuf == 2 ? (jc >> 1) : jc;
+        if (!mbar_wait(smem_u32(&acc_full[acc]), use & 1, p.err)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t t0 = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * (uint32_t)p.bn;
+        for (int t = 0; t < ju.mt_eff; ++t) {
+        GemmJob j = ju;
+        j.m_tile = ju.m_tile + t;
+        j.a_row0 = ju.a_row0 + t * 128;
+        j.m_valid = min(128, p.a_rows - j.m_tile * 128);
+        const uint32_t t0 = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * buf_cols + t * (uint32_t)p.bn;
         typename Epi::State st;
         epi.begin(j, row, st);
         const int nch = (j.n_valid + 15) >> 4;
@@ -307,6 +331,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
           }
         }
         epi.end(j, row, st);
+        }
         tc_fence_before();
         mbar_arrive(smem_u32(&acc_empty[acc]));
       }
@@ -320,20 +345,20 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
 }
 
 // Dynamic shared memory of one CTA for `stages` stages.
-inline size_t gemm_smem_bytes(int bn, int stages) {
-  return 1024 + (size_t)stages * (kATileBytes + (size_t)bn * 128) + (2 * stages + 5) * 8 + 16;
+inline size_t gemm_smem_bytes(int bn, int stages, int mt = 1) {
+  return 1024 + (size_t)stages * ((size_t)mt * kATileBytes + (size_t)bn * 128) + (2 * stages + 5) * 8 + 16;
 }
 
-// CTAs per SM: two when both fit (tensor memory: 2 x 2 x bn columns <= 512;
-// shared memory: at least three stages each), else one.
-inline int gemm_ctas_per_sm(int bn) { return bn <= 128 ? 2 : 1; }
+// CTAs per SM: two when both fit (tensor memory: 2 buffers x mt x bn columns
+// <= 256 each; shared memory: at least three stages each), else one.
+inline int gemm_ctas_per_sm(int bn, int mt = 1) { return mt * bn <= 128 ? 2 : 1; }
 
 // Stages that fit `ctas` CTAs in one SM's 228 KB (1 KB of each CTA's share is
 // reserved by the system).
-inline int gemm_pick_stages(int bn, int ctas, int max_stages = 8) {
+inline int gemm_pick_stages(int bn, int ctas, int max_stages = 8, int mt = 1) {
   const size_t budget = (size_t)228 * 1024 / ctas - 1024 - kGemmStaticSmem;
   int s = max_stages;
-  while (s > 2 && gemm_smem_bytes(bn, s) > budget) --s;
+  while (s > 2 && gemm_smem_bytes(bn, s, mt) > budget) --s;
   return s;
 }
 

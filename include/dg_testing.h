@@ -24,6 +24,12 @@ extern "C" {
 dg_status dg_test_gemm(const uint16_t* d_a, int32_t M, const uint16_t* d_b, int32_t N, int32_t K,
                        float* d_d, int32_t k_splits, void* stream);
 
+/* dg_test_gemm with the unit shape chosen: mt (1 or 2) 128-row A tiles and
+   bn (16..256, power of two) B rows per unit; bn = 0 picks the library's
+   choice for N.  Same output layout and split convention.  Synchronous. */
+dg_status dg_test_gemm_tiles(const uint16_t* d_a, int32_t M, const uint16_t* d_b, int32_t N, int32_t K,
+                             float* d_d, int32_t k_splits, int32_t mt, int32_t bn, void* stream);
+
 /* Grouped product as used by the expert layers: group g multiplies A rows
    [g * rows_per_group, (g + 1) * rows_per_group) with B rows
    [off[g], off[g+1]) and writes D[r, f] (fp32, [n_rows, rows_per_group]) for

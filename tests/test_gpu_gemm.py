@@ -74,3 +74,22 @@ def test_grouped_gemm(dg, bn, sizes):
 def test_gemm_rejects_bad_shapes(dg):
     with pytest.raises(dg.DgError):
         dg.check(dg.dg_test_gemm(None, 128, None, 16, 64, None, 1, None))
+
+
+@pytest.mark.parametrize("M,N,K,ks,mt,bn", [(256, 256, 512, 1, 2, 256), (384, 200, 320, 1, 2, 256),
+                                          (128 * 23, 256, 1024, 3, 2, 256), (128 * 45, 256, 2816, 3, 2, 128),
+                                          (640, 48, 704, 2, 2, 64), (128 * 300, 32, 640, 1, 2, 32)])
+def test_dense_gemm_two_a_tiles(dg, M, N, K, ks, mt, bn):
+    """Units of two 128-row A tiles (one B tile feeding two MMAs): odd tile
+    counts (a last unit with one tile), one or two accumulator buffers."""
+    rng = np.random.default_rng(M + N + K + mt)
+    a, b = _bf16(rng, (M, K)), _bf16(rng, (N, K))
+    da, db = a.cuda(), b.cuda()
+    dd = torch.full((ks, M, N), float("nan"), device="cuda")
+    st = torch.cuda.current_stream().cuda_stream
+    dg.check(dg.lib.dg_test_gemm_tiles(da.data_ptr(), M, db.data_ptr(), N, K, dd.data_ptr(), ks, mt, bn, st))
+    got = dd.sum(0).double().cpu().numpy()
+    ref = _ref(a, b)
+    tol = 1e-5 * np.sqrt(K) * 4 + 1e-6
+    assert np.isfinite(got).all()
+    assert np.abs(got - ref).max() <= tol * np.abs(ref).max() + 1e-4, np.abs(got - ref).max()
