@@ -220,6 +220,20 @@ def oracle_sample(wl, threads):
     return per_step, desc, t4 - t0
 
 
+def max_over_ranks(x, world):
+    """The largest value of x over the ranks of the job (a job's time is its
+    slowest rank's).  One process per GPU: NCCL tensors live on the rank's
+    GPU, gloo (the CPU tests of this path) on the host."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(x)], device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def cpu_cores():
     try:
         return len(os.sched_getaffinity(0))
@@ -339,11 +353,7 @@ def main():
     barrier()
     clk = clocks.stop()
     model.check_device()
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1), world)
     ms_per_step = ms / args.steps
     value = world * args.steps / (ms / 1000.0)
 
@@ -433,11 +443,7 @@ def main():
             h_sc.copy_(h_sc_out)
         f1.record(stream)
         barrier()
-        ms_e2e = f0.elapsed_time(f1)
-        if world > 1:
-            t = torch.tensor([ms_e2e], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms_e2e = float(t.item())
+        ms_e2e = max_over_ranks(f0.elapsed_time(f1), world)
         e2e = {"value": world * n_e2e / (ms_e2e / 1000.0), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "steps": n_e2e}
 
