@@ -117,7 +117,7 @@ WLayout weight_layout(const dg_model_config& c) {
 constexpr int kMaxAttnSplits = 8;
 
 struct WsLayout {
-  size_t err, flags, x, xn, qkv, opart, q, attn, attn_po, attn_pml, rpart, idx, w, off, choff, perm, inv, wperm,
+  size_t err, flags, x, xn, qkv, opart, q, attn, attn_po, attn_pml, rpart, rbar, rfill, off, choff, perm, inv, wperm,
       xperm, hperm, yperm, logits, vp_m, vp_z, vp_s, vp_av, vp_ai, vp_gv, vp_gi, st_m, st_iz, st_h,
       st_pmax, st_amax, st_samp, probs, epart, rope, stepdev, total;
   int T_alloc, P_alloc, ks_r, n_vt, attn_rows_cap;
@@ -190,8 +190,8 @@ WsLayout ws_layout(const dg_model_config& c, int batch, int num_sms) {
   L.attn_po = take((size_t)L.attn_rows_cap * DG_CANVAS * hq * 4);
   L.attn_pml = take((size_t)L.attn_rows_cap * DG_CANVAS * c.n_q_heads * 2 * 4);
   L.rpart = take((size_t)L.ks_r * T * E * 4);
-  L.idx = take(P * 4);
-  L.w = take(P * 4);
+  L.rbar = take(64);
+  L.rfill = take(E * 4);
   L.off = take((E + 1) * 4);
   L.choff = take((E + 1) * 4);
   L.perm = take(P * 4);
@@ -548,6 +548,8 @@ extern "C" dg_status dg_context_create(const dg_model_config* cfg, const void* d
     return fail(DG_ERR_WORKSPACE, "workspace too small: %zu < %zu", ws_bytes, need);
   }
   cudaError_t e = cudaMemset(c->ws + c->L.err, 0, 64);
+  if (e == cudaSuccess) e = cudaMemset(c->ws + c->L.rbar, 0, 64);
+  if (e == cudaSuccess) e = cudaMemset(c->ws + c->L.rfill, 0, (size_t)cfg->n_experts * 4);
   if (e != cudaSuccess) {
     delete c;
     return fail(DG_ERR_CUDA, "cudaMemset: %s", cudaGetErrorString(e));
@@ -722,17 +724,39 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
       DG_TRY(run_gemm(ta, tb, p, e, c->num_sms, st, &c->n_launch));
     }
     if (L.ks_r != kRouterSplits) return fail(DG_ERR_UNSUPPORTED, "router split count %d", L.ks_r);
-    router_topk_kernel<kRouterSplits><<<(T * 32 + 255) / 256, 256, 0, st>>>(
-        c->at<float>(L.rpart), T, E, k, c->at<int>(L.idx), c->at<float>(L.w),
-        dbg_idx ? dbg_idx + (size_t)l * T * k : nullptr, dbg_w ? dbg_w + (size_t)l * T * k : nullptr,
-        dbg_logits ? dbg_logits + (size_t)l * T * E : nullptr);
-        CNT(c);
-    permute_kernel<<<1, kPermThreads, (size_t)34 * E * sizeof(int), st>>>(
-        c->at<int>(L.idx), c->at<float>(L.w), P, E, bnG, c->at<int>(L.off), c->at<int>(L.choff),
-        c->at<int>(L.perm), c->at<int>(L.inv), c->at<float>(L.wperm), err);
-        CNT(c);
-    gather_rows_kernel<<<P, 128, 0, st>>>(xn, c->at<int>(L.perm), c->at<uint16_t>(L.xperm), P, k, d);
-    CNT(c);
+    {
+      // top-k, counting sort by expert and row gather in one cooperative launch
+      RouteParams rp;
+      rp.part = c->at<float>(L.rpart);
+      rp.xn = xn;
+      rp.T = T; rp.E = E; rp.k = k; rp.d = d; rp.bn = bnG;
+      rp.tpc = (T + c->num_sms - 1) / c->num_sms;
+      rp.off = c->at<int>(L.off);
+      rp.chunk_off = c->at<int>(L.choff);
+      rp.perm = c->at<int>(L.perm);
+      rp.inv = c->at<int>(L.inv);
+      rp.w_perm = c->at<float>(L.wperm);
+      rp.xperm = c->at<uint16_t>(L.xperm);
+      rp.fill = c->at<int>(L.rfill);
+      rp.bar = c->at<int>(L.rbar);
+      rp.dbg_idx = dbg_idx ? dbg_idx + (size_t)l * T * k : nullptr;
+      rp.dbg_w = dbg_w ? dbg_w + (size_t)l * T * k : nullptr;
+      rp.dbg_logits = dbg_logits ? dbg_logits + (size_t)l * T * E : nullptr;
+      rp.err = err;
+      const int nb = (T + rp.tpc - 1) / rp.tpc;
+      cudaLaunchConfig_t lc = {};
+      cudaLaunchAttribute at[1];
+      at[0].id = cudaLaunchAttributeCooperative;
+      at[0].val.cooperative = 1;
+      lc.gridDim = dim3(nb);
+      lc.blockDim = dim3(kRouteThreads);
+      lc.dynamicSmemBytes = route_smem_bytes(rp.tpc, k, E);
+      lc.stream = st;
+      lc.attrs = at;
+      lc.numAttrs = 1;
+      DG_CUDA(cudaLaunchKernelEx(&lc, route_kernel<kRouterSplits>, rp));
+      CNT(c);
+    }
     {
       ProfScope ps_(c, DG_PROF_EXPERT_GATE_UP, st);
       CUtensorMap ta;
@@ -1063,6 +1087,9 @@ extern "C" dg_status dg_check_device_error(dg_ctx* c, void* stream) {
   DG_CUDA(cudaMemcpy(&e, c->err(), sizeof(int), cudaMemcpyDeviceToHost));
   if (e) {
     DG_CUDA(cudaMemset(c->err(), 0, sizeof(int)));
+    // a wait that ran out may have left the routing counters mid-count
+    DG_CUDA(cudaMemset(c->ws + c->L.rbar, 0, 64));
+    DG_CUDA(cudaMemset(c->ws + c->L.rfill, 0, (size_t)c->cfg.n_experts * 4));
     if (e == kDevErrBadToken) return fail(DG_ERR_BAD_TOKEN, "a token id outside [0, vocab) reached the device");
     if (e == kDevErrTimeout) return fail(DG_ERR_TIMEOUT, "a bounded device wait ran out");
     return fail(DG_ERR_CUDA, "device error word %d", e);
@@ -1243,8 +1270,7 @@ extern "C" dg_status dg_test_workspace_buffer(dg_ctx* c, const char* name, void*
   const WsLayout& L = c->L;
   struct Entry { const char* n; size_t off, next; };
   const Entry tab[] = {{"x", L.x, L.xn}, {"xn", L.xn, L.qkv}, {"qkv", L.qkv, L.q}, {"q", L.q, L.attn},
-                       {"attn", L.attn, L.attn_po}, {"rpart", L.rpart, L.idx}, {"idx", L.idx, L.w},
-                       {"w", L.w, L.off},
+                       {"attn", L.attn, L.attn_po}, {"rpart", L.rpart, L.rbar},
                        {"off", L.off, L.perm}, {"perm", L.perm, L.inv}, {"inv", L.inv, L.wperm},
                        {"wperm", L.wperm, L.xperm}, {"xperm", L.xperm, L.hperm}, {"hperm", L.hperm, L.yperm},
                        {"yperm", L.yperm, L.logits}, {"logits", L.logits, L.vp_m},

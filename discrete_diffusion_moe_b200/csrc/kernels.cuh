@@ -250,156 +250,274 @@ __global__ void __launch_bounds__(256) rope_kv_kernel(const RopeParams p) {
 }
 
 // ---------------------------------------------------------------------------
-// Router: sum the split-k partial logits (fixed order), pick the top-k
-// experts by logit (ties to the lower id), softmax over the chosen k.
-// One warp per token; E <= 256.
+// Routing of the mixture-of-experts block in one launch: router top-k, the
+// stable counting sort of the (token, slot) pairs by expert, and the gather of
+// the normalised rows into expert order.
+//
+// Top-k of one token (one warp): sum the split-k partial logits (fixed
+// order), pick the k largest logits (ties to the lower expert id), softmax
+// over the chosen k.  E <= 256, k <= 8.
 template <int KS>
-__global__ void router_topk_kernel(const float* __restrict__ part, int T, int E, int k,
-                                   int* __restrict__ idx, float* __restrict__ w,
-                                   int* __restrict__ dbg_idx, float* __restrict__ dbg_w,
-                                   float* __restrict__ dbg_logits) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (warp >= T) return;
-  const int t = warp;
+__device__ __forceinline__ void route_topk_token(const float* __restrict__ part, int T, int E, int k, int t,
+                                                 int lane, int* sel_out, float* w_out, int* dbg_idx,
+                                                 float* dbg_w, float* dbg_logits) {
   float l[8];
-  bool taken[8];
 #pragma unroll
-  for (int q = 0; q < 8; ++q) { l[q] = 0.f; taken[q] = false; }
-  // split-k partials summed in split order; the 8 expert slots of a lane are
-  // independent, so their loads are issued together
+  for (int q = 0; q < 8; ++q) l[q] = 0.f;
+  // the 8 expert slots of a lane are independent, so their loads issue together
 #pragma unroll
   for (int p = 0; p < KS; ++p) {
     const float* row = part + ((long long)p * T + t) * E;
     float v[8];
 #pragma unroll
-    for (int q = 0; q < 8; ++q) v[q] = (lane + 32 * q < E) ? row[lane + 32 * q] : 0.f;
+    for (int q = 0; q < 8; ++q) v[q] = (lane + 32 * q < E) ? __ldcg(row + lane + 32 * q) : 0.f;
 #pragma unroll
     for (int q = 0; q < 8; ++q) l[q] += v[q];
   }
+  // order-preserving integer keys of the logits (larger logit, larger key);
+  // 0 marks an absent or already chosen expert
+  uint32_t key[8];
 #pragma unroll
   for (int q = 0; q < 8; ++q) {
-    if (lane + 32 * q >= E) l[q] = -INFINITY;
-    else if (dbg_logits) dbg_logits[(long long)t * E + lane + 32 * q] = l[q];
+    const bool ok = lane + 32 * q < E;
+    if (ok && dbg_logits) dbg_logits[(long long)t * E + lane + 32 * q] = l[q];
+    const uint32_t u = __float_as_uint(l[q]);
+    key[q] = ok ? ((u & 0x80000000u) ? ~u : (u | 0x80000000u)) : 0u;
+    if (ok && key[q] == 0u) key[q] = 1u;  // -NaN patterns: keep them selectable
   }
-  float sel_l[8];
+  // k rounds: the warp's largest key (one reduction), then the lowest expert
+  // id holding it (a second reduction); that expert leaves the candidates
+  uint32_t sel_k[8];
   int sel_e[8];
-  for (int r = 0; r < k; ++r) {
-    float bv = -INFINITY;
-    int be = 0x7fffffff;
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const int e = lane + 32 * q;
-      if (e < E && !taken[q] && (l[q] > bv || (l[q] == bv && e < be))) { bv = l[q]; be = e; }
-    }
+  for (int r = 0; r < 8; ++r) {
+    if (r >= k) break;
+    uint32_t best = 0u;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-      if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
-    }
+    for (int q = 0; q < 8; ++q) best = max(best, key[q]);
+    const uint32_t wmax = __reduce_max_sync(0xffffffffu, best);
+    uint32_t cand = 0xffffffffu;
+#pragma unroll
+    for (int q = 7; q >= 0; --q)
+      if (key[q] == wmax && wmax != 0u) cand = (uint32_t)(lane + 32 * q);
+    const uint32_t we = __reduce_min_sync(0xffffffffu, cand);
 #pragma unroll
     for (int q = 0; q < 8; ++q)
-      if (lane + 32 * q == be) taken[q] = true;
-    sel_l[r] = bv;
-    sel_e[r] = be;
+      if ((uint32_t)(lane + 32 * q) == we) key[q] = 0u;
+    sel_k[r] = wmax;
+    sel_e[r] = (int)we;
   }
-  if (lane == 0) {
-    float den = 0.f;
-    float ex[8];
-    for (int r = 0; r < k; ++r) { ex[r] = expf(sel_l[r] - sel_l[0]); den += ex[r]; }
-    for (int r = 0; r < k; ++r) {
-      idx[t * k + r] = sel_e[r];
-      w[t * k + r] = ex[r] / den;
-      if (dbg_idx) dbg_idx[t * k + r] = sel_e[r];
-      if (dbg_w) dbg_w[t * k + r] = ex[r] / den;
+  // softmax over the chosen logits, lane r handling choice r
+  float lr = 0.f;
+  int er = 0;
+#pragma unroll
+  for (int r = 0; r < 8; ++r)
+    if (r == lane && r < k) {
+      const uint32_t kk = sel_k[r];
+      lr = __uint_as_float((kk & 0x80000000u) ? (kk & 0x7fffffffu) : ~kk);
+      er = sel_e[r];
     }
+  const float l0 = __shfl_sync(0xffffffffu, lr, 0);
+  const float ex = lane < k ? expf(lr - l0) : 0.f;
+  float den = ex;
+#pragma unroll
+  for (int o = 1; o < 8; o <<= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+  if (lane < k) {
+    const float wv = ex / den;
+    sel_out[lane] = er;
+    w_out[lane] = wv;
+    if (dbg_idx) dbg_idx[t * k + lane] = er;
+    if (dbg_w) dbg_w[t * k + lane] = wv;
   }
 }
 
-// ---------------------------------------------------------------------------
-// Token permutation: stable counting sort of the T*k (token, slot) pairs by
-// expert.  One CTA of 1024 threads.  Outputs off[E+1], perm[slot] = pair,
-// inv[pair] = slot, w_perm[slot] = w[pair].  Within an expert, pairs keep
-// ascending pair order (token-major), so the layout is deterministic.
-constexpr int kPermThreads = 1024;
-__global__ void __launch_bounds__(kPermThreads) permute_kernel(const int* __restrict__ idx,
-                                                               const float* __restrict__ w, int P,
-                                                               int E, int bn, int* __restrict__ off,
-                                                               int* __restrict__ chunk_off,
-                                                               int* __restrict__ perm,
-                                                               int* __restrict__ inv,
-                                                               float* __restrict__ w_perm, int* err) {
-  extern __shared__ int sm[];
-  int* cnt = sm;                    // [E]
-  int* base = sm + E;               // [E] running base within expert
-  int* wcnt = sm + 2 * E;           // [32 warps][E]
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  for (int e = tid; e < E; e += kPermThreads) cnt[e] = 0;
+// All CTAs of the launch wait here until every CTA has arrived (the launch is
+// cooperative, so they are co-resident).  bar[0] counts arrivals, bar[1]
+// departures; the last CTA to leave zeroes both for the next launch.  Gives up
+// after kWaitLimitNs (error word kDevErrTimeout, returns false).
+__device__ __forceinline__ bool grid_barrier(int* bar, int nb, int* err) {
+  __shared__ int s_ok;
   __syncthreads();
-  for (int q = tid; q < P; q += kPermThreads) {
-    int e = idx[q];
-    if (e < 0 || e >= E) { set_error(err, kDevErrBadToken); e = 0; }
-    atomicAdd(&cnt[e], 1);
+  if (threadIdx.x == 0) {
+    red_release_gpu_add(bar, 1);
+    int ok = 1;
+    if (ld_acquire_gpu_s32(bar) < nb) {
+      const unsigned long long t0 = globaltimer_ns();
+      while (ld_acquire_gpu_s32(bar) < nb) {
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+          set_error(err, kDevErrTimeout);
+          ok = 0;
+          break;
+        }
+      }
+    }
+    if (atomicAdd(bar + 1, 1) == nb - 1) {
+      atomicExch(bar, 0);
+      atomicExch(bar + 1, 0);
+    }
+    s_ok = ok;
   }
   __syncthreads();
+  return s_ok != 0;
+}
+
+struct RouteParams {
+  const float* part;      // [KS, T, E] split-k router logits
+  const uint16_t* xn;     // [T, d] normalised rows (bf16)
+  int T, E, k, d, bn;     // bn: token chunk width of the grouped products
+  int tpc;                // tokens per CTA (CTA b owns tokens [b tpc, (b+1) tpc))
+  int* off;               // [E+1] first slot of each expert
+  int* chunk_off;         // [E+1] first chunk of each expert (chunks of bn slots)
+  int* perm;              // [P] slot -> pair (pair = token * k + j)
+  int* inv;               // [P] pair -> slot
+  float* w_perm;          // [P] routing weight of the slot's pair
+  uint16_t* xperm;        // [P, d] X_perm[slot] = xn[perm[slot] / k]
+  int* fill;              // [E] slots claimed per expert (zero between launches)
+  int* bar;               // [3] barrier and release counters (zero between launches)
+  int* dbg_idx;           // optional [T, k]
+  float* dbg_w;           // optional [T, k]
+  float* dbg_logits;      // optional [T, E]
+  int* err;
+};
+
+// The slots follow expert order.  Each CTA claims, per expert, a run of slots
+// for its pairs of that expert with one atomic add on fill[e] (before the
+// grid barrier, so the adds overlap the wait); after the barrier fill[] holds
+// the expert totals, which give the expert offsets.  Within a CTA's run the
+// pairs keep ascending pair order; the order of the runs of different CTAs
+// follows the atomics.  No result depends on it: every slot's expert row is
+// computed on its own, and the combine adds a token's k expert outputs in
+// the fixed order j = 0..k-1 through inv[].
+constexpr int kRouteThreads = 256;
+template <int KS>
+__global__ void __launch_bounds__(kRouteThreads) route_kernel(RouteParams p) {
+  extern __shared__ int rsm[];
+  const int E = p.E, k = p.k;
+  const int np_max = p.tpc * k;
+  int* s_e = rsm;                        // [np_max] expert of each local pair
+  float* s_w = (float*)(s_e + np_max);   // [np_max]
+  int* s_rank = (int*)(s_w + np_max);    // [np_max] rank among the CTA's pairs of its expert
+  int* s_slot = s_rank + np_max;         // [np_max]
+  int* s_cnt = s_slot + np_max;          // [E] the CTA's pairs per expert
+  int* s_bef = s_cnt + E;                // [E] first slot of the CTA's run within the expert
+  int* s_off = s_bef + E;                // [E+1]
+  int* s_tot = s_off + E + 1;            // [E]
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nw = kRouteThreads / 32;
+  const int b = blockIdx.x, nb = gridDim.x;
+  const int t0 = b * p.tpc;
+  const int nt = max(0, min(p.T, t0 + p.tpc) - t0);
+  const int np = nt * k;
+
+  // ---- top-k of the CTA's tokens ----
+  for (int lt = warp; lt < nt; lt += nw)
+    route_topk_token<KS>(p.part, p.T, E, k, t0 + lt, lane, s_e + lt * k, s_w + lt * k, p.dbg_idx, p.dbg_w,
+                         p.dbg_logits);
+  for (int e = tid; e < E; e += kRouteThreads) s_cnt[e] = 0;
+  __syncthreads();
+  // ---- stable ranks within the CTA: 32 pairs at a time in pair order ----
   if (warp == 0) {
-    // exclusive scans of the counts and chunk counts, 8 experts per lane (E <= 256)
+    for (int c0 = 0; c0 < np; c0 += 32) {
+      const int i = c0 + lane;
+      int e = i < np ? s_e[i] : -1;
+      if (e >= E || (i < np && e < 0)) { set_error(p.err, kDevErrBadToken); e = 0; }
+      const unsigned peers = __match_any_sync(0xffffffffu, e);
+      if (i < np) {
+        s_e[i] = e;
+        s_rank[i] = s_cnt[e] + __popc(peers & ((1u << lane) - 1));
+      }
+      __syncwarp();
+      if (i < np && (__ffs(peers) - 1) == lane) s_cnt[e] += __popc(peers);
+      __syncwarp();
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < E; e += kRouteThreads) {
+    const int c = s_cnt[e];
+    s_bef[e] = c ? atomicAdd(p.fill + e, c) : 0;
+  }
+
+  if (!grid_barrier(p.bar, nb, p.err)) return;
+
+  // ---- expert totals; the last CTA to read them zeroes fill[] ----
+  for (int e = tid; e < E; e += kRouteThreads) s_tot[e] = __ldcg(p.fill + e);
+  __syncthreads();
+  if (tid == 32 && atomicAdd(p.bar + 2, 1) == nb - 1) {
+    for (int e = 0; e < E; ++e) p.fill[e] = 0;
+    p.bar[2] = 0;
+  }
+  // exclusive scans of the counts and of the chunk counts (8 experts per lane)
+  if (warp == 0) {
     int c8[8], k8[8], sc = 0, sk = 0;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const int e = lane * 8 + j;
-      c8[j] = e < E ? cnt[e] : 0;
-      k8[j] = (c8[j] + bn - 1) / bn;
+      c8[j] = e < E ? s_tot[e] : 0;
+      k8[j] = (c8[j] + p.bn - 1) / p.bn;
       sc += c8[j];
       sk += k8[j];
     }
-    int ic = sc, ik = sk;  // inclusive lane sums
+    int ic = sc, ik = sk;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int a = __shfl_up_sync(0xffffffffu, ic, o), b2 = __shfl_up_sync(0xffffffffu, ik, o);
-      if (lane >= o) { ic += a; ik += b2; }
+      const int a = __shfl_up_sync(0xffffffffu, ic, o), a2 = __shfl_up_sync(0xffffffffu, ik, o);
+      if (lane >= o) { ic += a; ik += a2; }
     }
     int pc = ic - sc, pk = ik - sk;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const int e = lane * 8 + j;
-      if (e < E) { off[e] = pc; base[e] = pc; chunk_off[e] = pk; }
+      if (e < E) {
+        s_off[e] = pc;
+        if (b == 0) { p.off[e] = pc; p.chunk_off[e] = pk; }
+      }
       pc += c8[j];
       pk += k8[j];
     }
-    if (lane == 31) { off[E] = ic; chunk_off[E] = ik; }
+    if (lane == 31) {
+      s_off[E] = ic;
+      if (b == 0) { p.off[E] = ic; p.chunk_off[E] = ik; }
+    }
   }
   __syncthreads();
-  for (int c0 = 0; c0 < P; c0 += kPermThreads) {
-    const int q = c0 + tid;
-    int e = -1;
-    if (q < P) { e = idx[q]; if (e < 0 || e >= E) e = 0; }
-    for (int i = tid; i < 32 * E; i += kPermThreads) wcnt[i] = 0;
-    __syncthreads();
-    const unsigned peers = __match_any_sync(0xffffffffu, e);
-    const int rank_in_warp = __popc(peers & ((1u << lane) - 1));
-    if (e >= 0 && rank_in_warp == 0) wcnt[warp * E + e] = __popc(peers);
-    __syncthreads();
-    // exclusive scan over warps per expert (fixed order), then advance bases
-    for (int ee = tid; ee < E; ee += kPermThreads) {
-      int acc = base[ee];
-      for (int wv = 0; wv < 32; ++wv) {
-        const int c = wcnt[wv * E + ee];
-        wcnt[wv * E + ee] = acc;
-        acc += c;
-      }
-      base[ee] = acc;
-    }
-    __syncthreads();
-    if (e >= 0) {
-      const int slot = wcnt[warp * E + e] + rank_in_warp;
-      perm[slot] = q;
-      inv[q] = slot;
-      w_perm[slot] = w[q];
-    }
-    __syncthreads();
+  // ---- slots of the CTA's pairs ----
+  const int P = p.T * k;
+  for (int i = tid; i < np; i += kRouteThreads) {
+    const int e = s_e[i];
+    int slot = s_off[e] + s_bef[e] + s_rank[i];
+    if (slot < 0 || slot >= P) { set_error(p.err, kDevErrBadToken); slot = 0; }
+    const int q = t0 * k + i;
+    p.perm[slot] = q;
+    p.inv[q] = slot;
+    p.w_perm[slot] = s_w[i];
+    s_slot[i] = slot;
   }
+  __syncthreads();
+  // ---- gather: each 16-byte vector of a token row is loaded once and stored
+  // to the token's k slots; a thread's loads are all issued before its stores ----
+  const int nvec = p.d / 8;
+  const int nv_all = nt * nvec;
+  const uint4* src = reinterpret_cast<const uint4*>(p.xn + (long long)t0 * p.d);
+  for (int v0 = tid; v0 < nv_all; v0 += 4 * kRouteThreads) {
+    uint4 val[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int v = v0 + u * kRouteThreads;
+      if (v < nv_all) val[u] = __ldcg(src + v);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int v = v0 + u * kRouteThreads;
+      if (v < nv_all) {
+        const int lt = v / nvec, cv = v - lt * nvec;
+        for (int j = 0; j < k; ++j)
+          reinterpret_cast<uint4*>(p.xperm + (long long)s_slot[lt * k + j] * p.d)[cv] = val[u];
+      }
+    }
+  }
+}
+
+inline size_t route_smem_bytes(int tpc, int k, int E) {
+  return (size_t)tpc * k * 16 + (size_t)(4 * E + 1) * 4;
 }
 
 // chunk_off[g] = sum_{h < g} ceil((off[h+1] - off[h]) / bn)  (one thread)
@@ -412,17 +530,6 @@ __global__ void chunk_offsets_kernel(const int* __restrict__ off, int G, int bn,
     acc += n > 0 ? (n + bn - 1) / bn : 0;
   }
   chunk_off[G] = acc;
-}
-
-// X_perm[slot, :] = xn[perm[slot] / k, :]  (bf16 rows, 16-byte vectors)
-__global__ void gather_rows_kernel(const uint16_t* __restrict__ xn, const int* __restrict__ perm,
-                                   uint16_t* __restrict__ xp, int P, int k, int d) {
-  const int slot = blockIdx.x;
-  if (slot >= P) return;
-  const int t = perm[slot] / k;
-  const uint4* src = reinterpret_cast<const uint4*>(xn + (long long)t * d);
-  uint4* dst = reinterpret_cast<uint4*>(xp + (long long)slot * d);
-  for (int c = threadIdx.x; c < d / 8; c += blockDim.x) dst[c] = src[c];
 }
 
 // Mixture-of-experts combine + residual, fused with the next RMSNorm:
