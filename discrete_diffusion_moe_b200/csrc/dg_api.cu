@@ -191,7 +191,7 @@ WsLayout ws_layout(const dg_model_config& c, int batch, int num_sms) {
   L.attn_pml = take((size_t)L.attn_rows_cap * DG_CANVAS * c.n_q_heads * 2 * 4);
   L.rpart = take((size_t)L.ks_r * T * E * 4);
   L.rbar = take(64);
-  L.rfill = take(E * 4);
+  L.rfill = take(2 * E * 4);
   L.off = take((E + 1) * 4);
   L.choff = take((E + 1) * 4);
   L.perm = take(P * 4);
@@ -549,7 +549,7 @@ extern "C" dg_status dg_context_create(const dg_model_config* cfg, const void* d
   }
   cudaError_t e = cudaMemset(c->ws + c->L.err, 0, 64);
   if (e == cudaSuccess) e = cudaMemset(c->ws + c->L.rbar, 0, 64);
-  if (e == cudaSuccess) e = cudaMemset(c->ws + c->L.rfill, 0, (size_t)cfg->n_experts * 4);
+  if (e == cudaSuccess) e = cudaMemset(c->ws + c->L.rfill, 0, (size_t)cfg->n_experts * 8);
   if (e != cudaSuccess) {
     delete c;
     return fail(DG_ERR_CUDA, "cudaMemset: %s", cudaGetErrorString(e));
@@ -681,10 +681,12 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
       DG_TRY(run_gemm(ta, tb, p, e, c->num_sms, st, &c->n_launch));
     }
     {
-      const int v_blocks = B * Hkv * ((nq + kRopeVTok - 1) / kRopeVTok);
+      const int v_blocks = (int)(((long long)T * Hkv * (hd / 4) + 255) / 256);
       RopeParams rp{c->at<float>(L.qkv), ks_qkv, (long long)T * qkv_rows, c->at<double2>(L.rope),
                     c->at<uint16_t>(L.q), kc, vc, T, nq, L0, kv->c_max, Hq, Hkv, hd, v_blocks};
-      const int rot_blocks = T * ((Hq + Hkv + kRopeHeadsPerBlock - 1) / kRopeHeadsPerBlock);
+      if (ks_qkv > kRopeMaxSplits) return fail(DG_ERR_UNSUPPORTED, "QKV split count %d", ks_qkv);
+      const long long rot_threads = (long long)T * (Hq + Hkv) * (hd / 8);
+      const int rot_blocks = (int)((rot_threads + 255) / 256);
       rope_kv_kernel<<<rot_blocks + v_blocks, 256, 0, st>>>(rp);
       CNT(c);
     }
@@ -1089,7 +1091,7 @@ extern "C" dg_status dg_check_device_error(dg_ctx* c, void* stream) {
     DG_CUDA(cudaMemset(c->err(), 0, sizeof(int)));
     // a wait that ran out may have left the routing counters mid-count
     DG_CUDA(cudaMemset(c->ws + c->L.rbar, 0, 64));
-    DG_CUDA(cudaMemset(c->ws + c->L.rfill, 0, (size_t)c->cfg.n_experts * 4));
+    DG_CUDA(cudaMemset(c->ws + c->L.rfill, 0, (size_t)c->cfg.n_experts * 8));
     if (e == kDevErrBadToken) return fail(DG_ERR_BAD_TOKEN, "a token id outside [0, vocab) reached the device");
     if (e == kDevErrTimeout) return fail(DG_ERR_TIMEOUT, "a bounded device wait ran out");
     return fail(DG_ERR_CUDA, "device error word %d", e);

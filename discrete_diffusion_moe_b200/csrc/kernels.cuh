@@ -164,88 +164,91 @@ struct RopeParams {
   int v_blocks;       // blocks [0, v_blocks) transpose v; the rest rotate q and k
 };
 
-constexpr int kRopeVTok = 16;          // tokens per v-transpose block
-constexpr int kRopeHeadsPerBlock = 32; // q / k heads rotated per block
+constexpr int kRopeMaxSplits = 3; // split-k partials of the projection read by the kernel
 
-// Blocks [v_blocks, ...): one block per (token, group of up to 32 heads) rotates its
-// q heads (into the packed grouped-query layout) and k heads (into the
-// cache), one thread per rotated pair, the split-k partials summed in order.
-// Blocks [0, v_blocks) (scheduled first: they are the long ones): one block per
-// (canvas, kv head, 16 tokens) copies v into the transposed cache through
-// shared memory, so both the reads (along the head dimension) and the writes
-// (along positions) are contiguous; every thread issues the loads of several
-// elements before it uses them, so the block is not a chain of dependent
-// loads.
+// Blocks [v_blocks, ...): one thread per (token, q or k head, 4 consecutive
+// pairs) rotates the 4 pairs (i, i + hd/2) .. (i + 3, i + 3 + hd/2): 16-byte
+// loads of every split-k partial (summed in split order) and of the 4
+// (cos, sin), all issued before the first is used, then two 8-byte stores
+// (q into the packed grouped-query layout, k into the cache).
+// Threads [0, 256 v_blocks): one thread per (canvas, kv head, 4 consecutive
+// dims, position) moves 4 values of v into the transposed cache; the lanes of
+// a warp take consecutive positions, so each of the 4 stores of a warp is one
+// contiguous run along the cache's position axis.
 __global__ void __launch_bounds__(256) rope_kv_kernel(const RopeParams p) {
   const int half = p.hd / 2;
   const int row_w = (p.Hq + 2 * p.Hkv) * p.hd;
-  const int parts = (p.Hq + p.Hkv + kRopeHeadsPerBlock - 1) / kRopeHeadsPerBlock;
   const int rot_blk = (int)blockIdx.x - p.v_blocks;
   if (rot_blk >= 0) {
-    const int t = rot_blk / parts, part = rot_blk - t * parts;
-    const int G = p.Hq / p.Hkv;
+    const int n4 = half >> 2;  // groups of 4 pairs per head (hd % 8 == 0)
+    const int per_tok = (p.Hq + p.Hkv) * n4;
+    const long long gid = (long long)rot_blk * blockDim.x + threadIdx.x;
+    if (gid >= (long long)p.T * per_tok) return;
+    const int t = (int)(gid / per_tok);
+    const int rem = (int)(gid - (long long)t * per_tok);
+    const int h = rem / n4, i = (rem - h * n4) * 4;
     const int b = t / p.nq, pos_in = t - b * p.nq;
-    const int h0 = part * kRopeHeadsPerBlock;
-    const int n_pairs = (min(p.Hq + p.Hkv, h0 + kRopeHeadsPerBlock) - h0) * half;
-    const float* row = p.qkv + (long long)t * row_w;
-    const double2* tab = p.tab + (long long)pos_in * half;
-#pragma unroll 2
-    for (int j = threadIdx.x; j < n_pairs; j += blockDim.x) {
-      const int h = h0 + j / half, i = j - (h - h0) * half;
-      const float* src = row + h * p.hd + i;
-      float a1 = src[0], a2 = src[half];
-      for (int q = 1; q < p.ks; ++q) { a1 += src[q * p.split_stride]; a2 += src[q * p.split_stride + half]; }
-      const double2 cs = tab[i];
-      const double x1 = a1, x2 = a2;
-      const float o1 = (float)(x1 * cs.x - x2 * cs.y), o2 = (float)(x2 * cs.x + x1 * cs.y);
-      uint16_t* dst;
-      if (h < p.Hq) {
-        const int g = h / G, hh = h - g * G;
-        dst = p.q + ((((long long)b * p.Hkv + g) * p.nq + pos_in) * G + hh) * p.hd;
-      } else {
-        const int g = h - p.Hq;
-        dst = p.kc + (((long long)b * p.Hkv + g) * p.c_max + p.L0 + pos_in) * p.hd;
+    const float* src = p.qkv + (long long)t * row_w + h * p.hd + i;
+    float4 a1[kRopeMaxSplits], a2[kRopeMaxSplits];
+#pragma unroll
+    for (int q = 0; q < kRopeMaxSplits; ++q)
+      if (q < p.ks) {
+        a1[q] = __ldcg(reinterpret_cast<const float4*>(src + q * p.split_stride));
+        a2[q] = __ldcg(reinterpret_cast<const float4*>(src + q * p.split_stride + half));
       }
-      dst[i] = f32_to_bf16(o1);
-      dst[i + half] = f32_to_bf16(o2);
+    const double2* tab = p.tab + (long long)pos_in * half + i;
+    double2 cs[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) cs[u] = __ldg(tab + u);
+    float x1[4] = {a1[0].x, a1[0].y, a1[0].z, a1[0].w}, x2[4] = {a2[0].x, a2[0].y, a2[0].z, a2[0].w};
+#pragma unroll
+    for (int q = 1; q < kRopeMaxSplits; ++q)
+      if (q < p.ks) {
+        x1[0] += a1[q].x; x1[1] += a1[q].y; x1[2] += a1[q].z; x1[3] += a1[q].w;
+        x2[0] += a2[q].x; x2[1] += a2[q].y; x2[2] += a2[q].z; x2[3] += a2[q].w;
+      }
+    uint16_t o1[4], o2[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const double y1 = x1[u], y2 = x2[u];
+      o1[u] = f32_to_bf16((float)(y1 * cs[u].x - y2 * cs[u].y));
+      o2[u] = f32_to_bf16((float)(y2 * cs[u].x + y1 * cs[u].y));
     }
+    uint16_t* dst;
+    if (h < p.Hq) {
+      const int G = p.Hq / p.Hkv;
+      const int g = h / G, hh = h - g * G;
+      dst = p.q + ((((long long)b * p.Hkv + g) * p.nq + pos_in) * G + hh) * p.hd;
+    } else {
+      const int g = h - p.Hq;
+      dst = p.kc + (((long long)b * p.Hkv + g) * p.c_max + p.L0 + pos_in) * p.hd;
+    }
+    *reinterpret_cast<uint2*>(dst + i) =
+        make_uint2((uint32_t)o1[0] | ((uint32_t)o1[1] << 16), (uint32_t)o1[2] | ((uint32_t)o1[3] << 16));
+    *reinterpret_cast<uint2*>(dst + i + half) =
+        make_uint2((uint32_t)o2[0] | ((uint32_t)o2[1] << 16), (uint32_t)o2[2] | ((uint32_t)o2[3] << 16));
   } else {
-    __shared__ uint16_t tile[kRopeVTok * 256];  // [token][dim], hd <= 256
-    const int tiles_per_seq = (p.nq + kRopeVTok - 1) / kRopeVTok;
-    int blk = (int)blockIdx.x;
-    const int tt = blk % tiles_per_seq;
-    blk /= tiles_per_seq;
-    const int g = blk % p.Hkv, b = blk / p.Hkv;
-    const int pos0 = tt * kRopeVTok;
-    const int ntok = min(kRopeVTok, p.nq - pos0);
-    const int n = ntok * p.hd;
-    const float* base = p.qkv + (long long)(b * p.nq + pos0) * row_w + (p.Hq + p.Hkv + g) * p.hd;
-    constexpr int kPer = (kRopeVTok * 256 + 255) / 256;  // elements per thread at most
-    float a[kPer];
-    int off[kPer];
+    const int n4 = p.hd >> 2;
+    const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (gid >= (long long)(p.T / p.nq) * p.Hkv * n4 * p.nq) return;
+    const int pos = (int)(gid % p.nq);
+    long long rest = gid / p.nq;
+    const int d4 = (int)(rest % n4);
+    rest /= n4;
+    const int g = (int)(rest % p.Hkv), b = (int)(rest / p.Hkv);
+    const float* src = p.qkv + (long long)(b * p.nq + pos) * row_w + (p.Hq + p.Hkv + g) * p.hd + d4 * 4;
+    float4 a[kRopeMaxSplits];
 #pragma unroll
-    for (int u = 0; u < kPer; ++u) {
-      const int e = threadIdx.x + u * 256;
-      const int tok = e / p.hd, dim = e - tok * p.hd;
-      off[u] = tok * row_w + dim;
-      a[u] = e < n ? base[off[u]] : 0.f;
-    }
-    for (int q = 1; q < p.ks; ++q) {
+    for (int q = 0; q < kRopeMaxSplits; ++q)
+      if (q < p.ks) a[q] = __ldcg(reinterpret_cast<const float4*>(src + q * p.split_stride));
+    float v[4] = {a[0].x, a[0].y, a[0].z, a[0].w};
 #pragma unroll
-      for (int u = 0; u < kPer; ++u)
-        if (threadIdx.x + u * 256 < n) a[u] += base[q * p.split_stride + off[u]];
-    }
+    for (int q = 1; q < kRopeMaxSplits; ++q)
+      if (q < p.ks) { v[0] += a[q].x; v[1] += a[q].y; v[2] += a[q].z; v[3] += a[q].w; }
+    uint16_t* dst = p.vc + (((long long)b * p.Hkv + g) * p.hd + d4 * 4) * p.c_max + p.L0 + pos;
 #pragma unroll
-    for (int u = 0; u < kPer; ++u) {
-      const int e = threadIdx.x + u * 256;
-      if (e < n) tile[e] = bf16_to_f16(f32_to_bf16(a[u]));  // e = tok * hd + dim; the bf16 value, held in fp16
-    }
-    __syncthreads();
-    uint16_t* dst = p.vc + ((long long)b * p.Hkv + g) * p.hd * p.c_max + p.L0 + pos0;
-    for (int e = threadIdx.x; e < n; e += blockDim.x) {
-      const int dim = e / ntok, tok = e - dim * ntok;
-      dst[(long long)dim * p.c_max + tok] = tile[tok * p.hd + dim];
-    }
+    for (int u = 0; u < 4; ++u)
+      dst[(long long)u * p.c_max] = bf16_to_f16(f32_to_bf16(v[u]));  // the bf16 value, held in fp16
   }
 }
 
@@ -333,8 +336,9 @@ __device__ __forceinline__ void route_topk_token(const float* __restrict__ part,
 
 // All CTAs of the launch wait here until every CTA has arrived (the launch is
 // cooperative, so they are co-resident).  bar[0] counts arrivals, bar[1]
-// departures; the last CTA to leave zeroes both for the next launch.  Gives up
-// after kWaitLimitNs (error word kDevErrTimeout, returns false).
+// departures; the last CTA to leave zeroes both for the next launch and adds
+// 1 to bar[2], the count of completed barriers.  Gives up after kWaitLimitNs
+// (error word kDevErrTimeout, returns false).
 __device__ __forceinline__ bool grid_barrier(int* bar, int nb, int* err) {
   __shared__ int s_ok;
   __syncthreads();
@@ -354,6 +358,7 @@ __device__ __forceinline__ bool grid_barrier(int* bar, int nb, int* err) {
     if (atomicAdd(bar + 1, 1) == nb - 1) {
       atomicExch(bar, 0);
       atomicExch(bar + 1, 0);
+      atomicAdd(bar + 2, 1);
     }
     s_ok = ok;
   }
@@ -372,8 +377,8 @@ struct RouteParams {
   int* inv;               // [P] pair -> slot
   float* w_perm;          // [P] routing weight of the slot's pair
   uint16_t* xperm;        // [P, d] X_perm[slot] = xn[perm[slot] / k]
-  int* fill;              // [E] slots claimed per expert (zero between launches)
-  int* bar;               // [3] barrier and release counters (zero between launches)
+  int* fill;              // [2, E] slots claimed per expert, two buffers
+  int* bar;               // [3] grid barrier counters and completed-barrier count
   int* dbg_idx;           // optional [T, k]
   float* dbg_w;           // optional [T, k]
   float* dbg_logits;      // optional [T, E]
@@ -383,7 +388,9 @@ struct RouteParams {
 // The slots follow expert order.  Each CTA claims, per expert, a run of slots
 // for its pairs of that expert with one atomic add on fill[e] (before the
 // grid barrier, so the adds overlap the wait); after the barrier fill[] holds
-// the expert totals, which give the expert offsets.  Within a CTA's run the
+// the expert totals, which give the expert offsets.  Launches alternate
+// between the two fill buffers by the parity of the completed-barrier count;
+// CTA 0 zeroes the buffer of the previous launch, which the next one uses.  Within a CTA's run the
 // pairs keep ascending pair order; the order of the runs of different CTAs
 // follows the atomics.  No result depends on it: every slot's expert row is
 // computed on its own, and the combine adds a token's k expert outputs in
@@ -407,6 +414,10 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(RouteParams p) {
   const int t0 = b * p.tpc;
   const int nt = max(0, min(p.T, t0 + p.tpc) - t0);
   const int np = nt * k;
+  const int ep = __ldcg(p.bar + 2) & 1;  // this launch's fill buffer
+  int* fill = p.fill + ep * E;
+  if (b == 0)
+    for (int e = tid; e < E; e += kRouteThreads) p.fill[(ep ^ 1) * E + e] = 0;
 
   // ---- top-k of the CTA's tokens ----
   for (int lt = warp; lt < nt; lt += nw)
@@ -433,18 +444,14 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(RouteParams p) {
   __syncthreads();
   for (int e = tid; e < E; e += kRouteThreads) {
     const int c = s_cnt[e];
-    s_bef[e] = c ? atomicAdd(p.fill + e, c) : 0;
+    s_bef[e] = c ? atomicAdd(fill + e, c) : 0;
   }
 
   if (!grid_barrier(p.bar, nb, p.err)) return;
 
-  // ---- expert totals; the last CTA to read them zeroes fill[] ----
-  for (int e = tid; e < E; e += kRouteThreads) s_tot[e] = __ldcg(p.fill + e);
+  // ---- expert totals ----
+  for (int e = tid; e < E; e += kRouteThreads) s_tot[e] = __ldcg(fill + e);
   __syncthreads();
-  if (tid == 32 && atomicAdd(p.bar + 2, 1) == nb - 1) {
-    for (int e = 0; e < E; ++e) p.fill[e] = 0;
-    p.bar[2] = 0;
-  }
   // exclusive scans of the counts and of the chunk counts (8 experts per lane)
   if (warp == 0) {
     int c8[8], k8[8], sc = 0, sk = 0;
