@@ -11,7 +11,7 @@
 // [nq * G, hd] matrix, so one tile of K / V^T feeds every head of the group.
 //
 //   warp 0      TMA: the Q tile once, then K tile and V^T tile per stage
-//               (two stages); the V^T map's key extent is the number of valid
+//               (three stages); the V^T map's key extent is the number of valid
 //               keys, so keys past it arrive as zeros
 //   warp 1      tensor memory owner and MMA issuer:
 //                 S  = Q K^T            (M 128, N 64, K hd)    -> TMEM cols [0, 64)
@@ -29,8 +29,10 @@
 //               into shared memory in the 128-byte-swizzled K-major layout the
 //               MMA reads (the V^T cache holds the bf16-rounded values in
 //               fp16, exact above 2^-14, for this product);
-//               finally read O and write the normalised bf16 output or the
-//               split's unnormalised partial (with its max and sum).
+//               finally read O and write the normalised bf16 output, or
+//               stage the split's unnormalised partial in the freed K/V
+//               memory and store it with one bulk copy per 32 rows (with its
+//               max and sum).
 //
 // Every mbarrier wait is bounded; a thread whose wait ran out sets the error
 // word and stops issuing work, and the tensor memory is released only after
@@ -66,7 +68,13 @@ struct AttnTcShape {
   static constexpr uint32_t K_BYTES = NA * kAttnKeys * 128;
   static constexpr uint32_t V_BYTES = HD * 128;      // hd rows x 64 keys
   static constexpr uint32_t P_BYTES = kAttnRows * 128;
-  static constexpr size_t SMEM = 1024 + Q_BYTES + 2 * (K_BYTES + V_BYTES) + P_BYTES + 16 * 8 + 6 * 128 * 4;
+  static constexpr size_t FIXED = 1024 + Q_BYTES + 2 * P_BYTES + 24 * 8 + 6 * 128 * 4;
+  // K/V stages: three where they fit (the load of tile i + 3 is in flight while
+  // tiles i + 1, i + 2 are multiplied), else two
+  static constexpr int KV_STAGES = FIXED + 3 * (K_BYTES + V_BYTES) <= 227 * 1024 ? 3 : 2;
+  static constexpr size_t SMEM = FIXED + KV_STAGES * (K_BYTES + V_BYTES);
+  // the K/V stages hold the final O tile (fp32 rows) for its bulk store
+  static_assert((size_t)KV_STAGES * (K_BYTES + V_BYTES) >= (size_t)kAttnRows * HD * 4, "O staging");
   static constexpr uint32_t TMEM_COLS = (64 + HD) <= 128 ? 128 : 256;
 };
 
@@ -140,21 +148,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sQ = smem;
-  uint8_t* sK = sQ + S::Q_BYTES;               // 2 stages
-  uint8_t* sV = sK + 2 * S::K_BYTES;           // 2 stages
-  uint8_t* sP = sV + 2 * S::V_BYTES;           // P (fp16)
-  uint64_t* bars = (uint64_t*)(sP + S::P_BYTES);
+  constexpr int NS = S::KV_STAGES;
+  uint8_t* sK = sQ + S::Q_BYTES;               // NS stages
+  uint8_t* sV = sK + NS * S::K_BYTES;          // NS stages
+  uint8_t* sP = sV + NS * S::V_BYTES;          // P (fp16), two buffers by tile parity
+  uint64_t* bars = (uint64_t*)(sP + 2 * S::P_BYTES);
   uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;   // [2]
-  uint64_t* kv_empty = bars + 3;  // [2]
-  uint64_t* s_full = bars + 5;
-  uint64_t* s_free = bars + 6;
-  uint64_t* p_full = bars + 7;
-  uint64_t* pv_done = bars + 8;
-  uint64_t* drain = bars + 9;
-  uint64_t* pair_bar = bars + 10;  // [4] per tensor-memory lane quarter: the two halves of a row
-  uint32_t* tmem_slot = (uint32_t*)(bars + 14);
-  float* xchg = (float*)(bars + 16);  // [2 tile parities][2 halves][128 rows] maxima, then [2][128] sums
+  uint64_t* kv_full = bars + 1;        // [NS]
+  uint64_t* kv_empty = bars + 1 + NS;  // [NS]
+  uint64_t* s_full = bars + 1 + 2 * NS;
+  uint64_t* s_free = s_full + 1;
+  uint64_t* p_full = s_full + 2;      // [2] by tile parity
+  uint64_t* pv_done = s_full + 4;     // [2] by tile parity
+  uint64_t* drain = s_full + 6;
+  uint64_t* pair_bar = s_full + 7;     // [4] per tensor-memory lane quarter: the two halves of a row
+  uint32_t* tmem_slot = (uint32_t*)(s_full + 11);
+  float* xchg = (float*)(s_full + 13);  // [2 tile parities][2 halves][128 rows] maxima, then [2][128] sums
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.Hq / p.Hkv;
@@ -175,15 +184,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(q_full), 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < NS; ++s) {
       mbar_init(smem_u32(&kv_full[s]), 1);
       mbar_init(smem_u32(&kv_empty[s]), 1);
     }
     mbar_init(smem_u32(s_full), 1);
     mbar_init(smem_u32(s_free), 256);
-    mbar_init(smem_u32(p_full), 256);
+    mbar_init(smem_u32(&p_full[0]), 256);
+    mbar_init(smem_u32(&p_full[1]), 256);
     for (int q = 0; q < 4; ++q) mbar_init(smem_u32(&pair_bar[q]), 64);
-    mbar_init(smem_u32(pv_done), 1);
+    mbar_init(smem_u32(&pv_done[0]), 1);
+    mbar_init(smem_u32(&pv_done[1]), 1);
     mbar_init(smem_u32(drain), 1);
     fence_mbar_init();
     fence_proxy_async_smem();
@@ -210,8 +221,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       for (int a = 0; a < S::NA; ++a) tma_load_2d(smem_u32(sQ + a * 16384), &tmQ, qb, a * 64, q_row0);
       int issued = 0;
       for (int i = 0; i < n_tiles; ++i, ++issued) {
-        const int s = i & 1;
-        if (!mbar_wait(smem_u32(&kv_empty[s]), ((i >> 1) & 1) ^ 1, p.err)) break;
+        const int s = i % NS;
+        if (!mbar_wait(smem_u32(&kv_empty[s]), ((i / NS) & 1) ^ 1, p.err)) break;
         const uint32_t fb = smem_u32(&kv_full[s]);
         mbar_arrive_expect_tx(fb, S::K_BYTES + S::V_BYTES);
         const int key0 = (kt0 + i) * kAttnKeys;
@@ -221,9 +232,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tma_load_2d(smem_u32(sV + s * S::V_BYTES), &tmV, fb, key0, bg * HD);
       }
       // every issued copy must land before the CTA may exit
-      const int first = issued > 2 ? issued - 2 : 0;
+      const int first = issued > NS ? issued - NS : 0;
       mbar_wait(qb, 0, p.err);
-      for (int i = first; i < issued; ++i) mbar_wait(smem_u32(&kv_full[i & 1]), (i >> 1) & 1, p.err);
+      for (int i = first; i < issued; ++i) mbar_wait(smem_u32(&kv_full[i % NS]), (i / NS) & 1, p.err);
     }
   } else if (warp == 1) {
     if (lane == 0 && n_tiles > 0) {
@@ -232,8 +243,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint32_t id_o = idesc_f16_f32(128, HD);
       bool ok = mbar_wait(smem_u32(q_full), 0, p.err);
       auto issue_s = [&](int i) -> bool {
-        const int s = i & 1;
-        if (!mbar_wait(smem_u32(&kv_full[s]), (i >> 1) & 1, p.err)) return false;
+        const int s = i % NS;
+        if (!mbar_wait(smem_u32(&kv_full[s]), (i / NS) & 1, p.err)) return false;
         if (i > 0 && !mbar_wait(smem_u32(s_free), (i - 1) & 1, p.err)) return false;
         tc_fence_after();
         const uint32_t qa = smem_u32(sQ), ka = smem_u32(sK + s * S::K_BYTES);
@@ -249,15 +260,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (ok) ok = issue_s(0);
       for (int i = 0; i < n_tiles && ok; ++i) {
         if (i + 1 < n_tiles && !issue_s(i + 1)) { ok = false; break; }
-        if (!mbar_wait(smem_u32(p_full), i & 1, p.err)) { ok = false; break; }
+        if (!mbar_wait(smem_u32(&p_full[i & 1]), (i >> 1) & 1, p.err)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t va = smem_u32(sV + (i & 1) * S::V_BYTES);
-        const uint32_t pa = smem_u32(sP);
+        const uint32_t va = smem_u32(sV + (i % NS) * S::V_BYTES);
+        const uint32_t pa = smem_u32(sP + (i & 1) * S::P_BYTES);
 #pragma unroll
         for (int k = 0; k < kAttnKeys / 16; ++k)
           umma_bf16(t_o, sdesc_k128(pa + k * 32), sdesc_k128(va + k * 32), id_o, (i > 0 || k > 0) ? 1u : 0u);
-        umma_commit(smem_u32(pv_done));
-        umma_commit(smem_u32(&kv_empty[i & 1]));
+        umma_commit(smem_u32(&pv_done[i & 1]));
+        umma_commit(smem_u32(&kv_empty[i % NS]));
       }
       umma_commit(smem_u32(drain));
       mbar_wait(smem_u32(drain), 0, p.err);
@@ -274,7 +285,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const float scale = p.scale_log2;
     float m = -INFINITY, l = 0.f;  // reference max (scaled, log2 units) and this half's sum
     bool ok = true;
-    uint8_t* p_s = sP;
     const uint32_t prow = (uint32_t)row * 128;
     const uint32_t pb = smem_u32(&pair_bar[quarter]);
     constexpr int NCH = HD / 16;
@@ -330,11 +340,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       l = l * alpha + ((sq[0] + sq[1]) + (sq[2] + sq[3]));
       m = m_new;
-      // P of the previous tile has been consumed and O is up to date
-      if (i > 0) {
-        if (!wait_all(smem_u32(pv_done), (i - 1) & 1)) { ok = false; break; }
+      // O rescale: every product into O so far (up to tile i - 1) has completed
+      if (i > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        if (!wait_all(smem_u32(&pv_done[(i - 1) & 1]), ((i - 1) >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+        {
           for (int c = oc0; c < oc1; ++c) {
             float v[16];
             tmem_ld16(t_o + lane_off + c * 16, v);
@@ -345,7 +355,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           tmem_wait_st();
         }
       }
+      // this P buffer was last read by the product of tile i - 2
+      if (i > 1) {
+        if (!wait_all(smem_u32(&pv_done[i & 1]), ((i - 2) >> 1) & 1)) { ok = false; break; }
+      }
       // P rows (fp16) into the swizzled K-major operand tile
+      uint8_t* p_s = sP + (i & 1) * S::P_BYTES;
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
         const int ch = half * 4 + cc;
@@ -357,9 +372,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(smem_u32(p_full));
+      mbar_arrive(smem_u32(&p_full[i & 1]));
     }
-    if (ok && n_tiles > 0) ok = wait_all(smem_u32(pv_done), (n_tiles - 1) & 1);
+    if (ok && n_tiles > 0) ok = wait_all(smem_u32(&pv_done[(n_tiles - 1) & 1]), ((n_tiles - 1) >> 1) & 1);
     tc_fence_after();
     // total sum of the row: both halves used the same reference max
     float* xl = xchg + 512;
@@ -370,33 +385,70 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const bool valid = r < rows_total;
     const int h = g * G + (valid ? r % G : 0);
     const float inv = (have && l_row > 0.f) ? 1.f / l_row : 0.f;
-    const long long prow_g = (((long long)split * p.B + b) * p.Hq + h) * p.nq + t_in;
-    for (int c = oc0; c < oc1; ++c) {
-      float v[16];
-      if (have) {
-        tmem_ld16(t_o + lane_off + c * 16, v);
-      } else {
+    if (p.splits == 1) {
+      for (int c = oc0; c < oc1; ++c) {
+        float v[16];
+        if (have) {
+          tmem_ld16(t_o + lane_off + c * 16, v);
+        } else {
 #pragma unroll
-        for (int e = 0; e < 16; ++e) v[e] = 0.f;
-      }
-      if (!valid) continue;
-      if (p.splits == 1) {
+          for (int e = 0; e < 16; ++e) v[e] = 0.f;
+        }
+        if (!valid) continue;
         uint16_t* dst = p.out + ((long long)(b * p.nq + t_in) * p.Hq + h) * HD + c * 16;
         uint32_t w[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) w[e] = pack_bf16x2(v[2 * e] * inv, v[2 * e + 1] * inv);
         *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
         *reinterpret_cast<uint4*>(dst + 8) = make_uint4(w[4], w[5], w[6], w[7]);
-      } else {
-        float* dst = p.part_o + prow_g * HD + c * 16;
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          *reinterpret_cast<float4*>(dst + 4 * e) = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
       }
-    }
-    if (valid && p.splits > 1 && half == 0) {
-      p.part_ml[prow_g * 2] = have ? m : -INFINITY;
-      p.part_ml[prow_g * 2 + 1] = have ? l_row : 0.f;
+    } else {
+      // split partial: the unnormalised O rows (fp32) are staged in the K/V
+      // stage memory (every tensor-core operation and copy into it has
+      // completed) and leave in bulk copies of the tile's valid rows; the
+      // partial rows follow the packed query order [split][b][g][row]
+      float* so = reinterpret_cast<float*>(sK) + (size_t)row * HD;
+      // all of this half's O chunks are loaded before the one wait
+      constexpr int MAXC = (NCH + 1) / 2;
+      uint32_t rr[MAXC][16];
+#pragma unroll
+      for (int q = 0; q < MAXC; ++q)
+#pragma unroll
+        for (int e = 0; e < 16; ++e) rr[q][e] = 0u;
+      if (have) {
+#pragma unroll
+        for (int q = 0; q < MAXC; ++q)
+          if (oc0 + q < oc1) tmem_ld16_nowait(t_o + lane_off + (oc0 + q) * 16, rr[q]);
+#pragma unroll
+        for (int q = 0; q < MAXC; ++q)
+          if (oc0 + q < oc1) tmem_wait_ld16(rr[q]);
+      }
+#pragma unroll
+      for (int q = 0; q < MAXC; ++q)
+        if (oc0 + q < oc1) {
+          float4* d4 = reinterpret_cast<float4*>(so + (oc0 + q) * 16);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            d4[e] = make_float4(__uint_as_float(rr[q][4 * e]), __uint_as_float(rr[q][4 * e + 1]),
+                                __uint_as_float(rr[q][4 * e + 2]), __uint_as_float(rr[q][4 * e + 3]));
+        }
+      const long long prow_g = (((long long)split * p.B + b) * p.Hkv + g) * rows_total + r;
+      if (valid && half == 0) {
+        p.part_ml[prow_g * 2] = have ? m : -INFINITY;
+        p.part_ml[prow_g * 2 + 1] = have ? l_row : 0.f;
+      }
+      // each lane quarter's 32 rows leave in their own bulk copy once both
+      // halves have staged them
+      fence_proxy_async_smem();
+      mbar_arrive(pb);
+      const bool staged = wait_all(pb, (n_tiles + 1) & 1);
+      const int q0 = r0 + quarter * 32;
+      const int nvalid = min(32, rows_total - q0);
+      if (staged && half == 0 && lane == 0 && nvalid > 0) {
+        float* dst = p.part_o + ((((long long)split * p.B + b) * p.Hkv + g) * rows_total + q0) * HD;
+        bulk_store_wait_read(dst, smem_u32(reinterpret_cast<float*>(sK) + (size_t)quarter * 32 * HD),
+                             (uint32_t)nvalid * HD * 4);
+      }
     }
   }
 
@@ -408,37 +460,62 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
 // Merge split-KV partials (fixed split order) -> bf16 output.  One warp per
 // (canvas, head, query) row: the split maxima and sums are read once per row,
-// the row's HD values are merged with 16-byte vector loads.
+// the row's HD values are merged with 16-byte vector loads.  Partial rows are
+// in packed query order: [split][b][g][token * G + head-in-group].
+// MAXS: the largest split count the instantiation handles (4 or 8).
+template <int MAXS>
 __global__ void attn_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml,
-                                    uint16_t* __restrict__ out, int splits, int B, int Hq, int nq, int HD) {
+                                    uint16_t* __restrict__ out, int splits, int B, int Hq, int Hkv, int nq,
+                                    int HD) {
   const long long rows = (long long)B * Hq * nq;
   const long long row = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
-  float mx = -INFINITY;
-  for (int s = 0; s < splits; ++s) mx = fmaxf(mx, part_ml[(s * rows + row) * 2]);
-  float wgt[8];
-  float den = 0.f;
-#pragma unroll
-  for (int s = 0; s < 8; ++s) {
-    wgt[s] = 0.f;
-    if (s < splits) {
-      const float ms = part_ml[(s * rows + row) * 2];
-      if (ms != -INFINITY) wgt[s] = exp2f(ms - mx);
-      den += wgt[s] * part_ml[(s * rows + row) * 2 + 1];
-    }
-  }
-  const float inv = den > 0.f ? 1.f / den : 0.f;
   const int i = (int)(row % nq);
   const long long bh = row / nq;
   const int h = (int)(bh % Hq), b = (int)(bh / Hq);
+  const int G = Hq / Hkv, g = h / G;
+  const long long prow = (((long long)b * Hkv + g) * nq + i) * G + (h - g * G);
+  // every load (the split maxima and sums, and this lane's partial O vectors
+  // of every split) is issued before the first is used
+  constexpr int kMaxVec = 2;  // 16-byte vectors per lane and split (HD <= 256)
+  float2 ml[MAXS];
+  float4 po[MAXS][kMaxVec];
+#pragma unroll
+  for (int s = 0; s < MAXS; ++s)
+    if (s < splits) {
+      ml[s] = *reinterpret_cast<const float2*>(part_ml + (s * rows + prow) * 2);
+#pragma unroll
+      for (int u = 0; u < kMaxVec; ++u) {
+        const int c = lane * 4 + u * 128;
+        if (c < HD) po[s][u] = *reinterpret_cast<const float4*>(part_o + (s * rows + prow) * HD + c);
+      }
+    }
+  float mx = -INFINITY;
+#pragma unroll
+  for (int s = 0; s < MAXS; ++s)
+    if (s < splits) mx = fmaxf(mx, ml[s].x);
+  float wgt[MAXS];
+  float den = 0.f;
+#pragma unroll
+  for (int s = 0; s < MAXS; ++s) {
+    wgt[s] = 0.f;
+    if (s < splits) {
+      if (ml[s].x != -INFINITY) wgt[s] = exp2f(ml[s].x - mx);
+      den += wgt[s] * ml[s].y;
+    }
+  }
+  const float inv = den > 0.f ? 1.f / den : 0.f;
   uint16_t* dst = out + ((long long)(b * nq + i) * Hq + h) * HD;
-  for (int c = lane * 4; c < HD; c += 128) {
+#pragma unroll
+  for (int u = 0; u < kMaxVec; ++u) {
+    const int c = lane * 4 + u * 128;
+    if (c >= HD) break;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int s = 0; s < 8; ++s)
+    for (int s = 0; s < MAXS; ++s)
       if (s < splits) {
-        const float4 v = *reinterpret_cast<const float4*>(part_o + (s * rows + row) * HD + c);
+        const float4 v = po[s][u];
         acc.x += wgt[s] * v.x; acc.y += wgt[s] * v.y; acc.z += wgt[s] * v.z; acc.w += wgt[s] * v.w;
       }
     uint2 o;

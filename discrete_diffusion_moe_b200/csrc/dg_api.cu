@@ -599,8 +599,11 @@ static dg_status run_attention(const uint16_t* q, const uint16_t* kc, const uint
   if (launches) ++*launches;
   if (splits > 1) {
     const long long rows = (long long)B * Hq * nq;
-    attn_combine_kernel<<<(unsigned)((rows * 32 + 255) / 256), 256, 0, st>>>(part_o, part_ml, out, splits, B, Hq,
-                                                                             nq, hd);
+    const unsigned cgrid = (unsigned)((rows * 32 + 255) / 256);
+    if (splits <= 4)
+      attn_combine_kernel<4><<<cgrid, 256, 0, st>>>(part_o, part_ml, out, splits, B, Hq, Hkv, nq, hd);
+    else
+      attn_combine_kernel<8><<<cgrid, 256, 0, st>>>(part_o, part_ml, out, splits, B, Hq, Hkv, nq, hd);
     DG_CUDA(cudaGetLastError());
     if (launches) ++*launches;
   }
