@@ -124,8 +124,9 @@ struct WsLayout {
   long long epart_rows;
 };
 
-constexpr int kRouterSplits = 4;  // split-k of the router product (needs d_model >= 256)
-int router_splits(const dg_model_config&) { return kRouterSplits; }
+// split-k of the router product: 8 from 16 k-blocks on (d_model >= 1024), else 4
+// (d_model >= 256); the routing kernel is built for both
+int router_splits(const dg_model_config& c) { return c.d_model >= 1024 ? 8 : 4; }
 
 // Token columns per unit of the QKV and output projections: 128 from 256
 // tokens on (two CTAs share an SM, each weight tile is read by two CTAs at the
@@ -728,7 +729,7 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
       EpiStoreT e{c->at<float>(L.rpart), E, (long long)T * E, 0, nullptr, nullptr, 0, err};
       DG_TRY(run_gemm(ta, tb, p, e, c->num_sms, st, &c->n_launch));
     }
-    if (L.ks_r != kRouterSplits) return fail(DG_ERR_UNSUPPORTED, "router split count %d", L.ks_r);
+    if (L.ks_r != 4 && L.ks_r != 8) return fail(DG_ERR_UNSUPPORTED, "router split count %d", L.ks_r);
     {
       // top-k, counting sort by expert and row gather in one cooperative launch
       RouteParams rp;
@@ -759,7 +760,8 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
       lc.stream = st;
       lc.attrs = at;
       lc.numAttrs = 1;
-      DG_CUDA(cudaLaunchKernelEx(&lc, route_kernel<kRouterSplits>, rp));
+      if (L.ks_r == 8) DG_CUDA(cudaLaunchKernelEx(&lc, route_kernel<8>, rp));
+      else             DG_CUDA(cudaLaunchKernelEx(&lc, route_kernel<4>, rp));
       CNT(c);
     }
     {

@@ -122,13 +122,14 @@ struct EpiDown {
     float w[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) w[i] = i < nv ? __ldg(w_slot + j.n0 + c0 + i) : 0.f;
+    // plain stores: the combine reads y next, from L2
     if (nv >= 16) {
 #pragma unroll
-      for (int i = 0; i < 16; ++i) __stcs(y + (long long)(j.n0 + c0 + i) * d + f, w[i] * v[i]);
+      for (int i = 0; i < 16; ++i) y[(long long)(j.n0 + c0 + i) * d + f] = w[i] * v[i];
     } else {
 #pragma unroll
       for (int i = 0; i < 16; ++i)
-        if (i < nv) __stcs(y + (long long)(j.n0 + c0 + i) * d + f, w[i] * v[i]);
+        if (i < nv) y[(long long)(j.n0 + c0 + i) * d + f] = w[i] * v[i];
     }
   }
 };
