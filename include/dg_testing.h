@@ -49,7 +49,8 @@ dg_status dg_test_grouped_gemm(const uint16_t* d_a, int32_t rows_per_group, int3
    (token-major).  causal = 0: every query sees all L0 + nq keys; causal = 1:
    query i sees keys [0, L0 + i].  splits (1..8; 0 means 1) key splits; for
    splits > 1 the partial buffers come from the caller: part_o fp32
-   [splits * B * Hq * nq * hd] and part_ml fp32 [splits * B * Hq * nq * 2].
+   [splits * B * Hq * nq * hd] and part_ml fp32 [splits * B * Hq * nq * 2],
+   rows in packed query order [split][b][kv head][token * G + head in group].
    head_dim one of 32, 64, 128, 176.  Synchronous. */
 dg_status dg_test_attention(const uint16_t* d_q, const uint16_t* d_k, const uint16_t* d_v, uint16_t* d_out,
                             int32_t B, int32_t nq, int32_t L0, int32_t c_max, int32_t Hq, int32_t Hkv,
@@ -60,8 +61,7 @@ dg_status dg_test_attention(const uint16_t* d_q, const uint16_t* d_k, const uint
    workspace (for inspecting the last layer's intermediates after a call):
    "x" fp32 residual [T, d], "xn" bf16 normed activations, "qkv" fp32,
    "q" bf16 [T, Hq*hd], "attn" bf16 [T, Hq*hd], "rpart" fp32 split-k router
-   partial logits [splits, T, E], "idx" int32 [T, k],
-   "w" fp32 [T, k], "off" int32 [E+1], "perm", "inv" int32 [T*k],
+   partial logits [splits, T, E], "off" int32 [E+1], "perm", "inv" int32 [T*k],
    "wperm" fp32 [T*k], "xperm" bf16 [T*k, d], "hperm" bf16 [T*k, f],
    "yperm" fp32 [T*k, d], "logits" fp32 [T, V], "probs" bf16 [T, V]. */
 dg_status dg_test_workspace_buffer(dg_ctx* ctx, const char* name, void** d_ptr, size_t* bytes);
