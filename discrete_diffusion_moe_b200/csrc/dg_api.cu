@@ -325,7 +325,7 @@ dg_status run_gemm(const CUtensorMap& ta, const BOperand& tb, GemmPlan p, const 
   else units = (long long)((p.m_tiles + p.mt - 1) / p.mt) * ((p.n_total + p.bn - 1) / p.bn) * p.k_splits;
   if (units <= 0) return DG_OK;
   const int grid = (int)std::min<long long>(units, (long long)ctas * num_sms);
-  gemm_tc_kernel<Epi><<<grid, kGemmThreads, smem, st>>>(ta, tb.maps, p, epi, stages);
+  gemm_tc_kernel<Epi><<<grid, gemm_threads<Epi>(), smem, st>>>(ta, tb.maps, p, epi, stages);
   DG_CUDA(cudaGetLastError());
   if (launches) ++*launches;
   return DG_OK;
@@ -1166,6 +1166,7 @@ extern "C" dg_status dg_profile_stop(dg_ctx* c, dg_profile* out) {
 // test hooks
 namespace {
 struct EpiGroupedT {
+  static constexpr int kEpiWarps = 8;
   float* out;
   int ld;
   struct State {};
@@ -1182,6 +1183,7 @@ struct EpiGroupedT {
 
 // row-major store; k split s writes the matrix at D + s * M * N
 struct EpiSplitRows {
+  static constexpr int kEpiWarps = 8;
   float* out;
   long long M, N;
   struct State {};

@@ -16,6 +16,7 @@ namespace dg {
 //   mode 1: out += D           (residual add)
 //   mode 2: out  = E_emb[tok[t], f] + D   (canvas embedding + self-conditioning)
 struct EpiStoreT {
+  static constexpr int kEpiWarps = 8;
   float* out;
   long long ld;
   long long split_stride;
@@ -78,6 +79,7 @@ struct EpiStoreT {
 // divisions of different columns overlap instead of running one column at a
 // time behind a branch.
 struct EpiSwiGLU {
+  static constexpr int kEpiWarps = 8;
   uint16_t* h;   // [rows, f_dim] bf16, rows in expert (permuted) order
   int f_dim;
   struct State {};
@@ -108,6 +110,7 @@ struct EpiSwiGLU {
 
 // Grouped down projection: y[slot, f] = w[slot] * D (fp32), f = output feature.
 struct EpiDown {
+  static constexpr int kEpiWarps = 8;
   float* y;
   int d;
   const float* w_slot;
@@ -153,6 +156,7 @@ struct VocabPartials {
 };
 
 struct EpiLMHead {
+  static constexpr int kEpiWarps = 4;
   float* logits;         // [T, V]
   long long V;
   VocabPartials part;    // each [T, n_vt]
@@ -231,6 +235,7 @@ struct EpiLMHead {
 
 // Plain row-major store D[m, n] -> out[m * ld + n] (the GEMM test hook).
 struct EpiStoreRows {
+  static constexpr int kEpiWarps = 8;
   float* out;
   long long ld;
   struct State {};

@@ -146,7 +146,11 @@ __device__ __forceinline__ GemmJob gemm_job(const GemmPlan& p, const GemmTables&
   return j;
 }
 
-constexpr int kGemmThreads = 192;
+// Threads of a CTA: warp 0 copies, warp 1 issues the MMAs, Epi::kEpiWarps
+// warps (4 or 8) drain the accumulators.  With 8, warps w and w + 4 read the
+// same tensor-memory lane quarter (rows) and take alternate 16-column chunks.
+template <class Epi>
+__host__ __device__ constexpr int gemm_threads() { return 64 + 32 * Epi::kEpiWarps; }
 constexpr int kATileBytes = 128 * 128;  // 128 rows x 64 bf16
 
 // B tensor maps: boxes of b_rows[0] / b_rows[1] / b_rows[2] rows
@@ -155,7 +159,7 @@ struct BMaps {
 };
 
 template <class Epi>
-__global__ void __launch_bounds__(kGemmThreads, 2)
+__global__ void __launch_bounds__(gemm_threads<Epi>(), 2)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ BMaps tmB,
                    const GemmPlan p, const Epi epi, const int stages) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -189,7 +193,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(smem_u32(&acc_full[a]), 1);
-      mbar_init(smem_u32(&acc_empty[a]), 128);
+      mbar_init(smem_u32(&acc_empty[a]), 32 * Epi::kEpiWarps);
     }
     mbar_init(smem_u32(drain), 1);
     fence_mbar_init();
@@ -202,7 +206,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
     tmem_relinquish();
   }
   if (p.group_off && warp >= 2) {
-    for (int g = threadIdx.x - 64; g <= p.n_groups; g += kGemmThreads - 64) {
+    for (int g = threadIdx.x - 64; g <= p.n_groups; g += gemm_threads<Epi>() - 64) {
       tabs.chunk_off[g] = __ldg(p.chunk_off + g);
       tabs.group_off[g] = __ldg(p.group_off + g);
     }
@@ -293,7 +297,10 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
     }
   } else {
     // ---------------- epilogue (warps 2..5) ----------------
+    static_assert(Epi::kEpiWarps == 4 || Epi::kEpiWarps == 8, "epilogue warps");
+    constexpr int CSTEP = Epi::kEpiWarps / 4;  // chunk stride of a warp
     const int quarter = warp & 3;
+    const int cfirst = (warp - 2) >> 2;       // first chunk of this warp
     const int row = quarter * 32 + lane;
     uint32_t jc = 0;
     bool ok = true;
@@ -314,17 +321,20 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
         typename Epi::State st;
         epi.begin(j, row, st);
         const int nch = (j.n_valid + 15) >> 4;
-        // the load of chunk c + 1 is in flight while chunk c is processed
+        // the load of this warp's next chunk is in flight while the current
+        // one is processed
         uint32_t ra[16], rb[16];
-        tmem_ld16_nowait(t0, ra);
-        tmem_wait_ld16(ra);
-        for (int c = 0; c < nch; ++c) {
-          if (c + 1 < nch) tmem_ld16_nowait(t0 + (c + 1) * 16, rb);
+        if (cfirst < nch) {
+          tmem_ld16_nowait(t0 + cfirst * 16, ra);
+          tmem_wait_ld16(ra);
+        }
+        for (int c = cfirst; c < nch; c += CSTEP) {
+          if (c + CSTEP < nch) tmem_ld16_nowait(t0 + (c + CSTEP) * 16, rb);
           float v[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(ra[i]);
           epi.chunk(j, row, c * 16, v, st);
-          if (c + 1 < nch) {
+          if (c + CSTEP < nch) {
             tmem_wait_ld16(rb);
 #pragma unroll
             for (int i = 0; i < 16; ++i) ra[i] = rb[i];
