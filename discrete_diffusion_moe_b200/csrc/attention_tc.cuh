@@ -73,8 +73,10 @@ struct AttnTcShape {
   // tiles i + 1, i + 2 are multiplied), else two
   static constexpr int KV_STAGES = FIXED + 3 * (K_BYTES + V_BYTES) <= 227 * 1024 ? 3 : 2;
   static constexpr size_t SMEM = FIXED + KV_STAGES * (K_BYTES + V_BYTES);
-  // the K/V stages hold the final O tile (fp32 rows) for its bulk store
-  static_assert((size_t)KV_STAGES * (K_BYTES + V_BYTES) >= (size_t)kAttnRows * HD * 4, "O staging");
+  // the K/V stages hold the final O tile for its tensor stores: per lane
+  // quarter, NCB boxes of 32 rows x 32 fp32 columns (128-byte swizzle)
+  static constexpr int NCB = (HD + 31) / 32;
+  static_assert((size_t)KV_STAGES * (K_BYTES + V_BYTES) >= (size_t)4 * NCB * 4096, "O staging");
   static constexpr uint32_t TMEM_COLS = (64 + HD) <= 128 ? 128 : 256;
 };
 
@@ -143,7 +145,8 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
 template <int HD>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                   const __grid_constant__ CUtensorMap tmV, const AttnTcParams p) {
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                   const AttnTcParams p) {
   using S = AttnTcShape<HD>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -405,10 +408,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     } else {
       // split partial: the unnormalised O rows (fp32) are staged in the K/V
       // stage memory (every tensor-core operation and copy into it has
-      // completed) and leave in bulk copies of the tile's valid rows; the
+      // completed) as 32 x 32 boxes with the 128-byte swizzle (16-byte piece k
+      // of a box row r at k ^ (r % 8): the 8 rows of a quarter warp write 8
+      // different bank groups) and leave in tensor stores, one per box; the
       // partial rows follow the packed query order [split][b][g][row]
-      float* so = reinterpret_cast<float*>(sK) + (size_t)row * HD;
-      // all of this half's O chunks are loaded before the one wait
       constexpr int MAXC = (NCH + 1) / 2;
       uint32_t rr[MAXC][16];
 #pragma unroll
@@ -423,31 +426,37 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int q = 0; q < MAXC; ++q)
           if (oc0 + q < oc1) tmem_wait_ld16(rr[q]);
       }
+      uint8_t* qbox = sK + (size_t)quarter * S::NCB * 4096 + (size_t)lane * 128;
 #pragma unroll
       for (int q = 0; q < MAXC; ++q)
         if (oc0 + q < oc1) {
-          float4* d4 = reinterpret_cast<float4*>(so + (oc0 + q) * 16);
+          const int c = oc0 + q;
+          uint8_t* bx = qbox + (size_t)(c >> 1) * 4096;
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            d4[e] = make_float4(__uint_as_float(rr[q][4 * e]), __uint_as_float(rr[q][4 * e + 1]),
-                                __uint_as_float(rr[q][4 * e + 2]), __uint_as_float(rr[q][4 * e + 3]));
+          for (int e = 0; e < 4; ++e) {
+            const int piece = (c & 1) * 4 + e;
+            *reinterpret_cast<float4*>(bx + ((piece ^ (lane & 7)) << 4)) =
+                make_float4(__uint_as_float(rr[q][4 * e]), __uint_as_float(rr[q][4 * e + 1]),
+                            __uint_as_float(rr[q][4 * e + 2]), __uint_as_float(rr[q][4 * e + 3]));
+          }
         }
       const long long prow_g = (((long long)split * p.B + b) * p.Hkv + g) * rows_total + r;
       if (valid && half == 0) {
         p.part_ml[prow_g * 2] = have ? m : -INFINITY;
         p.part_ml[prow_g * 2 + 1] = have ? l_row : 0.f;
       }
-      // each lane quarter's 32 rows leave in their own bulk copy once both
-      // halves have staged them
+      // each lane quarter's boxes leave once both halves have staged them
+      // (rows past the pass's packed rows fall outside the tensor and are
+      // not written)
       fence_proxy_async_smem();
       mbar_arrive(pb);
       const bool staged = wait_all(pb, (n_tiles + 1) & 1);
       const int q0 = r0 + quarter * 32;
-      const int nvalid = min(32, rows_total - q0);
-      if (staged && half == 0 && lane == 0 && nvalid > 0) {
-        float* dst = p.part_o + ((((long long)split * p.B + b) * p.Hkv + g) * rows_total + q0) * HD;
-        bulk_store_wait_read(dst, smem_u32(reinterpret_cast<float*>(sK) + (size_t)quarter * 32 * HD),
-                             (uint32_t)nvalid * HD * 4);
+      if (staged && half == 0 && lane == 0 && q0 < rows_total) {
+        const int z = (split * p.B + b) * p.Hkv + g;
+        for (int cb = 0; cb < S::NCB; ++cb)
+          tma_store_3d(&tmO, smem_u32(sK + ((size_t)quarter * S::NCB + cb) * 4096), cb * 32, q0, z);
+        bulk_commit_wait_read();
       }
     }
   }

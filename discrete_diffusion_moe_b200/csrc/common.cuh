@@ -152,19 +152,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* er
 }
 
 // ---- TMA ------------------------------------------------------------------------------
-// Bulk copy shared -> global (addresses 16-byte aligned, bytes a multiple of
-// 16), then wait until the shared memory has been read (the writes to global
-// memory complete on their own, before the kernel's completion).
-__device__ __forceinline__ void bulk_store_wait_read(void* gdst, uint32_t ssrc, uint32_t bytes) {
-  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(ssrc), "r"(bytes)
-               : "memory");
-  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-// Barrier `id` (1..15) over `n` threads (a multiple of 32).
-__device__ __forceinline__ void named_bar_sync(int id, int n) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }
@@ -186,6 +173,19 @@ __device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const CUtensorMap
       "[%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
       "l"(map), "r"(bar), "r"(x), "r"(y), "l"(policy)
       : "memory");
+}
+// 3-D tiled bulk tensor store from this CTA's shared memory (box outside the
+// tensor is clipped); the caller commits and waits.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t src, int x, int y, int z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(map),
+               "r"(src), "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+// Commit this thread's bulk stores and wait until their shared-memory sources
+// have been read.
+__device__ __forceinline__ void bulk_commit_wait_read() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   uint64_t p;

@@ -274,6 +274,24 @@ dg_status make_tmap_2d(CUtensorMap* m, const void* base, long long inner, long l
   return DG_OK;
 }
 
+// fp32 tensor [slices][rows][inner] for tensor stores of 32 x 32 boxes with
+// the 128-byte swizzle (boxes reaching past `rows` or `inner` are clipped).
+dg_status make_tmap_f32_store(CUtensorMap* m, void* base, long long inner, long long rows, long long slices) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(DG_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  if (((uintptr_t)base & 15) || inner < 1 || (inner * 4) % 16 || rows < 1 || slices < 1)
+    return fail(DG_ERR_INVALID_ARG, "tensor map: bad fp32 store tensor (%p, %lld, %lld, %lld)", base, inner, rows,
+                slices);
+  cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)rows, (cuuint64_t)slices};
+  cuuint64_t strides[2] = {(cuuint64_t)inner * 4, (cuuint64_t)(inner * rows * 4)};
+  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(DG_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return DG_OK;
+}
+
 // B operand of a GEMM: three tensor maps of the same matrix with boxes of 16,
 // min(64, bn) and bn rows (each at most the matrix's rows).
 struct BOperand {
@@ -584,15 +602,19 @@ static dg_status run_attention(const uint16_t* q, const uint16_t* kc, const uint
   DG_TRY(make_tmap_2d(&tq, q, hd, (long long)B * Hkv * nq * G, (long long)hd * 2, 64, kAttnRows));
   DG_TRY(make_tmap_2d(&tk, kc, hd, (long long)B * Hkv * c_max, (long long)hd * 2, 64, kAttnKeys));
   DG_TRY(make_tmap_2d(&tv, vc, L0 + nq, (long long)B * Hkv * hd, (long long)c_max * 2, 64, hd));
+  CUtensorMap to;
+  memset(&to, 0, sizeof to);
+  if (splits > 1)
+    DG_TRY(make_tmap_f32_store(&to, part_o, hd, (long long)G * nq, (long long)splits * B * Hkv));
   AttnTcParams ap{out, part_o, part_ml, B, nq, L0, c_max, Hq, Hkv, splits, causal ? 1 : 0,
                   (float)(1.4426950408889634 / sqrt((double)hd)), err};
   dim3 grid((G * nq + kAttnRows - 1) / kAttnRows, Hkv, B * splits);
   bool ready = false;
   switch (hd) {
-    case 32: if ((ready = attn_tc_ready<32>())) attn_tc_kernel<32><<<grid, kAttnThreads, AttnTcShape<32>::SMEM, st>>>(tq, tk, tv, ap); break;
-    case 64: if ((ready = attn_tc_ready<64>())) attn_tc_kernel<64><<<grid, kAttnThreads, AttnTcShape<64>::SMEM, st>>>(tq, tk, tv, ap); break;
-    case 128: if ((ready = attn_tc_ready<128>())) attn_tc_kernel<128><<<grid, kAttnThreads, AttnTcShape<128>::SMEM, st>>>(tq, tk, tv, ap); break;
-    case 176: if ((ready = attn_tc_ready<176>())) attn_tc_kernel<176><<<grid, kAttnThreads, AttnTcShape<176>::SMEM, st>>>(tq, tk, tv, ap); break;
+    case 32: if ((ready = attn_tc_ready<32>())) attn_tc_kernel<32><<<grid, kAttnThreads, AttnTcShape<32>::SMEM, st>>>(tq, tk, tv, to, ap); break;
+    case 64: if ((ready = attn_tc_ready<64>())) attn_tc_kernel<64><<<grid, kAttnThreads, AttnTcShape<64>::SMEM, st>>>(tq, tk, tv, to, ap); break;
+    case 128: if ((ready = attn_tc_ready<128>())) attn_tc_kernel<128><<<grid, kAttnThreads, AttnTcShape<128>::SMEM, st>>>(tq, tk, tv, to, ap); break;
+    case 176: if ((ready = attn_tc_ready<176>())) attn_tc_kernel<176><<<grid, kAttnThreads, AttnTcShape<176>::SMEM, st>>>(tq, tk, tv, to, ap); break;
     default: return fail(DG_ERR_UNSUPPORTED, "head_dim %d", hd);
   }
   if (!ready) return fail(DG_ERR_CUDA, "attention shared-memory attribute");
