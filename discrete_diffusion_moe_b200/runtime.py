@@ -73,17 +73,32 @@ class Canvas:
 
 
 class StepOutputs:
+    """Device buffers a round writes.  The per-position and per-canvas results
+    (argmax, sample, entropy, pmax, lock, mean entropy, stop, final round) are
+    views of one contiguous block, `packed`, so the host can read them with a
+    single copy."""
+
     def __init__(self, cfg: dg_model_config, batch: int, logits=False, routing=False, hidden=False,
                  device="cuda"):
         T = batch * DG_CANVAS
-        self.argmax = torch.zeros(batch, DG_CANVAS, dtype=torch.int32, device=device)
-        self.sample = torch.zeros_like(self.argmax)
-        self.entropy = torch.zeros(batch, DG_CANVAS, dtype=torch.float32, device=device)
-        self.pmax = torch.zeros_like(self.entropy)
-        self.lock = torch.zeros(batch, DG_CANVAS, dtype=torch.uint8, device=device)
-        self.mean_entropy = torch.zeros(batch, dtype=torch.float32, device=device)
-        self.stop = torch.zeros(batch, dtype=torch.uint8, device=device)
-        self.final_round = torch.zeros(batch, dtype=torch.uint8, device=device)
+        parts = [("argmax", torch.int32, (batch, DG_CANVAS)), ("sample", torch.int32, (batch, DG_CANVAS)),
+                 ("entropy", torch.float32, (batch, DG_CANVAS)), ("pmax", torch.float32, (batch, DG_CANVAS)),
+                 ("lock", torch.uint8, (batch, DG_CANVAS)), ("mean_entropy", torch.float32, (batch,)),
+                 ("stop", torch.uint8, (batch,)), ("final_round", torch.uint8, (batch,))]
+        offs, total = [], 0
+        for _, dt, shape in parts:
+            nbytes = torch.empty(0, dtype=dt).element_size()
+            for n in shape:
+                nbytes *= n
+            offs.append(total)
+            total += (nbytes + 15) // 16 * 16
+        self.packed = torch.zeros(total, dtype=torch.uint8, device=device)
+        for (name, dt, shape), o in zip(parts, offs):
+            esz = torch.empty(0, dtype=dt).element_size()
+            n = 1
+            for v in shape:
+                n *= v
+            setattr(self, name, self.packed[o:o + n * esz].view(dt).view(*shape))
         self.logits = (torch.zeros(batch, DG_CANVAS, cfg.vocab, dtype=torch.float32, device=device)
                        if logits else None)
         self.route_idx = (torch.zeros(cfg.n_layers, T, cfg.top_k, dtype=torch.int32, device=device)
