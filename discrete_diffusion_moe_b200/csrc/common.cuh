@@ -29,12 +29,17 @@ __device__ __forceinline__ float bf16_to_f32(uint16_t b) {
 __device__ __forceinline__ uint16_t f32_to_bf16(float f) {
   return __bfloat16_as_ushort(__float2bfloat16_rn(f));
 }
+// two floats -> bf16 pair (round to nearest even), lo in the low half; one
+// paired conversion
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  return (uint32_t)f32_to_bf16(lo) | ((uint32_t)f32_to_bf16(hi) << 16);
+  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
 }
-// two floats -> fp16 pair (round to nearest even), lo in the low half
+// two floats -> fp16 pair (round to nearest even), lo in the low half; one
+// paired conversion
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
-  return (uint32_t)__half_as_ushort(__float2half_rn(lo)) | ((uint32_t)__half_as_ushort(__float2half_rn(hi)) << 16);
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
 }
 // bf16 value -> the same value in fp16 (exact for magnitudes in [2^-14, 65504])
 __device__ __forceinline__ uint16_t bf16_to_f16(uint16_t b) {
