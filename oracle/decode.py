@@ -76,9 +76,12 @@ def new_state(tokens, d_model) -> CanvasState:
 
 
 def encode_context(cfg: ModelConfig, W: Weights, kv: KVCache, tokens):
-    """Causal encoding of tokens [B, n] appended at kv.length (keys stored)."""
+    """Causal encoding of tokens [B, n] appended at kv.length (keys stored).
+    Encoding no tokens leaves the cache as it is."""
     tokens = np.asarray(tokens)
     B, n = tokens.shape
+    if n == 0:
+        return
     x = W.emb_rows(tokens).reshape(B, n, cfg.d_model)
     forward_layers(cfg, W, x, kv, causal=True, append=True)
 

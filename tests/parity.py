@@ -154,7 +154,7 @@ def run_case(case: Case, check_kv=True, verbose=True):
     model.check_device()
     assert gkv.length == okv.length == case.ctx_len
 
-    if check_kv:
+    if check_kv and case.ctx_len > 0:
         for l in range(L):
             gk, gv = gkv.layer_kv(l)
             gk = gk[:, :, :case.ctx_len].float().cpu().numpy().transpose(0, 2, 1, 3)

@@ -38,3 +38,14 @@ def test_single_layer_full_width_step():
     vocab 262144, 2048 context tokens, one canvas, one round."""
     rep = run_case(Case(cfg=LAYER1, ctx_len=2048, steps=1))
     assert rep.steps == 1, rep
+
+
+@pytest.mark.parametrize("n_experts,top_k,ctx_len", [(4, 4, 0), (6, 1, 17), (6, 3, 64)])
+def test_tiny_degenerate_routing_and_context(n_experts, top_k, ctx_len):
+    """Routing edge cases against the oracle: every expert chosen by every
+    token (top-k = E, the dense softmax mixture), a single expert per token,
+    an expert count that is not a multiple of 4; and a canvas with no context
+    at all (attention over the canvas keys only) or a ragged one."""
+    cfg = dict(TINY, n_experts=n_experts, top_k=top_k)
+    rep = run_case(Case(cfg=cfg, ctx_len=ctx_len, steps=2))
+    assert rep.steps == 2, rep
