@@ -75,15 +75,16 @@ def new_state(tokens, d_model) -> CanvasState:
                        prev_argmax=np.full((B, N), -1, np.int64), done=np.zeros(B, bool))
 
 
-def encode_context(cfg: ModelConfig, W: Weights, kv: KVCache, tokens):
+def encode_context(cfg: ModelConfig, W: Weights, kv: KVCache, tokens, record=None):
     """Causal encoding of tokens [B, n] appended at kv.length (keys stored).
-    Encoding no tokens leaves the cache as it is."""
+    Encoding no tokens leaves the cache as it is.  `record`, if a list,
+    receives the per-layer routing record of forward_layers."""
     tokens = np.asarray(tokens)
     B, n = tokens.shape
     if n == 0:
         return
     x = W.emb_rows(tokens).reshape(B, n, cfg.d_model)
-    forward_layers(cfg, W, x, kv, causal=True, append=True)
+    forward_layers(cfg, W, x, kv, causal=True, append=True, record=record)
 
 
 def _top2_gap(v):

@@ -143,7 +143,8 @@ def run_case(case: Case, check_kv=True, verbose=True):
     c_max = case.ctx_len + 256
     okv = oracle.KVCache(ocfg, case.batch, c_max)
     ctx = synth.context_tokens(case.batch, case.ctx_len, case.ctx_seed, V)
-    OD.encode_context(ocfg, W, okv, ctx)
+    enc_rec = []
+    OD.encode_context(ocfg, W, okv, ctx, record=enc_rec)
     sc = _sampler(case)
     floor = MARGIN * (case.lm_std or 0.02) / 0.02
 
@@ -155,12 +156,26 @@ def run_case(case: Case, check_kv=True, verbose=True):
     assert gkv.length == okv.length == case.ctx_len
 
     if check_kv and case.ctx_len > 0:
+        # A context token whose expert choice sits within MARGIN of a tie in
+        # layer j may route differently on the two sides: its keys and values
+        # from layer j + 1 on are not compared, nor (causal attention) those of
+        # the later tokens of its canvas from layer j + 2 on.
+        Bc, Cc = case.batch, case.ctx_len
+        skip = np.zeros((L, Bc, Cc), bool)
+        for j, (_, _, margin, _, _) in enumerate(enc_rec):
+            near = np.asarray(margin).reshape(Bc, Cc) < MARGIN
+            if j + 1 < L:
+                skip[j + 1:] |= near
+            if j + 2 < L:
+                skip[j + 2:] |= np.maximum.accumulate(near, axis=1)
+        rep.tainted_tokens += int(skip[-1].sum())
         for l in range(L):
             gk, gv = gkv.layer_kv(l)
             gk = gk[:, :, :case.ctx_len].float().cpu().numpy().transpose(0, 2, 1, 3)
             gv = gv[:, :, :case.ctx_len].float().cpu().numpy().transpose(0, 2, 1, 3)
+            keep = ~skip[l]
             for g_, o_ in ((gk, okv.k[l][:, :case.ctx_len]), (gv, okv.v[l][:, :case.ctx_len])):
-                err = np.abs(g_ - o_).max() / max(np.abs(o_).max(), 1e-30)
+                err = np.abs(g_ - o_)[keep].max() / max(np.abs(o_).max(), 1e-30)
                 assert err < LOGIT_REL, f"layer {l} KV cache differs: {err}"
 
     gcv = dg.Canvas(gcfg, case.batch)

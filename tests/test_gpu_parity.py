@@ -40,12 +40,21 @@ def test_single_layer_full_width_step():
     assert rep.steps == 1, rep
 
 
-@pytest.mark.parametrize("n_experts,top_k,ctx_len", [(4, 4, 0), (6, 1, 17), (6, 3, 64)])
+@pytest.mark.parametrize("n_experts,top_k,ctx_len", [(4, 4, 0), (6, 1, 17), (6, 3, 64), (256, 8, 0), (256, 8, 64)])
 def test_tiny_degenerate_routing_and_context(n_experts, top_k, ctx_len):
     """Routing edge cases against the oracle: every expert chosen by every
     token (top-k = E, the dense softmax mixture), a single expert per token,
-    an expert count that is not a multiple of 4; and a canvas with no context
-    at all (attention over the canvas keys only) or a ragged one."""
+    an expert count that is not a multiple of 4, the largest expert count
+    (256: 8 router logits per lane, 256 groups in the grouped products); and
+    a canvas with no context at all (attention over the canvas keys only) or a
+    ragged one."""
     cfg = dict(TINY, n_experts=n_experts, top_k=top_k)
     rep = run_case(Case(cfg=cfg, ctx_len=ctx_len, steps=2))
+    assert rep.steps == 2, rep
+
+
+def test_tiny_batch8_canvases():
+    """Eight canvases in one round (2,048 canvas tokens, 4,096 routed pairs
+    over 16 experts): every canvas against the oracle."""
+    rep = run_case(Case(cfg=TINY, ctx_len=40, batch=8, steps=2))
     assert rep.steps == 2, rep
