@@ -58,3 +58,16 @@ def test_tiny_batch8_canvases():
     over 16 experts): every canvas against the oracle."""
     rep = run_case(Case(cfg=TINY, ctx_len=40, batch=8, steps=2))
     assert rep.steps == 2, rep
+
+
+@pytest.mark.parametrize("shape", [
+    dict(d_model=4096, n_q_heads=32, n_kv_heads=8, head_dim=128),   # widest model, head_dim 128
+    dict(d_model=512, n_q_heads=8, n_kv_heads=2, head_dim=64),      # 4 query heads per kv head
+])
+def test_width_and_grouped_query_shapes(shape):
+    """One layer at the largest model width (d_model 4096: router split 8,
+    one float4 per thread of the 4096-wide rows) and at a wider grouped-query
+    ratio (G = 4, head_dim 64), end to end against the oracle."""
+    cfg = dict(n_layers=1, n_experts=8, top_k=2, d_ff=256, vocab=4096, **shape)
+    rep = run_case(Case(cfg=cfg, ctx_len=70, steps=2))
+    assert rep.steps == 2, rep
