@@ -71,3 +71,11 @@ def test_width_and_grouped_query_shapes(shape):
     cfg = dict(n_layers=1, n_experts=8, top_k=2, d_ff=256, vocab=4096, **shape)
     rep = run_case(Case(cfg=cfg, ctx_len=70, steps=2))
     assert rep.steps == 2, rep
+
+
+def test_tiny_largest_batch():
+    """The largest batch a context takes (64 canvases, 16,384 canvas tokens
+    and 32,768 routed pairs in one round; 111 tokens per routing CTA), one
+    round end to end against the oracle."""
+    rep = run_case(Case(cfg=TINY, ctx_len=16, batch=64, steps=1))
+    assert rep.steps == 1, rep
