@@ -134,8 +134,8 @@ class ClockSampler:
 
 def kernel_source_hash():
     h = hashlib.sha256()
-    for rel in ("discrete_diffusion_moe_b200/csrc/gemm_tc.cuh", "discrete_diffusion_moe_b200/csrc/epilogues.cuh",
-                "discrete_diffusion_moe_b200/csrc/common.cuh"):
+    for rel in ("discrete_diffusion_moe_b200/csrc/gemm_tc.cuh", "discrete_diffusion_moe_b200/csrc/gemm_pair.cuh",
+                "discrete_diffusion_moe_b200/csrc/epilogues.cuh", "discrete_diffusion_moe_b200/csrc/common.cuh"):
         h.update(open(os.path.join(ROOT, rel), "rb").read())
     return h.hexdigest()[:16]
 
@@ -476,7 +476,7 @@ def main():
                               "frac": t_roof / (ms_per_step / 1000.0),
                               "bound": "hbm" if nbytes / (peaks["hbm_gbs"] * 1e9) >= flops / (peaks["bf16_tflops_sustained"] * 1e12) else "tensor",
                               "peaks": f"{peaks['source']}: {peaks['hbm_gbs']} GB/s, {peaks['bf16_tflops_sustained']} TF/s sustained bf16"},
-            "roofline": {"kernel": "gemm_tc_kernel<EpiSwiGLU> (grouped expert gate/up + SwiGLU)", "bound": "hbm",
+            "roofline": {"kernel": "gemm_pair_kernel<EpiSwiGLU> (grouped expert gate/up + SwiGLU, CTA pairs)", "bound": "hbm",
                          "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / peaks["hbm_gbs"], "traffic": ncu_traffic("expert_gate_up"),
                          "bytes_per_launch": gu_bytes, "launch_ms": gu_ms,

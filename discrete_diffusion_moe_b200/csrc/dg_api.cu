@@ -17,6 +17,7 @@
 #include "../../synth/synth.h"
 #include "attention_tc.cuh"
 #include "epilogues.cuh"
+#include "gemm_pair.cuh"
 #include "gemm_tc.cuh"
 #include "kernels.cuh"
 
@@ -308,6 +309,16 @@ dg_status make_bop(BOperand* b, const void* base, long long K, long long rows, i
   return DG_OK;
 }
 
+// B maps of a pair schedule: each CTA of a pair copies half of a unit's rows.
+dg_status make_bop_half(BOperand* b, const void* base, long long K, long long rows, int bn) {
+  const int want[3] = {8, std::min(32, bn / 2), bn / 2};
+  for (int i = 0; i < 3; ++i) {
+    b->rows[i] = (int)std::min<long long>(want[i], rows);
+    DG_TRY(make_tmap(&b->maps.m[i], base, K, rows, b->rows[i]));
+  }
+  return DG_OK;
+}
+
 int device_sms() {
   int dev = 0, n = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
@@ -345,6 +356,45 @@ dg_status run_gemm(const CUtensorMap& ta, const BOperand& tb, GemmPlan p, const 
   const int grid = (int)std::min<long long>(units, (long long)ctas * num_sms);
   gemm_tc_kernel<Epi><<<grid, gemm_threads<Epi>(), smem, st>>>(ta, tb.maps, p, epi, stages);
   DG_CUDA(cudaGetLastError());
+  if (launches) ++*launches;
+  return DG_OK;
+}
+
+// The grouped schedule on 2-CTA clusters (see gemm_pair.cuh); tb from make_bop_half.
+template <class Epi>
+dg_status run_gemm_pair(const CUtensorMap& ta, const BOperand& tb, GemmPlan p, const Epi& epi, int num_sms,
+                        cudaStream_t st, long long* launches = nullptr) {
+  if (!p.group_off || p.n_groups < 1 || p.n_groups > kGemmMaxGroups || p.mt != 1)
+    return fail(DG_ERR_INVALID_ARG, "pair gemm: grouped plans only (%d groups)", p.n_groups);
+  if (p.bn < 16 || p.bn > 128 || (p.bn & (p.bn - 1)) || p.K % 64 || p.K < 64)
+    return fail(DG_ERR_INVALID_ARG, "pair gemm plan: bn %d K %d", p.bn, p.K);
+  for (int i = 0; i < 3; ++i) {
+    if (tb.rows[i] < 1 || (i && tb.rows[i] < tb.rows[i - 1]) || tb.rows[i] > p.bn / 2)
+      return fail(DG_ERR_INVALID_ARG, "pair gemm plan: B box rows %d of bn %d", tb.rows[i], p.bn);
+    p.b_rows[i] = tb.rows[i];
+  }
+  static bool attr_done = false;
+  if (!attr_done) {
+    DG_CUDA(cudaFuncSetAttribute(gemm_pair_kernel<Epi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)(227 * 1024 - kGemmStaticSmem)));
+    DG_CUDA(cudaFuncSetAttribute(gemm_pair_kernel<Epi>, cudaFuncAttributePreferredSharedMemoryCarveout, 100));
+    attr_done = true;
+  }
+  const int stages = gemm_pair_stages(p.bn);
+  const size_t smem = gemm_pair_smem_bytes(p.bn, stages);
+  cudaLaunchConfig_t lc = {};
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  lc.gridDim = dim3((unsigned)(2 * (num_sms / 2) * 2));  // two CTAs per SM, whole pairs
+  lc.blockDim = dim3(gemm_threads<Epi>());
+  lc.dynamicSmemBytes = smem;
+  lc.stream = st;
+  lc.attrs = at;
+  lc.numAttrs = 1;
+  DG_CUDA(cudaLaunchKernelEx(&lc, gemm_pair_kernel<Epi>, ta, tb.maps, p, epi, stages));
   if (launches) ++*launches;
   return DG_OK;
 }
@@ -667,6 +717,14 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
   BOperand t_xperm, t_hperm;
   DG_TRY(make_bop(&t_xperm, c->at<uint16_t>(L.xperm), d, L.P_alloc, bnG));
   DG_TRY(make_bop(&t_hperm, c->at<uint16_t>(L.hperm), f, L.P_alloc, bnG));
+  // grouped products of at most 128 tokens per chunk run on CTA pairs (two
+  // pairs per SM pair); 256-token chunks keep one CTA per tile
+  const bool pair = bnG <= 128;
+  BOperand h_xperm{}, h_hperm{};
+  if (pair) {
+    DG_TRY(make_bop_half(&h_xperm, c->at<uint16_t>(L.xperm), d, L.P_alloc, bnG));
+    DG_TRY(make_bop_half(&h_hperm, c->at<uint16_t>(L.hperm), f, L.P_alloc, bnG));
+  }
 
   // cos/sin of this pass's positions, shared by all layers
   {
@@ -794,7 +852,8 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
       p.a_hint = 1;
       p.b_hint = 2;
       EpiSwiGLU e{c->at<uint16_t>(L.hperm), f};
-      DG_TRY(run_gemm(ta, t_xperm, p, e, c->num_sms, st, &c->n_launch));
+      if (pair) DG_TRY(run_gemm_pair(ta, h_xperm, p, e, c->num_sms, st, &c->n_launch));
+      else      DG_TRY(run_gemm(ta, t_xperm, p, e, c->num_sms, st, &c->n_launch));
     }
     {
       ProfScope ps_(c, DG_PROF_EXPERT_DOWN, st);
@@ -804,7 +863,8 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
       p.a_hint = 1;
       p.b_hint = 2;
       EpiDown e{c->at<float>(L.yperm), d, c->at<float>(L.wperm)};
-      DG_TRY(run_gemm(ta, t_hperm, p, e, c->num_sms, st, &c->n_launch));
+      if (pair) DG_TRY(run_gemm_pair(ta, h_hperm, p, e, c->num_sms, st, &c->n_launch));
+      else      DG_TRY(run_gemm(ta, t_hperm, p, e, c->num_sms, st, &c->n_launch));
     }
     // combine + residual, fused with the next RMSNorm (next layer's attention
     // norm, or the final norm before the LM head)
@@ -1276,7 +1336,13 @@ extern "C" dg_status dg_test_grouped_gemm(const uint16_t* A, int32_t rows_per_gr
   chunk_offsets_kernel<<<1, 1, 0, st>>>(off, n_groups, bn, choff);
   GemmPlan p = grouped_plan(K, rows_per_group, off, choff, n_groups, bn, nullptr);
   EpiGroupedT e{D, rows_per_group};
-  DG_TRY(run_gemm(ta, tb, p, e, device_sms(), st));
+  if (bn <= 128) {  // as in the layers: CTA pairs up to 128 rows per chunk
+    BOperand th;
+    DG_TRY(make_bop_half(&th, B, K, n_rows, bn));
+    DG_TRY(run_gemm_pair(ta, th, p, e, device_sms(), st));
+  } else {
+    DG_TRY(run_gemm(ta, tb, p, e, device_sms(), st));
+  }
   DG_CUDA(cudaStreamSynchronize(st));
   return DG_OK;
 }

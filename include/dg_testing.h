@@ -36,7 +36,9 @@ dg_status dg_test_gemm_tiles(const uint16_t* d_a, int32_t M, const uint16_t* d_b
    each B row r of the group and each A row f of the group.  d_off is a
    device int32 array of n_groups + 1 non-decreasing offsets ending at n_rows.
    bn (16..256, power of two) is the number of B rows per unit; d_chunk_off
-   is caller-provided device scratch of n_groups + 1 int32.  Synchronous. */
+   is caller-provided device scratch of n_groups + 1 int32.  As in the expert
+   layers, bn <= 128 runs on CTA pairs (one 256-row tcgen05.mma.cta_group::2
+   per pair of A tiles) and bn = 256 on single CTAs.  Synchronous. */
 dg_status dg_test_grouped_gemm(const uint16_t* d_a, int32_t rows_per_group, int32_t n_groups,
                                const uint16_t* d_b, int32_t n_rows, int32_t K, const int32_t* d_off,
                                float* d_d, int32_t bn, int32_t* d_chunk_off, void* stream);

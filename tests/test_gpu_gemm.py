@@ -1,6 +1,7 @@
 """The tcgen05 GEMM core (through the C-ABI test hooks) against float64
 products on the CPU, over several tiles, ragged tails, split K and grouped
-(mixture-of-experts) schedules with empty groups and multi-pass groups."""
+(mixture-of-experts) schedules with empty groups and multi-pass groups, on
+single CTAs and on CTA pairs (tcgen05.mma.cta_group::2)."""
 
 import numpy as np
 import pytest
@@ -44,13 +45,17 @@ def test_dense_gemm(dg, M, N, K, ks):
     assert np.abs(got - ref).max() <= tol * np.abs(ref).max() + 1e-4, np.abs(got - ref).max()
 
 
-@pytest.mark.parametrize("bn,sizes", [(16, [17, 0, 43, 1, 90, 5]), (32, [17, 0, 43, 1, 90, 5]),
-                                      (64, [17, 0, 43, 1, 90, 5]), (256, [17, 0, 43, 1, 90, 5]),
-                                      # skewed routing: one group holds most rows
-                                      (64, [3, 600, 0, 0, 9, 300])])
-def test_grouped_gemm(dg, bn, sizes):
-    rng = np.random.default_rng(bn + len(sizes) + sizes[1])
-    G, R, K = 6, 256, 192
+@pytest.mark.parametrize("bn,sizes,R", [(16, [17, 0, 43, 1, 90, 5], 256), (32, [17, 0, 43, 1, 90, 5], 256),
+                                        (64, [17, 0, 43, 1, 90, 5], 256), (256, [17, 0, 43, 1, 90, 5], 256),
+                                        # skewed routing: one group holds most rows
+                                        (64, [3, 600, 0, 0, 9, 300], 256),
+                                        # CTA pairs: an odd tile count (the last pair's second tile
+                                        # is missing), a partial second tile, every B box size
+                                        (128, [17, 0, 43, 1, 90, 5], 384), (32, [33, 64, 0, 7], 200),
+                                        (16, [1, 2, 3, 15, 16, 17, 31, 33], 256)])
+def test_grouped_gemm(dg, bn, sizes, R):
+    rng = np.random.default_rng(bn + len(sizes) + sizes[1] + R)
+    G, K = len(sizes), 192
     off = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
     n = int(off[-1])
     a, b = _bf16(rng, (G * R, K)), _bf16(rng, (n, K))
