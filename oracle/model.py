@@ -23,9 +23,14 @@ attention equals a second, independent formulation on tiny shapes, is
 permutation-equivariant over canvas rows without a mask, returns the mean of
 V for identical keys, and with a causal mask row 0 returns v_0; routing with
 k = E equals the dense softmax mixture and E = k = 1 is a plain SwiGLU FFN;
-routing weights sum to 1 and ties go to the lower id.  The composition of
-the full random-init model (forward_layers over many layers) has no closed
-form: parity unpinned beyond those components.
+routing weights sum to 1 and ties go to the lower id.  One layer's wiring
+(layer_forward) is pinned by closed forms: zero output and down projections
+keep the stream; zero query/key weights give uniform attention, whose
+residual (grouped-query head mapping, head layout, causal prefix, context
+keys) is written out; with one expert the MoE reads the stream after the
+attention residual.  The composition of the full random-init model
+(forward_layers over many layers) has no closed form: parity unpinned beyond
+those pieces.
 """
 
 from dataclasses import dataclass, field

@@ -194,3 +194,102 @@ def test_route_weights_sum_to_one_and_ties_go_low():
     assert np.allclose(w.sum(1), 1.0, atol=1e-6)
     for t in range(20):
         assert set(idx[t]) == set(np.argsort(-logits[t], kind="stable")[:4])
+
+
+# ---- one layer: how the pieces are wired ---------------------------------------
+
+def _wired_layer(rng, d, Hq, Hkv, hd, E, f, zero_down=True):
+    """A layer whose attention has a closed form: zero query and key weights
+    make every score 0 (uniform attention over the visible keys); the value
+    projection copies the first Hkv * hd features of the normed input; the
+    output projection is the identity on the Hq * hd = d attention features."""
+    from oracle.numerics import f64_to_bf16_bits
+    assert Hq * hd == d
+    wv = np.zeros((Hkv * hd, d))
+    wv[:, :Hkv * hd] = np.eye(Hkv * hd)
+    mk = lambda *s: bf16_round(rng.standard_normal(s) * 0.3)  # noqa: E731
+    wd = np.zeros((E, d, f)) if zero_down else mk(E, d, f)
+    return {"wq": np.zeros((Hq * hd, d)), "wk": np.zeros((Hkv * hd, d)), "wv": wv, "wo": np.eye(d),
+            "wr": mk(E, d), "wg": f64_to_bf16_bits(mk(E, f, d)), "wu": f64_to_bf16_bits(mk(E, f, d)),
+            "wd": f64_to_bf16_bits(wd)}
+
+
+def _cfg(d, Hq, Hkv, hd, E, k, f):
+    return M.ModelConfig(n_layers=1, d_model=d, n_q_heads=Hq, n_kv_heads=Hkv, head_dim=hd, n_experts=E,
+                         top_k=k, d_ff=f, vocab=256)
+
+
+def _rms_bf16(x, eps=1e-6):
+    return bf16_round(x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps))
+
+
+def test_layer_with_zero_output_and_down_projections_keeps_the_stream():
+    rng = np.random.default_rng(20)
+    d, Hq, Hkv, hd, E, k, f = 16, 4, 2, 4, 4, 2, 8
+    cfg = _cfg(d, Hq, Hkv, hd, E, k, f)
+    lw = _wired_layer(rng, d, Hq, Hkv, hd, E, f)
+    lw["wo"] = np.zeros((d, Hq * hd))
+    x = f32_round(rng.standard_normal((1, 5, d)))
+    kk = np.zeros((1, 8, Hkv, hd), np.float32)
+    vv = np.zeros((1, 8, Hkv, hd), np.float32)
+    y, _ = M.layer_forward(cfg, lw, x, kk, vv, 0, causal=True, append=True)
+    assert np.array_equal(y, x)
+    # the values written to the cache are the copied features of the normed rows
+    h = _rms_bf16(x[0])
+    assert np.array_equal(vv[0, :5].reshape(5, -1), h[:, :Hkv * hd].astype(np.float32))
+    assert np.all(kk[0, :5] == 0) and np.all(vv[0, 5:] == 0)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_layer_attention_residual_in_closed_form(causal):
+    # uniform attention: query i of head h returns the mean over its visible keys
+    # of the copied features of kv head h // (Hq / Hkv); the identity output
+    # projection puts head h at features [h * hd, (h + 1) * hd)
+    rng = np.random.default_rng(21)
+    d, Hq, Hkv, hd, E, k, f = 16, 4, 2, 4, 4, 2, 8
+    G = Hq // Hkv
+    cfg = _cfg(d, Hq, Hkv, hd, E, k, f)
+    lw = _wired_layer(rng, d, Hq, Hkv, hd, E, f)
+    L0, n = 3, 5
+    x = f32_round(rng.standard_normal((1, n, d)))
+    ctx_v = bf16_round(rng.standard_normal((L0, Hkv * hd)))
+    kk = np.zeros((1, L0 + n, Hkv, hd), np.float32)
+    vv = np.zeros((1, L0 + n, Hkv, hd), np.float32)
+    vv[0, :L0] = ctx_v.reshape(L0, Hkv, hd)
+    y, _ = M.layer_forward(cfg, lw, x, kk, vv, L0, causal=causal, append=False)
+    vals = np.concatenate([ctx_v, _rms_bf16(x[0])[:, :Hkv * hd]])  # [L0 + n, Hkv * hd]
+    want = np.empty((n, d))
+    for i in range(n):
+        vis = vals[:L0 + i + 1] if causal else vals
+        mean = vis.mean(axis=0)
+        for h in range(Hq):
+            g = h // G
+            want[i, h * hd:(h + 1) * hd] = mean[g * hd:(g + 1) * hd]
+    want = f32_round(x[0] + bf16_round(want))
+    assert np.array_equal(y[0], want)
+
+
+def test_layer_moe_reads_the_stream_after_attention():
+    # one expert (E = k = 1): the layer adds the SwiGLU FFN of the normed
+    # stream AFTER the attention residual, not of the layer's input
+    from oracle.numerics import bf16_bits_to_f64 as dec
+    rng = np.random.default_rng(22)
+    d, Hq, Hkv, hd, E, k, f = 16, 4, 4, 4, 1, 1, 8
+    cfg = _cfg(d, Hq, Hkv, hd, E, k, f)
+    lw = _wired_layer(rng, d, Hq, Hkv, hd, E, f, zero_down=False)
+    n = 4
+    x = f32_round(rng.standard_normal((1, n, d)))
+    kk = np.zeros((1, n, Hkv, hd), np.float32)
+    vv = np.zeros((1, n, Hkv, hd), np.float32)
+    y, (idx, w, _, _) = M.layer_forward(cfg, lw, x, kk, vv, 0, causal=False, append=False)
+    x1 = f32_round(x[0] + bf16_round(np.broadcast_to(_rms_bf16(x[0]).mean(axis=0), (n, d))))
+    h2 = _rms_bf16(x1)
+    a = h2 @ dec(lw["wg"][0]).T
+    ffn = f32_round(bf16_round(a / (1.0 + np.exp(-a)) * (h2 @ dec(lw["wu"][0]).T)) @ dec(lw["wd"][0]).T)
+    assert np.all(idx == 0) and np.all(w == 1.0)
+    assert np.array_equal(y[0], f32_round(x1 + ffn))
+    # a layer that fed the MoE with its input instead would differ
+    h_in = _rms_bf16(x[0])
+    a_in = h_in @ dec(lw["wg"][0]).T
+    ffn_in = f32_round(bf16_round(a_in / (1.0 + np.exp(-a_in)) * (h_in @ dec(lw["wu"][0]).T)) @ dec(lw["wd"][0]).T)
+    assert not np.array_equal(y[0], f32_round(x1 + ffn_in))
