@@ -6,11 +6,11 @@
 // 128-byte swizzle (box: 64 elements of K x 128 rows for A).  B comes with
 // three tensor maps of 16, min(64, bn) and bn rows per box: every stage loads
 // its B rows with ONE copy, the smallest box that covers the unit's columns.
-// The per-CTA copy engine rate, not the number of bytes in flight, limits how
-// fast a CTA fills its stages (a few hundred cycles per 32 KB stage, plus
-// about a hundred per copy), so each stage is exactly two copies and, for
-// tiles of at most 128 columns, two CTAs share an SM.  Each CTA loops over
-// work units:
+// Each copy costs about a hundred cycles to issue, so each stage is exactly
+// two copies.  Two CTAs per SM (tiles of at most 128 columns) measured faster
+// than one CTA with twice the stages for every product: a CTA's main loop
+// advances at a near-fixed time per k block, whatever its bytes.  Each CTA
+// loops over work units:
 //   warp 0      TMA producer (one elected lane) filling a ring of smem stages
 //   warp 1      allocates tensor memory; one lane issues tcgen05.mma (M = 128,
 //               N = the unit's columns rounded up to 16) into one of two
