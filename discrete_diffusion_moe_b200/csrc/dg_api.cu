@@ -1347,6 +1347,40 @@ extern "C" dg_status dg_test_grouped_gemm(const uint16_t* A, int32_t rows_per_gr
   return DG_OK;
 }
 
+extern "C" dg_status dg_test_grouped_schedule(int32_t pair, int32_t rows_per_group, int32_t n_groups,
+                                              const int32_t* off, int32_t K, int32_t bn, int32_t* jobs,
+                                              int32_t max_jobs, int32_t* n_jobs) {
+  if (!off || !n_jobs || (!jobs && max_jobs > 0) || max_jobs < 0 || rows_per_group < 1 || n_groups < 1 ||
+      n_groups > kGemmMaxGroups || K < 64 || K % 64 || bn < 16 || bn > (pair ? 128 : 256) || (bn & (bn - 1)))
+    return fail(DG_ERR_INVALID_ARG, "dg_test_grouped_schedule: bad arguments");
+  GemmTables tb;
+  tb.chunk_off[0] = 0;
+  for (int g = 0; g <= n_groups; ++g) {
+    tb.group_off[g] = off[g];
+    if (g < n_groups) {
+      const int rows = off[g + 1] - off[g];
+      if (rows < 0) return fail(DG_ERR_INVALID_ARG, "dg_test_grouped_schedule: offsets decrease at %d", g);
+      tb.chunk_off[g + 1] = tb.chunk_off[g] + (rows + bn - 1) / bn;
+    }
+  }
+  GemmPlan p = grouped_plan(K, rows_per_group, off, tb.chunk_off, n_groups, bn, nullptr);
+  const int rows[3] = {pair ? 8 : 16, pair ? std::min(32, bn / 2) : std::min(64, bn), pair ? bn / 2 : bn};
+  for (int i = 0; i < 3; ++i) p.b_rows[i] = rows[i];
+  const int U = pair ? pair_num_units(p, tb) : gemm_num_units(p, tb);
+  const int ranks = pair ? 2 : 1;
+  int n = 0;
+  for (int u = 0; u < U; ++u)
+    for (int r = 0; r < ranks; ++r, ++n) {
+      if (n >= max_jobs) continue;
+      const GemmJob j = pair ? pair_job(p, tb, u, r) : gemm_job(p, tb, u, 0);
+      int32_t* o = jobs + (size_t)n * 10;
+      o[0] = u; o[1] = r; o[2] = j.group; o[3] = j.m_tile; o[4] = j.a_row0; o[5] = j.m_valid;
+      o[6] = j.n0; o[7] = j.n_valid; o[8] = j.kb1 - j.kb0; o[9] = pair ? pair_b_map(p, j.n_valid) : -1;
+    }
+  *n_jobs = n;
+  return DG_OK;
+}
+
 extern "C" dg_status dg_test_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out,
                                        int32_t B, int32_t nq, int32_t L0, int32_t c_max, int32_t Hq, int32_t Hkv,
                                        int32_t hd, int32_t causal, int32_t splits, float* part_o, float* part_ml,

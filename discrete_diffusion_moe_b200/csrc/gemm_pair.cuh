@@ -122,16 +122,16 @@ __device__ __forceinline__ void umma_commit_pair(uint32_t bar) {
 }
 
 // ---- schedule ---------------------------------------------------------------------------
-__device__ __forceinline__ int pair_tiles(const GemmPlan& p) { return (p.m_tiles + 1) >> 1; }
+__host__ __device__ __forceinline__ int pair_tiles(const GemmPlan& p) { return (p.m_tiles + 1) >> 1; }
 
-__device__ __forceinline__ int pair_num_units(const GemmPlan& p, const GemmTables& tb) {
+__host__ __device__ __forceinline__ int pair_num_units(const GemmPlan& p, const GemmTables& tb) {
   return pair_tiles(p) * tb.chunk_off[p.n_groups];
 }
 
 // The job of CTA `rank` in unit u: group g with P * chunk_off[g] <= u <
 // P * chunk_off[g + 1] (P tile pairs per group), then pair, then chunk.
 // m_valid <= 0 marks the missing second tile of a group with an odd tile count.
-__device__ __forceinline__ GemmJob pair_job(const GemmPlan& p, const GemmTables& tb, int u, int rank) {
+__host__ __device__ __forceinline__ GemmJob pair_job(const GemmPlan& p, const GemmTables& tb, int u, int rank) {
   const int P = pair_tiles(p);
   int lo = 0, hi = p.n_groups;
   while (hi - lo > 1) {
@@ -164,7 +164,7 @@ __device__ __forceinline__ GemmJob pair_job(const GemmPlan& p, const GemmTables&
 // B box rows of a pair unit: the smallest of the three maps (boxes of
 // b_rows[0] < b_rows[1] < b_rows[2] rows, the last bn / 2) that covers half
 // of the unit's columns rounded up to 16.
-__device__ __forceinline__ int pair_b_map(const GemmPlan& p, int n_valid) {
+__host__ __device__ __forceinline__ int pair_b_map(const GemmPlan& p, int n_valid) {
   const int half = ((n_valid + 15) & ~15) >> 1;
   return half <= p.b_rows[0] ? 0 : (half <= p.b_rows[1] ? 1 : 2);
 }

@@ -84,7 +84,7 @@ struct GemmTables {
 constexpr size_t kGemmStaticSmem = 4096;
 static_assert(sizeof(GemmTables) <= kGemmStaticSmem, "offset tables");
 
-__device__ __forceinline__ int gemm_num_units(const GemmPlan& p, const GemmTables& tb) {
+__host__ __device__ __forceinline__ int gemm_num_units(const GemmPlan& p, const GemmTables& tb) {
   if (p.group_off) return p.m_tiles * tb.chunk_off[p.n_groups];
   const int n_tiles = (p.n_total + p.bn - 1) / p.bn;
   const int m_units = (p.m_tiles + p.mt - 1) / p.mt;
@@ -92,9 +92,9 @@ __device__ __forceinline__ int gemm_num_units(const GemmPlan& p, const GemmTable
 }
 
 // Every unit is one pass (kept as a loop level so a unit could be split).
-__device__ __forceinline__ int gemm_unit_passes(const GemmPlan&, int) { return 1; }
+__host__ __device__ __forceinline__ int gemm_unit_passes(const GemmPlan&, int) { return 1; }
 
-__device__ __forceinline__ GemmJob gemm_job(const GemmPlan& p, const GemmTables& tb, int u, int) {
+__host__ __device__ __forceinline__ GemmJob gemm_job(const GemmPlan& p, const GemmTables& tb, int u, int) {
   GemmJob j;
   const int kb_total = p.K / 64;
   if (p.group_off) {

@@ -43,6 +43,19 @@ dg_status dg_test_grouped_gemm(const uint16_t* d_a, int32_t rows_per_group, int3
                                const uint16_t* d_b, int32_t n_rows, int32_t K, const int32_t* d_off,
                                float* d_d, int32_t bn, int32_t* d_chunk_off, void* stream);
 
+/* The work schedule of a grouped product, enumerated on the host (no GPU
+   call): pair = 1 is the CTA-pair schedule (bn <= 128), pair = 0 the
+   single-CTA one.  off is a HOST int32 array of n_groups + 1 non-decreasing B
+   row offsets; chunk offsets are ceil(rows / bn) prefix sums as on the
+   device.  For every unit u and CTA rank r (r = 0 only without pairs) one job
+   of 10 int32 goes to jobs[(u * ranks + r) * 10]: u, r, group, A tile index
+   within the group, first A row, valid A rows (<= 0 for the missing second
+   tile of a pair), first B row, valid B rows, k blocks, B map index (pairs;
+   -1 otherwise).  At most max_jobs jobs are written; *n_jobs receives the
+   total.  DG_ERR_INVALID_ARG on bad sizes or decreasing offsets. */
+dg_status dg_test_grouped_schedule(int32_t pair, int32_t rows_per_group, int32_t n_groups, const int32_t* off,
+                                   int32_t K, int32_t bn, int32_t* jobs, int32_t max_jobs, int32_t* n_jobs);
+
 /* The library's attention kernel on its own (tcgen05 tensor cores):
    q bf16 packed by kv head [B][Hkv][nq][G][hd] (G = Hq / Hkv, query head
    g * G + j is row j of token t's group g), K cache bf16 [B][Hkv][c_max][hd],
