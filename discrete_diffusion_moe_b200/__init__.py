@@ -111,6 +111,7 @@ def _load():
         "dg_test_gemm_tiles": (I32, [P, I32, P, I32, I32, P, I32, I32, I32, P]),
         "dg_test_grouped_gemm": (I32, [P, I32, I32, P, I32, I32, P, P, I32, P, P]),
         "dg_test_grouped_schedule": (I32, [I32, I32, I32, P, I32, I32, P, I32, P]),
+        "dg_test_dense_schedule": (I32, [I32, I32, I32, I32, I32, I32, I32, P, I32, P]),
         "dg_test_attention": (I32, [P, P, P, P, I32, I32, I32, I32, I32, I32, I32, I32, I32, P, P, P]),
         "dg_test_workspace_buffer": (I32, [P, ctypes.c_char_p, ctypes.POINTER(P), ctypes.POINTER(S)]),
         "dg_attention_static_scratch": (I32, [P, P, P, P, I32, I32, I32, I32, I32, I32, I32, I32, I32, P]),

@@ -1381,6 +1381,29 @@ extern "C" dg_status dg_test_grouped_schedule(int32_t pair, int32_t rows_per_gro
   return DG_OK;
 }
 
+extern "C" dg_status dg_test_dense_schedule(int32_t M, int32_t N, int32_t K, int32_t bn, int32_t k_splits,
+                                           int32_t mt, int32_t n_fast, int32_t* jobs, int32_t max_jobs,
+                                           int32_t* n_jobs) {
+  if (!n_jobs || (!jobs && max_jobs > 0) || max_jobs < 0 || M < 1 || N < 1 || K < 64 || K % 64 || bn < 16 ||
+      bn > 256 || (bn & (bn - 1)) || k_splits < 1 || k_splits > K / 64 || (mt != 1 && mt != 2))
+    return fail(DG_ERR_INVALID_ARG, "dg_test_dense_schedule: bad arguments");
+  GemmTables tb{};
+  GemmPlan p = dense_plan(K, M, N, bn, k_splits, nullptr);
+  p.mt = mt;
+  p.n_fast = n_fast != 0;
+  const int U = gemm_num_units(p, tb);
+  int n = 0;
+  for (int u = 0; u < U; ++u, ++n) {
+    if (n >= max_jobs) continue;
+    const GemmJob j = gemm_job(p, tb, u, 0);
+    int32_t* o = jobs + (size_t)n * 8;
+    o[0] = u; o[1] = j.m_tile; o[2] = j.mt_eff; o[3] = j.m_valid; o[4] = j.n0; o[5] = j.n_valid;
+    o[6] = j.kb0; o[7] = j.kb1;
+  }
+  *n_jobs = n;
+  return DG_OK;
+}
+
 extern "C" dg_status dg_test_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out,
                                        int32_t B, int32_t nq, int32_t L0, int32_t c_max, int32_t Hq, int32_t Hkv,
                                        int32_t hd, int32_t causal, int32_t splits, float* part_o, float* part_ml,

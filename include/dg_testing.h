@@ -56,6 +56,17 @@ dg_status dg_test_grouped_gemm(const uint16_t* d_a, int32_t rows_per_group, int3
 dg_status dg_test_grouped_schedule(int32_t pair, int32_t rows_per_group, int32_t n_groups, const int32_t* off,
                                    int32_t K, int32_t bn, int32_t* jobs, int32_t max_jobs, int32_t* n_jobs);
 
+/* The work schedule of a dense product D[M, N] = A[M, K] B[N, K]^T,
+   enumerated on the host (no GPU call): bn B rows per unit (16..256, power of
+   two), k_splits units along K (1..K/64), mt 128-row A tiles per unit (1 or
+   2), n_fast != 0 when consecutive units walk the column tiles of one A tile.
+   One job of 8 int32 per unit u goes to jobs[u * 8]: u, first A tile, A tiles
+   in the unit, valid rows of its first tile, first B row, valid B rows, first
+   and last (exclusive) k block.  At most max_jobs are written; *n_jobs
+   receives the total.  DG_ERR_INVALID_ARG on bad sizes. */
+dg_status dg_test_dense_schedule(int32_t M, int32_t N, int32_t K, int32_t bn, int32_t k_splits, int32_t mt,
+                                 int32_t n_fast, int32_t* jobs, int32_t max_jobs, int32_t* n_jobs);
+
 /* The library's attention kernel on its own (tcgen05 tensor cores):
    q bf16 packed by kv head [B][Hkv][nq][G][hd] (G = Hq / Hkv, query head
    g * G + j is row j of token t's group g), K cache bf16 [B][Hkv][c_max][hd],

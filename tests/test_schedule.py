@@ -1,9 +1,12 @@
-"""The work schedules of the grouped (mixture-of-experts) products, enumerated
-on the host through the C ABI (no GPU): every (expert, 128-row weight tile,
-chunk of at most bn tokens) is one job of exactly one CTA, with the right
-rows, columns and k range; on CTA pairs the two ranks of a unit share the
-chunk and take consecutive tiles, the only empty tile being the missing
-second tile of an odd tile count; units run expert, then tile, then chunk."""
+"""The work schedules of the GEMM core, enumerated on the host through the C
+ABI (no GPU).  Grouped (mixture-of-experts) products: every (expert, 128-row
+weight tile, chunk of at most bn tokens) is one job of exactly one CTA, with
+the right rows, columns and k range; on CTA pairs the two ranks of a unit
+share the chunk and take consecutive tiles, the only empty tile being the
+missing second tile of an odd tile count; units run expert, then tile, then
+chunk.  Dense products: every (A tile, column tile) is covered once per k
+split, the splits partition the k blocks, and units walk the splits, then
+the column tiles (or the A tiles)."""
 
 import ctypes
 import os
@@ -106,3 +109,60 @@ def test_rejects_bad_arguments(fn):
     assert fn(0, 128, 2, good.ctypes.data, 96, 32, None, 0, ctypes.byref(n)) != 0   # K % 64
     assert fn(0, 128, 2, good.ctypes.data, 64, 48, None, 0, ctypes.byref(n)) != 0   # bn not a power of 2
     assert fn(0, 128, 2, good.ctypes.data, 64, 32, None, 0, ctypes.byref(n)) == 0 and n.value > 0
+
+
+# ---- dense products (projections, LM head, expected embedding) ------------------
+
+@pytest.fixture(scope="module")
+def dense_fn():
+    lib = ctypes.CDLL(LIB)
+    f = lib.dg_test_dense_schedule
+    f.restype = I32
+    f.argtypes = [I32, I32, I32, I32, I32, I32, I32, P, I32, P]
+    return f
+
+
+def _dense_jobs(fn, M, N, K, bn, ks, mt, n_fast):
+    n = I32(0)
+    assert fn(M, N, K, bn, ks, mt, n_fast, None, 0, ctypes.byref(n)) == 0
+    jobs = np.zeros((max(n.value, 1), 8), np.int32)
+    assert fn(M, N, K, bn, ks, mt, n_fast, jobs.ctypes.data, n.value, ctypes.byref(n)) == 0
+    return jobs[:n.value]
+
+
+@pytest.mark.parametrize("M,N,K,bn,ks,mt,n_fast", [
+    (128, 16, 64, 16, 1, 1, 1), (5632, 256, 2816, 128, 3, 1, 1), (2816, 256, 2048, 64, 2, 2, 1),
+    (384, 200, 320, 64, 5, 2, 0), (200, 1000, 704, 256, 1, 2, 1), (128 * 44 + 3, 33, 192, 32, 3, 2, 0),
+    (256, 262144, 2816, 256, 1, 1, 0), (2816, 256, 262144 // 64 * 64, 128, 8, 1, 1)])
+def test_dense_schedule_covers_every_tile_once(dense_fn, M, N, K, bn, ks, mt, n_fast):
+    jobs = _dense_jobs(dense_fn, M, N, K, bn, ks, mt, n_fast)
+    m_tiles, n_tiles, kbt = -(-M // 128), -(-N // bn), K // 64
+    assert len(jobs) == -(-m_tiles // mt) * n_tiles * ks
+    pieces = {}
+    for u, t0, mte, mv, n0, nv, kb0, kb1 in jobs:
+        assert t0 % mt == 0 and mte == min(mt, m_tiles - t0) and mte >= 1
+        assert mv == min(128, M - 128 * t0) and mv >= 1
+        assert n0 % bn == 0 and nv == min(bn, N - n0) and nv >= 1
+        assert 0 <= kb0 < kb1 <= kbt
+        for t in range(t0, t0 + mte):
+            pieces.setdefault((t, n0 // bn), []).append((kb0, kb1))
+    assert set(pieces) == {(t, c) for t in range(m_tiles) for c in range(n_tiles)}
+    for key, ranges in pieces.items():  # the k splits partition the k blocks
+        ranges.sort()
+        assert len(ranges) == ks and ranges[0][0] == 0 and ranges[-1][1] == kbt, key
+        assert all(a[1] == b[0] for a, b in zip(ranges, ranges[1:])), key
+    # consecutive units: the k splits of one tile, then (n_fast) the column tiles of one A tile
+    first = jobs[::ks]
+    assert all(np.all(jobs[i * ks:(i + 1) * ks, 1] == first[i, 1]) and
+               np.all(jobs[i * ks:(i + 1) * ks, 4] == first[i, 4]) for i in range(len(first)))
+    if n_fast and n_tiles > 1:
+        assert first[0, 1] == first[1, 1] and first[1, 4] == first[0, 4] + bn
+    elif not n_fast and -(-m_tiles // mt) > 1:
+        assert first[0, 4] == first[1, 4] and first[1, 1] == first[0, 1] + mt
+
+
+def test_dense_schedule_rejects_bad_arguments(dense_fn):
+    n = I32(0)
+    assert dense_fn(128, 16, 64, 16, 2, 1, 1, None, 0, ctypes.byref(n)) != 0   # more splits than k blocks
+    assert dense_fn(128, 16, 64, 16, 1, 3, 1, None, 0, ctypes.byref(n)) != 0   # mt 3
+    assert dense_fn(128, 16, 100, 16, 1, 1, 1, None, 0, ctypes.byref(n)) != 0  # K % 64
