@@ -28,7 +28,10 @@ routing weights sum to 1 and ties go to the lower id.  One layer's wiring
 keep the stream; zero query/key weights give uniform attention, whose
 residual (grouped-query head mapping, head layout, causal prefix, context
 keys) is written out; with one expert the MoE reads the stream after the
-attention residual.  The composition of the full random-init model
+attention residual.  The final norm and LM head (lm_logits): identity
+vocabulary rows return the bf16 normed stream, vocabulary chunking changes
+no logit, and with eps 0 a power-of-two scale of the stream changes none.
+The composition of the full random-init model
 (forward_layers over many layers) has no closed form: parity unpinned beyond
 those pieces.
 """

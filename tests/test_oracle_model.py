@@ -293,3 +293,40 @@ def test_layer_moe_reads_the_stream_after_attention():
     a_in = h_in @ dec(lw["wg"][0]).T
     ffn_in = f32_round(bf16_round(a_in / (1.0 + np.exp(-a_in)) * (h_in @ dec(lw["wu"][0]).T)) @ dec(lw["wd"][0]).T)
     assert not np.array_equal(y[0], f32_round(x1 + ffn_in))
+
+
+# ---- final norm + LM head --------------------------------------------------------
+
+class _LmRows:
+    """Stands in for the weights: vocabulary rows of a given matrix."""
+
+    def __init__(self, rows):
+        self.rows = rows
+
+    def lm_chunk(self, v0, n):
+        return self.rows[v0:v0 + n]
+
+
+def test_lm_logits_closed_form_and_chunking():
+    rng = np.random.default_rng(23)
+    d, V = 16, 40
+    cfg = M.ModelConfig(n_layers=1, d_model=d, n_q_heads=4, n_kv_heads=4, head_dim=4, n_experts=4, top_k=2,
+                        d_ff=8, vocab=V)
+    rows = np.zeros((V, d))
+    rows[:d] = np.eye(d)          # ids 0..d-1 read one normed feature each
+    rows[d + 3] = 1.0             # id d+3 sums the normed features
+    x = f32_round(rng.standard_normal((5, d)) * 3.0)
+    got = M.lm_logits(cfg, _LmRows(rows), x, chunk=7)   # chunks that do not divide V
+    hn = _rms_bf16(x)
+    assert got.dtype == np.float32 and got.shape == (5, V)
+    assert np.array_equal(got[:, :d], hn.astype(np.float32))
+    assert np.array_equal(got[:, d + 3], hn.sum(axis=1).astype(np.float32))
+    assert np.all(got[:, d:d + 3] == 0) and np.all(got[:, d + 4:] == 0)
+    # chunking over the vocabulary does not change a logit
+    W2 = _LmRows(bf16_round(rng.standard_normal((V, d))))
+    assert np.array_equal(M.lm_logits(cfg, W2, x, chunk=V), M.lm_logits(cfg, W2, x, chunk=3))
+    # the final RMSNorm is applied: with eps 0 a power-of-two scale of the
+    # stream is exact through the norm and changes no logit
+    cfg0 = M.ModelConfig(n_layers=1, d_model=d, n_q_heads=4, n_kv_heads=4, head_dim=4, n_experts=4, top_k=2,
+                         d_ff=8, vocab=V, rms_eps=0.0)
+    assert np.array_equal(M.lm_logits(cfg0, W2, x * 4.0, chunk=V), M.lm_logits(cfg0, W2, x, chunk=V))
