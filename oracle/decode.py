@@ -30,7 +30,7 @@ import numpy as np
 from . import sampler as smp
 from .model import ModelConfig, Weights, KVCache, forward_layers, lm_logits
 from .numerics import f32_round
-from .philox import method_draw, uniform_token, PURPOSE_INIT
+from .philox import method_draw, uniform_token, gumbel_words, PURPOSE_INIT, PURPOSE_AR_GUMBEL
 
 
 @dataclass
@@ -39,6 +39,7 @@ class CanvasState:
     sc: np.ndarray                # [B, N, d] float64 (bf16 values); zeros before step 0
     prev_argmax: np.ndarray       # [B, N] int64, -1 before step 0
     done: np.ndarray              # [B] bool
+    locked: np.ndarray = None     # [B, N] bool, positions committed so far (persistent lock)
 
 
 @dataclass
@@ -72,7 +73,8 @@ def init_canvas(seed: int, block: int, batch: int, n_pos: int, vocab: int) -> np
 def new_state(tokens, d_model) -> CanvasState:
     B, N = tokens.shape
     return CanvasState(tokens=np.array(tokens, np.int64), sc=np.zeros((B, N, d_model)),
-                       prev_argmax=np.full((B, N), -1, np.int64), done=np.zeros(B, bool))
+                       prev_argmax=np.full((B, N), -1, np.int64), done=np.zeros(B, bool),
+                       locked=np.zeros((B, N), bool))
 
 
 def encode_context(cfg: ModelConfig, W: Weights, kv: KVCache, tokens, record=None):
@@ -101,15 +103,22 @@ def update_canvas(cfg: ModelConfig, sc: smp.SamplerConfig, state: CanvasState, b
     sample [B, N]): the mean entropy, the stop flag, the lock mask and the next
     canvas (locked positions keep their sample, the others get the re-noise
     draw; a stopping or last-budget canvas becomes its argmax and is frozen);
-    `state` is updated in place.  Returns (meanH, stop, final, lock)."""
+    `state` is updated in place.  With sc.persistent_lock (the masked-style
+    variant) a position locked in an earlier round keeps its token and counts
+    as locked.  Returns (meanH, stop, final, lock)."""
     B, N = state.tokens.shape
     V = cfg.vocab
     meanH = H.mean(axis=1)
     stop = np.zeros(B, bool)
     final = np.zeros(B, bool)
     lock = np.zeros((B, N), bool)
+    persistent = bool(getattr(sc, "persistent_lock", False))
+    if persistent and state.locked is None:
+        state.locked = np.zeros((B, N), bool)
     for b in range(B):
         lock[b] = smp.lock_mask(H[b], pmax[b], sc.lock_policy, sc.lock_threshold)
+        committed = state.locked[b].copy() if persistent else np.zeros(N, bool)
+        lock[b] |= committed
         if state.done[b]:
             continue
         prev = state.prev_argmax[b] if step > 0 else None
@@ -117,12 +126,14 @@ def update_canvas(cfg: ModelConfig, sc: smp.SamplerConfig, state: CanvasState, b
                                 amax[b], prev)
         final[b] = stop[b] or step == sc.max_steps - 1
         if final[b]:
-            state.tokens[b] = amax[b]
+            state.tokens[b] = np.where(committed, state.tokens[b], amax[b])
             state.done[b] = True
         else:
             noise = smp.renoise_tokens(sc.seed, b, block, step, N, V)
-            state.tokens[b] = np.where(lock[b], samp[b], noise)
+            state.tokens[b] = np.where(committed, state.tokens[b], np.where(lock[b], samp[b], noise))
         state.prev_argmax[b] = amax[b]
+        if persistent:
+            state.locked[b] |= lock[b]
         if cfg.self_cond and e_new is not None:
             state.sc[b] = e_new[b]
     return meanH, stop, final, lock
@@ -130,8 +141,10 @@ def update_canvas(cfg: ModelConfig, sc: smp.SamplerConfig, state: CanvasState, b
 
 def denoise_step(cfg: ModelConfig, W: Weights, kv: KVCache, state: CanvasState,
                  sc: smp.SamplerConfig, block: int, step: int, keep_logits: bool = True,
-                 record_routing: bool = False) -> StepOutput:
-    """One denoising round over every canvas of the batch; updates `state`."""
+                 record_routing: bool = False, force_routing=None) -> StepOutput:
+    """One denoising round over every canvas of the batch; updates `state`.
+    force_routing (optional): layer -> experts [B, N, k] the layer's MoE uses
+    (forward_layers' force); the routing record keeps the router's own choice."""
     B, N = state.tokens.shape
     d, V = cfg.d_model, cfg.vocab
     tokens_in = state.tokens.copy()
@@ -143,7 +156,7 @@ def denoise_step(cfg: ModelConfig, W: Weights, kv: KVCache, state: CanvasState,
 
     # a2-a6: transformer layers, bidirectional over the canvas
     routing = [] if record_routing else None
-    x = forward_layers(cfg, W, x, kv, causal=False, append=False, record=routing)
+    x = forward_layers(cfg, W, x, kv, causal=False, append=False, record=routing, force=force_routing)
 
     # a7: logits and per-position statistics / samples
     logits = lm_logits(cfg, W, x.reshape(B * N, d)).reshape(B, N, V)
@@ -162,7 +175,7 @@ def denoise_step(cfg: ModelConfig, W: Weights, kv: KVCache, state: CanvasState,
             s_gap[b, i] = _top2_gap(keys)
             a_gap[b, i] = _top2_gap(logits[b, i])
             if probs is not None:
-                probs[b, i] = p
+                probs[b, i] = smp.selfcond_probs(logits[b, i])
 
     # a8: expected embedding for the next round's self-conditioning input
     e_new = None
@@ -200,3 +213,31 @@ def decode_block(cfg: ModelConfig, W: Weights, kv: KVCache, sc: smp.SamplerConfi
     encode_context(cfg, W, kv, tokens)
     return tokens, steps, outs
 
+
+
+def ar_step(cfg: ModelConfig, W: Weights, kv: KVCache, tokens, temperature: float, seed: int):
+    """Retained autoregressive mode (the laozijiushiniubi.cn article, section
+    七: the same weights still generate one token at a time): tokens [B] are
+    appended at position P = kv.length with causal attention (the causal
+    encode of one token), and that position's logits give the next token:
+    its argmax and its Gumbel-max draw from softmax(l / temperature) (draw
+    purpose 5, canvas b, c2 = P, position 0).  Returns (logits [B, V] fp32,
+    argmax [B], sample [B], Gumbel-key top-2 gaps [B], logit top-2 gaps [B])."""
+    tokens = np.asarray(tokens).reshape(-1)
+    B = tokens.size
+    P = kv.length
+    x = W.emb_rows(tokens).reshape(B, 1, cfg.d_model)
+    x = forward_layers(cfg, W, x, kv, causal=True, append=True)
+    logits = lm_logits(cfg, W, x.reshape(B, cfg.d_model))
+    inv_t = np.float32(1.0 / float(np.float32(temperature)))
+    amax = np.empty(B, np.int64)
+    samp = np.empty(B, np.int64)
+    s_gap = np.empty(B)
+    a_gap = np.empty(B)
+    for b in range(B):
+        amax[b] = int(np.argmax(logits[b]))
+        words = gumbel_words(seed, b, 0, P, 0, cfg.vocab, purpose=PURPOSE_AR_GUMBEL)
+        samp[b], keys = smp.gumbel_sample(logits[b], inv_t, words)
+        s_gap[b] = _top2_gap(keys)
+        a_gap[b] = _top2_gap(logits[b])
+    return logits, amax, samp, s_gap, a_gap

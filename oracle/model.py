@@ -107,6 +107,14 @@ class Weights:
             self._layer_idx = l
         return self._layer
 
+    def router(self, l: int) -> dict:
+        """Layer l's router matrix alone ({"wr": [E, d]}), without generating
+        the rest of the layer (the same values as layer(l)["wr"])."""
+        if self._layer_idx == l:
+            return {"wr": self._layer["wr"]}
+        c = self.cfg
+        return {"wr": self._mat(0, c.n_experts, c.d_model, synth.layer_tid(l, synth.KIND_WR), synth.KIND_WR)}
+
     def emb_rows(self, tokens) -> np.ndarray:
         tokens = np.asarray(tokens).reshape(-1)
         d = self.cfg.d_model
@@ -198,12 +206,15 @@ def attention(q, k, v, q_pos, k_pos, causal):
     return out
 
 
-def route(h, wr, top_k):
+def route(h, wr, top_k, force_idx=None):
     """Router of the mixture of experts: fp32 logits h W_r^T, the top-k
     experts by logit (ties to the lower expert id; the softmax over all
     experts is monotone in the logit) and their softmax probabilities
     renormalised over the chosen k (the full-softmax denominator cancels).
     Returns (idx [T, k] int64, w [T, k] fp32 values, logits [T, E]).
+    With force_idx [T, k] those experts are used instead of the top-k (the
+    weights are still the softmax of their own logits): a comparison can run
+    this model on another implementation's expert choices.
     route_margin() gives each token's smallest gap between consecutive
     sorted logits among the first k + 1 (how close the choice is to a tie)."""
     logits = f32_round(h @ wr.T)
@@ -211,7 +222,10 @@ def route(h, wr, top_k):
     idx = np.empty((T, top_k), np.int64)
     w = np.empty((T, top_k))
     for t in range(T):
-        order = sorted(range(E), key=lambda e: (-logits[t, e], e))[:top_k]
+        if force_idx is None:
+            order = sorted(range(E), key=lambda e: (-logits[t, e], e))[:top_k]
+        else:
+            order = [int(e) for e in np.asarray(force_idx).reshape(T, top_k)[t]]
         idx[t] = order
         sel = logits[t, order]
         ex = np.exp(sel - sel.max())
@@ -237,13 +251,14 @@ def expert_ffn(x, wg, wu, wd):
     return f32_round(hh @ wd.T)
 
 
-def moe_ffn(h, layer, top_k):
-    """Mixture-of-experts FFN on bf16 inputs h [T, d]: route, run each
-    expert on the tokens sent to it, and combine sum_k w_k y_k (fp32 result).
+def moe_ffn(h, layer, top_k, force_idx=None):
+    """Mixture-of-experts FFN on bf16 inputs h [T, d]: route (or take the
+    experts force_idx names, see route), run each expert on the tokens sent
+    to it, and combine sum_k w_k y_k (fp32 result).
     Returns (out, idx, w, routing margin, router logits)."""
     wg, wu, wd = layer["wg"], layer["wu"], layer["wd"]
     E = wg.shape[0]
-    idx, w, logits = route(h, layer["wr"], top_k)
+    idx, w, logits = route(h, layer["wr"], top_k, force_idx)
     T = h.shape[0]
     y = np.zeros((T, top_k, h.shape[1]))
     for e in range(E):
@@ -256,14 +271,13 @@ def moe_ffn(h, layer, top_k):
     return out, idx, w, route_margin(logits, top_k), logits
 
 
-def layer_forward(cfg: ModelConfig, lw: dict, x, kv_k, kv_v, L0: int, causal: bool, append: bool):
-    """One transformer layer on the residual stream x [B, n, d] (fp32 values)
-    whose tokens sit at positions L0 .. L0 + n - 1.  kv_k / kv_v are this
-    layer's cached keys (after RoPE) and values [B, C_max, H_kv, hd]; the
-    pass attends to keys [0, L0) from the cache plus its own n keys, which are
-    written to the cache at [L0, L0 + n) when `append`.  Returns the residual
-    stream after the layer and (routing idx, weights, routing margin, router
-    logits)."""
+def attention_block(cfg: ModelConfig, lw: dict, x, kv_k, kv_v, L0: int, causal: bool, append: bool):
+    """The attention half of one transformer layer on the residual stream x
+    [B, n, d] (fp32 values) whose tokens sit at positions L0 .. L0 + n - 1:
+    RMSNorm, q/k/v projections, RoPE, attention over the cached keys [0, L0)
+    of kv_k / kv_v ([B, C_max, H_kv, hd], keys after RoPE) plus the pass's own
+    n keys (written to the cache at [L0, L0 + n) when `append`), output
+    projection and residual add.  Returns the residual stream after it."""
     c = cfg
     B, n, d = x.shape
     pos = np.arange(L0, L0 + n)
@@ -284,15 +298,51 @@ def layer_forward(cfg: ModelConfig, lw: dict, x, kv_k, kv_v, L0: int, causal: bo
         if append:
             kv_k[b, L0:L0 + n] = kb
             kv_v[b, L0:L0 + n] = vb
-    x = f32_round(x + f32_round(o @ lw["wo"].T))
-    h2 = bf16_round(rmsnorm(x, c.rms_eps)).reshape(B * n, d)
-    m, idx, w, margin, rlog = moe_ffn(h2, lw, c.top_k)
-    x = f32_round(x + m.reshape(B, n, d))
+    return f32_round(np.asarray(x, dtype=np.float64) + f32_round(o @ lw["wo"].T))
+
+
+def moe_block(cfg: ModelConfig, lw: dict, x, force_idx=None):
+    """The mixture-of-experts half of one transformer layer on the residual
+    stream x [B, n, d] after the attention half: RMSNorm, router, experts and
+    residual add (force_idx [B, n, k]: use these experts, see route).
+    Returns the residual stream after the layer and (routing idx, weights,
+    routing margin, router logits)."""
+    B, n, d = x.shape
+    h2 = bf16_round(rmsnorm(x, cfg.rms_eps)).reshape(B * n, d)
+    fi = None if force_idx is None else np.asarray(force_idx).reshape(B * n, -1)
+    m, idx, w, margin, rlog = moe_ffn(h2, lw, cfg.top_k, fi)
+    x = f32_round(np.asarray(x, dtype=np.float64) + m.reshape(B, n, d))
     return x, (idx.reshape(B, n, -1), w.reshape(B, n, -1), margin.reshape(B, n), rlog.reshape(B, n, -1))
 
 
+def router_block(cfg: ModelConfig, lw: dict, x):
+    """The router alone on the residual stream x [B, n, d] after the attention
+    half (the first steps of moe_block): routing idx, weights, margin and
+    router logits, shaped as moe_block returns them."""
+    B, n, d = x.shape
+    h2 = bf16_round(rmsnorm(x, cfg.rms_eps)).reshape(B * n, d)
+    idx, w, logits = route(h2, lw["wr"], cfg.top_k)
+    margin = route_margin(logits, cfg.top_k)
+    return idx.reshape(B, n, -1), w.reshape(B, n, -1), margin.reshape(B, n), logits.reshape(B, n, -1)
+
+
+def layer_forward(cfg: ModelConfig, lw: dict, x, kv_k, kv_v, L0: int, causal: bool, append: bool,
+                  force_idx=None):
+    """One transformer layer on the residual stream x [B, n, d] (fp32 values)
+    whose tokens sit at positions L0 .. L0 + n - 1: attention_block then
+    moe_block.  Returns the residual stream after the layer and (routing idx,
+    weights, routing margin, router logits).  With force_idx the experts are
+    those it names and the returned idx is the router's own top-k choice."""
+    x = attention_block(cfg, lw, x, kv_k, kv_v, L0, causal, append)
+    if force_idx is None:
+        return moe_block(cfg, lw, x)
+    own = router_block(cfg, lw, x)[0]
+    x, (_, w, margin, rlog) = moe_block(cfg, lw, x, force_idx)
+    return x, (own, w, margin, rlog)
+
+
 def forward_layers(cfg: ModelConfig, W: Weights, x, kv: KVCache, causal: bool, append: bool,
-                   record=None):
+                   record=None, force=None):
     """Run all transformer layers on the residual stream x [B, n, d] (fp32
     values) whose tokens sit at positions kv.length .. kv.length + n - 1.
 
@@ -302,12 +352,15 @@ def forward_layers(cfg: ModelConfig, W: Weights, x, kv: KVCache, causal: bool, a
     canvas attends to the whole context and to itself, and its keys are not
     kept).  Returns the final residual stream.  `record`, if a list, receives
     per layer (routing idx, weights, routing margin, residual stream after the
-    layer, router logits)."""
+    layer, router logits).  `force`, if given, maps a layer to the experts
+    [B, n, k] its MoE uses (layer_forward's force_idx); the record keeps the
+    router's own choice."""
     L0 = kv.length
     n = x.shape[1]
     x = f32_round(x)
     for l in range(cfg.n_layers):
-        x, (idx, w, margin, rlog) = layer_forward(cfg, W.layer(l), x, kv.k[l], kv.v[l], L0, causal, append)
+        fi = None if force is None else force(l)
+        x, (idx, w, margin, rlog) = layer_forward(cfg, W.layer(l), x, kv.k[l], kv.v[l], L0, causal, append, fi)
         if record is not None:
             record.append((idx, w, margin, x.copy(), rlog))
     if append:

@@ -31,6 +31,7 @@ _S32 = np.uint64(32)
 PURPOSE_INIT = 1
 PURPOSE_GUMBEL = 2
 PURPOSE_RENOISE = 3
+PURPOSE_AR_GUMBEL = 5   # the autoregressive mode's Gumbel draw (c1 = 0, c2 = the position)
 
 
 def philox4x32_10(c0, c1, c2, c3, k0, k1):
@@ -79,10 +80,10 @@ def gumbel_u(words):
     return ((r.astype(np.float32) + np.float32(0.5)) * np.float32(2.0 ** -23)).astype(np.float32)
 
 
-def gumbel_words(seed, canvas, block, step, position, vocab):
+def gumbel_words(seed, canvas, block, step, position, vocab, purpose=PURPOSE_GUMBEL):
     """One 32-bit word per vocabulary id for the Gumbel draw at one position:
     word for id v is output word (v % 4) of the block at c0 = v // 4."""
     n_blocks = (vocab + 3) // 4
     c0 = np.arange(n_blocks, dtype=np.uint64)
-    w = method_draw(seed, PURPOSE_GUMBEL, canvas, block, step, position, c0)
+    w = method_draw(seed, purpose, canvas, block, step, position, c0)
     return np.stack(w, axis=1).reshape(-1)[:vocab]

@@ -51,6 +51,7 @@ class SamplerConfig:
     stop_entropy: float = 0.5
     stop_require_stable_argmax: bool = False
     seed: int = 0
+    persistent_lock: bool = False   # masked-style variant: a locked position keeps its token
 
 
 def temperature(step: int, max_steps: int, t_start: float = 0.8, t_end: float = 0.4) -> float:
@@ -135,6 +136,17 @@ def renoise_tokens(seed, canvas, block, step, n_pos, vocab):
     w0, _, _, _ = method_draw(seed, PURPOSE_RENOISE, canvas, block, step,
                               np.arange(n_pos, dtype=np.uint64))
     return uniform_token(w0, vocab)
+
+
+def selfcond_probs(logits_f32):
+    """The expected embedding's probabilities of one position (precision
+    contract): the logits are stored as bf16 for this use only, so
+    p_v = exp(bf16(l_v) - m) / Z with m = max l and Z = sum_v exp(l_v - m) of
+    the fp32 logits (the statistics the entropy uses).  float64 result."""
+    l = np.asarray(logits_f32, dtype=np.float64)
+    m = l.max()
+    Z = np.exp(l - m).sum()
+    return np.exp(bf16_round(l) - m) / Z
 
 
 def expected_embedding(probs, W, chunk: int = 16384):

@@ -92,3 +92,70 @@ def test_canvas_init_uniform():
     assert toks.shape == (4, 256) and toks.min() >= 0 and toks.max() < 4096
     # 1024 draws from 4096 ids: about 906 distinct (sd ~13)
     assert 850 < len(np.unique(toks)) < 960
+
+
+def test_persistent_lock_keeps_committed_tokens():
+    # masked-style variant: once a position locks it keeps its token in every
+    # later round (the final argmax round included); without the flag the
+    # same rounds may change it again
+    from oracle import decode as D
+    from oracle import sampler as S
+    cfg = ModelConfig(n_layers=1, d_model=64, n_q_heads=2, n_kv_heads=1, head_dim=32, n_experts=4, top_k=2,
+                        d_ff=64, vocab=64)
+    rng = np.random.default_rng(5)
+    B, N, steps = 2, 16, 6
+    for persistent in (False, True):
+        sc = S.SamplerConfig(lock_threshold=0.5, max_steps=steps, stop_entropy=-1.0, seed=3,
+                             persistent_lock=persistent)
+        state = D.new_state(rng.integers(0, cfg.vocab, (B, N)), cfg.d_model)
+        first_lock = {}
+        history = []
+        for s in range(steps):
+            pmax = rng.uniform(0.0, 1.0, (B, N))
+            H = rng.uniform(0.0, 3.0, (B, N))
+            amax = rng.integers(0, cfg.vocab, (B, N))
+            samp = rng.integers(0, cfg.vocab, (B, N))
+            before = state.tokens.copy()
+            _, _, final, lock = D.update_canvas(cfg, sc, state, 0, s, H, pmax, amax, samp)
+            history.append(state.tokens.copy())
+            for b in range(B):
+                for i in range(N):
+                    if persistent and (b, i) in first_lock:
+                        assert lock[b, i] and state.tokens[b, i] == first_lock[(b, i)] == before[b, i]
+                    elif lock[b, i] and not final[b]:
+                        assert state.tokens[b, i] == samp[b, i]
+                        first_lock.setdefault((b, i), samp[b, i])
+            if persistent:
+                assert np.array_equal(state.locked, np.logical_or(state.locked, lock))
+        assert len(first_lock) > 0
+        changed_after_lock = any(history[-1][b][i] != v for (b, i), v in first_lock.items())
+        assert changed_after_lock != persistent
+
+
+def test_ar_step_is_the_causal_encode_of_one_token_then_the_lm_head():
+    # the autoregressive step appends exactly what the causal encode of the same
+    # token appends, and its logits are the LM head of that position's stream
+    from oracle import decode as D2
+    from oracle.model import forward_layers, lm_logits
+    cfg = ModelConfig(n_layers=2, d_model=64, n_q_heads=2, n_kv_heads=1, head_dim=32, n_experts=4, top_k=2,
+                      d_ff=64, vocab=256)
+    W = Weights(cfg, seed=1)
+    ctx = synth.context_tokens(2, 5, 3, cfg.vocab)
+    kv1, kv2 = KVCache(cfg, 2, 16), KVCache(cfg, 2, 16)
+    D2.encode_context(cfg, W, kv1, ctx)
+    D2.encode_context(cfg, W, kv2, ctx)
+    tok = np.array([7, 200])
+    logits, amax, samp, s_gap, a_gap = D2.ar_step(cfg, W, kv1, tok, 0.7, seed=9)
+    x = W.emb_rows(tok).reshape(2, 1, cfg.d_model)
+    x = forward_layers(cfg, W, x, kv2, causal=True, append=True)
+    assert kv1.length == kv2.length == 6
+    for l in range(cfg.n_layers):
+        assert np.array_equal(kv1.k[l], kv2.k[l]) and np.array_equal(kv1.v[l], kv2.v[l])
+    assert np.array_equal(logits, lm_logits(cfg, W, x.reshape(2, -1)))
+    assert list(amax) == [int(np.argmax(logits[b])) for b in range(2)]
+    # a tiny temperature makes the draw the argmax (the Gumbel noise is bounded
+    # for these words: |g| < 20 while the logits are scaled by 1e6)
+    kv3 = KVCache(cfg, 2, 16)
+    D2.encode_context(cfg, W, kv3, ctx)
+    _, amax3, samp3, _, _ = D2.ar_step(cfg, W, kv3, tok, 1e-6, seed=9)
+    assert list(samp3) == list(amax3)

@@ -330,3 +330,74 @@ def test_lm_logits_closed_form_and_chunking():
     cfg0 = M.ModelConfig(n_layers=1, d_model=d, n_q_heads=4, n_kv_heads=4, head_dim=4, n_experts=4, top_k=2,
                          d_ff=8, vocab=V, rms_eps=0.0)
     assert np.array_equal(M.lm_logits(cfg0, W2, x * 4.0, chunk=V), M.lm_logits(cfg0, W2, x, chunk=V))
+
+
+# ---- the layer's halves, as the stage checks call them ----------------------------
+
+def test_layer_halves_compose_to_the_layer_and_pin_the_attention_half():
+    # attention_block returns the closed-form stream after the uniform
+    # attention residual; moe_block on it reproduces the whole layer; the
+    # router alone makes moe_block's routing decisions
+    rng = np.random.default_rng(23)
+    d, Hq, Hkv, hd, E, k, f = 16, 4, 2, 4, 6, 2, 8
+    G = Hq // Hkv
+    cfg = _cfg(d, Hq, Hkv, hd, E, k, f)
+    lw = _wired_layer(rng, d, Hq, Hkv, hd, E, f, zero_down=False)
+    n = 6
+    x = f32_round(rng.standard_normal((1, n, d)))
+    kk = np.zeros((1, n, Hkv, hd), np.float32)
+    vv = np.zeros((1, n, Hkv, hd), np.float32)
+    xm = M.attention_block(cfg, lw, x, kk, vv, 0, causal=False, append=False)
+    mean = _rms_bf16(x[0])[:, :Hkv * hd].mean(axis=0)
+    want = np.concatenate([mean[(h // G) * hd:(h // G + 1) * hd] for h in range(Hq)])
+    assert np.array_equal(xm[0], f32_round(x[0] + bf16_round(np.broadcast_to(want, (n, d)))))
+    y, rec = M.moe_block(cfg, lw, xm)
+    y2, rec2 = M.layer_forward(cfg, lw, x, kk, vv, 0, causal=False, append=False)
+    assert np.array_equal(y, y2)
+    r = M.router_block(cfg, lw, xm)
+    for a, b in zip(r, rec):
+        assert np.array_equal(np.asarray(a), np.asarray(b))
+    # the router's choice is the top-k of its logits
+    logits = np.asarray(r[3]).reshape(n, E)
+    for t in range(n):
+        assert list(np.asarray(r[0]).reshape(n, k)[t]) == list(np.argsort(-logits[t], kind="stable")[:k])
+
+
+def test_router_weights_alone_equal_the_layer_router():
+    cfg = M.ModelConfig(n_layers=2, d_model=64, n_q_heads=2, n_kv_heads=1, head_dim=32, n_experts=8, top_k=2,
+                        d_ff=64, vocab=256)
+    W = M.Weights(cfg, seed=3)
+    wr1 = W.router(1)["wr"]
+    assert np.array_equal(wr1, W.layer(1)["wr"])
+    assert not np.array_equal(W.router(0)["wr"], wr1)
+
+
+def test_forced_routing_uses_the_named_experts_with_their_own_softmax_weights():
+    # forcing the router's own choice changes nothing; forcing other experts
+    # takes exactly those, weighted by the softmax of their own logits
+    rng = np.random.default_rng(24)
+    d, Hq, Hkv, hd, E, k, f = 16, 4, 2, 4, 6, 2, 8
+    cfg = _cfg(d, Hq, Hkv, hd, E, k, f)
+    lw = _wired_layer(rng, d, Hq, Hkv, hd, E, f, zero_down=False)
+    n = 5
+    xm = f32_round(rng.standard_normal((1, n, d)))
+    y, (idx, w, margin, rlog) = M.moe_block(cfg, lw, xm)
+    y2, (idx2, w2, _, _) = M.moe_block(cfg, lw, xm, force_idx=idx)
+    assert np.array_equal(y, y2) and np.array_equal(idx, idx2) and np.array_equal(w, w2)
+    other = (np.asarray(idx) + 1) % E
+    y3, (idx3, w3, margin3, rlog3) = M.moe_block(cfg, lw, xm, force_idx=other)
+    assert np.array_equal(idx3, other) and np.array_equal(margin3, margin) and np.array_equal(rlog3, rlog)
+    lg = np.asarray(rlog).reshape(n, E)
+    for t in range(n):
+        sel = lg[t, np.asarray(other).reshape(n, k)[t]]
+        e = np.exp(sel - sel.max())
+        assert np.array_equal(np.asarray(w3).reshape(n, k)[t], f32_round(e / e.sum()))
+    assert not np.array_equal(y3, y)
+    # layer_forward returns the router's own choice when forced
+    kk = np.zeros((1, n, Hkv, hd), np.float32)
+    vv = np.zeros((1, n, Hkv, hd), np.float32)
+    x = f32_round(rng.standard_normal((1, n, d)))
+    _, (own, _, _, _) = M.layer_forward(cfg, lw, x, kk, vv, 0, causal=False, append=False)
+    _, (own2, _, _, _) = M.layer_forward(cfg, lw, x, kk, vv, 0, causal=False, append=False,
+                                         force_idx=(np.asarray(own) + 1) % E)
+    assert np.array_equal(own, own2)

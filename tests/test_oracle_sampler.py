@@ -158,3 +158,22 @@ def test_renoise_uniform_and_deterministic():
     c = S.renoise_tokens(1, 0, 2, 4, 256, 4096)
     assert np.array_equal(a, b) and not np.array_equal(a, c)
     assert a.min() >= 0 and a.max() < 4096
+
+
+def test_selfcond_probs_round_only_the_stored_logits():
+    from oracle.numerics import bf16_round
+    # logits that bf16 holds exactly: the plain softmax
+    l = np.array([1.0, 0.5, -2.0, 0.25, 0.0], np.float32)
+    p = S.selfcond_probs(l)
+    e = np.exp(l.astype(np.float64) - 1.0)
+    assert np.allclose(p, e / e.sum(), rtol=0, atol=1e-15)
+    # a logit bf16 cannot hold: its numerator uses the rounded value, the
+    # normaliser (max and sum) the exact fp32 logits
+    a = np.float32(1.0 + 2.0 ** -10)          # between two bf16 values (1 and 1 + 2^-7)
+    l = np.array([a, 0.0, 0.0], np.float32)
+    p = S.selfcond_probs(l)
+    Z = 1.0 + 2.0 * np.exp(-float(a))
+    assert float(bf16_round(a)) == 1.0
+    assert p[0] == np.exp(1.0 - float(a)) / Z
+    assert p[1] == p[2] == np.exp(-float(a)) / Z
+    assert abs(p.sum() - 1.0) > 1e-6   # no longer a distribution: the rounding is visible
