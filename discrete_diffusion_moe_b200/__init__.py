@@ -43,7 +43,7 @@ class dg_sampler_config(ctypes.Structure):
     _fields_ = [("lock_policy", ctypes.c_int32), ("lock_threshold", ctypes.c_float),
                 ("t_start", ctypes.c_float), ("t_end", ctypes.c_float), ("max_steps", ctypes.c_int32),
                 ("stop_entropy", ctypes.c_float), ("stop_require_stable_argmax", ctypes.c_int32),
-                ("seed", ctypes.c_uint64)]
+                ("seed", ctypes.c_uint64), ("persistent_lock", ctypes.c_int32)]
 
 
 class dg_kv(ctypes.Structure):
@@ -53,7 +53,7 @@ class dg_kv(ctypes.Structure):
 
 class dg_canvas(ctypes.Structure):
     _fields_ = [("tokens", ctypes.c_void_p), ("sc_state", ctypes.c_void_p), ("prev_argmax", ctypes.c_void_p),
-                ("done", ctypes.c_void_p), ("batch", ctypes.c_int32)]
+                ("done", ctypes.c_void_p), ("batch", ctypes.c_int32), ("locked", ctypes.c_void_p)]
 
 
 class dg_step_args(ctypes.Structure):
@@ -65,7 +65,7 @@ class dg_step_out(ctypes.Structure):
                 ("pmax", ctypes.c_void_p), ("lock", ctypes.c_void_p), ("mean_entropy", ctypes.c_void_p),
                 ("stop", ctypes.c_void_p), ("final_round", ctypes.c_void_p), ("logits", ctypes.c_void_p),
                 ("route_idx", ctypes.c_void_p), ("route_w", ctypes.c_void_p), ("route_logits", ctypes.c_void_p),
-                ("hidden", ctypes.c_void_p)]
+                ("hidden", ctypes.c_void_p), ("hidden_attn", ctypes.c_void_p)]
 
 
 DG_PROF_EXPERT_GATE_UP, DG_PROF_EXPERT_DOWN, DG_PROF_LM_HEAD, DG_PROF_ATTENTION, DG_PROF_DENSE, \
@@ -93,6 +93,8 @@ def _load():
         "dg_weights_bytes": (S, [cfgp]),
         "dg_kv_bytes": (S, [cfgp, I32, I32]),
         "dg_workspace_bytes": (S, [cfgp, I32]),
+        "dg_workspace_bytes_ex": (S, [cfgp, I32, I32]),
+        "dg_context_create_ex": (I32, [cfgp, P, P, S, I32, I32, ctypes.POINTER(P)]),
         "dg_model_init_random": (I32, [cfgp, U64, P, P, P]),
         "dg_context_create": (I32, [cfgp, P, P, S, I32, ctypes.POINTER(P)]),
         "dg_context_destroy": (None, [P]),
@@ -114,6 +116,9 @@ def _load():
         "dg_test_dense_schedule": (I32, [I32, I32, I32, I32, I32, I32, I32, P, I32, P]),
         "dg_test_attention": (I32, [P, P, P, P, I32, I32, I32, I32, I32, I32, I32, I32, I32, P, P, P]),
         "dg_test_workspace_buffer": (I32, [P, ctypes.c_char_p, ctypes.POINTER(P), ctypes.POINTER(S)]),
+        "dg_test_wait_timeout": (I32, [P, ctypes.c_int64, P]),
+        "dg_router_probe": (I32, [P, I32, P, I32, P, P]),
+        "dg_ar_step": (I32, [P, ctypes.POINTER(dg_kv), P, F, U64, P, P, P, P]),
         "dg_attention_static_scratch": (I32, [P, P, P, P, I32, I32, I32, I32, I32, I32, I32, I32, I32, P]),
     }
     for name, (res, args) in sig.items():

@@ -16,7 +16,8 @@
 //   warp 1      tensor memory owner and MMA issuer:
 //                 S  = Q K^T            (M 128, N 64, K hd)    -> TMEM cols [0, 64)
 //                 O += P V              (M 128, N hd, K 64)    -> TMEM cols [64, 64 + hd)
-//                                       (P and V in fp16)
+//                                       (V in fp16, P as two fp16 parts:
+//                                        O += P_hi V + P_lo V)
 //               S of tile j + 1 is issued as soon as S of tile j has been read,
 //               before P V of tile j, so the next scores overlap the softmax.
 //   warps 2..9  softmax, two threads per query row (tensor-memory lane), each
@@ -24,8 +25,9 @@
 //               partial maxima through shared memory (bounded mbarrier wait),
 //               keeps an online max / sum in the exp2 domain, rescales its
 //               half of the row of O in tensor memory when the reference max
-//               moved, writes P in fp16 (11 significant bits; scaled by 2^7
-//               so that the values lie in (0, 2^15])
+//               moved, writes P as P_hi = fp16(P) and P_lo = fp16(P - P_hi)
+//               (about 22 significant bits together; scaled by 2^7 so that
+//               the values lie in (0, 2^15])
 //               into shared memory in the 128-byte-swizzled K-major layout the
 //               MMA reads (the V^T cache holds the bf16-rounded values in
 //               fp16, exact above 2^-14, for this product);
@@ -44,13 +46,22 @@
 namespace dg {
 
 struct AttnTcParams {
-  uint16_t* out;       // [B * nq, Hq * hd] bf16            (splits == 1)
-  float* part_o;       // [splits][B][Hq][nq][hd] unnormalised (splits > 1)
+  uint16_t* out;       // [B * nq, Hq * hd] bf16 (splits == 1, or merged in the cluster)
+  float* part_o;       // [splits][B][Hq][nq][hd] unnormalised (splits > 1 without cluster)
   float* part_ml;      // [splits][B][Hq][nq][2] (max in log2 units, sum)
   int B, nq, L0, c_max, Hq, Hkv, splits, causal;
   float scale_log2;    // log2(e) / sqrt(hd)
   int* err;
+  int cluster;         // splits > 1: the splits of a tile are one cluster and merge
+                       // through distributed shared memory (no partials in global memory)
 };
+
+// P in the P V product: 1 = two fp16 parts, P_hi + P_lo (about 22 significant
+// bits; two products per key tile), 0 = one fp16 part (11 bits).
+#ifndef DG_ATTN_P_SPLIT
+#define DG_ATTN_P_SPLIT 1
+#endif
+constexpr int kAttnPParts = DG_ATTN_P_SPLIT ? 2 : 1;
 
 constexpr int kAttnThreads = 320;
 constexpr int kAttnKeys = 64;   // keys per tile
@@ -67,8 +78,9 @@ struct AttnTcShape {
   static constexpr uint32_t Q_BYTES = NA * 128 * 128;
   static constexpr uint32_t K_BYTES = NA * kAttnKeys * 128;
   static constexpr uint32_t V_BYTES = HD * 128;      // hd rows x 64 keys
-  static constexpr uint32_t P_BYTES = kAttnRows * 128;
-  static constexpr size_t FIXED = 1024 + Q_BYTES + 2 * P_BYTES + 24 * 8 + 6 * 128 * 4;
+  static constexpr uint32_t P_BYTES = kAttnRows * 128;  // one fp16 P tile (128 rows x 64 keys)
+  // four P tiles: the high and low fp16 parts of P, two buffers of each by tile parity
+  static constexpr size_t FIXED = 1024 + Q_BYTES + 2 * kAttnPParts * P_BYTES + 24 * 8 + 6 * 128 * 4;
   // K/V stages: three where they fit (the load of tile i + 3 is in flight while
   // tiles i + 1, i + 2 are multiplied), else two
   static constexpr int KV_STAGES = FIXED + 3 * (K_BYTES + V_BYTES) <= 227 * 1024 ? 3 : 2;
@@ -76,7 +88,16 @@ struct AttnTcShape {
   // the K/V stages hold the final O tile for its tensor stores: per lane
   // quarter, NCB boxes of 32 rows x 32 fp32 columns (128-byte swizzle)
   static constexpr int NCB = (HD + 31) / 32;
-  static_assert((size_t)KV_STAGES * (K_BYTES + V_BYTES) >= (size_t)4 * NCB * 4096, "O staging");
+  // (the K/V stages and then the P tiles: one contiguous region, free at the end)
+  static_assert((size_t)KV_STAGES * (K_BYTES + V_BYTES) + 2 * kAttnPParts * P_BYTES >= (size_t)4 * NCB * 4096,
+                "O staging");
+  // cluster merge: the unnormalised O tile staged row-major in the K/V stage
+  // memory with a row pitch of HD + 4 floats (the 16-byte pieces of 8
+  // consecutive rows fall in different bank groups), then (max, sum) per row
+  static constexpr int OSTR = HD + 4;
+  static constexpr uint32_t O_STAGE = 128u * OSTR * 4u;
+  static_assert((size_t)KV_STAGES * (K_BYTES + V_BYTES) >= (size_t)O_STAGE + 128 * 8, "cluster O staging");
+  static_assert(2 * P_BYTES >= 128 * 8 * 4, "merge weights");
   static constexpr uint32_t TMEM_COLS = (64 + HD) <= 128 ? 128 : 256;
 };
 
@@ -154,8 +175,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   constexpr int NS = S::KV_STAGES;
   uint8_t* sK = sQ + S::Q_BYTES;               // NS stages
   uint8_t* sV = sK + NS * S::K_BYTES;          // NS stages
-  uint8_t* sP = sV + NS * S::V_BYTES;          // P (fp16), two buffers by tile parity
-  uint64_t* bars = (uint64_t*)(sP + 2 * S::P_BYTES);
+  uint8_t* sP = sV + NS * S::V_BYTES;          // P_hi [2] then P_lo [2] (fp16), by tile parity
+  uint64_t* bars = (uint64_t*)(sP + 2 * kAttnPParts * S::P_BYTES);
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;        // [NS]
   uint64_t* kv_empty = bars + 1 + NS;  // [NS]
@@ -267,9 +288,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tc_fence_after();
         const uint32_t va = smem_u32(sV + (i % NS) * S::V_BYTES);
         const uint32_t pa = smem_u32(sP + (i & 1) * S::P_BYTES);
+        const uint32_t pl = smem_u32(sP + (2 + (i & 1)) * S::P_BYTES);
+        // O += P_hi V + P_lo V: P to ~22 significant bits from two fp16 parts
 #pragma unroll
         for (int k = 0; k < kAttnKeys / 16; ++k)
           umma_bf16(t_o, sdesc_k128(pa + k * 32), sdesc_k128(va + k * 32), id_o, (i > 0 || k > 0) ? 1u : 0u);
+        if (kAttnPParts == 2) {
+#pragma unroll
+          for (int k = 0; k < kAttnKeys / 16; ++k)
+            umma_bf16(t_o, sdesc_k128(pl + k * 32), sdesc_k128(va + k * 32), id_o, 1u);
+        }
         umma_commit(smem_u32(&pv_done[i & 1]));
         umma_commit(smem_u32(&kv_empty[i % NS]));
       }
@@ -362,16 +390,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (i > 1) {
         if (!wait_all(smem_u32(&pv_done[i & 1]), ((i - 2) >> 1) & 1)) { ok = false; break; }
       }
-      // P rows (fp16) into the swizzled K-major operand tile
+      // P rows into the swizzled K-major operand tiles: P_hi = fp16(P) and
+      // P_lo = fp16(P - P_hi) (the difference is exact in fp32)
       uint8_t* p_s = sP + (i & 1) * S::P_BYTES;
+      uint8_t* p_l = sP + (2 + (i & 1)) * S::P_BYTES;
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
         const int ch = half * 4 + cc;
-        uint32_t hv[4];
+        uint32_t hv[4], lv[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) hv[e] = pack_f16x2(sv[cc * 8 + 2 * e], sv[cc * 8 + 2 * e + 1]);
+        for (int e = 0; e < 4; ++e) {
+          const float a = sv[cc * 8 + 2 * e], b2 = sv[cc * 8 + 2 * e + 1];
+          hv[e] = pack_f16x2(a, b2);
+          const __half2 hh = *reinterpret_cast<const __half2*>(&hv[e]);
+          lv[e] = pack_f16x2(a - __low2float(hh), b2 - __high2float(hh));
+        }
         const uint32_t off = prow + (((uint32_t)ch ^ ((uint32_t)row & 7)) << 4);
         *reinterpret_cast<uint4*>(p_s + off) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+        if (kAttnPParts == 2) *reinterpret_cast<uint4*>(p_l + off) = make_uint4(lv[0], lv[1], lv[2], lv[3]);
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -405,6 +441,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
         *reinterpret_cast<uint4*>(dst + 8) = make_uint4(w[4], w[5], w[6], w[7]);
       }
+    } else if (p.cluster) {
+      // cluster merge, part 1: stage this split's unnormalised O rows and the
+      // row's (reference max, sum) for the other CTAs of the cluster (every
+      // tensor-core operation and copy into the K/V stages has completed)
+      float* so = reinterpret_cast<float*>(sK) + (size_t)row * S::OSTR;
+      for (int c = oc0; c < oc1; ++c) {
+        float v[16];
+        if (have) {
+          tmem_ld16(t_o + lane_off + c * 16, v);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) v[e] = 0.f;
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          *reinterpret_cast<float4*>(so + c * 16 + 4 * e) = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+      }
+      if (half == 0)
+        reinterpret_cast<float2*>(sK + S::O_STAGE)[row] = make_float2(have ? m : -INFINITY, have ? l_row : 0.f);
     } else {
       // split partial: the unnormalised O rows (fp32) are staged in the K/V
       // stage memory (every tensor-core operation and copy into it has
@@ -464,6 +519,68 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (p.cluster && p.splits > 1) {
+    // cluster merge, part 2: CTA `rank` of the cluster (= its key split)
+    // finishes rows [q0, q1) of the tile from every split's staged rows, in
+    // split order: O = sum_s w_s O_s with w_s = 2^(m_s - M) / sum_s' 2^(m_s' - M) l_s'
+    cluster_sync_all();  // every split's rows and (max, sum) are staged
+    if (warp >= 2) {
+      const int S_ = p.splits;
+      const int rank = (int)cluster_ctarank();
+      const int per = (kAttnRows + S_ - 1) / S_;
+      const int q0 = rank * per, q1 = min(kAttnRows, q0 + per);
+      const int te = threadIdx.x - 64;
+      float* wts = reinterpret_cast<float*>(sP);  // [per rows][8 splits] merge weights
+      const uint32_t o_base = smem_u32(sK), ml_base = smem_u32(sK + S::O_STAGE);
+      if (te < q1 - q0) {
+        const int row = q0 + te;
+        float2 ml[8];
+        float M = -INFINITY;
+#pragma unroll
+        for (int s2 = 0; s2 < 8; ++s2)
+          if (s2 < S_) {
+            ml[s2] = ld_dsmem_f2(mapa_shared(ml_base + row * 8, (uint32_t)s2));
+            M = fmaxf(M, ml[s2].x);
+          }
+        float w[8], L = 0.f;
+#pragma unroll
+        for (int s2 = 0; s2 < 8; ++s2)
+          if (s2 < S_) {
+            w[s2] = ml[s2].x == -INFINITY ? 0.f : ex2_fast(ml[s2].x - M);
+            L += w[s2] * ml[s2].y;
+          }
+        const float inv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll
+        for (int s2 = 0; s2 < 8; ++s2)
+          if (s2 < S_) wts[te * 8 + s2] = w[s2] * inv;
+      }
+      named_bar_sync(1, 256);
+      constexpr int NC4 = HD / 4;
+      const int n_items = (q1 - q0) * NC4;
+      const int G = p.Hq / p.Hkv;
+      const int rows_total = G * p.nq;
+      for (int it = te; it < n_items; it += 256) {
+        const int rr = it / NC4, c4 = it - rr * NC4;
+        const int row = q0 + rr;
+        const int r = r0 + row;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        const uint32_t off = o_base + (uint32_t)(row * S::OSTR + c4 * 4) * 4u;
+#pragma unroll
+        for (int s2 = 0; s2 < 8; ++s2)
+          if (s2 < S_) {
+            const float ws = wts[rr * 8 + s2];
+            const float4 v = ld_dsmem_f4(mapa_shared(off, (uint32_t)s2));
+            acc.x += ws * v.x; acc.y += ws * v.y; acc.z += ws * v.z; acc.w += ws * v.w;
+          }
+        if (r < rows_total) {
+          const int t_in = r / G, h = g * G + r % G;
+          uint16_t* dst = p.out + ((long long)(b * p.nq + t_in) * p.Hq + h) * HD + c4 * 4;
+          *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+        }
+      }
+    }
+    cluster_sync_all();  // no CTA leaves while another reads its shared memory
+  }
   if (warp == 1) tmem_dealloc(tmem_base, S::TMEM_COLS);
 }
 

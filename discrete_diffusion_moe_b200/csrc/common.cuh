@@ -61,8 +61,9 @@ __device__ __forceinline__ float warp_max(float v) {
 // ---- Philox4x32-10 (Salmon, Moraes, Dror, Shaw, SC'11) -----------------------------
 // The method's random draws use key = (lo32(seed), hi32(seed)) and counter
 // (c0 = element index, c1 = position, c2 = block * 256 + step,
-//  c3 = purpose << 24 | canvas); purposes: 1 canvas init, 2 Gumbel, 3 re-noise.
-constexpr uint32_t kPurposeInit = 1, kPurposeGumbel = 2, kPurposeRenoise = 3;
+//  c3 = purpose << 24 | canvas); purposes: 1 canvas init, 2 Gumbel, 3 re-noise,
+// 5 the Gumbel draw of the autoregressive mode (c1 = 0, c2 = the position).
+constexpr uint32_t kPurposeInit = 1, kPurposeGumbel = 2, kPurposeRenoise = 3, kPurposeArGumbel = 5;
 
 struct Philox4 {
   uint32_t x, y, z, w;
@@ -141,19 +142,57 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 // Wait for the phase of parity `parity` to complete, giving up after
-// kWaitLimitNs: then the error word gets kDevErrTimeout and false is returned.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* err) {
+// limit_ns: then the error word gets kDevErrTimeout and false is returned.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* err,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
   for (;;) {
 #pragma unroll 1
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       set_error(err, kDevErrTimeout);
       return false;
     }
   }
+}
+
+// ---- thread-block clusters -----------------------------------------------------------
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// shared::cluster address of the same shared-memory location in CTA `rank`
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+// every thread of every CTA of the cluster (warps converged); the arrive
+// releases this thread's earlier shared-memory writes to the cluster, the wait
+// acquires the others'
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// loads from another CTA's shared memory (a shared::cluster address from mapa)
+__device__ __forceinline__ float4 ld_dsmem_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ float2 ld_dsmem_f2(uint32_t addr) {
+  float2 v;
+  asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr) : "memory");
+  return v;
+}
+// barrier of the `count` threads of warps that name barrier `id` (not 0)
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 // ---- TMA ------------------------------------------------------------------------------

@@ -10,7 +10,12 @@
 #include <string.h>
 
 #include <algorithm>
+#include <mutex>
+#include <set>
+#include <utility>
 #include <vector>
+
+#include <nvtx3/nvToolsExt.h>
 
 #include "../../include/dg.h"
 #include "../../include/dg_testing.h"
@@ -49,6 +54,15 @@ static dg_status fail(dg_status s, const char* fmt, ...) {
   } while (0)
 
 extern "C" const char* dg_last_error(void) { return g_err; }
+
+// NVTX range over one phase of the method (host side: brackets the phase's
+// launches for a profiler's timeline; a no-op when no tool is attached)
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 // ============================================================================
 // configuration checks and layouts
@@ -118,21 +132,46 @@ WLayout weight_layout(const dg_model_config& c) {
 constexpr int kMaxAttnSplits = 8;
 
 struct WsLayout {
-  size_t err, flags, x, xn, qkv, opart, q, attn, attn_po, attn_pml, rpart, rbar, rfill, off, choff, perm, inv, wperm,
+  size_t err, flags, x, xn, qkv, opart, q, attn, rpart, tok, rbar, rfill, off, choff, perm, inv, wperm,
       xperm, hperm, yperm, logits, vp_m, vp_z, vp_s, vp_av, vp_ai, vp_gv, vp_gi, st_m, st_iz, st_h,
       st_pmax, st_amax, st_samp, probs, epart, rope, stepdev, total;
-  int T_alloc, P_alloc, ks_r, n_vt, attn_rows_cap;
+  int T_alloc, P_alloc, ks_r, n_vt;  // T_alloc: token rows of a layer pass (>= the canvas tokens)
+  int T_canvas;                       // canvas tokens (batch * 256): rows of the vocabulary buffers
   long long epart_rows;
 };
 
 // split-k of the router product: 8 from 16 k-blocks on (d_model >= 1024), else 4
 // (d_model >= 256); the routing kernel is built for both
-int router_splits(const dg_model_config& c) { return c.d_model >= 1024 ? 8 : 4; }
+int router_splits(const dg_model_config& c) { return std::min(c.d_model >= 1024 ? 8 : 4, c.d_model / 64); }
+
+// Cluster scheduling preference of the split-k projections (1: pack the
+// CTAs of clusters onto SMs to balance load, 0: spread them over SMs).
+#ifndef DG_CLUSTER_POLICY
+#define DG_CLUSTER_POLICY 1
+#endif
+// How the split-k projections are summed: 1 = the k splits of a tile form a
+// thread-block cluster and add their accumulators through distributed shared
+// memory (the QKV projection then applies RoPE and writes q / K / V^T in its
+// epilogue); 0 = each split writes fp32 partials that the next kernel sums
+// (RoPE / KV write, residual + RMSNorm, routing).
+#ifndef DG_QKV_CLUSTER
+#define DG_QKV_CLUSTER 0
+#endif
+#ifndef DG_O_CLUSTER
+#define DG_O_CLUSTER 0
+#endif
+#ifndef DG_ROUTER_CLUSTER
+#define DG_ROUTER_CLUSTER 0
+#endif
+// Largest token tile of the QKV and output projections.
+#ifndef DG_PROJ_BN_MAX
+#define DG_PROJ_BN_MAX 128
+#endif
 
 // Token columns per unit of the QKV and output projections: 128 from 256
 // tokens on (two CTAs share an SM, each weight tile is read by two CTAs at the
 // same time, the second time from L2).
-int proj_bn(int T) { return T >= 256 ? 128 : std::min(256, std::max(16, next_pow2(T))); }
+int proj_bn(int T) { return T >= 256 ? DG_PROJ_BN_MAX : std::min(256, std::max(16, next_pow2(T))); }
 
 // Split-k of the QKV and output projections: enough units for two CTAs per
 // SM, at most 3 (every split is one more fp32 partial its consumer reads).
@@ -156,19 +195,22 @@ int esum_splits(const dg_model_config& c, int T, int num_sms) {
   return std::min(ks, c.vocab / 64);
 }
 
-WsLayout ws_layout(const dg_model_config& c, int batch, int num_sms) {
+// Workspace of a context for up to `batch` canvases whose causal encode passes
+// take up to `prefill` tokens (all canvases together; at least batch * 256).
+WsLayout ws_layout(const dg_model_config& c, int batch, int num_sms, int prefill = 0) {
   WsLayout L;
   size_t off = 0;
   auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes, 256); return o; };
-  const size_t T = (size_t)batch * DG_CANVAS;
+  const size_t Tc = (size_t)batch * DG_CANVAS;                          // canvas tokens
+  const size_t T = std::max(Tc, (size_t)align_up((size_t)std::max(prefill, 0), DG_CANVAS));  // layer rows
   const size_t d = c.d_model, V = c.vocab, k = c.top_k, E = c.n_experts;
   const size_t P = T * k;
   const size_t hq = (size_t)c.n_q_heads * c.head_dim;
   L.T_alloc = (int)T;
+  L.T_canvas = (int)Tc;
   L.P_alloc = (int)P;
   L.ks_r = router_splits(c);
   L.n_vt = c.vocab / 256;
-  L.attn_rows_cap = std::max(batch, kMaxAttnSplits);
   long long er = 0;
   for (int b = 1; b <= batch; ++b)
     er = std::max(er, (long long)esum_splits(c, b * DG_CANVAS, num_sms) * b * DG_CANVAS);
@@ -184,14 +226,12 @@ WsLayout ws_layout(const dg_model_config& c, int batch, int num_sms) {
       rq = std::max(rq, (size_t)proj_splits((qkv_rows + 127) / 128, tt, c.d_model / 64, num_sms) * tt);
       ro = std::max(ro, (size_t)proj_splits((c.d_model + 127) / 128, tt, (int)hq / 64, num_sms) * tt);
     }
-    L.qkv = take(rq * qkv_rows * 4);
-    L.opart = take(ro * d * 4);
+    L.qkv = DG_QKV_CLUSTER ? 0 : take(rq * qkv_rows * 4);
+    L.opart = DG_O_CLUSTER ? 0 : take(ro * d * 4);
   }
   L.q = take(T * hq * 2);
   L.attn = take(T * hq * 2);
-  L.attn_po = take((size_t)L.attn_rows_cap * DG_CANVAS * hq * 4);
-  L.attn_pml = take((size_t)L.attn_rows_cap * DG_CANVAS * c.n_q_heads * 2 * 4);
-  L.rpart = take((size_t)L.ks_r * T * E * 4);
+  L.rpart = take((size_t)(DG_ROUTER_CLUSTER ? 1 : L.ks_r) * T * E * 4);  // router logits (or split partials)
   L.rbar = take(64);
   L.rfill = take(2 * E * 4);
   L.off = take((E + 1) * 4);
@@ -202,15 +242,16 @@ WsLayout ws_layout(const dg_model_config& c, int batch, int num_sms) {
   L.xperm = take(P * d * 2);
   L.hperm = take(P * (size_t)c.d_ff * 2);
   L.yperm = take(P * d * 4);
-  L.logits = take(T * V * 4);
-  const size_t nvp = T * (size_t)L.n_vt * 4;
+  L.logits = take(Tc * V * 2);
+  const size_t nvp = Tc * (size_t)L.n_vt * 4;
   L.vp_m = take(nvp); L.vp_z = take(nvp); L.vp_s = take(nvp); L.vp_av = take(nvp);
   L.vp_ai = take(nvp); L.vp_gv = take(nvp); L.vp_gi = take(nvp);
-  L.st_m = take(T * 4); L.st_iz = take(T * 4); L.st_h = take(T * 4); L.st_pmax = take(T * 4);
-  L.st_amax = take(T * 4); L.st_samp = take(T * 4);
-  L.rope = take((size_t)DG_CANVAS * (c.head_dim / 2) * 16);
+  L.st_m = take(Tc * 4); L.st_iz = take(Tc * 4); L.st_h = take(Tc * 4); L.st_pmax = take(Tc * 4);
+  L.st_amax = take(Tc * 4); L.st_samp = take(Tc * 4);
+  L.tok = take(T * 4);
+  L.rope = take(T * (c.head_dim / 2) * 16);  // (cos, sin) of up to T positions of a pass
   L.stepdev = take(sizeof(StepDev));
-  L.probs = c.self_cond ? take(T * V * 2) : 0;
+  L.probs = c.self_cond ? take(Tc * V * 2) : 0;
   L.epart = c.self_cond ? take((size_t)er * d * 4) : 0;
   L.total = off;
   return L;
@@ -319,6 +360,22 @@ dg_status make_bop_half(BOperand* b, const void* base, long long K, long long ro
   return DG_OK;
 }
 
+// cudaFuncSetAttribute applies to the kernel in the current device's context:
+// set each (kernel, device) once, the first time a launch on that device
+// needs it.
+dg_status set_smem_attr(const void* fn, int bytes, bool max_carveout) {
+  static std::mutex mu;
+  static std::set<std::pair<const void*, int>> done;
+  int dev = 0;
+  DG_CUDA(cudaGetDevice(&dev));
+  std::lock_guard<std::mutex> lock(mu);
+  if (done.count({fn, dev})) return DG_OK;
+  DG_CUDA(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  if (max_carveout) DG_CUDA(cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, 100));
+  done.insert({fn, dev});
+  return DG_OK;
+}
+
 int device_sms() {
   int dev = 0, n = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
@@ -339,13 +396,7 @@ dg_status run_gemm(const CUtensorMap& ta, const BOperand& tb, GemmPlan p, const 
       return fail(DG_ERR_INVALID_ARG, "gemm plan: B box rows %d of bn %d", tb.rows[i], p.bn);
     p.b_rows[i] = tb.rows[i];
   }
-  static bool attr_done = false;
-  if (!attr_done) {
-    DG_CUDA(cudaFuncSetAttribute(gemm_tc_kernel<Epi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)(227 * 1024 - kGemmStaticSmem)));
-    DG_CUDA(cudaFuncSetAttribute(gemm_tc_kernel<Epi>, cudaFuncAttributePreferredSharedMemoryCarveout, 100));
-    attr_done = true;
-  }
+  DG_TRY(set_smem_attr((const void*)gemm_tc_kernel<Epi>, (int)(227 * 1024 - kGemmStaticSmem), true));
   const int ctas = gemm_ctas_per_sm(p.bn, p.mt);
   const int stages = gemm_pick_stages(p.bn, ctas, 8, p.mt);
   const size_t smem = gemm_smem_bytes(p.bn, stages, p.mt);
@@ -353,9 +404,36 @@ dg_status run_gemm(const CUtensorMap& ta, const BOperand& tb, GemmPlan p, const 
   if (p.group_off) units = (long long)ctas * num_sms;
   else units = (long long)((p.m_tiles + p.mt - 1) / p.mt) * ((p.n_total + p.bn - 1) / p.bn) * p.k_splits;
   if (units <= 0) return DG_OK;
-  const int grid = (int)std::min<long long>(units, (long long)ctas * num_sms);
-  gemm_tc_kernel<Epi><<<grid, gemm_threads<Epi>(), smem, st>>>(ta, tb.maps, p, epi, stages);
-  DG_CUDA(cudaGetLastError());
+  if (p.cluster_k <= 1) {
+    p.cluster_k = 0;
+    const int grid = (int)std::min<long long>(units, (long long)ctas * num_sms);
+    gemm_tc_kernel<Epi><<<grid, gemm_threads<Epi>(), smem, st>>>(ta, tb.maps, p, epi, stages);
+    DG_CUDA(cudaGetLastError());
+  } else {
+    // one unit per CTA; the k splits of a tile are consecutive units and one
+    // cluster; their accumulators are staged in the stage ring ([128][bn + 4] fp32)
+    if (p.group_off || p.mt != 1 || p.cluster_k != p.k_splits || p.cluster_k > 8)
+      return fail(DG_ERR_INVALID_ARG, "gemm plan: cluster of %d k splits (dense, one A tile, at most 8)",
+                  p.cluster_k);
+    if ((size_t)stages * ((size_t)kATileBytes + (size_t)p.bn * 128) < (size_t)128 * (p.bn + 4) * 4)
+      return fail(DG_ERR_INVALID_ARG, "gemm plan: the stage ring cannot hold a %d-column accumulator", p.bn);
+    cudaLaunchConfig_t lc = {};
+    cudaLaunchAttribute at[2];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = (unsigned)p.cluster_k;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    at[1].id = cudaLaunchAttributeClusterSchedulingPolicyPreference;
+    at[1].val.clusterSchedulingPolicyPreference =
+        DG_CLUSTER_POLICY ? cudaClusterSchedulingPolicyLoadBalancing : cudaClusterSchedulingPolicySpread;
+    lc.gridDim = dim3((unsigned)units);
+    lc.blockDim = dim3(gemm_threads<Epi>());
+    lc.dynamicSmemBytes = smem;
+    lc.stream = st;
+    lc.attrs = at;
+    lc.numAttrs = 2;
+    DG_CUDA(cudaLaunchKernelEx(&lc, gemm_tc_kernel<Epi>, ta, tb.maps, p, epi, stages));
+  }
   if (launches) ++*launches;
   return DG_OK;
 }
@@ -364,22 +442,16 @@ dg_status run_gemm(const CUtensorMap& ta, const BOperand& tb, GemmPlan p, const 
 template <class Epi>
 dg_status run_gemm_pair(const CUtensorMap& ta, const BOperand& tb, GemmPlan p, const Epi& epi, int num_sms,
                         cudaStream_t st, long long* launches = nullptr) {
-  if (!p.group_off || p.n_groups < 1 || p.n_groups > kGemmMaxGroups || p.mt != 1)
-    return fail(DG_ERR_INVALID_ARG, "pair gemm: grouped plans only (%d groups)", p.n_groups);
-  if (p.bn < 16 || p.bn > 128 || (p.bn & (p.bn - 1)) || p.K % 64 || p.K < 64)
+  if ((p.group_off && (p.n_groups < 1 || p.n_groups > kGemmMaxGroups)) || p.mt != 1 || p.k_splits != 1)
+    return fail(DG_ERR_INVALID_ARG, "pair gemm: %d groups, %d A tiles, %d k splits", p.n_groups, p.mt, p.k_splits);
+  if (p.bn < 16 || p.bn > (p.group_off ? 128 : 256) || (p.bn & (p.bn - 1)) || p.K % 64 || p.K < 64)
     return fail(DG_ERR_INVALID_ARG, "pair gemm plan: bn %d K %d", p.bn, p.K);
   for (int i = 0; i < 3; ++i) {
     if (tb.rows[i] < 1 || (i && tb.rows[i] < tb.rows[i - 1]) || tb.rows[i] > p.bn / 2)
       return fail(DG_ERR_INVALID_ARG, "pair gemm plan: B box rows %d of bn %d", tb.rows[i], p.bn);
     p.b_rows[i] = tb.rows[i];
   }
-  static bool attr_done = false;
-  if (!attr_done) {
-    DG_CUDA(cudaFuncSetAttribute(gemm_pair_kernel<Epi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)(227 * 1024 - kGemmStaticSmem)));
-    DG_CUDA(cudaFuncSetAttribute(gemm_pair_kernel<Epi>, cudaFuncAttributePreferredSharedMemoryCarveout, 100));
-    attr_done = true;
-  }
+  DG_TRY(set_smem_attr((const void*)gemm_pair_kernel<Epi>, (int)(227 * 1024 - kGemmStaticSmem), true));
   const int stages = gemm_pair_stages(p.bn);
   const size_t smem = gemm_pair_smem_bytes(p.bn, stages);
   cudaLaunchConfig_t lc = {};
@@ -388,7 +460,7 @@ dg_status run_gemm_pair(const CUtensorMap& ta, const BOperand& tb, GemmPlan p, c
   at[0].val.clusterDim.x = 2;
   at[0].val.clusterDim.y = 1;
   at[0].val.clusterDim.z = 1;
-  lc.gridDim = dim3((unsigned)(2 * (num_sms / 2) * 2));  // two CTAs per SM, whole pairs
+  lc.gridDim = dim3((unsigned)(2 * (num_sms / 2) * gemm_pair_ctas_per_sm(p.bn)));  // whole pairs
   lc.blockDim = dim3(gemm_threads<Epi>());
   lc.dynamicSmemBytes = smem;
   lc.stream = st;
@@ -535,10 +607,17 @@ extern "C" size_t dg_kv_bytes(const dg_model_config* cfg, int32_t batch, int32_t
   return (size_t)cfg->n_layers * batch * cfg->n_kv_heads * c_max * cfg->head_dim * 2;
 }
 
-extern "C" size_t dg_workspace_bytes(const dg_model_config* cfg, int32_t batch) {
+extern "C" size_t dg_workspace_bytes_ex(const dg_model_config* cfg, int32_t batch, int32_t prefill_tokens) {
   char why[256];
-  if (!cfg_ok(cfg, why, sizeof why) || batch < 1) { fail(DG_ERR_INVALID_ARG, "bad workspace query"); return 0; }
-  return ws_layout(*cfg, batch, device_sms()).total;
+  if (!cfg_ok(cfg, why, sizeof why) || batch < 1 || prefill_tokens < 0 || prefill_tokens > (1 << 20)) {
+    fail(DG_ERR_INVALID_ARG, "bad workspace query");
+    return 0;
+  }
+  return ws_layout(*cfg, batch, device_sms(), prefill_tokens).total;
+}
+
+extern "C" size_t dg_workspace_bytes(const dg_model_config* cfg, int32_t batch) {
+  return dg_workspace_bytes_ex(cfg, batch, 0);
 }
 
 extern "C" dg_status dg_model_init_random(const dg_model_config* cfg, uint64_t seed, const float* kind_std,
@@ -559,6 +638,12 @@ extern "C" dg_status dg_model_init_random(const dg_model_config* cfg, uint64_t s
     if (r) return fail(DG_ERR_CUDA, "weight init: %s", cudaGetErrorString((cudaError_t)r));
     return DG_OK;
   };
+  auto fill_rows = [&](uint16_t* dst, long long row0, long long rows, long long cols, long long sr, long long sc,
+                       uint32_t tid, int kind) -> dg_status {
+    int r = synth_fill_bf16_device(dst, row0, rows, cols, sr, sc, seed, tid, sd(kind), st);
+    if (r) return fail(DG_ERR_CUDA, "weight init: %s", cudaGetErrorString((cudaError_t)r));
+    return DG_OK;
+  };
   auto ones = [&](uint16_t* dst, long long n) -> dg_status {
     fill_u16_kernel<<<(unsigned)std::min<long long>((n + 255) / 256, 4096), 256, 0, st>>>(dst, n, 0x3F80);
     DG_CUDA(cudaGetLastError());
@@ -574,9 +659,16 @@ extern "C" dg_status dg_model_init_random(const dg_model_config* cfg, uint64_t s
   for (int l = 0; l < c.n_layers; ++l) {
     const LayerW& L = wl.layers[l];
     uint16_t* qkv = W + L.wqkv;
-    DG_TRY(fill(qkv, c.n_q_heads * hd, d, d, 1, synth_layer_tid(l, SYNTH_KIND_WQ), SYNTH_KIND_WQ));
-    DG_TRY(fill(qkv + (long long)c.n_q_heads * hd * d, c.n_kv_heads * hd, d, d, 1,
-                synth_layer_tid(l, SYNTH_KIND_WK), SYNTH_KIND_WK));
+    // q and k heads: rotation pairs (j, j + hd/2) of a head in adjacent physical
+    // rows 2j, 2j + 1 (the QKV epilogue rotates a pair across two lanes)
+    for (int h = 0; h < c.n_q_heads + c.n_kv_heads; ++h) {
+      const bool is_q = h < c.n_q_heads;
+      const int hl = is_q ? h : h - c.n_q_heads;
+      const int kind = is_q ? SYNTH_KIND_WQ : SYNTH_KIND_WK;
+      for (int hf = 0; hf < 2; ++hf)
+        DG_TRY(fill_rows(qkv + ((long long)h * hd + hf) * d, (long long)hl * hd + hf * (hd / 2), hd / 2, d, 2 * d, 1,
+                         synth_layer_tid(l, kind), kind));
+    }
     DG_TRY(fill(qkv + (long long)(c.n_q_heads + c.n_kv_heads) * hd * d, c.n_kv_heads * hd, d, d, 1,
                 synth_layer_tid(l, SYNTH_KIND_WV), SYNTH_KIND_WV));
     DG_TRY(fill(W + L.wo, d, c.n_q_heads * hd, c.n_q_heads * hd, 1, synth_layer_tid(l, SYNTH_KIND_WO),
@@ -594,7 +686,13 @@ extern "C" dg_status dg_model_init_random(const dg_model_config* cfg, uint64_t s
 
 extern "C" dg_status dg_context_create(const dg_model_config* cfg, const void* d_weights, void* d_workspace,
                                        size_t ws_bytes, int32_t batch, dg_ctx** out) {
+  return dg_context_create_ex(cfg, d_weights, d_workspace, ws_bytes, batch, 0, out);
+}
+
+extern "C" dg_status dg_context_create_ex(const dg_model_config* cfg, const void* d_weights, void* d_workspace,
+                                          size_t ws_bytes, int32_t batch, int32_t prefill_tokens, dg_ctx** out) {
   if (!out) return fail(DG_ERR_INVALID_ARG, "out is null");
+  if (prefill_tokens < 0 || prefill_tokens > (1 << 20)) return fail(DG_ERR_INVALID_ARG, "prefill_tokens outside [0, 2^20]");
   *out = nullptr;
   char why[256];
   if (!cfg_ok(cfg, why, sizeof why)) return fail(DG_ERR_INVALID_ARG, "%s", why);
@@ -610,7 +708,7 @@ extern "C" dg_status dg_context_create(const dg_model_config* cfg, const void* d
   c->batch_max = batch;
   c->num_sms = device_sms();
   c->wl = weight_layout(*cfg);
-  c->L = ws_layout(*cfg, batch, c->num_sms);
+  c->L = ws_layout(*cfg, batch, c->num_sms, prefill_tokens);
   if (ws_bytes < c->L.total) {
     size_t need = c->L.total;
     delete c;
@@ -633,20 +731,42 @@ extern "C" void dg_context_destroy(dg_ctx* ctx) { delete ctx; }
 // Attention of one pass on the tensor cores: q packed [B][Hkv][nq][G][hd],
 // K cache [B][Hkv][c_max][hd], V^T cache [B][Hkv][hd][c_max]; splits > 1
 // writes per-split partials and merges them (fixed split order) into out.
+
+// With `cluster`, the key splits of a tile run as one thread-block cluster and
+// merge through distributed shared memory (part_o / part_ml unused); without
+// it they write partials to part_o / part_ml and a second kernel merges them.
 template <int HD>
-static bool attn_tc_ready() {
-  static bool done = false;
-  if (!done)
-    done = cudaFuncSetAttribute(attn_tc_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)AttnTcShape<HD>::SMEM) == cudaSuccess;
-  return done;
+static dg_status launch_attn(dim3 grid, int splits, bool cluster, const CUtensorMap& tq, const CUtensorMap& tk,
+                             const CUtensorMap& tv, const CUtensorMap& to, const AttnTcParams& ap, cudaStream_t st) {
+  DG_TRY(set_smem_attr((const void*)attn_tc_kernel<HD>, (int)AttnTcShape<HD>::SMEM, false));
+  if (!cluster || splits <= 1) {
+    attn_tc_kernel<HD><<<grid, kAttnThreads, AttnTcShape<HD>::SMEM, st>>>(tq, tk, tv, to, ap);
+    DG_CUDA(cudaGetLastError());
+    return DG_OK;
+  }
+  cudaLaunchConfig_t lc = {};
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 1;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = (unsigned)splits;
+  lc.gridDim = grid;
+  lc.blockDim = dim3(kAttnThreads);
+  lc.dynamicSmemBytes = AttnTcShape<HD>::SMEM;
+  lc.stream = st;
+  lc.attrs = at;
+  lc.numAttrs = 1;
+  DG_CUDA(cudaLaunchKernelEx(&lc, attn_tc_kernel<HD>, tq, tk, tv, to, ap));
+  return DG_OK;
 }
 
 static dg_status run_attention(const uint16_t* q, const uint16_t* kc, const uint16_t* vc, uint16_t* out,
                                float* part_o, float* part_ml, int B, int nq, int L0, int c_max, int Hq, int Hkv,
-                               int hd, bool causal, int splits, int* err, cudaStream_t st, long long* launches) {
+                               int hd, bool causal, int splits, bool cluster, int* err, cudaStream_t st,
+                               long long* launches) {
   if (c_max % 8) return fail(DG_ERR_INVALID_ARG, "c_max %d is not a multiple of 8", c_max);
-  if (splits > 1 && (!part_o || !part_ml)) return fail(DG_ERR_INVALID_ARG, "split buffers are null");
+  if (splits > kMaxAttnSplits) return fail(DG_ERR_INVALID_ARG, "%d key splits (at most %d)", splits, kMaxAttnSplits);
+  if (splits > 1 && !cluster && (!part_o || !part_ml)) return fail(DG_ERR_INVALID_ARG, "split buffers are null");
   const int G = Hq / Hkv;
   CUtensorMap tq, tk, tv;
   DG_TRY(make_tmap_2d(&tq, q, hd, (long long)B * Hkv * nq * G, (long long)hd * 2, 64, kAttnRows));
@@ -654,23 +774,21 @@ static dg_status run_attention(const uint16_t* q, const uint16_t* kc, const uint
   DG_TRY(make_tmap_2d(&tv, vc, L0 + nq, (long long)B * Hkv * hd, (long long)c_max * 2, 64, hd));
   CUtensorMap to;
   memset(&to, 0, sizeof to);
-  if (splits > 1)
+  const bool merge_in_cluster = cluster && splits > 1;
+  if (splits > 1 && !merge_in_cluster)
     DG_TRY(make_tmap_f32_store(&to, part_o, hd, (long long)G * nq, (long long)splits * B * Hkv));
   AttnTcParams ap{out, part_o, part_ml, B, nq, L0, c_max, Hq, Hkv, splits, causal ? 1 : 0,
-                  (float)(1.4426950408889634 / sqrt((double)hd)), err};
+                  (float)(1.4426950408889634 / sqrt((double)hd)), err, merge_in_cluster ? 1 : 0};
   dim3 grid((G * nq + kAttnRows - 1) / kAttnRows, Hkv, B * splits);
-  bool ready = false;
   switch (hd) {
-    case 32: if ((ready = attn_tc_ready<32>())) attn_tc_kernel<32><<<grid, kAttnThreads, AttnTcShape<32>::SMEM, st>>>(tq, tk, tv, to, ap); break;
-    case 64: if ((ready = attn_tc_ready<64>())) attn_tc_kernel<64><<<grid, kAttnThreads, AttnTcShape<64>::SMEM, st>>>(tq, tk, tv, to, ap); break;
-    case 128: if ((ready = attn_tc_ready<128>())) attn_tc_kernel<128><<<grid, kAttnThreads, AttnTcShape<128>::SMEM, st>>>(tq, tk, tv, to, ap); break;
-    case 176: if ((ready = attn_tc_ready<176>())) attn_tc_kernel<176><<<grid, kAttnThreads, AttnTcShape<176>::SMEM, st>>>(tq, tk, tv, to, ap); break;
+    case 32: DG_TRY(launch_attn<32>(grid, splits, merge_in_cluster, tq, tk, tv, to, ap, st)); break;
+    case 64: DG_TRY(launch_attn<64>(grid, splits, merge_in_cluster, tq, tk, tv, to, ap, st)); break;
+    case 128: DG_TRY(launch_attn<128>(grid, splits, merge_in_cluster, tq, tk, tv, to, ap, st)); break;
+    case 176: DG_TRY(launch_attn<176>(grid, splits, merge_in_cluster, tq, tk, tv, to, ap, st)); break;
     default: return fail(DG_ERR_UNSUPPORTED, "head_dim %d", hd);
   }
-  if (!ready) return fail(DG_ERR_CUDA, "attention shared-memory attribute");
-  DG_CUDA(cudaGetLastError());
   if (launches) ++*launches;
-  if (splits > 1) {
+  if (splits > 1 && !merge_in_cluster) {
     const long long rows = (long long)B * Hq * nq;
     const unsigned cgrid = (unsigned)((rows * 32 + 255) / 256);
     if (splits <= 4)
@@ -699,7 +817,7 @@ static int attn_splits(int B, int nq, int L0, int Hq, int Hkv, int num_sms, int 
 // L0 .. L0 + nq - 1 (x already holds the embedded inputs)
 static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L0, bool causal,
                                 int32_t* dbg_idx, float* dbg_w, float* dbg_logits, float* dbg_hidden,
-                                cudaStream_t st) {
+                                float* dbg_hidden_attn, cudaStream_t st) {
   const dg_model_config& m = c->cfg;
   const WsLayout& L = c->L;
   const int T = B * nq, d = m.d_model, hd = m.head_dim, Hq = m.n_q_heads, Hkv = m.n_kv_heads;
@@ -739,8 +857,8 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
   const int ks_qkv = proj_splits((qkv_rows + 127) / 128, T, d / 64, c->num_sms);
   const int ks_o = proj_splits((d + 127) / 128, T, Hq * hd / 64, c->num_sms);
 
-  // attention key splits
-  const int splits = attn_splits(B, nq, L0, Hq, Hkv, c->num_sms, L.attn_rows_cap);
+  // attention key splits (merged inside each split cluster)
+  const int splits = attn_splits(B, nq, L0, Hq, Hkv, c->num_sms, 1 << 30);
 
   for (int l = 0; l < m.n_layers; ++l) {
     const LayerW& W = c->wl.layers[l];
@@ -748,6 +866,7 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
     uint16_t* vc = (uint16_t*)kv->v + (size_t)l * kv_layer;
 
     // --- attention block (its RMSNorm ran at the end of the previous layer) ---
+    NvtxRange nv_layer("dg.layer");  // the whole layer; its expert block nested
     if (l == 0) {
       rmsnorm_kernel<256><<<T, 256, 0, st>>>(x, c->wp(W.g_attn), xn, d, m.rms_eps);
       CNT(c);
@@ -761,10 +880,16 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
       DG_TRY(make_bop(&tb, xn, d, L.T_alloc, bn));
       GemmPlan p = dense_plan(d, qkv_rows, T, bn, ks_qkv, err);
       p.a_hint = 1;
-      EpiStoreT e{c->at<float>(L.qkv), qkv_rows, (long long)T * qkv_rows, 0, nullptr, nullptr, 0, err};
-      DG_TRY(run_gemm(ta, tb, p, e, c->num_sms, st, &c->n_launch));
+      if (DG_QKV_CLUSTER || ks_qkv == 1) {
+        p.cluster_k = ks_qkv;  // the k splits of a tile add up in their cluster
+        EpiQKV e{c->at<double2>(L.rope), c->at<uint16_t>(L.q), kc, vc, nq, L0, kv->c_max, Hq, Hkv, hd};
+        DG_TRY(run_gemm(ta, tb, p, e, c->num_sms, st, &c->n_launch));
+      } else {
+        EpiStoreT e{c->at<float>(L.qkv), qkv_rows, (long long)T * qkv_rows, 0, nullptr, nullptr, 0, err};
+        DG_TRY(run_gemm(ta, tb, p, e, c->num_sms, st, &c->n_launch));
+      }
     }
-    {
+    if (!DG_QKV_CLUSTER && ks_qkv > 1) {
       const int v_blocks = (int)(((long long)T * Hkv * (hd / 4) + 255) / 256);
       RopeParams rp{c->at<float>(L.qkv), ks_qkv, (long long)T * qkv_rows, c->at<double2>(L.rope),
                     c->at<uint16_t>(L.q), kc, vc, T, nq, L0, kv->c_max, Hq, Hkv, hd, v_blocks};
@@ -776,9 +901,8 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
     }
     {
       ProfScope ps_(c, DG_PROF_ATTENTION, st);
-      DG_TRY(run_attention(c->at<uint16_t>(L.q), kc, vc, c->at<uint16_t>(L.attn), c->at<float>(L.attn_po),
-                           c->at<float>(L.attn_pml), B, nq, L0, kv->c_max, Hq, Hkv, hd, causal, splits, err, st,
-                           &c->n_launch));
+      DG_TRY(run_attention(c->at<uint16_t>(L.q), kc, vc, c->at<uint16_t>(L.attn), nullptr, nullptr, B, nq, L0,
+                           kv->c_max, Hq, Hkv, hd, causal, splits, true, err, st, &c->n_launch));
     }
     {
       ProfScope ps_(c, DG_PROF_DENSE, st);
@@ -789,15 +913,28 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
       DG_TRY(make_bop(&tb, c->at<uint16_t>(L.attn), (long long)Hq * hd, L.T_alloc, bn));
       GemmPlan p = dense_plan(Hq * hd, d, T, bn, ks_o, err);
       p.a_hint = 1;
-      EpiStoreT e{c->at<float>(L.opart), d, (long long)T * d, 0, nullptr, nullptr, 0, err};
-      DG_TRY(run_gemm(ta, tb, p, e, c->num_sms, st, &c->n_launch));
+      if (DG_O_CLUSTER || ks_o == 1) {
+        p.cluster_k = ks_o;
+        EpiStoreT e{x, d, 0, 1, nullptr, nullptr, 0, err};  // residual add: x += attn W_o^T
+        DG_TRY(run_gemm(ta, tb, p, e, c->num_sms, st, &c->n_launch));
+      } else {
+        EpiStoreT e{c->at<float>(L.opart), d, (long long)T * d, 0, nullptr, nullptr, 0, err};
+        DG_TRY(run_gemm(ta, tb, p, e, c->num_sms, st, &c->n_launch));
+      }
     }
 
-    // --- mixture of experts block: residual add of the output projection + RMSNorm ---
-    residual_norm_kernel<1><<<T, row_launch(d).threads, 0, st>>>(x, c->at<float>(L.opart), ks_o,
-                                                                 (long long)T * d, d, c->wp(W.g_moe), xn,
-                                                                 m.rms_eps);
+    // --- mixture of experts block: residual add (split partials) + RMSNorm ---
+    NvtxRange nv_moe("dg.layer.moe_block");
+    {
+      const bool parts = !(DG_O_CLUSTER || ks_o == 1);
+      residual_norm_kernel<1><<<T, row_launch(d).threads, 0, st>>>(x, parts ? c->at<float>(L.opart) : nullptr,
+                                                                   parts ? ks_o : 0, (long long)T * d, d,
+                                                                   c->wp(W.g_moe), xn, m.rms_eps);
+    }
     CNT(c);
+    if (dbg_hidden_attn)
+      DG_CUDA(cudaMemcpyAsync(dbg_hidden_attn + (size_t)l * T * d, x, (size_t)T * d * 4,
+                              cudaMemcpyDeviceToDevice, st));
     {
       ProfScope ps_(c, DG_PROF_DENSE, st);
       CUtensorMap ta;
@@ -806,10 +943,15 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
       DG_TRY(make_tmap(&ta, c->wp(W.wr), d, c->wl.wr_rows, 128));
       DG_TRY(make_bop(&tb, xn, d, L.T_alloc, bn));
       GemmPlan p = dense_plan(d, E, T, bn, L.ks_r, err);
-      EpiStoreT e{c->at<float>(L.rpart), E, (long long)T * E, 0, nullptr, nullptr, 0, err};
-      DG_TRY(run_gemm(ta, tb, p, e, c->num_sms, st, &c->n_launch));
+      if (DG_ROUTER_CLUSTER) {
+        p.cluster_k = L.ks_r;  // final router logits [T, E]
+        EpiStoreT e{c->at<float>(L.rpart), E, 0, 0, nullptr, nullptr, 0, err};
+        DG_TRY(run_gemm(ta, tb, p, e, c->num_sms, st, &c->n_launch));
+      } else {
+        EpiStoreT e{c->at<float>(L.rpart), E, (long long)T * E, 0, nullptr, nullptr, 0, err};
+        DG_TRY(run_gemm(ta, tb, p, e, c->num_sms, st, &c->n_launch));
+      }
     }
-    if (L.ks_r != 4 && L.ks_r != 8) return fail(DG_ERR_UNSUPPORTED, "router split count %d", L.ks_r);
     {
       // top-k, counting sort by expert and row gather in one cooperative launch
       RouteParams rp;
@@ -840,8 +982,11 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
       lc.stream = st;
       lc.attrs = at;
       lc.numAttrs = 1;
-      if (L.ks_r == 8) DG_CUDA(cudaLaunchKernelEx(&lc, route_kernel<8>, rp));
-      else             DG_CUDA(cudaLaunchKernelEx(&lc, route_kernel<4>, rp));
+      const int ksr = DG_ROUTER_CLUSTER ? 1 : L.ks_r;
+      if (ksr == 8)      DG_CUDA(cudaLaunchKernelEx(&lc, route_kernel<8>, rp));
+      else if (ksr == 4) DG_CUDA(cudaLaunchKernelEx(&lc, route_kernel<4>, rp));
+      else if (ksr == 1) DG_CUDA(cudaLaunchKernelEx(&lc, route_kernel<1>, rp));
+      else return fail(DG_ERR_UNSUPPORTED, "router split count %d", ksr);
       CNT(c);
     }
     {
@@ -901,10 +1046,14 @@ extern "C" dg_status dg_encode_context(dg_ctx* c, dg_kv* kv, const int32_t* d_to
   if (n == 0) return DG_OK;
   if (!d_tokens) return fail(DG_ERR_INVALID_ARG, "tokens are null");
   cudaStream_t st = (cudaStream_t)stream;
+  NvtxRange nv("dg.encode_context");
   const int B = kv->batch, d = c->cfg.d_model;
-  int* tok_tmp = c->at<int>(c->L.st_samp);  // [T] staging of the chunk's token ids
-  for (int s0 = 0; s0 < n; s0 += DG_CANVAS) {
-    const int nq = std::min(DG_CANVAS, n - s0);
+  int* tok_tmp = c->at<int>(c->L.tok);  // [T] staging of the chunk's token ids
+  // chunks of as many tokens per canvas as a layer pass of the workspace holds
+  // (256, or more with a prefill workspace: one weight stream per chunk)
+  const int chunk = std::max(DG_CANVAS, c->L.T_alloc / B / 8 * 8);
+  for (int s0 = 0; s0 < n; s0 += chunk) {
+    const int nq = std::min(chunk, n - s0);
     const int T = B * nq;
     // gather the chunk's tokens into a dense [B, nq] block
     DG_CUDA(cudaMemcpy2DAsync(tok_tmp, (size_t)nq * 4, d_tokens + s0, (size_t)n * 4, (size_t)nq * 4, B,
@@ -912,7 +1061,7 @@ extern "C" dg_status dg_encode_context(dg_ctx* c, dg_kv* kv, const int32_t* d_to
     embed_kernel<<<T, 128, 0, st>>>(c->wp(c->wl.emb), tok_tmp, c->at<float>(c->L.x), T, d, c->cfg.vocab, c->err());
     CNT(c);
     DG_CUDA(cudaGetLastError());
-    DG_TRY(forward_layers(c, kv, B, nq, kv->length, true, nullptr, nullptr, nullptr, nullptr, st));
+    DG_TRY(forward_layers(c, kv, B, nq, kv->length, true, nullptr, nullptr, nullptr, nullptr, nullptr, st));
     kv->length += nq;
   }
   return DG_OK;
@@ -924,7 +1073,7 @@ extern "C" dg_status dg_canvas_init(dg_ctx* c, dg_canvas* cv, int32_t block, uin
   if (block < 0 || block > (1 << 23)) return fail(DG_ERR_INVALID_ARG, "block index");
   cudaStream_t st = (cudaStream_t)stream;
   const int n = cv->batch * DG_CANVAS;
-  canvas_init_kernel<<<(n + 255) / 256, 256, 0, st>>>(cv->tokens, cv->prev_argmax, cv->done, cv->batch, block,
+  canvas_init_kernel<<<(n + 255) / 256, 256, 0, st>>>(cv->tokens, cv->prev_argmax, cv->done, cv->locked, cv->batch, block,
                                                       (uint32_t)seed, (uint32_t)(seed >> 32), c->cfg.vocab);
                                                       CNT(c);
   DG_CUDA(cudaGetLastError());
@@ -951,6 +1100,7 @@ static StepDev step_dev(const dg_step_args* a) {
   v.require_stable = s.stop_require_stable_argmax;
   v.k0 = (uint32_t)s.seed;
   v.k1 = (uint32_t)(s.seed >> 32);
+  v.persistent = s.persistent_lock != 0;
   return v;
 }
 
@@ -967,6 +1117,7 @@ static dg_status check_round_args(dg_ctx* c, const dg_kv* kv, dg_canvas* cv, con
   if (s.lock_policy != DG_LOCK_PROB && s.lock_policy != DG_LOCK_ENTROPY_CUMSUM)
     return fail(DG_ERR_INVALID_ARG, "lock policy");
   if (!(s.t_start > 0.f) || !(s.t_end > 0.f)) return fail(DG_ERR_INVALID_ARG, "temperatures must be > 0");
+  if (s.persistent_lock && !cv->locked) return fail(DG_ERR_INVALID_ARG, "persistent lock needs canvas.locked");
   return DG_OK;
 }
 
@@ -996,6 +1147,7 @@ static dg_status enqueue_round(dg_ctx* c, const dg_kv* kv, dg_canvas* cv, const 
   }
 
   // a1: canvas embedding (+ self-conditioning input)
+  NvtxRange nv_round("dg.denoise_step");
   if (m.self_cond) {
     ProfScope ps_(c, DG_PROF_DENSE, st);
     CUtensorMap ta;
@@ -1018,11 +1170,12 @@ static dg_status enqueue_round(dg_ctx* c, const dg_kv* kv, dg_canvas* cv, const 
 
   // a2-a6: transformer layers, bidirectional over the canvas
   DG_TRY(forward_layers(c, kv, B, DG_CANVAS, kv->length, false, o->route_idx, o->route_w, o->route_logits,
-                        o->hidden, st));
+                        o->hidden, o->hidden_attn, st));
 
   // a7: final norm, LM head with online vocabulary statistics and sampling
+  NvtxRange nv_lm("dg.vocabulary_phase");  // a7-a9: LM head, statistics, expected embedding, update
   uint16_t* xn = c->at<uint16_t>(L.xn);  // final RMSNorm: fused into the last layer's combine
-  float* logits = o->logits ? o->logits : c->at<float>(L.logits);
+  uint16_t* logits = c->at<uint16_t>(L.logits);  // bf16, the expected embedding's input
   (void)s;
   VocabPartials vp{c->at<float>(L.vp_m), c->at<float>(L.vp_z), c->at<float>(L.vp_s), c->at<float>(L.vp_av),
                    c->at<int>(L.vp_ai), c->at<float>(L.vp_gv), c->at<int>(L.vp_gi)};
@@ -1030,14 +1183,17 @@ static dg_status enqueue_round(dg_ctx* c, const dg_kv* kv, dg_canvas* cv, const 
     ProfScope ps_(c, DG_PROF_LM_HEAD, st);
     CUtensorMap ta;
     BOperand tb;
+    // on CTA pairs: one tcgen05.mma.cta_group::2 covers 256 positions (both
+    // CTAs' 128-row A tiles) x 256 vocabulary ids, each CTA copying 128 of
+    // the ids; one CTA per SM (two 256-column accumulators per CTA)
     DG_TRY(make_tmap(&ta, xn, d, L.T_alloc, 128));
-    DG_TRY(make_bop(&tb, c->wp(c->wl.lm), d, V, 256));
+    DG_TRY(make_bop_half(&tb, c->wp(c->wl.lm), d, V, 256));
     GemmPlan p = dense_plan(d, T, V, 256, 1, err);
     p.n_fast = 0;
     p.a_hint = 2;
     p.b_hint = 1;
-    EpiLMHead e{logits, V, vp, L.n_vt, 256, sp, DG_CANVAS};
-    DG_TRY(run_gemm(ta, tb, p, e, c->num_sms, st, &c->n_launch));
+    EpiLMHead e{logits, o->logits, V, vp, L.n_vt, 256, sp, DG_CANVAS, kPurposeGumbel};
+    DG_TRY(run_gemm_pair(ta, tb, p, e, c->num_sms, st, &c->n_launch));
   }
   PosStats ps{c->at<float>(L.st_m), c->at<float>(L.st_iz), o->entropy ? o->entropy : c->at<float>(L.st_h),
               o->pmax ? o->pmax : c->at<float>(L.st_pmax), o->argmax ? o->argmax : c->at<int>(L.st_amax),
@@ -1049,17 +1205,18 @@ static dg_status enqueue_round(dg_ctx* c, const dg_kv* kv, dg_canvas* cv, const 
 
   // a8: expected embedding for the next round's self-conditioning input
   if (m.self_cond) {
+    NvtxRange nv_e("dg.expected_embedding");
     ProfScope ps_(c, DG_PROF_EXPECTED_EMB, st);
     uint16_t* probs = c->at<uint16_t>(L.probs);
-    const long long n4 = (long long)T * V / 4;
-    probs_kernel<<<(unsigned)std::min<long long>((n4 + 255) / 256, 148 * 16), 256, 0, st>>>(
+    const long long n8 = (long long)T * V / 8;
+    probs_kernel<<<(unsigned)std::min<long long>((n8 + 255) / 256, 148 * 16), 256, 0, st>>>(
         logits, ps.m, ps.inv_z, probs, T, V);
         CNT(c);
     const int ks = esum_splits(m, T, c->num_sms);
     CUtensorMap ta;
     BOperand tb;
     DG_TRY(make_tmap(&ta, c->wp(c->wl.embT), V, d, 128));
-    DG_TRY(make_bop(&tb, probs, V, L.T_alloc, bnT));
+    DG_TRY(make_bop(&tb, probs, V, L.T_canvas, bnT));
     GemmPlan p = dense_plan(V, d, T, bnT, ks, err);
     p.mt = kEsumMt;
     p.a_hint = 1;
@@ -1074,6 +1231,7 @@ static dg_status enqueue_round(dg_ctx* c, const dg_kv* kv, dg_canvas* cv, const 
   }
 
   // a9: mean entropy, stop, lock, next canvas
+  NvtxRange nv_u("dg.canvas_update");
   UpdateParams up{};
   up.entropy = ps.entropy;
   up.pmax = ps.pmax;
@@ -1087,6 +1245,7 @@ static dg_status enqueue_round(dg_ctx* c, const dg_kv* kv, dg_canvas* cv, const 
   up.stop_out = o->stop;
   up.final_out = o->final_round;
   up.flags = c->at<uint8_t>(L.flags);
+  up.locked = cv->locked;
   up.sp = sp;
   up.vocab = V;
   canvas_update_kernel<<<B, 256, 0, st>>>(up);
@@ -1107,10 +1266,11 @@ static bool same_key(const dg_ctx::GraphKey& a, const dg_ctx::GraphKey& b) {
   const dg_step_out &u = a.out, &w = b.out;
   return x.k == y.k && x.v == y.v && x.batch == y.batch && x.c_max == y.c_max && x.length == y.length &&
          p.tokens == q.tokens && p.sc_state == q.sc_state && p.prev_argmax == q.prev_argmax && p.done == q.done &&
-         p.batch == q.batch && u.argmax == w.argmax && u.sample == w.sample && u.entropy == w.entropy &&
+         p.batch == q.batch && p.locked == q.locked && u.argmax == w.argmax && u.sample == w.sample && u.entropy == w.entropy &&
          u.pmax == w.pmax && u.lock == w.lock && u.mean_entropy == w.mean_entropy && u.stop == w.stop &&
          u.final_round == w.final_round && u.logits == w.logits && u.route_idx == w.route_idx &&
-         u.route_w == w.route_w && u.route_logits == w.route_logits && u.hidden == w.hidden;
+         u.route_w == w.route_w && u.route_logits == w.route_logits && u.hidden == w.hidden &&
+         u.hidden_attn == w.hidden_attn;
 }
 
 extern "C" dg_status dg_denoise_step_graph(dg_ctx* c, const dg_kv* kv, dg_canvas* cv, const dg_step_args* a,
@@ -1169,6 +1329,61 @@ extern "C" dg_status dg_denoise_step_graph(dg_ctx* c, const dg_kv* kv, dg_canvas
   return DG_OK;
 }
 
+// Retained autoregressive mode: one token per canvas through the layers
+// (causal, appended to the context), then the final norm, LM head and
+// statistics of that position: argmax and the Gumbel-max draw of the next
+// token at `temperature`.
+extern "C" dg_status dg_ar_step(dg_ctx* c, dg_kv* kv, const int32_t* d_tokens, float temperature, uint64_t seed,
+                                int32_t* d_argmax, int32_t* d_sample, float* d_logits, void* stream) {
+  if (!c || !d_tokens || !d_argmax || !d_sample) return fail(DG_ERR_INVALID_ARG, "null argument");
+  if (!(temperature > 0.f)) return fail(DG_ERR_INVALID_ARG, "temperature must be > 0");
+  DG_TRY(check_kv(c, kv, 1));
+  cudaStream_t st = (cudaStream_t)stream;
+  NvtxRange nv("dg.ar_step");
+  const dg_model_config& m = c->cfg;
+  const WsLayout& L = c->L;
+  const int B = kv->batch, d = m.d_model, V = m.vocab, pos = kv->length;
+  int* err = c->err();
+  // round parameters of the draw: key = seed, c2 = the position
+  StepDev v{};
+  v.step = pos;
+  v.max_steps = 1;
+  v.block = 0;
+  v.inv_t = (float)(1.0 / (double)temperature);
+  v.k0 = (uint32_t)seed;
+  v.k1 = (uint32_t)(seed >> 32);
+  StepDev* sp = c->at<StepDev>(L.stepdev);
+  step_params_kernel<<<1, 32, 0, st>>>(sp, v);
+  CNT(c);
+  embed_kernel<<<B, 128, 0, st>>>(c->wp(c->wl.emb), d_tokens, c->at<float>(L.x), B, d, V, err);
+  CNT(c);
+  DG_CUDA(cudaGetLastError());
+  DG_TRY(forward_layers(c, kv, B, 1, pos, true, nullptr, nullptr, nullptr, nullptr, nullptr, st));
+  kv->length += 1;
+  uint16_t* xn = c->at<uint16_t>(L.xn);  // the final RMSNorm ran with the last layer's combine
+  VocabPartials vp{c->at<float>(L.vp_m), c->at<float>(L.vp_z), c->at<float>(L.vp_s), c->at<float>(L.vp_av),
+                   c->at<int>(L.vp_ai), c->at<float>(L.vp_gv), c->at<int>(L.vp_gi)};
+  {
+    CUtensorMap ta;
+    BOperand tb;
+    DG_TRY(make_tmap(&ta, xn, d, L.T_alloc, 128));
+    DG_TRY(make_bop_half(&tb, c->wp(c->wl.lm), d, V, 256));
+    GemmPlan p = dense_plan(d, B, V, 256, 1, err);
+    p.n_fast = 0;
+    p.a_hint = 2;
+    p.b_hint = 1;
+    EpiLMHead e{c->at<uint16_t>(L.logits), d_logits, V, vp, L.n_vt, 256, sp, 1, kPurposeArGumbel};
+    DG_TRY(run_gemm_pair(ta, tb, p, e, c->num_sms, st, &c->n_launch));
+  }
+  PosStats ps{c->at<float>(L.st_m), c->at<float>(L.st_iz), c->at<float>(L.st_h), c->at<float>(L.st_pmax), d_argmax,
+              d_sample};
+  vocab_merge_kernel<<<B, kMergeThreads, 0, st>>>(vp.m, vp.z, vp.s, vp.amax_v, vp.amax_i, vp.gkey_v, vp.gkey_i,
+                                                  L.n_vt, B, log((double)V), ps);
+  CNT(c);
+  DG_CUDA(cudaGetLastError());
+  return DG_OK;
+}
+
 extern "C" dg_status dg_check_device_error(dg_ctx* c, void* stream) {
   if (!c) return fail(DG_ERR_INVALID_ARG, "null context");
   DG_CUDA(cudaStreamSynchronize((cudaStream_t)stream));
@@ -1191,6 +1406,7 @@ extern "C" dg_status dg_decode_block(dg_ctx* c, dg_kv* kv, dg_canvas* cv, const 
   if (!c || !cv || !a || !d_out) return fail(DG_ERR_INVALID_ARG, "null argument");
   DG_TRY(check_kv(c, kv, DG_CANVAS));
   cudaStream_t st = (cudaStream_t)stream;
+  NvtxRange nv("dg.decode_block");
   const int B = cv->batch;
   DG_TRY(dg_canvas_init(c, cv, a->block, a->sampler.seed, stream));
   std::vector<uint8_t> flags(B, 0);
@@ -1215,6 +1431,71 @@ extern "C" dg_status dg_decode_block(dg_ctx* c, dg_kv* kv, dg_canvas* cv, const 
     h_stats->rounds = rounds;
     if (h_stats->steps_taken) memcpy(h_stats->steps_taken, steps.data(), B * sizeof(int32_t));
   }
+  return DG_OK;
+}
+
+// Router-load probe: the RMSNorm, router product and routing of one layer on
+// caller-given hidden states (the residual stream [T, d] fp32), as the layer
+// runs them in a round; writes each token's experts.
+extern "C" dg_status dg_router_probe(dg_ctx* c, int32_t layer, const float* d_x, int32_t T, int32_t* d_idx,
+                                     void* stream) {
+  if (!c || !d_x || !d_idx) return fail(DG_ERR_INVALID_ARG, "null argument");
+  const dg_model_config& m = c->cfg;
+  if (layer < 0 || layer >= m.n_layers) return fail(DG_ERR_INVALID_ARG, "layer %d outside [0, %d)", layer, m.n_layers);
+  if (T < 1 || T > c->L.T_alloc) return fail(DG_ERR_INVALID_ARG, "T %d outside [1, %d]", T, c->L.T_alloc);
+  cudaStream_t st = (cudaStream_t)stream;
+  const WsLayout& L = c->L;
+  const LayerW& W = c->wl.layers[layer];
+  const int d = m.d_model, E = m.n_experts, k = m.top_k;
+  int* err = c->err();
+  float* x = c->at<float>(L.x);
+  uint16_t* xn = c->at<uint16_t>(L.xn);
+  DG_CUDA(cudaMemcpyAsync(x, d_x, (size_t)T * d * 4, cudaMemcpyDeviceToDevice, st));
+  residual_norm_kernel<1><<<T, row_launch(d).threads, 0, st>>>(x, nullptr, 0, 0, d, c->wp(W.g_moe), xn, m.rms_eps);
+  DG_CUDA(cudaGetLastError());
+  {
+    CUtensorMap ta;
+    BOperand tb;
+    const int bn = std::max(32, dense_bn((E + 127) / 128, T, c->num_sms / L.ks_r));
+    DG_TRY(make_tmap(&ta, c->wp(W.wr), d, c->wl.wr_rows, 128));
+    DG_TRY(make_bop(&tb, xn, d, L.T_alloc, bn));
+    GemmPlan p = dense_plan(d, E, T, bn, L.ks_r, err);
+    if (DG_ROUTER_CLUSTER) p.cluster_k = L.ks_r;
+    EpiStoreT e{c->at<float>(L.rpart), E, DG_ROUTER_CLUSTER ? 0 : (long long)T * E, 0, nullptr, nullptr, 0, err};
+    DG_TRY(run_gemm(ta, tb, p, e, c->num_sms, st, &c->n_launch));
+  }
+  RouteParams rp;
+  rp.part = c->at<float>(L.rpart);
+  rp.xn = xn;
+  rp.T = T; rp.E = E; rp.k = k; rp.d = d; rp.bn = 128;
+  rp.tpc = (T + c->num_sms - 1) / c->num_sms;
+  rp.off = c->at<int>(L.off);
+  rp.chunk_off = c->at<int>(L.choff);
+  rp.perm = c->at<int>(L.perm);
+  rp.inv = c->at<int>(L.inv);
+  rp.w_perm = c->at<float>(L.wperm);
+  rp.xperm = c->at<uint16_t>(L.xperm);
+  rp.fill = c->at<int>(L.rfill);
+  rp.bar = c->at<int>(L.rbar);
+  rp.dbg_idx = d_idx;
+  rp.dbg_w = nullptr;
+  rp.dbg_logits = nullptr;
+  rp.err = err;
+  cudaLaunchConfig_t lc = {};
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeCooperative;
+  at[0].val.cooperative = 1;
+  lc.gridDim = dim3((T + rp.tpc - 1) / rp.tpc);
+  lc.blockDim = dim3(kRouteThreads);
+  lc.dynamicSmemBytes = route_smem_bytes(rp.tpc, k, E);
+  lc.stream = st;
+  lc.attrs = at;
+  lc.numAttrs = 1;
+  const int ksr = DG_ROUTER_CLUSTER ? 1 : L.ks_r;
+  if (ksr == 8)      DG_CUDA(cudaLaunchKernelEx(&lc, route_kernel<8>, rp));
+  else if (ksr == 4) DG_CUDA(cudaLaunchKernelEx(&lc, route_kernel<4>, rp));
+  else if (ksr == 1) DG_CUDA(cudaLaunchKernelEx(&lc, route_kernel<1>, rp));
+  else return fail(DG_ERR_UNSUPPORTED, "router split count %d", ksr);
   return DG_OK;
 }
 
@@ -1413,9 +1694,29 @@ extern "C" dg_status dg_test_attention(const uint16_t* q, const uint16_t* k, con
     return fail(DG_ERR_INVALID_ARG, "dg_test_attention: bad arguments");
   cudaStream_t st = (cudaStream_t)stream;
   if (splits == 0) splits = 1;
-  DG_TRY(run_attention(q, k, v, out, part_o, part_ml, B, nq, L0, c_max, Hq, Hkv, hd, causal != 0, splits, nullptr,
-                       st, nullptr));
+  // no partial buffers: the splits merge inside their cluster
+  const bool cluster = part_o == nullptr && part_ml == nullptr;
+  DG_TRY(run_attention(q, k, v, out, part_o, part_ml, B, nq, L0, c_max, Hq, Hkv, hd, causal != 0, splits, cluster,
+                       nullptr, st, nullptr));
   DG_CUDA(cudaStreamSynchronize(st));
+  return DG_OK;
+}
+
+// One thread waits, with a bounded wait of limit_ns, on an mbarrier that
+// nothing arrives on: the wait runs out, sets the error word and returns.
+__global__ void wait_timeout_kernel(int* err, unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x != 0) return;
+  mbar_init(smem_u32(&bar), 1);
+  fence_mbar_init();
+  mbar_wait(smem_u32(&bar), 0, err, limit_ns);
+}
+
+extern "C" dg_status dg_test_wait_timeout(dg_ctx* c, int64_t limit_ns, void* stream) {
+  if (!c || limit_ns <= 0 || limit_ns > 5000000000ll)
+    return fail(DG_ERR_INVALID_ARG, "dg_test_wait_timeout: limit must be in (0, 5 s]");
+  wait_timeout_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(c->err(), (unsigned long long)limit_ns);
+  DG_CUDA(cudaGetLastError());
   return DG_OK;
 }
 
@@ -1423,8 +1724,8 @@ extern "C" dg_status dg_test_workspace_buffer(dg_ctx* c, const char* name, void*
   if (!c || !name || !ptr || !bytes) return fail(DG_ERR_INVALID_ARG, "null argument");
   const WsLayout& L = c->L;
   struct Entry { const char* n; size_t off, next; };
-  const Entry tab[] = {{"x", L.x, L.xn}, {"xn", L.xn, L.qkv}, {"qkv", L.qkv, L.q}, {"q", L.q, L.attn},
-                       {"attn", L.attn, L.attn_po}, {"rpart", L.rpart, L.rbar},
+  const Entry tab[] = {{"x", L.x, L.xn}, {"xn", L.xn, L.qkv ? L.qkv : L.q}, {"q", L.q, L.attn},
+                       {"attn", L.attn, L.rpart}, {"rpart", L.rpart, L.rbar},
                        {"off", L.off, L.perm}, {"perm", L.perm, L.inv}, {"inv", L.inv, L.wperm},
                        {"wperm", L.wperm, L.xperm}, {"xperm", L.xperm, L.hperm}, {"hperm", L.hperm, L.yperm},
                        {"yperm", L.yperm, L.logits}, {"logits", L.logits, L.vp_m},
@@ -1442,7 +1743,6 @@ extern "C" dg_status dg_test_workspace_buffer(dg_ctx* c, const char* name, void*
 // ============================================================================
 // attention whose split-KV partials live in a fixed array of this library
 // (for callers that cannot allocate device memory)
-#include <mutex>
 
 static __device__ __align__(256) float g_attn_scratch[DG_ATTN_STATIC_SCRATCH_BYTES / sizeof(float)];
 

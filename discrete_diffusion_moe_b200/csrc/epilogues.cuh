@@ -70,6 +70,86 @@ struct EpiStoreT {
   }
 };
 
+// QKV projection with RoPE and the KV-cache write (the product's final values:
+// it runs with the cluster split-k reduction).  A = Wqkv with the rows of every
+// q and k head interleaved: head row j (j < hd/2) at physical row 2j and its
+// rotation partner j + hd/2 at 2j + 1, so a rotated pair sits in adjacent
+// accumulator lanes; v rows in natural order.  B = tokens t of the pass (B
+// canvases x nq positions, position L0 + t % nq).  Per pair: the even lane
+// outputs x_j cos - x_{j+hd/2} sin, the odd lane x_{j+hd/2} cos + x_j sin,
+// rotated in double from the fp32 sums and rounded once to bf16 (the angle's
+// (cos, sin) from the pass's table).  q goes to the packed grouped-query
+// layout, k to the K cache, v (its bf16 value held in fp16) to the transposed
+// V cache, each at the token's position.
+struct EpiQKV {
+  static constexpr int kEpiWarps = 8;
+  const double2* rope;  // [nq][hd / 2] (cos, sin) of positions L0 .. L0 + nq - 1
+  uint16_t* q;          // packed queries [B][Hkv][nq][G][hd] bf16
+  uint16_t* kc;         // layer base of the K cache [B][Hkv][c_max][hd] bf16
+  uint16_t* vc;         // layer base of the V^T cache [B][Hkv][hd][c_max] fp16
+  int nq, L0, c_max, Hq, Hkv, hd;
+  struct State {};
+  __device__ __forceinline__ void begin(const GemmJob&, int, State&) const {}
+  __device__ __forceinline__ void end(const GemmJob&, int, State&) const {}
+  __device__ __forceinline__ void chunk(const GemmJob& j, int row, int c0, const float (&v)[16],
+                                        State&) const {
+    float o[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) o[i] = __shfl_xor_sync(0xffffffffu, v[i], 1);
+    if (row >= j.m_valid) return;
+    const int f = j.m_tile * 128 + row;
+    const int qk_rows = (Hq + Hkv) * hd;
+    const int half = hd >> 1;
+    const int G = Hq / Hkv;
+    const int nv = min(16, j.n_valid - c0);
+    if (f < qk_rows) {
+      const int h = f / hd, w = f - h * hd;
+      const int jj = w >> 1, odd = w & 1;
+      const int dim = jj + odd * half;
+      const double sgn = odd ? 1.0 : -1.0;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        if (i >= nv) break;
+        const int t = j.n0 + c0 + i;
+        const int b = t / nq, pos = t - b * nq;
+        const double2 cs = __ldg(rope + (long long)pos * half + jj);
+        const uint16_t r = f32_to_bf16((float)((double)v[i] * cs.x + sgn * (double)o[i] * cs.y));
+        if (h < Hq) {
+          const int g = h / G, hh = h - g * G;
+          q[((((long long)b * Hkv + g) * nq + pos) * G + hh) * hd + dim] = r;
+        } else {
+          const int g = h - Hq;
+          kc[(((long long)b * Hkv + g) * c_max + L0 + pos) * hd + dim] = r;
+        }
+      }
+    } else {
+      const int g = (f - qk_rows) / hd, dim = (f - qk_rows) - g * hd;
+      const int t0 = j.n0 + c0;
+      const int b0 = t0 / nq, pos0 = t0 - b0 * nq;
+      uint16_t hv[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) hv[i] = bf16_to_f16(f32_to_bf16(v[i]));  // the bf16 value, held in fp16
+      if (nv == 16 && pos0 + 15 < nq && ((L0 + pos0) & 7) == 0) {
+        // 16 consecutive positions of one canvas: two 16-byte stores
+        uint16_t* dst = vc + (((long long)b0 * Hkv + g) * hd + dim) * c_max + L0 + pos0;
+        uint32_t w[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) w[e] = (uint32_t)hv[2 * e] | ((uint32_t)hv[2 * e + 1] << 16);
+        reinterpret_cast<uint4*>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        reinterpret_cast<uint4*>(dst)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          if (i >= nv) break;
+          const int t = t0 + i;
+          const int b = t / nq, pos = t - b * nq;
+          vc[(((long long)b * Hkv + g) * hd + dim) * c_max + L0 + pos] = hv[i];
+        }
+      }
+    }
+  }
+};
+
 // Grouped gate/up projection with SwiGLU.  The expert's [2 f, d] weight has
 // gate row j at 2j and up row j at 2j+1, so the pair sits in adjacent lanes:
 // h[slot, j] = bf16(silu(gate) * up) with silu(z) = z / (1 + e^-z).  The two
@@ -138,7 +218,8 @@ struct EpiDown {
 };
 
 // LM head (A = final normalised hidden states, one row per canvas position;
-// B = W_lm rows = vocabulary ids).  Stores the fp32 logits and keeps, per
+// B = W_lm rows = vocabulary ids).  Stores the logits in bf16 (the expected
+// embedding's input; fp32 too when a debug buffer is given) and keeps, per
 // position and per vocabulary tile, the online softmax statistics
 //   m = max l, Z = sum e^(l - m), S = sum e^(l - m) l,
 // the argmax (first maximum) and the Gumbel-max key argmax_v (l_v / T + g_v)
@@ -157,13 +238,15 @@ struct VocabPartials {
 
 struct EpiLMHead {
   static constexpr int kEpiWarps = 4;
-  float* logits;         // [T, V]
+  uint16_t* logits_bf16; // [T, V] bf16: the expected embedding's input (a8)
+  float* logits;         // optional [T, V] fp32 (debug output), may be null
   long long V;
   VocabPartials part;    // each [T, n_vt]
   int n_vt;              // vocabulary tiles (V / bn)
   int bn;
   const StepDev* sp;     // round parameters: Philox key, block, step, 1 / T_step
-  int canvas;            // positions per canvas (256)
+  int canvas;            // positions per canvas (256; 1 in the autoregressive mode)
+  uint32_t purpose;      // Philox purpose of the Gumbel draw
   struct State {
     float m, z, s, av, gv;
     int ai, gi;
@@ -182,9 +265,19 @@ struct EpiLMHead {
     if (row >= j.m_valid) return;
     const int t = j.m_tile * 128 + row;
     const int vb = j.n0 + c0;  // first vocabulary id of this chunk (multiple of 16)
-    float4* dst = reinterpret_cast<float4*>(logits + (long long)t * V + vb);
+    {
+      uint32_t w[8];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+      for (int e = 0; e < 8; ++e) w[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
+      uint4* dst = reinterpret_cast<uint4*>(logits_bf16 + (long long)t * V + vb);
+      dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+      dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    }
+    if (logits) {
+      float4* dst = reinterpret_cast<float4*>(logits + (long long)t * V + vb);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+    }
 
     float cm = v[0];
 #pragma unroll
@@ -203,7 +296,7 @@ struct EpiLMHead {
       if (v[i] > st.av) { st.av = v[i]; st.ai = vb + i; }
     }
     const int b = t / canvas, pos = t - b * canvas;
-    const uint32_t c3 = (kPurposeGumbel << 24) | (uint32_t)b;
+    const uint32_t c3 = (purpose << 24) | (uint32_t)b;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const Philox4 r = philox4x32_10((uint32_t)(vb >> 2) + q, (uint32_t)pos, st.c2, c3, st.k0, st.k1);

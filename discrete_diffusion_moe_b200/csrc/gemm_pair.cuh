@@ -5,7 +5,8 @@
 //
 //   D[m, n] = sum_k A[m, k] * B[n, k]      (bf16 inputs, fp32 accumulate)
 //
-// A unit is (group, pair of 128-row A tiles, chunk of at most bn B rows).
+// A unit is (group, pair of 128-row A tiles, chunk of at most bn B rows); a
+// dense plan (no groups, the LM head) has units (pair of A tiles, column tile).
 // CTA rank r of the pair copies its own A tile (tile 2 * pair + r) and half
 // of the unit's B rows (rows [r * N / 2, (r + 1) * N / 2) of the N = the
 // chunk's rows rounded up to 16); the MMA reads A from each CTA for its 128
@@ -35,22 +36,7 @@
 
 namespace dg {
 
-// ---- cluster / CTA-pair PTX ----------------------------------------------------------
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-// shared::cluster address of the same shared-memory location in CTA `rank`
-__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
-  return r;
-}
-// every thread of both CTAs (warps converged)
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
+// ---- CTA-pair PTX (cluster rank, mapa and the cluster barrier are in common.cuh) ----------
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t bar_cluster) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
 }
@@ -125,6 +111,7 @@ __device__ __forceinline__ void umma_commit_pair(uint32_t bar) {
 __host__ __device__ __forceinline__ int pair_tiles(const GemmPlan& p) { return (p.m_tiles + 1) >> 1; }
 
 __host__ __device__ __forceinline__ int pair_num_units(const GemmPlan& p, const GemmTables& tb) {
+  if (!p.group_off) return pair_tiles(p) * ((p.n_total + p.bn - 1) / p.bn);
   return pair_tiles(p) * tb.chunk_off[p.n_groups];
 }
 
@@ -133,6 +120,24 @@ __host__ __device__ __forceinline__ int pair_num_units(const GemmPlan& p, const 
 // m_valid <= 0 marks the missing second tile of a group with an odd tile count.
 __host__ __device__ __forceinline__ GemmJob pair_job(const GemmPlan& p, const GemmTables& tb, int u, int rank) {
   const int P = pair_tiles(p);
+  if (!p.group_off) {
+    // dense: unit u = (tile pair u % P, column tile u / P); consecutive units
+    // share a column tile (its B rows are read from L2 after the first)
+    GemmJob j;
+    const int pr = u % P, nt = u / P;
+    j.m_tile = 2 * pr + rank;
+    j.group = -1;
+    j.a_row0 = j.m_tile * 128;
+    j.m_valid = min(128, p.a_rows - j.m_tile * 128);
+    j.n_local0 = nt * p.bn;
+    j.n0 = j.n_local0;
+    j.n_valid = min(p.bn, p.n_total - j.n0);
+    j.ks = 0;
+    j.kb0 = 0;
+    j.kb1 = p.K / 64;
+    j.mt_eff = 1;
+    return j;
+  }
   int lo = 0, hi = p.n_groups;
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
@@ -191,7 +196,7 @@ __global__ void __launch_bounds__(gemm_threads<Epi>(), 2)
   const uint32_t rank = cluster_ctarank();
   const int cidx = (int)(blockIdx.x >> 1), ncl = (int)(gridDim.x >> 1);
   const uint32_t buf_cols = (uint32_t)p.bn;
-  const uint32_t tmem_cols = 2u * buf_cols <= 32u ? 32u : (2u * buf_cols <= 64u ? 64u : (2u * buf_cols <= 128u ? 128u : 256u));
+  const uint32_t tmem_cols = 2u * buf_cols <= 32u ? 32u : (2u * buf_cols <= 64u ? 64u : (2u * buf_cols <= 128u ? 128u : (2u * buf_cols <= 256u ? 256u : 512u)));
   const uint32_t acc_stride = tmem_cols / 2;  // two accumulator buffers
 
   if (threadIdx.x == 0) {
@@ -209,7 +214,7 @@ __global__ void __launch_bounds__(gemm_threads<Epi>(), 2)
     tma_prefetch_desc(&tmA);
     for (int i = 0; i < 3; ++i) tma_prefetch_desc(&tmB.m[i]);
   }
-  if (warp >= 2) {
+  if (warp >= 2 && p.group_off) {
     for (int g = threadIdx.x - 64; g <= p.n_groups; g += gemm_threads<Epi>() - 64) {
       tabs.chunk_off[g] = __ldg(p.chunk_off + g);
       tabs.group_off[g] = __ldg(p.group_off + g);
@@ -352,9 +357,13 @@ inline size_t gemm_pair_smem_bytes(int bn, int stages) {
   return 1024 + (size_t)stages * ((size_t)kATileBytes + (size_t)(bn / 2) * 128) + (2 * stages + 5) * 8 + 16;
 }
 
-// Stages that fit two pair CTAs in one SM's 228 KB.
+// CTAs per SM of the pair kernel: two, unless the two 256-column accumulator
+// buffers of a CTA take the whole tensor memory.
+inline int gemm_pair_ctas_per_sm(int bn) { return bn <= 128 ? 2 : 1; }
+
+// Stages that fit the pair CTAs of one SM in its 228 KB.
 inline int gemm_pair_stages(int bn, int max_stages = 8) {
-  const size_t budget = (size_t)228 * 1024 / 2 - 1024 - kGemmStaticSmem;
+  const size_t budget = (size_t)228 * 1024 / gemm_pair_ctas_per_sm(bn) - 1024 - kGemmStaticSmem;
   int s = max_stages;
   while (s > 2 && gemm_pair_smem_bytes(bn, s) > budget) --s;
   return s;

@@ -55,6 +55,9 @@ struct GemmPlan {
   int a_rows_per_group;  // grouped: A row stride between groups
   int a_hint, b_hint;    // L2 policy of the A / B loads: 0 none, 1 evict_first, 2 evict_last
   int mt;                // dense: 128-row A tiles per unit (1 or 2; grouped: 1)
+  int cluster_k;         // dense, > 1: the k_splits (== cluster_k) units of a tile are one
+                         // cluster and add their accumulators through distributed shared
+                         // memory before a single epilogue (one unit per CTA)
   int* err;              // device error word
 };
 
@@ -295,6 +298,32 @@ __global__ void __launch_bounds__(gemm_threads<Epi>(), 2)
       umma_commit(smem_u32(drain));
       mbar_wait(smem_u32(drain), 0, p.err);
     }
+  } else if (p.cluster_k > 1) {
+    // ---------------- cluster split-k, part 1: stage the accumulator ----------------
+    // (one unit per CTA; every copy into the stage ring has been consumed and
+    // every MMA has completed once acc_full fires, so the ring is free)
+    constexpr int CSTEP = Epi::kEpiWarps / 4;
+    const int quarter = warp & 3;
+    const int cfirst = (warp - 2) >> 2;
+    const int row = quarter * 32 + lane;
+    const GemmJob j = gemm_job(p, tabs, blockIdx.x, 0);
+    const bool ok = blockIdx.x < (unsigned)U && __all_sync(0xffffffffu, mbar_wait(smem_u32(&acc_full[0]), 0, p.err));
+    tc_fence_after();
+    const int pitch = p.bn + 4;
+    float* stg = reinterpret_cast<float*>(sA) + (size_t)row * pitch;
+    const int nch = (j.n_valid + 15) >> 4;
+    for (int c = cfirst; c < nch; c += CSTEP) {
+      float v[16];
+      if (ok) {
+        tmem_ld16(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(c * 16), v);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = 0.f;
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        *reinterpret_cast<float4*>(stg + c * 16 + 4 * e) = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+    }
   } else {
     // ---------------- epilogue (warps 2..5) ----------------
     static_assert(Epi::kEpiWarps == 4 || Epi::kEpiWarps == 8, "epilogue warps");
@@ -351,6 +380,47 @@ __global__ void __launch_bounds__(gemm_threads<Epi>(), 2)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (p.cluster_k > 1) {
+    // ---------------- cluster split-k, part 2: reduce and run the epilogue ----------------
+    // CTA `rank` of the cluster (its k split) takes the 16-column chunks
+    // c == rank (mod cluster_k) of the tile: each thread adds its row of the
+    // chunk from every CTA's staged accumulator in rank order (a fixed order:
+    // deterministic) and hands the sum to the functor, as split 0.
+    cluster_sync_all();  // every CTA's accumulator is staged
+    if (warp >= 2) {
+      constexpr int CSTEP = Epi::kEpiWarps / 4;
+      const int quarter = warp & 3;
+      const int cfirst = (warp - 2) >> 2;
+      const int row = quarter * 32 + lane;
+      const int rank = (int)cluster_ctarank();
+      GemmJob j = gemm_job(p, tabs, blockIdx.x, 0);
+      j.ks = 0;
+      j.kb0 = 0;
+      j.kb1 = p.K / 64;
+      const int nch = (j.n_valid + 15) >> 4;
+      const uint32_t stg = smem_u32(sA) + (uint32_t)(row * (p.bn + 4)) * 4u;
+      typename Epi::State st;
+      epi.begin(j, row, st);
+      int idx = 0;
+      for (int c = rank; c < nch; c += p.cluster_k, ++idx) {
+        if ((idx % CSTEP) != cfirst) continue;
+        float v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = 0.f;
+        for (int r = 0; r < p.cluster_k; ++r) {
+          const uint32_t src = mapa_shared(stg + (uint32_t)c * 64u, (uint32_t)r);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float4 a = ld_dsmem_f4(src + 16u * e);
+            v[4 * e] += a.x; v[4 * e + 1] += a.y; v[4 * e + 2] += a.z; v[4 * e + 3] += a.w;
+          }
+        }
+        epi.chunk(j, row, c * 16, v, st);
+      }
+      epi.end(j, row, st);
+    }
+    cluster_sync_all();  // no CTA leaves while another reads its shared memory
+  }
   if (warp == 1) tmem_dealloc(tmem_base, tmem_cols);
 }
 

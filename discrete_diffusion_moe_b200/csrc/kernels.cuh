@@ -1,5 +1,5 @@
 // kernels.cuh - bandwidth-bound kernels of the denoising step: embedding,
-// RMSNorm, RoPE + KV write, router top-k, token permutation, expert combine,
+// RMSNorm, RoPE table, router top-k, token permutation, expert combine,
 // vocabulary statistics merge, softmax probabilities, split-k reduction of
 // the expected embedding, the canvas update (entropy / lock / stop /
 // re-noise) and canvas initialisation.  All reductions that carry results
@@ -69,8 +69,8 @@ __global__ void __launch_bounds__(THREADS) rmsnorm_kernel(const float* __restric
 }
 
 // ---------------------------------------------------------------------------
-// x[t, :] += sum_s part[s, t, :] (split-k partials of the output projection, in
-// split order), then xn = bf16(x / rms(x) * gain).  One CTA per token with
+// x[t, :] += sum_s part[s, t, :] (ks split-k partials, in split order; none
+// when ks == 0), then xn = bf16(x / rms(x) * gain).  One CTA per token with
 // one float4 of the row per thread (NV per thread when the row is longer than
 // 4096): every load of the row is in flight at once and all tokens' CTAs are
 // resident together; the row stays in registers between the two passes.
@@ -89,15 +89,17 @@ __global__ void __launch_bounds__(1024) residual_norm_kernel(float* __restrict__
     const int c = (q * nt + threadIdx.x) * 4;
     r[q] = make_float4(0.f, 0.f, 0.f, 0.f);
     if (c < d) {
-      const float* pp = part + (long long)t * d + c;
-      float4 sum = *reinterpret_cast<const float4*>(pp);
-      for (int sp = 1; sp < ks; ++sp) {
-        const float4 v = *reinterpret_cast<const float4*>(pp + sp * split_stride);
-        sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
-      }
       float4 acc = *reinterpret_cast<const float4*>(xr + c);
-      acc.x += sum.x; acc.y += sum.y; acc.z += sum.z; acc.w += sum.w;
-      *reinterpret_cast<float4*>(xr + c) = acc;
+      if (ks > 0) {
+        const float* pp = part + (long long)t * d + c;
+        float4 sum = *reinterpret_cast<const float4*>(pp);
+        for (int sp = 1; sp < ks; ++sp) {
+          const float4 v = *reinterpret_cast<const float4*>(pp + sp * split_stride);
+          sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
+        }
+        acc.x += sum.x; acc.y += sum.y; acc.z += sum.z; acc.w += sum.w;
+        *reinterpret_cast<float4*>(xr + c) = acc;
+      }
       r[q] = acc;
       ss += acc.x * acc.x + acc.y * acc.y + acc.z * acc.z + acc.w * acc.w;
     }
@@ -138,10 +140,10 @@ inline RowLaunch row_launch(int d) {
 // ---------------------------------------------------------------------------
 // RoPE: pairs (i, i + hd/2) rotated by the angle pos * theta^(-2i/hd).  The
 // cos/sin of each (position, pair) are computed once per pass in double
-// (rope_table_kernel) and shared by all layers; the rotation is done in
-// double from the fp32 projection and rounded once to bf16.
-// q -> bf16 [T, Hq*hd]; k, v -> bf16 KV cache of this layer at position
-// L0 + i of each canvas ([B][Hkv][c_max][hd]).
+// (rope_table_kernel) and shared by all layers; the rotation runs in double
+// from the fp32 sums, rounded once to bf16: in the QKV projection's epilogue
+// (EpiQKV, when the projection's k splits add up in a cluster) or in
+// rope_kv_kernel from the projection's split-k partials.
 __global__ void rope_table_kernel(double2* __restrict__ tab, int nq, int L0, int half, int hd, double theta) {
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
   if (e >= nq * half) return;
@@ -167,10 +169,11 @@ struct RopeParams {
 constexpr int kRopeMaxSplits = 3; // split-k partials of the projection read by the kernel
 
 // Blocks [v_blocks, ...): one thread per (token, q or k head, 4 consecutive
-// pairs) rotates the 4 pairs (i, i + hd/2) .. (i + 3, i + 3 + hd/2): 16-byte
-// loads of every split-k partial (summed in split order) and of the 4
-// (cos, sin), all issued before the first is used, then two 8-byte stores
-// (q into the packed grouped-query layout, k into the cache).
+// pairs) rotates the 4 pairs (i, i + hd/2) .. (i + 3, i + 3 + hd/2) (rows
+// interleaved by pair, see EpiQKV): two 16-byte loads of every split-k
+// partial (summed in split order) and the 4 (cos, sin), all issued before the
+// first is used, then two 8-byte stores (q into the packed grouped-query
+// layout, k into the cache).
 // Threads [0, 256 v_blocks): one thread per (canvas, kv head, 4 consecutive
 // dims, position) moves 4 values of v into the transposed cache; the lanes of
 // a warp take consecutive positions, so each of the 4 stores of a warp is one
@@ -188,24 +191,26 @@ __global__ void __launch_bounds__(256) rope_kv_kernel(const RopeParams p) {
     const int rem = (int)(gid - (long long)t * per_tok);
     const int h = rem / n4, i = (rem - h * n4) * 4;
     const int b = t / p.nq, pos_in = t - b * p.nq;
-    const float* src = p.qkv + (long long)t * row_w + h * p.hd + i;
+    // q / k rows are interleaved by rotation pair: dim j at physical row 2j,
+    // dim j + hd/2 at 2j + 1, so pairs i .. i + 3 are 8 consecutive values
+    const float* src = p.qkv + (long long)t * row_w + h * p.hd + 2 * i;
     float4 a1[kRopeMaxSplits], a2[kRopeMaxSplits];
 #pragma unroll
     for (int q = 0; q < kRopeMaxSplits; ++q)
       if (q < p.ks) {
         a1[q] = __ldcg(reinterpret_cast<const float4*>(src + q * p.split_stride));
-        a2[q] = __ldcg(reinterpret_cast<const float4*>(src + q * p.split_stride + half));
+        a2[q] = __ldcg(reinterpret_cast<const float4*>(src + q * p.split_stride + 4));
       }
     const double2* tab = p.tab + (long long)pos_in * half + i;
     double2 cs[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) cs[u] = __ldg(tab + u);
-    float x1[4] = {a1[0].x, a1[0].y, a1[0].z, a1[0].w}, x2[4] = {a2[0].x, a2[0].y, a2[0].z, a2[0].w};
+    float x1[4] = {a1[0].x, a1[0].z, a2[0].x, a2[0].z}, x2[4] = {a1[0].y, a1[0].w, a2[0].y, a2[0].w};
 #pragma unroll
     for (int q = 1; q < kRopeMaxSplits; ++q)
       if (q < p.ks) {
-        x1[0] += a1[q].x; x1[1] += a1[q].y; x1[2] += a1[q].z; x1[3] += a1[q].w;
-        x2[0] += a2[q].x; x2[1] += a2[q].y; x2[2] += a2[q].z; x2[3] += a2[q].w;
+        x1[0] += a1[q].x; x1[1] += a1[q].z; x1[2] += a2[q].x; x1[3] += a2[q].z;
+        x2[0] += a1[q].y; x2[1] += a1[q].w; x2[2] += a2[q].y; x2[3] += a2[q].w;
       }
     uint16_t o1[4], o2[4];
 #pragma unroll
@@ -680,21 +685,25 @@ __global__ void __launch_bounds__(kMergeThreads) vocab_merge_kernel(
   }
 }
 
-// p[t, v] = bf16(exp(l[t, v] - m_t) / Z_t) — the softmax operand of the
-// expected-embedding product.
-__global__ void probs_kernel(const float* __restrict__ logits, const float* __restrict__ m,
+// p[t, v] = bf16(exp(l[t, v] - m_t) / Z_t) from the bf16 logits, with m_t
+// and Z_t the statistics of the fp32 logits — the softmax operand of the
+// expected-embedding product.  Eight values per thread (16-byte loads and
+// stores).
+__global__ void probs_kernel(const uint16_t* __restrict__ logits, const float* __restrict__ m,
                              const float* __restrict__ inv_z, uint16_t* __restrict__ p, int T,
                              long long V) {
-  const long long n4 = (long long)T * V / 4;
-  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n4;
+  const long long n8 = (long long)T * V / 8;
+  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n8;
        e += (long long)gridDim.x * blockDim.x) {
-    const long long t = (e * 4) / V;
+    const long long t = (e * 8) / V;
     const float mm = m[t], iz = inv_z[t];
-    const float4 l = reinterpret_cast<const float4*>(logits)[e];
-    uint2 o;
-    o.x = pack_bf16x2(__expf(l.x - mm) * iz, __expf(l.y - mm) * iz);
-    o.y = pack_bf16x2(__expf(l.z - mm) * iz, __expf(l.w - mm) * iz);
-    reinterpret_cast<uint2*>(p)[e] = o;
+    const uint4 l = reinterpret_cast<const uint4*>(logits)[e];
+    const uint32_t w[4] = {l.x, l.y, l.z, l.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      o[q] = pack_bf16x2(__expf(bf16_to_f32(w[q] & 0xFFFF) - mm) * iz, __expf(bf16_to_f32(w[q] >> 16) - mm) * iz);
+    reinterpret_cast<uint4*>(p)[e] = make_uint4(o[0], o[1], o[2], o[3]);
   }
 }
 
@@ -720,6 +729,7 @@ struct StepDev {
   float lock_threshold, stop_entropy, inv_t;
   int require_stable;
   uint32_t k0, k1;
+  int persistent;   // a locked position keeps its token for the rest of the block
 };
 
 __global__ void step_params_kernel(StepDev* dst, const StepDev v) {
@@ -740,6 +750,7 @@ struct UpdateParams {
   uint8_t* stop_out;    // may be null
   uint8_t* final_out;   // may be null
   uint8_t* flags;       // [B] internal copy of done after the update (host readback)
+  uint8_t* locked;      // [B, 256] committed positions (persistent lock; null otherwise)
   const StepDev* sp;    // round parameters
   int vocab;
 };
@@ -802,6 +813,9 @@ __global__ void __launch_bounds__(256) canvas_update_kernel(const UpdateParams p
     for (int r = 0; r < 256; ++r)
       if (kid[r] == i) { lock = csum[r] <= sp.lock_threshold; break; }
   }
+  // persistent lock: a position committed in an earlier round keeps its token
+  const bool committed = sp.persistent && p.locked && p.locked[t];
+  lock = lock || committed;
   if (p.lock_out) p.lock_out[t] = lock ? 1 : 0;
 
   const bool stable = sp.step > 0 && all_same;
@@ -809,7 +823,9 @@ __global__ void __launch_bounds__(256) canvas_update_kernel(const UpdateParams p
   const bool fin = !was_done && (stop || sp.step == sp.max_steps - 1);
   if (!was_done) {
     int nt;
-    if (fin) {
+    if (committed) {
+      nt = p.tokens[t];
+    } else if (fin) {
       nt = am;
     } else if (lock) {
       nt = smp;
@@ -820,6 +836,7 @@ __global__ void __launch_bounds__(256) canvas_update_kernel(const UpdateParams p
     }
     p.tokens[t] = nt;
     p.prev_argmax[t] = am;
+    if (sp.persistent && p.locked && lock) p.locked[t] = 1;
   }
   __syncthreads();
   if (i == 0) {
@@ -831,8 +848,9 @@ __global__ void __launch_bounds__(256) canvas_update_kernel(const UpdateParams p
   }
 }
 
-// Canvas initialisation: uniform tokens (purpose 1), prev_argmax = -1, done = 0.
-__global__ void canvas_init_kernel(int* tokens, int* prev_argmax, uint8_t* done, int B, int block,
+// Canvas initialisation: uniform tokens (purpose 1), prev_argmax = -1, done = 0,
+// locked = 0 (when given).
+__global__ void canvas_init_kernel(int* tokens, int* prev_argmax, uint8_t* done, uint8_t* locked, int B, int block,
                                    uint32_t k0, uint32_t k1, int vocab) {
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
   if (t >= B * 256) return;
@@ -841,6 +859,7 @@ __global__ void canvas_init_kernel(int* tokens, int* prev_argmax, uint8_t* done,
                                   (kPurposeInit << 24) | (uint32_t)b, k0, k1);
   tokens[t] = uniform_token(r.x, (uint32_t)vocab);
   prev_argmax[t] = -1;
+  if (locked) locked[t] = 0;
   if (i == 0) done[b] = 0;
 }
 

@@ -17,9 +17,10 @@ def model_config(n_layers, d_model, n_q_heads, n_kv_heads, head_dim, n_experts, 
 
 
 def sampler_config(lock_policy=DG_LOCK_PROB, lock_threshold=0.9, t_start=0.8, t_end=0.4, max_steps=48,
-                   stop_entropy=0.5, stop_require_stable_argmax=False, seed=0) -> dg_sampler_config:
+                   stop_entropy=0.5, stop_require_stable_argmax=False, seed=0,
+                   persistent_lock=False) -> dg_sampler_config:
     return dg_sampler_config(lock_policy, lock_threshold, t_start, t_end, max_steps, stop_entropy,
-                             int(bool(stop_require_stable_argmax)), seed)
+                             int(bool(stop_require_stable_argmax)), seed, int(bool(persistent_lock)))
 
 
 def _stream(stream=None):
@@ -68,8 +69,9 @@ class Canvas:
         self.sc_state = torch.zeros(batch, DG_CANVAS, cfg.d_model, dtype=torch.bfloat16, device=device)
         self.prev_argmax = torch.full((batch, DG_CANVAS), -1, dtype=torch.int32, device=device)
         self.done = torch.zeros(batch, dtype=torch.uint8, device=device)
+        self.locked = torch.zeros(batch, DG_CANVAS, dtype=torch.uint8, device=device)
         self.s = dg_canvas(self.tokens.data_ptr(), self.sc_state.data_ptr(), self.prev_argmax.data_ptr(),
-                           self.done.data_ptr(), batch)
+                           self.done.data_ptr(), batch, self.locked.data_ptr())
 
 
 class StepOutputs:
@@ -109,35 +111,45 @@ class StepOutputs:
                              if routing else None)
         self.hidden = (torch.zeros(cfg.n_layers + 1, T, cfg.d_model, dtype=torch.float32, device=device)
                        if hidden else None)
+        self.hidden_attn = (torch.zeros(cfg.n_layers, T, cfg.d_model, dtype=torch.float32, device=device)
+                            if hidden else None)
         self.s = dg_step_out(*[t.data_ptr() if t is not None else None for t in (
             self.argmax, self.sample, self.entropy, self.pmax, self.lock, self.mean_entropy, self.stop,
-            self.final_round, self.logits, self.route_idx, self.route_w, self.route_logits, self.hidden)])
+            self.final_round, self.logits, self.route_idx, self.route_w, self.route_logits, self.hidden,
+            self.hidden_attn)])
 
 
 class Model:
     """Weights + workspace + context handle for up to `batch` canvases."""
 
     def __init__(self, cfg: dg_model_config, batch: int, seed: int = 0, kind_std=None, device="cuda",
-                 stream=None):
+                 stream=None, weights_of=None, prefill_tokens: int = 0):
+        """weights_of: another Model whose weight buffer this one shares (a
+        second context, e.g. for a larger batch, on the same weights).
+        prefill_tokens: encode passes of up to that many tokens."""
         self.cfg = cfg
         self.batch = batch
         nw = lib.dg_weights_bytes(ctypes.byref(cfg))
         if nw == 0:
             raise ValueError(lib.dg_last_error().decode())
-        self.weights = torch.empty(nw, dtype=torch.uint8, device=device)
-        nws = lib.dg_workspace_bytes(ctypes.byref(cfg), batch)
+        nws = lib.dg_workspace_bytes_ex(ctypes.byref(cfg), batch, prefill_tokens)
         self.workspace = torch.empty(nws, dtype=torch.uint8, device=device)
-        std = None
-        if kind_std:
-            arr = (ctypes.c_float * 32)()
-            for kind, v in kind_std.items():
-                arr[kind] = v
-            std = ctypes.cast(arr, ctypes.c_void_p)
-            self._std = arr
-        check(lib.dg_model_init_random(ctypes.byref(cfg), seed, std, _ptr(self.weights), _stream(stream)))
+        if weights_of is not None:
+            assert weights_of.weights.numel() == nw
+            self.weights = weights_of.weights
+        else:
+            self.weights = torch.empty(nw, dtype=torch.uint8, device=device)
+            std = None
+            if kind_std:
+                arr = (ctypes.c_float * 32)()
+                for kind, v in kind_std.items():
+                    arr[kind] = v
+                std = ctypes.cast(arr, ctypes.c_void_p)
+                self._std = arr
+            check(lib.dg_model_init_random(ctypes.byref(cfg), seed, std, _ptr(self.weights), _stream(stream)))
         ctx = ctypes.c_void_p()
-        check(lib.dg_context_create(ctypes.byref(cfg), _ptr(self.weights), _ptr(self.workspace), nws, batch,
-                                    ctypes.byref(ctx)))
+        check(lib.dg_context_create_ex(ctypes.byref(cfg), _ptr(self.weights), _ptr(self.workspace), nws, batch,
+                                       prefill_tokens, ctypes.byref(ctx)))
         self.ctx = ctx
 
     def close(self):
@@ -177,3 +189,17 @@ class Model:
 
     def check_device(self, stream=None):
         check(lib.dg_check_device_error(self.ctx, _stream(stream)))
+
+    def ar_step(self, kv: KVCache, tokens: torch.Tensor, temperature: float, seed: int, out_argmax: torch.Tensor,
+                out_sample: torch.Tensor, out_logits: torch.Tensor = None, stream=None):
+        """Autoregressive mode: append tokens [B] (int32) to the context and
+        write the next token's argmax and sample [B] (int32)."""
+        assert tokens.dtype == torch.int32 and out_argmax.dtype == torch.int32 and out_sample.dtype == torch.int32
+        check(lib.dg_ar_step(self.ctx, ctypes.byref(kv.s), _ptr(tokens), float(temperature), int(seed),
+                             _ptr(out_argmax), _ptr(out_sample), _ptr(out_logits), _stream(stream)))
+
+    def router_probe(self, layer: int, x: torch.Tensor, out_idx: torch.Tensor, stream=None):
+        """Route hidden states x [T, d] (fp32) with layer `layer`'s router into
+        out_idx [T, top_k] (int32)."""
+        assert x.dtype == torch.float32 and x.is_contiguous() and out_idx.dtype == torch.int32
+        check(lib.dg_router_probe(self.ctx, layer, _ptr(x), x.shape[0], _ptr(out_idx), _stream(stream)))

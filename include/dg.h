@@ -93,6 +93,11 @@ typedef struct dg_sampler_config {
   float stop_entropy;                  /* stop when mean entropy < this (nats) */
   int32_t stop_require_stable_argmax;  /* also require argmax == previous round's */
   uint64_t seed;                       /* Philox4x32-10 key of the method's draws */
+  int32_t persistent_lock;             /* 0: the lock mask is recomputed every round and locked
+                                          tokens may change later (the method: laozijiushiniubi.cn
+                                          article §一); 1: the masked-style variant, a position once
+                                          locked keeps its token for the rest of the block (needs
+                                          dg_canvas.locked) */
 } dg_sampler_config;
 
 /* Causally encoded context, one K and one V buffer of dg_kv_bytes() each:
@@ -120,6 +125,8 @@ typedef struct dg_canvas {
   int32_t* prev_argmax;  /* [B, 256] argmax of the previous round */
   uint8_t* done;         /* [B] 1 once the canvas has stopped (frozen) */
   int32_t batch;
+  uint8_t* locked;       /* [B, 256] positions committed so far (persistent_lock only; may be
+                            NULL otherwise); dg_canvas_init clears it */
 } dg_canvas;
 
 typedef struct dg_step_args {
@@ -144,6 +151,8 @@ typedef struct dg_step_out {
   float* route_logits;    /* optional [n_layers, B*256, n_experts] fp32 router logits */
   float* hidden;          /* optional [n_layers + 1, B*256, d_model] fp32 residual stream after
                              the embedding (a1) and after each layer */
+  float* hidden_attn;     /* optional [n_layers, B*256, d_model] fp32 residual stream after each
+                             layer's attention block (the input of its router and experts) */
 } dg_step_out;
 
 /* Host-side statistics of one dg_decode_block call. */
@@ -165,6 +174,13 @@ size_t dg_weights_bytes(const dg_model_config* cfg);
 size_t dg_kv_bytes(const dg_model_config* cfg, int32_t batch, int32_t c_max);
 /* Bytes of the scratch workspace for up to `batch` canvases. */
 size_t dg_workspace_bytes(const dg_model_config* cfg, int32_t batch);
+/* The same for a context whose causal encodes (dg_encode_context) run passes
+   of up to prefill_tokens tokens (all canvases together; 0 or anything up to
+   batch * 256 gives dg_workspace_bytes).  Larger passes read every layer's
+   weights once per pass instead of once per 256 tokens: the prompt's
+   prefill becomes compute-bound (laozijiushiniubi.cn article §二: the prompt
+   is encoded causally, in one go). */
+size_t dg_workspace_bytes_ex(const dg_model_config* cfg, int32_t batch, int32_t prefill_tokens);
 
 /* Fill the weight buffer with seeded random-init weights: every matrix from
    the seeded generator of synth/synth.h (approximately N(0, std^2), bf16)
@@ -179,17 +195,24 @@ dg_status dg_model_init_random(const dg_model_config* cfg, uint64_t seed, const 
    overlap on the GPU.  *out is NULL on failure. */
 dg_status dg_context_create(const dg_model_config* cfg, const void* d_weights, void* d_workspace,
                             size_t ws_bytes, int32_t batch, dg_ctx** out);
+/* dg_context_create for a workspace of dg_workspace_bytes_ex(cfg, batch,
+   prefill_tokens) bytes. */
+dg_status dg_context_create_ex(const dg_model_config* cfg, const void* d_weights, void* d_workspace,
+                               size_t ws_bytes, int32_t batch, int32_t prefill_tokens, dg_ctx** out);
 void dg_context_destroy(dg_ctx* ctx);
 
 /* Causal encoding (laozijiushiniubi.cn article §二: the prompt is encoded with
    causal attention): tokens [kv->batch, n] (device int32) are appended at
    positions kv->length .. kv->length + n - 1 of every layer's K/V, then
-   kv->length += n.  Processed in chunks of 256 tokens per canvas. */
+   kv->length += n.  Processed in passes of up to max(256, prefill_tokens /
+   batch) tokens per canvas (prefill_tokens of dg_context_create_ex; the
+   canvas batch of the context). */
 dg_status dg_encode_context(dg_ctx* ctx, dg_kv* kv, const int32_t* d_tokens, int32_t n,
                             void* stream);
 
 /* Initialise a canvas for block `block`: uniform random tokens (Philox draw
-   purpose 1), zero self-conditioning state, prev_argmax = -1, done = 0. */
+   purpose 1), zero self-conditioning state, prev_argmax = -1, done = 0,
+   locked = 0 (when given). */
 dg_status dg_canvas_init(dg_ctx* ctx, dg_canvas* cv, int32_t block, uint64_t seed, void* stream);
 
 /* One denoising round over every canvas (the steps a1-a9: embedding plus
@@ -200,7 +223,9 @@ dg_status dg_canvas_init(dg_ctx* ctx, dg_canvas* cv, int32_t block, uint64_t see
    and the next canvas: locked positions keep their sample, the others are
    re-noised uniformly; on stop or at the last budgeted round the canvas
    becomes the argmax sequence and is frozen).  Canvases already done are
-   left unchanged. */
+   left unchanged.  With sampler.persistent_lock a position locked in an
+   earlier round keeps its token (and counts as locked) in every later round,
+   the final round included; the other positions follow the rules above. */
 dg_status dg_denoise_step(dg_ctx* ctx, const dg_kv* kv, dg_canvas* cv, const dg_step_args* args,
                           const dg_step_out* out, void* stream);
 
@@ -219,6 +244,20 @@ dg_status dg_denoise_step_graph(dg_ctx* ctx, const dg_kv* kv, dg_canvas* cv, con
    dg_encode_context.  `args->step` is ignored.  h_stats may be NULL. */
 dg_status dg_decode_block(dg_ctx* ctx, dg_kv* kv, dg_canvas* cv, const dg_step_args* args,
                           int32_t* d_out, dg_block_stats* h_stats, void* stream);
+
+/* Retained autoregressive mode (laozijiushiniubi.cn article §七: the same
+   weights still generate one token at a time), the comparison workload of
+   the method: d_tokens [kv->batch] (device int32) are appended at position
+   P = kv->length of each canvas's context with causal attention (the causal
+   encode of one token), then that position's final RMSNorm, LM head and
+   vocabulary statistics give the next token: its argmax (ties to the lower
+   id) to d_argmax [batch] and its Gumbel-max draw from softmax(l /
+   temperature) to d_sample [batch] (Philox4x32-10 with key = seed, counter
+   (c0 = v / 4, c1 = 0, c2 = P, c3 = 5 << 24 | canvas), word v % 4).
+   d_logits (optional, NULL for none) [batch, vocab] fp32.  kv->length += 1.
+   Asynchronous on `stream`; uses the context's workspace. */
+dg_status dg_ar_step(dg_ctx* ctx, dg_kv* kv, const int32_t* d_tokens, float temperature, uint64_t seed,
+                     int32_t* d_argmax, int32_t* d_sample, float* d_logits, void* stream);
 
 /* Synchronise `stream` and report (then clear) the device error word:
    DG_OK, DG_ERR_BAD_TOKEN or DG_ERR_TIMEOUT. */
@@ -249,6 +288,15 @@ dg_status dg_profile_start(dg_ctx* ctx);
 /* Stop, synchronise the recorded events and fill *out. */
 dg_status dg_profile_stop(dg_ctx* ctx, dg_profile* out);
 
+/* Router-load probe (measurement hook): layer `layer`'s RMSNorm, router
+   product and top-k routing on T (1 <= T <= the context's batch * 256) given
+   hidden states d_x [T, d_model] fp32 (device), exactly as that layer routes
+   its residual stream in a round; d_idx [T, top_k] int32 (device) receives
+   each token's experts (selection order).  It uses the context's workspace,
+   so it must not overlap other calls on the context.  Asynchronous. */
+dg_status dg_router_probe(dg_ctx* ctx, int32_t layer, const float* d_x, int32_t T, int32_t* d_idx,
+                          void* stream);
+
 /* ---- attention without caller-provided scratch ---------------------------
    The pages have no counterpart for this call.  It is for callers that cannot
    allocate device memory when they call in: code that runs inside a memory
@@ -271,12 +319,13 @@ dg_status dg_profile_stop(dg_ctx* ctx, dg_profile* out);
    alignment) must fit the array; a larger request returns DG_ERR_INVALID_ARG
    and launches nothing.  splits 0 or 1 uses no scratch.
    Set-up: the first call on each GPU (that GPU current) looks up the array's
-   address; make that first call before any stream capture begins.
+   address (cudaGetSymbolAddress; nothing is allocated); make that first call
+   before any stream capture begins.
    Nothing has to start at zero: each call writes every partial it reads.
    One array per GPU: calls on the same GPU that may run at the same time
    (several host threads, or streams with no ordering between them) race on
-   it, so the caller serialises them.  The call returns after its work on
-   `stream` has finished. */
+   it, so the caller serialises them.  Every call synchronises `stream` (it
+   waits for its work there to finish) before it returns. */
 #define DG_ATTN_STATIC_SCRATCH_BYTES (16u << 20)
 dg_status dg_attention_static_scratch(const uint16_t* d_q, const uint16_t* d_k, const uint16_t* d_v,
                                       uint16_t* d_out, int32_t B, int32_t nq, int32_t L0, int32_t c_max,

@@ -73,15 +73,25 @@ dg_status dg_test_dense_schedule(int32_t M, int32_t N, int32_t K, int32_t bn, in
    V cache transposed, fp16 [B][Hkv][hd][c_max], both holding keys
    [0, L0 + nq); c_max a multiple of 8; out bf16 [B * nq, Hq * hd]
    (token-major).  causal = 0: every query sees all L0 + nq keys; causal = 1:
-   query i sees keys [0, L0 + i].  splits (1..8; 0 means 1) key splits; for
-   splits > 1 the partial buffers come from the caller: part_o fp32
-   [splits * B * Hq * nq * hd] and part_ml fp32 [splits * B * Hq * nq * 2],
-   rows in packed query order [split][b][kv head][token * G + head in group].
+   query i sees keys [0, L0 + i].  splits (1..8; 0 means 1) key splits.  For
+   splits > 1 with part_o and part_ml both NULL, the splits of each tile run
+   as one thread-block cluster and merge through distributed shared memory
+   (the form the layers use); otherwise the partial buffers come from the
+   caller: part_o fp32 [splits * B * Hq * nq * hd] and part_ml fp32
+   [splits * B * Hq * nq * 2], rows in packed query order
+   [split][b][kv head][token * G + head in group], merged by a second kernel.
    head_dim one of 32, 64, 128, 176.  Synchronous. */
 dg_status dg_test_attention(const uint16_t* d_q, const uint16_t* d_k, const uint16_t* d_v, uint16_t* d_out,
                             int32_t B, int32_t nq, int32_t L0, int32_t c_max, int32_t Hq, int32_t Hkv,
                             int32_t hd, int32_t causal, int32_t splits, float* d_part_o,
                             float* d_part_ml, void* stream);
+
+/* Failure-path hook: one thread of a one-CTA kernel waits, with a bounded
+   wait of limit_ns (0 < limit_ns <= 5e9), on an mbarrier that nothing arrives
+   on.  The wait runs out, the kernel latches DG_ERR_TIMEOUT in the context's
+   device error word and returns, so the next dg_check_device_error reports
+   (and clears) it and the context stays usable.  Asynchronous on `stream`. */
+dg_status dg_test_wait_timeout(dg_ctx* ctx, int64_t limit_ns, void* stream);
 
 /* Device address and size of one named scratch buffer of a context's
    workspace (for inspecting the last layer's intermediates after a call):
@@ -89,7 +99,7 @@ dg_status dg_test_attention(const uint16_t* d_q, const uint16_t* d_k, const uint
    "q" bf16 [T, Hq*hd], "attn" bf16 [T, Hq*hd], "rpart" fp32 split-k router
    partial logits [splits, T, E], "off" int32 [E+1], "perm", "inv" int32 [T*k],
    "wperm" fp32 [T*k], "xperm" bf16 [T*k, d], "hperm" bf16 [T*k, f],
-   "yperm" fp32 [T*k, d], "logits" fp32 [T, V], "probs" bf16 [T, V]. */
+   "yperm" fp32 [T*k, d], "logits" bf16 [T, V], "probs" bf16 [T, V]. */
 dg_status dg_test_workspace_buffer(dg_ctx* ctx, const char* name, void** d_ptr, size_t* bytes);
 
 #ifdef __cplusplus
