@@ -28,14 +28,15 @@ def bound(ref, n_keys, ref_abs):
     oracle:
       - one bf16 ulp of the output (2^-7 relative: the final rounding plus the
         small error that can push it across a rounding boundary);
-      - the probabilities enter the P V product as fp16 (relative rounding
-        error <= 2^-11 each), so the output moves by at most
-        2^-11 * sum_j p_j |v_j| = 2^-11 * (attention over |V|), given as
-        ref_abs; 2^-10 leaves a factor 2;
+      - the probabilities enter the P V product as two fp16 parts, P_hi =
+        fp16(P) and P_lo = fp16(P - P_hi) (relative error <= 2^-22 each,
+        plus fp16 subnormals of P_lo for the smallest probabilities), so the
+        output moves by at most about 2^-22 * (attention over |V|), given as
+        ref_abs; 2^-20 leaves a factor 4;
       - an absolute floor for fp32 accumulation in the tensor cores' own
         order: the rounding noise of a sum over n_keys terms grows like
         sqrt(n_keys) * 2^-24 times the size of the partial sums (at most
         max|ref|-sized after normalisation); 2^-22 * sqrt(n_keys) * max|ref|
         leaves a factor 4."""
-    return (2.0 ** -7 * np.abs(ref) + 2.0 ** -10 * ref_abs
+    return (2.0 ** -7 * np.abs(ref) + 2.0 ** -20 * ref_abs
             + 2.0 ** -22 * np.sqrt(n_keys) * np.abs(ref).max())

@@ -71,3 +71,24 @@ def test_size_queries_and_argument_errors_without_gpu(lib):
     with pytest.raises(dg.DgError) as e:
         dg.dg_context_create(cfg, None, None, 0, 1)
     assert e.value.status == dg.DG_ERR_INVALID_ARG
+
+
+def test_workspace_too_small_is_refused_before_any_device_work(lib):
+    # the size check comes before the context touches the workspace, so fake
+    # (aligned, never dereferenced) addresses suffice and no GPU is needed
+    import discrete_diffusion_moe_b200 as dg
+    cfg = dg.model_config(2, 256, 8, 8, 32, 16, 2, 512, 4096)
+    need = dg.dg_workspace_bytes(cfg, 2)
+    assert need > 0
+    with pytest.raises(dg.DgError) as e:
+        dg.dg_context_create(cfg, 1 << 20, 2 << 20, need - 256, 2)
+    assert e.value.status == dg.DG_ERR_WORKSPACE
+    assert "workspace too small" in dg.last_error()
+    # a misaligned workspace is an argument error
+    with pytest.raises(dg.DgError) as e:
+        dg.dg_context_create(cfg, 1 << 20, (2 << 20) + 8, need, 2)
+    assert e.value.status == dg.DG_ERR_INVALID_ARG
+    # so is a batch outside [1, 64]
+    with pytest.raises(dg.DgError) as e:
+        dg.dg_context_create(cfg, 1 << 20, 2 << 20, need, 65)
+    assert e.value.status == dg.DG_ERR_INVALID_ARG

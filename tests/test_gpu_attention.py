@@ -20,15 +20,21 @@ pytestmark = pytest.mark.gpu
     (1, 256, 300, 8, 8, 32, 0, 8), (1, 256, 2048, 16, 8, 176, 0, 5), (2, 256, 77, 8, 8, 32, 0, 4),
     (1, 256, 1024, 8, 4, 64, 0, 4), (1, 130, 70, 8, 2, 128, 1, 2), (3, 256, 1024, 16, 8, 176, 0, 1),
     (1, 1, 0, 16, 8, 176, 0, 1), (1, 256, 8000, 16, 8, 176, 0, 8)])
-def test_attention_matches_oracle(B, nq, L0, Hq, Hkv, hd, causal, splits):
+@pytest.mark.parametrize("merge", ["cluster", "scratch"])
+def test_attention_matches_oracle(B, nq, L0, Hq, Hkv, hd, causal, splits, merge):
+    """merge: the key splits of a tile merge inside their thread-block cluster
+    (the layers' form), or through caller scratch and a second kernel."""
     import discrete_diffusion_moe_b200 as dg
+    if merge == "scratch" and splits == 1:
+        pytest.skip("one split has nothing to merge")
     dev, ref = attn_inputs.make(B, nq, L0, Hq, Hkv, hd, seed=nq + L0 + hd + splits)
-    out = torch.zeros(B * nq, Hq * hd, dtype=torch.bfloat16, device="cuda")
+    out = torch.full((B * nq, Hq * hd), float("nan"), dtype=torch.bfloat16, device="cuda")
     po = torch.zeros(max(splits, 1) * B * Hq * nq * hd, device="cuda")
     pml = torch.zeros(max(splits, 1) * B * Hq * nq * 2, device="cuda")
+    p_o, p_ml = (None, None) if merge == "cluster" else (po.data_ptr(), pml.data_ptr())
     dg.check(dg.lib.dg_test_attention(dev["q"].data_ptr(), dev["k"].data_ptr(), dev["v"].data_ptr(), out.data_ptr(),
-                                      B, nq, L0, dev["c_max"], Hq, Hkv, hd, causal, splits, po.data_ptr(),
-                                      pml.data_ptr(), torch.cuda.current_stream().cuda_stream))
+                                      B, nq, L0, dev["c_max"], Hq, Hkv, hd, causal, splits, p_o, p_ml,
+                                      torch.cuda.current_stream().cuda_stream))
     got = out.float().cpu().numpy().reshape(B, nq, Hq, hd)
     for b in range(B):
         pos, kpos = np.arange(L0, L0 + nq), np.arange(L0 + nq)

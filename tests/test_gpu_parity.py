@@ -1,7 +1,8 @@
 """GPU (C ABI) vs oracle parity of the denoising step on seeded synthetic
 inputs: context encoding, canvas initialisation, logits, routing, per-position
 statistics, samples, lock masks, stop flags, the next canvas and the
-self-conditioning state, step by step."""
+self-conditioning state, step by step -- every stage on the GPU's own input
+(strict decision gate) and the whole step free-running (tests/parity.py)."""
 
 import pytest
 
@@ -10,11 +11,19 @@ from parity import Case, TINY, LAYER1, run_case
 pytestmark = pytest.mark.gpu
 
 
+def _compared(rep, steps, batch=1):
+    """Every step compared every stage at every position, and some positions
+    end to end."""
+    assert rep.steps == steps, rep
+    assert rep.tf_decisions > 0 and rep.tf_positions == steps * 256 * batch, rep
+    assert rep.compared_positions > 0 and rep.logit_rel > 0 and rep.tf_logit_rel > 0, rep
+
+
 def test_tiny_decode_prob_lock():
     """2 layers, d 256, 8 heads x 32, 16 experts top-2, vocab 4096, 64 context
     tokens, one canvas, 4 rounds, lock on max prob > 0.9, Philox seed 1234."""
     rep = run_case(Case(cfg=TINY, ctx_len=64, steps=4))
-    assert rep.steps == 4 and rep.compared_positions > 0, rep
+    _compared(rep, 4)
 
 
 def test_tiny_self_cond_entropy_cumsum_lock_batch2():
@@ -23,21 +32,30 @@ def test_tiny_self_cond_entropy_cumsum_lock_batch2():
     ragged context length (not a multiple of 64)."""
     rep = run_case(Case(cfg=TINY, self_cond=True, ctx_len=77, batch=2, steps=3, lm_std=2.0,
                         sampler=dict(lock_policy="entropy_cumsum", lock_threshold=0.1)))
-    assert rep.steps >= 1, rep
+    _compared(rep, 3, batch=2)
 
 
 def test_tiny_peaked_prob_lock_and_stop():
     """Locks fire (pmax > 0.9) and the adaptive stop fires at its threshold."""
     rep = run_case(Case(cfg=TINY, ctx_len=300, steps=3, lm_std=2.5,
                         sampler=dict(stop_entropy=3.0, stop_require_stable_argmax=False)))
-    assert rep.steps >= 1, rep
+    _compared(rep, 3)
+
+
+def test_tiny_persistent_lock_variant():
+    """The masked-style variant (persistent lock): a position locked in an
+    earlier round keeps its token in every later round; peaked LM head so
+    that positions lock, four rounds."""
+    rep = run_case(Case(cfg=TINY, ctx_len=48, steps=4, lm_std=2.5,
+                        sampler=dict(persistent_lock=True, stop_entropy=0.0)))
+    _compared(rep, 4)
 
 
 def test_single_layer_full_width_step():
     """1 layer, d 2816, 16 q / 8 kv heads x 176, 128 experts top-8, ffn 704,
     vocab 262144, 2048 context tokens, one canvas, one round."""
     rep = run_case(Case(cfg=LAYER1, ctx_len=2048, steps=1))
-    assert rep.steps == 1, rep
+    _compared(rep, 1)
 
 
 @pytest.mark.parametrize("n_experts,top_k,ctx_len", [(4, 4, 0), (6, 1, 17), (6, 3, 64), (256, 8, 0), (256, 8, 64)])
@@ -50,14 +68,14 @@ def test_tiny_degenerate_routing_and_context(n_experts, top_k, ctx_len):
     ragged one."""
     cfg = dict(TINY, n_experts=n_experts, top_k=top_k)
     rep = run_case(Case(cfg=cfg, ctx_len=ctx_len, steps=2))
-    assert rep.steps == 2, rep
+    _compared(rep, 2)
 
 
 def test_tiny_batch8_canvases():
     """Eight canvases in one round (2,048 canvas tokens, 4,096 routed pairs
     over 16 experts): every canvas against the oracle."""
     rep = run_case(Case(cfg=TINY, ctx_len=40, batch=8, steps=2))
-    assert rep.steps == 2, rep
+    _compared(rep, 2, batch=8)
 
 
 @pytest.mark.parametrize("shape", [
@@ -70,7 +88,7 @@ def test_width_and_grouped_query_shapes(shape):
     ratio (G = 4, head_dim 64), end to end against the oracle."""
     cfg = dict(n_layers=1, n_experts=8, top_k=2, d_ff=256, vocab=4096, **shape)
     rep = run_case(Case(cfg=cfg, ctx_len=70, steps=2))
-    assert rep.steps == 2, rep
+    _compared(rep, 2)
 
 
 def test_tiny_largest_batch():
@@ -78,4 +96,4 @@ def test_tiny_largest_batch():
     and 32,768 routed pairs in one round; 111 tokens per routing CTA), one
     round end to end against the oracle."""
     rep = run_case(Case(cfg=TINY, ctx_len=16, batch=64, steps=1))
-    assert rep.steps == 1, rep
+    _compared(rep, 1, batch=64)

@@ -40,4 +40,6 @@ def test_step_outputs_pack_results_in_one_block(batch):
     assert tuple(full.route_idx.shape) == (2, batch * 256, 2)
     assert tuple(full.route_logits.shape) == (2, batch * 256, 16)
     assert tuple(full.hidden.shape) == (3, batch * 256, 256)
+    assert tuple(full.hidden_attn.shape) == (2, batch * 256, 256)
+    assert full.s.hidden_attn == full.hidden_attn.data_ptr()
     assert full.s.logits == full.logits.data_ptr()
