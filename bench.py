@@ -220,6 +220,120 @@ def oracle_sample(wl, threads):
     return per_step, desc, t4 - t0
 
 
+def time_steps(dg, model, kv, cv, samp, block, steps, warm, stream):
+    """Mean ms of `steps` graph-replayed rounds after `warm` untimed ones."""
+    model.canvas_init(cv, block, SEED)
+    s_ = 0
+    for _ in range(warm):
+        model.step(kv, cv, block, s_, samp, graph=True)
+        s_ += 1
+    import torch
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        model.step(kv, cv, block, s_, samp, graph=True)
+        s_ += 1
+    e1.record(stream)
+    torch.cuda.synchronize()
+    model.check_device()
+    return e0.elapsed_time(e1) / steps
+
+
+def routed_distinct(dg, cfg, model, kv, cv, samp, B, n_layers):
+    """Distinct experts per layer (over all canvases) of one more round."""
+    import torch
+    out = dg.StepOutputs(cfg, B, routing=True)
+    model.canvas_init(cv, 1, SEED)
+    model.step(kv, cv, 1, 0, samp, out)
+    torch.cuda.synchronize()
+    ridx = out.route_idx.cpu()
+    return [int(torch.unique(ridx[l]).numel()) for l in range(n_layers)]
+
+
+def line_roofline(cfg_d, B, ctx, distinct, ms, peaks):
+    flops, nbytes = step_cost(cfg_d, B, ctx, distinct)
+    t_f = flops / (peaks["bf16_tflops_sustained"] * 1e12)
+    t_b = nbytes / (peaks["hbm_gbs"] * 1e9)
+    return {"flops": flops, "bytes": nbytes, "t_ms": 1000 * max(t_f, t_b), "bound": "hbm" if t_b >= t_f else "tensor",
+            "frac": max(t_f, t_b) / (ms / 1000.0)}
+
+
+def other_configs(dg, synth, model, wl, rank, peaks, stream, steps=5, warm=3):
+    """The benchmark's other configurations, measured in the same run:
+    the single-layer full-width step (context 2048, one canvas), the batch x
+    context sweep on the full-size model (B canvases of 256 tokens, B in
+    {1, 2, 4, 8, 16}, each with its own causal context of C in {1024, 8192,
+    32768} random tokens), and the router-load probe (every layer's router on
+    N(0, 1) hidden states of 256 tokens)."""
+    import torch
+    res = {}
+    samp = dg.sampler_config(max_steps=MAX_STEPS, stop_entropy=0.5, lock_threshold=0.9, seed=SEED + rank)
+    # single-layer full-width step
+    w1 = WORKLOADS["layer1"]
+    c1 = w1["cfg"]
+    cfg1 = dg.model_config(**c1)
+    m1 = dg.Model(cfg1, 1, seed=0)
+    kv1 = dg.KVCache(cfg1, 1, w1["ctx"] + CANVAS)
+    m1.encode(kv1, torch.from_numpy(synth.context_tokens(1, w1["ctx"], 1234 + rank, c1["vocab"])).cuda())
+    cv1 = dg.Canvas(cfg1, 1)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    ms_list = []
+    for _ in range(steps):        # its 3 GB of weights fit in L2 twice over: flush L2 before each round
+        flush.zero_()
+        ms_list.append(time_steps(dg, m1, kv1, cv1, samp, 0, 1, warm if not ms_list else 0, stream))
+    ms1 = statistics.median(ms_list)
+    dist1 = routed_distinct(dg, cfg1, m1, kv1, cv1, samp, 1, 1)
+    res["single_layer_full_width"] = {"workload": "1 layer, d 2816, 128 experts top-8, vocab 262144, context 2048, "
+                                                  "one canvas; L2 flushed before each round",
+                                      "ms_per_step": ms1, "steps_per_s": 1000.0 / ms1,
+                                      "distinct_experts": dist1[0],
+                                      "roofline": line_roofline(c1, 1, w1["ctx"], dist1, ms1, peaks)}
+    m1.close()
+    del m1, kv1, cv1, flush
+    torch.cuda.empty_cache()
+    # batch x context sweep on the full-size model (shared weights, one context per batch)
+    c = wl["cfg"]
+    cfg = dg.model_config(**c)
+    sweep = []
+    for B in (16, 8, 4, 2, 1):
+        mb = dg.Model(cfg, B, weights_of=model)
+        kvb = dg.KVCache(cfg, B, 32768 + CANVAS)
+        mb.encode(kvb, torch.from_numpy(synth.context_tokens(B, 32768, 1234 + rank, c["vocab"])).cuda())
+        mb.check_device()
+        cvb = dg.Canvas(cfg, B)
+        for C in (32768, 8192, 1024):   # descending: a round's canvas keys overwrite [C, C + 256)
+            kvb.s.length = C
+            ms = time_steps(dg, mb, kvb, cvb, samp, 0, steps, warm, stream)
+            dist = routed_distinct(dg, cfg, mb, kvb, cvb, samp, B, c["n_layers"])
+            sweep.append({"batch": B, "context": C, "ms_per_step": ms, "steps_per_s": 1000.0 / ms,
+                          "canvas_tok_per_s": B * CANVAS * 1000.0 / ms,
+                          "distinct_experts_per_layer": sum(dist) / len(dist),
+                          "roofline": line_roofline(c, B, C, dist, ms, peaks)})
+        mb.close()
+        del mb, kvb, cvb
+        torch.cuda.empty_cache()
+    res["batch_context_sweep"] = sweep
+    # router-load probe: N(0, 1) hidden states of 256 tokens through every layer's router
+    x = torch.from_numpy(synth.f32_tensor(CANVAS * c["d_model"], 7, 905, 1.0).reshape(CANVAS, c["d_model"])).cuda()
+    idx = torch.zeros(CANVAS, c["top_k"], dtype=torch.int32, device="cuda")
+    per_layer = []
+    for l in range(c["n_layers"]):
+        model.router_probe(l, x, idx)
+        cnt = torch.bincount(idx.reshape(-1).long(), minlength=c["n_experts"]).cpu()
+        per_layer.append({"distinct": int((cnt > 0).sum()), "max_load": int(cnt.max()),
+                          "cv": float(cnt.float().std() / cnt.float().mean())})
+    model.check_device()
+    res["router_load_probe"] = {
+        "inputs": "256 hidden states N(0, 1) (seeded generator), each layer's RMSNorm + router + top-8",
+        "distinct_experts_mean": sum(p["distinct"] for p in per_layer) / len(per_layer),
+        "max_load_mean": sum(p["max_load"] for p in per_layer) / len(per_layer),
+        "load_cv_mean": sum(p["cv"] for p in per_layer) / len(per_layer),
+        "per_layer_distinct": [p["distinct"] for p in per_layer]}
+    return res
+
+
 def max_over_ranks(x, world):
     """The largest value of x over the ranks of the job (a job's time is its
     slowest rank's).  One process per GPU: NCCL tensors live on the rank's
@@ -289,6 +403,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode-loop", action="store_true")
+    ap.add_argument("--no-other-configs", action="store_true")
     args = ap.parse_args()
     wl = WORKLOADS[args.workload]
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -444,6 +559,9 @@ def main():
                "d2h_bytes_per_step": d2h, "steps": n_e2e}
 
     peaks = load_peaks()
+    extra = None
+    if not args.no_other_configs and args.workload == "full":
+        extra = other_configs(dg, synth, model, wl, rank, peaks, stream)
     flops, nbytes = step_cost(c, B, ctx, distinct)
     t_roof = max(flops / (peaks["bf16_tflops_sustained"] * 1e12), nbytes / (peaks["hbm_gbs"] * 1e9))
     # dominant kernel: grouped expert gate/up projection + SwiGLU (one launch per layer)
@@ -488,6 +606,7 @@ def main():
             "clocks": clk,
             "e2e": e2e,
             "cpu_baseline": cpu,
+            "other_configs": extra,
         }
         print(json.dumps(line), flush=True)
     model.close()
