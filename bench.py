@@ -42,6 +42,11 @@ WORKLOADS = {
     "moe1": dict(cfg=dict(n_layers=1, d_model=2816, n_q_heads=16, n_kv_heads=8, head_dim=176,
                           n_experts=128, top_k=8, d_ff=704, vocab=16384, self_cond=False),
                  ctx=1024, batch=1),
+    # the same with the self-conditioning product and expected embedding (vocabulary 16384):
+    # the workload for captures of the LM-head / expected-embedding kernels
+    "moe1sc": dict(cfg=dict(n_layers=1, d_model=2816, n_q_heads=16, n_kv_heads=8, head_dim=176,
+                            n_experts=128, top_k=8, d_ff=704, vocab=16384, self_cond=True),
+                   ctx=1024, batch=1),
     # tiny: 2 layers, d 256, 16 experts top-2, vocab 4096, context 64
     "tiny": dict(cfg=dict(n_layers=2, d_model=256, n_q_heads=8, n_kv_heads=8, head_dim=32, n_experts=16,
                           top_k=2, d_ff=512, vocab=4096, self_cond=False),
@@ -156,68 +161,98 @@ def ncu_traffic(kernel_key):
 # ---------------------------------------------------------------------------
 # CPU baseline: the oracle, timed on a bounded sample of the workload
 
-def oracle_sample(wl, threads):
-    """Time the oracle on a sample of one step and scale it to the whole
-    step.  Sample: transformer layer 0 over the 256 canvas tokens (keys: a
-    synthetic context of the workload's length + the canvas), the LM head over
-    one 16384-id block of the vocabulary, and the per-position statistics,
-    Gumbel sample and expected embedding of 8 positions over the full
-    vocabulary.  Weights are generated before timing (inputs).  Returns
-    (seconds per step, description)."""
-    import numpy as np
+def oracle_setup(wl, threads):
+    """The oracle's inputs for timing one step of the workload (generated, not
+    timed: weights and tokens are inputs): the model, a context KV cache of the
+    workload's length (synthetic keys / values, as the GPU's encode would
+    leave), the canvas and its embedding."""
     import oracle
     import synth
     from oracle import decode as OD
-    from oracle import sampler as OS
-    from oracle.model import forward_layers, lm_logits
     c = wl["cfg"]
-    ocfg1 = oracle.ModelConfig(**dict(c, n_layers=1))
-    W = oracle.Weights(ocfg1, seed=0, threads=threads, keep_chunks=True)
-    W.layer(0)
+    ocfg = oracle.ModelConfig(**c)
+    W = oracle.Weights(ocfg, seed=0, threads=threads, keep_chunks=True)
     ctx = wl["ctx"]
-    kv = oracle.KVCache(ocfg1, 1, ctx + CANVAS)
-    kv.k[0][:, :ctx] = synth.f32_tensor(ctx * c["n_kv_heads"] * c["head_dim"], 3, 900, 1.0).reshape(
-        1, ctx, c["n_kv_heads"], c["head_dim"])
-    kv.v[0][:, :ctx] = synth.f32_tensor(ctx * c["n_kv_heads"] * c["head_dim"], 3, 901, 1.0).reshape(
-        1, ctx, c["n_kv_heads"], c["head_dim"])
+    kv = oracle.KVCache(ocfg, 1, ctx + CANVAS)
+    for l in range(c["n_layers"]):
+        kv.k[l][:, :ctx] = synth.f32_tensor(ctx * c["n_kv_heads"] * c["head_dim"], 3, 900 + 2 * l, 1.0).reshape(
+            1, ctx, c["n_kv_heads"], c["head_dim"])
+        kv.v[l][:, :ctx] = synth.f32_tensor(ctx * c["n_kv_heads"] * c["head_dim"], 3, 901 + 2 * l, 1.0).reshape(
+            1, ctx, c["n_kv_heads"], c["head_dim"])
     kv.length = ctx
     toks = OD.init_canvas(SEED, 0, 1, CANVAS, c["vocab"])
     x0 = W.emb_rows(toks).reshape(1, CANVAS, c["d_model"])
-    chunk = 16384
+    return ocfg, W, kv, x0
+
+
+def oracle_tail_sample(wl, W, x, threads, n_pos=8, chunk=16384):
+    """Seconds of the oracle's vocabulary phase of one step, from timed
+    samples: the LM head over one 16384-id block (x V / 16384), the statistics
+    and Gumbel sample of n_pos positions (x 256 / n_pos) and the expected
+    embedding over one 16384-id block (x V / 16384).  Returns (seconds, desc)."""
+    import numpy as np
+    import oracle
+    import synth
+    from oracle import sampler as OS
+    from oracle.model import lm_logits
+    c = wl["cfg"]
     vcfg = oracle.ModelConfig(**dict(c, n_layers=1, vocab=chunk))
     Wv = oracle.Weights(vcfg, seed=0, threads=threads, keep_chunks=True)
     Wv.lm_chunk(0, chunk)
-    n_pos = 8
-    W.emb_chunk(0, chunk)
+    Wv.emb_chunk(0, chunk)
     t0 = time.perf_counter()
-    x = forward_layers(ocfg1, W, x0, kv, causal=False, append=False)
-    t1 = time.perf_counter()
     lm_logits(vcfg, Wv, x.reshape(CANVAS, -1), chunk=chunk)
-    t2 = time.perf_counter()
+    t1 = time.perf_counter()
     rng_logits = synth.f32_tensor(n_pos * c["vocab"], 5, 902, 1.0).reshape(n_pos, c["vocab"])
-    probs = []
     for i in range(n_pos):
-        _, _, _, p = OS.position_stats(rng_logits[i])
+        OS.position_stats(rng_logits[i])
         OS.position_sample(rng_logits[i], np.float32(1.25), SEED, 0, 0, 0, i)
-        probs.append(p)
-    t3 = time.perf_counter()
-    t4 = t3
+        OS.selfcond_probs(rng_logits[i])
+    t2 = time.perf_counter()
+    t3 = t2
     if c["self_cond"]:
-        vc = oracle.ModelConfig(**dict(c, n_layers=1, vocab=chunk))
-        We = oracle.Weights(vc, seed=0, threads=threads, keep_chunks=True)
-        We._chunks[(synth.KIND_EMB, 0, chunk)] = W.emb_chunk(0, chunk)
         p_all = np.full((CANVAS, chunk), 1.0 / c["vocab"])
+        t2 = time.perf_counter()
+        OS.expected_embedding(p_all, Wv, chunk=chunk)
         t3 = time.perf_counter()
-        OS.expected_embedding(p_all, We, chunk=chunk)
-        t4 = time.perf_counter()
-    per_step = ((t1 - t0) * c["n_layers"] + (t2 - t1) * (c["vocab"] / chunk)
-                + (t3 - t2) * (CANVAS / n_pos) + (t4 - t3) * (c["vocab"] / chunk))
-    desc = (f"oracle (numpy float64) timed on: layer 0 of {c['n_layers']} over the 256-token canvas with "
-            f"{ctx} context keys (x{c['n_layers']}), LM head over 16384 of {c['vocab']} ids "
-            f"(x{c['vocab'] // chunk}), statistics and Gumbel sample of {n_pos} of 256 positions "
-            f"(x{CANVAS // n_pos}), expected embedding over 16384 ids (x{c['vocab'] // chunk}); "
-            f"weight generation excluded")
-    return per_step, desc, t4 - t0
+    reps = c["vocab"] / chunk
+    sec = (t1 - t0) * reps + (t2 - t1) * (CANVAS / n_pos) + (t3 - t2) * reps
+    desc = (f"LM head over {chunk} of {c['vocab']} ids (x{reps:g}), statistics and Gumbel sample of {n_pos} of "
+            f"256 positions (x{CANVAS // n_pos})" + (f", expected embedding over {chunk} ids (x{reps:g})"
+                                                   if c["self_cond"] else ""))
+    return sec, desc
+
+
+def oracle_sample(wl, threads, distinct):
+    """The oracle's seconds per step from timed samples: layer 0's attention
+    block, router and experts timed separately (seconds per routed expert
+    from its experts block), every layer costed as attention + router +
+    (its measured distinct experts) x (seconds per expert), plus the timed
+    vocabulary-phase samples.  `distinct`: experts per layer of the GPU's
+    own round.  Returns (seconds per step, description, wall seconds)."""
+    import numpy as np
+    from oracle import model as OM
+    c = wl["cfg"]
+    w0 = time.perf_counter()
+    ocfg, W, kv, x0 = oracle_setup(dict(wl, cfg=dict(c, n_layers=1)), threads)
+    lw = W.layer(0)
+    t0 = time.perf_counter()
+    xm = OM.attention_block(ocfg, lw, x0, kv.k[0], kv.v[0], wl["ctx"], causal=False, append=False)
+    t1 = time.perf_counter()
+    OM.router_block(ocfg, lw, xm)
+    t2 = time.perf_counter()
+    x1, (idx, _, _, _) = OM.moe_block(ocfg, lw, xm)
+    t3 = time.perf_counter()
+    e0 = len(np.unique(np.asarray(idx)))
+    t_attn, t_route = t1 - t0, t2 - t1
+    t_exp = max(0.0, (t3 - t2) - t_route) / max(e0, 1)
+    layers = sum(t_attn + t_route + e * t_exp for e in distinct)
+    tail, tdesc = oracle_tail_sample(wl, W, x1, threads)
+    desc = (f"oracle (numpy float64): layer 0 timed (attention {t_attn:.2f} s, router {t_route:.2f} s, "
+            f"{e0} experts {t3 - t2 - t_route:.2f} s); each of the {c['n_layers']} layers costed as attention + "
+            f"router + its routed experts (the GPU round's distinct experts per layer, mean "
+            f"{sum(distinct) / len(distinct):.1f}) x {t_exp:.3f} s; {tdesc}; inputs generated outside the timing")
+    return layers + tail, desc, time.perf_counter() - w0
 
 
 def time_steps(dg, model, kv, cv, samp, block, steps, warm, stream):
@@ -356,21 +391,47 @@ def cpu_cores():
 
 
 def reference_arm(args, wl, rank, world):
+    """The oracle on the host cores.  Each step times one real layer of the
+    oracle's own chain for the workload's canvas (step i runs layer i mod L on
+    the stream the previous step left) plus the vocabulary-phase samples; a
+    step's value is the whole round costed from them: the layers timed so
+    far, each untimed layer at the mean of the timed layers past layer 0,
+    plus the vocabulary phase."""
     if rank != 0:
         return 0
+    import numpy as np
+    from oracle import model as OM
     cores = cpu_cores()
-    times = []
-    desc = ""
+    c = wl["cfg"]
+    L = c["n_layers"]
+    ocfg, W, kv, x = oracle_setup(wl, cores)
+    layer_s = {}
+    times, sample_s = [], []
+    tail, descs = oracle_tail_sample(wl, W, x, cores)   # the vocabulary phase, timed once
     for i in range(args.warmup + args.steps):
-        per_step, desc, _ = oracle_sample(wl, threads=cores)
+        l = i % L
+        lw = W.layer(l)                       # generated outside the timing
+        t0 = time.perf_counter()
+        x, _ = OM.layer_forward(ocfg, lw, x, kv.k[l], kv.v[l], wl["ctx"], causal=False, append=False)
+        t1 = time.perf_counter()
+        layer_s[l] = t1 - t0
+        deep = [v for k, v in layer_s.items() if k > 0] or [layer_s[0]]
+        est = sum(layer_s.get(k, sum(deep) / len(deep)) for k in range(L)) + tail
         if i >= args.warmup:
-            times.append(per_step)
+            times.append(est)
+            sample_s.append(t1 - t0)
     v = 1.0 / statistics.mean(times)
+    desc = (f"oracle (numpy float64) on {cores} cores: one real layer of its own {L}-layer chain per step "
+            f"(layers 0..{min(L, args.warmup + args.steps) - 1} timed), the untimed layers at the mean of the "
+            f"timed ones past layer 0; once per run: {descs}; inputs generated outside the timing")
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * statistics.mean(times),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": workload_config(args, wl, world),
-            "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc,
+                             "sample_s_per_step": statistics.mean(sample_s),
+                             "note": "ms_per_step is the whole round costed from the timed samples; the "
+                                     "timed work per step is sample_s_per_step"},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -381,6 +442,7 @@ def workload_config(args, wl, world):
     return {"workload": {"full": "full-size single step (30 layers, self-conditioning, context 1024, batch 1)",
                          "layer1": "single-layer full-width step (context 2048, batch 1)",
                          "moe1": "single full-width layer, vocabulary 16384 (context 1024, batch 1)",
+                         "moe1sc": "single full-width layer, vocabulary 16384, self-conditioning (context 1024, batch 1)",
                          "tiny": "tiny 2-layer step (context 64, batch 1)"}[args.workload],
             "n_layers": c["n_layers"], "d_model": c["d_model"], "heads": f"{c['n_q_heads']}q/{c['n_kv_heads']}kv x {c['head_dim']}",
             "experts": f"{c['n_experts']} top-{c['top_k']} ffn {c['d_ff']}", "vocab": c["vocab"],
@@ -579,7 +641,7 @@ def main():
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
             cores = cpu_cores()
-            per_step, desc, wall = oracle_sample(wl, threads=cores)
+            per_step, desc, wall = oracle_sample(wl, threads=cores, distinct=distinct)
             cpu = {"value": 1.0 / per_step, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc,
                    "sample_wall_s": wall}
         line = {
