@@ -305,6 +305,8 @@ def other_configs(dg, synth, model, wl, rank, peaks, stream, steps=5, warm=3):
     import torch
     res = {}
     samp = dg.sampler_config(max_steps=MAX_STEPS, stop_entropy=0.5, lock_threshold=0.9, seed=SEED + rank)
+    samp_topk = dg.sampler_config(max_steps=MAX_STEPS, stop_entropy=0.5, lock_threshold=0.9, seed=SEED + rank,
+                                  selfcond_topk=64)
     # single-layer full-width step
     w1 = WORKLOADS["layer1"]
     c1 = w1["cfg"]
@@ -346,6 +348,14 @@ def other_configs(dg, synth, model, wl, rank, peaks, stream, steps=5, warm=3):
                           "canvas_tok_per_s": B * CANVAS * 1000.0 / ms,
                           "distinct_experts_per_layer": sum(dist) / len(dist),
                           "roofline": line_roofline(c, B, C, dist, ms, peaks)})
+            if B == 16 and C == 1024 and c.get("self_cond"):
+                # the high-batch variant: expected embedding over each position's 64 largest logits
+                ms_k = time_steps(dg, mb, kvb, cvb, samp_topk, 0, steps, warm, stream)
+                res["selfcond_topk_variant"] = {
+                    "workload": "full-size model, 16 canvases, context 1024, self-conditioning input over the "
+                                "64 largest logits of each position",
+                    "k": 64, "ms_per_step": ms_k, "full_vocabulary_ms_per_step": ms,
+                    "canvas_tok_per_s": B * CANVAS * 1000.0 / ms_k}
         mb.close()
         del mb, kvb, cvb
         torch.cuda.empty_cache()
@@ -572,9 +582,11 @@ def main():
         barrier()
         g0.record(stream)
         passes = 0
+        block_stats = []
         for blk in range(n_blocks):
             st_, _ = model.decode_block(kv_l, cv_l, blk, samp, toks)
             passes += st_[0]
+            block_stats.append(model.last_block_stats)
         g1.record(stream)
         barrier()
         model.check_device()
@@ -582,6 +594,9 @@ def main():
         loop = {"blocks": n_blocks, "max_steps_per_block": MAX_STEPS, "output_tokens": n_blocks * CANVAS,
                 "denoise_passes": passes, "tokens_per_pass": n_blocks * CANVAS / passes, "ms": ms_l,
                 "output_tok_per_s": n_blocks * CANVAS / (ms_l / 1000.0),
+                "library_tokens_per_pass": [round(b["tokens_per_pass"], 3) for b in block_stats],
+                "distinct_experts_per_layer": [round(sum(b["distinct_experts"]) / len(b["distinct_experts"]), 2)
+                                               for b in block_stats],
                 "note": "random-init weights: predictions stay near uniform, so no position locks and the "
                         "entropy stop never fires; every block runs its full step budget"}
         del kv_l

@@ -18,6 +18,7 @@ DG_CANVAS = 256
 DG_OK, DG_ERR_INVALID_ARG, DG_ERR_CUDA, DG_ERR_WORKSPACE, DG_ERR_TIMEOUT, DG_ERR_UNSUPPORTED, \
     DG_ERR_BAD_TOKEN = range(7)
 DG_LOCK_PROB, DG_LOCK_ENTROPY_CUMSUM = 0, 1
+DG_DECODE_DEFER_APPEND = 1
 
 # size of the library's fixed split-KV scratch array (dg_attention_static_scratch)
 DG_ATTN_STATIC_SCRATCH_BYTES = 16 << 20
@@ -43,7 +44,7 @@ class dg_sampler_config(ctypes.Structure):
     _fields_ = [("lock_policy", ctypes.c_int32), ("lock_threshold", ctypes.c_float),
                 ("t_start", ctypes.c_float), ("t_end", ctypes.c_float), ("max_steps", ctypes.c_int32),
                 ("stop_entropy", ctypes.c_float), ("stop_require_stable_argmax", ctypes.c_int32),
-                ("seed", ctypes.c_uint64), ("persistent_lock", ctypes.c_int32)]
+                ("seed", ctypes.c_uint64), ("persistent_lock", ctypes.c_int32), ("selfcond_topk", ctypes.c_int32)]
 
 
 class dg_kv(ctypes.Structure):
@@ -77,7 +78,8 @@ class dg_profile(ctypes.Structure):
 
 
 class dg_block_stats(ctypes.Structure):
-    _fields_ = [("steps_taken", ctypes.POINTER(ctypes.c_int32)), ("rounds", ctypes.c_int32)]
+    _fields_ = [("steps_taken", ctypes.POINTER(ctypes.c_int32)), ("rounds", ctypes.c_int32),
+                ("tokens_per_pass", ctypes.c_float), ("distinct_experts", ctypes.POINTER(ctypes.c_float))]
 
 
 def _load():
@@ -107,6 +109,10 @@ def _load():
         "dg_decode_block": (I32, [P, ctypes.POINTER(dg_kv), ctypes.POINTER(dg_canvas),
                                   ctypes.POINTER(dg_step_args), P, ctypes.POINTER(dg_block_stats), P]),
         "dg_check_device_error": (I32, [P, P]),
+        "dg_denoise_step_append": (I32, [P, ctypes.POINTER(dg_kv), ctypes.POINTER(dg_canvas),
+                                         ctypes.POINTER(dg_step_args), P, ctypes.POINTER(dg_step_out), P]),
+        "dg_decode_block_ex": (I32, [P, ctypes.POINTER(dg_kv), ctypes.POINTER(dg_canvas),
+                                     ctypes.POINTER(dg_step_args), P, I32, P, ctypes.POINTER(dg_block_stats), P]),
         "dg_profile_start": (I32, [P]),
         "dg_profile_stop": (I32, [P, ctypes.POINTER(dg_profile)]),
         "dg_test_gemm": (I32, [P, I32, P, I32, I32, P, I32, P]),
@@ -117,6 +123,7 @@ def _load():
         "dg_test_attention": (I32, [P, P, P, P, I32, I32, I32, I32, I32, I32, I32, I32, I32, P, P, P]),
         "dg_test_workspace_buffer": (I32, [P, ctypes.c_char_p, ctypes.POINTER(P), ctypes.POINTER(S)]),
         "dg_test_wait_timeout": (I32, [P, ctypes.c_int64, P]),
+        "dg_test_struct_size": (S, [ctypes.c_char_p]),
         "dg_router_probe": (I32, [P, I32, P, I32, P, P]),
         "dg_ar_step": (I32, [P, ctypes.POINTER(dg_kv), P, F, U64, P, P, P, P]),
         "dg_attention_static_scratch": (I32, [P, P, P, P, I32, I32, I32, I32, I32, I32, I32, I32, I32, P]),

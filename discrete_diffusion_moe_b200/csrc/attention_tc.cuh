@@ -1,9 +1,11 @@
 // attention_tc.cuh - attention of one pass of queries over the keys of a
 // KV cache on the tcgen05 tensor cores (sm_100a).
 //
-//   canvas pass (causal = 0): every query sees keys [0, L0 + nq)   (no mask:
+//   canvas pass (causal_n = 0): every query sees keys [0, L0 + nq)   (no mask:
 //     bidirectional over the canvas, full view of the context)
-//   context encoding (causal = 1): query i sees keys [0, L0 + i]
+//   context encoding (causal_n = nq): query i sees keys [0, L0 + i]
+//   a finished block appended in the same pass as the next canvas round
+//     (causal_n = 256): the block's queries causal, the canvas's see all keys
 //
 // One CTA computes one 128-row tile of packed queries against a range of
 // 64-key tiles (a key split).  Grouped-query packing: the G = Hq / Hkv query
@@ -49,7 +51,9 @@ struct AttnTcParams {
   uint16_t* out;       // [B * nq, Hq * hd] bf16 (splits == 1, or merged in the cluster)
   float* part_o;       // [splits][B][Hq][nq][hd] unnormalised (splits > 1 without cluster)
   float* part_ml;      // [splits][B][Hq][nq][2] (max in log2 units, sum)
-  int B, nq, L0, c_max, Hq, Hkv, splits, causal;
+  int B, nq, L0, c_max, Hq, Hkv, splits;
+  int causal_n;        // queries of the first causal_n tokens of a canvas are causal
+                       // (token i sees keys [0, L0 + i]); the others see every key
   float scale_log2;    // log2(e) / sqrt(hd)
   int* err;
   int cluster;         // splits > 1: the splits of a tile are one cluster and merge
@@ -199,9 +203,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int n_kt = (kv_len + kAttnKeys - 1) / kAttnKeys;
   const int kt0 = (int)((long long)n_kt * split / p.splits);
   int kt1 = (int)((long long)n_kt * (split + 1) / p.splits);
-  if (p.causal) {
+  {
+    // the tile's last row sees the most keys (visibility grows with the token)
     const int r_last = min(r0 + kAttnRows - 1, rows_total - 1);
-    kt1 = min(kt1, (p.L0 + r_last / G) / kAttnKeys + 1);
+    if (r_last / G < p.causal_n) kt1 = min(kt1, (p.L0 + r_last / G) / kAttnKeys + 1);
   }
   const int n_tiles = max(0, kt1 - kt0);
   const int bg = b * p.Hkv + g;
@@ -230,6 +235,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     tmem_alloc(smem_u32(tmem_slot), S::TMEM_COLS);
     tmem_relinquish();
   }
+  grid_dep_wait();
+  grid_dep_launch();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -312,7 +319,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const int r = r0 + row;
     const int t_in = (r < rows_total ? r : rows_total - 1) / G;  // token within the pass
-    const int lim = p.causal ? min(kv_len - 1, p.L0 + t_in) : kv_len - 1;
+    const int lim = t_in < p.causal_n ? min(kv_len - 1, p.L0 + t_in) : kv_len - 1;
     const float scale = p.scale_log2;
     float m = -INFINITY, l = 0.f;  // reference max (scaled, log2 units) and this half's sum
     bool ok = true;
@@ -593,6 +600,8 @@ template <int MAXS>
 __global__ void attn_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml,
                                     uint16_t* __restrict__ out, int splits, int B, int Hq, int Hkv, int nq,
                                     int HD) {
+  grid_dep_wait();
+  grid_dep_launch();
   const long long rows = (long long)B * Hq * nq;
   const long long row = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;

@@ -22,6 +22,17 @@ __device__ __forceinline__ void set_error(int* err, int code) {
   if (err) atomicCAS(err, 0, code);
 }
 
+// ---- programmatic dependent launch --------------------------------------------
+// The round's kernels are launched so that a kernel's CTAs may start while
+// the previous kernel of the stream is still finishing.  Every kernel calls
+// grid_dep_wait() before it reads or writes memory that another kernel
+// writes or reads (before it, only its own shared / tensor memory set-up and
+// the tensor maps), and grid_dep_launch() right after, which lets the next
+// kernel's CTAs be scheduled once every CTA of this grid has got that far.
+// Outside such a launch both are no-ops.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---- bf16 ---------------------------------------------------------------------
 __device__ __forceinline__ float bf16_to_f32(uint16_t b) {
   return __uint_as_float(((uint32_t)b) << 16);

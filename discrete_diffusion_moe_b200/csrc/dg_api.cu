@@ -64,6 +64,56 @@ struct NvtxRange {
   NvtxRange& operator=(const NvtxRange&) = delete;
 };
 
+// One kernel launch.  With DG_PDL (programmatic dependent launch) its CTAs
+// may be scheduled while the stream's previous kernel finishes: every kernel
+// of the library waits (griddepcontrol.wait) before it touches memory that
+// another kernel writes, so only its launch latency and its own set-up
+// (barriers, tensor memory, tensor-map prefetch) overlap the predecessor's
+// tail.  Optional cluster shape and cluster scheduling policy.
+#ifndef DG_PDL
+#define DG_PDL 1
+#endif
+// token rows per grouped (expert) unit: 0 chooses 128 on CTA pairs, or 256 on
+// single CTAs when experts average more than 64 tokens; 256 takes 256-token
+// chunks on CTA pairs (one read of an expert's weight tile for up to 256 tokens)
+#ifndef DG_GROUPED_BN
+#define DG_GROUPED_BN 0
+#endif
+struct Launch {
+  cudaLaunchConfig_t lc = {};
+  cudaLaunchAttribute at[3];
+  Launch(dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl = DG_PDL) {
+    lc.gridDim = grid;
+    lc.blockDim = block;
+    lc.dynamicSmemBytes = smem;
+    lc.stream = st;
+    lc.attrs = at;
+    if (pdl) {
+      at[lc.numAttrs].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      at[lc.numAttrs].val.programmaticStreamSerializationAllowed = 1;
+      ++lc.numAttrs;
+    }
+  }
+  Launch& cluster(unsigned x, unsigned y, unsigned z) {
+    at[lc.numAttrs].id = cudaLaunchAttributeClusterDimension;
+    at[lc.numAttrs].val.clusterDim.x = x;
+    at[lc.numAttrs].val.clusterDim.y = y;
+    at[lc.numAttrs].val.clusterDim.z = z;
+    ++lc.numAttrs;
+    return *this;
+  }
+  Launch& policy(cudaClusterSchedulingPolicy pol) {
+    at[lc.numAttrs].id = cudaLaunchAttributeClusterSchedulingPolicyPreference;
+    at[lc.numAttrs].val.clusterSchedulingPolicyPreference = pol;
+    ++lc.numAttrs;
+    return *this;
+  }
+  template <typename... KArgs, typename... Args>
+  cudaError_t operator()(void (*k)(KArgs...), Args&&... args) {
+    return cudaLaunchKernelEx(&lc, k, std::forward<Args>(args)...);
+  }
+};
+
 // ============================================================================
 // configuration checks and layouts
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -132,9 +182,9 @@ WLayout weight_layout(const dg_model_config& c) {
 constexpr int kMaxAttnSplits = 8;
 
 struct WsLayout {
-  size_t err, flags, x, xn, qkv, opart, q, attn, rpart, tok, rbar, rfill, off, choff, perm, inv, wperm,
+  size_t err, flags, x, xn, qkv, opart, q, attn, rpart, tok, xnc, rbar, rfill, off, choff, perm, inv, wperm,
       xperm, hperm, yperm, logits, vp_m, vp_z, vp_s, vp_av, vp_ai, vp_gv, vp_gi, st_m, st_iz, st_h,
-      st_pmax, st_amax, st_samp, probs, epart, rope, stepdev, total;
+      st_pmax, st_amax, st_samp, probs, epart, rope, stepdev, dstat, total;
   int T_alloc, P_alloc, ks_r, n_vt;  // T_alloc: token rows of a layer pass (>= the canvas tokens)
   int T_canvas;                       // canvas tokens (batch * 256): rows of the vocabulary buffers
   long long epart_rows;
@@ -249,8 +299,10 @@ WsLayout ws_layout(const dg_model_config& c, int batch, int num_sms, int prefill
   L.st_m = take(Tc * 4); L.st_iz = take(Tc * 4); L.st_h = take(Tc * 4); L.st_pmax = take(Tc * 4);
   L.st_amax = take(Tc * 4); L.st_samp = take(Tc * 4);
   L.tok = take(T * 4);
+  L.xnc = take(Tc * d * 2);  // canvas rows of the normed stream after a fused append pass
   L.rope = take(T * (c.head_dim / 2) * 16);  // (cos, sin) of up to T positions of a pass
   L.stepdev = take(sizeof(StepDev));
+  L.dstat = take((size_t)c.n_layers * 4);  // distinct experts per layer, summed over passes
   L.probs = c.self_cond ? take(Tc * V * 2) : 0;
   L.epart = c.self_cond ? take((size_t)er * d * 4) : 0;
   L.total = off;
@@ -407,8 +459,8 @@ dg_status run_gemm(const CUtensorMap& ta, const BOperand& tb, GemmPlan p, const 
   if (p.cluster_k <= 1) {
     p.cluster_k = 0;
     const int grid = (int)std::min<long long>(units, (long long)ctas * num_sms);
-    gemm_tc_kernel<Epi><<<grid, gemm_threads<Epi>(), smem, st>>>(ta, tb.maps, p, epi, stages);
-    DG_CUDA(cudaGetLastError());
+    DG_CUDA(Launch(dim3(grid), dim3(gemm_threads<Epi>()), smem, st)(gemm_tc_kernel<Epi>, ta, tb.maps, p, epi,
+                                                                       stages));
   } else {
     // one unit per CTA; the k splits of a tile are consecutive units and one
     // cluster; their accumulators are staged in the stage ring ([128][bn + 4] fp32)
@@ -417,22 +469,11 @@ dg_status run_gemm(const CUtensorMap& ta, const BOperand& tb, GemmPlan p, const 
                   p.cluster_k);
     if ((size_t)stages * ((size_t)kATileBytes + (size_t)p.bn * 128) < (size_t)128 * (p.bn + 4) * 4)
       return fail(DG_ERR_INVALID_ARG, "gemm plan: the stage ring cannot hold a %d-column accumulator", p.bn);
-    cudaLaunchConfig_t lc = {};
-    cudaLaunchAttribute at[2];
-    at[0].id = cudaLaunchAttributeClusterDimension;
-    at[0].val.clusterDim.x = (unsigned)p.cluster_k;
-    at[0].val.clusterDim.y = 1;
-    at[0].val.clusterDim.z = 1;
-    at[1].id = cudaLaunchAttributeClusterSchedulingPolicyPreference;
-    at[1].val.clusterSchedulingPolicyPreference =
-        DG_CLUSTER_POLICY ? cudaClusterSchedulingPolicyLoadBalancing : cudaClusterSchedulingPolicySpread;
-    lc.gridDim = dim3((unsigned)units);
-    lc.blockDim = dim3(gemm_threads<Epi>());
-    lc.dynamicSmemBytes = smem;
-    lc.stream = st;
-    lc.attrs = at;
-    lc.numAttrs = 2;
-    DG_CUDA(cudaLaunchKernelEx(&lc, gemm_tc_kernel<Epi>, ta, tb.maps, p, epi, stages));
+    DG_CUDA(Launch(dim3((unsigned)units), dim3(gemm_threads<Epi>()), smem, st)
+                .cluster((unsigned)p.cluster_k, 1, 1)
+                .policy(DG_CLUSTER_POLICY ? cudaClusterSchedulingPolicyLoadBalancing
+                                          : cudaClusterSchedulingPolicySpread)(gemm_tc_kernel<Epi>, ta, tb.maps, p,
+                                                                               epi, stages));
   }
   if (launches) ++*launches;
   return DG_OK;
@@ -444,7 +485,7 @@ dg_status run_gemm_pair(const CUtensorMap& ta, const BOperand& tb, GemmPlan p, c
                         cudaStream_t st, long long* launches = nullptr) {
   if ((p.group_off && (p.n_groups < 1 || p.n_groups > kGemmMaxGroups)) || p.mt != 1 || p.k_splits != 1)
     return fail(DG_ERR_INVALID_ARG, "pair gemm: %d groups, %d A tiles, %d k splits", p.n_groups, p.mt, p.k_splits);
-  if (p.bn < 16 || p.bn > (p.group_off ? 128 : 256) || (p.bn & (p.bn - 1)) || p.K % 64 || p.K < 64)
+  if (p.bn < 16 || p.bn > 256 || (p.bn & (p.bn - 1)) || p.K % 64 || p.K < 64)
     return fail(DG_ERR_INVALID_ARG, "pair gemm plan: bn %d K %d", p.bn, p.K);
   for (int i = 0; i < 3; ++i) {
     if (tb.rows[i] < 1 || (i && tb.rows[i] < tb.rows[i - 1]) || tb.rows[i] > p.bn / 2)
@@ -454,19 +495,9 @@ dg_status run_gemm_pair(const CUtensorMap& ta, const BOperand& tb, GemmPlan p, c
   DG_TRY(set_smem_attr((const void*)gemm_pair_kernel<Epi>, (int)(227 * 1024 - kGemmStaticSmem), true));
   const int stages = gemm_pair_stages(p.bn);
   const size_t smem = gemm_pair_smem_bytes(p.bn, stages);
-  cudaLaunchConfig_t lc = {};
-  cudaLaunchAttribute at[1];
-  at[0].id = cudaLaunchAttributeClusterDimension;
-  at[0].val.clusterDim.x = 2;
-  at[0].val.clusterDim.y = 1;
-  at[0].val.clusterDim.z = 1;
-  lc.gridDim = dim3((unsigned)(2 * (num_sms / 2) * gemm_pair_ctas_per_sm(p.bn)));  // whole pairs
-  lc.blockDim = dim3(gemm_threads<Epi>());
-  lc.dynamicSmemBytes = smem;
-  lc.stream = st;
-  lc.attrs = at;
-  lc.numAttrs = 1;
-  DG_CUDA(cudaLaunchKernelEx(&lc, gemm_pair_kernel<Epi>, ta, tb.maps, p, epi, stages));
+  const unsigned grid = (unsigned)(2 * (num_sms / 2) * gemm_pair_ctas_per_sm(p.bn));  // whole pairs
+  DG_CUDA(Launch(dim3(grid), dim3(gemm_threads<Epi>()), smem, st).cluster(2, 1, 1)(gemm_pair_kernel<Epi>, ta,
+                                                                                    tb.maps, p, epi, stages));
   if (launches) ++*launches;
   return DG_OK;
 }
@@ -546,6 +577,7 @@ struct dg_ctx {
     dg_kv kv;
     dg_canvas cv;
     dg_step_out out;
+    int32_t topk;   // the a8 form the graph was captured with
   };
   bool g_valid = false;
   GraphKey g_key;
@@ -739,30 +771,15 @@ template <int HD>
 static dg_status launch_attn(dim3 grid, int splits, bool cluster, const CUtensorMap& tq, const CUtensorMap& tk,
                              const CUtensorMap& tv, const CUtensorMap& to, const AttnTcParams& ap, cudaStream_t st) {
   DG_TRY(set_smem_attr((const void*)attn_tc_kernel<HD>, (int)AttnTcShape<HD>::SMEM, false));
-  if (!cluster || splits <= 1) {
-    attn_tc_kernel<HD><<<grid, kAttnThreads, AttnTcShape<HD>::SMEM, st>>>(tq, tk, tv, to, ap);
-    DG_CUDA(cudaGetLastError());
-    return DG_OK;
-  }
-  cudaLaunchConfig_t lc = {};
-  cudaLaunchAttribute at[1];
-  at[0].id = cudaLaunchAttributeClusterDimension;
-  at[0].val.clusterDim.x = 1;
-  at[0].val.clusterDim.y = 1;
-  at[0].val.clusterDim.z = (unsigned)splits;
-  lc.gridDim = grid;
-  lc.blockDim = dim3(kAttnThreads);
-  lc.dynamicSmemBytes = AttnTcShape<HD>::SMEM;
-  lc.stream = st;
-  lc.attrs = at;
-  lc.numAttrs = 1;
-  DG_CUDA(cudaLaunchKernelEx(&lc, attn_tc_kernel<HD>, tq, tk, tv, to, ap));
+  Launch l(grid, dim3(kAttnThreads), AttnTcShape<HD>::SMEM, st);
+  if (cluster && splits > 1) l.cluster(1, 1, (unsigned)splits);
+  DG_CUDA(l(attn_tc_kernel<HD>, tq, tk, tv, to, ap));
   return DG_OK;
 }
 
 static dg_status run_attention(const uint16_t* q, const uint16_t* kc, const uint16_t* vc, uint16_t* out,
                                float* part_o, float* part_ml, int B, int nq, int L0, int c_max, int Hq, int Hkv,
-                               int hd, bool causal, int splits, bool cluster, int* err, cudaStream_t st,
+                               int hd, int causal_n, int splits, bool cluster, int* err, cudaStream_t st,
                                long long* launches) {
   if (c_max % 8) return fail(DG_ERR_INVALID_ARG, "c_max %d is not a multiple of 8", c_max);
   if (splits > kMaxAttnSplits) return fail(DG_ERR_INVALID_ARG, "%d key splits (at most %d)", splits, kMaxAttnSplits);
@@ -777,7 +794,7 @@ static dg_status run_attention(const uint16_t* q, const uint16_t* kc, const uint
   const bool merge_in_cluster = cluster && splits > 1;
   if (splits > 1 && !merge_in_cluster)
     DG_TRY(make_tmap_f32_store(&to, part_o, hd, (long long)G * nq, (long long)splits * B * Hkv));
-  AttnTcParams ap{out, part_o, part_ml, B, nq, L0, c_max, Hq, Hkv, splits, causal ? 1 : 0,
+  AttnTcParams ap{out, part_o, part_ml, B, nq, L0, c_max, Hq, Hkv, splits, causal_n,
                   (float)(1.4426950408889634 / sqrt((double)hd)), err, merge_in_cluster ? 1 : 0};
   dim3 grid((G * nq + kAttnRows - 1) / kAttnRows, Hkv, B * splits);
   switch (hd) {
@@ -792,9 +809,9 @@ static dg_status run_attention(const uint16_t* q, const uint16_t* kc, const uint
     const long long rows = (long long)B * Hq * nq;
     const unsigned cgrid = (unsigned)((rows * 32 + 255) / 256);
     if (splits <= 4)
-      attn_combine_kernel<4><<<cgrid, 256, 0, st>>>(part_o, part_ml, out, splits, B, Hq, Hkv, nq, hd);
+      DG_CUDA(Launch(dim3(cgrid), dim3(256), 0, st)(attn_combine_kernel<4>, part_o, part_ml, out, splits, B, Hq, Hkv, nq, hd));
     else
-      attn_combine_kernel<8><<<cgrid, 256, 0, st>>>(part_o, part_ml, out, splits, B, Hq, Hkv, nq, hd);
+      DG_CUDA(Launch(dim3(cgrid), dim3(256), 0, st)(attn_combine_kernel<8>, part_o, part_ml, out, splits, B, Hq, Hkv, nq, hd));
     DG_CUDA(cudaGetLastError());
     if (launches) ++*launches;
   }
@@ -815,7 +832,7 @@ static int attn_splits(int B, int nq, int L0, int Hq, int Hkv, int num_sms, int 
 // ============================================================================
 // one pass of the transformer layers over T = B * nq tokens at positions
 // L0 .. L0 + nq - 1 (x already holds the embedded inputs)
-static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L0, bool causal,
+static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L0, int causal_n,
                                 int32_t* dbg_idx, float* dbg_w, float* dbg_logits, float* dbg_hidden,
                                 float* dbg_hidden_attn, cudaStream_t st) {
   const dg_model_config& m = c->cfg;
@@ -829,7 +846,7 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
   // token rows per grouped unit: 128 (256 for large batches).  Routing can be
   // very uneven; one unit per 128 tokens of an expert keeps the number of times
   // a weight tile is read small while the units of one tile run side by side.
-  const int bnG = P / E > 64 ? 256 : 128;
+  const int bnG = DG_GROUPED_BN ? DG_GROUPED_BN : (P / E > 64 ? 256 : 128);
   const size_t kv_layer = (size_t)kv->batch * Hkv * kv->c_max * hd;
 
   BOperand t_xperm, t_hperm;
@@ -837,7 +854,7 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
   DG_TRY(make_bop(&t_hperm, c->at<uint16_t>(L.hperm), f, L.P_alloc, bnG));
   // grouped products of at most 128 tokens per chunk run on CTA pairs (two
   // pairs per SM pair); 256-token chunks keep one CTA per tile
-  const bool pair = bnG <= 128;
+  const bool pair = bnG <= 128 || DG_GROUPED_BN == 256;
   BOperand h_xperm{}, h_hperm{};
   if (pair) {
     DG_TRY(make_bop_half(&h_xperm, c->at<uint16_t>(L.xperm), d, L.P_alloc, bnG));
@@ -847,8 +864,8 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
   // cos/sin of this pass's positions, shared by all layers
   {
     const int n = nq * (hd / 2);
-    rope_table_kernel<<<(n + 255) / 256, 256, 0, st>>>(c->at<double2>(L.rope), nq, L0, hd / 2, hd,
-                                                       (double)m.rope_theta);
+    DG_CUDA(Launch(dim3((n + 255) / 256), dim3(256), 0, st)(rope_table_kernel, c->at<double2>(L.rope), nq, L0, hd / 2, hd,
+                                                       (double)m.rope_theta));
     CNT(c);
   }
 
@@ -868,7 +885,7 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
     // --- attention block (its RMSNorm ran at the end of the previous layer) ---
     NvtxRange nv_layer("dg.layer");  // the whole layer; its expert block nested
     if (l == 0) {
-      rmsnorm_kernel<256><<<T, 256, 0, st>>>(x, c->wp(W.g_attn), xn, d, m.rms_eps);
+      DG_CUDA(Launch(dim3(T), dim3(256), 0, st)(rmsnorm_kernel<256>, x, c->wp(W.g_attn), xn, d, m.rms_eps));
       CNT(c);
     }
     {
@@ -896,13 +913,13 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
       if (ks_qkv > kRopeMaxSplits) return fail(DG_ERR_UNSUPPORTED, "QKV split count %d", ks_qkv);
       const long long rot_threads = (long long)T * (Hq + Hkv) * (hd / 8);
       const int rot_blocks = (int)((rot_threads + 255) / 256);
-      rope_kv_kernel<<<rot_blocks + v_blocks, 256, 0, st>>>(rp);
+      DG_CUDA(Launch(dim3(rot_blocks + v_blocks), dim3(256), 0, st)(rope_kv_kernel, rp));
       CNT(c);
     }
     {
       ProfScope ps_(c, DG_PROF_ATTENTION, st);
       DG_TRY(run_attention(c->at<uint16_t>(L.q), kc, vc, c->at<uint16_t>(L.attn), nullptr, nullptr, B, nq, L0,
-                           kv->c_max, Hq, Hkv, hd, causal, splits, true, err, st, &c->n_launch));
+                           kv->c_max, Hq, Hkv, hd, causal_n, splits, true, err, st, &c->n_launch));
     }
     {
       ProfScope ps_(c, DG_PROF_DENSE, st);
@@ -927,9 +944,9 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
     NvtxRange nv_moe("dg.layer.moe_block");
     {
       const bool parts = !(DG_O_CLUSTER || ks_o == 1);
-      residual_norm_kernel<1><<<T, row_launch(d).threads, 0, st>>>(x, parts ? c->at<float>(L.opart) : nullptr,
+      DG_CUDA(Launch(dim3(T), dim3(row_launch(d).threads), 0, st)(residual_norm_kernel<1>, x, parts ? c->at<float>(L.opart) : nullptr,
                                                                    parts ? ks_o : 0, (long long)T * d, d,
-                                                                   c->wp(W.g_moe), xn, m.rms_eps);
+                                                                   c->wp(W.g_moe), xn, m.rms_eps));
     }
     CNT(c);
     if (dbg_hidden_attn)
@@ -967,9 +984,14 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
       rp.xperm = c->at<uint16_t>(L.xperm);
       rp.fill = c->at<int>(L.rfill);
       rp.bar = c->at<int>(L.rbar);
-      rp.dbg_idx = dbg_idx ? dbg_idx + (size_t)l * T * k : nullptr;
-      rp.dbg_w = dbg_w ? dbg_w + (size_t)l * T * k : nullptr;
-      rp.dbg_logits = dbg_logits ? dbg_logits + (size_t)l * T * E : nullptr;
+      // an appending pass records the routing of its canvas rows only
+      rp.dbg_nq = causal_n > 0 && causal_n < nq ? nq : 0;
+      rp.dbg_skip = rp.dbg_nq ? causal_n : 0;
+      const size_t T_dbg = rp.dbg_nq ? (size_t)B * (nq - causal_n) : (size_t)T;
+      rp.dbg_idx = dbg_idx ? dbg_idx + (size_t)l * T_dbg * k : nullptr;
+      rp.dbg_w = dbg_w ? dbg_w + (size_t)l * T_dbg * k : nullptr;
+      rp.dbg_logits = dbg_logits ? dbg_logits + (size_t)l * T_dbg * E : nullptr;
+      rp.distinct = c->at<int>(L.dstat) + l;
       rp.err = err;
       const int nb = (T + rp.tpc - 1) / rp.tpc;
       cudaLaunchConfig_t lc = {};
@@ -1017,8 +1039,8 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
       const uint16_t* g_next = l + 1 < m.n_layers ? c->wp(c->wl.layers[l + 1].g_attn) : c->wp(c->wl.g_final);
       // two float4s per thread: the eight expert rows per float4 keep the
       // register count high, and two CTAs per SM keep every token resident
-      moe_combine_norm_kernel<2><<<T, ((d / 4 + 1) / 2 + 31) / 32 * 32, 0, st>>>(x, c->at<float>(L.yperm), c->at<int>(L.inv), T, k, d, g_next,
-                                                 xn, m.rms_eps);
+      DG_CUDA(Launch(dim3(T), dim3(((d / 4 + 1) / 2 + 31) / 32 * 32), 0, st)(moe_combine_norm_kernel<2>, x, c->at<float>(L.yperm), c->at<int>(L.inv), T, k, d, g_next,
+                                                 xn, m.rms_eps));
       CNT(c);
     }
     DG_CUDA(cudaGetLastError());
@@ -1058,10 +1080,10 @@ extern "C" dg_status dg_encode_context(dg_ctx* c, dg_kv* kv, const int32_t* d_to
     // gather the chunk's tokens into a dense [B, nq] block
     DG_CUDA(cudaMemcpy2DAsync(tok_tmp, (size_t)nq * 4, d_tokens + s0, (size_t)n * 4, (size_t)nq * 4, B,
                               cudaMemcpyDeviceToDevice, st));
-    embed_kernel<<<T, 128, 0, st>>>(c->wp(c->wl.emb), tok_tmp, c->at<float>(c->L.x), T, d, c->cfg.vocab, c->err());
+    DG_CUDA(Launch(dim3(T), dim3(128), 0, st)(embed_kernel, c->wp(c->wl.emb), tok_tmp, c->at<float>(c->L.x), T, d, c->cfg.vocab, c->err()));
     CNT(c);
     DG_CUDA(cudaGetLastError());
-    DG_TRY(forward_layers(c, kv, B, nq, kv->length, true, nullptr, nullptr, nullptr, nullptr, nullptr, st));
+    DG_TRY(forward_layers(c, kv, B, nq, kv->length, nq, nullptr, nullptr, nullptr, nullptr, nullptr, st));
     kv->length += nq;
   }
   return DG_OK;
@@ -1118,13 +1140,21 @@ static dg_status check_round_args(dg_ctx* c, const dg_kv* kv, dg_canvas* cv, con
     return fail(DG_ERR_INVALID_ARG, "lock policy");
   if (!(s.t_start > 0.f) || !(s.t_end > 0.f)) return fail(DG_ERR_INVALID_ARG, "temperatures must be > 0");
   if (s.persistent_lock && !cv->locked) return fail(DG_ERR_INVALID_ARG, "persistent lock needs canvas.locked");
+  if (s.selfcond_topk < 0 || s.selfcond_topk > std::min(kTopkMax, c->cfg.vocab))
+    return fail(DG_ERR_INVALID_ARG, "selfcond_topk %d outside [0, %d]", s.selfcond_topk,
+                std::min(kTopkMax, c->cfg.vocab));
   return DG_OK;
 }
 
 // Enqueue one round.  The first launch writes the round parameters to the
-// device (its node is returned when the stream is being captured).
+// device (its node is returned when the stream is being captured).  With
+// `append` ([B, 256] tokens of a finished block), the block is appended to
+// the context in the same pass: each canvas's pass holds 512 tokens, the
+// block's (causal, positions L0 ..) then the canvas's (bidirectional,
+// positions L0 + 256 ..); the vocabulary phase runs on the canvas rows only.
 static dg_status enqueue_round(dg_ctx* c, const dg_kv* kv, dg_canvas* cv, const dg_step_args* a,
-                               const dg_step_out* o, cudaStream_t st, cudaGraphNode_t* param_node) {
+                               const dg_step_out* o, cudaStream_t st, cudaGraphNode_t* param_node,
+                               const int32_t* append = nullptr) {
   const dg_model_config& m = c->cfg;
   const WsLayout& L = c->L;
   const dg_sampler_config& s = a->sampler;
@@ -1148,6 +1178,18 @@ static dg_status enqueue_round(dg_ctx* c, const dg_kv* kv, dg_canvas* cv, const 
 
   // a1: canvas embedding (+ self-conditioning input)
   NvtxRange nv_round("dg.denoise_step");
+  const int nq = append ? 2 * DG_CANVAS : DG_CANVAS;   // tokens per canvas in the pass
+  if (append) {
+    // the pass's token ids, [B][block | canvas]; the embedding of all of them
+    int* tok = c->at<int>(L.tok);
+    DG_CUDA(cudaMemcpy2DAsync(tok, (size_t)nq * 4, append, (size_t)DG_CANVAS * 4, (size_t)DG_CANVAS * 4, B,
+                              cudaMemcpyDeviceToDevice, st));
+    DG_CUDA(cudaMemcpy2DAsync(tok + DG_CANVAS, (size_t)nq * 4, cv->tokens, (size_t)DG_CANVAS * 4,
+                              (size_t)DG_CANVAS * 4, B, cudaMemcpyDeviceToDevice, st));
+    DG_CUDA(Launch(dim3(B * nq), dim3(128), 0, st)(embed_kernel, c->wp(c->wl.emb), tok, c->at<float>(L.x), B * nq, d, V, err));
+    CNT(c);
+    DG_CUDA(cudaGetLastError());
+  }
   if (m.self_cond) {
     ProfScope ps_(c, DG_PROF_DENSE, st);
     CUtensorMap ta;
@@ -1158,9 +1200,14 @@ static dg_status enqueue_round(dg_ctx* c, const dg_kv* kv, dg_canvas* cv, const 
     GemmPlan p = dense_plan(d, d, T, bn, 1, err);
     p.a_hint = 1;
     EpiStoreT e{c->at<float>(L.x), d, 0, 2, c->wp(c->wl.emb), cv->tokens, V, err};
+    if (append) {  // canvas token t goes to pass row (t / 256) * 512 + 256 + t % 256
+      e.row_group = DG_CANVAS;
+      e.row_pitch = nq;
+      e.row_off = DG_CANVAS;
+    }
     DG_TRY(run_gemm(ta, tb, p, e, c->num_sms, st, &c->n_launch));
-  } else {
-    embed_kernel<<<T, 128, 0, st>>>(c->wp(c->wl.emb), cv->tokens, c->at<float>(L.x), T, d, V, err);
+  } else if (!append) {
+    DG_CUDA(Launch(dim3(T), dim3(128), 0, st)(embed_kernel, c->wp(c->wl.emb), cv->tokens, c->at<float>(L.x), T, d, V, err));
     CNT(c);
     DG_CUDA(cudaGetLastError());
   }
@@ -1168,15 +1215,23 @@ static dg_status enqueue_round(dg_ctx* c, const dg_kv* kv, dg_canvas* cv, const 
   if (o->hidden)
     DG_CUDA(cudaMemcpyAsync(o->hidden, c->at<float>(L.x), (size_t)T * d * 4, cudaMemcpyDeviceToDevice, st));
 
-  // a2-a6: transformer layers, bidirectional over the canvas
-  DG_TRY(forward_layers(c, kv, B, DG_CANVAS, kv->length, false, o->route_idx, o->route_w, o->route_logits,
-                        o->hidden, o->hidden_attn, st));
+  // a2-a6: transformer layers, bidirectional over the canvas (the appended
+  // block's tokens causal)
+  DG_TRY(forward_layers(c, kv, B, nq, kv->length, append ? DG_CANVAS : 0, o->route_idx, o->route_w,
+                        o->route_logits, o->hidden, o->hidden_attn, st));
+  if (append) {
+    // the canvas rows of the final normed stream, compacted for the LM head
+    const size_t row = (size_t)d * 2;
+    DG_CUDA(cudaMemcpy2DAsync(c->at<uint16_t>(L.xnc), (size_t)DG_CANVAS * row, c->at<uint16_t>(L.xn) +
+                              (size_t)DG_CANVAS * d, (size_t)nq * row, (size_t)DG_CANVAS * row, B,
+                              cudaMemcpyDeviceToDevice, st));
+  }
 
   // a7: final norm, LM head with online vocabulary statistics and sampling
   NvtxRange nv_lm("dg.vocabulary_phase");  // a7-a9: LM head, statistics, expected embedding, update
-  uint16_t* xn = c->at<uint16_t>(L.xn);  // final RMSNorm: fused into the last layer's combine
+  // final RMSNorm: fused into the last layer's combine
+  uint16_t* xn = append ? c->at<uint16_t>(L.xnc) : c->at<uint16_t>(L.xn);
   uint16_t* logits = c->at<uint16_t>(L.logits);  // bf16, the expected embedding's input
-  (void)s;
   VocabPartials vp{c->at<float>(L.vp_m), c->at<float>(L.vp_z), c->at<float>(L.vp_s), c->at<float>(L.vp_av),
                    c->at<int>(L.vp_ai), c->at<float>(L.vp_gv), c->at<int>(L.vp_gi)};
   {
@@ -1198,19 +1253,28 @@ static dg_status enqueue_round(dg_ctx* c, const dg_kv* kv, dg_canvas* cv, const 
   PosStats ps{c->at<float>(L.st_m), c->at<float>(L.st_iz), o->entropy ? o->entropy : c->at<float>(L.st_h),
               o->pmax ? o->pmax : c->at<float>(L.st_pmax), o->argmax ? o->argmax : c->at<int>(L.st_amax),
               o->sample ? o->sample : c->at<int>(L.st_samp)};
-  vocab_merge_kernel<<<T, kMergeThreads, 0, st>>>(vp.m, vp.z, vp.s, vp.amax_v, vp.amax_i, vp.gkey_v,
-                                                  vp.gkey_i, L.n_vt, T, log((double)V), ps);
+  DG_CUDA(Launch(dim3(T), dim3(kMergeThreads), 0, st)(vocab_merge_kernel, vp.m, vp.z, vp.s, vp.amax_v, vp.amax_i, vp.gkey_v,
+                                                  vp.gkey_i, L.n_vt, T, log((double)V), ps));
                                                            CNT(c);
   DG_CUDA(cudaGetLastError());
 
   // a8: expected embedding for the next round's self-conditioning input
-  if (m.self_cond) {
+  if (m.self_cond && s.selfcond_topk > 0) {
+    // high-batch variant: over each position's K largest logits only
+    NvtxRange nv_e("dg.expected_embedding");
+    ProfScope ps_(c, DG_PROF_EXPECTED_EMB, st);
+    DG_TRY(set_smem_attr((const void*)topk_esum_kernel, (int)sizeof(TopkSmem), false));
+    DG_CUDA(Launch(dim3(std::min(T, c->num_sms)), dim3(kTopkThreads), sizeof(TopkSmem), st)(
+        topk_esum_kernel, logits, (long long)V, s.selfcond_topk, c->wp(c->wl.emb), d, DG_CANVAS, T, cv->done,
+        cv->sc_state));
+    CNT(c);
+    DG_CUDA(cudaGetLastError());
+  } else if (m.self_cond) {
     NvtxRange nv_e("dg.expected_embedding");
     ProfScope ps_(c, DG_PROF_EXPECTED_EMB, st);
     uint16_t* probs = c->at<uint16_t>(L.probs);
     const long long n8 = (long long)T * V / 8;
-    probs_kernel<<<(unsigned)std::min<long long>((n8 + 255) / 256, 148 * 16), 256, 0, st>>>(
-        logits, ps.m, ps.inv_z, probs, T, V);
+    DG_CUDA(Launch(dim3((unsigned)std::min<long long>((n8 + 255) / 256, 148 * 16)), dim3(256), 0, st)(probs_kernel, logits, ps.m, ps.inv_z, probs, T, V));
         CNT(c);
     const int ks = esum_splits(m, T, c->num_sms);
     CUtensorMap ta;
@@ -1224,8 +1288,7 @@ static dg_status enqueue_round(dg_ctx* c, const dg_kv* kv, dg_canvas* cv, const 
     EpiStoreT e{c->at<float>(L.epart), d, (long long)T * d, 0, nullptr, nullptr, 0, err};
     DG_TRY(run_gemm(ta, tb, p, e, c->num_sms, st, &c->n_launch));
     const long long n = (long long)T * d;
-    esum_kernel<<<(unsigned)std::min<long long>((n + 255) / 256, 148 * 16), 256, 0, st>>>(
-        c->at<float>(L.epart), ks, T, d, DG_CANVAS, cv->done, cv->sc_state);
+    DG_CUDA(Launch(dim3((unsigned)std::min<long long>((n + 255) / 256, 148 * 16)), dim3(256), 0, st)(esum_kernel, c->at<float>(L.epart), ks, T, d, DG_CANVAS, cv->done, cv->sc_state));
         CNT(c);
     DG_CUDA(cudaGetLastError());
   }
@@ -1248,7 +1311,7 @@ static dg_status enqueue_round(dg_ctx* c, const dg_kv* kv, dg_canvas* cv, const 
   up.locked = cv->locked;
   up.sp = sp;
   up.vocab = V;
-  canvas_update_kernel<<<B, 256, 0, st>>>(up);
+  DG_CUDA(Launch(dim3(B), dim3(256), 0, st)(canvas_update_kernel, up));
   CNT(c);
   DG_CUDA(cudaGetLastError());
   return DG_OK;
@@ -1260,11 +1323,27 @@ extern "C" dg_status dg_denoise_step(dg_ctx* c, const dg_kv* kv, dg_canvas* cv, 
   return enqueue_round(c, kv, cv, a, o, (cudaStream_t)stream, nullptr);
 }
 
+extern "C" dg_status dg_denoise_step_append(dg_ctx* c, dg_kv* kv, dg_canvas* cv, const dg_step_args* a,
+                                            const int32_t* d_append, const dg_step_out* o, void* stream) {
+  DG_TRY(check_round_args(c, kv, cv, a));
+  if (!d_append) return fail(DG_ERR_INVALID_ARG, "append tokens are null");
+  DG_TRY(check_kv(c, kv, 2 * DG_CANVAS));
+  if (c->L.T_alloc < 2 * cv->batch * DG_CANVAS)
+    return fail(DG_ERR_WORKSPACE, "an appending round needs layer passes of %d tokens (dg_workspace_bytes_ex)",
+                2 * cv->batch * DG_CANVAS);
+  if (o && (o->hidden || o->hidden_attn))
+    return fail(DG_ERR_INVALID_ARG, "an appending round has no hidden-state outputs");
+  DG_TRY(enqueue_round(c, kv, cv, a, o, (cudaStream_t)stream, nullptr, d_append));
+  kv->length += DG_CANVAS;
+  return DG_OK;
+}
+
 static bool same_key(const dg_ctx::GraphKey& a, const dg_ctx::GraphKey& b) {
   const dg_kv &x = a.kv, &y = b.kv;
   const dg_canvas &p = a.cv, &q = b.cv;
   const dg_step_out &u = a.out, &w = b.out;
-  return x.k == y.k && x.v == y.v && x.batch == y.batch && x.c_max == y.c_max && x.length == y.length &&
+  return a.topk == b.topk && x.k == y.k && x.v == y.v && x.batch == y.batch && x.c_max == y.c_max &&
+         x.length == y.length &&
          p.tokens == q.tokens && p.sc_state == q.sc_state && p.prev_argmax == q.prev_argmax && p.done == q.done &&
          p.batch == q.batch && p.locked == q.locked && u.argmax == w.argmax && u.sample == w.sample && u.entropy == w.entropy &&
          u.pmax == w.pmax && u.lock == w.lock && u.mean_entropy == w.mean_entropy && u.stop == w.stop &&
@@ -1282,6 +1361,7 @@ extern "C" dg_status dg_denoise_step_graph(dg_ctx* c, const dg_kv* kv, dg_canvas
   key.kv = *kv;
   key.cv = *cv;
   if (o) key.out = *o;
+  key.topk = a->sampler.selfcond_topk;
   if (!c->g_valid || !same_key(key, c->g_key)) {
     c->drop_graph();
     if (!c->g_stream) DG_CUDA(cudaStreamCreateWithFlags(&c->g_stream, cudaStreamNonBlocking));
@@ -1355,10 +1435,10 @@ extern "C" dg_status dg_ar_step(dg_ctx* c, dg_kv* kv, const int32_t* d_tokens, f
   StepDev* sp = c->at<StepDev>(L.stepdev);
   step_params_kernel<<<1, 32, 0, st>>>(sp, v);
   CNT(c);
-  embed_kernel<<<B, 128, 0, st>>>(c->wp(c->wl.emb), d_tokens, c->at<float>(L.x), B, d, V, err);
+  DG_CUDA(Launch(dim3(B), dim3(128), 0, st)(embed_kernel, c->wp(c->wl.emb), d_tokens, c->at<float>(L.x), B, d, V, err));
   CNT(c);
   DG_CUDA(cudaGetLastError());
-  DG_TRY(forward_layers(c, kv, B, 1, pos, true, nullptr, nullptr, nullptr, nullptr, nullptr, st));
+  DG_TRY(forward_layers(c, kv, B, 1, pos, 1, nullptr, nullptr, nullptr, nullptr, nullptr, st));
   kv->length += 1;
   uint16_t* xn = c->at<uint16_t>(L.xn);  // the final RMSNorm ran with the last layer's combine
   VocabPartials vp{c->at<float>(L.vp_m), c->at<float>(L.vp_z), c->at<float>(L.vp_s), c->at<float>(L.vp_av),
@@ -1377,8 +1457,8 @@ extern "C" dg_status dg_ar_step(dg_ctx* c, dg_kv* kv, const int32_t* d_tokens, f
   }
   PosStats ps{c->at<float>(L.st_m), c->at<float>(L.st_iz), c->at<float>(L.st_h), c->at<float>(L.st_pmax), d_argmax,
               d_sample};
-  vocab_merge_kernel<<<B, kMergeThreads, 0, st>>>(vp.m, vp.z, vp.s, vp.amax_v, vp.amax_i, vp.gkey_v, vp.gkey_i,
-                                                  L.n_vt, B, log((double)V), ps);
+  DG_CUDA(Launch(dim3(B), dim3(kMergeThreads), 0, st)(vocab_merge_kernel, vp.m, vp.z, vp.s, vp.amax_v, vp.amax_i, vp.gkey_v, vp.gkey_i,
+                                                  L.n_vt, B, log((double)V), ps));
   CNT(c);
   DG_CUDA(cudaGetLastError());
   return DG_OK;
@@ -1403,33 +1483,59 @@ extern "C" dg_status dg_check_device_error(dg_ctx* c, void* stream) {
 
 extern "C" dg_status dg_decode_block(dg_ctx* c, dg_kv* kv, dg_canvas* cv, const dg_step_args* a, int32_t* d_out,
                                      dg_block_stats* h_stats, void* stream) {
+  return dg_decode_block_ex(c, kv, cv, a, nullptr, 0, d_out, h_stats, stream);
+}
+
+extern "C" dg_status dg_decode_block_ex(dg_ctx* c, dg_kv* kv, dg_canvas* cv, const dg_step_args* a,
+                                        const int32_t* d_pending, int32_t flags, int32_t* d_out,
+                                        dg_block_stats* h_stats, void* stream) {
   if (!c || !cv || !a || !d_out) return fail(DG_ERR_INVALID_ARG, "null argument");
-  DG_TRY(check_kv(c, kv, DG_CANVAS));
+  if (flags & ~DG_DECODE_DEFER_APPEND) return fail(DG_ERR_INVALID_ARG, "unknown decode flags %d", flags);
+  if (d_pending && d_pending == d_out) return fail(DG_ERR_INVALID_ARG, "the pending block and the output alias");
+  DG_TRY(check_kv(c, kv, d_pending ? 2 * DG_CANVAS : DG_CANVAS));
   cudaStream_t st = (cudaStream_t)stream;
   NvtxRange nv("dg.decode_block");
   const int B = cv->batch;
   DG_TRY(dg_canvas_init(c, cv, a->block, a->sampler.seed, stream));
-  std::vector<uint8_t> flags(B, 0);
+  std::vector<uint8_t> done_flags(B, 0);
   std::vector<int32_t> steps(B, 0);
-  int rounds = 0;
+  int rounds = 0, counted = 0;
+  int* dstat = c->at<int>(c->L.dstat);
+  const size_t dstat_bytes = (size_t)c->cfg.n_layers * 4;
+  DG_CUDA(cudaMemsetAsync(dstat, 0, dstat_bytes, st));
   for (int s = 0; s < a->sampler.max_steps; ++s) {
     dg_step_args sa = *a;
     sa.step = s;
-    DG_TRY(dg_denoise_step_graph(c, kv, cv, &sa, nullptr, stream));
+    if (s == 0 && d_pending) {
+      DG_TRY(dg_denoise_step_append(c, kv, cv, &sa, d_pending, nullptr, stream));
+      DG_CUDA(cudaMemsetAsync(dstat, 0, dstat_bytes, st));  // its pass routed the block's tokens too
+    } else {
+      DG_TRY(dg_denoise_step_graph(c, kv, cv, &sa, nullptr, stream));
+      ++counted;
+    }
     ++rounds;
     for (int b = 0; b < B; ++b)
-      if (!flags[b]) ++steps[b];
-    DG_CUDA(cudaMemcpyAsync(flags.data(), c->at<uint8_t>(c->L.flags), B, cudaMemcpyDeviceToHost, st));
+      if (!done_flags[b]) ++steps[b];
+    DG_CUDA(cudaMemcpyAsync(done_flags.data(), c->at<uint8_t>(c->L.flags), B, cudaMemcpyDeviceToHost, st));
     DG_TRY(dg_check_device_error(c, stream));  // synchronises the stream
     bool all = true;
-    for (int b = 0; b < B; ++b) all = all && flags[b];
+    for (int b = 0; b < B; ++b) all = all && done_flags[b];
     if (all) break;
   }
+  std::vector<int32_t> dsum(c->cfg.n_layers, 0);
+  if (h_stats && h_stats->distinct_experts) {
+    DG_CUDA(cudaMemcpyAsync(dsum.data(), dstat, dstat_bytes, cudaMemcpyDeviceToHost, st));
+    DG_CUDA(cudaStreamSynchronize(st));
+  }
   DG_CUDA(cudaMemcpyAsync(d_out, cv->tokens, (size_t)B * DG_CANVAS * 4, cudaMemcpyDeviceToDevice, st));
-  DG_TRY(dg_encode_context(c, kv, d_out, DG_CANVAS, stream));
+  if (!(flags & DG_DECODE_DEFER_APPEND)) DG_TRY(dg_encode_context(c, kv, d_out, DG_CANVAS, stream));
   if (h_stats) {
     h_stats->rounds = rounds;
+    h_stats->tokens_per_pass = rounds ? (float)(B * DG_CANVAS) / (float)rounds : 0.f;
     if (h_stats->steps_taken) memcpy(h_stats->steps_taken, steps.data(), B * sizeof(int32_t));
+    if (h_stats->distinct_experts)
+      for (int l = 0; l < c->cfg.n_layers; ++l)
+        h_stats->distinct_experts[l] = counted ? (float)dsum[l] / (float)counted : 0.f;
   }
   return DG_OK;
 }
@@ -1451,7 +1557,7 @@ extern "C" dg_status dg_router_probe(dg_ctx* c, int32_t layer, const float* d_x,
   float* x = c->at<float>(L.x);
   uint16_t* xn = c->at<uint16_t>(L.xn);
   DG_CUDA(cudaMemcpyAsync(x, d_x, (size_t)T * d * 4, cudaMemcpyDeviceToDevice, st));
-  residual_norm_kernel<1><<<T, row_launch(d).threads, 0, st>>>(x, nullptr, 0, 0, d, c->wp(W.g_moe), xn, m.rms_eps);
+  DG_CUDA(Launch(dim3(T), dim3(row_launch(d).threads), 0, st)(residual_norm_kernel<1>, x, nullptr, 0, 0, d, c->wp(W.g_moe), xn, m.rms_eps));
   DG_CUDA(cudaGetLastError());
   {
     CUtensorMap ta;
@@ -1480,6 +1586,8 @@ extern "C" dg_status dg_router_probe(dg_ctx* c, int32_t layer, const float* d_x,
   rp.dbg_idx = d_idx;
   rp.dbg_w = nullptr;
   rp.dbg_logits = nullptr;
+  rp.dbg_nq = rp.dbg_skip = 0;
+  rp.distinct = nullptr;
   rp.err = err;
   cudaLaunchConfig_t lc = {};
   cudaLaunchAttribute at[1];
@@ -1696,8 +1804,9 @@ extern "C" dg_status dg_test_attention(const uint16_t* q, const uint16_t* k, con
   if (splits == 0) splits = 1;
   // no partial buffers: the splits merge inside their cluster
   const bool cluster = part_o == nullptr && part_ml == nullptr;
-  DG_TRY(run_attention(q, k, v, out, part_o, part_ml, B, nq, L0, c_max, Hq, Hkv, hd, causal != 0, splits, cluster,
-                       nullptr, st, nullptr));
+  if (causal < 0 || causal > nq) return fail(DG_ERR_INVALID_ARG, "dg_test_attention: causal %d", causal);
+  DG_TRY(run_attention(q, k, v, out, part_o, part_ml, B, nq, L0, c_max, Hq, Hkv, hd, causal == 1 ? nq : causal,
+                       splits, cluster, nullptr, st, nullptr));
   DG_CUDA(cudaStreamSynchronize(st));
   return DG_OK;
 }
@@ -1718,6 +1827,18 @@ extern "C" dg_status dg_test_wait_timeout(dg_ctx* c, int64_t limit_ns, void* str
   wait_timeout_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(c->err(), (unsigned long long)limit_ns);
   DG_CUDA(cudaGetLastError());
   return DG_OK;
+}
+
+extern "C" size_t dg_test_struct_size(const char* name) {
+  if (!name) return 0;
+  const struct { const char* n; size_t s; } tab[] = {
+      {"dg_model_config", sizeof(dg_model_config)}, {"dg_sampler_config", sizeof(dg_sampler_config)},
+      {"dg_kv", sizeof(dg_kv)}, {"dg_canvas", sizeof(dg_canvas)}, {"dg_step_args", sizeof(dg_step_args)},
+      {"dg_step_out", sizeof(dg_step_out)}, {"dg_block_stats", sizeof(dg_block_stats)},
+      {"dg_profile", sizeof(dg_profile)}};
+  for (const auto& e : tab)
+    if (strcmp(e.n, name) == 0) return e.s;
+  return 0;
 }
 
 extern "C" dg_status dg_test_workspace_buffer(dg_ctx* c, const char* name, void** ptr, size_t* bytes) {

@@ -25,6 +25,9 @@ struct EpiStoreT {
   const int* tokens;     // mode 2: [T]
   int vocab;             // mode 2
   int* err;
+  // mode 2: token t goes to row (t / row_group) * row_pitch + row_off + t % row_group
+  // (row_group 0: row t)
+  int row_group = 0, row_pitch = 0, row_off = 0;
   struct State {};
   __device__ __forceinline__ void begin(const GemmJob&, int, State&) const {}
   __device__ __forceinline__ void end(const GemmJob&, int, State&) const {}
@@ -65,7 +68,11 @@ struct EpiStoreT {
       }
 #pragma unroll
       for (int i = 0; i < 16; ++i)
-        if (i < nv) base[(long long)(j.n0 + c0 + i) * ld] = e[i] + v[i];
+        if (i < nv) {
+          const int t = j.n0 + c0 + i;
+          const long long r = row_group ? (long long)(t / row_group) * row_pitch + row_off + t % row_group : t;
+          base[r * ld] = e[i] + v[i];
+        }
     }
   }
 };

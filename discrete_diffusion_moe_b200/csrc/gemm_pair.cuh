@@ -214,6 +214,8 @@ __global__ void __launch_bounds__(gemm_threads<Epi>(), 2)
     tma_prefetch_desc(&tmA);
     for (int i = 0; i < 3; ++i) tma_prefetch_desc(&tmB.m[i]);
   }
+  grid_dep_wait();
+  grid_dep_launch();
   if (warp >= 2 && p.group_off) {
     for (int g = threadIdx.x - 64; g <= p.n_groups; g += gemm_threads<Epi>() - 64) {
       tabs.chunk_off[g] = __ldg(p.chunk_off + g);

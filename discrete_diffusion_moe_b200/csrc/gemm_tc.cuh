@@ -208,6 +208,8 @@ __global__ void __launch_bounds__(gemm_threads<Epi>(), 2)
     tmem_alloc(smem_u32(tmem_slot), tmem_cols);
     tmem_relinquish();
   }
+  grid_dep_wait();
+  grid_dep_launch();
   if (p.group_off && warp >= 2) {
     for (int g = threadIdx.x - 64; g <= p.n_groups; g += gemm_threads<Epi>() - 64) {
       tabs.chunk_off[g] = __ldg(p.chunk_off + g);

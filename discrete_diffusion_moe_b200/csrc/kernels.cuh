@@ -14,6 +14,8 @@ namespace dg {
 // a1: x[t, :] = E_emb[tok[t], :]   (fp32 residual stream)
 __global__ void embed_kernel(const uint16_t* __restrict__ emb, const int* __restrict__ tokens,
                              float* __restrict__ x, int T, int d, int vocab, int* err) {
+  grid_dep_wait();
+  grid_dep_launch();
   const int t = blockIdx.x;
   if (t >= T) return;
   int tok = tokens[t];
@@ -42,6 +44,8 @@ template <int THREADS>
 __global__ void __launch_bounds__(THREADS) rmsnorm_kernel(const float* __restrict__ x,
                                                           const uint16_t* __restrict__ gain,
                                                           uint16_t* __restrict__ y, int d, float eps) {
+  grid_dep_wait();
+  grid_dep_launch();
   const int t = blockIdx.x;
   const float* xr = x + (long long)t * d;
   float ss = 0.f;
@@ -79,6 +83,8 @@ __global__ void __launch_bounds__(1024) residual_norm_kernel(float* __restrict__
                                                              int ks, long long split_stride, int d,
                                                              const uint16_t* __restrict__ gain,
                                                              uint16_t* __restrict__ xn, float eps) {
+  grid_dep_wait();
+  grid_dep_launch();
   const int t = blockIdx.x;
   const int nt = blockDim.x;
   float* xr = x + (long long)t * d;
@@ -145,6 +151,8 @@ inline RowLaunch row_launch(int d) {
 // (EpiQKV, when the projection's k splits add up in a cluster) or in
 // rope_kv_kernel from the projection's split-k partials.
 __global__ void rope_table_kernel(double2* __restrict__ tab, int nq, int L0, int half, int hd, double theta) {
+  grid_dep_wait();
+  grid_dep_launch();
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
   if (e >= nq * half) return;
   const int pos_in = e / half, i = e - pos_in * half;
@@ -179,6 +187,8 @@ constexpr int kRopeMaxSplits = 3; // split-k partials of the projection read by 
 // a warp take consecutive positions, so each of the 4 stores of a warp is one
 // contiguous run along the cache's position axis.
 __global__ void __launch_bounds__(256) rope_kv_kernel(const RopeParams p) {
+  grid_dep_wait();
+  grid_dep_launch();
   const int half = p.hd / 2;
   const int row_w = (p.Hq + 2 * p.Hkv) * p.hd;
   const int rot_blk = (int)blockIdx.x - p.v_blocks;
@@ -267,7 +277,7 @@ __global__ void __launch_bounds__(256) rope_kv_kernel(const RopeParams p) {
 // over the chosen k.  E <= 256, k <= 8.
 template <int KS>
 __device__ __forceinline__ void route_topk_token(const float* __restrict__ part, int T, int E, int k, int t,
-                                                 int lane, int* sel_out, float* w_out, int* dbg_idx,
+                                                 int lane, int* sel_out, float* w_out, int dbg_t, int* dbg_idx,
                                                  float* dbg_w, float* dbg_logits) {
   float l[8];
 #pragma unroll
@@ -288,7 +298,7 @@ __device__ __forceinline__ void route_topk_token(const float* __restrict__ part,
 #pragma unroll
   for (int q = 0; q < 8; ++q) {
     const bool ok = lane + 32 * q < E;
-    if (ok && dbg_logits) dbg_logits[(long long)t * E + lane + 32 * q] = l[q];
+    if (ok && dbg_logits) dbg_logits[(long long)dbg_t * E + lane + 32 * q] = l[q];
     const uint32_t u = __float_as_uint(l[q]);
     key[q] = ok ? ((u & 0x80000000u) ? ~u : (u | 0x80000000u)) : 0u;
     if (ok && key[q] == 0u) key[q] = 1u;  // -NaN patterns: keep them selectable
@@ -334,8 +344,8 @@ __device__ __forceinline__ void route_topk_token(const float* __restrict__ part,
     const float wv = ex / den;
     sel_out[lane] = er;
     w_out[lane] = wv;
-    if (dbg_idx) dbg_idx[t * k + lane] = er;
-    if (dbg_w) dbg_w[t * k + lane] = wv;
+    if (dbg_idx) dbg_idx[dbg_t * k + lane] = er;
+    if (dbg_w) dbg_w[dbg_t * k + lane] = wv;
   }
 }
 
@@ -387,6 +397,9 @@ struct RouteParams {
   int* dbg_idx;           // optional [T, k]
   float* dbg_w;           // optional [T, k]
   float* dbg_logits;      // optional [T, E]
+  int dbg_nq, dbg_skip;   // dbg_nq > 0: of each dbg_nq tokens the first dbg_skip are not recorded
+                          // (an appending pass: only the canvas rows, compacted)
+  int* distinct;          // optional: += number of experts given at least one token
   int* err;
 };
 
@@ -403,6 +416,8 @@ struct RouteParams {
 constexpr int kRouteThreads = 256;
 template <int KS>
 __global__ void __launch_bounds__(kRouteThreads) route_kernel(RouteParams p) {
+  grid_dep_wait();
+  grid_dep_launch();
   extern __shared__ int rsm[];
   const int E = p.E, k = p.k;
   const int np_max = p.tpc * k;
@@ -425,9 +440,18 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(RouteParams p) {
     for (int e = tid; e < E; e += kRouteThreads) p.fill[(ep ^ 1) * E + e] = 0;
 
   // ---- top-k of the CTA's tokens ----
-  for (int lt = warp; lt < nt; lt += nw)
-    route_topk_token<KS>(p.part, p.T, E, k, t0 + lt, lane, s_e + lt * k, s_w + lt * k, p.dbg_idx, p.dbg_w,
-                         p.dbg_logits);
+  for (int lt = warp; lt < nt; lt += nw) {
+    const int t = t0 + lt;
+    int r = t;
+    bool rec = true;
+    if (p.dbg_nq > 0) {
+      const int in = t % p.dbg_nq;
+      rec = in >= p.dbg_skip;
+      r = (t / p.dbg_nq) * (p.dbg_nq - p.dbg_skip) + in - p.dbg_skip;
+    }
+    route_topk_token<KS>(p.part, p.T, E, k, t, lane, s_e + lt * k, s_w + lt * k, r, rec ? p.dbg_idx : nullptr,
+                         rec ? p.dbg_w : nullptr, rec ? p.dbg_logits : nullptr);
+  }
   for (int e = tid; e < E; e += kRouteThreads) s_cnt[e] = 0;
   __syncthreads();
   // ---- stable ranks within the CTA: 32 pairs at a time in pair order ----
@@ -489,6 +513,13 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(RouteParams p) {
       s_off[E] = ic;
       if (b == 0) { p.off[E] = ic; p.chunk_off[E] = ik; }
     }
+    if (b == 0 && p.distinct) {
+      int nz = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) nz += c8[j] > 0;
+      nz = __reduce_add_sync(0xffffffffu, nz);
+      if (lane == 0) atomicAdd(p.distinct, nz);
+    }
   }
   __syncthreads();
   // ---- slots of the CTA's pairs ----
@@ -534,6 +565,8 @@ inline size_t route_smem_bytes(int tpc, int k, int E) {
 
 // chunk_off[g] = sum_{h < g} ceil((off[h+1] - off[h]) / bn)  (one thread)
 __global__ void chunk_offsets_kernel(const int* __restrict__ off, int G, int bn, int* __restrict__ chunk_off) {
+  grid_dep_wait();
+  grid_dep_launch();
   if (blockIdx.x != 0 || threadIdx.x != 0) return;
   int acc = 0;
   for (int g = 0; g < G; ++g) {
@@ -554,6 +587,8 @@ __global__ void __launch_bounds__(1024) moe_combine_norm_kernel(float* __restric
                                                                 const int* __restrict__ inv, int T, int k, int d,
                                                                 const uint16_t* __restrict__ gain,
                                                                 uint16_t* __restrict__ xn, float eps) {
+  grid_dep_wait();
+  grid_dep_launch();
   const int t = blockIdx.x;
   if (t >= T) return;
   const int nt = blockDim.x;
@@ -637,6 +672,8 @@ __global__ void __launch_bounds__(kMergeThreads) vocab_merge_kernel(
     const float* __restrict__ pm, const float* __restrict__ pz, const float* __restrict__ ps,
     const float* __restrict__ pav, const int* __restrict__ pai, const float* __restrict__ pgv,
     const int* __restrict__ pgi, int n_vt, int T, double log_v, PosStats out) {
+  grid_dep_wait();
+  grid_dep_launch();
   __shared__ double sm_m[kMergeThreads], sm_z[kMergeThreads], sm_s[kMergeThreads];
   __shared__ float sa_v[kMergeThreads], sg_v[kMergeThreads];
   __shared__ int sa_i[kMergeThreads], sg_i[kMergeThreads];
@@ -692,6 +729,8 @@ __global__ void __launch_bounds__(kMergeThreads) vocab_merge_kernel(
 __global__ void probs_kernel(const uint16_t* __restrict__ logits, const float* __restrict__ m,
                              const float* __restrict__ inv_z, uint16_t* __restrict__ p, int T,
                              long long V) {
+  grid_dep_wait();
+  grid_dep_launch();
   const long long n8 = (long long)T * V / 8;
   for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n8;
        e += (long long)gridDim.x * blockDim.x) {
@@ -710,6 +749,8 @@ __global__ void probs_kernel(const uint16_t* __restrict__ logits, const float* _
 // e[t, f] = bf16(sum_s part[s, t, f]) for canvases that are still running.
 __global__ void esum_kernel(const float* __restrict__ part, int ks, int T, int d, int canvas,
                             const uint8_t* __restrict__ done, uint16_t* __restrict__ sc_state) {
+  grid_dep_wait();
+  grid_dep_launch();
   const long long n = (long long)T * d;
   for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n;
        e += (long long)gridDim.x * blockDim.x) {
@@ -733,6 +774,8 @@ struct StepDev {
 };
 
 __global__ void step_params_kernel(StepDev* dst, const StepDev v) {
+  grid_dep_wait();
+  grid_dep_launch();
   if (threadIdx.x == 0 && blockIdx.x == 0) *dst = v;
 }
 
@@ -756,6 +799,8 @@ struct UpdateParams {
 };
 
 __global__ void __launch_bounds__(256) canvas_update_kernel(const UpdateParams p) {
+  grid_dep_wait();
+  grid_dep_launch();
   const int b = blockIdx.x, i = threadIdx.x;
   const int t = b * 256 + i;
   __shared__ float red[8];
@@ -852,6 +897,8 @@ __global__ void __launch_bounds__(256) canvas_update_kernel(const UpdateParams p
 // locked = 0 (when given).
 __global__ void canvas_init_kernel(int* tokens, int* prev_argmax, uint8_t* done, uint8_t* locked, int B, int block,
                                    uint32_t k0, uint32_t k1, int vocab) {
+  grid_dep_wait();
+  grid_dep_launch();
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
   if (t >= B * 256) return;
   const int b = t / 256, i = t % 256;
@@ -867,6 +914,381 @@ __global__ void fill_u16_kernel(uint16_t* p, long long n, uint16_t v) {
   for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n;
        e += (long long)gridDim.x * blockDim.x)
     p[e] = v;
+}
+
+}  // namespace dg
+
+namespace dg {
+
+// ---------------------------------------------------------------------------
+// a8, high-batch variant (top-k vocabulary truncation): per position, the K
+// ids with the largest bf16-stored logits (ties to the lower id), weights
+// p = bf16(exp(l - M) / sum_sel exp(l - M)) over those K (M their largest),
+// e = bf16(sum_j p_j E_emb[id_j]) in ascending id order.  One CTA per
+// position: a two-pass radix select on order-preserving 16-bit keys of the
+// bf16 logits (per-warp histograms of the high, then the low byte), an
+// index-ordered collect (each thread owns a contiguous id range; block scans
+// give every thread its output slots), then the K-row gather-sum (fixed
+// order).  Positions of canvases that are done keep their state.
+constexpr int kTopkThreads = 1024;
+constexpr int kTopkMax = 1024;     // largest K
+constexpr int kTopkBins = 512;     // first level: the key's top 9 bits (sign and exponent: one octave)
+constexpr int kTopkBins2 = 128;    // second level: the 7 mantissa bits
+constexpr int kTopkStash = 8192;   // candidates held in shared memory after the second pass
+
+__device__ __forceinline__ uint32_t bf16_order_key(uint16_t b) {
+  return (b & 0x8000u) ? (~(uint32_t)b & 0xFFFFu) : ((uint32_t)b | 0x8000u);
+}
+
+// exclusive block scan of one int per thread (kTopkThreads threads); the
+// total goes to *total.  Uses `ws` [kTopkThreads / 32 + 1] ints of shared memory.
+__device__ __forceinline__ int block_excl_scan(int v, int* ws, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  if (lane == 31) ws[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int t = lane < kTopkThreads / 32 ? ws[lane] : 0;
+    int c = t;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, c, o);
+      if (lane >= o) c += n;
+    }
+    if (lane < kTopkThreads / 32) ws[lane] = c - t;
+    if (lane == 31) ws[kTopkThreads / 32] = c;
+  }
+  __syncthreads();
+  const int r = ws[warp] + incl - v;
+  *total = ws[kTopkThreads / 32];
+  __syncthreads();
+  return r;
+}
+
+// order keys of the two bf16 values packed in w (low half: the lower id)
+__device__ __forceinline__ uint32_t bf16x2_order_keys(uint32_t w) {
+  const uint32_t sgn = (w >> 15) & 0x00010001u;      // the halves' sign bits
+  return w ^ ((sgn * 0x7FFFu) | 0x80008000u);        // negative: ~b, positive: b | 0x8000
+}
+
+// dynamic shared memory of topk_esum_kernel
+struct TopkSmem {
+  int lh[kTopkBins * 32];  // lane-private histogram [bin][lane]: a warp's 32 adds never share an address
+  int hist[kTopkBins];     // first level, summed over lanes
+  int hist2[kTopkBins2];   // second level
+  int sel_idx[kTopkMax];
+  float sel_w[kTopkMax];
+  int scan_ws[kTopkThreads / 32 + 1];
+  float red[kTopkThreads / 32];
+  int s_b1, s_above1, s_thr, s_above, s_ns, s_nsel, s_maxkey, s_stash_ok;
+  union {
+    struct {
+      int id[kTopkStash];
+      uint16_t key[kTopkStash];
+    } stash;
+    float part[8192];  // the gather's per-group partial sums [groups][d]
+  } u;
+};
+
+// warp-aggregated append: the lanes with `take` get consecutive slots of
+// `counter` (one atomic per warp); returns this lane's slot (or -1)
+__device__ __forceinline__ int warp_append(bool take, int* counter) {
+  const unsigned mask = __ballot_sync(0xffffffffu, take);
+  if (!mask) return -1;
+  const int lane = threadIdx.x & 31, leader = __ffs(mask) - 1;
+  int base = 0;
+  if (lane == leader) base = atomicAdd(counter, __popc(mask));
+  base = __shfl_sync(0xffffffffu, base, leader);
+  return take ? base + __popc(mask & ((1u << lane) - 1u)) : -1;
+}
+
+// The high-batch variant of the self-conditioning input: per position t, the
+// K largest bf16 logits (ties to the lower id), p_v = bf16(exp(l_v - M) /
+// sum over the K of exp(l_u - M)) with M the row's largest, and
+// e_t = bf16(sum_v p_v E_emb[v]) over those K rows only.  A persistent grid
+// of one 1024-thread CTA per SM walks the positions, so the rows in flight
+// (one 512 KB row of a 262144-id vocabulary per SM) stay in L2 between the
+// passes.  Keys are the logits' bf16 bits mapped to an unsigned order; the
+// histograms are lane-private ([bin][lane]) so that the many keys that share
+// a bin never serialise a warp's shared-memory adds.
+//   pass 1 (from DRAM): histogram of the key's top 9 bits (one octave per
+//     bin) and the row's largest key; the bin b1 holding the K-th largest;
+//   pass 2 (from L2): histogram of the 7 low bits inside b1 (exact keys), and
+//     every key in bins >= b1 appended (id, key) to a shared stash when they
+//     fit; the K-th largest key thr follows, with the keys equal to it to take;
+//   selection: from the stash when it holds every candidate and every key
+//     equal to thr is taken, else a third pass over the row in id order; the
+//     K ids sorted ascending (bitonic) so that the sums below run in id order;
+//   gather: 8 columns per thread, the K rows split over thread groups, the
+//     groups' partial sums added in group order (deterministic).
+// V is a multiple of 256, so the uint4 units of a warp are all in range or
+// all out of it (the warp-collective steps below never diverge).
+__global__ void __launch_bounds__(kTopkThreads, 1) topk_esum_kernel(const uint16_t* __restrict__ logits, long long V,
+                                                                     int K, const uint16_t* __restrict__ emb, int d,
+                                                                     int canvas, int T, const uint8_t* __restrict__ done,
+                                                                     uint16_t* __restrict__ sc_state) {
+  grid_dep_wait();
+  grid_dep_launch();
+  extern __shared__ __align__(16) uint8_t topk_smem_raw[];
+  TopkSmem& sm = *reinterpret_cast<TopkSmem*>(topk_smem_raw);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const long long nv8 = V / 8;
+  for (int t = blockIdx.x; t < T; t += gridDim.x) {
+    if (done[t / canvas]) continue;  // block-uniform
+    const uint4* lr = reinterpret_cast<const uint4*>(logits + (long long)t * V);
+    // ---- pass 1: octave histogram and the largest key ----
+    for (int e = tid; e < kTopkBins * 32 / 4; e += kTopkThreads) reinterpret_cast<int4*>(sm.lh)[e] = make_int4(0, 0, 0, 0);
+    __syncthreads();
+    uint32_t kmax2 = 0;
+    for (long long u0 = tid; u0 < nv8; u0 += 4 * kTopkThreads) {
+      uint4 w[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const long long u = u0 + (long long)r * kTopkThreads;
+        w[r] = u < nv8 ? __ldcg(lr + u) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        if (u0 + (long long)r * kTopkThreads >= nv8) break;
+        const uint32_t w4[4] = {w[r].x, w[r].y, w[r].z, w[r].w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t k2 = bf16x2_order_keys(w4[q]);
+          kmax2 = __vmaxu2(kmax2, k2);
+          atomicAdd(&sm.lh[(((k2 >> 7) & 0x1FFu) << 5) | lane], 1);
+          atomicAdd(&sm.lh[((k2 >> 23) << 5) | lane], 1);
+        }
+      }
+    }
+    uint32_t kmax = max(kmax2 & 0xFFFFu, kmax2 >> 16);
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    if (lane == 0) sm.red[warp] = __int_as_float((int)kmax);
+    __syncthreads();
+    for (int b = warp; b < kTopkBins; b += kTopkThreads / 32) {
+      const int v = __reduce_add_sync(0xffffffffu, sm.lh[b * 32 + lane]);
+      if (lane == 0) sm.hist[b] = v;
+    }
+    __syncthreads();
+    {
+      // bins from the top: thread i < 512 owns bin 511 - i
+      const int c = tid < kTopkBins ? sm.hist[kTopkBins - 1 - tid] : 0;
+      int total;
+      const int before = block_excl_scan(c, sm.scan_ws, &total);
+      if (tid < kTopkBins && before < K && before + c >= K) {
+        sm.s_b1 = kTopkBins - 1 - tid;
+        sm.s_above1 = before;
+      }
+      if (tid == 0) {
+        uint32_t km = 0;
+        for (int w_ = 0; w_ < kTopkThreads / 32; ++w_) km = max(km, (uint32_t)__float_as_int(sm.red[w_]));
+        sm.s_maxkey = (int)km;
+        sm.s_ns = 0;
+        sm.s_nsel = 0;
+      }
+      for (int e = tid; e < kTopkBins2 * 32 / 4; e += kTopkThreads) reinterpret_cast<int4*>(sm.lh)[e] = make_int4(0, 0, 0, 0);
+    }
+    __syncthreads();
+    const uint32_t b1 = (uint32_t)sm.s_b1;
+    const bool stash_ok = sm.s_above1 + sm.hist[b1] <= kTopkStash;
+    // ---- pass 2: mantissa histogram inside b1; stash the candidates ----
+    for (long long u0 = tid; u0 < nv8; u0 += 4 * kTopkThreads) {
+      uint4 w[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const long long u = u0 + (long long)r * kTopkThreads;
+        w[r] = u < nv8 ? __ldcg(lr + u) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const long long u = u0 + (long long)r * kTopkThreads;
+        if (u >= nv8) break;  // warp-uniform
+        const uint32_t w4[4] = {w[r].x, w[r].y, w[r].z, w[r].w};
+        uint32_t k2[4], mx2 = 0;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          k2[q] = bf16x2_order_keys(w4[q]);
+          mx2 = __vmaxu2(mx2, k2[q]);
+        }
+        // most 8-key groups hold no key in bins >= b1: one vote for the warp
+        const bool cand = max(mx2 & 0xFFFFu, mx2 >> 16) >= (b1 << 7);
+        if (__any_sync(0xffffffffu, cand)) {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const uint32_t key = (k2[q >> 1] >> (16 * (q & 1))) & 0xFFFFu;
+            const uint32_t bin = key >> 7;
+            if (bin == b1) atomicAdd(&sm.lh[(key & 127u) * 32 + lane], 1);
+            const int pos = warp_append(stash_ok && bin >= b1, &sm.s_ns);
+            if (pos >= 0) {
+              sm.u.stash.id[pos] = (int)(u * 8 + q);
+              sm.u.stash.key[pos] = (uint16_t)key;
+            }
+          }
+        }
+      }
+    }
+    __syncthreads();
+    for (int b = warp; b < kTopkBins2; b += kTopkThreads / 32) {
+      const int v = __reduce_add_sync(0xffffffffu, sm.lh[b * 32 + lane]);
+      if (lane == 0) sm.hist2[b] = v;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      // the K-th largest key: lane l owns the low-bit bins 127 - 4l .. 124 - 4l
+      const int hi = kTopkBins2 - 1 - 4 * lane;
+      int c4[4], loc = 0;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) { c4[q] = sm.hist2[hi - q]; loc += c4[q]; }
+      int incl = loc;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += n;
+      }
+      int cum = sm.s_above1 + incl - loc;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (cum < K && cum + c4[q] >= K) {
+          sm.s_thr = (int)((b1 << 7) | (uint32_t)(hi - q));
+          sm.s_above = cum;                                // keys larger than thr
+          sm.s_stash_ok = stash_ok && cum + c4[q] == K;    // every key equal to thr is taken
+        }
+        cum += c4[q];
+      }
+    }
+    __syncthreads();
+    const uint32_t thr = (uint32_t)sm.s_thr;
+    if (sm.s_stash_ok) {
+      // ---- selection from the stash (exactly K keys >= thr), then ids ascending ----
+      const int ns = sm.s_ns;
+      for (int e0 = 0; e0 < ns; e0 += kTopkThreads) {
+        const int e = e0 + tid;
+        const bool take = e < ns && (uint32_t)sm.u.stash.key[e] >= thr;
+        const int pos = warp_append(take, &sm.s_nsel);
+        if (pos >= 0) sm.sel_idx[pos] = sm.u.stash.id[e];
+      }
+      __syncthreads();
+      int n2 = 1;
+      while (n2 < K) n2 <<= 1;
+      for (int e = K + tid; e < n2; e += kTopkThreads) sm.sel_idx[e] = 0x7FFFFFFF;
+      __syncthreads();
+      for (int k2 = 2; k2 <= n2; k2 <<= 1)
+        for (int j2 = k2 >> 1; j2 > 0; j2 >>= 1) {
+          const int e = tid, f = e ^ j2;
+          if (e < n2 && f > e) {
+            const int a = sm.sel_idx[e], b = sm.sel_idx[f];
+            if (((e & k2) == 0) == (a > b)) { sm.sel_idx[e] = b; sm.sel_idx[f] = a; }
+          }
+          __syncthreads();
+        }
+    } else {
+      // ---- pass 3: collect in id order (each thread a contiguous id range) ----
+      const int ties_needed = K - sm.s_above;
+      const long long per = (nv8 + kTopkThreads - 1) / kTopkThreads;  // uint4 units per thread
+      const long long v0 = min(nv8, (long long)tid * per), v1 = min(nv8, v0 + per);
+      int n_gt = 0, n_eq = 0;
+      for (long long u = v0; u < v1; ++u) {
+        const uint4 w = __ldcg(lr + u);
+        const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const uint32_t key = bf16_order_key((uint16_t)(w4[q >> 1] >> (16 * (q & 1))));
+          n_gt += key > thr;
+          n_eq += key == thr;
+        }
+      }
+      int total;
+      const int eq_before = block_excl_scan(n_eq, sm.scan_ws, &total);
+      const int take_eq = max(0, min(n_eq, ties_needed - eq_before));
+      int slot = block_excl_scan(n_gt + take_eq, sm.scan_ws, &total);
+      int eq_taken = 0;
+      const uint16_t* lr16 = logits + (long long)t * V;
+      for (long long i = v0 * 8; i < v1 * 8 && slot < K; ++i) {
+        const uint32_t key = bf16_order_key(lr16[i]);
+        if (key > thr || (key == thr && eq_taken < take_eq)) {
+          if (key == thr) ++eq_taken;
+          sm.sel_idx[slot++] = (int)i;
+        }
+      }
+      __syncthreads();
+    }
+    // ---- weights: softmax over the selected bf16 logits (fixed-order sum) ----
+    const uint16_t* lr16 = logits + (long long)t * V;
+    const uint32_t mk = (uint32_t)sm.s_maxkey;
+    const uint16_t mbits = (uint16_t)((mk & 0x8000u) ? (mk & 0x7FFFu) : (~mk & 0xFFFFu));
+    const float M = bf16_to_f32(mbits);
+    float part = 0.f;
+    for (int j = tid; j < K; j += kTopkThreads) {
+      const float w = expf(bf16_to_f32(lr16[sm.sel_idx[j]]) - M);
+      sm.sel_w[j] = w;
+      part += w;
+    }
+    part = warp_sum(part);
+    if (lane == 0) sm.red[warp] = part;
+    __syncthreads();
+    float den = 0.f;
+#pragma unroll
+    for (int w_ = 0; w_ < kTopkThreads / 32; ++w_) den += sm.red[w_];
+    for (int j = tid; j < K; j += kTopkThreads) sm.sel_w[j] = bf16_to_f32(f32_to_bf16(sm.sel_w[j] / den));
+    __syncthreads();
+    // ---- e = sum_j p_j E_emb[id_j]: groups of d/8 threads, group g takes j = g, g + G, ... ----
+    const int cpt = d / 8, G = min(kTopkThreads / cpt, (int)(8192 / d));
+    const int g = tid / cpt, c8 = tid - g * cpt;
+    if (g < G) {
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      int j = g;
+      for (; j + 3 * G < K; j += 4 * G) {
+        uint4 w[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+          w[r] = __ldg(reinterpret_cast<const uint4*>(emb + (long long)sm.sel_idx[j + r * G] * d) + c8);
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const float p = sm.sel_w[j + r * G];
+          const uint32_t w4[4] = {w[r].x, w[r].y, w[r].z, w[r].w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            acc[2 * q] = fmaf(p, bf16_to_f32(w4[q] & 0xFFFF), acc[2 * q]);
+            acc[2 * q + 1] = fmaf(p, bf16_to_f32(w4[q] >> 16), acc[2 * q + 1]);
+          }
+        }
+      }
+      for (; j < K; j += G) {
+        const uint4 w = __ldg(reinterpret_cast<const uint4*>(emb + (long long)sm.sel_idx[j] * d) + c8);
+        const float p = sm.sel_w[j];
+        const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          acc[2 * q] = fmaf(p, bf16_to_f32(w4[q] & 0xFFFF), acc[2 * q]);
+          acc[2 * q + 1] = fmaf(p, bf16_to_f32(w4[q] >> 16), acc[2 * q + 1]);
+        }
+      }
+      float* dst = sm.u.part + (long long)g * d + c8 * 8;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) dst[q] = acc[q];
+    }
+    __syncthreads();
+    if (tid < cpt) {
+      float acc[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) acc[q] = sm.u.part[tid * 8 + q];
+      for (int g2 = 1; g2 < G; ++g2) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[q] += sm.u.part[(long long)g2 * d + tid * 8 + q];
+      }
+      uint4 o;
+      o.x = pack_bf16x2(acc[0], acc[1]);
+      o.y = pack_bf16x2(acc[2], acc[3]);
+      o.z = pack_bf16x2(acc[4], acc[5]);
+      o.w = pack_bf16x2(acc[6], acc[7]);
+      reinterpret_cast<uint4*>(sc_state + (long long)t * d)[tid] = o;
+    }
+    __syncthreads();  // the shared buffers are reused by the next position
+  }
 }
 
 }  // namespace dg

@@ -18,9 +18,10 @@ def model_config(n_layers, d_model, n_q_heads, n_kv_heads, head_dim, n_experts, 
 
 def sampler_config(lock_policy=DG_LOCK_PROB, lock_threshold=0.9, t_start=0.8, t_end=0.4, max_steps=48,
                    stop_entropy=0.5, stop_require_stable_argmax=False, seed=0,
-                   persistent_lock=False) -> dg_sampler_config:
+                   persistent_lock=False, selfcond_topk=0) -> dg_sampler_config:
     return dg_sampler_config(lock_policy, lock_threshold, t_start, t_end, max_steps, stop_entropy,
-                             int(bool(stop_require_stable_argmax)), seed, int(bool(persistent_lock)))
+                             int(bool(stop_require_stable_argmax)), seed, int(bool(persistent_lock)),
+                             int(selfcond_topk))
 
 
 def _stream(stream=None):
@@ -179,13 +180,30 @@ class Model:
                  ctypes.byref(out.s) if out is not None else None, _stream(stream)))
 
     def decode_block(self, kv: KVCache, cv: Canvas, block: int, sampler: dg_sampler_config, out_tokens,
-                     stream=None):
+                     stream=None, pending=None, defer_append=False):
+        """One block (dg_decode_block_ex): `pending` is a finished block not
+        yet in the context, appended in this block's first round;
+        `defer_append` leaves this block out of the context (the next call's
+        pending)."""
         steps = (ctypes.c_int32 * cv.s.batch)()
-        stats = dg_block_stats(steps, 0)
+        distinct = (ctypes.c_float * self.cfg.n_layers)()
+        stats = dg_block_stats(steps, 0, 0.0, distinct)
         args = dg_step_args(block, 0, sampler)
-        check(lib.dg_decode_block(self.ctx, ctypes.byref(kv.s), ctypes.byref(cv.s), ctypes.byref(args),
-                                  _ptr(out_tokens), ctypes.byref(stats), _stream(stream)))
+        check(lib.dg_decode_block_ex(self.ctx, ctypes.byref(kv.s), ctypes.byref(cv.s), ctypes.byref(args),
+                                     _ptr(pending), 1 if defer_append else 0, _ptr(out_tokens), ctypes.byref(stats),
+                                     _stream(stream)))
+        self.last_block_stats = dict(tokens_per_pass=stats.tokens_per_pass, distinct_experts=list(distinct))
         return list(steps), stats.rounds
+
+    def step_append(self, kv: KVCache, cv: Canvas, block: int, step: int, sampler: dg_sampler_config,
+                    append: torch.Tensor, out: StepOutputs = None, stream=None):
+        """dg_denoise_step_append: append `append` [B, 256] to the context in
+        the same pass as this round."""
+        assert append.dtype == torch.int32 and append.is_contiguous()
+        args = dg_step_args(block, step, sampler)
+        check(lib.dg_denoise_step_append(self.ctx, ctypes.byref(kv.s), ctypes.byref(cv.s), ctypes.byref(args),
+                                         _ptr(append), ctypes.byref(out.s) if out is not None else None,
+                                         _stream(stream)))
 
     def check_device(self, stream=None):
         check(lib.dg_check_device_error(self.ctx, _stream(stream)))

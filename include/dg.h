@@ -98,6 +98,11 @@ typedef struct dg_sampler_config {
                                           article §一); 1: the masked-style variant, a position once
                                           locked keeps its token for the rest of the block (needs
                                           dg_canvas.locked) */
+  int32_t selfcond_topk;               /* 0: the expected embedding over the whole vocabulary (the
+                                          method); K in [1, min(1024, vocab)]: the high-batch variant
+                                          (laozijiushiniubi.cn article §九, top-k vocabulary
+                                          truncation): over each position's K largest bf16 logits
+                                          (ties to the lower id), renormalised over them */
 } dg_sampler_config;
 
 /* Causally encoded context, one K and one V buffer of dg_kv_bytes() each:
@@ -157,8 +162,15 @@ typedef struct dg_step_out {
 
 /* Host-side statistics of one dg_decode_block call. */
 typedef struct dg_block_stats {
-  int32_t* steps_taken;   /* host [B]: rounds run for each canvas (may be NULL) */
-  int32_t rounds;         /* rounds launched for the batch */
+  int32_t* steps_taken;      /* host [B]: rounds run for each canvas (may be NULL) */
+  int32_t rounds;            /* rounds launched for the batch */
+  float tokens_per_pass;     /* tokens finished per round launched: B * 256 / rounds (the pages'
+                                tokens per forward pass, laozijiushiniubi.cn article §四, §五) */
+  float* distinct_experts;   /* host [n_layers] (may be NULL): per layer, the number of distinct
+                                experts the router gave at least one of the batch's canvas tokens,
+                                averaged over the block's canvas rounds (a round that also
+                                appends a pending block is not counted); the article's "about 84
+                                of 128 experts per 256 tokens" (§五) */
 } dg_block_stats;
 
 typedef struct dg_ctx dg_ctx;
@@ -229,6 +241,21 @@ dg_status dg_canvas_init(dg_ctx* ctx, dg_canvas* cv, int32_t block, uint64_t see
 dg_status dg_denoise_step(dg_ctx* ctx, const dg_kv* kv, dg_canvas* cv, const dg_step_args* args,
                           const dg_step_out* out, void* stream);
 
+/* A round that first appends a finished block to the context, in the same
+   pass (one read of every layer's weights for both): d_append [kv->batch,
+   256] (device int32) are appended causally at positions kv->length ..
+   kv->length + 255 of each canvas's context, exactly as dg_encode_context
+   would (laozijiushiniubi.cn article §二, §四: a finished block becomes
+   context), while the canvas round of dg_denoise_step runs on the positions
+   after them, seeing the appended block; then kv->length += 256.  Needs
+   c_max >= length + 512 and a workspace for layer passes of 512 tokens per
+   canvas (dg_workspace_bytes_ex, prefill_tokens >= batch * 512, else
+   DG_ERR_WORKSPACE).  The routing outputs hold the canvas rows' routing
+   ([n_layers, B*256, ...], as in dg_denoise_step); the hidden-state outputs
+   are not available (must be NULL, else DG_ERR_INVALID_ARG).  Asynchronous. */
+dg_status dg_denoise_step_append(dg_ctx* ctx, dg_kv* kv, dg_canvas* cv, const dg_step_args* args,
+                                 const int32_t* d_append, const dg_step_out* out, void* stream);
+
 /* The same round as dg_denoise_step, replayed from a CUDA graph that the
    context captures on first use and keeps while the KV cache (pointers and
    length), canvas and output pointers stay the same (a change re-captures
@@ -244,6 +271,19 @@ dg_status dg_denoise_step_graph(dg_ctx* ctx, const dg_kv* kv, dg_canvas* cv, con
    dg_encode_context.  `args->step` is ignored.  h_stats may be NULL. */
 dg_status dg_decode_block(dg_ctx* ctx, dg_kv* kv, dg_canvas* cv, const dg_step_args* args,
                           int32_t* d_out, dg_block_stats* h_stats, void* stream);
+
+/* dg_decode_block with the block append fused into the next block's first
+   round: d_pending (device [batch, 256], may be NULL) is a finished block
+   not yet in the context; this block's round 0 appends it
+   (dg_denoise_step_append).  With DG_DECODE_DEFER_APPEND in `flags` the
+   block decoded here is not appended at the end (the caller passes d_out as
+   the next call's d_pending, a different buffer from that call's d_out).
+   Needs a context created with dg_context_create_ex(prefill_tokens >=
+   batch * 512) when d_pending is given. */
+#define DG_DECODE_DEFER_APPEND 1
+dg_status dg_decode_block_ex(dg_ctx* ctx, dg_kv* kv, dg_canvas* cv, const dg_step_args* args,
+                             const int32_t* d_pending, int32_t flags, int32_t* d_out,
+                             dg_block_stats* h_stats, void* stream);
 
 /* Retained autoregressive mode (laozijiushiniubi.cn article §七: the same
    weights still generate one token at a time), the comparison workload of

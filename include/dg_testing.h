@@ -73,7 +73,9 @@ dg_status dg_test_dense_schedule(int32_t M, int32_t N, int32_t K, int32_t bn, in
    V cache transposed, fp16 [B][Hkv][hd][c_max], both holding keys
    [0, L0 + nq); c_max a multiple of 8; out bf16 [B * nq, Hq * hd]
    (token-major).  causal = 0: every query sees all L0 + nq keys; causal = 1:
-   query i sees keys [0, L0 + i].  splits (1..8; 0 means 1) key splits.  For
+   query i sees keys [0, L0 + i]; 1 < causal <= nq: queries i < causal are
+   causal and the rest see all keys (a pass that appends a finished block
+   ahead of a canvas, causal = 256).  splits (1..8; 0 means 1) key splits.  For
    splits > 1 with part_o and part_ml both NULL, the splits of each tile run
    as one thread-block cluster and merge through distributed shared memory
    (the form the layers use); otherwise the partial buffers come from the
@@ -92,6 +94,12 @@ dg_status dg_test_attention(const uint16_t* d_q, const uint16_t* d_k, const uint
    device error word and returns, so the next dg_check_device_error reports
    (and clears) it and the context stays usable.  Asynchronous on `stream`. */
 dg_status dg_test_wait_timeout(dg_ctx* ctx, int64_t limit_ns, void* stream);
+
+/* sizeof of one of the ABI's structs by its name ("dg_model_config",
+   "dg_sampler_config", "dg_kv", "dg_canvas", "dg_step_args", "dg_step_out",
+   "dg_block_stats", "dg_profile"), 0 for another name.  Host only: lets a
+   binding check its mirrors of the structs against this build. */
+size_t dg_test_struct_size(const char* name);
 
 /* Device address and size of one named scratch buffer of a context's
    workspace (for inspecting the last layer's intermediates after a call):

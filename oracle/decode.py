@@ -167,7 +167,8 @@ def denoise_step(cfg: ModelConfig, W: Weights, kv: KVCache, state: CanvasState,
     samp = np.empty((B, N), np.int64)
     s_gap = np.empty((B, N))
     a_gap = np.empty((B, N))
-    probs = np.empty((B, N, V)) if cfg.self_cond else None
+    topk = int(getattr(sc, "selfcond_topk", 0))
+    probs = np.empty((B, N, V)) if cfg.self_cond and topk == 0 else None
     for b in range(B):
         for i in range(N):
             H[b, i], pmax[b, i], amax[b, i], p = smp.position_stats(logits[b, i])
@@ -179,7 +180,9 @@ def denoise_step(cfg: ModelConfig, W: Weights, kv: KVCache, state: CanvasState,
 
     # a8: expected embedding for the next round's self-conditioning input
     e_new = None
-    if cfg.self_cond:
+    if cfg.self_cond and topk > 0:
+        e_new = smp.expected_embedding_topk(logits.reshape(B * N, V), W, topk)[0].reshape(B, N, d)
+    elif cfg.self_cond:
         e_new = smp.expected_embedding(probs.reshape(B * N, V), W).reshape(B, N, d)
 
     # a9: stop, lock and the next canvas
@@ -241,3 +244,14 @@ def ar_step(cfg: ModelConfig, W: Weights, kv: KVCache, tokens, temperature: floa
         s_gap[b] = _top2_gap(keys)
         a_gap[b] = _top2_gap(logits[b])
     return logits, amax, samp, s_gap, a_gap
+
+
+def denoise_step_append(cfg: ModelConfig, W: Weights, kv: KVCache, state: CanvasState,
+                        sc: smp.SamplerConfig, block: int, step: int, append_tokens, **kw) -> StepOutput:
+    """A round that first appends a finished block to the context (the
+    laozijiushiniubi.cn article, sections 二 and 四: a finished block becomes
+    context, encoded causally): the causal encode of append_tokens [B, N],
+    then the canvas round over the grown context.  The GPU runs both in one
+    pass; this is its definition."""
+    encode_context(cfg, W, kv, append_tokens)
+    return denoise_step(cfg, W, kv, state, sc, block, step, **kw)

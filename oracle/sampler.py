@@ -52,6 +52,7 @@ class SamplerConfig:
     stop_require_stable_argmax: bool = False
     seed: int = 0
     persistent_lock: bool = False   # masked-style variant: a locked position keeps its token
+    selfcond_topk: int = 0          # 0: full-vocabulary expected embedding; K: top-K variant
 
 
 def temperature(step: int, max_steps: int, t_start: float = 0.8, t_end: float = 0.4) -> float:
@@ -158,3 +159,28 @@ def expected_embedding(probs, W, chunk: int = 16384):
         n = min(chunk, V - v0)
         acc += pb[:, v0:v0 + n] @ W.emb_chunk(v0, n)
     return bf16_round(acc)
+
+
+def expected_embedding_topk(logits_f32, W, k: int):
+    """The high-batch variant of the self-conditioning input (top-k
+    vocabulary truncation, the laozijiushiniubi.cn article, section 九): per
+    position, the k ids with the largest bf16-stored logits (ties to the lower
+    id), p_v = exp(bf16(l_v) - M) / sum over those k of exp(bf16(l_u) - M) with
+    M the largest of them, rounded to bf16, and e = bf16(sum_v p_v E_emb[v])
+    over those k rows only.  logits_f32 [T, V]; returns (e [T, d] float64
+    bf16 values, ids [T, k] in ascending id order)."""
+    lb = bf16_round(np.asarray(logits_f32, dtype=np.float64))
+    T, V = lb.shape
+    k = int(min(k, V))
+    e = np.zeros((T, W.cfg.d_model))
+    ids = np.empty((T, k), np.int64)
+    for t in range(T):
+        order = np.lexsort((np.arange(V), -lb[t]))[:k]   # by value descending, then id ascending
+        sel = np.sort(order)
+        ids[t] = sel
+        M = lb[t, sel].max()
+        w = np.exp(lb[t, sel] - M)
+        p = bf16_round(w / w.sum())
+        rows = np.stack([W.emb_rows([int(v)])[0] for v in sel])
+        e[t] = p @ rows
+    return bf16_round(e), ids

@@ -301,6 +301,16 @@ def tf_expected_embedding(rep, W, gl, ge, rows):
     assert not bad.any(), f"expected embedding differs at {int(bad.sum())} elements"
 
 
+def tf_expected_embedding_topk(rep, W, gl, ge, k):
+    """a8's top-k variant on the GPU's logits: the K ids are chosen on the
+    bf16 logits both sides store (ties to the lower id), so the set is exact;
+    e within one bf16 ulp plus the rounding of each bf16 p_v (2^-8 of max |e|)."""
+    e, _ = OS.expected_embedding_topk(gl, W, k)
+    tol = 2.0 ** -7 * np.abs(e) + 2.0 ** -8 * np.abs(e).max()
+    bad = np.abs(ge - e) > tol
+    assert not bad.any(), f"top-{k} expected embedding differs at {int(bad.sum())} elements"
+
+
 # ---------------------------------------------------------------------------
 # one case: context encoding, canvas initialisation, then steps
 
@@ -316,6 +326,8 @@ class Case:
     lm_std: float = None
     ctx_seed: int = 1234
     block: int = 0
+    ctx_split: int = 0      # > 0: the GPU encodes the context in two calls, split there
+    prefill: int = 0        # the GPU context's prefill_tokens (encode passes of that many tokens)
 
 
 def _sampler(case: Case):
@@ -330,7 +342,7 @@ def gpu_sampler(dg, sc):
                              lock_threshold=sc.lock_threshold, t_start=sc.t_start, t_end=sc.t_end,
                              max_steps=sc.max_steps, stop_entropy=sc.stop_entropy,
                              stop_require_stable_argmax=sc.stop_require_stable_argmax, seed=sc.seed,
-                             persistent_lock=sc.persistent_lock)
+                             persistent_lock=sc.persistent_lock, selfcond_topk=sc.selfcond_topk)
 
 
 def check_context_kv(rep, ocfg, gkv, okv, enc_rec, B, C):
@@ -375,9 +387,13 @@ def run_case(case: Case, check_kv=True, verbose=True):
     sc = _sampler(case)
 
     gcfg = dg.model_config(**c, self_cond=case.self_cond)
-    model = dg.Model(gcfg, case.batch, seed=0, kind_std=std)
+    model = dg.Model(gcfg, case.batch, seed=0, kind_std=std, prefill_tokens=case.prefill)
     gkv = dg.KVCache(gcfg, case.batch, c_max)
-    model.encode(gkv, torch.from_numpy(ctx.astype(np.int32)).cuda())
+    if case.ctx_split:
+        model.encode(gkv, torch.from_numpy(np.ascontiguousarray(ctx[:, :case.ctx_split]).astype(np.int32)).cuda())
+        model.encode(gkv, torch.from_numpy(np.ascontiguousarray(ctx[:, case.ctx_split:]).astype(np.int32)).cuda())
+    else:
+        model.encode(gkv, torch.from_numpy(ctx.astype(np.int32)).cuda())
     model.check_device()
     assert gkv.length == okv.length == case.ctx_len
     if check_kv and case.ctx_len > 0:
@@ -429,7 +445,10 @@ def run_case(case: Case, check_kv=True, verbose=True):
             live_rows = np.nonzero(np.repeat(~done_in, 256))[0]
             if live_rows.size:
                 ge = gcv.sc_state.float().cpu().numpy().astype(np.float64).reshape(T, d)
-                tf_expected_embedding(rep, W, gl[live_rows], ge[live_rows], live_rows)
+                if sc.selfcond_topk > 0:
+                    tf_expected_embedding_topk(rep, W, gl[live_rows], ge[live_rows], sc.selfcond_topk)
+                else:
+                    tf_expected_embedding(rep, W, gl[live_rows], ge[live_rows], live_rows)
 
         # ---- 2. the oracle's own chain from the step's inputs ---------------------------
         state = OD.CanvasState(tokens=tokens_in.astype(np.int64).copy(), sc=sc_in.copy(),

@@ -92,3 +92,16 @@ def test_workspace_too_small_is_refused_before_any_device_work(lib):
     with pytest.raises(dg.DgError) as e:
         dg.dg_context_create(cfg, 1 << 20, 2 << 20, need, 65)
     assert e.value.status == dg.DG_ERR_INVALID_ARG
+
+
+def test_binding_structs_match_the_header():
+    """The Python binding's ctypes mirrors of the ABI structs have the sizes
+    the C build gives them (a field added on one side only shifts every later
+    one)."""
+    import discrete_diffusion_moe_b200 as dg
+    for name in ("dg_model_config", "dg_sampler_config", "dg_kv", "dg_canvas", "dg_step_args",
+                 "dg_step_out", "dg_block_stats", "dg_profile"):
+        c_size = dg.lib.dg_test_struct_size(name.encode())
+        assert c_size > 0, name
+        assert ctypes.sizeof(getattr(dg, name)) == c_size, (name, ctypes.sizeof(getattr(dg, name)), c_size)
+    assert dg.lib.dg_test_struct_size(b"no_such_struct") == 0

@@ -19,7 +19,12 @@ pytestmark = pytest.mark.gpu
     (1, 256, 256, 16, 8, 176, 1, 4), (1, 200, 0, 16, 8, 176, 1, 1),
     (1, 256, 300, 8, 8, 32, 0, 8), (1, 256, 2048, 16, 8, 176, 0, 5), (2, 256, 77, 8, 8, 32, 0, 4),
     (1, 256, 1024, 8, 4, 64, 0, 4), (1, 130, 70, 8, 2, 128, 1, 2), (3, 256, 1024, 16, 8, 176, 0, 1),
-    (1, 1, 0, 16, 8, 176, 0, 1), (1, 256, 8000, 16, 8, 176, 0, 8)])
+    (1, 1, 0, 16, 8, 176, 0, 1), (1, 256, 8000, 16, 8, 176, 0, 8),
+    # passes after a context appended at a ragged offset, and appending passes
+    # (the first 256 queries causal, the canvas's 256 bidirectional)
+    (1, 256, 296, 8, 8, 32, 0, 8), (2, 256, 333, 8, 8, 32, 0, 4), (1, 256, 40, 8, 8, 32, 1, 5),
+    (2, 256, 77, 8, 8, 32, 1, 4), (1, 512, 40, 8, 8, 32, 256, 4), (2, 512, 77, 8, 8, 32, 256, 2),
+    (2, 512, 40, 8, 8, 32, 256, 2), (1, 512, 77, 16, 8, 176, 256, 4)])
 @pytest.mark.parametrize("merge", ["cluster", "scratch"])
 def test_attention_matches_oracle(B, nq, L0, Hq, Hkv, hd, causal, splits, merge):
     """merge: the key splits of a tile merge inside their thread-block cluster
@@ -38,8 +43,15 @@ def test_attention_matches_oracle(B, nq, L0, Hq, Hkv, hd, causal, splits, merge)
     got = out.float().cpu().numpy().reshape(B, nq, Hq, hd)
     for b in range(B):
         pos, kpos = np.arange(L0, L0 + nq), np.arange(L0 + nq)
-        want = oracle_attention(ref["q"][b], ref["k"][b], ref["v"][b], pos, kpos, bool(causal))
-        want_abs = oracle_attention(ref["q"][b], ref["k"][b], np.abs(ref["v"][b]), pos, kpos, bool(causal))
+        n_c = nq if causal == 1 else causal   # queries [0, n_c) causal, the rest bidirectional
+        want, want_abs = [], []
+        for rows, cz in ((slice(0, n_c), True), (slice(n_c, nq), False)):
+            if rows.start == rows.stop:
+                continue
+            want.append(oracle_attention(ref["q"][b][rows], ref["k"][b], ref["v"][b], pos[rows], kpos, cz))
+            want_abs.append(oracle_attention(ref["q"][b][rows], ref["k"][b], np.abs(ref["v"][b]), pos[rows],
+                                             kpos, cz))
+        want, want_abs = np.concatenate(want), np.concatenate(want_abs)
         # bf16 rounding of the output, fp16 probabilities in the P V product and
         # fp32 accumulation noise (see attn_inputs.bound)
         err = np.abs(got[b] - want)

@@ -51,6 +51,25 @@ def test_tiny_persistent_lock_variant():
     _compared(rep, 4)
 
 
+@pytest.mark.parametrize("k", [1, 64, 1024])
+def test_tiny_self_cond_topk_variant(k):
+    """The high-batch variant of the self-conditioning input: the expected
+    embedding over each position's K largest logits only (K = 1: the argmax
+    embedding; K = 1024: the largest K the kernel takes), three rounds."""
+    rep = run_case(Case(cfg=TINY, self_cond=True, ctx_len=40, steps=3, lm_std=1.5,
+                        sampler=dict(selfcond_topk=k)))
+    _compared(rep, 3)
+
+
+@pytest.mark.parametrize("split,ctx_len,batch,prefill", [(40, 296, 1, 512), (77, 333, 2, 1024), (40, 296, 2, 0),
+                                                        (64, 320, 1, 512), (100, 612, 1, 0)])
+def test_tiny_context_encoded_in_two_calls(split, ctx_len, batch, prefill):
+    """The context appended in two encode calls, the second starting at a
+    ragged position (passes of 256 or of `prefill` tokens), then two rounds."""
+    rep = run_case(Case(cfg=TINY, ctx_len=ctx_len, batch=batch, steps=2, ctx_split=split, prefill=prefill))
+    _compared(rep, 2, batch=batch)
+
+
 def test_single_layer_full_width_step():
     """1 layer, d 2816, 16 q / 8 kv heads x 176, 128 experts top-8, ffn 704,
     vocab 262144, 2048 context tokens, one canvas, one round."""

@@ -177,3 +177,50 @@ def test_selfcond_probs_round_only_the_stored_logits():
     assert p[0] == np.exp(1.0 - float(a)) / Z
     assert p[1] == p[2] == np.exp(-float(a)) / Z
     assert abs(p.sum() - 1.0) > 1e-6   # no longer a distribution: the rounding is visible
+
+
+class _EmbRows:
+    """Stands in for the weights: embedding rows of a given matrix."""
+
+    def __init__(self, rows):
+        self.rows = rows
+
+        class _C:
+            d_model = rows.shape[1]
+        self.cfg = _C()
+
+    def emb_rows(self, toks):
+        return self.rows[np.asarray(toks)]
+
+
+def test_expected_embedding_topk_selection_and_weights():
+    from oracle.numerics import bf16_round
+    rng = np.random.default_rng(11)
+    V, d = 40, 8
+    E = bf16_round(rng.standard_normal((V, d)))
+    W = _EmbRows(E)
+    # k = 1: the embedding row of the largest bf16 logit
+    l = rng.standard_normal((3, V)).astype(np.float32)
+    e, ids = S.expected_embedding_topk(l, W, 1)
+    for t in range(3):
+        am = int(np.argmax(bf16_round(l[t].astype(np.float64))))
+        assert ids[t, 0] == am and np.array_equal(e[t], bf16_round(E[am]))
+    # ties go to the lower ids: equal logits select ids 0..k-1 with equal weights
+    l = np.zeros((1, V), np.float32)
+    e, ids = S.expected_embedding_topk(l, W, 4)
+    assert list(ids[0]) == [0, 1, 2, 3]
+    assert np.array_equal(e[0], bf16_round(bf16_round(np.full(4, 0.25)) @ E[:4]))
+    # brute force: the selected set is the k largest bf16 logits, the weights their softmax
+    l = rng.standard_normal((2, V)).astype(np.float32) * 3
+    k = 7
+    e, ids = S.expected_embedding_topk(l, W, k)
+    for t in range(2):
+        lb = bf16_round(l[t].astype(np.float64))
+        ranked = sorted(range(V), key=lambda v: (-lb[v], v))[:k]
+        assert list(ids[t]) == sorted(ranked)
+        w = np.exp(lb[sorted(ranked)] - lb[ranked[0]])
+        want = bf16_round(bf16_round(w / w.sum()) @ E[sorted(ranked)])
+        assert np.array_equal(e[t], want)
+    # k >= V keeps every id
+    e, ids = S.expected_embedding_topk(l, W, V + 5)
+    assert ids.shape == (2, V)
