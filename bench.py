@@ -47,6 +47,11 @@ WORKLOADS = {
     "moe1sc": dict(cfg=dict(n_layers=1, d_model=2816, n_q_heads=16, n_kv_heads=8, head_dim=176,
                             n_experts=128, top_k=8, d_ff=704, vocab=16384, self_cond=True),
                    ctx=1024, batch=1),
+    # one full-width layer with 16 experts and the full vocabulary, self-conditioning (3.3 GB of
+    # weights): the workload for captures of the vocabulary-phase kernels at their real width
+    "vocab1": dict(cfg=dict(n_layers=1, d_model=2816, n_q_heads=16, n_kv_heads=8, head_dim=176,
+                            n_experts=16, top_k=8, d_ff=704, vocab=262144, self_cond=True),
+                   ctx=1024, batch=1),
     # tiny: 2 layers, d 256, 16 experts top-2, vocab 4096, context 64
     "tiny": dict(cfg=dict(n_layers=2, d_model=256, n_q_heads=8, n_kv_heads=8, head_dim=32, n_experts=16,
                           top_k=2, d_ff=512, vocab=4096, self_cond=False),
@@ -453,11 +458,14 @@ def workload_config(args, wl, world):
                          "layer1": "single-layer full-width step (context 2048, batch 1)",
                          "moe1": "single full-width layer, vocabulary 16384 (context 1024, batch 1)",
                          "moe1sc": "single full-width layer, vocabulary 16384, self-conditioning (context 1024, batch 1)",
+                         "vocab1": "single full-width layer with 16 experts, vocabulary 262144, self-conditioning "
+                                   "(context 1024)",
                          "tiny": "tiny 2-layer step (context 64, batch 1)"}[args.workload],
             "n_layers": c["n_layers"], "d_model": c["d_model"], "heads": f"{c['n_q_heads']}q/{c['n_kv_heads']}kv x {c['head_dim']}",
             "experts": f"{c['n_experts']} top-{c['top_k']} ffn {c['d_ff']}", "vocab": c["vocab"],
             "self_cond": bool(c["self_cond"]), "context": wl["ctx"], "canvas": CANVAS, "batch_per_gpu": wl["batch"],
             "global_batch": wl["batch"] * world, "parallelism": f"replicas x{world}",
+            "selfcond_topk": getattr(args, "selfcond_topk", 0),
             "l2": "inputs larger than L2: every step streams the full weight set (no flush needed)"
             if args.workload != "tiny" else "L2 flushed between steps (256 MiB write)",
             "weights": "random-init bf16, seeded generator, std 0.02"}
@@ -476,8 +484,14 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode-loop", action="store_true")
     ap.add_argument("--no-other-configs", action="store_true")
+    ap.add_argument("--batch", type=int, default=0, help="canvases per GPU (0: the workload's)")
+    ap.add_argument("--selfcond-topk", type=int, default=0,
+                    help="time the round with the self-conditioning input over each position's K largest "
+                         "logits (the high-batch variant); 0 = the method")
     args = ap.parse_args()
-    wl = WORKLOADS[args.workload]
+    wl = dict(WORKLOADS[args.workload])
+    if args.batch > 0:
+        wl["batch"] = args.batch
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
@@ -508,7 +522,8 @@ def main():
     model.encode(kv, ctx_tok)
     cv = dg.Canvas(cfg, B)
     model.canvas_init(cv, 0, SEED + rank)
-    samp = dg.sampler_config(max_steps=MAX_STEPS, stop_entropy=0.5, lock_threshold=0.9, seed=SEED + rank)
+    samp = dg.sampler_config(max_steps=MAX_STEPS, stop_entropy=0.5, lock_threshold=0.9, seed=SEED + rank,
+                             selfcond_topk=args.selfcond_topk)
     model.check_device()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda") if args.workload == "tiny" else None
 

@@ -124,6 +124,7 @@ def _load():
         "dg_test_workspace_buffer": (I32, [P, ctypes.c_char_p, ctypes.POINTER(P), ctypes.POINTER(S)]),
         "dg_test_wait_timeout": (I32, [P, ctypes.c_int64, P]),
         "dg_test_struct_size": (S, [ctypes.c_char_p]),
+        "dg_test_expected_embedding_topk": (I32, [P, ctypes.c_int64, I32, P, I32, I32, P, P]),
         "dg_router_probe": (I32, [P, I32, P, I32, P, P]),
         "dg_ar_step": (I32, [P, ctypes.POINTER(dg_kv), P, F, U64, P, P, P, P]),
         "dg_attention_static_scratch": (I32, [P, P, P, P, I32, I32, I32, I32, I32, I32, I32, I32, I32, P]),

@@ -1829,6 +1829,20 @@ extern "C" dg_status dg_test_wait_timeout(dg_ctx* c, int64_t limit_ns, void* str
   return DG_OK;
 }
 
+extern "C" dg_status dg_test_expected_embedding_topk(const uint16_t* d_logits, int64_t V, int32_t K,
+                                                     const uint16_t* d_emb, int32_t d, int32_t T, uint16_t* d_out,
+                                                     void* stream) {
+  if (!d_logits || !d_emb || !d_out || V < 256 || V % 256 || K < 1 || K > std::min<int64_t>(kTopkMax, V) ||
+      d < 64 || d % 64 || d > 4096 || T < 1)
+    return fail(DG_ERR_INVALID_ARG, "dg_test_expected_embedding_topk: bad arguments");
+  cudaStream_t st = (cudaStream_t)stream;
+  DG_TRY(set_smem_attr((const void*)topk_esum_kernel, (int)sizeof(TopkSmem), false));
+  DG_CUDA(Launch(dim3(std::min(T, device_sms())), dim3(kTopkThreads), sizeof(TopkSmem), st, false)(
+      topk_esum_kernel, d_logits, (long long)V, K, d_emb, d, DG_CANVAS, T, (const uint8_t*)nullptr, d_out));
+  DG_CUDA(cudaStreamSynchronize(st));
+  return DG_OK;
+}
+
 extern "C" size_t dg_test_struct_size(const char* name) {
   if (!name) return 0;
   const struct { const char* n; size_t s; } tab[] = {

@@ -932,8 +932,8 @@ namespace dg {
 // order).  Positions of canvases that are done keep their state.
 constexpr int kTopkThreads = 1024;
 constexpr int kTopkMax = 1024;     // largest K
-constexpr int kTopkBins = 512;     // first level: the key's top 9 bits (sign and exponent: one octave)
-constexpr int kTopkBins2 = 128;    // second level: the 7 mantissa bits
+constexpr int kTopkBins = 2048;    // first level: the key's top 11 bits (a quarter octave)
+constexpr int kTopkBins2 = 32;     // second level: the 5 low bits
 constexpr int kTopkStash = 8192;   // candidates held in shared memory after the second pass
 
 __device__ __forceinline__ uint32_t bf16_order_key(uint16_t b) {
@@ -978,14 +978,18 @@ __device__ __forceinline__ uint32_t bf16x2_order_keys(uint32_t w) {
 
 // dynamic shared memory of topk_esum_kernel
 struct TopkSmem {
-  int lh[kTopkBins * 32];  // lane-private histogram [bin][lane]: a warp's 32 adds never share an address
+  // lane-private histograms [bin][lane]: a warp's 32 adds never share an
+  // address; the first level packs two 16-bit counters per word (a lane sees
+  // at most V / 32 keys of a row)
+  uint32_t lh[kTopkBins / 2 * 32];
+  int lh2[kTopkBins2 * 32];
   int hist[kTopkBins];     // first level, summed over lanes
   int hist2[kTopkBins2];   // second level
   int sel_idx[kTopkMax];
   float sel_w[kTopkMax];
   int scan_ws[kTopkThreads / 32 + 1];
   float red[kTopkThreads / 32];
-  int s_b1, s_above1, s_thr, s_above, s_ns, s_nsel, s_maxkey, s_stash_ok;
+  int s_b1, s_above1, s_thr, s_above, s_cthr, s_ns, s_nsel, s_ntie, s_maxkey;
   union {
     struct {
       int id[kTopkStash];
@@ -994,6 +998,24 @@ struct TopkSmem {
     float part[8192];  // the gather's per-group partial sums [groups][d]
   } u;
 };
+
+// warp-aggregated append of up to 8 items per lane (bits of m8): returns the
+// slot of this lane's first item (its items take consecutive slots); one
+// atomic per warp
+__device__ __forceinline__ int warp_append8(uint32_t m8, int* counter) {
+  const int lane = threadIdx.x & 31;
+  const int cnt = __popc(m8);
+  int incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  int base = 0;
+  if (lane == 31 && incl) base = atomicAdd(counter, incl);
+  base = __shfl_sync(0xffffffffu, base, 31);
+  return base + incl - cnt;
+}
 
 // warp-aggregated append: the lanes with `take` get consecutive slots of
 // `counter` (one atomic per warp); returns this lane's slot (or -1)
@@ -1016,14 +1038,16 @@ __device__ __forceinline__ int warp_append(bool take, int* counter) {
 // passes.  Keys are the logits' bf16 bits mapped to an unsigned order; the
 // histograms are lane-private ([bin][lane]) so that the many keys that share
 // a bin never serialise a warp's shared-memory adds.
-//   pass 1 (from DRAM): histogram of the key's top 9 bits (one octave per
-//     bin) and the row's largest key; the bin b1 holding the K-th largest;
-//   pass 2 (from L2): histogram of the 7 low bits inside b1 (exact keys), and
+//   pass 1 (from DRAM): histogram of the key's top 11 bits (a quarter octave
+//     per bin) and the row's largest key; the bin b1 holding the K-th largest;
+//   pass 2 (from L2): histogram of the 5 low bits inside b1 (exact keys), and
 //     every key in bins >= b1 appended (id, key) to a shared stash when they
-//     fit; the K-th largest key thr follows, with the keys equal to it to take;
-//   selection: from the stash when it holds every candidate and every key
-//     equal to thr is taken, else a third pass over the row in id order; the
-//     K ids sorted ascending (bitonic) so that the sums below run in id order;
+//     fit (a second such pass with the exact threshold when they do not); the
+//     K-th largest key thr follows, with the number of keys equal to it;
+//   selection: the stashed keys above thr, then the lowest ids of the keys
+//     equal to it (sorted when not all are taken); a third pass over the row in
+//     id order only when more than 1024 keys tie at thr; the K ids sorted
+//     ascending (bitonic) so that the sums below run in id order;
 //   gather: 8 columns per thread, the K rows split over thread groups, the
 //     groups' partial sums added in group order (deterministic).
 // V is a multiple of 256, so the uint4 units of a warp are all in range or
@@ -1039,10 +1063,10 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_esum_kernel(const uint16
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const long long nv8 = V / 8;
   for (int t = blockIdx.x; t < T; t += gridDim.x) {
-    if (done[t / canvas]) continue;  // block-uniform
+    if (done && done[t / canvas]) continue;  // block-uniform
     const uint4* lr = reinterpret_cast<const uint4*>(logits + (long long)t * V);
     // ---- pass 1: octave histogram and the largest key ----
-    for (int e = tid; e < kTopkBins * 32 / 4; e += kTopkThreads) reinterpret_cast<int4*>(sm.lh)[e] = make_int4(0, 0, 0, 0);
+    for (int e = tid; e < kTopkBins / 2 * 32 / 4; e += kTopkThreads) reinterpret_cast<int4*>(sm.lh)[e] = make_int4(0, 0, 0, 0);
     __syncthreads();
     uint32_t kmax2 = 0;
     for (long long u0 = tid; u0 < nv8; u0 += 4 * kTopkThreads) {
@@ -1060,8 +1084,9 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_esum_kernel(const uint16
         for (int q = 0; q < 4; ++q) {
           const uint32_t k2 = bf16x2_order_keys(w4[q]);
           kmax2 = __vmaxu2(kmax2, k2);
-          atomicAdd(&sm.lh[(((k2 >> 7) & 0x1FFu) << 5) | lane], 1);
-          atomicAdd(&sm.lh[((k2 >> 23) << 5) | lane], 1);
+          const uint32_t b_lo = (k2 & 0xFFFFu) >> 5, b_hi = k2 >> 21;
+          atomicAdd(&sm.lh[((b_lo >> 1) << 5) | lane], 1u << ((b_lo & 1u) << 4));
+          atomicAdd(&sm.lh[((b_hi >> 1) << 5) | lane], 1u << ((b_hi & 1u) << 4));
         }
       }
     }
@@ -1069,19 +1094,22 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_esum_kernel(const uint16
     kmax = __reduce_max_sync(0xffffffffu, kmax);
     if (lane == 0) sm.red[warp] = __int_as_float((int)kmax);
     __syncthreads();
-    for (int b = warp; b < kTopkBins; b += kTopkThreads / 32) {
-      const int v = __reduce_add_sync(0xffffffffu, sm.lh[b * 32 + lane]);
-      if (lane == 0) sm.hist[b] = v;
+    for (int wi = warp; wi < kTopkBins / 2; wi += kTopkThreads / 32) {
+      const uint32_t v = sm.lh[wi * 32 + lane];
+      const int lo = (int)__reduce_add_sync(0xffffffffu, v & 0xFFFFu);
+      const int hi = (int)__reduce_add_sync(0xffffffffu, v >> 16);
+      if (lane == 0) { sm.hist[2 * wi] = lo; sm.hist[2 * wi + 1] = hi; }
     }
     __syncthreads();
     {
-      // bins from the top: thread i < 512 owns bin 511 - i
-      const int c = tid < kTopkBins ? sm.hist[kTopkBins - 1 - tid] : 0;
+      // bins from the top: thread i owns bins 2047 - 2i and 2046 - 2i
+      const int hb = kTopkBins - 1 - 2 * tid;
+      const int c0 = sm.hist[hb], c1 = sm.hist[hb - 1];
       int total;
-      const int before = block_excl_scan(c, sm.scan_ws, &total);
-      if (tid < kTopkBins && before < K && before + c >= K) {
-        sm.s_b1 = kTopkBins - 1 - tid;
-        sm.s_above1 = before;
+      const int before = block_excl_scan(c0 + c1, sm.scan_ws, &total);
+      if (before < K && before + c0 + c1 >= K) {
+        if (before + c0 >= K) { sm.s_b1 = hb;     sm.s_above1 = before; }
+        else                  { sm.s_b1 = hb - 1; sm.s_above1 = before + c0; }
       }
       if (tid == 0) {
         uint32_t km = 0;
@@ -1090,7 +1118,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_esum_kernel(const uint16
         sm.s_ns = 0;
         sm.s_nsel = 0;
       }
-      for (int e = tid; e < kTopkBins2 * 32 / 4; e += kTopkThreads) reinterpret_cast<int4*>(sm.lh)[e] = make_int4(0, 0, 0, 0);
+      for (int e = tid; e < kTopkBins2 * 32; e += kTopkThreads) sm.lh2[e] = 0;
     }
     __syncthreads();
     const uint32_t b1 = (uint32_t)sm.s_b1;
@@ -1115,63 +1143,127 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_esum_kernel(const uint16
           mx2 = __vmaxu2(mx2, k2[q]);
         }
         // most 8-key groups hold no key in bins >= b1: one vote for the warp
-        const bool cand = max(mx2 & 0xFFFFu, mx2 >> 16) >= (b1 << 7);
+        const bool cand = max(mx2 & 0xFFFFu, mx2 >> 16) >= (b1 << 5);
         if (__any_sync(0xffffffffu, cand)) {
+          uint32_t m8 = 0;
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
             const uint32_t key = (k2[q >> 1] >> (16 * (q & 1))) & 0xFFFFu;
-            const uint32_t bin = key >> 7;
-            if (bin == b1) atomicAdd(&sm.lh[(key & 127u) * 32 + lane], 1);
-            const int pos = warp_append(stash_ok && bin >= b1, &sm.s_ns);
-            if (pos >= 0) {
-              sm.u.stash.id[pos] = (int)(u * 8 + q);
-              sm.u.stash.key[pos] = (uint16_t)key;
-            }
+            const uint32_t bin = key >> 5;
+            if (bin == b1) atomicAdd(&sm.lh2[((key & 31u) << 5) | lane], 1);
+            m8 |= (uint32_t)(bin >= b1) << q;
+          }
+          if (stash_ok) {
+            int pos = warp_append8(m8, &sm.s_ns);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              if (m8 & (1u << q)) {
+                sm.u.stash.id[pos] = (int)(u * 8 + q);
+                sm.u.stash.key[pos] = (uint16_t)((k2[q >> 1] >> (16 * (q & 1))) & 0xFFFFu);
+                ++pos;
+              }
           }
         }
       }
     }
     __syncthreads();
     for (int b = warp; b < kTopkBins2; b += kTopkThreads / 32) {
-      const int v = __reduce_add_sync(0xffffffffu, sm.lh[b * 32 + lane]);
+      const int v = __reduce_add_sync(0xffffffffu, sm.lh2[b * 32 + lane]);
       if (lane == 0) sm.hist2[b] = v;
     }
     __syncthreads();
     if (warp == 0) {
-      // the K-th largest key: lane l owns the low-bit bins 127 - 4l .. 124 - 4l
-      const int hi = kTopkBins2 - 1 - 4 * lane;
-      int c4[4], loc = 0;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) { c4[q] = sm.hist2[hi - q]; loc += c4[q]; }
-      int incl = loc;
+      // the K-th largest key: lane l owns the low-bit bin 31 - l
+      const int c = sm.hist2[kTopkBins2 - 1 - lane];
+      int incl = c;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int n = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += n;
       }
-      int cum = sm.s_above1 + incl - loc;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        if (cum < K && cum + c4[q] >= K) {
-          sm.s_thr = (int)((b1 << 7) | (uint32_t)(hi - q));
-          sm.s_above = cum;                                // keys larger than thr
-          sm.s_stash_ok = stash_ok && cum + c4[q] == K;    // every key equal to thr is taken
-        }
-        cum += c4[q];
+      const int cum = sm.s_above1 + incl - c;
+      if (cum < K && cum + c >= K) {
+        sm.s_thr = (int)((b1 << 5) | (uint32_t)(kTopkBins2 - 1 - lane));
+        sm.s_above = cum;   // keys larger than thr
+        sm.s_cthr = c;      // keys equal to it
       }
+      if (lane == 0) sm.s_ntie = 0;
     }
     __syncthreads();
     const uint32_t thr = (uint32_t)sm.s_thr;
-    if (sm.s_stash_ok) {
-      // ---- selection from the stash (exactly K keys >= thr), then ids ascending ----
+    const int above = sm.s_above, c_thr = sm.s_cthr, ties_needed = K - above;
+    // the stash holds every key >= thr when it took all of bins >= b1; else one
+    // more pass collects exactly the keys >= thr when they fit
+    bool have = stash_ok;
+    if (!have && above + c_thr <= kTopkStash) {
+      if (tid == 0) sm.s_ns = 0;
+      __syncthreads();
+      for (long long u0 = tid; u0 < nv8; u0 += 4 * kTopkThreads) {
+        uint4 w[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const long long u = u0 + (long long)r * kTopkThreads;
+          w[r] = u < nv8 ? __ldcg(lr + u) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const long long u = u0 + (long long)r * kTopkThreads;
+          if (u >= nv8) break;  // warp-uniform
+          const uint32_t w4[4] = {w[r].x, w[r].y, w[r].z, w[r].w};
+          uint32_t k2[4], mx2 = 0;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            k2[q] = bf16x2_order_keys(w4[q]);
+            mx2 = __vmaxu2(mx2, k2[q]);
+          }
+          if (__any_sync(0xffffffffu, max(mx2 & 0xFFFFu, mx2 >> 16) >= thr)) {
+            uint32_t m8 = 0;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) m8 |= (uint32_t)(((k2[q >> 1] >> (16 * (q & 1))) & 0xFFFFu) >= thr) << q;
+            int pos = warp_append8(m8, &sm.s_ns);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              if (m8 & (1u << q)) {
+                sm.u.stash.id[pos] = (int)(u * 8 + q);
+                sm.u.stash.key[pos] = (uint16_t)((k2[q >> 1] >> (16 * (q & 1))) & 0xFFFFu);
+                ++pos;
+              }
+          }
+        }
+      }
+      __syncthreads();
+      have = true;
+    }
+    if (have && c_thr <= kTopkMax) {
+      // ---- selection from the stash: the keys above thr, then the ties_needed
+      // lowest ids of the keys equal to it; finally the K ids ascending ----
+      int* tie_ids = reinterpret_cast<int*>(sm.sel_w);  // free until the weights
       const int ns = sm.s_ns;
       for (int e0 = 0; e0 < ns; e0 += kTopkThreads) {
         const int e = e0 + tid;
-        const bool take = e < ns && (uint32_t)sm.u.stash.key[e] >= thr;
-        const int pos = warp_append(take, &sm.s_nsel);
+        const uint32_t key = e < ns ? (uint32_t)sm.u.stash.key[e] : 0u;
+        const int pos = warp_append(e < ns && key > thr, &sm.s_nsel);
         if (pos >= 0) sm.sel_idx[pos] = sm.u.stash.id[e];
+        const int pt = warp_append(e < ns && key == thr, &sm.s_ntie);
+        if (pt >= 0) tie_ids[pt] = sm.u.stash.id[e];
       }
       __syncthreads();
+      if (ties_needed < c_thr) {
+        int n2 = 1;
+        while (n2 < c_thr) n2 <<= 1;
+        for (int e = c_thr + tid; e < n2; e += kTopkThreads) tie_ids[e] = 0x7FFFFFFF;
+        __syncthreads();
+        for (int k2 = 2; k2 <= n2; k2 <<= 1)
+          for (int j2 = k2 >> 1; j2 > 0; j2 >>= 1) {
+            const int e = tid, f = e ^ j2;
+            if (e < n2 && f > e) {
+              const int a = tie_ids[e], b = tie_ids[f];
+              if (((e & k2) == 0) == (a > b)) { tie_ids[e] = b; tie_ids[f] = a; }
+            }
+            __syncthreads();
+          }
+      }
+      for (int e = tid; e < ties_needed; e += kTopkThreads) sm.sel_idx[above + e] = tie_ids[e];
       int n2 = 1;
       while (n2 < K) n2 <<= 1;
       for (int e = K + tid; e < n2; e += kTopkThreads) sm.sel_idx[e] = 0x7FFFFFFF;
@@ -1186,8 +1278,8 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_esum_kernel(const uint16
           __syncthreads();
         }
     } else {
-      // ---- pass 3: collect in id order (each thread a contiguous id range) ----
-      const int ties_needed = K - sm.s_above;
+      // ---- pass 3 (more than kTopkMax keys tie at thr, or too many above it):
+      // collect in id order, each thread a contiguous id range ----
       const long long per = (nv8 + kTopkThreads - 1) / kTopkThreads;  // uint4 units per thread
       const long long v0 = min(nv8, (long long)tid * per), v1 = min(nv8, v0 + per);
       int n_gt = 0, n_eq = 0;

@@ -95,6 +95,15 @@ dg_status dg_test_attention(const uint16_t* d_q, const uint16_t* d_k, const uint
    (and clears) it and the context stays usable.  Asynchronous on `stream`. */
 dg_status dg_test_wait_timeout(dg_ctx* ctx, int64_t limit_ns, void* stream);
 
+/* The top-k form of the expected embedding on its own (dg_sampler_config.
+   selfcond_topk): for each of T rows of bf16 logits d_logits [T, V] (V a
+   multiple of 256), the K (1 <= K <= min(1024, V)) largest (ties to the lower
+   id), p = bf16(softmax over those K), d_out [T, d] bf16 = bf16(sum p_v
+   E_emb[v]) with d_emb [V, d] bf16 (d a multiple of 64, at most 4096).
+   Synchronous. */
+dg_status dg_test_expected_embedding_topk(const uint16_t* d_logits, int64_t V, int32_t K, const uint16_t* d_emb,
+                                          int32_t d, int32_t T, uint16_t* d_out, void* stream);
+
 /* sizeof of one of the ABI's structs by its name ("dg_model_config",
    "dg_sampler_config", "dg_kv", "dg_canvas", "dg_step_args", "dg_step_out",
    "dg_block_stats", "dg_profile"), 0 for another name.  Host only: lets a
