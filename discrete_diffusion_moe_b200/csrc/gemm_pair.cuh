@@ -193,8 +193,14 @@ __global__ void __launch_bounds__(gemm_threads<Epi>(), 2)
   uint32_t* tmem_slot = (uint32_t*)(drain + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  touch_plan(p);
   const uint32_t rank = cluster_ctarank();
   const int cidx = (int)(blockIdx.x >> 1), ncl = (int)(gridDim.x >> 1);
+  // a dense plan's first job needs no table: computed before any wait
+  const bool dense = p.group_off == nullptr;
+  const GemmJob j_first = dense ? pair_job(p, tabs, cidx, (int)rank) : GemmJob{};
+  const GemmJob j_first0 = dense ? pair_job(p, tabs, cidx, 0) : GemmJob{};
+  const int U_dense = dense ? pair_num_units(p, tabs) : 0;
   const uint32_t buf_cols = (uint32_t)p.bn;
   const uint32_t tmem_cols = 2u * buf_cols <= 32u ? 32u : (2u * buf_cols <= 64u ? 64u : (2u * buf_cols <= 128u ? 128u : (2u * buf_cols <= 256u ? 256u : 512u)));
   const uint32_t acc_stride = tmem_cols / 2;  // two accumulator buffers
@@ -233,7 +239,7 @@ __global__ void __launch_bounds__(gemm_threads<Epi>(), 2)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int U = pair_num_units(p, tabs);
+  const int U = dense ? U_dense : pair_num_units(p, tabs);
 
   if (warp == 0) {
     if (lane == 0) {
@@ -244,7 +250,7 @@ __global__ void __launch_bounds__(gemm_threads<Epi>(), 2)
       const uint64_t pol_a = p.a_hint == 1 ? pol_first : pol_last;
       const uint64_t pol_b = p.b_hint == 1 ? pol_first : pol_last;
       for (int u = cidx; u < U && ok; u += ncl) {
-        const GemmJob j = pair_job(p, tabs, u, (int)rank);
+        const GemmJob j = (dense && u == cidx) ? j_first : pair_job(p, tabs, u, (int)rank);
         const int bi = pair_b_map(p, j.n_valid);
         const int half = ((j.n_valid + 15) & ~15) >> 1;
         const bool a_mine = j.m_valid > 0;
@@ -275,7 +281,7 @@ __global__ void __launch_bounds__(gemm_threads<Epi>(), 2)
       uint32_t it = 0, jc = 0;
       bool ok = true;
       for (int u = cidx; u < U && ok; u += ncl, ++jc) {
-        const GemmJob j = pair_job(p, tabs, u, 0);
+        const GemmJob j = (dense && u == cidx) ? j_first0 : pair_job(p, tabs, u, 0);
         const int n_mma = (j.n_valid + 15) & ~15;
         const uint32_t idesc = idesc_bf16_f32(256, n_mma);
         const uint32_t acc = jc & 1, use = jc >> 1;
@@ -311,7 +317,7 @@ __global__ void __launch_bounds__(gemm_threads<Epi>(), 2)
     uint32_t jc = 0;
     bool ok = true;
     for (int u = cidx; u < U && ok; u += ncl, ++jc) {
-      const GemmJob j = pair_job(p, tabs, u, (int)rank);
+      const GemmJob j = (dense && u == cidx) ? j_first : pair_job(p, tabs, u, (int)rank);
       const uint32_t acc = jc & 1, use = jc >> 1;
       if (!mbar_wait(smem_u32(&acc_full[acc]), use & 1, p.err)) { ok = false; break; }
       tc_fence_after();
