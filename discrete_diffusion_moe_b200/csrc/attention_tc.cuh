@@ -84,7 +84,7 @@ struct AttnTcShape {
   static constexpr uint32_t V_BYTES = HD * 128;      // hd rows x 64 keys
   static constexpr uint32_t P_BYTES = kAttnRows * 128;  // one fp16 P tile (128 rows x 64 keys)
   // four P tiles: the high and low fp16 parts of P, two buffers of each by tile parity
-  static constexpr size_t FIXED = 1024 + Q_BYTES + 2 * kAttnPParts * P_BYTES + 24 * 8 + 6 * 128 * 4;
+  static constexpr size_t FIXED = 1024 + Q_BYTES + 2 * kAttnPParts * P_BYTES + 32 * 8 + 6 * 128 * 4;
   // K/V stages: three where they fit (the load of tile i + 3 is in flight while
   // tiles i + 1, i + 2 are multiplied), else two
   static constexpr int KV_STAGES = FIXED + 3 * (K_BYTES + V_BYTES) <= 227 * 1024 ? 3 : 2;
@@ -182,9 +182,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint8_t* sP = sV + NS * S::V_BYTES;          // P_hi [2] then P_lo [2] (fp16), by tile parity
   uint64_t* bars = (uint64_t*)(sP + 2 * kAttnPParts * S::P_BYTES);
   uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;        // [NS]
-  uint64_t* kv_empty = bars + 1 + NS;  // [NS]
-  uint64_t* s_full = bars + 1 + 2 * NS;
+  // K and V of a stage are released separately: K as soon as the scores of
+  // its tile are computed (so the next K load overlaps the softmax), V after
+  // the P V product
+  uint64_t* k_full = bars + 1;          // [NS]
+  uint64_t* k_empty = bars + 1 + NS;    // [NS]
+  uint64_t* v_full = bars + 1 + 2 * NS; // [NS]
+  uint64_t* v_empty = bars + 1 + 3 * NS;// [NS]
+  uint64_t* s_full = bars + 1 + 4 * NS;
   uint64_t* s_free = s_full + 1;
   uint64_t* p_full = s_full + 2;      // [2] by tile parity
   uint64_t* pv_done = s_full + 4;     // [2] by tile parity
@@ -214,8 +219,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(q_full), 1);
     for (int s = 0; s < NS; ++s) {
-      mbar_init(smem_u32(&kv_full[s]), 1);
-      mbar_init(smem_u32(&kv_empty[s]), 1);
+      mbar_init(smem_u32(&k_full[s]), 1);
+      mbar_init(smem_u32(&k_empty[s]), 1);
+      mbar_init(smem_u32(&v_full[s]), 1);
+      mbar_init(smem_u32(&v_empty[s]), 1);
     }
     mbar_init(smem_u32(s_full), 1);
     mbar_init(smem_u32(s_free), 256);
@@ -251,21 +258,30 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int q_row0 = bg * rows_total + r0;
       for (int a = 0; a < S::NA; ++a) tma_load_2d(smem_u32(sQ + a * 16384), &tmQ, qb, a * 64, q_row0);
       int issued = 0;
-      for (int i = 0; i < n_tiles; ++i, ++issued) {
+      int issued_v = 0;
+      for (int i = 0; i < n_tiles; ++i) {
         const int s = i % NS;
-        if (!mbar_wait(smem_u32(&kv_empty[s]), ((i / NS) & 1) ^ 1, p.err)) break;
-        const uint32_t fb = smem_u32(&kv_full[s]);
-        mbar_arrive_expect_tx(fb, S::K_BYTES + S::V_BYTES);
+        const uint32_t par = ((i / NS) & 1) ^ 1;
         const int key0 = (kt0 + i) * kAttnKeys;
+        if (!mbar_wait(smem_u32(&k_empty[s]), par, p.err)) break;
+        const uint32_t kb = smem_u32(&k_full[s]);
+        mbar_arrive_expect_tx(kb, S::K_BYTES);
         for (int a = 0; a < S::NA; ++a)
-          tma_load_2d(smem_u32(sK + s * S::K_BYTES + a * kAttnKeys * 128), &tmK, fb, a * 64,
+          tma_load_2d(smem_u32(sK + s * S::K_BYTES + a * kAttnKeys * 128), &tmK, kb, a * 64,
                       bg * p.c_max + key0);
-        tma_load_2d(smem_u32(sV + s * S::V_BYTES), &tmV, fb, key0, bg * HD);
+        ++issued;
+        if (!mbar_wait(smem_u32(&v_empty[s]), par, p.err)) break;
+        const uint32_t vb = smem_u32(&v_full[s]);
+        mbar_arrive_expect_tx(vb, S::V_BYTES);
+        tma_load_2d(smem_u32(sV + s * S::V_BYTES), &tmV, vb, key0, bg * HD);
+        ++issued_v;
       }
       // every issued copy must land before the CTA may exit
-      const int first = issued > NS ? issued - NS : 0;
       mbar_wait(qb, 0, p.err);
-      for (int i = first; i < issued; ++i) mbar_wait(smem_u32(&kv_full[i % NS]), (i / NS) & 1, p.err);
+      for (int i = issued > NS ? issued - NS : 0; i < issued; ++i)
+        mbar_wait(smem_u32(&k_full[i % NS]), (i / NS) & 1, p.err);
+      for (int i = issued_v > NS ? issued_v - NS : 0; i < issued_v; ++i)
+        mbar_wait(smem_u32(&v_full[i % NS]), (i / NS) & 1, p.err);
     }
   } else if (warp == 1) {
     if (lane == 0 && n_tiles > 0) {
@@ -275,7 +291,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       bool ok = mbar_wait(smem_u32(q_full), 0, p.err);
       auto issue_s = [&](int i) -> bool {
         const int s = i % NS;
-        if (!mbar_wait(smem_u32(&kv_full[s]), (i / NS) & 1, p.err)) return false;
+        if (!mbar_wait(smem_u32(&k_full[s]), (i / NS) & 1, p.err)) return false;
         if (i > 0 && !mbar_wait(smem_u32(s_free), (i - 1) & 1, p.err)) return false;
         tc_fence_after();
         const uint32_t qa = smem_u32(sQ), ka = smem_u32(sK + s * S::K_BYTES);
@@ -286,12 +302,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     id_s, k > 0 ? 1u : 0u);
         }
         umma_commit(smem_u32(s_full));
+        umma_commit(smem_u32(&k_empty[s]));  // K of this stage is consumed once the scores are
         return true;
       };
       if (ok) ok = issue_s(0);
       for (int i = 0; i < n_tiles && ok; ++i) {
         if (i + 1 < n_tiles && !issue_s(i + 1)) { ok = false; break; }
         if (!mbar_wait(smem_u32(&p_full[i & 1]), (i >> 1) & 1, p.err)) { ok = false; break; }
+        if (!mbar_wait(smem_u32(&v_full[i % NS]), (i / NS) & 1, p.err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t va = smem_u32(sV + (i % NS) * S::V_BYTES);
         const uint32_t pa = smem_u32(sP + (i & 1) * S::P_BYTES);
@@ -306,7 +324,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             umma_bf16(t_o, sdesc_k128(pl + k * 32), sdesc_k128(va + k * 32), id_o, 1u);
         }
         umma_commit(smem_u32(&pv_done[i & 1]));
-        umma_commit(smem_u32(&kv_empty[i % NS]));
+        umma_commit(smem_u32(&v_empty[i % NS]));
       }
       umma_commit(smem_u32(drain));
       mbar_wait(smem_u32(drain), 0, p.err);
@@ -566,23 +584,38 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int n_items = (q1 - q0) * NC4;
       const int G = p.Hq / p.Hkv;
       const int rows_total = G * p.nq;
-      for (int it = te; it < n_items; it += 256) {
-        const int rr = it / NC4, c4 = it - rr * NC4;
-        const int row = q0 + rr;
-        const int r = r0 + row;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        const uint32_t off = o_base + (uint32_t)(row * S::OSTR + c4 * 4) * 4u;
+      // two items per pass: all of their remote loads are issued before the
+      // first is used (a remote load's latency, not its bandwidth, bounds this)
+      constexpr int kItems = 2;
+      for (int it0 = te; it0 < n_items; it0 += 256 * kItems) {
+        float4 v[kItems][8];
 #pragma unroll
-        for (int s2 = 0; s2 < 8; ++s2)
-          if (s2 < S_) {
-            const float ws = wts[rr * 8 + s2];
-            const float4 v = ld_dsmem_f4(mapa_shared(off, (uint32_t)s2));
-            acc.x += ws * v.x; acc.y += ws * v.y; acc.z += ws * v.z; acc.w += ws * v.w;
+        for (int u = 0; u < kItems; ++u) {
+          const int it = it0 + u * 256;
+          const int rr = it / NC4, c4 = it - rr * NC4;
+          const uint32_t off = o_base + (uint32_t)((q0 + rr) * S::OSTR + c4 * 4) * 4u;
+#pragma unroll
+          for (int s2 = 0; s2 < 8; ++s2)
+            if (s2 < S_ && it < n_items) v[u][s2] = ld_dsmem_f4(mapa_shared(off, (uint32_t)s2));
+        }
+#pragma unroll
+        for (int u = 0; u < kItems; ++u) {
+          const int it = it0 + u * 256;
+          if (it >= n_items) break;
+          const int rr = it / NC4, c4 = it - rr * NC4;
+          const int r = r0 + q0 + rr;
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int s2 = 0; s2 < 8; ++s2)
+            if (s2 < S_) {
+              const float ws = wts[rr * 8 + s2];
+              acc.x += ws * v[u][s2].x; acc.y += ws * v[u][s2].y; acc.z += ws * v[u][s2].z; acc.w += ws * v[u][s2].w;
+            }
+          if (r < rows_total) {
+            const int t_in = r / G, h = g * G + r % G;
+            uint16_t* dst = p.out + ((long long)(b * p.nq + t_in) * p.Hq + h) * HD + c4 * 4;
+            *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
           }
-        if (r < rows_total) {
-          const int t_in = r / G, h = g * G + r % G;
-          uint16_t* dst = p.out + ((long long)(b * p.nq + t_in) * p.Hq + h) * HD + c4 * 4;
-          *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
         }
       }
     }
