@@ -73,6 +73,11 @@ struct NvtxRange {
 #ifndef DG_PDL
 #define DG_PDL 1
 #endif
+// 1: the QKV and output projections run on CTA pairs (each CTA of a pair
+// copies half of the unit's token rows), with the same k splits and partials
+#ifndef DG_PROJ_PAIR
+#define DG_PROJ_PAIR 0
+#endif
 // token rows per grouped (expert) unit: 0 chooses 128 on CTA pairs, or 256 on
 // single CTAs when experts average more than 64 tokens; 256 takes 256-token
 // chunks on CTA pairs (one read of an expert's weight tile for up to 256 tokens)
@@ -483,7 +488,8 @@ dg_status run_gemm(const CUtensorMap& ta, const BOperand& tb, GemmPlan p, const 
 template <class Epi>
 dg_status run_gemm_pair(const CUtensorMap& ta, const BOperand& tb, GemmPlan p, const Epi& epi, int num_sms,
                         cudaStream_t st, long long* launches = nullptr) {
-  if ((p.group_off && (p.n_groups < 1 || p.n_groups > kGemmMaxGroups)) || p.mt != 1 || p.k_splits != 1)
+  if ((p.group_off && (p.n_groups < 1 || p.n_groups > kGemmMaxGroups || p.k_splits != 1)) || p.mt != 1 ||
+      p.k_splits < 1 || p.k_splits > p.K / 64)
     return fail(DG_ERR_INVALID_ARG, "pair gemm: %d groups, %d A tiles, %d k splits", p.n_groups, p.mt, p.k_splits);
   if (p.bn < 16 || p.bn > 256 || (p.bn & (p.bn - 1)) || p.K % 64 || p.K < 64)
     return fail(DG_ERR_INVALID_ARG, "pair gemm plan: bn %d K %d", p.bn, p.K);
@@ -894,10 +900,20 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
       BOperand tb;
       const int bn = dense_bn_x;
       DG_TRY(make_tmap(&ta, c->wp(W.wqkv), d, qkv_rows, 128));
-      DG_TRY(make_bop(&tb, xn, d, L.T_alloc, bn));
       GemmPlan p = dense_plan(d, qkv_rows, T, bn, ks_qkv, err);
       p.a_hint = 1;
-      if (DG_QKV_CLUSTER || ks_qkv == 1) {
+      const bool pair_qkv = DG_PROJ_PAIR && !DG_QKV_CLUSTER;
+      if (pair_qkv) DG_TRY(make_bop_half(&tb, xn, d, L.T_alloc, bn));
+      else          DG_TRY(make_bop(&tb, xn, d, L.T_alloc, bn));
+      if (pair_qkv) {
+        if (ks_qkv == 1) {
+          EpiQKV e{c->at<double2>(L.rope), c->at<uint16_t>(L.q), kc, vc, nq, L0, kv->c_max, Hq, Hkv, hd};
+          DG_TRY(run_gemm_pair(ta, tb, p, e, c->num_sms, st, &c->n_launch));
+        } else {
+          EpiStoreT e{c->at<float>(L.qkv), qkv_rows, (long long)T * qkv_rows, 0, nullptr, nullptr, 0, err};
+          DG_TRY(run_gemm_pair(ta, tb, p, e, c->num_sms, st, &c->n_launch));
+        }
+      } else if (DG_QKV_CLUSTER || ks_qkv == 1) {
         p.cluster_k = ks_qkv;  // the k splits of a tile add up in their cluster
         EpiQKV e{c->at<double2>(L.rope), c->at<uint16_t>(L.q), kc, vc, nq, L0, kv->c_max, Hq, Hkv, hd};
         DG_TRY(run_gemm(ta, tb, p, e, c->num_sms, st, &c->n_launch));
@@ -927,10 +943,20 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
       BOperand tb;
       const int bn = dense_bn_x;
       DG_TRY(make_tmap(&ta, c->wp(W.wo), (long long)Hq * hd, d, 128));
-      DG_TRY(make_bop(&tb, c->at<uint16_t>(L.attn), (long long)Hq * hd, L.T_alloc, bn));
       GemmPlan p = dense_plan(Hq * hd, d, T, bn, ks_o, err);
       p.a_hint = 1;
-      if (DG_O_CLUSTER || ks_o == 1) {
+      const bool pair_o = DG_PROJ_PAIR && !DG_O_CLUSTER;
+      if (pair_o) DG_TRY(make_bop_half(&tb, c->at<uint16_t>(L.attn), (long long)Hq * hd, L.T_alloc, bn));
+      else        DG_TRY(make_bop(&tb, c->at<uint16_t>(L.attn), (long long)Hq * hd, L.T_alloc, bn));
+      if (pair_o) {
+        if (ks_o == 1) {
+          EpiStoreT e{x, d, 0, 1, nullptr, nullptr, 0, err};  // residual add: x += attn W_o^T
+          DG_TRY(run_gemm_pair(ta, tb, p, e, c->num_sms, st, &c->n_launch));
+        } else {
+          EpiStoreT e{c->at<float>(L.opart), d, (long long)T * d, 0, nullptr, nullptr, 0, err};
+          DG_TRY(run_gemm_pair(ta, tb, p, e, c->num_sms, st, &c->n_launch));
+        }
+      } else if (DG_O_CLUSTER || ks_o == 1) {
         p.cluster_k = ks_o;
         EpiStoreT e{x, d, 0, 1, nullptr, nullptr, 0, err};  // residual add: x += attn W_o^T
         DG_TRY(run_gemm(ta, tb, p, e, c->num_sms, st, &c->n_launch));

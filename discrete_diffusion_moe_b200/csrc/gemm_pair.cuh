@@ -111,7 +111,7 @@ __device__ __forceinline__ void umma_commit_pair(uint32_t bar) {
 __host__ __device__ __forceinline__ int pair_tiles(const GemmPlan& p) { return (p.m_tiles + 1) >> 1; }
 
 __host__ __device__ __forceinline__ int pair_num_units(const GemmPlan& p, const GemmTables& tb) {
-  if (!p.group_off) return pair_tiles(p) * ((p.n_total + p.bn - 1) / p.bn);
+  if (!p.group_off) return pair_tiles(p) * ((p.n_total + p.bn - 1) / p.bn) * p.k_splits;
   return pair_tiles(p) * tb.chunk_off[p.n_groups];
 }
 
@@ -121,10 +121,12 @@ __host__ __device__ __forceinline__ int pair_num_units(const GemmPlan& p, const 
 __host__ __device__ __forceinline__ GemmJob pair_job(const GemmPlan& p, const GemmTables& tb, int u, int rank) {
   const int P = pair_tiles(p);
   if (!p.group_off) {
-    // dense: unit u = (tile pair u % P, column tile u / P); consecutive units
-    // share a column tile (its B rows are read from L2 after the first)
+    // dense: unit u = (k split u % k_splits, then tile pair, then column
+    // tile); consecutive units share a column tile (its B rows are read from
+    // L2 after the first)
     GemmJob j;
-    const int pr = u % P, nt = u / P;
+    const int ks = u % p.k_splits, r = u / p.k_splits;
+    const int pr = r % P, nt = r / P;
     j.m_tile = 2 * pr + rank;
     j.group = -1;
     j.a_row0 = j.m_tile * 128;
@@ -132,9 +134,9 @@ __host__ __device__ __forceinline__ GemmJob pair_job(const GemmPlan& p, const Ge
     j.n_local0 = nt * p.bn;
     j.n0 = j.n_local0;
     j.n_valid = min(p.bn, p.n_total - j.n0);
-    j.ks = 0;
-    j.kb0 = 0;
-    j.kb1 = p.K / 64;
+    j.ks = ks;
+    j.kb0 = (p.K / 64) * ks / p.k_splits;       // K / 64 * k_splits < 2^31
+    j.kb1 = (p.K / 64) * (ks + 1) / p.k_splits;
     j.mt_eff = 1;
     return j;
   }
