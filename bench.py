@@ -150,17 +150,24 @@ def kernel_source_hash():
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(kernel_key):
-    """DRAM bytes per launch of the dominant kernel from the committed ncu
-    summary, or None when missing or taken on a different kernel source."""
+def ncu_traffic(kernel_key, distinct_mean):
+    """DRAM bytes per launch of the dominant kernel, scaled from the committed
+    ncu capture of one launch on the one-layer workload, or None when missing
+    or taken on a different kernel source.  The capture's bytes beyond the
+    launch's expert-independent part (the permuted inputs and the outputs of
+    the same 256 canvas tokens) grow with the distinct experts the launch
+    streams, so a full-size launch is that part plus the rest times the
+    round's mean distinct experts per layer over the capture's count."""
     p = os.path.join(ROOT, "profiles", "dram_traffic.json")
     if not os.path.exists(p):
         return None
     j = json.load(open(p))
     e = j.get(kernel_key)
-    if not e or e.get("source_hash") != kernel_source_hash():
+    if not e or e.get("source_hash") != kernel_source_hash() or not distinct_mean:
         return None
-    return e.get("bytes_per_launch_full")
+    measured = e["read_bytes"] + e["write_bytes"]
+    fixed = e["fixed_bytes"]
+    return fixed + (measured - fixed) * distinct_mean / e["distinct_experts"]
 
 
 # ---------------------------------------------------------------------------
@@ -688,7 +695,7 @@ def main():
                               "peaks": f"{peaks['source']}: {peaks['hbm_gbs']} GB/s, {peaks['bf16_tflops_sustained']} TF/s sustained bf16"},
             "roofline": {"kernel": "gemm_pair_kernel<EpiSwiGLU> (grouped expert gate/up + SwiGLU, CTA pairs)", "bound": "hbm",
                          "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": achieved / peaks["hbm_gbs"], "traffic": ncu_traffic("expert_gate_up"),
+                         "frac": achieved / peaks["hbm_gbs"], "traffic": ncu_traffic("expert_gate_up", avg_distinct),
                          "bytes_per_launch": gu_bytes, "launch_ms": gu_ms,
                          "peak_source": f"{peaks['source']} (of {peaks['source']})"},
             "kernel_breakdown": breakdown,
