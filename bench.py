@@ -669,6 +669,11 @@ def main():
     P = B * CANVAS * c["top_k"]
     avg_distinct = sum(distinct) / len(distinct)
     gu_bytes = avg_distinct * 2 * c["d_ff"] * c["d_model"] * 2 + P * c["d_model"] * 2 + P * c["d_ff"] * 2
+    # with the fused expert kernel (no separate down launches) the launch also
+    # streams the down weights, reads the SwiGLU outputs and writes the fp32 outputs
+    fused = prof.launches[1] == 0
+    if fused:
+        gu_bytes += avg_distinct * c["d_model"] * c["d_ff"] * 2 + P * c["d_ff"] * 2 + P * c["d_model"] * 4
     achieved = gu_bytes / (gu_ms / 1000.0) / 1e9
     kinds = ["expert_gate_up", "expert_down", "lm_head", "attention", "dense_proj", "expected_emb"]
     breakdown = {kinds[i]: {"ms_per_step": prof.ms[i] / args.steps, "launches_per_step": prof.launches[i] / args.steps}
@@ -693,9 +698,13 @@ def main():
                               "frac": t_roof / (ms_per_step / 1000.0),
                               "bound": "hbm" if nbytes / (peaks["hbm_gbs"] * 1e9) >= flops / (peaks["bf16_tflops_sustained"] * 1e12) else "tensor",
                               "peaks": f"{peaks['source']}: {peaks['hbm_gbs']} GB/s, {peaks['bf16_tflops_sustained']} TF/s sustained bf16"},
-            "roofline": {"kernel": "gemm_pair_kernel<EpiSwiGLU> (grouped expert gate/up + SwiGLU, CTA pairs)", "bound": "hbm",
+            "roofline": {"kernel": ("moe_pair_kernel<EpiSwiGLU, EpiDown> (both grouped expert products in one launch, "
+                                    "CTA pairs)" if fused else
+                                    "gemm_pair_kernel<EpiSwiGLU> (grouped expert gate/up + SwiGLU, CTA pairs)"),
+                         "bound": "hbm",
                          "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": achieved / peaks["hbm_gbs"], "traffic": ncu_traffic("expert_gate_up", avg_distinct),
+                         "frac": achieved / peaks["hbm_gbs"],
+                         "traffic": ncu_traffic("expert_block" if fused else "expert_gate_up", avg_distinct),
                          "bytes_per_launch": gu_bytes, "launch_ms": gu_ms,
                          "peak_source": f"{peaks['source']} (of {peaks['source']})"},
             "kernel_breakdown": breakdown,

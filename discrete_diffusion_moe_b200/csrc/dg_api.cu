@@ -24,6 +24,7 @@
 #include "epilogues.cuh"
 #include "gemm_pair.cuh"
 #include "gemm_tc.cuh"
+#include "moe_pair.cuh"
 #include "kernels.cuh"
 
 using namespace dg;
@@ -77,6 +78,12 @@ struct NvtxRange {
 // copies half of the unit's token rows), with the same k splits and partials
 #ifndef DG_PROJ_PAIR
 #define DG_PROJ_PAIR 0
+#endif
+// 1: the two grouped expert products run as one persistent launch on CTA
+// pairs (moe_pair.cuh), a chunk's down product starting as soon as its
+// gate/up outputs are stored
+#ifndef DG_MOE_FUSED
+#define DG_MOE_FUSED 1
 #endif
 // token rows per grouped (expert) unit: 0 chooses 128 on CTA pairs, or 256 on
 // single CTAs when experts average more than 64 tokens; 256 takes 256-token
@@ -189,7 +196,7 @@ constexpr int kMaxAttnSplits = 8;
 struct WsLayout {
   size_t err, flags, x, xn, qkv, opart, q, attn, rpart, tok, xnc, rbar, rfill, off, choff, perm, inv, wperm,
       xperm, hperm, yperm, logits, vp_m, vp_z, vp_s, vp_av, vp_ai, vp_gv, vp_gi, st_m, st_iz, st_h,
-      st_pmax, st_amax, st_samp, probs, epart, rope, stepdev, dstat, total;
+      st_pmax, st_amax, st_samp, probs, epart, rope, stepdev, dstat, dep, total;
   int T_alloc, P_alloc, ks_r, n_vt;  // T_alloc: token rows of a layer pass (>= the canvas tokens)
   int T_canvas;                       // canvas tokens (batch * 256): rows of the vocabulary buffers
   long long epart_rows;
@@ -308,6 +315,7 @@ WsLayout ws_layout(const dg_model_config& c, int batch, int num_sms, int prefill
   L.rope = take(T * (c.head_dim / 2) * 16);  // (cos, sin) of up to T positions of a pass
   L.stepdev = take(sizeof(StepDev));
   L.dstat = take((size_t)c.n_layers * 4);  // distinct experts per layer, summed over passes
+  L.dep = take((P / 16 + E + 1) * 4);       // the fused expert kernel's chunk counters (chunks of >= 16 slots)
   L.probs = c.self_cond ? take(Tc * V * 2) : 0;
   L.epart = c.self_cond ? take((size_t)er * d * 4) : 0;
   L.total = off;
@@ -504,6 +512,38 @@ dg_status run_gemm_pair(const CUtensorMap& ta, const BOperand& tb, GemmPlan p, c
   const unsigned grid = (unsigned)(2 * (num_sms / 2) * gemm_pair_ctas_per_sm(p.bn));  // whole pairs
   DG_CUDA(Launch(dim3(grid), dim3(gemm_threads<Epi>()), smem, st).cluster(2, 1, 1)(gemm_pair_kernel<Epi>, ta,
                                                                                     tb.maps, p, epi, stages));
+  if (launches) ++*launches;
+  return DG_OK;
+}
+
+// Both grouped expert products in one launch on 2-CTA clusters (moe_pair.cuh);
+// tb1 / tb2 from make_bop_half.
+template <class EpiU, class EpiD>
+dg_status run_moe_pair(const CUtensorMap& ta1, const BOperand& tb1, const CUtensorMap& ta2, const BOperand& tb2,
+                       MoePlan mp, const EpiU& e1, const EpiD& e2, int num_sms, cudaStream_t st,
+                       long long* launches = nullptr) {
+  GemmPlan* ps[2] = {&mp.up, &mp.down};
+  const BOperand* tbs[2] = {&tb1, &tb2};
+  for (int q = 0; q < 2; ++q) {
+    GemmPlan& p = *ps[q];
+    if (!p.group_off || p.n_groups < 1 || p.n_groups > kGemmMaxGroups || p.mt != 1 || p.k_splits != 1 ||
+        p.bn < 16 || p.bn > 128 || (p.bn & (p.bn - 1)) || p.K % 64 || p.K < 64)
+      return fail(DG_ERR_INVALID_ARG, "expert kernel plan %d: groups %d bn %d K %d", q, p.n_groups, p.bn, p.K);
+    for (int i = 0; i < 3; ++i) {
+      if (tbs[q]->rows[i] < 1 || (i && tbs[q]->rows[i] < tbs[q]->rows[i - 1]) || tbs[q]->rows[i] > p.bn / 2)
+        return fail(DG_ERR_INVALID_ARG, "expert kernel plan %d: B box rows %d of bn %d", q, tbs[q]->rows[i], p.bn);
+      p.b_rows[i] = tbs[q]->rows[i];
+    }
+  }
+  if (mp.up.bn != mp.down.bn || mp.up.n_groups != mp.down.n_groups || mp.up.group_off != mp.down.group_off ||
+      mp.up.chunk_off != mp.down.chunk_off || !mp.dep)
+    return fail(DG_ERR_INVALID_ARG, "expert kernel: the two products must share groups and chunks");
+  DG_TRY(set_smem_attr((const void*)moe_pair_kernel<EpiU, EpiD>, (int)(227 * 1024 - kGemmStaticSmem), true));
+  const int stages = gemm_pair_stages(mp.up.bn);
+  const size_t smem = gemm_pair_smem_bytes(mp.up.bn, stages);
+  const unsigned grid = (unsigned)(2 * (num_sms / 2) * gemm_pair_ctas_per_sm(mp.up.bn));  // whole pairs
+  DG_CUDA(Launch(dim3(grid), dim3(gemm_threads<EpiU>()), smem, st).cluster(2, 1, 1)(
+      moe_pair_kernel<EpiU, EpiD>, ta1, tb1.maps, ta2, tb2.maps, mp, e1, e2, stages));
   if (launches) ++*launches;
   return DG_OK;
 }
@@ -1018,6 +1058,8 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
       rp.dbg_w = dbg_w ? dbg_w + (size_t)l * T_dbg * k : nullptr;
       rp.dbg_logits = dbg_logits ? dbg_logits + (size_t)l * T_dbg * E : nullptr;
       rp.distinct = c->at<int>(L.dstat) + l;
+      rp.dep = c->at<int>(L.dep);
+      rp.dep_n = (int)(L.P_alloc / 16 + E + 1);
       rp.err = err;
       const int nb = (T + rp.tpc - 1) / rp.tpc;
       cudaLaunchConfig_t lc = {};
@@ -1037,6 +1079,22 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
       else return fail(DG_ERR_UNSUPPORTED, "router split count %d", ksr);
       CNT(c);
     }
+    if (pair && DG_MOE_FUSED) {
+      // gate/up + SwiGLU and down in one launch
+      ProfScope ps_(c, DG_PROF_EXPERT_GATE_UP, st);
+      CUtensorMap ta1, ta2;
+      DG_TRY(make_tmap(&ta1, c->wp(W.wgu), d, (long long)E * 2 * f, 128));
+      DG_TRY(make_tmap(&ta2, c->wp(W.wd), f, (long long)E * d, 128));
+      MoePlan mp;
+      mp.up = grouped_plan(d, 2 * f, c->at<int>(L.off), c->at<int>(L.choff), E, bnG, err);
+      mp.down = grouped_plan(f, d, c->at<int>(L.off), c->at<int>(L.choff), E, bnG, err);
+      mp.up.a_hint = mp.down.a_hint = 1;
+      mp.up.b_hint = mp.down.b_hint = 2;
+      mp.dep = c->at<int>(L.dep);
+      EpiSwiGLU e1{c->at<uint16_t>(L.hperm), f};
+      EpiDown e2{c->at<float>(L.yperm), d, c->at<float>(L.wperm)};
+      DG_TRY(run_moe_pair(ta1, h_xperm, ta2, h_hperm, mp, e1, e2, c->num_sms, st, &c->n_launch));
+    } else {
     {
       ProfScope ps_(c, DG_PROF_EXPERT_GATE_UP, st);
       CUtensorMap ta;
@@ -1058,6 +1116,7 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
       EpiDown e{c->at<float>(L.yperm), d, c->at<float>(L.wperm)};
       if (pair) DG_TRY(run_gemm_pair(ta, h_hperm, p, e, c->num_sms, st, &c->n_launch));
       else      DG_TRY(run_gemm(ta, t_hperm, p, e, c->num_sms, st, &c->n_launch));
+    }
     }
     // combine + residual, fused with the next RMSNorm (next layer's attention
     // norm, or the final norm before the LM head)
@@ -1614,6 +1673,8 @@ extern "C" dg_status dg_router_probe(dg_ctx* c, int32_t layer, const float* d_x,
   rp.dbg_logits = nullptr;
   rp.dbg_nq = rp.dbg_skip = 0;
   rp.distinct = nullptr;
+  rp.dep = nullptr;
+  rp.dep_n = 0;
   rp.err = err;
   cudaLaunchConfig_t lc = {};
   cudaLaunchAttribute at[1];

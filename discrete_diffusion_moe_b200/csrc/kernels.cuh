@@ -400,6 +400,8 @@ struct RouteParams {
   int dbg_nq, dbg_skip;   // dbg_nq > 0: of each dbg_nq tokens the first dbg_skip are not recorded
                           // (an appending pass: only the canvas rows, compacted)
   int* distinct;          // optional: += number of experts given at least one token
+  int* dep;               // optional [dep_n]: zeroed (the fused expert kernel's chunk counters)
+  int dep_n;
   int* err;
 };
 
@@ -436,8 +438,11 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(RouteParams p) {
   const int np = nt * k;
   const int ep = __ldcg(p.bar + 2) & 1;  // this launch's fill buffer
   int* fill = p.fill + ep * E;
-  if (b == 0)
+  if (b == 0) {
     for (int e = tid; e < E; e += kRouteThreads) p.fill[(ep ^ 1) * E + e] = 0;
+    if (p.dep)
+      for (int i = tid; i < p.dep_n; i += kRouteThreads) p.dep[i] = 0;
+  }
 
   // ---- top-k of the CTA's tokens ----
   for (int lt = warp; lt < nt; lt += nw) {
