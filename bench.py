@@ -145,7 +145,8 @@ class ClockSampler:
 def kernel_source_hash():
     h = hashlib.sha256()
     for rel in ("discrete_diffusion_moe_b200/csrc/gemm_tc.cuh", "discrete_diffusion_moe_b200/csrc/gemm_pair.cuh",
-                "discrete_diffusion_moe_b200/csrc/epilogues.cuh", "discrete_diffusion_moe_b200/csrc/common.cuh"):
+                "discrete_diffusion_moe_b200/csrc/epilogues.cuh", "discrete_diffusion_moe_b200/csrc/common.cuh",
+                "discrete_diffusion_moe_b200/csrc/moe_pair.cuh"):
         h.update(open(os.path.join(ROOT, rel), "rb").read())
     return h.hexdigest()[:16]
 
