@@ -79,6 +79,11 @@ struct NvtxRange {
 #ifndef DG_PROJ_PAIR
 #define DG_PROJ_PAIR 0
 #endif
+// most k splits of the output projection (its partials are summed by the
+// residual + RMSNorm kernel, which takes any count)
+#ifndef DG_O_SPLITS
+#define DG_O_SPLITS 3
+#endif
 // 1: the two grouped expert products run as one persistent launch on CTA
 // pairs (moe_pair.cuh), a chunk's down product starting as soon as its
 // gate/up outputs are stored
@@ -237,10 +242,10 @@ int proj_bn(int T) { return T >= 256 ? DG_PROJ_BN_MAX : std::min(256, std::max(1
 
 // Split-k of the QKV and output projections: enough units for two CTAs per
 // SM, at most 3 (every split is one more fp32 partial its consumer reads).
-int proj_splits(int m_tiles, int T, int kb, int num_sms) {
+int proj_splits(int m_tiles, int T, int kb, int num_sms, int cap = 3) {
   const int n_tiles = (T + proj_bn(T) - 1) / proj_bn(T);
   const int ks = (2 * num_sms) / std::max(1, m_tiles * n_tiles);
-  return std::max(1, std::min({ks, 3, kb / 4}));
+  return std::max(1, std::min({ks, cap, kb / 4}));
 }
 
 // Split-k (over the vocabulary) of the expected-embedding product
@@ -286,7 +291,7 @@ WsLayout ws_layout(const dg_model_config& c, int batch, int num_sms, int prefill
     size_t rq = 0, ro = 0;
     for (int tt = DG_CANVAS; tt <= (int)T; tt += DG_CANVAS) {
       rq = std::max(rq, (size_t)proj_splits((qkv_rows + 127) / 128, tt, c.d_model / 64, num_sms) * tt);
-      ro = std::max(ro, (size_t)proj_splits((c.d_model + 127) / 128, tt, (int)hq / 64, num_sms) * tt);
+      ro = std::max(ro, (size_t)proj_splits((c.d_model + 127) / 128, tt, (int)hq / 64, num_sms, DG_O_SPLITS) * tt);
     }
     L.qkv = DG_QKV_CLUSTER ? 0 : take(rq * qkv_rows * 4);
     L.opart = DG_O_CLUSTER ? 0 : take(ro * d * 4);
@@ -918,7 +923,7 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
   // split-k of the two dense projections (partials summed by their consumers)
   const int dense_bn_x = proj_bn(T);
   const int ks_qkv = proj_splits((qkv_rows + 127) / 128, T, d / 64, c->num_sms);
-  const int ks_o = proj_splits((d + 127) / 128, T, Hq * hd / 64, c->num_sms);
+  const int ks_o = proj_splits((d + 127) / 128, T, Hq * hd / 64, c->num_sms, DG_O_SPLITS);
 
   // attention key splits (merged inside each split cluster)
   const int splits = attn_splits(B, nq, L0, Hq, Hkv, c->num_sms, 1 << 30);
