@@ -1127,10 +1127,12 @@ static dg_status forward_layers(dg_ctx* c, const dg_kv* kv, int B, int nq, int L
     // norm, or the final norm before the LM head)
     {
       const uint16_t* g_next = l + 1 < m.n_layers ? c->wp(c->wl.layers[l + 1].g_attn) : c->wp(c->wl.g_final);
+      // the next layer's QKV weights go to L2 during the combine
+      const void* pf = l + 1 < m.n_layers ? (const void*)c->wp(c->wl.layers[l + 1].wqkv) : nullptr;
       // two float4s per thread: the eight expert rows per float4 keep the
       // register count high, and two CTAs per SM keep every token resident
       DG_CUDA(Launch(dim3(T), dim3(((d / 4 + 1) / 2 + 31) / 32 * 32), 0, st)(moe_combine_norm_kernel<2>, x, c->at<float>(L.yperm), c->at<int>(L.inv), T, k, d, g_next,
-                                                 xn, m.rms_eps));
+                                                 xn, m.rms_eps, pf, (long long)qkv_rows * d * 2));
       CNT(c);
     }
     DG_CUDA(cudaGetLastError());

@@ -7,6 +7,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "l2_prefetch.cuh"
 
 namespace dg {
 
@@ -591,7 +592,11 @@ template <int NV>
 __global__ void __launch_bounds__(1024) moe_combine_norm_kernel(float* __restrict__ x, const float* __restrict__ y,
                                                                 const int* __restrict__ inv, int T, int k, int d,
                                                                 const uint16_t* __restrict__ gain,
-                                                                uint16_t* __restrict__ xn, float eps) {
+                                                                uint16_t* __restrict__ xn, float eps,
+                                                                const void* pf, long long pf_bytes) {
+  // the next projection's weights (pf, pf_bytes: none when null) into L2; they
+  // depend on nothing, so this comes before the wait for the previous kernel
+  if (threadIdx.x == 0) l2_prefetch_share(pf, pf_bytes, blockIdx.x, gridDim.x);
   grid_dep_wait();
   grid_dep_launch();
   const int t = blockIdx.x;
