@@ -18,7 +18,8 @@
 //   warp 1      tensor memory owner and MMA issuer:
 //                 S  = Q K^T            (M 128, N 64, K hd)    -> TMEM cols [0, 64)
 //                 O += P V              (M 128, N hd, K 64)    -> TMEM cols [64, 64 + hd)
-//                                       (V in fp16, P as two fp16 parts:
+//                                       (V in fp16 from shared memory, P as
+//                                        two fp16 parts from tensor memory:
 //                                        O += P_hi V + P_lo V)
 //               S of tile j + 1 is issued as soon as S of tile j has been read,
 //               before P V of tile j, so the next scores overlap the softmax.
@@ -30,8 +31,8 @@
 //               moved, writes P as P_hi = fp16(P) and P_lo = fp16(P - P_hi)
 //               (about 22 significant bits together; scaled by 2^7 so that
 //               the values lie in (0, 2^15])
-//               into shared memory in the 128-byte-swizzled K-major layout the
-//               MMA reads (the V^T cache holds the bf16-rounded values in
+//               into tensor memory, where the P V product takes its A
+//               operand (the V^T cache holds the bf16-rounded values in
 //               fp16, exact above 2^-14, for this product);
 //               finally read O and write the normalised bf16 output, or
 //               stage the split's unnormalised partial in the freed K/V
@@ -82,9 +83,8 @@ struct AttnTcShape {
   static constexpr uint32_t Q_BYTES = NA * 128 * 128;
   static constexpr uint32_t K_BYTES = NA * kAttnKeys * 128;
   static constexpr uint32_t V_BYTES = HD * 128;      // hd rows x 64 keys
-  static constexpr uint32_t P_BYTES = kAttnRows * 128;  // one fp16 P tile (128 rows x 64 keys)
-  // four P tiles: the high and low fp16 parts of P, two buffers of each by tile parity
-  static constexpr size_t FIXED = 1024 + Q_BYTES + 2 * kAttnPParts * P_BYTES + 32 * 8 + 6 * 128 * 4;
+  // P lives in tensor memory (the A operand of the P V product), not here
+  static constexpr size_t FIXED = 1024 + Q_BYTES + 32 * 8 + 6 * 128 * 4;
   // K/V stages: three where they fit (the load of tile i + 3 is in flight while
   // tiles i + 1, i + 2 are multiplied), else two
   static constexpr int KV_STAGES = FIXED + 3 * (K_BYTES + V_BYTES) <= 227 * 1024 ? 3 : 2;
@@ -92,17 +92,23 @@ struct AttnTcShape {
   // the K/V stages hold the final O tile for its tensor stores: per lane
   // quarter, NCB boxes of 32 rows x 32 fp32 columns (128-byte swizzle)
   static constexpr int NCB = (HD + 31) / 32;
-  // (the K/V stages and then the P tiles: one contiguous region, free at the end)
-  static_assert((size_t)KV_STAGES * (K_BYTES + V_BYTES) + 2 * kAttnPParts * P_BYTES >= (size_t)4 * NCB * 4096,
-                "O staging");
+  // (the K/V stages: one contiguous region, free at the end)
+  static_assert((size_t)KV_STAGES * (K_BYTES + V_BYTES) >= (size_t)4 * NCB * 4096, "O staging");
   // cluster merge: the unnormalised O tile staged row-major in the K/V stage
   // memory with a row pitch of HD + 4 floats (the 16-byte pieces of 8
   // consecutive rows fall in different bank groups), then (max, sum) per row
   static constexpr int OSTR = HD + 4;
   static constexpr uint32_t O_STAGE = 128u * OSTR * 4u;
-  static_assert((size_t)KV_STAGES * (K_BYTES + V_BYTES) >= (size_t)O_STAGE + 128 * 8, "cluster O staging");
-  static_assert(2 * P_BYTES >= 128 * 8 * 4, "merge weights");
-  static constexpr uint32_t TMEM_COLS = (64 + HD) <= 128 ? 128 : 256;
+  // then the merge weights, [at most 64 rows][8 splits]
+  static constexpr uint32_t WTS_OFF = O_STAGE + 128 * 8;
+  static_assert((size_t)KV_STAGES * (K_BYTES + V_BYTES) >= (size_t)WTS_OFF + 64 * 8 * 4, "cluster O staging");
+  // tensor memory: S in columns [0, 64), O in [64, 64 + HD), then P from P_COL:
+  // per tile parity P_hi (and P_lo) as 32 columns each, two fp16 keys per column
+  static constexpr uint32_t P_COL = (64 + HD + 31) / 32 * 32;
+  static constexpr uint32_t P_BUF_COLS = 32 * kAttnPParts;
+  static constexpr uint32_t TMEM_NEED = P_COL + 2 * P_BUF_COLS;
+  static constexpr uint32_t TMEM_COLS = TMEM_NEED <= 128 ? 128 : (TMEM_NEED <= 256 ? 256 : 512);
+  static_assert(TMEM_NEED <= 512, "tensor memory");
 };
 
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
@@ -117,6 +123,26 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) 
       : "memory");
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+// 32 lanes x 16 consecutive 32-bit columns from registers (raw words)
+__device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+// D[tmem] (+)= A[tmem] * B[smem]^T, fp16 inputs, fp32 accumulate; A is M rows
+// in tensor-memory lanes, K packed two 16-bit elements per 32-bit column.
+__device__ __forceinline__ void umma_f16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                                uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 
 // 32 lanes x 32 consecutive fp32 columns in one load and one wait.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
@@ -179,8 +205,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   constexpr int NS = S::KV_STAGES;
   uint8_t* sK = sQ + S::Q_BYTES;               // NS stages
   uint8_t* sV = sK + NS * S::K_BYTES;          // NS stages
-  uint8_t* sP = sV + NS * S::V_BYTES;          // P_hi [2] then P_lo [2] (fp16), by tile parity
-  uint64_t* bars = (uint64_t*)(sP + 2 * kAttnPParts * S::P_BYTES);
+  uint64_t* bars = (uint64_t*)(sV + NS * S::V_BYTES);
   uint64_t* q_full = bars;
   // K and V of a stage are released separately: K as soon as the scores of
   // its tile are computed (so the next K load overlaps the softmax), V after
@@ -248,7 +273,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const uint32_t t_s = tmem_base, t_o = tmem_base + 64;
+  const uint32_t t_s = tmem_base, t_o = tmem_base + 64, t_p = tmem_base + S::P_COL;
 
   if (warp == 0) {
     if (lane == 0 && n_tiles > 0) {
@@ -312,16 +337,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (!mbar_wait(smem_u32(&v_full[i % NS]), (i / NS) & 1, p.err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t va = smem_u32(sV + (i % NS) * S::V_BYTES);
-        const uint32_t pa = smem_u32(sP + (i & 1) * S::P_BYTES);
-        const uint32_t pl = smem_u32(sP + (2 + (i & 1)) * S::P_BYTES);
-        // O += P_hi V + P_lo V: P to ~22 significant bits from two fp16 parts
+        // O += P_hi V + P_lo V: P to ~22 significant bits from two fp16 parts,
+        // both read from tensor memory (8 columns of 16 keys per product)
+        const uint32_t pa = t_p + (uint32_t)(i & 1) * S::P_BUF_COLS;
 #pragma unroll
         for (int k = 0; k < kAttnKeys / 16; ++k)
-          umma_bf16(t_o, sdesc_k128(pa + k * 32), sdesc_k128(va + k * 32), id_o, (i > 0 || k > 0) ? 1u : 0u);
+          umma_f16_tmem_a(t_o, pa + k * 8, sdesc_k128(va + k * 32), id_o, (i > 0 || k > 0) ? 1u : 0u);
         if (kAttnPParts == 2) {
 #pragma unroll
-          for (int k = 0; k < kAttnKeys / 16; ++k)
-            umma_bf16(t_o, sdesc_k128(pl + k * 32), sdesc_k128(va + k * 32), id_o, 1u);
+          for (int k = 0; k < kAttnKeys / 16; ++k) umma_f16_tmem_a(t_o, pa + 32 + k * 8, sdesc_k128(va + k * 32), id_o, 1u);
         }
         umma_commit(smem_u32(&pv_done[i & 1]));
         umma_commit(smem_u32(&v_empty[i % NS]));
@@ -341,7 +365,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const float scale = p.scale_log2;
     float m = -INFINITY, l = 0.f;  // reference max (scaled, log2 units) and this half's sum
     bool ok = true;
-    const uint32_t prow = (uint32_t)row * 128;
     const uint32_t pb = smem_u32(&pair_bar[quarter]);
     constexpr int NCH = HD / 16;
     const int oc0 = half ? (NCH + 1) / 2 : 0, oc1 = half ? NCH : (NCH + 1) / 2;  // this half's O chunks
@@ -415,26 +438,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (i > 1) {
         if (!wait_all(smem_u32(&pv_done[i & 1]), ((i - 2) >> 1) & 1)) { ok = false; break; }
       }
-      // P rows into the swizzled K-major operand tiles: P_hi = fp16(P) and
-      // P_lo = fp16(P - P_hi) (the difference is exact in fp32)
-      uint8_t* p_s = sP + (i & 1) * S::P_BYTES;
-      uint8_t* p_l = sP + (2 + (i & 1)) * S::P_BYTES;
+      // P into tensor memory, the A operand of the P V product: the row's lane,
+      // two keys per 32-bit column (the even key in the low half), this half's
+      // 32 keys in columns [16 half, 16 half + 16); P_hi = fp16(P) and
+      // P_lo = fp16(P - P_hi) (the difference is exact in fp32) 32 columns apart
+      {
+        uint32_t hv[16], lv[16];
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        const int ch = half * 4 + cc;
-        uint32_t hv[4], lv[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float a = sv[cc * 8 + 2 * e], b2 = sv[cc * 8 + 2 * e + 1];
+        for (int e = 0; e < 16; ++e) {
+          const float a = sv[2 * e], b2 = sv[2 * e + 1];
           hv[e] = pack_f16x2(a, b2);
           const __half2 hh = *reinterpret_cast<const __half2*>(&hv[e]);
           lv[e] = pack_f16x2(a - __low2float(hh), b2 - __high2float(hh));
         }
-        const uint32_t off = prow + (((uint32_t)ch ^ ((uint32_t)row & 7)) << 4);
-        *reinterpret_cast<uint4*>(p_s + off) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-        if (kAttnPParts == 2) *reinterpret_cast<uint4*>(p_l + off) = make_uint4(lv[0], lv[1], lv[2], lv[3]);
+        const uint32_t tp = t_p + lane_off + (uint32_t)(i & 1) * S::P_BUF_COLS + (uint32_t)half * 16;
+        tmem_st16u(tp, hv);
+        if (kAttnPParts == 2) tmem_st16u(tp + 32, lv);
+        tmem_wait_st();
       }
-      fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(smem_u32(&p_full[i & 1]));
     }
@@ -555,7 +576,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int per = (kAttnRows + S_ - 1) / S_;
       const int q0 = rank * per, q1 = min(kAttnRows, q0 + per);
       const int te = threadIdx.x - 64;
-      float* wts = reinterpret_cast<float*>(sP);  // [per rows][8 splits] merge weights
+      float* wts = reinterpret_cast<float*>(sK + S::WTS_OFF);  // [per rows][8 splits] merge weights
       const uint32_t o_base = smem_u32(sK), ml_base = smem_u32(sK + S::O_STAGE);
       if (te < q1 - q0) {
         const int row = q0 + te;
