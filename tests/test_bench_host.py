@@ -12,7 +12,7 @@ import bench
 FULL = bench.WORKLOADS["full"]["cfg"]
 
 
-def test_step_cost_matches_the_per_step_totals_of_the_scope_table():
+def test_step_cost_matches_the_stage_by_stage_totals():
     """With every expert touched in every layer, the full-size round is
     1.97 TFLOP and 50.27 GB, summed stage by stage from the model's shapes:
     experts 45.68 GB, attention projections 1.43, attention at context 1024
