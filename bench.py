@@ -242,7 +242,8 @@ def oracle_sample(wl, threads, distinct):
     from its experts block), every layer costed as attention + router +
     (its measured distinct experts) x (seconds per expert), plus the timed
     vocabulary-phase samples.  `distinct`: experts per layer of the GPU's
-    own round.  Returns (seconds per step, description, wall seconds)."""
+    own round (None: a one-layer workload, whose layer 0 is timed whole).
+    Returns (seconds per step, description, wall seconds)."""
     import numpy as np
     from oracle import model as OM
     c = wl["cfg"]
@@ -259,13 +260,52 @@ def oracle_sample(wl, threads, distinct):
     e0 = len(np.unique(np.asarray(idx)))
     t_attn, t_route = t1 - t0, t2 - t1
     t_exp = max(0.0, (t3 - t2) - t_route) / max(e0, 1)
-    layers = sum(t_attn + t_route + e * t_exp for e in distinct)
     tail, tdesc = oracle_tail_sample(wl, W, x1, threads)
+    if distinct is None:
+        layers = t1 - t0 + t3 - t2
+        desc = (f"oracle (numpy float64): the layer timed whole (attention {t_attn:.2f} s, router {t_route:.2f} s, "
+                f"{e0} experts {t3 - t2 - t_route:.2f} s); {tdesc}; inputs generated outside the timing")
+        return layers + tail, desc, time.perf_counter() - w0
+    layers = sum(t_attn + t_route + e * t_exp for e in distinct)
     desc = (f"oracle (numpy float64): layer 0 timed (attention {t_attn:.2f} s, router {t_route:.2f} s, "
             f"{e0} experts {t3 - t2 - t_route:.2f} s); each of the {c['n_layers']} layers costed as attention + "
             f"router + its routed experts (the GPU round's distinct experts per layer, mean "
             f"{sum(distinct) / len(distinct):.1f}) x {t_exp:.3f} s; {tdesc}; inputs generated outside the timing")
     return layers + tail, desc, time.perf_counter() - w0
+
+
+def oracle_other_configs(cores, full_width=True):
+    """The oracle on the smaller configurations, on the host cores: the tiny
+    model's whole 4-round loop (seed 1234, lock above 0.9) on all cores and on
+    one thread, and one full-width layer at context 2048 (timed as the main
+    line's sample, the layer whole).  Returns a list of cpu_baseline-style
+    entries with their workload named."""
+    from threadpoolctl import threadpool_limits
+    from oracle import decode as OD
+    from oracle import sampler as OS
+    out = []
+    wl = WORKLOADS["tiny"]
+    c = wl["cfg"]
+    for threads in (cores, 1):
+        with threadpool_limits(limits=threads):
+            ocfg, W, kv, _ = oracle_setup(wl, threads)
+            state = OD.new_state(OD.init_canvas(1234, 0, 1, CANVAS, c["vocab"]), c["d_model"])
+            sc = OS.SamplerConfig(max_steps=4, lock_threshold=0.9, seed=1234)
+            W.layer(0)
+            t0 = time.perf_counter()
+            for s_ in range(4):
+                OD.denoise_step(ocfg, W, kv, state, sc, 0, s_, keep_logits=False)
+            sec = time.perf_counter() - t0
+        out.append({"workload": "tiny 2-layer model (d 256, 16 experts top-2, vocab 4096), context 64, "
+                                "the whole 4-round loop",
+                    "value": 4.0 / sec, "unit": UNIT, "cores": threads, "kind": "oracle",
+                    "sample": "every round of the loop computed and timed (weights generated outside the timing)"})
+    if full_width:
+        with threadpool_limits(limits=cores):
+            per_step, desc, _ = oracle_sample(WORKLOADS["layer1"], cores, distinct=None)
+        out.append({"workload": "one full-width layer, context 2048, one round", "value": 1.0 / per_step,
+                    "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc})
+    return out
 
 
 def time_steps(dg, model, kv, cv, samp, block, steps, warm, stream):
@@ -682,11 +722,17 @@ def main():
 
     if rank == 0:
         cpu = None
+        cpu_other = None
         if world == 1 and not args.no_cpu_baseline:
             cores = cpu_cores()
             per_step, desc, wall = oracle_sample(wl, threads=cores, distinct=distinct)
             cpu = {"value": 1.0 / per_step, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc,
                    "sample_wall_s": wall}
+            if args.workload == "full" and not args.no_other_configs:
+                try:
+                    cpu_other = oracle_other_configs(cores)
+                except Exception as e:  # reported; the main line stands without these figures
+                    cpu_other = {"error": f"{type(e).__name__}: {e}"}
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
@@ -715,6 +761,7 @@ def main():
             "clocks": clk,
             "e2e": e2e,
             "cpu_baseline": cpu,
+            "cpu_baseline_other_configs": cpu_other,
             "other_configs": extra,
         }
         print(json.dumps(line), flush=True)

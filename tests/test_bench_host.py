@@ -83,3 +83,13 @@ def test_peaks_fall_back_to_the_stated_figures_without_the_measured_file(monkeyp
     (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"hbm_gbs": 6500.0, "bf16_tflops": 1600.0}))
     p = bench.load_peaks()
     assert p["source"] == "measured" and p["bf16_tflops_sustained"] == 1600.0
+
+
+def test_oracle_timing_of_the_tiny_loop_on_all_cores_and_one_thread():
+    """The oracle baselines of the smaller configurations: the tiny model's
+    whole 4-round loop, timed on the cores it is given and on one thread."""
+    out = bench.oracle_other_configs(2, full_width=False)
+    assert [e["cores"] for e in out] == [2, 1]
+    for e in out:
+        assert e["kind"] == "oracle" and e["unit"] == bench.UNIT and e["value"] > 0
+        assert "4-round loop" in e["workload"]
