@@ -6,7 +6,9 @@ share the chunk and take consecutive tiles, the only empty tile being the
 missing second tile of an odd tile count; units run expert, then tile, then
 chunk.  Dense products: every (A tile, column tile) is covered once per k
 split, the splits partition the k blocks, and units walk the splits, then
-the column tiles (or the A tiles)."""
+the column tiles (or the A tiles).  The one-launch expert block: the chunk
+counters its down units wait on, and the unit order that makes those waits
+end."""
 
 import ctypes
 import os
@@ -166,3 +168,46 @@ def test_dense_schedule_rejects_bad_arguments(dense_fn):
     assert dense_fn(128, 16, 64, 16, 2, 1, 1, None, 0, ctypes.byref(n)) != 0   # more splits than k blocks
     assert dense_fn(128, 16, 64, 16, 1, 3, 1, None, 0, ctypes.byref(n)) != 0   # mt 3
     assert dense_fn(128, 16, 100, 16, 1, 1, 1, None, 0, ctypes.byref(n)) != 0  # K % 64
+
+
+@pytest.mark.parametrize("seed,E,k,T", [(0, 128, 8, 256), (1, 128, 8, 256), (2, 16, 2, 256), (3, 128, 8, 512)])
+def test_fused_expert_block_dependencies(fn, seed, E, k, T):
+    """The one-launch expert block (gate/up units, then down units, on CTA
+    pairs; pair c takes units c, c + clusters, ...): a down unit of token chunk
+    q waits until every CTA of the gate/up units of q has published, i.e. for
+    2 x (gate/up tile pairs) arrivals.  On random routings: each chunk has
+    exactly that many gate/up CTAs and one down unit per down tile pair, both
+    phases number the chunks alike and within the counter array, and every
+    pair reaches all of its gate/up units before its first down unit."""
+    d, f, bn, clusters = 2816, 704, 128, 148
+    rng = np.random.default_rng(seed)
+    counts = np.bincount(np.concatenate([rng.choice(E, k, replace=False) for _ in range(T)]), minlength=E)
+    sizes = [int(x) for x in counts]
+    chunk_off = np.concatenate([[0], np.cumsum([-(-s // bn) for s in sizes])])
+    n_chunks = int(chunk_off[-1])
+
+    def units(R, K):
+        off, jobs = _jobs(fn, 1, R, sizes, K, bn)
+        out = {}
+        for u, r, g, t, a0, mv, n0, nv, kb, bmap in jobs:
+            out.setdefault(int(u), []).append(int(chunk_off[g] + (n0 - off[g]) // bn))
+        assert all(len(set(v)) == 1 and len(v) == 2 for v in out.values())  # both ranks, one chunk
+        return {u: v[0] for u, v in out.items()}
+
+    up, down = units(2 * f, d), units(d, f)
+    p_up, p_down = (2 * f // 128 + 1) // 2, (d // 128 + 1) // 2
+    assert len(up) == p_up * n_chunks and len(down) == p_down * n_chunks
+    arrivals = np.bincount([q for q in up.values()], minlength=n_chunks) * 2  # both CTAs of a unit add one
+    assert np.all(arrivals == 2 * p_up)
+    assert np.all(np.bincount([q for q in down.values()], minlength=n_chunks) == p_down)
+    assert n_chunks <= T * k // 16 + E + 1  # the counters the workspace holds
+    U1 = len(up)
+    for c in range(clusters):
+        mine = list(range(c, U1 + len(down), clusters))
+        first_down = next((i for i, u in enumerate(mine) if u >= U1), len(mine))
+        assert all(u < U1 for u in mine[:first_down]) and all(u >= U1 for u in mine[first_down:])
+        # every chunk this pair waits for has its gate/up units among units that
+        # some pair reaches before any of its own down units
+        for u in mine[first_down:]:
+            q = down[u - U1]
+            assert all(v < U1 for v, qq in up.items() if qq == q)
