@@ -11,9 +11,16 @@ baseline leg use it.
 It shares no code with the CUDA library.  Its only shared dependency is the
 seeded input generator in ``synth/`` (weights and token ids are inputs).
 
+A second, plain C++ implementation of the same round and of the causal
+encoding (``dg_oracle.cpp``, double precision with plain loops, reached
+through ``oracle.cpp``) shares no code with this one either; the tests run
+both on the same seeded weights and inputs and require them to agree at
+every decision point.
+
 Parity status per function is recorded in each module's docstring; the one
-part with no independent pin is the composition of the full random-init
-model (``forward_logits``): "parity unpinned" beyond its pinned components.
+part with no independent closed-form pin is the composition of the full
+random-init model (``forward_layers`` over many layers): "parity unpinned"
+beyond its pinned components, and cross-checked only by the C++ oracle.
 """
 
 from .philox import philox4x32_10, uniform_token, gumbel_u  # noqa: F401
