@@ -274,12 +274,18 @@ def oracle_sample(wl, threads, distinct):
     return layers + tail, desc, time.perf_counter() - w0
 
 
+def oracle_cfg(c):
+    import oracle
+    return oracle.ModelConfig(**c)
+
+
 def oracle_other_configs(cores, full_width=True):
     """The oracle on the smaller configurations, on the host cores: the tiny
     model's whole 4-round loop (seed 1234, lock above 0.9) on all cores and on
-    one thread, and one full-width layer at context 2048 (timed as the main
-    line's sample, the layer whole).  Returns a list of cpu_baseline-style
-    entries with their workload named."""
+    one thread, the same loop on the plain C++ oracle (one thread), and one
+    full-width layer at context 2048 (timed as the main line's sample, the
+    layer whole).  Returns a list of cpu_baseline-style entries with their
+    workload named."""
     from threadpoolctl import threadpool_limits
     from oracle import decode as OD
     from oracle import sampler as OS
@@ -300,6 +306,26 @@ def oracle_other_configs(cores, full_width=True):
                                 "the whole 4-round loop",
                     "value": 4.0 / sec, "unit": UNIT, "cores": threads, "kind": "oracle",
                     "sample": "every round of the loop computed and timed (weights generated outside the timing)"})
+    # the plain C++ oracle (one thread, plain loops) on the same loop
+    from oracle import cpp
+    import synth
+    m = cpp.Model(oracle_cfg(c), seed=0)
+    cache = cpp.Cache(m.cfg, 1, wl["ctx"] + CANVAS)
+    cpp.encode_context(m, cache, synth.context_tokens(1, wl["ctx"], 1234, c["vocab"]).astype("int64"))
+    import numpy as np
+    st = {"tokens": cpp.init_canvas(1234, 0, 1, CANVAS, c["vocab"]), "sc": np.zeros((1, CANVAS, c["d_model"])),
+          "prev_argmax": np.full((1, CANVAS), -1, np.int64), "done": np.zeros(1, np.uint8),
+          "locked": np.zeros((1, CANVAS), np.uint8)}
+    samp = cpp.sampler(max_steps=4, lock_threshold=0.9, seed=1234)
+    t0 = time.perf_counter()
+    for s_ in range(4):
+        cpp.denoise_step(m, cache, st, samp, 0, s_)
+    sec = time.perf_counter() - t0
+    out.append({"workload": "tiny 2-layer model (d 256, 16 experts top-2, vocab 4096), context 64, "
+                            "the whole 4-round loop", "value": 4.0 / sec, "unit": UNIT, "cores": 1,
+                "kind": "oracle (plain C++, double, plain loops)",
+                "sample": "every round of the loop computed and timed (weights and the context encode outside "
+                          "the timing)"})
     if full_width:
         with threadpool_limits(limits=cores):
             per_step, desc, _ = oracle_sample(WORKLOADS["layer1"], cores, distinct=None)

@@ -87,9 +87,11 @@ def test_peaks_fall_back_to_the_stated_figures_without_the_measured_file(monkeyp
 
 def test_oracle_timing_of_the_tiny_loop_on_all_cores_and_one_thread():
     """The oracle baselines of the smaller configurations: the tiny model's
-    whole 4-round loop, timed on the cores it is given and on one thread."""
+    whole 4-round loop, timed on the cores it is given and on one thread, and
+    on the plain C++ oracle."""
     out = bench.oracle_other_configs(2, full_width=False)
-    assert [e["cores"] for e in out] == [2, 1]
+    assert [e["cores"] for e in out] == [2, 1, 1]
+    assert "C++" in out[2]["kind"]
     for e in out:
-        assert e["kind"] == "oracle" and e["unit"] == bench.UNIT and e["value"] > 0
+        assert e["kind"].startswith("oracle") and e["unit"] == bench.UNIT and e["value"] > 0
         assert "4-round loop" in e["workload"]
