@@ -158,3 +158,13 @@ def test_topk_self_conditioning_and_the_persistent_lock_agree():
     rep = _run(dict(TINY, self_cond=True), dict(max_steps=8, seed=5, selfcond_topk=16, persistent_lock=True,
                                                 lock_threshold=7.6e-4), rounds=3, batch=1)
     assert rep["locked"] > 0 and rep["kept"] > 0, rep
+
+
+def test_grouped_query_attention_and_wider_routing_agree():
+    """Two query heads per kv head (head_dim 64), top-4 of 32 experts, three
+    layers, a longer context and a round later in the block."""
+    cfg = dict(n_layers=3, d_model=512, n_q_heads=8, n_kv_heads=4, head_dim=64, n_experts=32, top_k=4,
+               d_ff=256, vocab=2048)
+    rep = _run(cfg, dict(max_steps=12, lock_threshold=1e-3, seed=99), rounds=2, batch=1, ctx=200)
+    assert rep["decisions"] + rep["excused"] == 2 * (3 * 256 + 2 * 256)
+    assert rep["excused"] <= 0.01 * rep["decisions"], rep
