@@ -168,3 +168,35 @@ def test_grouped_query_attention_and_wider_routing_agree():
     rep = _run(cfg, dict(max_steps=12, lock_threshold=1e-3, seed=99), rounds=2, batch=1, ctx=200)
     assert rep["decisions"] + rep["excused"] == 2 * (3 * 256 + 2 * 256)
     assert rep["excused"] <= 0.01 * rep["decisions"], rep
+
+
+def test_round_invariants_of_the_cpp_oracle():
+    """What the pages fix, checked on the C++ oracle's own outputs: entropy in
+    [0, ln V] and 1/V <= pmax <= 1; a locked position's next token is its
+    sample; the stop fires exactly when the mean entropy is below the
+    threshold (thresholds just above and just below the round's value)."""
+    ocfg = oracle.ModelConfig(**TINY)
+    m = cpp.Model(ocfg, seed=0)
+    V = ocfg.vocab
+
+    def one_round(stop_entropy, lock_threshold):
+        cache = cpp.Cache(ocfg, 1, 64 + 256)
+        cpp.encode_context(m, cache, synth.context_tokens(1, 64, 1234, V).astype(np.int64))
+        st = {"tokens": cpp.init_canvas(3, 0, 1, 256, V), "sc": np.zeros((1, 256, ocfg.d_model)),
+              "prev_argmax": np.full((1, 256), -1, np.int64), "done": np.zeros(1, np.uint8),
+              "locked": np.zeros((1, 256), np.uint8)}
+        o = cpp.denoise_step(m, cache, st, cpp.sampler(max_steps=48, seed=3, stop_entropy=stop_entropy,
+                                                       lock_threshold=lock_threshold), 0, 0)
+        return o, st
+
+    o, st = one_round(0.5, 7.6e-4)
+    assert np.all(o["entropy"] >= 0) and np.all(o["entropy"] <= np.log(V) + 1e-12)
+    assert np.all(o["pmax"] >= 1.0 / V - 1e-15) and np.all(o["pmax"] <= 1.0)
+    lock = o["lock"].astype(bool)
+    assert 0 < lock.sum() < lock.size
+    assert np.array_equal(st["tokens"][lock], o["sample"][lock])
+    mh = float(o["mean_entropy"][0])
+    below, _ = one_round(np.nextafter(mh, np.inf), 7.6e-4)
+    above, _ = one_round(mh, 7.6e-4)
+    assert below["stop"][0] == 1 and below["final"][0] == 1
+    assert above["stop"][0] == 0 and above["final"][0] == 0
